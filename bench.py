@@ -1,0 +1,386 @@
+#!/usr/bin/env python3
+"""Throughput of the DLRM hot path on B200, as one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload large] [--impl ours|reference]
+
+A step is one forward pass of the whole hot path over one batch: bottom MLP,
+fused embedding-bag gather + pairwise interaction + concat, top MLP and
+sigmoid. Default workload: the large memory-bound configuration (B = 65536,
+26 tables with log-spaced row counts 1e3 .. 4e7 = 29.6 GB of bf16, d = 128,
+one-hot Zipf(1.05) bags, bottom MLP 13-512-256-128, top MLP
+479-1024-1024-512-256-1). Inputs are seeded synthetic stand-ins for a click
+log; the benchmark cycles a pool of 8 batches.
+
+value:  samples/s with inputs resident in HBM, device time (CUDA events),
+        max over ranks; each rank runs an independent replica (weak scaling).
+e2e:    the same through dlrm_forward with the batch copied from pinned host
+        memory and y_hat copied back inside the timed region.
+roofline: the fused gather + interaction kernel against measured HBM
+        bandwidth, with algorithmic bytes = gathered rows + indices + offsets +
+        x_dense read + concat write.
+cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload.
+
+--impl reference times that oracle alone (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import CONFIGS, gen  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+POOL = 8
+
+
+def workload_desc(cfg) -> str:
+    rows = f"{min(cfg.rows)}..{max(cfg.rows)} rows" if len(set(cfg.rows)) > 1 else f"{cfg.rows[0]} rows each"
+    tb = sum(cfg.rows) * cfg.d * (4 if cfg.table_dtype == "f32" else 2) / 1e9
+    return (f"{cfg.name}: B={cfg.B}, K={cfg.K} tables ({rows}, {tb:.1f} GB {cfg.table_dtype}), d={cfg.d}, "
+            f"bags={cfg.bag}, indices={cfg.index}, bottom={'-'.join(map(str, cfg.bottom))}, "
+            f"top={'-'.join(map(str, cfg.top))}")
+
+
+def algorithmic_bytes(cfg, batch) -> int:
+    """Bytes the fused gather + interaction must move for one batch."""
+    es_t = 4 if cfg.table_dtype == "f32" else 2
+    es_o = 4 if cfg.mlp_dtype == "f32" else 2
+    rows = int(batch.indices.size) * cfg.d * es_t
+    return rows + 4 * batch.indices.size + 4 * (cfg.K * cfg.B + 1) + 4 * cfg.B * cfg.d + es_o * cfg.B * cfg.concat_width
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_traffic(path_rel: str, src_rel: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, path_rel)
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    src = open(os.path.join(ROOT, src_rel), "rb").read()
+    if j.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    return j.get("dram_bytes_per_launch_full")
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(self.REASONS, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle (CPU baseline)
+
+def oracle_rate(cfg, batch, n_samples: int, seed: int = 0):
+    """samples/s of the fp64 oracle forward on n_samples drawn from the batch (excluding input prep)."""
+    from oracle import oracle as O
+    rng = np.random.default_rng(seed)
+    samples = np.sort(rng.choice(cfg.B, size=min(n_samples, cfg.B), replace=False))
+    Bs, dense, offs, idx, _, rows, used = O.sub_batch(cfg, batch, samples)
+    model = O.model_for_rows(cfg, used)
+    t0 = time.perf_counter()
+    O.forward(model, dense, offs, idx)
+    dt = time.perf_counter() - t0
+    return Bs / dt, dt, O.threads(), Bs
+
+
+def calibrated_oracle(cfg, batch, target_s: float):
+    n = 64
+    rate, dt, cores, used = oracle_rate(cfg, batch, n)
+    n2 = int(min(cfg.B, max(n, rate * target_s)))
+    if n2 > n:
+        rate, dt, cores, used = oracle_rate(cfg, batch, n2, seed=1)
+    return rate, dt, cores, used
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return 0
+    batch = gen.make_batches(cfg, (0,))[0]
+    # size one step at about 1/(steps + warmup) of ~2 minutes of CPU time
+    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    rate0, _, cores, _ = oracle_rate(cfg, batch, 32)
+    n = int(min(cfg.B, max(16, rate0 * budget)))
+    for w in range(args.warmup):
+        oracle_rate(cfg, batch, n, seed=100 + w)
+    total_s, total_n = 0.0, 0
+    for s in range(args.steps):
+        r, dt, cores, used = oracle_rate(cfg, batch, n, seed=s)
+        total_s += dt
+        total_n += used
+    value = total_n / total_s
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": workload_desc(cfg), "global_batch": cfg.B, "parallelism": "cpu-oracle"},
+           "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
+                            "sample": f"{n} random samples of batch 0 per step (fp64 forward, host cores)"},
+           "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+METRIC = "DLRM samples/s on 1 B200; EmbeddingBag+interaction HBM GB/s as % of peak"
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import embedding_bags_dot_b200 as E
+    from synth import device as sd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    E.lib()
+    sd.build_fill()
+
+    # model
+    tables = sd.tables_on_device(cfg, device=dev)
+    T = E.Tables(tables, cfg.rows, cfg.d)
+    bW, bb, bd = sd.mlp_on_device(cfg, "bottom", dev)
+    tW, tb, td = sd.mlp_on_device(cfg, "top", dev)
+    bot, top = E.MLP(bW, bb, bd), E.MLP(tW, tb, td)
+    ws = E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, cfg.B, 0), dev)
+
+    # batch pool (independent per rank)
+    ids = tuple(rank * POOL + j for j in range(POOL))
+    perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
+    batches = gen.make_batches(cfg, ids, perms=perms)
+    dev_b = [sd.batch_on_device(b, dev) for b in batches]
+    host_b = [sd.batch_on_device(b, pin=True) for b in batches]
+    algo_bytes = [algorithmic_bytes(cfg, b) for b in batches]
+    pool_bytes = sum(sum(t.numel() * t.element_size() for t in d.values()) for d in dev_b)
+
+    ldc = cfg.concat_ld
+    out_t = sd.TORCH_DT[cfg.mlp_dtype]
+    x_dense = torch.empty((cfg.B, cfg.d), dtype=torch.float32, device=dev)
+    concat = torch.zeros((cfg.B, ldc), dtype=out_t, device=dev)
+    y = torch.empty(cfg.B, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        b = dev_b[i % POOL]
+        if ev is not None:
+            ev[0].record(stream)
+        E.dlrm_mlp_fwd(bot, cfg.B, b["dense"], cfg.n_dense, x_dense, cfg.d, E.ACT_RELU, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        E.dlrm_embbag_interact_fwd(T, cfg.B, b["offsets"], b["indices"], x_dense, concat, ldc, cfg.mlp_dtype, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        E.dlrm_mlp_fwd(top, cfg.B, concat, ldc, y, 1, E.ACT_SIGMOID, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for i in range(args.warmup):
+        step(i)
+    st = E.dlrm_check_error(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device error record after warm-up: {st}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    barrier()
+    clocks.start()
+    n0 = E.dlrm_launch_count()
+    for i in range(args.steps):
+        step(i, evs[i])
+    n1 = E.dlrm_launch_count()
+    barrier()
+    clk = clocks.stop()
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    k2_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bot_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    top_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    st = E.dlrm_check_error(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device error record after timing: {st}")
+
+    # end to end through dlrm_forward with host buffers
+    stage = {k: torch.empty_like(v, device=dev) for k, v in dev_b[0].items()}
+    y_host = torch.empty(cfg.B, dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        hb = host_b[i % POOL]
+        for k in ("dense", "offsets", "indices"):
+            if stage[k].numel() != hb[k].numel():
+                stage[k] = torch.empty(hb[k].shape, dtype=hb[k].dtype, device=dev)
+            stage[k].copy_(hb[k], non_blocking=True)
+        E.dlrm_forward(T, bot, top, cfg.B, stage["dense"], stage["offsets"], stage["indices"], y, ws, stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = int(np.mean([sum(hb[k].numel() * hb[k].element_size() for k in ("dense", "offsets", "indices"))
+                       for hb in host_b]))
+    d2h = cfg.B * 4
+
+    # max over ranks
+    def maxr(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    total_ms, e2e_ms = maxr(total_ms), maxr(e2e_ms)
+    k2_avg = maxr(float(np.mean(k2_ms)))
+    peak_hbm, peak_bf16, peak_kind = read_peaks()
+    avg_algo = float(np.mean([algo_bytes[i % POOL] for i in range(args.steps)]))
+    achieved = avg_algo / (k2_avg * 1e-3) / 1e9
+    samples = cfg.B * args.steps * world
+    value = samples / (total_ms * 1e-3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, cores, used = calibrated_oracle(cfg, batches[0], args.cpu_seconds)
+        cpu = {"value": rate, "unit": "samples/s", "cores": cores, "kind": "oracle",
+               "sample": f"{used} random samples of batch 0, fp64 forward in {dt:.1f} s"}
+
+    if rank == 0:
+        traffic = kernel_traffic("profiles/embbag_interact_large_traffic.json",
+                                 "embedding_bags_dot_b200/csrc/embbag.cu")
+        out = {
+            "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.table_dtype, "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "per_gpu_batch": cfg.B,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"no flush: tables {sum(cfg.rows) * cfg.d * (4 if cfg.table_dtype == 'f32' else 2) / 1e9:.1f} GB "
+                             f"and a {POOL}-batch pool of {pool_bytes / 1e6:.0f} MB exceed the {L2_BYTES >> 20} MB L2"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
+                         "frac": achieved / peak_hbm, "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": "embbag_interact_kernel (dlrm_embbag_interact_fwd)",
+                         "algorithmic_bytes_per_launch": avg_algo, "avg_launch_ms": k2_avg},
+            "kernels_ms_per_step": {"bottom_mlp": float(np.mean(bot_ms)), "embbag_interact": float(np.mean(k2_ms)),
+                                    "top_mlp": float(np.mean(top_ms))},
+            "cpu_baseline": cpu,
+            "e2e": {"value": samples / (e2e_ms * 1e-3), "unit": "samples/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": int(n1 - n0),
+            "clocks": clk,
+        }
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="large", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

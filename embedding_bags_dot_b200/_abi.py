@@ -1,0 +1,208 @@
+"""ctypes binding of libdlrm.so.
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of libdlrm.so. PyTorch provides device memory and streams. The
+functions keep the C names (``dlrm_forward`` ...) and take torch tensors;
+a non-OK status raises ``DlrmError`` carrying the status code.
+
+There is no CPU fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdlrm.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_INDEX_OOB, ERR_BAD_OFFSETS, ERR_TIMEOUT, ERR_CUDA, ERR_WORKSPACE = range(8)
+F32, F16, BF16 = 0, 1, 2
+ACT_NONE, ACT_RELU, ACT_SIGMOID = 0, 1, 2
+MAX_TABLES = 256
+MAX_LAYERS = 16
+ERR_RECORD_BYTES = 256
+
+DT_CODE = {"f32": F32, "f16": F16, "bf16": BF16, torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+DT_TORCH = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
+
+
+class DlrmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: status {status} ({status_str(status)})")
+
+
+class dlrm_tables(C.Structure):
+    _fields_ = [("data", C.c_void_p), ("rows", C.POINTER(C.c_int64)), ("K", C.c_int), ("d", C.c_int), ("dt", C.c_int)]
+
+
+class dlrm_mlp(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("dims", C.POINTER(C.c_int)), ("W", C.POINTER(C.c_void_p)),
+                ("b", C.POINTER(C.c_void_p)), ("dt", C.c_int)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+_SIGS = {
+    "dlrm_launch_count": (C.c_uint64, []),
+    "dlrm_ld": (C.c_int, [C.c_int, C.c_int]),
+    "dlrm_status_str": (C.c_char_p, [C.c_int]),
+    "dlrm_workspace_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
+    "dlrm_check_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_embbag_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
+                                  C.c_void_p, C.c_void_p]),
+    "dlrm_interact_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int,
+                                    C.c_void_p]),
+    "dlrm_embbag_interact_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p,
+                                           C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "dlrm_mlp_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int,
+                               C.c_void_p, C.c_void_p]),
+    "dlrm_forward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                               C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+}
+
+
+def lib():
+    """Load libdlrm.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libdlrm.so is not built ({LIB_PATH}); run `python -m embedding_bags_dot_b200.build`")
+            L = C.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def status_str(s: int) -> str:
+    try:
+        return lib().dlrm_status_str(int(s)).decode()
+    except Exception:  # noqa: BLE001 - only used for messages
+        return "?"
+
+
+def _check(status: int, where: str) -> int:
+    if status != OK:
+        raise DlrmError(status, where)
+    return status
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr() if t.numel() else None
+
+
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def dlrm_launch_count() -> int:
+    return int(lib().dlrm_launch_count())
+
+
+def dlrm_ld(n: int, dt) -> int:
+    return int(lib().dlrm_ld(int(n), DT_CODE.get(dt, dt)))
+
+
+# ----------------------------------------------------------------- model containers
+
+class Tables:
+    """K tables in one contiguous device buffer ([sum rows][d]) plus host row counts."""
+
+    def __init__(self, data: torch.Tensor, rows, d: int):
+        assert data.is_cuda and data.is_contiguous()
+        self.data = data
+        self.rows = [int(r) for r in rows]
+        self.d = int(d)
+        self._rows = (C.c_int64 * len(self.rows))(*self.rows)
+        self.struct = dlrm_tables(data.data_ptr(), self._rows, len(self.rows), self.d, DT_CODE[data.dtype])
+
+    @property
+    def K(self):
+        return len(self.rows)
+
+    def ref(self):
+        return C.byref(self.struct)
+
+
+class MLP:
+    """Layers W[l] ([out][dlrm_ld(in)] device tensors) and fp32 biases b[l]."""
+
+    def __init__(self, Ws, bs, dims):
+        self.Ws, self.bs, self.dims = list(Ws), list(bs), [int(x) for x in dims]
+        assert len(self.Ws) == len(self.bs) == len(self.dims) - 1
+        self.dt = DT_CODE[self.Ws[0].dtype]
+        self._dims = (C.c_int * len(self.dims))(*self.dims)
+        self._W = (C.c_void_p * len(self.Ws))(*[w.data_ptr() for w in self.Ws])
+        self._b = (C.c_void_p * len(self.bs))(*[b.data_ptr() for b in self.bs])
+        self.struct = dlrm_mlp(len(self.Ws), self._dims, self._W, self._b, self.dt)
+
+    def ref(self):
+        return C.byref(self.struct)
+
+
+def _ref(x):
+    return None if x is None else x.ref()
+
+
+# ----------------------------------------------------------------- entry points (C names)
+
+def dlrm_workspace_size(T: Tables, bot: MLP, top: MLP, B: int, training: int = 0) -> int:
+    return int(lib().dlrm_workspace_size(_ref(T), _ref(bot), _ref(top), int(B), int(training)))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace (the error record must start at zero)."""
+    return torch.zeros(max(int(nbytes), ERR_RECORD_BYTES), dtype=torch.uint8, device=device)
+
+
+def dlrm_check_error(ws: torch.Tensor, stream=None):
+    """Returns (status, flags, n_skipped_indices, n_bad_bags) and clears the record."""
+    info = (C.c_int64 * 3)()
+    s = lib().dlrm_check_error(_ptr(ws), _stream(stream), info)
+    return int(s), int(info[0]), int(info[1]), int(info[2])
+
+
+def dlrm_embbag_fwd(T: Tables, B: int, offsets, indices, pooled, bag_len=None, ws=None, stream=None):
+    return _check(lib().dlrm_embbag_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
+                                        _ptr(pooled), _ptr(bag_len), _ptr(ws), _stream(stream)), "dlrm_embbag_fwd")
+
+
+def dlrm_interact_fwd(B: int, K: int, d: int, x_dense, pooled, concat, ld: int, out_dt=None, stream=None):
+    out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
+    return _check(lib().dlrm_interact_fwd(int(B), int(K), int(d), _ptr(x_dense), _ptr(pooled), _ptr(concat), int(ld),
+                                          int(out_dt), _stream(stream)), "dlrm_interact_fwd")
+
+
+def dlrm_embbag_interact_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,
+                             stream=None):
+    out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
+    return _check(lib().dlrm_embbag_interact_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
+                                                 _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
+                                                 _stream(stream)), "dlrm_embbag_interact_fwd")
+
+
+def dlrm_mlp_fwd(mlp: MLP, B: int, inp, ld_in: int, out, ld_out: int, final_act: int, ws, stream=None):
+    return _check(lib().dlrm_mlp_fwd(mlp.ref(), int(B), _ptr(inp), DT_CODE[inp.dtype], int(ld_in), _ptr(out),
+                                     int(ld_out), int(final_act), _ptr(ws), _stream(stream)), "dlrm_mlp_fwd")
+
+
+def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
+    return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
+                                     _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
+                  "dlrm_forward")

@@ -1,0 +1,249 @@
+// extern "C" entry points of libdlrm: argument checks, workspace carving and
+// launch order. Every operation runs in the kernels of this library; nothing
+// here computes on the host beyond sizes and table bases.
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace dlrm;
+
+namespace dlrm {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace dlrm
+
+namespace {
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline bool valid_dt(int dt) { return dt == DLRM_F32 || dt == DLRM_F16 || dt == DLRM_BF16; }
+inline cudaStream_t cs(dlrm_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+dlrm_status check_tables(const dlrm_tables* T, TableMeta& tm) {
+    if (!T || !T->rows || !T->data) return DLRM_ERR_INVALID_ARG;
+    if (T->K < 1 || T->d < 1 || !valid_dt(T->dt)) return DLRM_ERR_INVALID_ARG;
+    if (T->K > DLRM_MAX_TABLES) return DLRM_ERR_UNSUPPORTED;
+    if (!aligned16(T->data)) return DLRM_ERR_INVALID_ARG;
+    long long acc = 0;
+    for (int k = 0; k < T->K; ++k) {
+        if (T->rows[k] < 1) return DLRM_ERR_INVALID_ARG;
+        tm.base[k] = acc;
+        tm.rows[k] = T->rows[k];
+        acc += T->rows[k];
+    }
+    if (!gather_supported(T->d, T->dt)) return DLRM_ERR_UNSUPPORTED;
+    return DLRM_OK;
+}
+
+dlrm_status check_bags(int B, const int32_t* offsets, const int32_t* indices, int64_t nnz) {
+    if (B < 0 || nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
+    if (B > 0 && !offsets) return DLRM_ERR_INVALID_ARG;
+    if (nnz > 0 && !indices) return DLRM_ERR_INVALID_ARG;
+    return DLRM_OK;
+}
+
+dlrm_status check_mlp(const dlrm_mlp* m) {
+    if (!m || !m->dims || !m->W || !m->b) return DLRM_ERR_INVALID_ARG;
+    if (m->n_layers < 1 || m->n_layers > DLRM_MAX_LAYERS || !valid_dt(m->dt)) return DLRM_ERR_INVALID_ARG;
+    for (int l = 0; l <= m->n_layers; ++l)
+        if (m->dims[l] < 1) return DLRM_ERR_INVALID_ARG;
+    for (int l = 0; l < m->n_layers; ++l)
+        if (!m->W[l] || !m->b[l] || !aligned16(m->W[l])) return DLRM_ERR_INVALID_ARG;
+    return DLRM_OK;
+}
+
+// Bytes of one hidden-activation buffer for the widest hidden layer of m.
+size_t hidden_bytes(const dlrm_mlp* m, int B) {
+    size_t w = 0;
+    for (int l = 1; l < m->n_layers; ++l) {
+        const size_t b = (size_t)dlrm_ld(m->dims[l], m->dt) * esize(m->dt);
+        if (b > w) w = b;
+    }
+    return w * (size_t)B;
+}
+
+struct FwdLayout {
+    size_t x_dense, concat, act0, act1, total;
+};
+
+FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
+    FwdLayout L;
+    size_t off = DLRM_ERR_RECORD_BYTES;
+    const int K = T->K, d = T->d;
+    const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
+    L.x_dense = off;
+    off = align_up(off + sizeof(float) * (size_t)B * d, 256);
+    L.concat = off;
+    off = align_up(off + (size_t)B * ldc * esize(top->dt), 256);
+    size_t h = hidden_bytes(bot, B);
+    const size_t ht = hidden_bytes(top, B);
+    if (ht > h) h = ht;
+    L.act0 = off;
+    off = align_up(off + h, 256);
+    L.act1 = off;
+    off = align_up(off + h, 256);
+    L.total = off;
+    return L;
+}
+
+// The MLP chain: ReLU after hidden layers, final_act after the last layer.
+dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out, int ld_out,
+                    int final_act, void* act0, void* act1, cudaStream_t st) {
+    const void* cur = in;
+    dlrm_dtype cur_dt = in_dt;
+    int cur_ld = ld_in;
+    for (int l = 0; l < m->n_layers; ++l) {
+        const int K = m->dims[l], N = m->dims[l + 1];
+        const int ldw = dlrm_ld(K, m->dt);
+        dlrm_status r;
+        if (l == m->n_layers - 1) {
+            r = launch_linear(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l], out, DLRM_F32, ld_out,
+                              final_act, st);
+        } else {
+            void* dst = (l & 1) ? act1 : act0;
+            const int ldd = dlrm_ld(N, m->dt);
+            r = launch_linear(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l], dst, m->dt, ldd,
+                              DLRM_ACT_RELU, st);
+            cur = dst;
+            cur_dt = m->dt;
+            cur_ld = ldd;
+        }
+        if (r != DLRM_OK) return r;
+    }
+    return DLRM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t dlrm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int dlrm_ld(int n, dlrm_dtype dt) {
+    const int per = 16 / (int)esize(dt);
+    return (n + per - 1) / per * per;
+}
+
+const char* dlrm_status_str(dlrm_status s) {
+    switch (s) {
+        case DLRM_OK: return "ok";
+        case DLRM_ERR_INVALID_ARG: return "invalid argument";
+        case DLRM_ERR_UNSUPPORTED: return "unsupported";
+        case DLRM_ERR_INDEX_OOB: return "index out of range (skipped)";
+        case DLRM_ERR_BAD_OFFSETS: return "bad bag offsets (bag pooled to zero)";
+        case DLRM_ERR_TIMEOUT: return "bounded wait timed out";
+        case DLRM_ERR_CUDA: return "CUDA error";
+        case DLRM_ERR_WORKSPACE: return "workspace too small or misaligned";
+    }
+    return "unknown status";
+}
+
+size_t dlrm_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int training) {
+    TableMeta tm;
+    if (check_tables(T, tm) != DLRM_OK || check_mlp(bot) != DLRM_OK || check_mlp(top) != DLRM_OK || B < 0) return 0;
+    (void)training;
+    return fwd_layout(T, bot, top, B).total;
+}
+
+dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info) {
+    if (!ws) return DLRM_ERR_INVALID_ARG;
+    ErrRecord h;
+    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess) return DLRM_ERR_CUDA;
+    if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return DLRM_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(h), cs(stream)) != cudaSuccess) return DLRM_ERR_CUDA;
+    if (info) {
+        info[0] = h.flags;
+        info[1] = (int64_t)h.n_oob;
+        info[2] = (int64_t)h.n_bad;
+    }
+    if (h.flags & ERR_BAD_OFFSETS) return DLRM_ERR_BAD_OFFSETS;
+    if (h.flags & ERR_OOB) return DLRM_ERR_INDEX_OOB;
+    if (h.flags & ERR_TIMEOUT) return DLRM_ERR_TIMEOUT;
+    return DLRM_OK;
+}
+
+dlrm_status dlrm_embbag_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_tables(T, tm);
+    if (r != DLRM_OK) return r;
+    if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (B > 0 && (!pooled || !aligned16(pooled))) return DLRM_ERR_INVALID_ARG;
+    if (B == 0) return DLRM_OK;
+    return launch_embbag(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, pooled, bag_len,
+                         static_cast<ErrRecord*>(ws), cs(stream));
+}
+
+dlrm_status dlrm_interact_fwd(int B, int K, int d, const float* x_dense, const float* pooled, void* concat, int ld,
+                              dlrm_dtype out_dt, dlrm_stream stream) {
+    if (B < 0 || K < 1 || d < 1 || !valid_dt(out_dt)) return DLRM_ERR_INVALID_ARG;
+    if (K > DLRM_MAX_TABLES) return DLRM_ERR_UNSUPPORTED;
+    if (ld < d + K * (K + 1) / 2) return DLRM_ERR_INVALID_ARG;
+    if (B == 0) return DLRM_OK;
+    if (!x_dense || !pooled || !concat || !aligned16(x_dense) || !aligned16(pooled) || !aligned16(concat))
+        return DLRM_ERR_INVALID_ARG;
+    return launch_interact(B, K, d, x_dense, pooled, concat, ld, out_dt, cs(stream));
+}
+
+dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                                     int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt,
+                                     void* ws, dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_tables(T, tm);
+    if (r != DLRM_OK) return r;
+    if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
+    if (!valid_dt(out_dt) || ld < T->d + T->K * (T->K + 1) / 2) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    if (!x_dense || !concat || !aligned16(x_dense) || !aligned16(concat)) return DLRM_ERR_INVALID_ARG;
+    return launch_embbag_interact(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, x_dense, concat, ld,
+                                  out_dt, static_cast<ErrRecord*>(ws), cs(stream));
+}
+
+dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out,
+                         int ld_out, int final_act, void* ws, dlrm_stream stream) {
+    dlrm_status r = check_mlp(mlp);
+    if (r != DLRM_OK) return r;
+    if (B < 0 || !valid_dt(in_dt) || ld_in < mlp->dims[0] || ld_out < mlp->dims[mlp->n_layers]) return DLRM_ERR_INVALID_ARG;
+    if (final_act < DLRM_ACT_NONE || final_act > DLRM_ACT_SIGMOID) return DLRM_ERR_INVALID_ARG;
+    if (B == 0) return DLRM_OK;
+    if (!in || !out) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    const size_t h = align_up(hidden_bytes(mlp, B), 256);
+    char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
+    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, cs(stream));
+}
+
+dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                         const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
+                         dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_tables(T, tm);
+    if (r != DLRM_OK) return r;
+    if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
+    if ((r = check_mlp(bot)) != DLRM_OK || (r = check_mlp(top)) != DLRM_OK) return r;
+    const int K = T->K, d = T->d;
+    if (bot->dims[bot->n_layers] != d || top->dims[0] != d + K * (K + 1) / 2 || top->dims[top->n_layers] != 1)
+        return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    if (!dense || !y_hat) return DLRM_ERR_INVALID_ARG;
+    const FwdLayout L = fwd_layout(T, bot, top, B);
+    char* w = static_cast<char*>(ws);
+    cudaStream_t st = cs(stream);
+    float* x_dense = reinterpret_cast<float*>(w + L.x_dense);
+    void* concat = w + L.concat;
+    const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
+    if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1, st)))
+        return r;
+    if ((r = launch_embbag_interact(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt,
+                                    reinterpret_cast<ErrRecord*>(w), st)))
+        return r;
+    return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, st);
+}
+
+}  // extern "C"

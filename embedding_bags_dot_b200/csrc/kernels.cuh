@@ -1,0 +1,29 @@
+// Launchers shared between the kernel files and the C ABI layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace dlrm {
+
+bool gather_supported(int d, dlrm_dtype dt);
+size_t interact_smem_per_sample(int K, int d);
+
+dlrm_status launch_embbag(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
+                          const int32_t* offsets, const int32_t* indices, long long nnz, float* pooled,
+                          int32_t* bag_len, ErrRecord* err, cudaStream_t st);
+
+dlrm_status launch_interact(int B, int K, int d, const float* x_dense, const float* pooled, void* out, int ld,
+                            dlrm_dtype out_dt, cudaStream_t st);
+
+dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
+                                   const int32_t* offsets, const int32_t* indices, long long nnz,
+                                   const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
+                                   cudaStream_t st);
+
+// One fully connected layer: C[M][N] = act(A[M][K] W[N][K]^T + bias), fp32 accumulation.
+// A has dtype a_dt (ld lda), W has dtype w_dt (ld ldw), C has dtype c_dt (ld ldc).
+dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                          dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
+                          cudaStream_t st);
+
+}  // namespace dlrm

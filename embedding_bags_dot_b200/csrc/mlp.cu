@@ -1,0 +1,164 @@
+// Fully connected layers y = act(x W^T + b) of the bottom and top MLPs
+// ("Deep Learning Recommendation Model (DLRM)", nadeemcite summary, Key Method
+// Details: FC layers with ReLU; "DLRM", briansu.co, section 4, equation
+// "Output": a sigmoid on the top MLP's output).
+//
+// This file holds the CUDA-core paths: a tiled FFMA GEMM used for fp32
+// layers and for layers the tensor-core path does not take, and a
+// warp-per-row GEMV for the single-logit last layer with its activation.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dlrm {
+
+template <int ACT>
+__device__ __forceinline__ float activate(float v) {
+    if constexpr (ACT == DLRM_ACT_RELU) return v > 0.f ? v : 0.f;
+    if constexpr (ACT == DLRM_ACT_SIGMOID) return 1.f / (1.f + expf(-v));
+    return v;
+}
+
+// 64 x 64 output tile per 256-thread block, 16-deep k slices through smem,
+// 4 x 4 outputs per thread.
+template <typename TA, typename TW, typename TC, int ACT>
+__global__ void __launch_bounds__(256) linear_ffma_kernel(int M, int N, int K, const TA* __restrict__ A, int lda,
+                                                          const TW* __restrict__ W, int ldw,
+                                                          const float* __restrict__ bias, TC* __restrict__ C,
+                                                          int ldc) {
+    __shared__ float As[16][64 + 4];
+    __shared__ float Ws[16][64 + 4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const long long m0 = (long long)blockIdx.y * 64;
+    const int n0 = blockIdx.x * 64;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    const int lr = threadIdx.x >> 2, lk = (threadIdx.x & 3) * 4;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int gk = k0 + lk + e;
+            const long long gm = m0 + lr;
+            const int gn = n0 + lr;
+            As[lk + e][lr] = (gm < M && gk < K) ? Cvt<TA>::to_f(A[gm * lda + gk]) : 0.f;
+            Ws[lk + e][lr] = (gn < N && gk < K) ? Cvt<TW>::to_f(W[(long long)gn * ldw + gk]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = As[kk][ty * 4 + i];
+                w[i] = Ws[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const long long m = m0 + ty * 4 + i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx * 4 + j;
+            if (n < N) C[m * ldc + n] = Cvt<TC>::from_f(activate<ACT>(acc[i][j] + bias[n]));
+        }
+    }
+}
+
+// N == 1: one warp per row.
+template <typename TA, typename TW, int ACT>
+__global__ void __launch_bounds__(256) gemv_kernel(int M, int K, const TA* __restrict__ A, int lda,
+                                                   const TW* __restrict__ w, const float* __restrict__ bias,
+                                                   float* __restrict__ y, int ldy) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const TA* a = A + row * lda;
+    float s = 0.f;
+    for (int k = lane; k < K; k += 32) s = fmaf(Cvt<TA>::to_f(a[k]), Cvt<TW>::to_f(w[k]), s);
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) y[row * ldy] = activate<ACT>(s + bias[0]);
+}
+
+template <typename TA, typename TW, typename TC, int ACT>
+static void run_ffma(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias, void* C,
+                     int ldc, cudaStream_t st) {
+    const dim3 grid((N + 63) / 64, (M + 63) / 64);
+    linear_ffma_kernel<TA, TW, TC, ACT><<<grid, 256, 0, st>>>(M, N, K, static_cast<const TA*>(A), lda,
+                                                              static_cast<const TW*>(W), ldw, bias,
+                                                              static_cast<TC*>(C), ldc);
+}
+
+template <typename TA, typename TW, int ACT>
+static void run_gemv(int M, int K, const void* A, int lda, const void* W, const float* bias, void* C, int ldc,
+                     cudaStream_t st) {
+    gemv_kernel<TA, TW, ACT><<<(M + 7) / 8, 256, 0, st>>>(M, K, static_cast<const TA*>(A), lda,
+                                                          static_cast<const TW*>(W), bias, static_cast<float*>(C), ldc);
+}
+
+template <typename TA, typename TW, typename TC>
+static void dispatch_act(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias,
+                         void* C, int ldc, int act, cudaStream_t st) {
+    if (act == DLRM_ACT_RELU) run_ffma<TA, TW, TC, DLRM_ACT_RELU>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+    else if (act == DLRM_ACT_SIGMOID) run_ffma<TA, TW, TC, DLRM_ACT_SIGMOID>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+    else run_ffma<TA, TW, TC, DLRM_ACT_NONE>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+}
+
+template <typename TA, typename TW>
+static dlrm_status dispatch_out(int M, int N, int K, const void* A, int lda, const void* W, int ldw,
+                                const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, cudaStream_t st) {
+    if (N == 1 && c_dt == DLRM_F32) {
+        if (act == DLRM_ACT_RELU) run_gemv<TA, TW, DLRM_ACT_RELU>(M, K, A, lda, W, bias, C, ldc, st);
+        else if (act == DLRM_ACT_SIGMOID) run_gemv<TA, TW, DLRM_ACT_SIGMOID>(M, K, A, lda, W, bias, C, ldc, st);
+        else run_gemv<TA, TW, DLRM_ACT_NONE>(M, K, A, lda, W, bias, C, ldc, st);
+        return DLRM_OK;
+    }
+    switch (c_dt) {
+        case DLRM_F32: dispatch_act<TA, TW, float>(M, N, K, A, lda, W, ldw, bias, C, ldc, act, st); break;
+        case DLRM_BF16: dispatch_act<TA, TW, __nv_bfloat16>(M, N, K, A, lda, W, ldw, bias, C, ldc, act, st); break;
+        case DLRM_F16: dispatch_act<TA, TW, __half>(M, N, K, A, lda, W, ldw, bias, C, ldc, act, st); break;
+    }
+    return DLRM_OK;
+}
+
+template <typename TA>
+static dlrm_status dispatch_w(int M, int N, int K, const void* A, int lda, const void* W, dlrm_dtype w_dt, int ldw,
+                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, cudaStream_t st) {
+    switch (w_dt) {
+        case DLRM_F32: return dispatch_out<TA, float>(M, N, K, A, lda, W, ldw, bias, C, c_dt, ldc, act, st);
+        case DLRM_BF16: return dispatch_out<TA, __nv_bfloat16>(M, N, K, A, lda, W, ldw, bias, C, c_dt, ldc, act, st);
+        case DLRM_F16: return dispatch_out<TA, __half>(M, N, K, A, lda, W, ldw, bias, C, c_dt, ldc, act, st);
+    }
+    return DLRM_ERR_UNSUPPORTED;
+}
+
+dlrm_status launch_linear_ffma(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                               dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc,
+                               int act, cudaStream_t st) {
+    dlrm_status r = DLRM_ERR_UNSUPPORTED;
+    switch (a_dt) {
+        case DLRM_F32: r = dispatch_w<float>(M, N, K, A, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st); break;
+        case DLRM_BF16: r = dispatch_w<__nv_bfloat16>(M, N, K, A, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st); break;
+        case DLRM_F16: r = dispatch_w<__half>(M, N, K, A, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st); break;
+    }
+    if (r != DLRM_OK) return r;
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                          dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
+                          cudaStream_t st) {
+    if (M == 0) return DLRM_OK;
+    return launch_linear_ffma(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st);
+}
+
+}  // namespace dlrm

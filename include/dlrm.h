@@ -1,0 +1,153 @@
+/*
+ * dlrm.h -- C ABI of the B200 (sm_100a) DLRM hot-path library, libdlrm.so.
+ *
+ * The operations follow the DLRM architecture as two pages state it:
+ *   [N] "Deep Learning Recommendation Model (DLRM)" (nadeemcite summary):
+ *       Core Idea; Key Method Details.
+ *   [S] "DLRM" (briansu.co/recsys/dlrm): section 3 "How it works";
+ *       section 4 "Key equations" (equations "Interaction" and "Output");
+ *       section 6 "Limitations & trade-offs".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are DEVICE pointers unless marked "host". The caller owns every
+ *    buffer (tables, weights, inputs, outputs, workspace); the library never
+ *    allocates device memory and keeps no pointer after a call returns.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *    Host-detectable argument errors return a status before anything is
+ *    launched. Errors found on the device (an index outside its table, bag
+ *    offsets that decrease or leave [0, nnz]) never trap: the offending
+ *    index contributes nothing, the offending bag pools to zero, and the
+ *    event is recorded in the error record at the start of the workspace;
+ *    dlrm_check_error() reads and clears it.
+ *  - Bags are CSR, table-major: bag (k, b) of table k and sample b holds
+ *    indices[offsets[k*B + b] .. offsets[k*B + b + 1]), each a row id local to
+ *    table k. offsets has K*B + 1 int32 entries; nnz < 2^31.
+ *  - All K tables live in one contiguous row-major buffer; table k starts at
+ *    row base_k = rows[0] + ... + rows[k-1]. Rows are d elements wide (all
+ *    features share d: [N] Key Method Details, [S] section 6).
+ *  - A matrix with a leading dimension `ld` stores row i at element i*ld;
+ *    ld must make every row start on a 16-byte boundary (dlrm_ld()). Padding
+ *    columns are never read by the library; outputs zero their padding.
+ *  - Limits: 1 <= K <= DLRM_MAX_TABLES; 1 <= d, and d*sizeof(elem) <= 2048
+ *    when d*sizeof(elem) is a multiple of 16, else d <= 256.
+ */
+#ifndef DLRM_H
+#define DLRM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DLRM_MAX_TABLES 256
+#define DLRM_MAX_LAYERS 16
+#define DLRM_ERR_RECORD_BYTES 256
+
+typedef struct CUstream_st* dlrm_stream; /* a cudaStream_t */
+
+typedef enum {
+    DLRM_OK = 0,
+    DLRM_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer or leading dimension */
+    DLRM_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement (dtype, d, K) */
+    DLRM_ERR_INDEX_OOB = 3,     /* device: some index was outside [0, m_k); it was skipped */
+    DLRM_ERR_BAD_OFFSETS = 4,   /* device: some bag had decreasing offsets or left [0, nnz]; it pooled to 0 */
+    DLRM_ERR_TIMEOUT = 5,       /* device: a bounded wait gave up */
+    DLRM_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch, copy) */
+    DLRM_ERR_WORKSPACE = 7      /* workspace too small or misaligned */
+} dlrm_status;
+
+typedef enum { DLRM_F32 = 0, DLRM_F16 = 1, DLRM_BF16 = 2 } dlrm_dtype;
+
+typedef enum { DLRM_ACT_NONE = 0, DLRM_ACT_RELU = 1, DLRM_ACT_SIGMOID = 2 } dlrm_act;
+
+/* K embedding tables of m_k x d ([N] Key Method Details). */
+typedef struct {
+    void* data;             /* device, all tables, row-major, 16-byte aligned */
+    const int64_t* rows;    /* host, K row counts m_k >= 1 */
+    int K;
+    int d;
+    dlrm_dtype dt;          /* storage dtype of the table values; pooling accumulates in fp32 */
+} dlrm_tables;
+
+/* A stack of fully connected layers y = act(x W^T + b) ([N] Key Method Details). */
+typedef struct {
+    int n_layers;           /* 1 .. DLRM_MAX_LAYERS */
+    const int* dims;        /* host, n_layers + 1 widths */
+    void* const* W;         /* host array of device pointers: W[l] is [dims[l+1]][dlrm_ld(dims[l], dt)] */
+    float* const* b;        /* host array of device pointers: b[l] is fp32 [dims[l+1]] */
+    dlrm_dtype dt;          /* dtype of weights and of hidden activations */
+} dlrm_mlp;
+
+/* Smallest leading dimension >= n whose rows are 16-byte multiples for dtype dt. */
+int dlrm_ld(int n, dlrm_dtype dt);
+
+/* Number of kernels this library has launched in the calling process so far
+ * (all devices, all streams). Used to count launches inside a timed region. */
+uint64_t dlrm_launch_count(void);
+
+/* Human-readable name of a status code (static string). */
+const char* dlrm_status_str(dlrm_status s);
+
+/* Bytes of device workspace dlrm_forward (training = 0) or dlrm_backward
+ * (training = 1) needs for batch B. Also enough for every single-step entry
+ * point on the same model and batch. The first DLRM_ERR_RECORD_BYTES bytes
+ * hold the error record: zero the whole workspace once after allocating it. */
+size_t dlrm_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int training);
+
+/* Reads the error record of `ws` (synchronising `stream`), clears it, and
+ * returns DLRM_ERR_BAD_OFFSETS if any bag had bad offsets, else
+ * DLRM_ERR_INDEX_OOB if any index was out of range, else DLRM_ERR_TIMEOUT if
+ * a bounded wait gave up, else DLRM_OK. If `info` (host, 3 entries) is not
+ * NULL it receives {flags, skipped indices, bad bags}. */
+dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info);
+
+/* Sum-pooled embedding bags ([S] section 3: each sparse feature looks up a
+ * row of its own table; a bag of several ids sums their rows, an empty bag
+ * gives zeros).
+ *   pooled   out, fp32 [B][K][d]
+ *   bag_len  out, optional (may be NULL): int32 [K*B], end - start of each bag
+ *            (0 for a bag with bad offsets)
+ *   ws       workspace holding the error record (>= DLRM_ERR_RECORD_BYTES) */
+dlrm_status dlrm_embbag_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, dlrm_stream stream);
+
+/* Pairwise dot-product interaction and concat ([S] section 4, equations
+ * "Interaction" and "Output"; [N] Core Idea: self-interactions excluded).
+ * With X = [x_dense; e_1; ...; e_K] ((K+1) x d), writes per sample the row
+ *   [x_dense (d values), Z_10, Z_20, Z_21, Z_30, ..., Z_K(K-1)],  Z_ij = <X_i, X_j>,
+ * i.e. d + K(K+1)/2 values, then zeros up to ld.
+ *   x_dense  fp32 [B][d];  pooled fp32 [B][K][d]
+ *   concat   out, [B][ld] of out_dt, ld >= d + K(K+1)/2 */
+dlrm_status dlrm_interact_fwd(int B, int K, int d, const float* x_dense, const float* pooled,
+                              void* concat, int ld, dlrm_dtype out_dt, dlrm_stream stream);
+
+/* dlrm_embbag_fwd fused with dlrm_interact_fwd: the pooled vectors stay on
+ * chip and only the concat rows are written. Same arguments and errors. */
+dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                                     int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt,
+                                     void* ws, dlrm_stream stream);
+
+/* MLP forward ([N] Key Method Details: FC layers with ReLU). ReLU after every
+ * hidden layer; after the last layer `final_act` (none, ReLU or sigmoid).
+ *   in    [B][ld_in] of in_dt, dims[0] logical columns
+ *   out   out, fp32 [B][ld_out], dims[n_layers] logical columns
+ *   ws    workspace from dlrm_workspace_size for this MLP as `top` (or bottom) */
+dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in,
+                         float* out, int ld_out, int final_act, void* ws, dlrm_stream stream);
+
+/* Whole forward pass ([S] sections 3-4):
+ *   y_hat = sigmoid(top([x_dense, vec(Z)])),  x_dense = bottom(dense) with ReLU after every bottom layer,
+ * hidden top layers with ReLU, last top layer linear (dims must end in 1).
+ *   dense  fp32 [B][bot->dims[0]];  y_hat out, fp32 [B] */
+dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                         const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat,
+                         void* ws, dlrm_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLRM_H */

@@ -1,0 +1,83 @@
+"""Helpers for the GPU parity tests: seeded models on the device and the
+element-wise tolerance rule.
+
+Tolerance (the same rule everywhere, applied element by element against the
+fp64 oracle): |gpu - oracle| <= rtol * (|oracle| + 1e-3 * max|oracle|) + atol
+with rtol = 1e-5, atol = 0 for fp32 tables and rtol = 2e-2, atol = 1e-3 for
+bf16 / fp16 tables. The 1e-3 * max term keeps entries that cancel to nearly
+zero (an fp32 dot product of length d carries an absolute error of order
+d * 2^-24 * |x||y|) from demanding more than fp32 can give.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import embedding_bags_dot_b200 as E
+from synth import device as sd
+from synth import gen
+
+TOL = {"f32": (1e-5, 0.0), "bf16": (2e-2, 1e-3), "f16": (2e-2, 1e-3)}
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64) if t.dtype != torch.float64 else t.cpu().numpy()
+
+
+def assert_close(got, want, dtype: str, what: str):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, f"{what}: shape {got.shape} vs {want.shape}"
+    if want.size == 0:
+        return
+    rtol, atol = TOL[dtype]
+    scale = float(np.abs(want).max())
+    lim = rtol * (np.abs(want) + 1e-3 * scale) + atol
+    err = np.abs(got - want)
+    bad = ~(err <= lim)
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(bad, err - lim, -np.inf)), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance ({dtype}); "
+                             f"worst at {i}: gpu {got[i]!r} oracle {want[i]!r} (max |oracle| {scale:.3g})")
+
+
+def max_rel(got, want) -> float:
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    den = np.abs(want) + 1e-3 * (np.abs(want).max() if want.size else 0) + 1e-300
+    return float((np.abs(got - want) / den).max()) if want.size else 0.0
+
+
+class GpuModel:
+    """A seeded model on cuda:0 wrapped for the C ABI."""
+
+    def __init__(self, cfg, on_device_fill=None, training=None):
+        self.cfg = cfg
+        self.tables = sd.tables_on_device(cfg, on_device_fill=on_device_fill)
+        self.T = E.Tables(self.tables, cfg.rows, cfg.d)
+        bW, bb, bd = sd.mlp_on_device(cfg, "bottom")
+        tW, tb, td = sd.mlp_on_device(cfg, "top")
+        self.bot = E.MLP(bW, bb, bd)
+        self.top = E.MLP(tW, tb, td)
+        tr = cfg.training if training is None else training
+        self.ws = E.alloc_workspace(E.dlrm_workspace_size(self.T, self.bot, self.top, cfg.B, int(tr)))
+
+    def forward(self, bt: dict, B=None):
+        B = self.cfg.B if B is None else B
+        y = torch.empty(B, dtype=torch.float32, device="cuda")
+        E.dlrm_forward(self.T, self.bot, self.top, B, bt["dense"], bt["offsets"], bt["indices"], y, self.ws)
+        return y
+
+
+def random_pooled(B, K, d, seed=0, scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((B, d)) * scale).astype(np.float32)
+    p = (rng.standard_normal((B, K, d)) * scale).astype(np.float32)
+    return x, p
+
+
+def concat_width(K, d):
+    return d + K * (K + 1) // 2
+
+
+def batch_dev(batch: gen.Batch):
+    return sd.batch_on_device(batch)
