@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import embedding_bags_dot_b200 as E
-from gpucase import GpuModel, assert_close, to_np
+from gpucase import GpuModel, assert_close, scale_pooled, to_np
 from oracle import oracle as O
 from synth import CONFIGS, gen, shrink
 from synth import device as sd
@@ -44,7 +44,7 @@ def test_out_of_range_indices_are_skipped_and_counted(tiny):
     assert counts == (25, 0)
     assert st == (E.ERR_INDEX_OOB, 1, 25, 0)
     assert np.array_equal(blen.cpu().numpy(), wlen)
-    assert_close(to_np(pooled), want, "f32", "pooled with skipped indices")
+    assert_close(to_np(pooled), want, "f32", "pooled with skipped indices", scale_pooled(model, cfg.B, batch.offsets, idx))
     # the record was cleared by the read
     assert E.dlrm_check_error(g.ws) == (0, 0, 0, 0)
 
@@ -63,7 +63,7 @@ def test_bad_offsets_pool_to_zero_and_are_counted(tiny):
     assert counts[1] >= 3
     assert st == (E.ERR_BAD_OFFSETS, 2 | (1 if counts[0] else 0), counts[0], counts[1])
     assert np.array_equal(blen.cpu().numpy(), wlen)
-    assert_close(to_np(pooled), want, "f32", "pooled with bad bags")
+    assert_close(to_np(pooled), want, "f32", "pooled with bad bags", scale_pooled(model, cfg.B, offs, batch.indices))
 
 
 def test_forward_records_errors_and_completes(tiny):

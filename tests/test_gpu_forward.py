@@ -4,7 +4,8 @@ import pytest
 import torch
 
 import embedding_bags_dot_b200 as E
-from gpucase import GpuModel, assert_close, batch_dev, concat_width, random_pooled, to_np
+from gpucase import (GpuModel, assert_close, batch_dev, concat_width, random_pooled, scale_concat,
+                     scale_mlp, scale_pooled, to_np)
 from oracle import oracle as O
 from synth import CONFIGS, gen, shrink
 from synth import device as sd
@@ -68,7 +69,9 @@ def test_embbag_fwd(name):
     want, wlen, counts = _oracle_pool(cfg, batch)
     assert st == (0, 0, counts[0], counts[1])
     assert np.array_equal(blen.cpu().numpy(), wlen)
-    assert_close(to_np(pooled), want, cfg.table_dtype, f"pooled {name}")
+    model = O.model_from_config(cfg)
+    sc = scale_pooled(model, cfg.B, batch.offsets, batch.indices)
+    assert_close(to_np(pooled), want, cfg.table_dtype, f"pooled {name}", sc)
 
 
 @pytest.mark.parametrize("K,d,dt", [(8, 16, "f32"), (26, 64, "f32"), (26, 128, "bf16"), (100, 64, "bf16"),
@@ -82,7 +85,7 @@ def test_interact_fwd(K, d, dt):
     torch.cuda.synchronize()
     want = O.interact(x, p)
     got = to_np(out)
-    assert_close(got[:, :want.shape[1]], want, dt, f"interaction K={K} d={d} {dt}")
+    assert_close(got[:, :want.shape[1]], want, dt, f"interaction K={K} d={d} {dt}", scale_concat(x, np.abs(p)))
     assert np.all(got[:, want.shape[1]:] == 0.0), "padding columns must be zero"
 
 
@@ -104,7 +107,9 @@ def test_embbag_interact_fwd(name):
     want = O.interact(x, pooled)
     got = to_np(out)
     tol_dt = "f32" if (cfg.table_dtype == "f32" and cfg.mlp_dtype == "f32") else "bf16"
-    assert_close(got[:, :want.shape[1]], want, tol_dt, f"fused concat {name}")
+    model = O.model_from_config(cfg)
+    sc = scale_concat(x, scale_pooled(model, cfg.B, batch.offsets, batch.indices))
+    assert_close(got[:, :want.shape[1]], want, tol_dt, f"fused concat {name}", sc)
     assert np.all(got[:, want.shape[1]:] == 0.0)
 
 
@@ -130,7 +135,8 @@ def test_mlp_fwd(name):
         want = O.mlp(Ws, bs, x_used, relu_last=(which == "bottom"))
         if which == "top":
             want = 1.0 / (1.0 + np.exp(-want))
-        assert_close(to_np(out), want, cfg.mlp_dtype, f"{which} MLP {name}")
+        sc = scale_mlp(Ws, bs, x_used, sigmoid=(which == "top"))
+        assert_close(to_np(out), want, cfg.mlp_dtype, f"{which} MLP {name}", sc)
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
