@@ -357,10 +357,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="smaller batch (profiling captures only)")
+    ap.add_argument("--rows-cap", type=int, default=None, help="cap table rows (profiling captures only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = CONFIGS[args.workload]
+    if args.batch or args.rows_cap:
+        from synth import shrink
+        cfg = shrink(cfg, B=args.batch, rows_cap=args.rows_cap, name=f"{cfg.name}-profile")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
