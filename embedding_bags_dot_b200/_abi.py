@@ -24,6 +24,7 @@ ACT_NONE, ACT_RELU, ACT_SIGMOID = 0, 1, 2
 MAX_TABLES = 256
 MAX_LAYERS = 16
 ERR_RECORD_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 DT_CODE = {"f32": F32, "f16": F16, "bf16": BF16, torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 DT_TORCH = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
@@ -63,6 +64,8 @@ _SIGS = {
                                C.c_void_p, C.c_void_p]),
     "dlrm_forward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
                                C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                       C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
 }
 
 
@@ -206,3 +209,12 @@ def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices,
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                      _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
                   "dlrm_forward")
+
+
+def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, err_flags=None,
+                         stream=None):
+    """dlrm_forward without a workspace: the library's fixed device scratch array is used instead
+    (for callers that cannot allocate device memory; see include/dlrm.h)."""
+    return _check(lib().dlrm_forward_noalloc(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
+                                             _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(err_flags),
+                                             _stream(stream)), "dlrm_forward_noalloc")

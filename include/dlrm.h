@@ -146,6 +146,43 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat,
                          void* ws, dlrm_stream stream);
 
+/* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
+#define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* dlrm_forward for callers that cannot allocate device memory. The pages
+ * describe no counterpart: this is a deployment convenience, not part of the
+ * method.
+ *
+ * Some callers are not allowed to call cudaMalloc: a plugin inside a host
+ * application or serving runtime that owns all device memory and hands the
+ * plugin only its input and output buffers; a latency-bound request path on
+ * which an allocation, and the device-wide synchronisation that
+ * cudaMalloc/cudaFree may cause, is not acceptable; a plain C caller with no
+ * device allocator. This entry point takes the same inputs and outputs as
+ * dlrm_forward but no workspace: its scratch is one fixed array of
+ * DLRM_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that
+ * loads the library holds until the process exits. It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ *  - Limit: dlrm_workspace_size(T, bot, top, B, 0) must not exceed
+ *    DLRM_NOALLOC_SCRATCH_BYTES; larger requests return DLRM_ERR_WORKSPACE
+ *    before anything is launched (split the batch, or use dlrm_forward).
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (with that device current). Make that first call before any
+ *    stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    previous call's contents. Calls whose work overlaps on the GPU (other
+ *    streams, other host threads) race on it; order them on one stream or
+ *    serialise them.
+ *  - Errors: device-detected input errors are handled as in dlrm_forward
+ *    (skipped index, empty bag). The error record is cleared at the start
+ *    of each call; if err_flags (device, optional) is not NULL it receives
+ *    this call's flags once the call's work completes: bit 0 = an index was
+ *    out of range, bit 1 = a bag had bad offsets. */
+dlrm_status dlrm_forward_noalloc(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
+                                 const float* dense, const int32_t* offsets, const int32_t* indices, int64_t nnz,
+                                 float* y_hat, uint32_t* err_flags, dlrm_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
