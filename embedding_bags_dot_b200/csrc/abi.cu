@@ -91,7 +91,7 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
 
 // The MLP chain: ReLU after hidden layers, final_act after the last layer.
 dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out, int ld_out,
-                    int final_act, void* act0, void* act1, cudaStream_t st) {
+                    int final_act, void* act0, void* act1, ErrRecord* err, cudaStream_t st) {
     const void* cur = in;
     dlrm_dtype cur_dt = in_dt;
     int cur_ld = ld_in;
@@ -101,12 +101,12 @@ dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, 
         dlrm_status r;
         if (l == m->n_layers - 1) {
             r = launch_linear(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l], out, DLRM_F32, ld_out,
-                              final_act, st);
+                              final_act, err, st);
         } else {
             void* dst = (l & 1) ? act1 : act0;
             const int ldd = dlrm_ld(N, m->dt);
             r = launch_linear(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l], dst, m->dt, ldd,
-                              DLRM_ACT_RELU, st);
+                              DLRM_ACT_RELU, err, st);
             cur = dst;
             cur_dt = m->dt;
             cur_ld = ldd;
@@ -215,7 +215,8 @@ dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype 
     if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
     const size_t h = align_up(hidden_bytes(mlp, B), 256);
     char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
-    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, cs(stream));
+    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, static_cast<ErrRecord*>(ws),
+                   cs(stream));
 }
 
 dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
@@ -238,12 +239,14 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
     float* x_dense = reinterpret_cast<float*>(w + L.x_dense);
     void* concat = w + L.concat;
     const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
-    if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1, st)))
+    ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
+    if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1, err,
+                     st)))
         return r;
     if ((r = launch_embbag_interact(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt,
                                     reinterpret_cast<ErrRecord*>(w), st)))
         return r;
-    return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, st);
+    return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, err, st);
 }
 
 }  // extern "C"

@@ -1,0 +1,407 @@
+// Tensor-core fully connected layer for 16-bit activations and weights:
+//   C[M][N] = act(A[M][K] W[N][K]^T + bias)      (fp32 accumulation in TMEM)
+// the bottom/top MLP layers of DLRM ("Deep Learning Recommendation Model
+// (DLRM)", nadeemcite summary, Key Method Details: FC layers with ReLU).
+//
+// sm_100a design: a persistent kernel, one 192-thread CTA per SM.
+//   warp 0      TMA producer: 128x64 tiles of A and 256x64 tiles of W (both
+//               K-major, 128-byte swizzle) into a 4-stage shared-memory ring;
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
+//               and one thread issues tcgen05.mma (M=128, N=256, K=16);
+//   warps 2..5  epilogue: tcgen05.ld of the finished accumulator (each warp
+//               owns the 32 TMEM lanes of its quadrant), bias, activation,
+//               conversion and global stores, while the MMA warp already
+//               fills the other accumulator.
+// Shared-memory stages are released by tcgen05.commit onto an mbarrier. All
+// waits are bounded: on timeout the kernel records DLRM_ERR_TIMEOUT in the
+// error record, drains its own copies and MMAs (again bounded), frees TMEM
+// and returns. No cluster multicast is used.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dlrm {
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr long long WAIT_LIMIT = 1ll << 26;
+
+struct Bars {
+    unsigned long long full[STAGES];
+    unsigned long long empty[STAGES];
+    unsigned long long tfull[2];
+    unsigned long long tempty[2];
+    unsigned long long drain;
+    unsigned int tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(unsigned long long* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(unsigned long long* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity to complete. Gives up
+// early when another role has already aborted (unless ignore_abort).
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, volatile int* abort,
+                                          bool ignore_abort = false) {
+    for (long long i = 0; i < WAIT_LIMIT; ++i) {
+        if (mbar_try(b, parity)) return true;
+        if (!ignore_abort && (i & 255) == 255 && *abort) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, unsigned long long* bar, int x,
+                                            int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand tile with 128-byte swizzle: 8-row groups of 1024 bytes.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
+    uint64_t d = (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;            // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;            // descriptor version
+    d |= (uint64_t)2 << 61;            // 128-byte swizzle
+    return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, A/B bf16 (1) or fp16 (0), both K-major.
+__host__ __device__ constexpr uint32_t idesc(int ab_fmt) {
+    return (1u << 4) | ((uint32_t)ab_fmt << 7) | ((uint32_t)ab_fmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accum) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(id), "r"(accum));
+}
+__device__ __forceinline__ void umma_commit(unsigned long long* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
+        "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_fn(float v) {
+    if constexpr (ACT == DLRM_ACT_RELU) return v > 0.f ? v : 0.f;
+    if constexpr (ACT == DLRM_ACT_SIGMOID) return 1.f / (1.f + expf(-v));
+    return v;
+}
+
+template <typename TC>
+__device__ __forceinline__ void store_chunk(TC* __restrict__ C, long long ldc, long long m, int n, int N, const float* v) {
+    TC* row = C + m * ldc;
+    if (n + 32 <= N) {
+        if constexpr (sizeof(TC) == 2) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                TC lo = Cvt<TC>::from_f(v[2 * j]), hi = Cvt<TC>::from_f(v[2 * j + 1]);
+                w[j] = (uint32_t)(*reinterpret_cast<uint16_t*>(&lo)) | ((uint32_t)(*reinterpret_cast<uint16_t*>(&hi)) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(row + n);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        } else {
+            float4* dst = reinterpret_cast<float4*>(row + n);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+    } else {
+        for (int j = 0; j < 32 && n + j < N; ++j) row[n + j] = Cvt<TC>::from_f(v[j]);
+    }
+}
+
+template <typename TC, int ACT>
+__global__ void __launch_bounds__(THREADS, 1)
+    linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, int M, int N,
+                     int K, const float* __restrict__ bias, TC* __restrict__ C, long long ldc, uint32_t id,
+                     ErrRecord* err) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = su32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    Bars* bars = reinterpret_cast<Bars*>(gbase + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nbn = (N + BN - 1) / BN;
+    const int ntiles = ((M + BM - 1) / BM) * nbn;
+    const int nk = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bars->tfull[a], 1);
+            mbar_init(&bars->tempty[a], 128);
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars->tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int* abort = &bars->abort;
+    bool timed_out = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW)) : "memory");
+            int s = 0;
+            uint32_t ph = 0;
+            for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x) {
+                const int mb = t / nbn, nb = t - mb * nbn;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&bars->empty[s], ph ^ 1u, abort)) {
+                        timed_out = true;
+                        break;
+                    }
+                    const uint32_t sa = base + s * STAGE_BYTES;
+                    mbar_expect_tx(&bars->full[s], STAGE_BYTES);
+                    tma_load_2d(sa, &mapA, &bars->full[s], kb * BK, mb * BM);
+                    tma_load_2d(sa + A_BYTES, &mapW, &bars->full[s], kb * BK, nb * BN);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (timed_out) {
+                *abort = 1;
+                // drain: every stage whose load may still be in flight completes its full phase
+                for (int q = 0; q < STAGES; ++q) {
+                    if (--s < 0) {
+                        s = STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    mbar_wait(&bars->full[s], ph, abort, true);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_ = id;
+            int s = 0;
+            uint32_t ph = 0;
+            int i = 0;
+            for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
+                const int acc = i & 1;
+                const uint32_t use = (uint32_t)(i >> 1);
+                if (!mbar_wait(&bars->tempty[acc], (use & 1u) ^ 1u, abort)) {
+                    timed_out = true;
+                    break;
+                }
+                fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&bars->full[s], ph, abort)) {
+                        timed_out = true;
+                        break;
+                    }
+                    fence_after();
+                    const uint32_t sa = base + s * STAGE_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma(d, sdesc(sa + k * 32), sdesc(sa + A_BYTES + k * 32), id_, (kb | k) != 0);
+                    umma_commit(&bars->empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (timed_out) break;
+                umma_commit(&bars->tfull[acc]);
+            }
+            if (timed_out) *abort = 1;
+            // all MMAs issued by this thread have completed once this fires
+            umma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0, abort, true);
+        }
+    } else {
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
+            const int acc = i & 1;
+            const uint32_t use = (uint32_t)(i >> 1);
+            if (!mbar_wait(&bars->tfull[acc], use & 1u, abort)) {
+                timed_out = true;
+                break;
+            }
+            fence_after();
+            const int mb = t / nbn, nb = t - mb * nbn;
+            const long long m = (long long)mb * BM + q * 32 + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = nb * BN + c * 32;
+                if (n0 >= N) break;  // uniform across the warp
+                uint32_t r[32];
+                tmem_ld32(taddr + c * 32, r);
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float b = (n0 + j < N) ? __ldg(bias + n0 + j) : 0.f;
+                    v[j] = act_fn<ACT>(__uint_as_float(r[j]) + b);
+                }
+                if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
+            }
+            fence_before();
+            mbar_arrive(&bars->tempty[acc]);
+        }
+        if (timed_out) *abort = 1;
+    }
+
+    if (timed_out && lane == 0) atomicOr(&err->flags, (unsigned)ERR_TIMEOUT);
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+static bool make_map(CUtensorMap* map, const void* ptr, dlrm_dtype dt, int inner, int outer, int ld, int box_outer) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType t = dt == DLRM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return enc(map, t, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+    static int n[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 148;
+    }
+    return n[dev];
+}
+
+template <typename TC, int ACT>
+static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, int M, int N, int K, const float* bias,
+                            void* C, int ldc, uint32_t id, ErrRecord* err, cudaStream_t st) {
+    auto kern = linear_tc_kernel<TC, ACT>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    const int ntiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = ntiles < sm_count() ? ntiles : sm_count();
+    kern<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mw, M, N, K, bias, static_cast<TC*>(C), (long long)ldc, id, err);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+}  // namespace tc
+
+bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
+                         int ldw, void* C, dlrm_dtype c_dt, int ldc) {
+    if (a_dt != w_dt || a_dt == DLRM_F32) return false;
+    if (M < 1 || N < 2 || K < 16) return false;
+    if ((lda % 8) || (ldw % 8)) return false;
+    if (((uintptr_t)A & 15) || ((uintptr_t)W & 15) || ((uintptr_t)C & 15)) return false;
+    if (c_dt != DLRM_F32 && c_dt != a_dt) return false;
+    if (ldc % (c_dt == DLRM_F32 ? 4 : 8)) return false;
+    return tc::encode_fn() != nullptr;
+}
+
+dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
+                             const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
+                             cudaStream_t st) {
+    CUtensorMap ma, mw;
+    if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) || !tc::make_map(&mw, W, a_dt, K, N, ldw, tc::BN))
+        return DLRM_ERR_CUDA;
+    const uint32_t id = tc::idesc(a_dt == DLRM_BF16 ? 1 : 0);
+#define DLRM_TC(TC)                                                                                             \
+    switch (act) {                                                                                              \
+        case DLRM_ACT_RELU: return tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st);       \
+        case DLRM_ACT_SIGMOID: return tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st); \
+        default: return tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st);                  \
+    }
+    if (c_dt == DLRM_F32) {
+        DLRM_TC(float)
+    } else if (c_dt == DLRM_BF16) {
+        DLRM_TC(__nv_bfloat16)
+    } else {
+        DLRM_TC(__half)
+    }
+#undef DLRM_TC
+}
+
+}  // namespace dlrm

@@ -22,8 +22,16 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
 
 // One fully connected layer: C[M][N] = act(A[M][K] W[N][K]^T + bias), fp32 accumulation.
 // A has dtype a_dt (ld lda), W has dtype w_dt (ld ldw), C has dtype c_dt (ld ldc).
+// Takes the tcgen05 path when linear_tc_supported(), else CUDA-core FFMA (or the N = 1 GEMV).
+// err receives DLRM_ERR_TIMEOUT if a bounded wait of the tensor-core kernel gives up.
 dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
-                          cudaStream_t st);
+                          ErrRecord* err, cudaStream_t st);
+
+bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
+                         int ldw, void* C, dlrm_dtype c_dt, int ldc);
+dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
+                             const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
+                             cudaStream_t st);
 
 }  // namespace dlrm

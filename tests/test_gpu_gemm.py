@@ -1,0 +1,72 @@
+"""Tensor-core (tcgen05) fully connected layer against the fp64 oracle, through
+dlrm_mlp_fwd with one layer, on shapes that exercise a single tile, ragged
+M / N / K edges, K below one 64-wide slice and many tiles per CTA.
+
+bf16 x bf16 products are exact in fp32 and the accumulation is fp32, so with
+an fp32 output the layer is held to the fp32 rule (rtol 1e-5 against the sum
+of |terms|); a layout or descriptor mistake shows up as O(1) errors."""
+import numpy as np
+import pytest
+import torch
+
+import embedding_bags_dot_b200 as E
+from gpucase import assert_close, scale_mlp, to_np
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TD = {"bf16": torch.bfloat16, "f16": torch.float16}
+
+
+def _layer(M, N, K, dt, seed):
+    g = torch.Generator().manual_seed(seed)
+    ld = E.dlrm_ld(K, dt)
+    x = torch.zeros((M, ld), dtype=TD[dt])
+    x[:, :K] = torch.randn((M, K), generator=g).to(TD[dt])
+    W = torch.zeros((N, ld), dtype=TD[dt])
+    W[:, :K] = (torch.randn((N, K), generator=g) / np.sqrt(K)).to(TD[dt])
+    b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
+    return x, W, b, ld
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (333, 200, 100), (1000, 1024, 479), (65, 40, 16),
+                                   (4096, 512, 1024), (300, 768, 256), (129, 257, 65)])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_linear_tc_fp32_out(M, N, K, dt):
+    x, W, b, ld = _layer(M, N, K, dt, seed=M * 7 + N + K)
+    mlp = E.MLP([W.cuda()], [b.cuda()], [K, N])
+    out = torch.full((M, N + 4 - N % 4 if N % 4 else N), float("nan"), device="cuda")
+    ldo = out.shape[1]
+    ws = E.alloc_workspace(1 << 20)
+    E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, ldo, E.ACT_NONE, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    xs = x[:, :K].double().numpy()
+    Ws = W[:, :K].double().numpy()
+    want = O.mlp([Ws], [b.double().numpy()], xs, relu_last=False)
+    assert_close(to_np(out)[:, :N], want, "f32", f"tc linear {M}x{N}x{K} {dt}", scale_mlp([Ws], [b.double().numpy()], xs))
+
+
+@pytest.mark.parametrize("act", [E.ACT_RELU, E.ACT_SIGMOID])
+def test_linear_tc_two_layers_bf16_hidden(act):
+    # hidden layer output is stored in bf16 (tcgen05 epilogue with ReLU); final layer fp32 with act
+    M, K, H, N = 777, 300, 512, 96
+    x, W1, b1, ld = _layer(M, K, K, "bf16", seed=1)
+    x = x[:, :ld]
+    g = torch.Generator().manual_seed(2)
+    W1 = torch.zeros((H, E.dlrm_ld(K, "bf16")), dtype=torch.bfloat16)
+    W1[:, :K] = (torch.randn((H, K), generator=g) / np.sqrt(K)).bfloat16()
+    b1 = torch.randn(H, generator=g) * 0.1
+    W2 = (torch.randn((N, H), generator=g) / np.sqrt(H)).bfloat16()
+    b2 = torch.randn(N, generator=g) * 0.1
+    mlp = E.MLP([W1.cuda(), W2.cuda()], [b1.cuda(), b2.cuda()], [K, H, N])
+    out = torch.empty((M, N), device="cuda")
+    ws = E.alloc_workspace(1 << 22)
+    E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, N, act, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    Ws = [W1[:, :K].double().numpy(), W2.double().numpy()]
+    bs = [b1.double().numpy(), b2.double().numpy()]
+    xs = x[:, :K].double().numpy()
+    want = O.mlp(Ws, bs, xs, relu_last=(act == E.ACT_RELU))
+    if act == E.ACT_SIGMOID:
+        want = 1 / (1 + np.exp(-want))
+    assert_close(to_np(out), want, "bf16", "two-layer bf16 MLP", scale_mlp(Ws, bs, xs, sigmoid=(act == E.ACT_SIGMOID)))
