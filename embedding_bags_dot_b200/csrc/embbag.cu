@@ -457,6 +457,8 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                    cudaStream_t st) {
     Geometry g;
     if (!gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
+    if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt))
+        return launch_embbag_interact_mma(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st);
     switch (dt) {
         case DLRM_F32: return launch_fused_t<float>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
         case DLRM_BF16: return launch_fused_t<__nv_bfloat16>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);

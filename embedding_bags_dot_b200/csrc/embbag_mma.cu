@@ -1,0 +1,332 @@
+// Fused gather + interaction for bf16 tables on the tensor cores.
+//
+// Same operation as embbag.cu's fused kernel: per sample b, pool the K bags
+// into e_1..e_K ("DLRM", briansu.co, section 3), form X = [x_dense; e_1..e_K]
+// and write [x_dense, Z_10, Z_20, Z_21, ...] with Z_ij = <X_i, X_j>, j < i
+// ("DLRM", briansu.co, section 4, equations "Interaction" and "Output").
+//
+// One warp owns one sample at a time:
+//  1. gather: lanes form groups of GL = d/8 lanes, one 16-byte chunk of a bf16
+//     row per lane; each group takes every (32/GL)-th table and issues the
+//     first row of up to TB bags before consuming any, so a warp keeps up to
+//     TB * 32/GL rows in flight. Bags with more rows add them in fp32; the
+//     pooled row is rounded to bf16 (exact for one-row bags of bf16 tables).
+//  2. x_dense (fp32) is split into hi = bf16(x) and lo = bf16(x - hi); hi is
+//     row 0 of X and lo row K+1, so that Z_i0 = G[i][0] + G[K+1][i] keeps the
+//     dense vector's fp32 precision.
+//  3. Gram G = X X^T of the Kp = 16*MT padded rows by mma.sync.m16n8k16
+//     (bf16 in, fp32 accumulate), lower-triangle tiles only. The same
+//     ldmatrix fragments serve as A and as B (B = X^T), so X is read from
+//     shared memory once per sample.
+//  4. G is staged in shared memory and the warp writes the concat row with
+//     16-byte stores (bf16 output) or element stores.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dlrm {
+
+namespace {
+
+constexpr int WARPS = 8;
+constexpr int SPW = 2;               // samples per warp per block
+constexpr int S = WARPS * SPW;       // samples per block
+constexpr int TB = 8;                // bags per group whose first row is loaded before any is consumed
+
+__device__ __forceinline__ void bf16x8_add(const uint4& v, float* a) { Chunk16<__nv_bfloat16>::add(v, a); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+}  // namespace
+
+// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2). GL: lanes per row (d = 8 GL).
+template <int MT, int GL>
+__global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_mma_kernel(
+    const __nv_bfloat16* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
+    const float* __restrict__ x_dense, void* out, int ld, int out_dt, int warp_bytes, ErrRecord* err) {
+    constexpr int d = 8 * GL;
+    constexpr int KP = 16 * MT;
+    constexpr int RS = 2 * d + 16;   // X row stride in bytes (odd multiple of 16: conflict-free ldmatrix)
+    constexpr int GS = KP + 1;       // G row stride in floats
+    constexpr int NG = 32 / GL;      // row groups per warp
+    constexpr int NTILE = MT * (MT + 1);
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = K * (K + 1) / 2;
+    const int L = K + 1;             // row holding the low half of x_dense
+    unsigned char* xw = smem + (size_t)warp * warp_bytes;
+    unsigned char* tail = smem + (size_t)WARPS * warp_bytes;
+    int* off_s = reinterpret_cast<int*>(tail);
+    unsigned char* bad_s = reinterpret_cast<unsigned char*>(off_s + K * (S + 1));
+    uint16_t* src1 = reinterpret_cast<uint16_t*>(bad_s + ((K * S + 15) & ~15));
+    uint16_t* src2 = src1 + ld;
+
+    const int b0 = blockIdx.x * S;
+    const int nb = min(S, B - b0);
+    unsigned oob = 0, bad = 0;
+
+    // ---- block prologue: offsets of the tile, bad-bag flags, concat column sources
+    for (int q = threadIdx.x; q < K * (nb + 1); q += blockDim.x) {
+        const int k = q / (nb + 1), s = q - k * (nb + 1);
+        off_s[k * (S + 1) + s] = offsets[(long long)k * B + b0 + s];
+    }
+    for (int c = threadIdx.x; c < ld; c += blockDim.x) {
+        uint16_t s1 = 0xFFFFu, s2 = 0xFFFFu;
+        const int p = c - d;
+        if (p >= 0 && p < P) {
+            int i = (int)((1.0f + sqrtf(8.0f * (float)p + 1.0f)) * 0.5f);
+            while (i * (i - 1) / 2 > p) --i;
+            while ((i + 1) * i / 2 <= p) ++i;
+            const int j = p - i * (i - 1) / 2;
+            s1 = (uint16_t)(i * GS + j);
+            if (j == 0) s2 = (uint16_t)(L * GS + i);
+        }
+        src1[c] = s1;
+        src2[c] = s2;
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < K * nb; q += blockDim.x) {
+        const int k = q / nb, s = q - k * nb;
+        const long long st = off_s[k * (S + 1) + s], en = off_s[k * (S + 1) + s + 1];
+        const bool isbad = st < 0 || en < st || en > nnz;
+        bad_s[k * S + s] = isbad;
+        bad += isbad;
+    }
+    __syncthreads();
+
+    const uint32_t xw_s = (uint32_t)__cvta_generic_to_shared(xw);
+    float* G = reinterpret_cast<float*>(xw + RS);
+    const int gi = lane / GL, g = lane % GL;
+
+    for (int r = 0; r < SPW; ++r) {
+        const int s = warp * SPW + r;
+        if (s >= nb) break;
+        const long long b = b0 + s;
+
+        // zero the padding rows K+2 .. KP-1
+        for (int q = lane; q < (KP - K - 2) * (RS / 16); q += 32)
+            reinterpret_cast<uint4*>(xw + (size_t)(K + 2) * RS)[q] = make_uint4(0, 0, 0, 0);
+
+        // ---- 1. gather the K pooled rows into X rows 1..K (bf16)
+        for (int k0 = gi; k0 < K; k0 += NG * TB) {
+            uint4 v[TB];
+            int st[TB], en[TB];
+#pragma unroll
+            for (int u = 0; u < TB; ++u) {
+                const int k = k0 + u * NG;
+                st[u] = 0;
+                en[u] = 0;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (k < K && !bad_s[k * S + s]) {
+                    st[u] = off_s[k * (S + 1) + s];
+                    en[u] = off_s[k * (S + 1) + s + 1];
+                    if (en[u] > st[u]) {
+                        const int idx = __ldg(indices + st[u]);
+                        if (idx >= 0 && (long long)idx < tm.rows[k])
+                            v[u] = ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g);
+                        else if (g == 0)
+                            ++oob;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < TB; ++u) {
+                const int k = k0 + u * NG;
+                if (k < K) {
+                    uint4 packed = v[u];
+                    if (en[u] - st[u] > 1) {
+                        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        bf16x8_add(v[u], a);
+                        for (int p = st[u] + 1; p < en[u]; ++p) {
+                            const int idx = __ldg(indices + p);
+                            if (idx >= 0 && (long long)idx < tm.rows[k])
+                                bf16x8_add(ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g), a);
+                            else if (g == 0)
+                                ++oob;
+                        }
+                        packed = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                                            pack_bf16(a[6], a[7]));
+                    }
+                    *reinterpret_cast<uint4*>(xw + (size_t)(k + 1) * RS + 16 * g) = packed;
+                }
+            }
+        }
+
+        // ---- 2. x_dense -> rows 0 (hi) and K+1 (lo)
+        for (int c = 4 * lane; c < d; c += 128) {
+            const float4 x = *reinterpret_cast<const float4*>(x_dense + b * d + c);
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
+            const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+            const uint32_t lo01 = pack_bf16(x.x - f01.x, x.y - f01.y), lo23 = pack_bf16(x.z - f23.x, x.w - f23.y);
+            *reinterpret_cast<uint2*>(xw + 2 * c) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+            *reinterpret_cast<uint2*>(xw + (size_t)L * RS + 2 * c) = make_uint2(lo01, lo23);
+        }
+        __syncwarp();
+
+        // ---- 3. lower-triangle Gram tiles on the tensor cores
+        float acc[NTILE][4];
+#pragma unroll
+        for (int t = 0; t < NTILE; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < d / 16; ++ks) {
+            uint32_t a[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+                ldmatrix_x4(xw_s + (uint32_t)((16 * mt + (lane & 15)) * RS + ks * 32 + (lane >> 4) * 16), a[mt]);
+            int t = 0;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                for (int nt = 0; nt <= 2 * mt + 1; ++nt, ++t) {
+                    const uint32_t b0r = a[nt >> 1][(nt & 1) ? 1 : 0];
+                    const uint32_t b1r = a[nt >> 1][(nt & 1) ? 3 : 2];
+                    mma_bf16(acc[t], a[mt], b0r, b1r);
+                }
+            }
+        }
+        __syncwarp();  // every lane's ldmatrix of X is done before G overwrites it
+
+        // ---- 4. stage G (rows 0..KP-1, row stride GS floats, starting after X row 0)
+        {
+            const int gr = lane >> 2, tc = (lane & 3) * 2;
+            int t = 0;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                for (int nt = 0; nt <= 2 * mt + 1; ++nt, ++t) {
+                    float* p0 = G + (16 * mt + gr) * GS + 8 * nt + tc;
+                    float* p1 = p0 + 8 * GS;
+                    p0[0] = acc[t][0];
+                    p0[1] = acc[t][1];
+                    p1[0] = acc[t][2];
+                    p1[1] = acc[t][3];
+                }
+            }
+        }
+        __syncwarp();
+
+        // ---- 5. concat row: x_dense (hi = bf16(x)), Z, zero padding
+        if (out_dt == DLRM_BF16) {
+            uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + b * ld);
+            for (int c8 = lane; c8 < ld / 8; c8 += 32) {
+                const int c = 8 * c8;
+                if (c + 8 <= d) {
+                    orow[c8] = *reinterpret_cast<const uint4*>(xw + 2 * c);
+                } else {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int cc = c + e;
+                        float val = 0.f;
+                        if (cc < d) {
+                            val = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[cc]);
+                        } else {
+                            const uint16_t i1 = src1[cc], i2 = src2[cc];
+                            if (i1 != 0xFFFFu) val = G[i1];
+                            if (i2 != 0xFFFFu) val += G[i2];
+                        }
+                        f[e] = val;
+                    }
+                    orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                          pack_bf16(f[6], f[7]));
+                }
+            }
+        } else {
+            for (int c = lane; c < ld; c += 32) {
+                float val = 0.f;
+                if (c < d) {
+                    val = x_dense[b * d + c];
+                } else {
+                    const uint16_t i1 = src1[c], i2 = src2[c];
+                    if (i1 != 0xFFFFu) val = G[i1];
+                    if (i2 != 0xFFFFu) val += G[i2];
+                }
+                store_as(out, (size_t)b * ld + c, val, out_dt);
+            }
+        }
+        __syncwarp();  // X / G reused by the next sample
+    }
+    report_warp(err, oob, bad);
+}
+
+// ------------------------------------------------------------------ host side
+
+static int mma_warp_bytes(int K, int d, int& MT) {
+    MT = (K + 2 + 15) / 16;
+    const int KP = 16 * MT;
+    const int RS = 2 * d + 16;
+    const int x = KP * RS;
+    const int gbytes = RS + KP * (KP + 1) * 4;
+    return ((x > gbytes ? x : gbytes) + 15) & ~15;
+}
+
+static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
+    warp_bytes = mma_warp_bytes(K, d, MT);
+    return (size_t)WARPS * warp_bytes + sizeof(int) * (size_t)K * (S + 1) + (((size_t)K * S + 15) & ~(size_t)15) +
+           2 * sizeof(uint16_t) * (size_t)ld;
+}
+
+bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt) {
+    if (dt != DLRM_BF16) return false;
+    if (!(d == 32 || d == 64 || d == 128 || d == 256)) return false;
+    if (K + 2 > 64) return false;
+    if (out_dt == DLRM_BF16 && (ld % 8 || ((uintptr_t)out & 15))) return false;
+    int MT, wb;
+    const int P = K * (K + 1) / 2;
+    if ((K + 2) * (K + 3) > 0xFFFF || ld > 0x7FFF || P + d > ld) return false;
+    return mma_smem(K, d, ld, MT, wb) <= 227 * 1024;
+}
+
+template <int MT, int GL>
+static void launch_mma_t(const TableMeta& tm, const void* tables, int K, int B, const int32_t* offsets,
+                         const int32_t* indices, long long nnz, const float* x_dense, void* out, int ld, int out_dt,
+                         int warp_bytes, size_t smem, ErrRecord* err, cudaStream_t st) {
+    auto kern = embbag_interact_mma_kernel<MT, GL>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<(B + S - 1) / S, WARPS * 32, smem, st>>>(static_cast<const __nv_bfloat16*>(tables), tm, K, B, offsets,
+                                                    indices, nnz, x_dense, out, ld, out_dt, warp_bytes, err);
+}
+
+dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, int K, int d, int B,
+                                       const int32_t* offsets, const int32_t* indices, long long nnz,
+                                       const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
+                                       cudaStream_t st) {
+    int MT, wb;
+    const size_t smem = mma_smem(K, d, ld, MT, wb);
+#define DLRM_MMA_GL(MTV)                                                                                       \
+    switch (d) {                                                                                               \
+        case 32: launch_mma_t<MTV, 4>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \
+        case 64: launch_mma_t<MTV, 8>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \
+        case 128: launch_mma_t<MTV, 16>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break; \
+        default: launch_mma_t<MTV, 32>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;  \
+    }
+    switch (MT) {
+        case 1: DLRM_MMA_GL(1) break;
+        case 2: DLRM_MMA_GL(2) break;
+        case 3: DLRM_MMA_GL(3) break;
+        default: DLRM_MMA_GL(4) break;
+    }
+#undef DLRM_MMA_GL
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+}  // namespace dlrm

@@ -20,6 +20,14 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                    const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                    cudaStream_t st);
 
+// Tensor-core (mma.sync) variant of launch_embbag_interact for bf16 tables with
+// d in {32, 64, 128, 256} and K + 2 <= 64; launch_embbag_interact picks it when supported.
+bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt);
+dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, int K, int d, int B,
+                                       const int32_t* offsets, const int32_t* indices, long long nnz,
+                                       const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
+                                       cudaStream_t st);
+
 // One fully connected layer: C[M][N] = act(A[M][K] W[N][K]^T + bias), fp32 accumulation.
 // A has dtype a_dt (ld lda), W has dtype w_dt (ld ldw), C has dtype c_dt (ld ldc).
 // Takes the tcgen05 path when linear_tc_supported(), else CUDA-core FFMA (or the N = 1 GEMV).

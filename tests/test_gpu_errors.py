@@ -16,9 +16,14 @@ from synth import device as sd
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def tiny():
-    cfg = shrink(CONFIGS["tiny"], B=70).with_(bag="mix", seed=4)
+@pytest.fixture(scope="module", params=["f32", "bf16"])
+def tiny(request):
+    # bf16 with d = 16 x 8 = 128 takes the tensor-core fused path; f32 the CUDA-core one
+    if request.param == "f32":
+        cfg = shrink(CONFIGS["tiny"], B=70).with_(bag="mix", seed=4)
+    else:
+        cfg = shrink(CONFIGS["large"], B=70, rows_cap=1000).with_(rows=(1000,) * 8, bag="mix", seed=4,
+                                                                  top=(128 + 36, 64, 1))
     return cfg, gen.make_batches(cfg, (0,))[0], GpuModel(cfg)
 
 
@@ -36,7 +41,7 @@ def test_out_of_range_indices_are_skipped_and_counted(tiny):
     rng = np.random.default_rng(0)
     pos = rng.choice(idx.size, 25, replace=False)
     idx[pos[:10]] = -1
-    idx[pos[10:20]] = 1000            # == m_k: one past the end
+    idx[pos[10:20]] = cfg.rows[0]     # == m_k: one past the end
     idx[pos[20:]] = 2 ** 31 - 1
     pooled, blen, st = _run_pool(cfg, g, batch.offsets, idx)
     model = O.model_from_config(cfg)
@@ -44,7 +49,8 @@ def test_out_of_range_indices_are_skipped_and_counted(tiny):
     assert counts == (25, 0)
     assert st == (E.ERR_INDEX_OOB, 1, 25, 0)
     assert np.array_equal(blen.cpu().numpy(), wlen)
-    assert_close(to_np(pooled), want, "f32", "pooled with skipped indices", scale_pooled(model, cfg.B, batch.offsets, idx))
+    assert_close(to_np(pooled), want, cfg.table_dtype, "pooled with skipped indices",
+                 scale_pooled(model, cfg.B, batch.offsets, idx))
     # the record was cleared by the read
     assert E.dlrm_check_error(g.ws) == (0, 0, 0, 0)
 
@@ -63,13 +69,14 @@ def test_bad_offsets_pool_to_zero_and_are_counted(tiny):
     assert counts[1] >= 3
     assert st == (E.ERR_BAD_OFFSETS, 2 | (1 if counts[0] else 0), counts[0], counts[1])
     assert np.array_equal(blen.cpu().numpy(), wlen)
-    assert_close(to_np(pooled), want, "f32", "pooled with bad bags", scale_pooled(model, cfg.B, offs, batch.indices))
+    assert_close(to_np(pooled), want, cfg.table_dtype, "pooled with bad bags",
+                 scale_pooled(model, cfg.B, offs, batch.indices))
 
 
 def test_forward_records_errors_and_completes(tiny):
     cfg, batch, g = tiny
     idx = batch.indices.copy()
-    idx[::7] = 5000
+    idx[::7] = 50000
     bt = sd.batch_on_device(batch)
     bt["indices"] = torch.from_numpy(idx).cuda()
     y = g.forward(bt)
@@ -77,7 +84,7 @@ def test_forward_records_errors_and_completes(tiny):
     model = O.model_from_config(cfg)
     want, _, counts = O.forward(model, batch.dense, batch.offsets, idx)
     assert st == (E.ERR_INDEX_OOB, 1, counts[0], 0)
-    assert_close(to_np(y), want, "f32", "forward with skipped indices")
+    assert_close(to_np(y), want, cfg.table_dtype, "forward with skipped indices")
 
 
 def test_host_argument_errors(tiny):
@@ -130,4 +137,4 @@ def test_all_bags_empty(tiny):
                    "indices": torch.zeros(0, dtype=torch.int32, device="cuda")})
     model = O.model_from_config(cfg)
     want, _, _ = O.forward(model, batch.dense, offs, idx)
-    assert_close(to_np(y), want, "f32", "forward with empty bags")
+    assert_close(to_np(y), want, cfg.table_dtype, "forward with empty bags")

@@ -29,6 +29,13 @@ def _cases():
         "f32-d512-K3": shrink(t, B=19, rows_cap=300).with_(rows=(300, 17, 5), d=512, bag="poisson20",
                                                            bottom=(13, 32, 512), top=(512 + 6, 16, 1)),
         "bf16-K1": shrink(l, B=33, rows_cap=100).with_(rows=(100,), bottom=(13, 16, 128), top=(129, 8, 1)),
+        # tensor-core fused path: multi-hot and empty bags, every supported width and tile count
+        "bf16-d64-K40-mix": shrink(m, B=83).with_(rows=(2000,) * 40, table_dtype="bf16", mlp_dtype="bf16", bag="mix",
+                                                   bottom=(13, 32, 64), top=(64 + 820, 32, 1)),
+        "bf16-d256-K8-mix": shrink(t, B=51, rows_cap=400).with_(d=256, table_dtype="bf16", mlp_dtype="bf16",
+                                                                bag="mix", bottom=(13, 32, 256), top=(256 + 36, 32, 1)),
+        "bf16-d32-K62": shrink(t, B=35).with_(rows=(300,) * 62, d=32, table_dtype="bf16", mlp_dtype="bf16",
+                                               bottom=(13, 16, 32), top=(32 + 1953, 16, 1)),
     }
 
 
@@ -164,3 +171,28 @@ def test_two_batches_back_to_back_are_independent():
     assert np.array_equal(y0, y0b), "same inputs must give bit-identical outputs"
     model = O.model_from_config(cfg)
     assert_close(y1, O.forward(model, b1.dense, b1.offsets, b1.indices)[0], "f32", "second batch")
+
+
+@pytest.mark.parametrize("name", ["large-small", "bf16-K1", "bf16-d32-K62"])
+def test_fused_bf16_one_hot_keeps_fp32_precision(name):
+    """One-row bags of bf16 tables are exact in bf16 and x_dense is split into
+    two bf16 halves, so the tensor-core Gram with an fp32 output is accurate to
+    about 2^-16 of the terms' magnitude (checked at 1e-4)."""
+    cfg = CASES[name]
+    batch = gen.make_batches(cfg, (0,))[0]
+    g = GpuModel(cfg)
+    bt = batch_dev(batch)
+    x = np.random.default_rng(9).standard_normal((cfg.B, cfg.d)).astype(np.float32)
+    ld = E.dlrm_ld(cfg.concat_width, "f32")
+    out = torch.full((cfg.B, ld), float("nan"), device="cuda")
+    E.dlrm_embbag_interact_fwd(g.T, cfg.B, bt["offsets"], bt["indices"], torch.from_numpy(x).cuda(), out, ld, "f32",
+                               g.ws)
+    assert E.dlrm_check_error(g.ws)[0] == 0
+    model = O.model_from_config(cfg)
+    pooled, _, _ = O.embbag(model.tables, cfg.rows, cfg.d, cfg.B, batch.offsets, batch.indices)
+    want = O.interact(x, pooled)
+    got = to_np(out)
+    sc = scale_concat(x, scale_pooled(model, cfg.B, batch.offsets, batch.indices))
+    err = np.abs(got[:, :want.shape[1]] - want)
+    assert np.all(err <= 1e-4 * (np.abs(want) + sc)), float((err / (np.abs(want) + sc)).max())
+    assert np.all(got[:, want.shape[1]:] == 0)
