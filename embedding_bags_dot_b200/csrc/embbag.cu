@@ -457,7 +457,7 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                    cudaStream_t st) {
     Geometry g;
     if (!gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
-    if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt))
+    if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt, tm.base[K - 1] + tm.rows[K - 1]))
         return launch_embbag_interact_mma(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st);
     switch (dt) {
         case DLRM_F32: return launch_fused_t<float>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);

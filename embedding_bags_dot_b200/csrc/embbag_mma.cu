@@ -5,21 +5,23 @@
 // and write [x_dense, Z_10, Z_20, Z_21, ...] with Z_ij = <X_i, X_j>, j < i
 // ("DLRM", briansu.co, section 4, equations "Interaction" and "Output").
 //
-// One warp owns one sample at a time:
+// Block prologue (all threads): the tile's CSR offsets are read once,
+// coalesced, and every bag is resolved to a code: the global row of a
+// one-row bag, "empty" (no rows, bad offsets or an out-of-range index), or
+// "several rows". Then one warp owns one sample at a time:
 //  1. gather: lanes form groups of GL = d/8 lanes, one 16-byte chunk of a bf16
-//     row per lane; each group takes every (32/GL)-th table and issues the
-//     first row of up to TB bags before consuming any, so a warp keeps up to
-//     TB * 32/GL rows in flight. Bags with more rows add them in fp32; the
-//     pooled row is rounded to bf16 (exact for one-row bags of bf16 tables).
+//     row per lane. A one-row bag is copied global -> shared with cp.async,
+//     so every row of the sample is in flight at once without registers;
+//     a bag of several rows is summed in fp32 and rounded to bf16.
 //  2. x_dense (fp32) is split into hi = bf16(x) and lo = bf16(x - hi); hi is
 //     row 0 of X and lo row K+1, so that Z_i0 = G[i][0] + G[K+1][i] keeps the
 //     dense vector's fp32 precision.
-//  3. Gram G = X X^T of the Kp = 16*MT padded rows by mma.sync.m16n8k16
-//     (bf16 in, fp32 accumulate), lower-triangle tiles only. The same
-//     ldmatrix fragments serve as A and as B (B = X^T), so X is read from
-//     shared memory once per sample.
-//  4. G is staged in shared memory and the warp writes the concat row with
-//     16-byte stores (bf16 output) or element stores.
+//  3. Gram G = X X^T over the Kp = 16*MT padded rows with
+//     mma.sync.m16n8k16 (bf16 in, fp32 accumulate), lower-triangle tiles only.
+//     The same ldmatrix fragments serve as A and as B (B = X^T), so X is read
+//     from shared memory once per sample.
+//  4. G is staged in shared memory; each lane owns fixed 8-column chunks of
+//     the concat row, whose sources in G are computed once per block.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -30,9 +32,9 @@ namespace {
 constexpr int WARPS = 8;
 constexpr int SPW = 2;               // samples per warp per block
 constexpr int S = WARPS * SPW;       // samples per block
-constexpr int TB = 8;                // bags per group whose first row is loaded before any is consumed
-
-__device__ __forceinline__ void bf16x8_add(const uint4& v, float* a) { Chunk16<__nv_bfloat16>::add(v, a); }
+constexpr uint32_t CODE_EMPTY = 0xFFFFFFFFu;
+constexpr uint32_t CODE_MULTI = 0xFFFFFFFEu;
+constexpr int SRC_CACHE = 2;         // concat chunks per lane whose sources stay in registers
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -53,6 +55,33 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// Source of concat column c in the staged Gram G (row stride GS): i*GS + j for
+// Z_ij, 0xFFFF for a padding column. Columns below d come from x_dense.
+__device__ __forceinline__ uint32_t column_source(int c, int d, int P, int GS) {
+    const int p = c - d;
+    if (p < 0 || p >= P) return 0xFFFFu;
+    int i = (int)((1.0f + sqrtf(8.0f * (float)p + 1.0f)) * 0.5f);
+    while (i * (i - 1) / 2 > p) --i;
+    while ((i + 1) * i / 2 <= p) ++i;
+    return (uint32_t)(i * GS + (p - i * (i - 1) / 2));
+}
+
+// Z_ij from G; for j = 0 the low half of x_dense (row L) adds G[L][i].
+template <int GS>
+__device__ __forceinline__ float column_value(uint32_t s1, const float* G, int L) {
+    if (s1 == 0xFFFFu) return 0.f;
+    float v = G[s1];
+    if (s1 % GS == 0) v += G[L * GS + s1 / GS];
+    return v;
+}
+
 }  // namespace
 
 // MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2). GL: lanes per row (d = 8 GL).
@@ -64,7 +93,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     constexpr int d = 8 * GL;
     constexpr int KP = 16 * MT;
     constexpr int RS = 2 * d + 16;   // X row stride in bytes (odd multiple of 16: conflict-free ldmatrix)
-    constexpr int GS = KP + 1;       // G row stride in floats
+    constexpr int GS = KP + 8;       // G row stride in floats (float2 staging without bank conflicts)
     constexpr int NG = 32 / GL;      // row groups per warp
     constexpr int NTILE = MT * (MT + 1);
     extern __shared__ __align__(16) unsigned char smem[];
@@ -74,42 +103,51 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     unsigned char* xw = smem + (size_t)warp * warp_bytes;
     unsigned char* tail = smem + (size_t)WARPS * warp_bytes;
     int* off_s = reinterpret_cast<int*>(tail);
-    unsigned char* bad_s = reinterpret_cast<unsigned char*>(off_s + K * (S + 1));
-    uint16_t* src1 = reinterpret_cast<uint16_t*>(bad_s + ((K * S + 15) & ~15));
-    uint16_t* src2 = src1 + ld;
+    uint32_t* code_s = reinterpret_cast<uint32_t*>(off_s + K * (S + 1));
+    uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + K * S);
+    const int nchunk = ld / 8;
+    const bool bf16_out = out_dt == DLRM_BF16;
 
     const int b0 = blockIdx.x * S;
     const int nb = min(S, B - b0);
     unsigned oob = 0, bad = 0;
 
-    // ---- block prologue: offsets of the tile, bad-bag flags, concat column sources
+    // ---- block prologue: tile offsets, bag codes, concat column sources
     for (int q = threadIdx.x; q < K * (nb + 1); q += blockDim.x) {
         const int k = q / (nb + 1), s = q - k * (nb + 1);
         off_s[k * (S + 1) + s] = offsets[(long long)k * B + b0 + s];
     }
-    for (int c = threadIdx.x; c < ld; c += blockDim.x) {
-        uint16_t s1 = 0xFFFFu, s2 = 0xFFFFu;
-        const int p = c - d;
-        if (p >= 0 && p < P) {
-            int i = (int)((1.0f + sqrtf(8.0f * (float)p + 1.0f)) * 0.5f);
-            while (i * (i - 1) / 2 > p) --i;
-            while ((i + 1) * i / 2 <= p) ++i;
-            const int j = p - i * (i - 1) / 2;
-            s1 = (uint16_t)(i * GS + j);
-            if (j == 0) s2 = (uint16_t)(L * GS + i);
-        }
-        src1[c] = s1;
-        src2[c] = s2;
-    }
+    for (int c = threadIdx.x; c < ld; c += blockDim.x) src_s[c] = (uint16_t)column_source(c, d, P, GS);
     __syncthreads();
     for (int q = threadIdx.x; q < K * nb; q += blockDim.x) {
         const int k = q / nb, s = q - k * nb;
         const long long st = off_s[k * (S + 1) + s], en = off_s[k * (S + 1) + s + 1];
-        const bool isbad = st < 0 || en < st || en > nnz;
-        bad_s[k * S + s] = isbad;
-        bad += isbad;
+        uint32_t code = CODE_EMPTY;
+        if (st < 0 || en < st || en > nnz) {
+            ++bad;
+        } else if (en - st == 1) {
+            const int idx = __ldg(indices + st);
+            if (idx >= 0 && (long long)idx < tm.rows[k])
+                code = (uint32_t)(tm.base[k] + idx);
+            else
+                ++oob;
+        } else if (en - st > 1) {
+            code = CODE_MULTI;
+        }
+        code_s[k * S + s] = code;
     }
     __syncthreads();
+
+    // per-lane concat chunk sources (two 16-bit sources per register), fixed for the whole block
+    uint32_t srcr[SRC_CACHE][4];
+#pragma unroll
+    for (int j = 0; j < SRC_CACHE; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = 8 * (lane + 32 * j) + 2 * e;
+            const uint32_t lo = c < ld ? src_s[c] : 0xFFFFu, hi = c + 1 < ld ? src_s[c + 1] : 0xFFFFu;
+            srcr[j][e] = lo | (hi << 16);
+        }
 
     const uint32_t xw_s = (uint32_t)__cvta_generic_to_shared(xw);
     float* G = reinterpret_cast<float*>(xw + RS);
@@ -120,65 +158,55 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         if (s >= nb) break;
         const long long b = b0 + s;
 
-        // zero the padding rows K+2 .. KP-1
+        // x_dense in flight alongside the rows
+        float4 xv[(d + 127) / 128];
+#pragma unroll
+        for (int q = 0; q < (d + 127) / 128; ++q) {
+            const int c = 4 * lane + 128 * q;
+            xv[q] = c < d ? *reinterpret_cast<const float4*>(x_dense + b * d + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+
+        // ---- 1. gather: X rows 1..K
+        for (int k = gi; k < K; k += NG) {
+            const uint32_t code = code_s[k * S + s];
+            const uint32_t dst = xw_s + (uint32_t)((k + 1) * RS + 16 * g);
+            if (code < CODE_MULTI) {
+                cp_async16(dst, tables + (long long)code * d + 8 * g);
+            } else if (code == CODE_EMPTY) {
+                *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) = make_uint4(0, 0, 0, 0);
+            } else {
+                const int st = off_s[k * (S + 1) + s], en = off_s[k * (S + 1) + s + 1];
+                float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int p = st; p < en; ++p) {
+                    const int idx = __ldg(indices + p);
+                    if (idx >= 0 && (long long)idx < tm.rows[k])
+                        Chunk16<__nv_bfloat16>::add(ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g), a);
+                    else if (g == 0)
+                        ++oob;
+                }
+                *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) =
+                    make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+            }
+        }
+        // zero the padding rows K+2 .. KP-1 (G of the previous sample may have overwritten them)
         for (int q = lane; q < (KP - K - 2) * (RS / 16); q += 32)
             reinterpret_cast<uint4*>(xw + (size_t)(K + 2) * RS)[q] = make_uint4(0, 0, 0, 0);
 
-        // ---- 1. gather the K pooled rows into X rows 1..K (bf16)
-        for (int k0 = gi; k0 < K; k0 += NG * TB) {
-            uint4 v[TB];
-            int st[TB], en[TB];
-#pragma unroll
-            for (int u = 0; u < TB; ++u) {
-                const int k = k0 + u * NG;
-                st[u] = 0;
-                en[u] = 0;
-                v[u] = make_uint4(0, 0, 0, 0);
-                if (k < K && !bad_s[k * S + s]) {
-                    st[u] = off_s[k * (S + 1) + s];
-                    en[u] = off_s[k * (S + 1) + s + 1];
-                    if (en[u] > st[u]) {
-                        const int idx = __ldg(indices + st[u]);
-                        if (idx >= 0 && (long long)idx < tm.rows[k])
-                            v[u] = ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g);
-                        else if (g == 0)
-                            ++oob;
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < TB; ++u) {
-                const int k = k0 + u * NG;
-                if (k < K) {
-                    uint4 packed = v[u];
-                    if (en[u] - st[u] > 1) {
-                        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        bf16x8_add(v[u], a);
-                        for (int p = st[u] + 1; p < en[u]; ++p) {
-                            const int idx = __ldg(indices + p);
-                            if (idx >= 0 && (long long)idx < tm.rows[k])
-                                bf16x8_add(ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g), a);
-                            else if (g == 0)
-                                ++oob;
-                        }
-                        packed = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
-                                            pack_bf16(a[6], a[7]));
-                    }
-                    *reinterpret_cast<uint4*>(xw + (size_t)(k + 1) * RS + 16 * g) = packed;
-                }
-            }
-        }
-
         // ---- 2. x_dense -> rows 0 (hi) and K+1 (lo)
-        for (int c = 4 * lane; c < d; c += 128) {
-            const float4 x = *reinterpret_cast<const float4*>(x_dense + b * d + c);
-            const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
-            const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-            const uint32_t lo01 = pack_bf16(x.x - f01.x, x.y - f01.y), lo23 = pack_bf16(x.z - f23.x, x.w - f23.y);
-            *reinterpret_cast<uint2*>(xw + 2 * c) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
-            *reinterpret_cast<uint2*>(xw + (size_t)L * RS + 2 * c) = make_uint2(lo01, lo23);
+#pragma unroll
+        for (int q = 0; q < (d + 127) / 128; ++q) {
+            const int c = 4 * lane + 128 * q;
+            if (c < d) {
+                const float4 x = xv[q];
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
+                const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+                *reinterpret_cast<uint2*>(xw + 2 * c) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+                *reinterpret_cast<uint2*>(xw + (size_t)L * RS + 2 * c) =
+                    make_uint2(pack_bf16(x.x - f01.x, x.y - f01.y), pack_bf16(x.z - f23.x, x.w - f23.y));
+            }
         }
+        cp_async_wait_all();
         __syncwarp();
 
         // ---- 3. lower-triangle Gram tiles on the tensor cores
@@ -204,7 +232,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         }
         __syncwarp();  // every lane's ldmatrix of X is done before G overwrites it
 
-        // ---- 4. stage G (rows 0..KP-1, row stride GS floats, starting after X row 0)
+        // ---- 4. stage G (row stride GS floats, after X row 0, which keeps bf16(x_dense))
         {
             const int gr = lane >> 2, tc = (lane & 3) * 2;
             int t = 0;
@@ -213,52 +241,48 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
 #pragma unroll
                 for (int nt = 0; nt <= 2 * mt + 1; ++nt, ++t) {
                     float* p0 = G + (16 * mt + gr) * GS + 8 * nt + tc;
-                    float* p1 = p0 + 8 * GS;
-                    p0[0] = acc[t][0];
-                    p0[1] = acc[t][1];
-                    p1[0] = acc[t][2];
-                    p1[1] = acc[t][3];
+                    *reinterpret_cast<float2*>(p0) = make_float2(acc[t][0], acc[t][1]);
+                    *reinterpret_cast<float2*>(p0 + 8 * GS) = make_float2(acc[t][2], acc[t][3]);
                 }
             }
         }
         __syncwarp();
 
-        // ---- 5. concat row: x_dense (hi = bf16(x)), Z, zero padding
-        if (out_dt == DLRM_BF16) {
+        // ---- 5. concat row: x_dense, Z, zero padding
+        if (bf16_out) {
             uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + b * ld);
-            for (int c8 = lane; c8 < ld / 8; c8 += 32) {
-                const int c = 8 * c8;
-                if (c + 8 <= d) {
-                    orow[c8] = *reinterpret_cast<const uint4*>(xw + 2 * c);
-                } else {
-                    float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int cc = c + e;
-                        float val = 0.f;
-                        if (cc < d) {
-                            val = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[cc]);
-                        } else {
-                            const uint16_t i1 = src1[cc], i2 = src2[cc];
-                            if (i1 != 0xFFFFu) val = G[i1];
-                            if (i2 != 0xFFFFu) val += G[i2];
-                        }
-                        f[e] = val;
+            for (int j = 0; j < SRC_CACHE; ++j) {
+                const int c8 = lane + 32 * j;
+                if (c8 < nchunk) {
+                    if (8 * c8 + 8 <= d) {
+                        orow[c8] = *reinterpret_cast<const uint4*>(xw + 16 * c8);
+                    } else {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            f[e] = (8 * c8 + e < d)
+                                       ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[8 * c8 + e])
+                                       : column_value<GS>((srcr[j][e >> 1] >> (16 * (e & 1))) & 0xFFFFu, G, L);
+                        orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                              pack_bf16(f[6], f[7]));
                     }
-                    orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                          pack_bf16(f[6], f[7]));
                 }
+            }
+            for (int c8 = lane + 32 * SRC_CACHE; c8 < nchunk; c8 += 32) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = 8 * c8 + e;
+                    f[e] = c < d ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[c])
+                                 : column_value<GS>(src_s[c], G, L);
+                }
+                orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                      pack_bf16(f[6], f[7]));
             }
         } else {
             for (int c = lane; c < ld; c += 32) {
-                float val = 0.f;
-                if (c < d) {
-                    val = x_dense[b * d + c];
-                } else {
-                    const uint16_t i1 = src1[c], i2 = src2[c];
-                    if (i1 != 0xFFFFu) val = G[i1];
-                    if (i2 != 0xFFFFu) val += G[i2];
-                }
+                const float val = c < d ? x_dense[b * d + c] : column_value<GS>(src_s[c], G, L);
                 store_as(out, (size_t)b * ld + c, val, out_dt);
             }
         }
@@ -274,24 +298,26 @@ static int mma_warp_bytes(int K, int d, int& MT) {
     const int KP = 16 * MT;
     const int RS = 2 * d + 16;
     const int x = KP * RS;
-    const int gbytes = RS + KP * (KP + 1) * 4;
+    const int gbytes = RS + KP * (KP + 8) * 4;
     return ((x > gbytes ? x : gbytes) + 15) & ~15;
 }
 
 static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
     warp_bytes = mma_warp_bytes(K, d, MT);
-    return (size_t)WARPS * warp_bytes + sizeof(int) * (size_t)K * (S + 1) + (((size_t)K * S + 15) & ~(size_t)15) +
-           2 * sizeof(uint16_t) * (size_t)ld;
+    return (size_t)WARPS * warp_bytes + sizeof(int) * (size_t)K * (S + 1) + sizeof(uint32_t) * (size_t)K * S +
+           sizeof(uint16_t) * (size_t)ld;
 }
 
-bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt) {
+bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
+                                   long long total_rows) {
     if (dt != DLRM_BF16) return false;
     if (!(d == 32 || d == 64 || d == 128 || d == 256)) return false;
     if (K + 2 > 64) return false;
+    if (total_rows >= (long long)CODE_MULTI) return false;
     if (out_dt == DLRM_BF16 && (ld % 8 || ((uintptr_t)out & 15))) return false;
-    int MT, wb;
     const int P = K * (K + 1) / 2;
-    if ((K + 2) * (K + 3) > 0xFFFF || ld > 0x7FFF || P + d > ld) return false;
+    if (P + d > ld || ld > 0x7FFF) return false;
+    int MT, wb;
     return mma_smem(K, d, ld, MT, wb) <= 227 * 1024;
 }
 

@@ -22,7 +22,8 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
 
 // Tensor-core (mma.sync) variant of launch_embbag_interact for bf16 tables with
 // d in {32, 64, 128, 256} and K + 2 <= 64; launch_embbag_interact picks it when supported.
-bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt);
+bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
+                                   long long total_rows);
 dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, int K, int d, int B,
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
