@@ -20,8 +20,9 @@
 //     mma.sync.m16n8k16 (bf16 in, fp32 accumulate), lower-triangle tiles only.
 //     The same ldmatrix fragments serve as A and as B (B = X^T), so X is read
 //     from shared memory once per sample.
-//  4. G is staged in shared memory; each lane owns fixed 8-column chunks of
-//     the concat row, whose sources in G are computed once per block.
+//  4. G is staged in shared memory, the x_dense low-half terms are folded into
+//     column 0, and each lane writes fixed 8-column chunks of the concat row
+//     whose sources in G are computed once per block.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -30,11 +31,11 @@ namespace dlrm {
 namespace {
 
 constexpr int WARPS = 8;
-constexpr int SPW = 2;               // samples per warp per block
+constexpr int SPW = 4;               // samples per warp per block
 constexpr int S = WARPS * SPW;       // samples per block
 constexpr uint32_t CODE_EMPTY = 0xFFFFFFFFu;
 constexpr uint32_t CODE_MULTI = 0xFFFFFFFEu;
-constexpr int SRC_CACHE = 2;         // concat chunks per lane whose sources stay in registers
+constexpr int SRC_CACHE = 1;         // concat chunks per lane whose sources stay in registers
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -62,24 +63,15 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
-// Source of concat column c in the staged Gram G (row stride GS): i*GS + j for
-// Z_ij, 0xFFFF for a padding column. Columns below d come from x_dense.
-__device__ __forceinline__ uint32_t column_source(int c, int d, int P, int GS) {
+// Source of concat column c (c >= d) in the staged Gram G (row stride GS):
+// i*GS + j for Z_ij, or `zero` (a slot holding 0) for a padding column.
+__device__ __forceinline__ uint32_t column_source(int c, int d, int P, int GS, uint32_t zero) {
     const int p = c - d;
-    if (p < 0 || p >= P) return 0xFFFFu;
+    if (p < 0 || p >= P) return zero;
     int i = (int)((1.0f + sqrtf(8.0f * (float)p + 1.0f)) * 0.5f);
     while (i * (i - 1) / 2 > p) --i;
     while ((i + 1) * i / 2 <= p) ++i;
     return (uint32_t)(i * GS + (p - i * (i - 1) / 2));
-}
-
-// Z_ij from G; for j = 0 the low half of x_dense (row L) adds G[L][i].
-template <int GS>
-__device__ __forceinline__ float column_value(uint32_t s1, const float* G, int L) {
-    if (s1 == 0xFFFFu) return 0.f;
-    float v = G[s1];
-    if (s1 % GS == 0) v += G[L * GS + s1 / GS];
-    return v;
 }
 
 }  // namespace
@@ -104,8 +96,9 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     unsigned char* tail = smem + (size_t)WARPS * warp_bytes;
     int* off_s = reinterpret_cast<int*>(tail);
     uint32_t* code_s = reinterpret_cast<uint32_t*>(off_s + K * (S + 1));
-    uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + K * S);
-    const int nchunk = ld / 8;
+    uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + K * S);   // sources of columns d .. ld-1
+    const int nzc = (ld - d) / 8;                                    // 8-column chunks after x_dense
+    constexpr uint32_t ZERO_SLOT = KP * GS;
     const bool bf16_out = out_dt == DLRM_BF16;
 
     const int b0 = blockIdx.x * S;
@@ -117,7 +110,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         const int k = q / (nb + 1), s = q - k * (nb + 1);
         off_s[k * (S + 1) + s] = offsets[(long long)k * B + b0 + s];
     }
-    for (int c = threadIdx.x; c < ld; c += blockDim.x) src_s[c] = (uint16_t)column_source(c, d, P, GS);
+    for (int c = d + threadIdx.x; c < ld; c += blockDim.x) src_s[c - d] = (uint16_t)column_source(c, d, P, GS, ZERO_SLOT);
     __syncthreads();
     for (int q = threadIdx.x; q < K * nb; q += blockDim.x) {
         const int k = q / nb, s = q - k * nb;
@@ -138,14 +131,14 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     }
     __syncthreads();
 
-    // per-lane concat chunk sources (two 16-bit sources per register), fixed for the whole block
+    // per-lane sources of its Z chunks (two 16-bit sources per register), fixed for the whole block
     uint32_t srcr[SRC_CACHE][4];
 #pragma unroll
     for (int j = 0; j < SRC_CACHE; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int c = 8 * (lane + 32 * j) + 2 * e;
-            const uint32_t lo = c < ld ? src_s[c] : 0xFFFFu, hi = c + 1 < ld ? src_s[c + 1] : 0xFFFFu;
+            const uint32_t lo = c < ld - d ? src_s[c] : ZERO_SLOT, hi = c + 1 < ld - d ? src_s[c + 1] : ZERO_SLOT;
             srcr[j][e] = lo | (hi << 16);
         }
 
@@ -245,44 +238,39 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                     *reinterpret_cast<float2*>(p0 + 8 * GS) = make_float2(acc[t][2], acc[t][3]);
                 }
             }
+            if (lane == 0) G[ZERO_SLOT] = 0.f;
         }
+        __syncwarp();
+        // Z_i0 = <e_i, x_hi> + <e_i, x_lo>: fold the low half (row L) into column 0
+        for (int i = 1 + lane; i <= K; i += 32) G[i * GS] += G[L * GS + i];
         __syncwarp();
 
         // ---- 5. concat row: x_dense, Z, zero padding
         if (bf16_out) {
             uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + b * ld);
+            for (int c8 = lane; c8 < d / 8; c8 += 32) orow[c8] = *reinterpret_cast<const uint4*>(xw + 16 * c8);
+            uint4* zrow = orow + d / 8;
 #pragma unroll
             for (int j = 0; j < SRC_CACHE; ++j) {
                 const int c8 = lane + 32 * j;
-                if (c8 < nchunk) {
-                    if (8 * c8 + 8 <= d) {
-                        orow[c8] = *reinterpret_cast<const uint4*>(xw + 16 * c8);
-                    } else {
-                        float f[8];
+                if (c8 < nzc) {
+                    float f[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            f[e] = (8 * c8 + e < d)
-                                       ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[8 * c8 + e])
-                                       : column_value<GS>((srcr[j][e >> 1] >> (16 * (e & 1))) & 0xFFFFu, G, L);
-                        orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                                              pack_bf16(f[6], f[7]));
-                    }
+                    for (int e = 0; e < 8; ++e) f[e] = G[(srcr[j][e >> 1] >> (16 * (e & 1))) & 0xFFFFu];
+                    zrow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                          pack_bf16(f[6], f[7]));
                 }
             }
-            for (int c8 = lane + 32 * SRC_CACHE; c8 < nchunk; c8 += 32) {
+            for (int c8 = lane + 32 * SRC_CACHE; c8 < nzc; c8 += 32) {
                 float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = 8 * c8 + e;
-                    f[e] = c < d ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(xw)[c])
-                                 : column_value<GS>(src_s[c], G, L);
-                }
-                orow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                for (int e = 0; e < 8; ++e) f[e] = G[src_s[8 * c8 + e]];
+                zrow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                                       pack_bf16(f[6], f[7]));
             }
         } else {
             for (int c = lane; c < ld; c += 32) {
-                const float val = c < d ? x_dense[b * d + c] : column_value<GS>(src_s[c], G, L);
+                const float val = c < d ? x_dense[b * d + c] : G[src_s[c - d]];
                 store_as(out, (size_t)b * ld + c, val, out_dt);
             }
         }
@@ -298,14 +286,14 @@ static int mma_warp_bytes(int K, int d, int& MT) {
     const int KP = 16 * MT;
     const int RS = 2 * d + 16;
     const int x = KP * RS;
-    const int gbytes = RS + KP * (KP + 8) * 4;
+    const int gbytes = RS + (KP * (KP + 8) + 1) * 4;
     return ((x > gbytes ? x : gbytes) + 15) & ~15;
 }
 
 static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
     warp_bytes = mma_warp_bytes(K, d, MT);
     return (size_t)WARPS * warp_bytes + sizeof(int) * (size_t)K * (S + 1) + sizeof(uint32_t) * (size_t)K * S +
-           sizeof(uint16_t) * (size_t)ld;
+           sizeof(uint16_t) * (size_t)(ld - d + 8);
 }
 
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
@@ -315,6 +303,7 @@ bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const vo
     if (K + 2 > 64) return false;
     if (total_rows >= (long long)CODE_MULTI) return false;
     if (out_dt == DLRM_BF16 && (ld % 8 || ((uintptr_t)out & 15))) return false;
+    if (ld - d > 8 * 0x1FFF) return false;
     const int P = K * (K + 1) / 2;
     if (P + d > ld || ld > 0x7FFF) return false;
     int MT, wb;
