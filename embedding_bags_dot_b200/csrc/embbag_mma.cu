@@ -84,18 +84,23 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, int warp_bytes, ErrRecord* err) {
     constexpr int d = 8 * GL;
     constexpr int KP = 16 * MT;
-    constexpr int RS = 2 * d + 16;   // X row stride in bytes (odd multiple of 16: conflict-free ldmatrix)
+    // X rows: d >= 64 uses 2d-byte rows whose 16-byte chunks are XOR-swizzled by (row & 7); d = 32
+    // pads rows to an odd number of chunks. Either way ldmatrix reads 8 rows without bank conflicts.
+    constexpr bool SWZ = d >= 64;
+    constexpr int RS = SWZ ? 2 * d : 2 * d + 16;
     constexpr int GS = KP + 8;       // G row stride in floats (float2 staging without bank conflicts)
     constexpr int NG = 32 / GL;      // row groups per warp
     constexpr int NTILE = MT * (MT + 1);
+    // byte offset of 16-byte chunk c of X row r
+    auto xoff = [](int r, int c) { return r * RS + 16 * (SWZ ? (c ^ (r & 7)) : c); };
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = K * (K + 1) / 2;
     const int L = K + 1;             // row holding the low half of x_dense
     unsigned char* xw = smem + (size_t)warp * warp_bytes;
     unsigned char* tail = smem + (size_t)WARPS * warp_bytes;
-    int* off_s = reinterpret_cast<int*>(tail);
-    uint32_t* code_s = reinterpret_cast<uint32_t*>(off_s + K * (S + 1));
+    int* off_s = reinterpret_cast<int*>(smem);   // prologue only: lives in the X regions until samples start
+    uint32_t* code_s = reinterpret_cast<uint32_t*>(tail);
     uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + K * S);   // sources of columns d .. ld-1
     const int nzc = (ld - d) / 8;                                    // 8-column chunks after x_dense
     constexpr uint32_t ZERO_SLOT = KP * GS;
@@ -162,13 +167,13 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         // ---- 1. gather: X rows 1..K
         for (int k = gi; k < K; k += NG) {
             const uint32_t code = code_s[k * S + s];
-            const uint32_t dst = xw_s + (uint32_t)((k + 1) * RS + 16 * g);
+            const uint32_t dst = xw_s + (uint32_t)xoff(k + 1, g);
             if (code < CODE_MULTI) {
                 cp_async16(dst, tables + (long long)code * d + 8 * g);
             } else if (code == CODE_EMPTY) {
-                *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) = make_uint4(0, 0, 0, 0);
             } else {
-                const int st = off_s[k * (S + 1) + s], en = off_s[k * (S + 1) + s + 1];
+                const int st = offsets[(long long)k * B + b], en = offsets[(long long)k * B + b + 1];
                 float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int p = st; p < en; ++p) {
                     const int idx = __ldg(indices + p);
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                     else if (g == 0)
                         ++oob;
                 }
-                *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) =
+                *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) =
                     make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
             }
         }
@@ -193,9 +198,9 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                 const float4 x = xv[q];
                 const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
                 const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-                *reinterpret_cast<uint2*>(xw + 2 * c) =
+                *reinterpret_cast<uint2*>(xw + xoff(0, c / 8) + 2 * (c % 8)) =
                     make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
-                *reinterpret_cast<uint2*>(xw + (size_t)L * RS + 2 * c) =
+                *reinterpret_cast<uint2*>(xw + xoff(L, c / 8) + 2 * (c % 8)) =
                     make_uint2(pack_bf16(x.x - f01.x, x.y - f01.y), pack_bf16(x.z - f23.x, x.w - f23.y));
             }
         }
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
             uint32_t a[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
-                ldmatrix_x4(xw_s + (uint32_t)((16 * mt + (lane & 15)) * RS + ks * 32 + (lane >> 4) * 16), a[mt]);
+                ldmatrix_x4(xw_s + (uint32_t)xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a[mt]);
             int t = 0;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
 static int mma_warp_bytes(int K, int d, int& MT) {
     MT = (K + 2 + 15) / 16;
     const int KP = 16 * MT;
-    const int RS = 2 * d + 16;
+    const int RS = d >= 64 ? 2 * d : 2 * d + 16;
     const int x = KP * RS;
     const int gbytes = RS + (KP * (KP + 8) + 1) * 4;
     return ((x > gbytes ? x : gbytes) + 15) & ~15;
@@ -292,8 +297,7 @@ static int mma_warp_bytes(int K, int d, int& MT) {
 
 static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
     warp_bytes = mma_warp_bytes(K, d, MT);
-    return (size_t)WARPS * warp_bytes + sizeof(int) * (size_t)K * (S + 1) + sizeof(uint32_t) * (size_t)K * S +
-           sizeof(uint16_t) * (size_t)(ld - d + 8);
+    return (size_t)WARPS * warp_bytes + sizeof(uint32_t) * (size_t)K * S + sizeof(uint16_t) * (size_t)(ld - d + 8);
 }
 
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
