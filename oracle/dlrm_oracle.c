@@ -254,7 +254,8 @@ double oracle_bce(int B, const double* z, const double* y) {
  *   dA  [B][n_in]   gradient w.r.t. the input (may be NULL)
  * ReLU'(0) is taken as 0. */
 static void linear_backward(int B, int n_in, int n_out, const double* W, const double* A, const double* Y,
-                            double* dY, double* dW, double* db, double* dA, int relu) {
+                            double* dY, double* dW, double* db, double* dA, int relu,
+                            double* dW_scale, double* db_scale) {
     if (relu) {
         for (int64_t q = 0; q < (int64_t)B * n_out; ++q)
             if (!(Y[q] > 0.0)) dY[q] = 0.0;
@@ -268,6 +269,19 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
             double s = 0.0;
             for (int b = 0; b < B; ++b) s += dY[(int64_t)b * n_out + o] * A[(int64_t)b * n_in + i];
             dW[(int64_t)o * n_in + i] = s;
+        }
+        /* magnitude of each batch sum (sum of |terms|), for judging rounding error */
+        if (db_scale) {
+            double a = 0.0;
+            for (int b = 0; b < B; ++b) a += fabs(dY[(int64_t)b * n_out + o]);
+            db_scale[o] = a;
+        }
+        if (dW_scale) {
+            for (int i = 0; i < n_in; ++i) {
+                double a = 0.0;
+                for (int b = 0; b < B; ++b) a += fabs(dY[(int64_t)b * n_out + o] * A[(int64_t)b * n_in + i]);
+                dW_scale[(int64_t)o * n_in + i] = a;
+            }
         }
     }
     if (dA) {
@@ -289,12 +303,17 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
  *   bot_dW[l] [out][in], bot_db[l] [out], top_dW[l], top_db[l]: batch-summed gradients of the mean loss
  *   table_grad [sum rows][d]  gradient of every table row (zero for rows no valid index touches)
  *   row_count  [sum rows]     number of valid occurrences of each row in the batch
- *   counts[0..1]              as oracle_embbag */
+ *   counts[0..1]              as oracle_embbag
+ * Optional (NULL to skip): *_scale arrays of the same shapes receive the sum of
+ * |terms| of each batch-summed gradient, and table_grad_scale the sum over
+ * occurrences of |dE| (an error yardstick; not part of the method). */
 void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* dense,
                         const int32_t* offsets, const int32_t* indices, const double* labels,
                         double* loss, double* y_hat,
                         double* const* bot_dW, double* const* bot_db, double* const* top_dW, double* const* top_db,
-                        double* table_grad, int64_t* row_count, long* counts) {
+                        double* table_grad, int64_t* row_count, long* counts,
+                        double* const* bot_dW_s, double* const* bot_db_s, double* const* top_dW_s,
+                        double* const* top_db_s, double* table_grad_s) {
     int K = M->K, d = M->d;
     int width = d + K * (K + 1) / 2;
     int64_t* base = (int64_t*)malloc(sizeof(int64_t) * (K > 0 ? K : 1));
@@ -349,7 +368,8 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
     for (int l = M->n_top - 1; l >= 0; --l) {
         double* dA = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
         linear_backward(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], top_act[l], top_act[l + 1],
-                        dY, top_dW[l], top_db[l], dA, l < M->n_top - 1);
+                        dY, top_dW[l], top_db[l], dA, l < M->n_top - 1,
+                        top_dW_s ? top_dW_s[l] : NULL, top_db_s ? top_db_s[l] : NULL);
         free(dY);
         dY = dA;
     }
@@ -380,13 +400,15 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
     for (int l = M->n_bot - 1; l >= 0; --l) {
         double* dA = (l > 0) ? (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]) : NULL;
         linear_backward(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], bot_act[l], bot_act[l + 1],
-                        dB, bot_dW[l], bot_db[l], dA, 1);
+                        dB, bot_dW[l], bot_db[l], dA, 1,
+                        bot_dW_s ? bot_dW_s[l] : NULL, bot_db_s ? bot_db_s[l] : NULL);
         free(dB);
         dB = dA;
     }
     /* embedding rows: every valid occurrence of row r in bag (k, b) adds dE_k[b] */
     memset(table_grad, 0, sizeof(double) * (size_t)total_rows * d);
     memset(row_count, 0, sizeof(int64_t) * (size_t)total_rows);
+    if (table_grad_s) memset(table_grad_s, 0, sizeof(double) * (size_t)total_rows * d);
     for (int k = 0; k < K; ++k) {
         for (int b = 0; b < B; ++b) {
             int64_t start = offsets[(int64_t)k * B + b], end = offsets[(int64_t)k * B + b + 1];
@@ -398,6 +420,8 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
                 double* tg = table_grad + (base[k] + r) * d;
                 for (int t = 0; t < d; ++t) tg[t] += g[t];
                 row_count[base[k] + r] += 1;
+                if (table_grad_s)
+                    for (int t = 0; t < d; ++t) table_grad_s[(base[k] + r) * d + t] += fabs(g[t]);
             }
         }
     }
