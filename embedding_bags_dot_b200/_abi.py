@@ -64,6 +64,15 @@ _SIGS = {
                                C.c_void_p, C.c_void_p]),
     "dlrm_forward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
                                C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_grads_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64]),
+    "dlrm_grads_offsets": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_backward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                                C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_sparse_sgd": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_void_p,
+                                  C.c_void_p, C.c_void_p]),
+    "dlrm_embedding_row_grads": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_void_p,
+                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
 }
@@ -218,3 +227,47 @@ def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, 
     return _check(lib().dlrm_forward_noalloc(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                              _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(err_flags),
                                              _stream(stream)), "dlrm_forward_noalloc")
+
+
+# ----------------------------------------------------------------- training step (fp32)
+
+def dlrm_grads_size(T: Tables, bot: MLP, top: MLP, B: int, nnz: int) -> int:
+    return int(lib().dlrm_grads_size(T.ref(), bot.ref(), top.ref(), int(B), int(nnz)))
+
+
+def dlrm_grads_offsets(T: Tables, bot: MLP, top: MLP, B: int, nnz: int) -> dict:
+    """Byte offsets of every gradient inside the gradient buffer."""
+    nb, nt = len(bot.Ws), len(top.Ws)
+    arrs = [(C.c_size_t * n)() for n in (nb, nb, nt, nt)]
+    dE, loss = C.c_size_t(), C.c_size_t()
+    _check(lib().dlrm_grads_offsets(T.ref(), bot.ref(), top.ref(), int(B), int(nnz), *arrs, C.byref(dE),
+                                    C.byref(loss)), "dlrm_grads_offsets")
+    return {"bot_dW": list(arrs[0]), "bot_db": list(arrs[1]), "top_dW": list(arrs[2]), "top_db": list(arrs[3]),
+            "dE": dE.value, "loss": loss.value}
+
+
+def dlrm_backward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, labels, grads, ws, loss=None,
+                  y_hat=None, stream=None):
+    return _check(lib().dlrm_backward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
+                                      _ptr(indices), int(indices.numel()), _ptr(labels), _ptr(loss), _ptr(y_hat),
+                                      _ptr(grads), _ptr(ws), _stream(stream)), "dlrm_backward")
+
+
+def dlrm_sparse_sgd(T: Tables, bot: MLP, top: MLP, B: int, nnz: int, lr: float, grads, n_touched=None, stream=None):
+    return _check(lib().dlrm_sparse_sgd(T.ref(), bot.ref(), top.ref(), int(B), int(nnz), float(lr), _ptr(grads),
+                                        _ptr(n_touched), _stream(stream)), "dlrm_sparse_sgd")
+
+
+def dlrm_embedding_row_grads(T: Tables, bot: MLP, top: MLP, B: int, nnz: int, grads, rows, row_grads, n_rows,
+                             stream=None):
+    return _check(lib().dlrm_embedding_row_grads(T.ref(), bot.ref(), top.ref(), int(B), int(nnz), _ptr(grads),
+                                                 _ptr(rows), _ptr(row_grads), _ptr(n_rows), _stream(stream)),
+                  "dlrm_embedding_row_grads")
+
+
+def grads_view(grads: torch.Tensor, off: int, shape) -> torch.Tensor:
+    """fp32 view of part of a gradient buffer at a byte offset."""
+    n = 1
+    for x in shape:
+        n *= int(x)
+    return grads[off:off + 4 * n].view(torch.float32).view(*shape)

@@ -144,8 +144,11 @@ const char* dlrm_status_str(dlrm_status s) {
 size_t dlrm_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int training) {
     TableMeta tm;
     if (check_tables(T, tm) != DLRM_OK || check_mlp(bot) != DLRM_OK || check_mlp(top) != DLRM_OK || B < 0) return 0;
-    (void)training;
-    return fwd_layout(T, bot, top, B).total;
+    const size_t f = fwd_layout(T, bot, top, B).total;
+    if (!training) return f;
+    const size_t t = train_workspace_size(T, bot, top, B);
+    if (t == 0) return 0;
+    return t > f ? t : f;
 }
 
 dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info) {

@@ -43,4 +43,40 @@ dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st);
 
+// ---- training (fp32)
+dlrm_status train_linear_fwd(int M, int N, int K, const float* x, int ldx, const float* W, int ldw, const float* b,
+                             float* y, int ldy, bool relu, cudaStream_t st);
+dlrm_status train_linear_dgrad(int M, int N, int K, const float* dy, int lddy, const float* W, int ldw,
+                               const float* relu_of, int ldr, float* dx, int lddx, cudaStream_t st);
+int train_wgrad_splits(int N, int K, int M);
+size_t train_wgrad_scratch_floats(int N, int K, int M);
+dlrm_status train_linear_wgrad(int M, int N, int K, const float* dy, int lddy, const float* x, int ldx, float* dW,
+                               int ldw, float* db, float* scratch, cudaStream_t st);
+
+dlrm_status launch_bce(int B, const float* z, const float* y, float* dz, float* y_hat, float* partial, float* loss,
+                       cudaStream_t st);
+size_t interact_bwd_smem(int K, int d);
+// dx_dense receives the gradient w.r.t. the pre-activation of the bottom MLP's last (ReLU) layer.
+dlrm_status launch_interact_bwd(int B, int K, int d, const float* x_dense, const float* E, const float* dconcat,
+                                int ldc, float* dx_dense, float* dE, cudaStream_t st);
+
+constexpr int SPARSE_PIECE = 64;   // occurrences summed per warp before the per-row combine
+
+// Byte offsets of the sparse-update arrays inside the gradient buffer.
+struct SparseLayout {
+    long long cap;
+    size_t counts, bag_len, occ_off, keys[2], vals[2], hist, hist_off, head, seg_id, seg_start, seg_row, seg_pieces,
+        piece_base, piece_seg, partial, scan_sums, total;
+};
+SparseLayout sparse_layout(long long KB, long long nnz, int d);
+int radix_passes(long long total_rows);
+dlrm_status launch_sparse_prepare(int K, int B, const TableMeta& tm, long long total_rows, const int32_t* offsets,
+                                  const int32_t* indices, long long nnz, char* base, const SparseLayout& L,
+                                  ErrRecord* err, int* sorted_buf, cudaStream_t st);
+dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, int sorted_buf, const float* dE,
+                                float lr, float* table, float* grad_out, uint32_t* rows_out, int32_t* n_rows_out,
+                                cudaStream_t st);
+dlrm_status launch_sgd(long long n, float lr, float* w, const float* g, cudaStream_t st);
+size_t train_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B);
+
 }  // namespace dlrm

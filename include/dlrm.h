@@ -146,6 +146,51 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat,
                          void* ws, dlrm_stream stream);
 
+/* ------------------------------------------------------------ training step
+ * fp32 tables and MLPs only (DLRM_ERR_UNSUPPORTED otherwise); d % 4 == 0.
+ * The pages state the loss ([N] Key Method Details: binary cross-entropy);
+ * the gradients are the calculus of the forward definition and the update is
+ * plain SGD, w <- w - lr * grad, applied to the MLP parameters and to the
+ * embedding rows the batch touched (no other row is written). */
+
+/* Bytes of the gradient buffer for batch B with nnz indices. No zeroing needed. */
+size_t dlrm_grads_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz);
+
+/* Byte offsets inside the gradient buffer (host arrays of n_layers entries; any may be NULL):
+ * dW[l] is fp32 [dims[l+1]][dlrm_ld(dims[l], DLRM_F32)], db[l] fp32 [dims[l+1]],
+ * dE fp32 [B][K][d] (gradient of each pooled bag), loss one fp32. */
+dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
+                               size_t* bot_dW, size_t* bot_db, size_t* top_dW, size_t* top_db, size_t* dE,
+                               size_t* loss);
+
+/* Forward (as dlrm_forward, keeping every activation in `ws`, which must
+ * come from dlrm_workspace_size(..., training = 1)), then the mean BCE loss
+ * against labels (fp32 [B] of 0/1), then the backward pass: batch-summed
+ * gradients of the mean loss for every MLP weight and bias, the gradient of
+ * every pooled bag, and the occurrences of the batch sorted by table row
+ * (stable, so equal rows keep occurrence order). loss (device, 1 float) and
+ * y_hat (device, fp32 [B]) are optional outputs. Bit-reproducible. */
+dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                          const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
+                          float* loss, float* y_hat, void* grads, void* ws, dlrm_stream stream);
+
+/* SGD step from a gradient buffer filled by dlrm_backward on the same batch
+ * shape: every table row the batch touched gets T[r] -= lr * g_r, where g_r
+ * sums the gradients of the bags that use row r (once per occurrence) in
+ * occurrence order; untouched rows are not written. Then W -= lr * dW and
+ * b -= lr * db for every MLP layer. n_touched (device int32, optional)
+ * receives the number of distinct rows updated. */
+dlrm_status dlrm_sparse_sgd(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
+                            float lr, void* grads, int32_t* n_touched, dlrm_stream stream);
+
+/* The per-row embedding gradients dlrm_sparse_sgd would apply, without
+ * applying them: rows (device uint32 [nnz]) gets the touched rows as global
+ * row ids (base_k + r) in increasing order, row_grads (device fp32 [nnz][d])
+ * their summed gradients, n_rows (device int32) their count. */
+dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
+                                     int64_t nnz, void* grads, uint32_t* rows, float* row_grads,
+                                     int32_t* n_rows, dlrm_stream stream);
+
 /* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
 #define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
 

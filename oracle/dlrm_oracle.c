@@ -254,8 +254,7 @@ double oracle_bce(int B, const double* z, const double* y) {
  *   dA  [B][n_in]   gradient w.r.t. the input (may be NULL)
  * ReLU'(0) is taken as 0. */
 static void linear_backward(int B, int n_in, int n_out, const double* W, const double* A, const double* Y,
-                            double* dY, double* dW, double* db, double* dA, int relu,
-                            double* dW_scale, double* db_scale) {
+                            double* dY, double* dW, double* db, double* dA, int relu) {
     if (relu) {
         for (int64_t q = 0; q < (int64_t)B * n_out; ++q)
             if (!(Y[q] > 0.0)) dY[q] = 0.0;
@@ -270,19 +269,6 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
             for (int b = 0; b < B; ++b) s += dY[(int64_t)b * n_out + o] * A[(int64_t)b * n_in + i];
             dW[(int64_t)o * n_in + i] = s;
         }
-        /* magnitude of each batch sum (sum of |terms|), for judging rounding error */
-        if (db_scale) {
-            double a = 0.0;
-            for (int b = 0; b < B; ++b) a += fabs(dY[(int64_t)b * n_out + o]);
-            db_scale[o] = a;
-        }
-        if (dW_scale) {
-            for (int i = 0; i < n_in; ++i) {
-                double a = 0.0;
-                for (int b = 0; b < B; ++b) a += fabs(dY[(int64_t)b * n_out + o] * A[(int64_t)b * n_in + i]);
-                dW_scale[(int64_t)o * n_in + i] = a;
-            }
-        }
     }
     if (dA) {
 #pragma omp parallel for schedule(static)
@@ -296,6 +282,41 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
     }
 }
 
+/* Magnitude companion of linear_backward (error yardstick, not part of the
+ * method): given sY >= |dY| (an elementwise bound on the size of the output
+ * gradient and of its rounding error), masks it like dY, and returns
+ * sW = sum_b sY |A|, sb = sum_b sY and sA = sY |W|. */
+static void linear_backward_magnitude(int B, int n_in, int n_out, const double* W, const double* A, const double* Y,
+                                      double* sY, double* sW, double* sb, double* sA, int relu) {
+    if (relu) {
+        for (int64_t q = 0; q < (int64_t)B * n_out; ++q)
+            if (!(Y[q] > 0.0)) sY[q] = 0.0;
+    }
+#pragma omp parallel for schedule(static)
+    for (int o = 0; o < n_out; ++o) {
+        double a = 0.0;
+        for (int b = 0; b < B; ++b) a += sY[(int64_t)b * n_out + o];
+        if (sb) sb[o] = a;
+        if (sW) {
+            for (int i = 0; i < n_in; ++i) {
+                double s = 0.0;
+                for (int b = 0; b < B; ++b) s += sY[(int64_t)b * n_out + o] * fabs(A[(int64_t)b * n_in + i]);
+                sW[(int64_t)o * n_in + i] = s;
+            }
+        }
+    }
+    if (sA) {
+#pragma omp parallel for schedule(static)
+        for (int b = 0; b < B; ++b) {
+            for (int i = 0; i < n_in; ++i) {
+                double s = 0.0;
+                for (int o = 0; o < n_out; ++o) s += sY[(int64_t)b * n_out + o] * fabs(W[(int64_t)o * n_in + i]);
+                sA[(int64_t)b * n_in + i] = s;
+            }
+        }
+    }
+}
+
 /* Forward + backward of the whole model on one batch.
  * Outputs:
  *   loss                      mean BCE
@@ -304,9 +325,10 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
  *   table_grad [sum rows][d]  gradient of every table row (zero for rows no valid index touches)
  *   row_count  [sum rows]     number of valid occurrences of each row in the batch
  *   counts[0..1]              as oracle_embbag
- * Optional (NULL to skip): *_scale arrays of the same shapes receive the sum of
- * |terms| of each batch-summed gradient, and table_grad_scale the sum over
- * occurrences of |dE| (an error yardstick; not part of the method). */
+ * Optional (NULL to skip): *_s arrays of the same shapes receive, for every
+ * gradient, the size of what it sums: the same backward chain run on
+ * magnitudes (|dL/dz|, |W|, |activations|), an error yardstick for the fp32
+ * GPU result; not part of the method. */
 void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* dense,
                         const int32_t* offsets, const int32_t* indices, const double* labels,
                         double* loss, double* y_hat,
@@ -368,8 +390,7 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
     for (int l = M->n_top - 1; l >= 0; --l) {
         double* dA = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
         linear_backward(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], top_act[l], top_act[l + 1],
-                        dY, top_dW[l], top_db[l], dA, l < M->n_top - 1,
-                        top_dW_s ? top_dW_s[l] : NULL, top_db_s ? top_db_s[l] : NULL);
+                        dY, top_dW[l], top_db[l], dA, l < M->n_top - 1);
         free(dY);
         dY = dA;
     }
@@ -400,15 +421,13 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
     for (int l = M->n_bot - 1; l >= 0; --l) {
         double* dA = (l > 0) ? (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]) : NULL;
         linear_backward(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], bot_act[l], bot_act[l + 1],
-                        dB, bot_dW[l], bot_db[l], dA, 1,
-                        bot_dW_s ? bot_dW_s[l] : NULL, bot_db_s ? bot_db_s[l] : NULL);
+                        dB, bot_dW[l], bot_db[l], dA, 1);
         free(dB);
         dB = dA;
     }
     /* embedding rows: every valid occurrence of row r in bag (k, b) adds dE_k[b] */
     memset(table_grad, 0, sizeof(double) * (size_t)total_rows * d);
     memset(row_count, 0, sizeof(int64_t) * (size_t)total_rows);
-    if (table_grad_s) memset(table_grad_s, 0, sizeof(double) * (size_t)total_rows * d);
     for (int k = 0; k < K; ++k) {
         for (int b = 0; b < B; ++b) {
             int64_t start = offsets[(int64_t)k * B + b], end = offsets[(int64_t)k * B + b + 1];
@@ -420,12 +439,70 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
                 double* tg = table_grad + (base[k] + r) * d;
                 for (int t = 0; t < d; ++t) tg[t] += g[t];
                 row_count[base[k] + r] += 1;
-                if (table_grad_s)
-                    for (int t = 0; t < d; ++t) table_grad_s[(base[k] + r) * d + t] += fabs(g[t]);
             }
         }
     }
     free(dX); free(dY);
+
+    /* Magnitude companion pass (only when scales are requested): the same
+     * backward chain on sizes, sY >= |dY|, so that each gradient can be judged
+     * against the sizes of the terms it sums, including upstream gradients. */
+    if (bot_dW_s || bot_db_s || top_dW_s || top_db_s || table_grad_s) {
+        double* sY = (double*)malloc(sizeof(double) * (size_t)B);
+        for (int b = 0; b < B; ++b) sY[b] = fabs(sigmoid(z[b]) - labels[b]) / B;
+        for (int l = M->n_top - 1; l >= 0; --l) {
+            double* sA = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
+            linear_backward_magnitude(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], top_act[l], top_act[l + 1],
+                                      sY, top_dW_s ? top_dW_s[l] : NULL, top_db_s ? top_db_s[l] : NULL, sA,
+                                      l < M->n_top - 1);
+            free(sY);
+            sY = sA;
+        }
+        double* sX = (double*)calloc((size_t)B * (K + 1) * d, sizeof(double));
+#pragma omp parallel for schedule(static)
+        for (int b = 0; b < B; ++b) {
+            const double* sc = sY + (int64_t)b * width;
+            double* g = sX + (int64_t)b * (K + 1) * d;
+            for (int t = 0; t < d; ++t) g[t] += sc[t];
+            int p = d;
+            for (int i = 1; i <= K; ++i) {
+                const double* xi = E + ((int64_t)b * K + (i - 1)) * d;
+                for (int j = 0; j < i; ++j) {
+                    const double* xj = (j == 0) ? xd + (int64_t)b * d : E + ((int64_t)b * K + (j - 1)) * d;
+                    double sz = sc[p++];
+                    for (int t = 0; t < d; ++t) {
+                        g[(int64_t)i * d + t] += sz * fabs(xj[t]);
+                        g[(int64_t)j * d + t] += sz * fabs(xi[t]);
+                    }
+                }
+            }
+        }
+        double* sB = (double*)malloc(sizeof(double) * (size_t)B * d);
+        for (int b = 0; b < B; ++b) memcpy(sB + (int64_t)b * d, sX + (int64_t)b * (K + 1) * d, sizeof(double) * d);
+        for (int l = M->n_bot - 1; l >= 0; --l) {
+            double* sA = (l > 0) ? (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]) : NULL;
+            linear_backward_magnitude(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], bot_act[l], bot_act[l + 1],
+                                      sB, bot_dW_s ? bot_dW_s[l] : NULL, bot_db_s ? bot_db_s[l] : NULL, sA, 1);
+            free(sB);
+            sB = sA;
+        }
+        if (table_grad_s) {
+            memset(table_grad_s, 0, sizeof(double) * (size_t)total_rows * d);
+            for (int k = 0; k < K; ++k)
+                for (int b = 0; b < B; ++b) {
+                    int64_t start = offsets[(int64_t)k * B + b], end = offsets[(int64_t)k * B + b + 1];
+                    if (start < 0 || end < start || end > nnz) continue;
+                    const double* g = sX + ((int64_t)b * (K + 1) + (k + 1)) * d;
+                    for (int64_t p = start; p < end; ++p) {
+                        int64_t r = indices[p];
+                        if (r < 0 || r >= M->rows[k]) continue;
+                        for (int t = 0; t < d; ++t) table_grad_s[(base[k] + r) * d + t] += g[t];
+                    }
+                }
+        }
+        free(sX);
+        free(sY);
+    }
     for (int l = 0; l <= M->n_bot; ++l) free(bot_act[l]);
     for (int l = 0; l <= M->n_top; ++l) free(top_act[l]);
     free(bot_act); free(top_act); free(E); free(lens); free(base);

@@ -1,0 +1,161 @@
+"""Training step on the GPU (fp32) against the fp64 oracle, through the C ABI:
+loss, every MLP gradient, the row-sorted embedding gradients (bit-exact row
+set and counts), the SGD update of touched rows only, and bit-reproducibility.
+
+Gradients are batch sums; each is judged against its own sum of |terms|
+(from the oracle): |gpu - oracle| <= 1e-5 * (|oracle| + sum|terms|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import embedding_bags_dot_b200 as E
+from gpucase import GpuModel, to_np
+from oracle import oracle as O
+from synth import CONFIGS, gen, shrink
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-5
+
+
+def _cases():
+    tr = CONFIGS["train"]
+    return {
+        "train-small": shrink(tr, B=300, rows_cap=3000),
+        "train-mix": shrink(tr, B=97, rows_cap=400).with_(bag="mix", seed=2),
+        "tiny-train": CONFIGS["tiny"].with_(training=True, B=203),
+        "train-hot-rows": shrink(tr, B=2000, rows_cap=50),   # long segments: many occurrences per row
+    }
+
+
+CASES = _cases()
+
+
+def _close(got, want, scale, what):
+    got, want, scale = (np.asarray(a, np.float64) for a in (got, want, scale))
+    lim = RTOL * (np.abs(want) + scale) + 1e-30
+    err = np.abs(got - want)
+    bad = ~(err <= lim)
+    assert not bad.any(), (f"{what}: {int(bad.sum())}/{bad.size} outside; worst rel "
+                           f"{float((err / (np.abs(want) + scale + 1e-30)).max()):.3g}")
+
+
+class Trainer:
+    def __init__(self, cfg):
+        self.cfg = cfg
+        self.g = GpuModel(cfg, training=True)
+        self.batch = gen.make_batches(cfg, (0,))[0]
+        self.bt = {k: torch.from_numpy(v).cuda() for k, v in
+                   (("dense", self.batch.dense), ("offsets", self.batch.offsets), ("indices", self.batch.indices),
+                    ("labels", self.batch.labels))}
+        self.nnz = self.batch.indices.size
+        g = self.g
+        self.grads = torch.zeros(E.dlrm_grads_size(g.T, g.bot, g.top, cfg.B, self.nnz), dtype=torch.uint8, device="cuda")
+        self.off = E.dlrm_grads_offsets(g.T, g.bot, g.top, cfg.B, self.nnz)
+
+    def backward(self):
+        g, cfg = self.g, self.cfg
+        loss = torch.zeros(1, device="cuda")
+        y = torch.zeros(cfg.B, device="cuda")
+        E.dlrm_backward(g.T, g.bot, g.top, cfg.B, self.bt["dense"], self.bt["offsets"], self.bt["indices"],
+                        self.bt["labels"], self.grads, g.ws, loss=loss, y_hat=y)
+        st = E.dlrm_check_error(g.ws)
+        assert st[0] == 0, st
+        return float(loss.item()), to_np(y)
+
+    def dense_grads(self):
+        g, o = self.g, self.off
+        out = {}
+        for key, mlp in (("bot", g.bot), ("top", g.top)):
+            out[key + "_dW"] = [to_np(E.grads_view(self.grads, o[key + "_dW"][l], (mlp.dims[l + 1], E.dlrm_ld(mlp.dims[l], "f32"))))[:, :mlp.dims[l]]
+                                for l in range(len(mlp.Ws))]
+            out[key + "_db"] = [to_np(E.grads_view(self.grads, o[key + "_db"][l], (mlp.dims[l + 1],)))
+                                for l in range(len(mlp.Ws))]
+        return out
+
+
+@pytest.fixture(scope="module", params=sorted(CASES))
+def case(request):
+    cfg = CASES[request.param]
+    t = Trainer(cfg)
+    model = O.model_from_config(cfg)
+    ref = O.train_grads(model, t.batch.dense, t.batch.offsets, t.batch.indices, t.batch.labels, scales=True)
+    return cfg, t, model, ref
+
+
+def test_loss_and_dense_gradients(case):
+    cfg, t, model, ref = case
+    loss, y = t.backward()
+    assert abs(loss - ref["loss"]) <= RTOL * abs(ref["loss"]), (loss, ref["loss"])
+    assert np.abs(y - ref["y_hat"]).max() <= RTOL * 1.0
+    grads = t.dense_grads()
+    for key in ("bot_dW", "bot_db", "top_dW", "top_db"):
+        for l, (gg, oo, ss) in enumerate(zip(grads[key], ref[key], ref[key + "_s"])):
+            _close(gg, oo, ss, f"{cfg.name} {key}[{l}]")
+
+
+def test_embedding_row_gradients_and_bookkeeping(case):
+    cfg, t, model, ref = case
+    t.backward()
+    g = t.g
+    rows = torch.full((max(t.nnz, 1),), 0xFFFFFFF, dtype=torch.int32, device="cuda")
+    rg = torch.zeros((max(t.nnz, 1), cfg.d), device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    E.dlrm_embedding_row_grads(g.T, g.bot, g.top, cfg.B, t.nnz, t.grads, rows, rg, n)
+    torch.cuda.synchronize()
+    nr = int(n.item())
+    touched = np.nonzero(ref["row_count"])[0]
+    assert nr == touched.size
+    got_rows = rows.cpu().numpy()[:nr].astype(np.int64)
+    assert np.array_equal(got_rows, touched), "touched rows must match bit-exactly, in increasing order"
+    _close(to_np(rg)[:nr], ref["table_grad"][touched], ref["table_grad_s"][touched], f"{cfg.name} row grads")
+
+
+def test_sparse_sgd_updates_touched_rows_only(case):
+    cfg, t, model, ref = case
+    g = t.g
+    before = g.tables.clone()
+    Ws_before = [w.clone() for w in g.bot.Ws + g.top.Ws]
+    t.backward()
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    E.dlrm_sparse_sgd(g.T, g.bot, g.top, cfg.B, t.nnz, cfg.lr, t.grads, n)
+    torch.cuda.synchronize()
+    touched = ref["row_count"] > 0
+    assert int(n.item()) == int(touched.sum())
+    after = g.tables.cpu()
+    assert torch.equal(after[torch.from_numpy(~touched)], before.cpu()[torch.from_numpy(~touched)]), \
+        "untouched rows must be bit-identical"
+    want = O.sgd(model.tables[touched], ref["table_grad"][touched], cfg.lr)
+    scale = np.abs(model.tables[touched]) + cfg.lr * ref["table_grad_s"][touched]
+    _close(after.double().numpy()[touched], want, scale, f"{cfg.name} updated rows")
+    # dense parameters
+    refs = [(ref["bot_dW"], ref["bot_db"], ref["bot_dW_s"], ref["bot_db_s"], g.bot, model.bot_W, model.bot_b),
+            (ref["top_dW"], ref["top_db"], ref["top_dW_s"], ref["top_db_s"], g.top, model.top_W, model.top_b)]
+    for dW, db, dWs, dbs, mlp, W0, b0 in refs:
+        for l in range(len(mlp.Ws)):
+            k = mlp.dims[l]
+            _close(to_np(mlp.Ws[l])[:, :k], O.sgd(W0[l], dW[l], cfg.lr), np.abs(W0[l]) + cfg.lr * dWs[l], "W update")
+            _close(to_np(mlp.bs[l]), O.sgd(b0[l], db[l], cfg.lr), np.abs(b0[l]) + cfg.lr * dbs[l], "b update")
+            assert torch.all(mlp.Ws[l][:, k:] == 0), "weight padding untouched"
+    # restore for the other tests of this module
+    g.tables.copy_(before)
+    for w, w0 in zip(g.bot.Ws + g.top.Ws, Ws_before):
+        w.copy_(w0)
+    for mlp, b0s in ((g.bot, model.bot_b), (g.top, model.top_b)):
+        for l, b in enumerate(mlp.bs):
+            b.copy_(torch.from_numpy(b0s[l].astype(np.float32)))
+
+
+def test_training_step_is_bit_reproducible():
+    cfg = CASES["train-mix"]
+    results = []
+    for _ in range(2):
+        t = Trainer(cfg)
+        for _step in range(2):
+            t.backward()
+            E.dlrm_sparse_sgd(t.g.T, t.g.bot, t.g.top, cfg.B, t.nnz, cfg.lr, t.grads)
+        torch.cuda.synchronize()
+        results.append([t.g.tables.cpu()] + [w.cpu() for w in t.g.bot.Ws + t.g.top.Ws + t.g.bot.bs + t.g.top.bs])
+    for a, b in zip(*results):
+        assert torch.equal(a, b)
