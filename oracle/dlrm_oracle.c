@@ -285,12 +285,28 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
 /* Magnitude companion of linear_backward (error yardstick, not part of the
  * method): given sY >= |dY| (an elementwise bound on the size of the output
  * gradient and of its rounding error), masks it like dY, and returns
- * sW = sum_b sY |A|, sb = sum_b sY and sA = sY |W|. */
-static void linear_backward_magnitude(int B, int n_in, int n_out, const double* W, const double* A, const double* Y,
-                                      double* sY, double* sW, double* sb, double* sA, int relu) {
+ * sW = sum_b sY |A|, sb = sum_b sY and sA = sY |W|. A ReLU unit whose
+ * pre-activation lies within kink_eps of its own size (|b| + sum |W||A|) may
+ * fall on either side of zero in fp32, so its gradient size is kept. */
+static void linear_backward_magnitude(int B, int n_in, int n_out, const double* W, const double* bias,
+                                      const double* A, const double* Y, double* sY, double* sW, double* sb,
+                                      double* sA, int relu, double kink_eps) {
     if (relu) {
-        for (int64_t q = 0; q < (int64_t)B * n_out; ++q)
-            if (!(Y[q] > 0.0)) sY[q] = 0.0;
+#pragma omp parallel for schedule(static)
+        for (int b = 0; b < B; ++b) {
+            for (int o = 0; o < n_out; ++o) {
+                const int64_t q = (int64_t)b * n_out + o;
+                if (Y[q] > 0.0) continue;
+                double pre = bias[o], size = fabs(bias[o]);
+                const double* w = W + (int64_t)o * n_in;
+                const double* a = A + (int64_t)b * n_in;
+                for (int i = 0; i < n_in; ++i) {
+                    pre += w[i] * a[i];
+                    size += fabs(w[i] * a[i]);
+                }
+                if (!(fabs(pre) <= kink_eps * size)) sY[q] = 0.0;
+            }
+        }
     }
 #pragma omp parallel for schedule(static)
     for (int o = 0; o < n_out; ++o) {
@@ -448,13 +464,14 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
      * backward chain on sizes, sY >= |dY|, so that each gradient can be judged
      * against the sizes of the terms it sums, including upstream gradients. */
     if (bot_dW_s || bot_db_s || top_dW_s || top_db_s || table_grad_s) {
+        const double KINK_EPS = 1e-4;   /* well above the fp32 forward's relative rounding */
         double* sY = (double*)malloc(sizeof(double) * (size_t)B);
         for (int b = 0; b < B; ++b) sY[b] = fabs(sigmoid(z[b]) - labels[b]) / B;
         for (int l = M->n_top - 1; l >= 0; --l) {
             double* sA = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
-            linear_backward_magnitude(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], top_act[l], top_act[l + 1],
-                                      sY, top_dW_s ? top_dW_s[l] : NULL, top_db_s ? top_db_s[l] : NULL, sA,
-                                      l < M->n_top - 1);
+            linear_backward_magnitude(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], M->top_b[l], top_act[l],
+                                      top_act[l + 1], sY, top_dW_s ? top_dW_s[l] : NULL,
+                                      top_db_s ? top_db_s[l] : NULL, sA, l < M->n_top - 1, KINK_EPS);
             free(sY);
             sY = sA;
         }
@@ -481,8 +498,9 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
         for (int b = 0; b < B; ++b) memcpy(sB + (int64_t)b * d, sX + (int64_t)b * (K + 1) * d, sizeof(double) * d);
         for (int l = M->n_bot - 1; l >= 0; --l) {
             double* sA = (l > 0) ? (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]) : NULL;
-            linear_backward_magnitude(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], bot_act[l], bot_act[l + 1],
-                                      sB, bot_dW_s ? bot_dW_s[l] : NULL, bot_db_s ? bot_db_s[l] : NULL, sA, 1);
+            linear_backward_magnitude(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], M->bot_b[l], bot_act[l],
+                                      bot_act[l + 1], sB, bot_dW_s ? bot_dW_s[l] : NULL,
+                                      bot_db_s ? bot_db_s[l] : NULL, sA, 1, KINK_EPS);
             free(sB);
             sB = sA;
         }
