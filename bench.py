@@ -348,6 +348,87 @@ def run_ours(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_train(args, cfg, rank, world, local_rank):
+    """Training workload: a step is dlrm_backward (forward with saved activations, BCE, backward, row sort)
+    plus dlrm_sparse_sgd (touched rows and MLP parameters) on one batch."""
+    import torch
+    import torch.distributed as dist
+
+    import embedding_bags_dot_b200 as E
+    from synth import device as sd
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    E.lib()
+    sd.build_fill()
+    tables = sd.tables_on_device(cfg, device=dev)
+    T = E.Tables(tables, cfg.rows, cfg.d)
+    bot = E.MLP(*sd.mlp_on_device(cfg, "bottom", dev))
+    top = E.MLP(*sd.mlp_on_device(cfg, "top", dev))
+    ws = E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, cfg.B, 1), dev)
+    ids = tuple(rank * POOL + j for j in range(POOL))
+    perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
+    batches = gen.make_batches(cfg, ids, perms=perms)
+    dev_b = [sd.batch_on_device(b, dev) for b in batches]
+    nnz_max = max(b.indices.size for b in batches)
+    grads = torch.zeros(max(E.dlrm_grads_size(T, bot, top, cfg.B, int(b.indices.size)) for b in batches),
+                        dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    loss = torch.zeros(1, device=dev)
+
+    def step(i, ev=None):
+        b = dev_b[i % POOL]
+        nnz = int(b["indices"].numel())
+        if ev is not None:
+            ev[0].record(stream)
+        E.dlrm_backward(T, bot, top, cfg.B, b["dense"], b["offsets"], b["indices"], b["labels"], grads, ws, loss=loss,
+                        stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        E.dlrm_sparse_sgd(T, bot, top, cfg.B, nnz, cfg.lr, grads, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    st = E.dlrm_check_error(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device error record after warm-up: {st}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    n0 = E.dlrm_launch_count()
+    for i in range(args.steps):
+        step(i, evs[i])
+    n1 = E.dlrm_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    bwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    sgd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    samples = cfg.B * args.steps * world
+    if rank == 0:
+        out = {"metric": "DLRM training samples/s on 1 B200 (forward + backward + sparse SGD)",
+               "value": samples / (total_ms * 1e-3), "unit": "samples/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+               "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "lr": cfg.lr,
+                          "nnz_max": nnz_max},
+               "kernels_ms_per_step": {"dlrm_backward": bwd, "dlrm_sparse_sgd": sgd},
+               "loss_last": float(loss.item()), "gpu_launches": int(n1 - n0), "clocks": clk}
+        print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,6 +461,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if cfg.training:
+            return run_train(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
