@@ -312,6 +312,243 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+
+// ------------------------------------------------------------------ 2-SM variant
+//
+// A cluster of two CTAs (one per SM of a pair) computes a 256x256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): CTA r loads rows
+// [128 r, 128 r + 128) of the A tile and of the W tile (its halves of M and
+// N), so each SM streams 32 KB per 64-deep k-block instead of 48 KB. The
+// leader (rank 0) issues the MMAs; both CTAs' TMA loads complete on the
+// leader's full barrier; the MMA commits are multicast to both CTAs' empty and
+// accumulator-full barriers; both CTAs' epilogues release the accumulator on
+// the leader's barrier. Each CTA's TMEM holds the 128 rows of its M half.
+constexpr int BN2 = 256, STAGES2 = 6;
+constexpr int A2_BYTES = 128 * BK * 2;
+constexpr int B2_BYTES = (BN2 / 2) * BK * 2;
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512;
+
+struct Bars2 {
+    unsigned long long full[STAGES2];
+    unsigned long long empty[STAGES2];
+    unsigned long long tfull[2];
+    unsigned long long tempty[2];
+    unsigned long long drain;
+    unsigned int tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_rank(uint32_t shared_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(shared_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t leader_bar, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void umma2(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accum) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(id), "r"(accum));
+}
+// arrive on the barrier at this offset in both CTAs of the pair once all prior MMAs complete
+__device__ __forceinline__ void umma2_commit_both(unsigned long long* bar) {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            su32(bar)),
+        "h"(mask)
+        : "memory");
+}
+
+__host__ __device__ constexpr uint32_t idesc2(int ab_fmt) {
+    return (1u << 4) | ((uint32_t)ab_fmt << 7) | ((uint32_t)ab_fmt << 10) | ((uint32_t)(BN2 >> 3) << 17) |
+           ((uint32_t)(256 >> 4) << 24);
+}
+
+template <typename TC, int ACT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    linear_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, int M, int N,
+                      int K, const float* __restrict__ bias, TC* __restrict__ C, long long ldc, uint32_t id,
+                      ErrRecord* err) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = su32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    Bars2* bars = reinterpret_cast<Bars2*>(gbase + STAGES2 * STAGE2_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int npair = gridDim.x >> 1, pair = blockIdx.x >> 1;
+    const int nbn = (N + BN2 - 1) / BN2;
+    const int ntiles = ((M + 255) / 256) * nbn;
+    const int nk = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES2; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bars->tfull[a], 1);
+            mbar_init(&bars->tempty[a], 8);   // lane 0 of 4 epilogue warps in each CTA
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars->tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    fence_before();
+    cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA signal
+    fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int* abort = &bars->abort;
+    bool timed_out = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW)) : "memory");
+            int s = 0;
+            uint32_t ph = 0;
+            for (int t = pair; t < ntiles && !timed_out; t += npair) {
+                const int mb = t / nbn, nb = t - mb * nbn;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&bars->empty[s], ph ^ 1u, abort)) {
+                        timed_out = true;
+                        break;
+                    }
+                    const uint32_t sa = base + s * STAGE2_BYTES;
+                    const uint32_t lead_full = map_rank(su32(&bars->full[s]), 0);
+                    if (leader) mbar_expect_tx(&bars->full[s], 2 * STAGE2_BYTES);
+                    tma_load_2d_pair(sa, &mapA, lead_full, kb * BK, mb * 256 + (int)rank * 128);
+                    tma_load_2d_pair(sa + A2_BYTES, &mapW, lead_full, kb * BK, nb * BN2 + (int)rank * (BN2 / 2));
+                    if (++s == STAGES2) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (timed_out) *abort = 1;
+            // every load this CTA issued completes before it may exit: wait (bounded) for the
+            // empty barriers, which the leader's MMA commits after consuming each stage
+            for (int q = 0; q < STAGES2; ++q) {
+                mbar_wait(&bars->empty[s], ph ^ 1u, abort, true);
+                if (++s == STAGES2) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            int s = 0;
+            uint32_t ph = 0;
+            int i = 0;
+            for (int t = pair; t < ntiles && !timed_out; t += npair, ++i) {
+                const int acc = i & 1;
+                const uint32_t use = (uint32_t)(i >> 1);
+                if (!mbar_wait(&bars->tempty[acc], (use & 1u) ^ 1u, abort)) {
+                    timed_out = true;
+                    break;
+                }
+                fence_after();
+                const uint32_t d = tmem + (uint32_t)(acc * BN2);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&bars->full[s], ph, abort)) {
+                        timed_out = true;
+                        break;
+                    }
+                    fence_after();
+                    const uint32_t sa = base + s * STAGE2_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma2(d, sdesc(sa + k * 32), sdesc(sa + A2_BYTES + k * 32), id, (kb | k) != 0);
+                    umma2_commit_both(&bars->empty[s]);
+                    if (++s == STAGES2) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (timed_out) break;
+                umma2_commit_both(&bars->tfull[acc]);
+            }
+            if (timed_out) *abort = 1;
+            umma2_commit_both(&bars->drain);
+            mbar_wait(&bars->drain, 0, abort, true);
+        } else if (lane == 0) {
+            // the peer's MMA-issue thread has nothing to issue; it waits for the leader's drain
+            mbar_wait(&bars->drain, 0, abort, true);
+        }
+    } else {
+        const int q = warp & 3;
+        const uint32_t lead_tempty0 = map_rank(su32(&bars->tempty[0]), 0);
+        const uint32_t lead_tempty1 = map_rank(su32(&bars->tempty[1]), 0);
+        int i = 0;
+        for (int t = pair; t < ntiles && !timed_out; t += npair, ++i) {
+            const int acc = i & 1;
+            const uint32_t use = (uint32_t)(i >> 1);
+            if (!mbar_wait(&bars->tfull[acc], use & 1u, abort)) {
+                timed_out = true;
+                break;
+            }
+            fence_after();
+            const int mb = t / nbn, nb = t - mb * nbn;
+            const long long m = (long long)mb * 256 + (long long)rank * 128 + q * 32 + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2);
+#pragma unroll 1
+            for (int c = 0; c < BN2 / 32; ++c) {
+                const int n0 = nb * BN2 + c * 32;
+                if (n0 >= N) break;
+                uint32_t r[32];
+                tmem_ld32(taddr + c * 32, r);
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float bj = (n0 + j < N) ? __ldg(bias + n0 + j) : 0.f;
+                    v[j] = act_fn<ACT>(__uint_as_float(r[j]) + bj);
+                }
+                if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
+            }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc ? lead_tempty1 : lead_tempty0);
+        }
+        if (timed_out) *abort = 1;
+    }
+
+    if (timed_out && lane == 0) atomicOr(&err->flags, (unsigned)ERR_TIMEOUT);
+    fence_before();
+    cluster_sync_all();   // no CTA frees TMEM or exits while its pair still signals it
+    fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -368,6 +605,19 @@ static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, int M,
     return DLRM_OK;
 }
 
+template <typename TC, int ACT>
+static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, int M, int N, int K, const float* bias,
+                             void* C, int ldc, uint32_t id, ErrRecord* err, cudaStream_t st) {
+    auto kern = linear_tc2_kernel<TC, ACT>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+    const int ntiles = ((M + 255) / 256) * ((N + BN2 - 1) / BN2);
+    const int pairs = sm_count() / 2;
+    const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
+    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, M, N, K, bias, static_cast<TC*>(C), (long long)ldc, id, err);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
 }  // namespace tc
 
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
@@ -384,15 +634,25 @@ bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, in
 dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st) {
+    // 256-row tiles on SM pairs when there are enough of them to fill the GPU, 128-row tiles otherwise
+    const bool pair = M >= 256 * 16;
     CUtensorMap ma, mw;
-    if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) || !tc::make_map(&mw, W, a_dt, K, N, ldw, tc::BN))
+    if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) ||
+        !tc::make_map(&mw, W, a_dt, K, N, ldw, pair ? tc::BN2 / 2 : tc::BN))
         return DLRM_ERR_CUDA;
-    const uint32_t id = tc::idesc(a_dt == DLRM_BF16 ? 1 : 0);
+    const int fmt = a_dt == DLRM_BF16 ? 1 : 0;
+    const uint32_t id = pair ? tc::idesc2(fmt) : tc::idesc(fmt);
 #define DLRM_TC(TC)                                                                                             \
     switch (act) {                                                                                              \
-        case DLRM_ACT_RELU: return tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st);       \
-        case DLRM_ACT_SIGMOID: return tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st); \
-        default: return tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st);                  \
+        case DLRM_ACT_RELU:                                                                                     \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st)          \
+                        : tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st);          \
+        case DLRM_ACT_SIGMOID:                                                                                  \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st)       \
+                        : tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st);       \
+        default:                                                                                                \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st)          \
+                        : tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st);          \
     }
     if (c_dt == DLRM_F32) {
         DLRM_TC(float)
