@@ -112,7 +112,7 @@ __device__ __forceinline__ void umma_commit(unsigned long long* bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
         "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -121,8 +121,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 template <int ACT>
 __device__ __forceinline__ float act_fn(float v) {
@@ -151,7 +151,51 @@ __device__ __forceinline__ void store_chunk(TC* __restrict__ C, long long ldc, l
             for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
     } else {
-        for (int j = 0; j < 32 && n + j < N; ++j) row[n + j] = Cvt<TC>::from_f(v[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n + j < N) row[n + j] = Cvt<TC>::from_f(v[j]);
+    }
+}
+
+// Epilogue of one 128-row accumulator slice: this warp's 32 TMEM lanes, BN columns from
+// column `col0` of TMEM, output rows m, columns n_base.. . The TMEM load of chunk c + 1 is in
+// flight while chunk c is converted and stored.
+template <typename TC, int ACT, int NCOL>
+__device__ __forceinline__ void epilogue_rows(uint32_t taddr, long long m, int M, int n_base, int N,
+                                              const float* __restrict__ bias, TC* __restrict__ C, long long ldc) {
+    constexpr int NCH = NCOL / 32;
+    uint32_t ra[32], rb[32];
+    int nch = (N - n_base + 31) / 32;
+    nch = nch < NCH ? nch : NCH;
+    if (nch <= 0) return;
+    tmem_ld32_issue(taddr, ra);
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+        tmem_ld_wait();
+        uint32_t cur[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) cur[j] = ra[j];
+        if (c + 1 < nch) tmem_ld32_issue(taddr + (c + 1) * 32, rb);
+        const int n0 = n_base + c * 32;
+        float v[32];
+        if (n0 + 32 <= N) {
+            const float4* b4 = reinterpret_cast<const float4*>(bias + n0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 bq = __ldg(b4 + q);
+                v[4 * q + 0] = act_fn<ACT>(__uint_as_float(cur[4 * q + 0]) + bq.x);
+                v[4 * q + 1] = act_fn<ACT>(__uint_as_float(cur[4 * q + 1]) + bq.y);
+                v[4 * q + 2] = act_fn<ACT>(__uint_as_float(cur[4 * q + 2]) + bq.z);
+                v[4 * q + 3] = act_fn<ACT>(__uint_as_float(cur[4 * q + 3]) + bq.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                v[j] = act_fn<ACT>(__uint_as_float(cur[j]) + ((n0 + j < N) ? __ldg(bias + n0 + j) : 0.f));
+        }
+        if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
     }
 }
 
@@ -283,20 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int mb = t / nbn, nb = t - mb * nbn;
             const long long m = (long long)mb * BM + q * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n0 = nb * BN + c * 32;
-                if (n0 >= N) break;  // uniform across the warp
-                uint32_t r[32];
-                tmem_ld32(taddr + c * 32, r);
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float b = (n0 + j < N) ? __ldg(bias + n0 + j) : 0.f;
-                    v[j] = act_fn<ACT>(__uint_as_float(r[j]) + b);
-                }
-                if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
-            }
+            epilogue_rows<TC, ACT, BN>(taddr, m, M, nb * BN, N, bias, C, ldc);
             fence_before();
             mbar_arrive(&bars->tempty[acc]);
         }
@@ -519,20 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int mb = t / nbn, nb = t - mb * nbn;
             const long long m = (long long)mb * 256 + (long long)rank * 128 + q * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2);
-#pragma unroll 1
-            for (int c = 0; c < BN2 / 32; ++c) {
-                const int n0 = nb * BN2 + c * 32;
-                if (n0 >= N) break;
-                uint32_t r[32];
-                tmem_ld32(taddr + c * 32, r);
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float bj = (n0 + j < N) ? __ldg(bias + n0 + j) : 0.f;
-                    v[j] = act_fn<ACT>(__uint_as_float(r[j]) + bj);
-                }
-                if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
-            }
+            epilogue_rows<TC, ACT, BN2>(taddr, m, M, nb * BN2, N, bias, C, ldc);
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? lead_tempty1 : lead_tempty0);
@@ -621,11 +639,11 @@ static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, int M
 }  // namespace tc
 
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
-                         int ldw, void* C, dlrm_dtype c_dt, int ldc) {
+                         int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc) {
     if (a_dt != w_dt || a_dt == DLRM_F32) return false;
     if (M < 1 || N < 2 || K < 16) return false;
     if ((lda % 8) || (ldw % 8)) return false;
-    if (((uintptr_t)A & 15) || ((uintptr_t)W & 15) || ((uintptr_t)C & 15)) return false;
+    if (((uintptr_t)A & 15) || ((uintptr_t)W & 15) || ((uintptr_t)C & 15) || ((uintptr_t)bias & 15)) return false;
     if (c_dt != DLRM_F32 && c_dt != a_dt) return false;
     if (ldc % (c_dt == DLRM_F32 ? 4 : 8)) return false;
     return tc::encode_fn() != nullptr;

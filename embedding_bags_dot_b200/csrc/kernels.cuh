@@ -38,7 +38,7 @@ dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, i
                           ErrRecord* err, cudaStream_t st);
 
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
-                         int ldw, void* C, dlrm_dtype c_dt, int ldc);
+                         int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc);
 dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st);

@@ -158,7 +158,7 @@ dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, i
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
                           ErrRecord* err, cudaStream_t st) {
     if (M == 0) return DLRM_OK;
-    if (N > 1 && linear_tc_supported(M, N, K, A, a_dt, lda, W, w_dt, ldw, C, c_dt, ldc))
+    if (N > 1 && linear_tc_supported(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc))
         return launch_linear_tc(M, N, K, A, a_dt, lda, W, ldw, bias, C, c_dt, ldc, act, err, st);
     return launch_linear_ffma(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st);
 }
