@@ -8,10 +8,11 @@
 //               K-major, 128-byte swizzle) into a 4-stage shared-memory ring;
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
 //               and one thread issues tcgen05.mma (M=128, N=256, K=16);
-//   warps 2..5  epilogue: tcgen05.ld of the finished accumulator (each warp
-//               owns the 32 TMEM lanes of its quadrant), bias, activation,
-//               conversion and global stores, while the MMA warp already
-//               fills the other accumulator.
+//   warps 2..9  epilogue: tcgen05.ld of the finished accumulator (each warp
+//               owns the 32 TMEM lanes of its quadrant and half of the
+//               columns), bias, activation, conversion into a 128-byte
+//               swizzled shared-memory stage written out by TMA bulk tensor
+//               stores, while the MMA warp already fills the other accumulator.
 // Shared-memory stages are released by tcgen05.commit onto an mbarrier. All
 // waits are bounded: on timeout the kernel records DLRM_ERR_TIMEOUT in the
 // error record, drains its own copies and MMAs (again bounded), frees TMEM
@@ -29,8 +30,11 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int EPI_WARPS = 8;                       // two per TMEM lane quadrant, each half of the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int STAGE_OUT_BYTES = 32 * 128;          // per epilogue warp: 32 rows x 128 bytes, 128-byte swizzle
+constexpr int OUT_BYTES = EPI_WARPS * STAGE_OUT_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + 1024 + 256;
 constexpr long long WAIT_LIMIT = 1ll << 26;
 
 struct Bars {
@@ -131,84 +135,88 @@ __device__ __forceinline__ float act_fn(float v) {
     return v;
 }
 
-template <typename TC>
-__device__ __forceinline__ void store_chunk(TC* __restrict__ C, long long ldc, long long m, int n, int N, const float* v) {
-    TC* row = C + m * ldc;
-    if (n + 32 <= N) {
-        if constexpr (sizeof(TC) == 2) {
-            uint32_t w[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                TC lo = Cvt<TC>::from_f(v[2 * j]), hi = Cvt<TC>::from_f(v[2 * j + 1]);
-                w[j] = (uint32_t)(*reinterpret_cast<uint16_t*>(&lo)) | ((uint32_t)(*reinterpret_cast<uint16_t*>(&hi)) << 16);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(row + n);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        } else {
-            float4* dst = reinterpret_cast<float4*>(row + n);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (n + j < N) row[n + j] = Cvt<TC>::from_f(v[j]);
-    }
+// Output tile rows of one epilogue warp, written through shared memory by TMA: for
+// each 128-byte wide column chunk, the 32 lanes (one row each) convert their
+// TMEM values, store them 128-byte swizzled into the warp's staging buffer,
+// and lane 0 issues a bulk tensor store of the 32 x chunk box (rows and
+// columns beyond the tensor are clipped by the TMA unit).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Epilogue of one 128-row accumulator slice: this warp's 32 TMEM lanes, BN columns from
-// column `col0` of TMEM, output rows m, columns n_base.. . The TMEM load of chunk c + 1 is in
-// flight while chunk c is converted and stored.
-template <typename TC, int ACT, int NCOL>
-__device__ __forceinline__ void epilogue_rows(uint32_t taddr, long long m, int M, int n_base, int N,
-                                              const float* __restrict__ bias, TC* __restrict__ C, long long ldc) {
-    constexpr int NCH = NCOL / 32;
-    uint32_t ra[32], rb[32];
-    int nch = (N - n_base + 31) / 32;
-    nch = nch < NCH ? nch : NCH;
-    if (nch <= 0) return;
-    tmem_ld32_issue(taddr, ra);
+template <typename TC, int ACT, int NCOLS>
+__device__ __forceinline__ void epilogue_tma(uint32_t taddr, int m0, int n_base, int N, const float* __restrict__ bias,
+                                             const CUtensorMap* mapC, unsigned char* stage, uint32_t stage_s) {
+    constexpr int CW = 128 / (int)sizeof(TC);   // columns per chunk: 64 (16-bit) or 32 (fp32)
+    constexpr int NL = CW / 32;                 // 32-column TMEM loads per chunk
+    const int lane = threadIdx.x & 31;
 #pragma unroll 1
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < NCOLS / CW; ++c) {
+        const int n0 = n_base + c * CW;
+        if (n0 >= N) break;   // uniform across the warp
+        uint32_t r[NL][32];
+#pragma unroll
+        for (int h = 0; h < NL; ++h) tmem_ld32_issue(taddr + c * CW + 32 * h, r[h]);
         tmem_ld_wait();
-        uint32_t cur[32];
+        float v[CW];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) cur[j] = ra[j];
-        if (c + 1 < nch) tmem_ld32_issue(taddr + (c + 1) * 32, rb);
-        const int n0 = n_base + c * 32;
-        float v[32];
-        if (n0 + 32 <= N) {
-            const float4* b4 = reinterpret_cast<const float4*>(bias + n0);
+        for (int h = 0; h < NL; ++h) {
+            const int nh = n0 + 32 * h;
+            if (nh + 32 <= N) {
+                const float4* b4 = reinterpret_cast<const float4*>(bias + nh);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 bq = __ldg(b4 + q);
-                v[4 * q + 0] = act_fn<ACT>(__uint_as_float(cur[4 * q + 0]) + bq.x);
-                v[4 * q + 1] = act_fn<ACT>(__uint_as_float(cur[4 * q + 1]) + bq.y);
-                v[4 * q + 2] = act_fn<ACT>(__uint_as_float(cur[4 * q + 2]) + bq.z);
-                v[4 * q + 3] = act_fn<ACT>(__uint_as_float(cur[4 * q + 3]) + bq.w);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 bq = __ldg(b4 + q);
+                    v[32 * h + 4 * q + 0] = act_fn<ACT>(__uint_as_float(r[h][4 * q + 0]) + bq.x);
+                    v[32 * h + 4 * q + 1] = act_fn<ACT>(__uint_as_float(r[h][4 * q + 1]) + bq.y);
+                    v[32 * h + 4 * q + 2] = act_fn<ACT>(__uint_as_float(r[h][4 * q + 2]) + bq.z);
+                    v[32 * h + 4 * q + 3] = act_fn<ACT>(__uint_as_float(r[h][4 * q + 3]) + bq.w);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    v[32 * h + j] = act_fn<ACT>(__uint_as_float(r[h][j]) + ((nh + j < N) ? __ldg(bias + nh + j) : 0.f));
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                v[j] = act_fn<ACT>(__uint_as_float(cur[j]) + ((n0 + j < N) ? __ldg(bias + n0 + j) : 0.f));
         }
-        if (m < M) store_chunk<TC>(C, ldc, m, n0, N, v);
+        if (lane == 0) bulk_wait_read0();   // the previous chunk's store has read the staging buffer
+        __syncwarp();
+        unsigned char* row = stage + lane * 128;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
+        for (int q = 0; q < 8; ++q) {
+            uint4 w;
+            if constexpr (sizeof(TC) == 2) {
+                TC t[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = Cvt<TC>::from_f(v[8 * q + e]);
+                w = *reinterpret_cast<const uint4*>(t);
+            } else {
+                w = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                               __float_as_uint(v[4 * q + 3]));
+            }
+            *reinterpret_cast<uint4*>(row + 16 * (q ^ (lane & 7))) = w;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) tma_store_2d(mapC, stage_s, n0, m0);
     }
 }
 
 template <typename TC, int ACT>
 __global__ void __launch_bounds__(THREADS, 1)
-    linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, int M, int N,
-                     int K, const float* __restrict__ bias, TC* __restrict__ C, long long ldc, uint32_t id,
-                     ErrRecord* err) {
+    linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
+                     const __grid_constant__ CUtensorMap mapC, int M, int N, int K, const float* __restrict__ bias,
+                     uint32_t id, ErrRecord* err) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    Bars* bars = reinterpret_cast<Bars*>(gbase + STAGES * STAGE_BYTES);
+    Bars* bars = reinterpret_cast<Bars*>(gbase + STAGES * STAGE_BYTES + OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nbn = (N + BN - 1) / BN;
     const int ntiles = ((M + BM - 1) / BM) * nbn;
@@ -221,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&bars->tfull[a], 1);
-            mbar_init(&bars->tempty[a], 128);
+            mbar_init(&bars->tempty[a], EPI_WARPS);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -314,7 +322,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_wait(&bars->drain, 0, abort, true);
         }
     } else {
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int ew = warp - 2;   // epilogue warp 0..7
+        const int q = warp & 3;    // TMEM lane quadrant this warp may access
+        const int h = ew >> 2;     // which half of the tile's columns
+        unsigned char* stage = gbase + STAGES * STAGE_BYTES + ew * STAGE_OUT_BYTES;
+        const uint32_t stage_s = base + STAGES * STAGE_BYTES + ew * STAGE_OUT_BYTES;
         int i = 0;
         for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
             const int acc = i & 1;
@@ -325,13 +337,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             fence_after();
             const int mb = t / nbn, nb = t - mb * nbn;
-            const long long m = (long long)mb * BM + q * 32 + lane;
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            epilogue_rows<TC, ACT, BN>(taddr, m, M, nb * BN, N, bias, C, ldc);
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + h * (BN / 2));
+            epilogue_tma<TC, ACT, BN / 2>(taddr, mb * BM + q * 32, nb * BN + h * (BN / 2), N, bias, &mapC, stage,
+                                          stage_s);
             fence_before();
-            mbar_arrive(&bars->tempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tempty[acc]);
         }
         if (timed_out) *abort = 1;
+        if (lane == 0) bulk_wait_all0();
     }
 
     if (timed_out && lane == 0) atomicOr(&err->flags, (unsigned)ERR_TIMEOUT);
@@ -358,7 +372,7 @@ constexpr int BN2 = 256, STAGES2 = 6;
 constexpr int A2_BYTES = 128 * BK * 2;
 constexpr int B2_BYTES = (BN2 / 2) * BK * 2;
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
-constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + OUT_BYTES + 1024 + 256;
 
 struct Bars2 {
     unsigned long long full[STAGES2];
@@ -418,14 +432,14 @@ __host__ __device__ constexpr uint32_t idesc2(int ab_fmt) {
 
 template <typename TC, int ACT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    linear_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, int M, int N,
-                      int K, const float* __restrict__ bias, TC* __restrict__ C, long long ldc, uint32_t id,
-                      ErrRecord* err) {
+    linear_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
+                      const __grid_constant__ CUtensorMap mapC, int M, int N, int K, const float* __restrict__ bias,
+                      uint32_t id, ErrRecord* err) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    Bars2* bars = reinterpret_cast<Bars2*>(gbase + STAGES2 * STAGE2_BYTES);
+    Bars2* bars = reinterpret_cast<Bars2*>(gbase + STAGES2 * STAGE2_BYTES + OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
@@ -441,7 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&bars->tfull[a], 1);
-            mbar_init(&bars->tempty[a], 8);   // lane 0 of 4 epilogue warps in each CTA
+            mbar_init(&bars->tempty[a], 2 * EPI_WARPS);   // lane 0 of every epilogue warp of both CTAs
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -535,7 +549,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_wait(&bars->drain, 0, abort, true);
         }
     } else {
+        const int ew = warp - 2;
         const int q = warp & 3;
+        const int h = ew >> 2;
+        unsigned char* stage = gbase + STAGES2 * STAGE2_BYTES + ew * STAGE_OUT_BYTES;
+        const uint32_t stage_s = base + STAGES2 * STAGE2_BYTES + ew * STAGE_OUT_BYTES;
         const uint32_t lead_tempty0 = map_rank(su32(&bars->tempty[0]), 0);
         const uint32_t lead_tempty1 = map_rank(su32(&bars->tempty[1]), 0);
         int i = 0;
@@ -548,14 +566,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             fence_after();
             const int mb = t / nbn, nb = t - mb * nbn;
-            const long long m = (long long)mb * 256 + (long long)rank * 128 + q * 32 + lane;
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2);
-            epilogue_rows<TC, ACT, BN2>(taddr, m, M, nb * BN2, N, bias, C, ldc);
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2 + h * (BN2 / 2));
+            epilogue_tma<TC, ACT, BN2 / 2>(taddr, mb * 256 + (int)rank * 128 + q * 32, nb * BN2 + h * (BN2 / 2), N,
+                                           bias, &mapC, stage, stage_s);
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? lead_tempty1 : lead_tempty0);
         }
         if (timed_out) *abort = 1;
+        if (lane == 0) bulk_wait_all0();
     }
 
     if (timed_out && lane == 0) atomicOr(&err->flags, (unsigned)ERR_TIMEOUT);
@@ -585,14 +604,18 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-static bool make_map(CUtensorMap* map, const void* ptr, dlrm_dtype dt, int inner, int outer, int ld, int box_outer) {
+static bool make_map(CUtensorMap* map, const void* ptr, dlrm_dtype dt, int inner, int outer, int ld, int box_outer,
+                     int box_inner = BK) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_outer};
+    const size_t es = dt == DLRM_F32 ? 4 : 2;
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * es};
+    const cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType t = dt == DLRM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType t = dt == DLRM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                  : dt == DLRM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     return enc(map, t, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -612,26 +635,26 @@ static int sm_count() {
 }
 
 template <typename TC, int ACT>
-static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, int M, int N, int K, const float* bias,
-                            void* C, int ldc, uint32_t id, ErrRecord* err, cudaStream_t st) {
+static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc, int M, int N, int K,
+                            const float* bias, uint32_t id, ErrRecord* err, cudaStream_t st) {
     auto kern = linear_tc_kernel<TC, ACT>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     const int ntiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = ntiles < sm_count() ? ntiles : sm_count();
-    kern<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mw, M, N, K, bias, static_cast<TC*>(C), (long long)ldc, id, err);
+    kern<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
 
 template <typename TC, int ACT>
-static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, int M, int N, int K, const float* bias,
-                             void* C, int ldc, uint32_t id, ErrRecord* err, cudaStream_t st) {
+static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc, int M, int N, int K,
+                             const float* bias, uint32_t id, ErrRecord* err, cudaStream_t st) {
     auto kern = linear_tc2_kernel<TC, ACT>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
     const int ntiles = ((M + 255) / 256) * ((N + BN2 - 1) / BN2);
     const int pairs = sm_count() / 2;
     const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, M, N, K, bias, static_cast<TC*>(C), (long long)ldc, id, err);
+    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -654,23 +677,24 @@ dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt
                              cudaStream_t st) {
     // 256-row tiles on SM pairs when there are enough of them to fill the GPU, 128-row tiles otherwise
     const bool pair = M >= 256 * 16;
-    CUtensorMap ma, mw;
+    CUtensorMap ma, mw, mc;
     if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) ||
-        !tc::make_map(&mw, W, a_dt, K, N, ldw, pair ? tc::BN2 / 2 : tc::BN))
+        !tc::make_map(&mw, W, a_dt, K, N, ldw, pair ? tc::BN2 / 2 : tc::BN) ||
+        !tc::make_map(&mc, C, c_dt, N, M, ldc, 32, c_dt == DLRM_F32 ? 32 : 64))
         return DLRM_ERR_CUDA;
     const int fmt = a_dt == DLRM_BF16 ? 1 : 0;
     const uint32_t id = pair ? tc::idesc2(fmt) : tc::idesc(fmt);
 #define DLRM_TC(TC)                                                                                             \
     switch (act) {                                                                                              \
         case DLRM_ACT_RELU:                                                                                     \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st)          \
-                        : tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, M, N, K, bias, C, ldc, id, err, st);          \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_RELU>(ma, mw, mc, M, N, K, bias, id, err, st)              \
+                        : tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, mc, M, N, K, bias, id, err, st);              \
         case DLRM_ACT_SIGMOID:                                                                                  \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st)       \
-                        : tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, M, N, K, bias, C, ldc, id, err, st);       \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_SIGMOID>(ma, mw, mc, M, N, K, bias, id, err, st)           \
+                        : tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, mc, M, N, K, bias, id, err, st);           \
         default:                                                                                                \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st)          \
-                        : tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, M, N, K, bias, C, ldc, id, err, st);          \
+            return pair ? tc::launch_t2<TC, DLRM_ACT_NONE>(ma, mw, mc, M, N, K, bias, id, err, st)              \
+                        : tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, mc, M, N, K, bias, id, err, st);              \
     }
     if (c_dt == DLRM_F32) {
         DLRM_TC(float)
