@@ -55,10 +55,11 @@ dlrm_status check_mlp(const dlrm_mlp* m) {
     return DLRM_OK;
 }
 
-// Bytes of one hidden-activation buffer for the widest hidden layer of m.
+// Bytes of one activation buffer: the widest layer input of m (the first layer's input
+// is converted into such a buffer when it does not come in the MLP's dtype).
 size_t hidden_bytes(const dlrm_mlp* m, int B) {
     size_t w = 0;
-    for (int l = 1; l < m->n_layers; ++l) {
+    for (int l = 0; l < m->n_layers; ++l) {
         const size_t b = (size_t)dlrm_ld(m->dims[l], m->dt) * esize(m->dt);
         if (b > w) w = b;
     }
@@ -66,7 +67,7 @@ size_t hidden_bytes(const dlrm_mlp* m, int B) {
 }
 
 struct FwdLayout {
-    size_t x_dense, concat, act0, act1, total;
+    size_t x_dense, concat, act0, act1, cvt, total;
 };
 
 FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
@@ -85,16 +86,28 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
     off = align_up(off + h, 256);
     L.act1 = off;
     off = align_up(off + h, 256);
+    L.cvt = off;
+    off = align_up(off + h, 256);
     L.total = off;
     return L;
 }
 
-// The MLP chain: ReLU after hidden layers, final_act after the last layer.
+// The MLP chain: ReLU after hidden layers, final_act after the last layer. An fp32 input
+// to a 16-bit MLP is first converted (into cvt) so that every layer can take the
+// tensor-core path.
 dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out, int ld_out,
-                    int final_act, void* act0, void* act1, ErrRecord* err, cudaStream_t st) {
+                    int final_act, void* act0, void* act1, void* cvt, ErrRecord* err, cudaStream_t st) {
     const void* cur = in;
     dlrm_dtype cur_dt = in_dt;
     int cur_ld = ld_in;
+    if (in_dt != m->dt && m->dt != DLRM_F32 && cvt) {
+        const int ldk = dlrm_ld(m->dims[0], m->dt);
+        dlrm_status r = launch_convert(B, m->dims[0], in, in_dt, ld_in, cvt, m->dt, ldk, st);
+        if (r != DLRM_OK) return r;
+        cur = cvt;
+        cur_dt = m->dt;
+        cur_ld = ldk;
+    }
     for (int l = 0; l < m->n_layers; ++l) {
         const int K = m->dims[l], N = m->dims[l + 1];
         const int ldw = dlrm_ld(K, m->dt);
@@ -218,8 +231,8 @@ dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype 
     if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
     const size_t h = align_up(hidden_bytes(mlp, B), 256);
     char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
-    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, static_cast<ErrRecord*>(ws),
-                   cs(stream));
+    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, w + 2 * h,
+                   static_cast<ErrRecord*>(ws), cs(stream));
 }
 
 dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
@@ -243,13 +256,14 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
     void* concat = w + L.concat;
     const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
-    if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1, err,
-                     st)))
+    if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1,
+                     w + L.cvt, err, st)))
         return r;
     if ((r = launch_embbag_interact(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt,
                                     reinterpret_cast<ErrRecord*>(w), st)))
         return r;
-    return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, err, st);
+    return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, w + L.cvt, err,
+                   st);
 }
 
 }  // extern "C"

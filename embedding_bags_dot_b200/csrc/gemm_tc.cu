@@ -664,7 +664,7 @@ static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, const
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
                          int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc) {
     if (a_dt != w_dt || a_dt == DLRM_F32) return false;
-    if (M < 1 || N < 2 || K < 16) return false;
+    if (M < 1 || N < 2 || K < 1) return false;
     if ((lda % 8) || (ldw % 8)) return false;
     if (((uintptr_t)A & 15) || ((uintptr_t)W & 15) || ((uintptr_t)C & 15) || ((uintptr_t)bias & 15)) return false;
     if (c_dt != DLRM_F32 && c_dt != a_dt) return false;

@@ -37,6 +37,10 @@ dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, i
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
                           ErrRecord* err, cudaStream_t st);
 
+// out[b][c] = in[b][c] (converted) for c < K, zero up to ldo.
+dlrm_status launch_convert(int B, int K, const void* in, dlrm_dtype in_dt, int ldi, void* out, dlrm_dtype out_dt,
+                           int ldo, cudaStream_t st);
+
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
                          int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc);
 dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,

@@ -154,6 +154,41 @@ dlrm_status launch_linear_ffma(int M, int N, int K, const void* A, dlrm_dtype a_
     return DLRM_OK;
 }
 
+// out[b][c] = in[b][c] converted to out_dt for c < K, 0 for K <= c < ldo.
+template <typename TI, typename TO>
+__global__ void convert_kernel(int B, int K, const TI* __restrict__ in, int ldi, TO* __restrict__ out, int ldo) {
+    const long long n = (long long)B * ldo;
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+        const long long b = q / ldo;
+        const int c = (int)(q - b * ldo);
+        out[q] = Cvt<TO>::from_f(c < K ? Cvt<TI>::to_f(in[b * ldi + c]) : 0.f);
+    }
+}
+
+template <typename TI>
+static void convert_to(int B, int K, const void* in, int ldi, void* out, dlrm_dtype out_dt, int ldo, cudaStream_t st) {
+    long long blocks = ((long long)B * ldo + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    const TI* i = static_cast<const TI*>(in);
+    if (out_dt == DLRM_BF16)
+        convert_kernel<TI, __nv_bfloat16><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__nv_bfloat16*>(out), ldo);
+    else if (out_dt == DLRM_F16)
+        convert_kernel<TI, __half><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__half*>(out), ldo);
+    else
+        convert_kernel<TI, float><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<float*>(out), ldo);
+}
+
+dlrm_status launch_convert(int B, int K, const void* in, dlrm_dtype in_dt, int ldi, void* out, dlrm_dtype out_dt,
+                           int ldo, cudaStream_t st) {
+    if (B == 0) return DLRM_OK;
+    if (in_dt == DLRM_F32) convert_to<float>(B, K, in, ldi, out, out_dt, ldo, st);
+    else if (in_dt == DLRM_BF16) convert_to<__nv_bfloat16>(B, K, in, ldi, out, out_dt, ldo, st);
+    else convert_to<__half>(B, K, in, ldi, out, out_dt, ldo, st);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
 dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
                           ErrRecord* err, cudaStream_t st) {
