@@ -192,6 +192,29 @@ def run_reference(args, cfg, rank):
 METRIC = "DLRM samples/s on 1 B200; EmbeddingBag+interaction HBM GB/s as % of peak"
 
 
+# --------------------------------------------------------------------------- multi-rank plumbing (replicas)
+
+def rank_batch_ids(rank: int) -> tuple:
+    """Each rank benchmarks its own pool of seeded batches (independent replicas, weak scaling)."""
+    return tuple(rank * POOL + j for j in range(POOL))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the slowest rank's time bounds the whole job)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(samples_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job samples/s: every rank's samples over the slowest rank's time."""
+    return samples_per_rank * world / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def run_ours(args, cfg, rank, world, local_rank):
@@ -215,7 +238,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     ws = E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, cfg.B, 0), dev)
 
     # batch pool (independent per rank)
-    ids = tuple(rank * POOL + j for j in range(POOL))
+    ids = rank_batch_ids(rank)
     perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
     batches = gen.make_batches(cfg, ids, perms=perms)
     dev_b = [sd.batch_on_device(b, dev) for b in batches]
@@ -316,20 +339,14 @@ def run_ours(args, cfg, rank, world, local_rank):
     d2h = cfg.B * 4
 
     # max over ranks
-    def maxr(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    total_ms, e2e_ms = maxr(total_ms), maxr(e2e_ms)
-    k2_avg = maxr(float(np.mean(k2_ms)))
+    total_ms = max_over_ranks(total_ms, world, dev)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    k2_avg = max_over_ranks(float(np.mean(k2_ms)), world, dev)
     peak_hbm, peak_bf16, peak_kind = read_peaks()
     avg_algo = float(np.mean([algo_bytes[i % POOL] for i in range(args.steps)]))
     achieved = avg_algo / (k2_avg * 1e-3) / 1e9
     samples = cfg.B * args.steps * world
-    value = samples / (total_ms * 1e-3)
+    value = aggregate_rate(cfg.B * args.steps, world, total_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -356,7 +373,8 @@ def run_ours(args, cfg, rank, world, local_rank):
             "kernels_ms_per_step": {"bottom_mlp": float(np.mean(bot_ms)), "embbag_interact": float(np.mean(k2_ms)),
                                     "top_mlp": float(np.mean(top_ms))},
             "cpu_baseline": cpu,
-            "e2e": {"value": samples / (e2e_ms * 1e-3), "unit": "samples/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": aggregate_rate(cfg.B * args.steps, world, e2e_ms), "unit": "samples/s",
+                    "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
             "gpu_launches": int(n1 - n0),
             "clocks": clk,
@@ -383,7 +401,7 @@ def run_train(args, cfg, rank, world, local_rank):
     bot = E.MLP(*sd.mlp_on_device(cfg, "bottom", dev))
     top = E.MLP(*sd.mlp_on_device(cfg, "top", dev))
     ws = E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, cfg.B, 1), dev)
-    ids = tuple(rank * POOL + j for j in range(POOL))
+    ids = rank_batch_ids(rank)
     perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
     batches = gen.make_batches(cfg, ids, perms=perms)
     dev_b = [sd.batch_on_device(b, dev) for b in batches]
@@ -425,17 +443,14 @@ def run_train(args, cfg, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
-    total_ms = evs[0][0].elapsed_time(evs[-1][2])
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][2]), world, dev)
     bwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     sgd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     samples = cfg.B * args.steps * world
     if rank == 0:
         out = {"metric": "DLRM training samples/s on 1 B200 (forward + backward + sparse SGD)",
-               "value": samples / (total_ms * 1e-3), "unit": "samples/s", "n_gpus": world, "steps": args.steps,
+               "value": aggregate_rate(cfg.B * args.steps, world, total_ms), "unit": "samples/s", "n_gpus": world,
+               "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "lr": cfg.lr,
