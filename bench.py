@@ -461,6 +461,85 @@ def run_train(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_latency(args, cfg, rank, world, local_rank):
+    """Latency-bounded inference: forward latency and throughput against batch size, and the
+    aggregate throughput of several streams serving small batches side by side (batching and
+    co-location, as the companion paper's CPU study measures them)."""
+    import torch
+
+    import embedding_bags_dot_b200 as E
+    from synth import device as sd
+    from synth import shrink
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    E.lib()
+    sd.build_fill()
+    T = E.Tables(sd.tables_on_device(cfg, device=dev), cfg.rows, cfg.d)
+    bot = E.MLP(*sd.mlp_on_device(cfg, "bottom", dev))
+    top = E.MLP(*sd.mlp_on_device(cfg, "top", dev))
+    perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
+    sizes = [b for b in (1, 8, 64, 256, 1024, 4096, 16384, 65536) if b <= cfg.B]
+    rows = []
+    for B in sizes:
+        c = shrink(cfg, B=B)
+        bt = sd.batch_on_device(gen.make_batches(c, (rank * 100 + 1,), perms=perms)[0], dev)
+        ws = E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, B, 0), dev)
+        y = torch.empty(B, dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream(dev)
+        for _ in range(args.warmup):
+            E.dlrm_forward(T, bot, top, B, bt["dense"], bt["offsets"], bt["indices"], y, ws, st)
+        ms = []
+        for _ in range(max(args.steps, 20)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            E.dlrm_forward(T, bot, top, B, bt["dense"], bt["offsets"], bt["indices"], y, ws, st)
+            e1.record(st)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        ms.sort()
+        med, p99 = ms[len(ms) // 2], ms[min(len(ms) - 1, int(0.99 * len(ms)))]
+        rows.append({"batch": B, "latency_ms_p50": med, "latency_ms_p99": p99, "samples_per_s": B / (med * 1e-3)})
+    # co-location: S streams, each serving its own small batches
+    coloc = []
+    Bc = min(256, cfg.B)
+    c = shrink(cfg, B=Bc)
+    bts = [sd.batch_on_device(b, dev) for b in gen.make_batches(c, tuple(rank * 100 + 10 + j for j in range(4)),
+                                                                perms=perms)]
+    for S in (1, 2, 4):
+        streams = [torch.cuda.Stream(dev) for _ in range(S)]
+        wss = [E.alloc_workspace(E.dlrm_workspace_size(T, bot, top, Bc, 0), dev) for _ in range(S)]
+        ys = [torch.empty(Bc, dtype=torch.float32, device=dev) for _ in range(S)]
+        n_iter = max(args.steps, 20)
+
+        def burst():
+            for it in range(n_iter):
+                for j in range(S):
+                    b = bts[j]
+                    E.dlrm_forward(T, bot, top, Bc, b["dense"], b["offsets"], b["indices"], ys[j], wss[j], streams[j])
+
+        burst()
+        torch.cuda.synchronize(dev)
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(torch.cuda.current_stream(dev))
+        for sj in streams:
+            sj.wait_event(start)
+        burst()
+        ends = [torch.cuda.Event(enable_timing=True) for _ in streams]
+        for e, sj in zip(ends, streams):
+            e.record(sj)
+        torch.cuda.synchronize(dev)
+        dt = max(start.elapsed_time(e) for e in ends) * 1e-3
+        coloc.append({"streams": S, "batch": Bc, "samples_per_s": S * n_iter * Bc / dt,
+                      "ms_per_round": 1e3 * dt / n_iter})
+    if rank == 0:
+        print(json.dumps({"metric": "DLRM inference latency and throughput vs batch size on 1 B200",
+                          "unit": "ms", "higher_is_better": False, "data": "synthetic",
+                          "config": {"workload": workload_desc(cfg)}, "latency": rows, "colocation": coloc}),
+              flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,6 +551,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="smaller batch (profiling captures only)")
     ap.add_argument("--rows-cap", type=int, default=None, help="cap table rows (profiling captures only)")
+    ap.add_argument("--latency", action="store_true", help="latency vs batch size and co-located streams")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -493,6 +573,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.latency:
+            return run_latency(args, cfg, rank, world, local_rank)
         if cfg.training:
             return run_train(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
