@@ -75,6 +75,9 @@ _SIGS = {
                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_gemm_f32_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
+    "dlrm_gemm_f32": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
+                                C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
 }
 
 
@@ -227,6 +230,20 @@ def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, 
     return _check(lib().dlrm_forward_noalloc(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                              _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(err_flags),
                                              _stream(stream)), "dlrm_forward_noalloc")
+
+
+# ----------------------------------------------------------------- fp32 GEMM (tensor cores, 3xTF32)
+
+def dlrm_gemm_f32_workspace_size(I: int, J: int, R: int, a_mn: bool, b_mn: bool) -> int:
+    return int(lib().dlrm_gemm_f32_workspace_size(int(I), int(J), int(R), int(bool(a_mn)), int(bool(b_mn))))
+
+
+def dlrm_gemm_f32(I: int, J: int, R: int, A, lda: int, a_mn: bool, B, ldb: int, b_mn: bool, C, ldc: int, ws,
+                  stream=None):
+    """C[i][j] = sum_r A(i, r) B(j, r) in fp32 on the tensor cores; A(i, r) = A[i][r], or A[r][i] when a_mn
+    (B likewise)."""
+    return _check(lib().dlrm_gemm_f32(int(I), int(J), int(R), _ptr(A), int(lda), int(bool(a_mn)), _ptr(B), int(ldb),
+                                      int(bool(b_mn)), _ptr(C), int(ldc), _ptr(ws), _stream(stream)), "dlrm_gemm_f32")
 
 
 # ----------------------------------------------------------------- training step (fp32)

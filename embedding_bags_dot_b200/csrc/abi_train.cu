@@ -16,8 +16,20 @@ namespace {
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline cudaStream_t cs(dlrm_stream s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Workspace of the training step. Every tensor that a GEMM reads is kept as a
+// 3xTF32 (hi, lo) pair (F32Pair); x_dense, the concat vector, the logit and the
+// gradients that feed the interaction backward are also (or only) plain fp32.
 struct TrainWs {
-    size_t bact[DLRM_MAX_LAYERS], E, concat, tact[DLRM_MAX_LAYERS], g0, g1, wscratch, lpart, total;
+    size_t bW[DLRM_MAX_LAYERS][2], tW[DLRM_MAX_LAYERS][2];   // weight pairs, ld ldf(in)
+    size_t bact[DLRM_MAX_LAYERS][2];                         // bottom outputs (pairs), ld ldb
+    size_t xd;                                               // x_dense plain [B][d]
+    size_t E;                                                // pooled [B][K][d]
+    size_t concat, concat_p[2];                              // [B][ldc] plain and pair
+    size_t tact[DLRM_MAX_LAYERS][2];                         // top hidden outputs (pairs), ld ldt
+    size_t z, dz;                                            // logit and dL/dz [B]
+    size_t g[2][2];                                          // gradient ping-pong pairs [B][gmax]
+    size_t dcat, dxd;                                        // plain d(concat) [B][ldc], d(x_dense pre-act) [B][d]
+    size_t wscratch, lpart, total;
     int ldb[DLRM_MAX_LAYERS], ldt[DLRM_MAX_LAYERS], ldc, gmax;
 };
 
@@ -38,29 +50,39 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
         return o;
     };
     const int K = T->K, d = T->d;
+    const int nb = bot->n_layers, nt = top->n_layers;
+    for (int l = 0; l < nb; ++l)
+        for (int h = 0; h < 2; ++h) W.bW[l][h] = take(sizeof(float) * (size_t)bot->dims[l + 1] * ldf(bot->dims[l]));
+    for (int l = 0; l < nt; ++l)
+        for (int h = 0; h < 2; ++h) W.tW[l][h] = take(sizeof(float) * (size_t)top->dims[l + 1] * ldf(top->dims[l]));
     int gmax = 0;
-    for (int l = 0; l < bot->n_layers; ++l) {
+    for (int l = 0; l < nb; ++l) {
         W.ldb[l] = ldf(bot->dims[l + 1]);
-        W.bact[l] = take(sizeof(float) * (size_t)B * W.ldb[l]);
+        for (int h = 0; h < 2; ++h) W.bact[l][h] = take(sizeof(float) * (size_t)B * W.ldb[l]);
         gmax = std::max(gmax, W.ldb[l]);
     }
+    W.xd = take(sizeof(float) * (size_t)B * d);
     W.E = take(sizeof(float) * (size_t)B * K * d);
     W.ldc = ldf(d + K * (K + 1) / 2);
     W.concat = take(sizeof(float) * (size_t)B * W.ldc);
-    gmax = std::max(gmax, W.ldc);
-    for (int l = 0; l < top->n_layers; ++l) {
-        // the logit (last layer, one column) is stored densely: BCE reads z[B]
-        W.ldt[l] = (l == top->n_layers - 1 && top->dims[l + 1] == 1) ? 1 : ldf(top->dims[l + 1]);
-        W.tact[l] = take(sizeof(float) * (size_t)B * W.ldt[l]);
+    for (int h = 0; h < 2; ++h) W.concat_p[h] = take(sizeof(float) * (size_t)B * W.ldc);
+    for (int l = 0; l < nt - 1; ++l) {
+        W.ldt[l] = ldf(top->dims[l + 1]);
+        for (int h = 0; h < 2; ++h) W.tact[l][h] = take(sizeof(float) * (size_t)B * W.ldt[l]);
         gmax = std::max(gmax, W.ldt[l]);
     }
+    W.ldt[nt - 1] = 1;   // the logit is stored densely: BCE reads z[B]
+    W.z = take(sizeof(float) * (size_t)B);
+    W.dz = take(sizeof(float) * (size_t)B);
     W.gmax = gmax;
-    W.g0 = take(sizeof(float) * (size_t)B * gmax);
-    W.g1 = take(sizeof(float) * (size_t)B * gmax);
+    for (int p = 0; p < 2; ++p)
+        for (int h = 0; h < 2; ++h) W.g[p][h] = take(sizeof(float) * (size_t)B * gmax);
+    W.dcat = take(sizeof(float) * (size_t)B * W.ldc);
+    W.dxd = take(sizeof(float) * (size_t)B * d);
     size_t ws = 0;
-    for (int l = 0; l < bot->n_layers; ++l)
+    for (int l = 0; l < nb; ++l)
         ws = std::max(ws, train_wgrad_scratch_floats(bot->dims[l + 1], bot->dims[l], B));
-    for (int l = 0; l < top->n_layers; ++l)
+    for (int l = 0; l < nt; ++l)
         ws = std::max(ws, train_wgrad_scratch_floats(top->dims[l + 1], top->dims[l], B));
     W.wscratch = take(sizeof(float) * ws);
     W.lpart = take(sizeof(float) * ((size_t)(B + 255) / 256 + 1));
@@ -190,74 +212,89 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
 
     // dW padding columns stay zero so that SGD leaves the weights' padding untouched
     if (cudaMemsetAsync(g, 0, G.dE, st) != cudaSuccess) return DLRM_ERR_CUDA;
+    auto P = [&](const size_t (&o)[2], int ld) { return F32Pair{F(o[0]), F(o[1]), ld}; };
+
+    // ---- weights as (hi, lo) pairs (they change with every SGD step)
+    for (int l = 0; l < nb; ++l)
+        if ((r = launch_split_pair(bot->dims[l + 1], bot->dims[l], static_cast<const float*>(bot->W[l]),
+                                   ldf(bot->dims[l]), F(W.bW[l][0]), F(W.bW[l][1]), ldf(bot->dims[l]), st)))
+            return r;
+    for (int l = 0; l < nt; ++l)
+        if ((r = launch_split_pair(top->dims[l + 1], top->dims[l], static_cast<const float*>(top->W[l]),
+                                   ldf(top->dims[l]), F(W.tW[l][0]), F(W.tW[l][1]), ldf(top->dims[l]), st)))
+            return r;
 
     // ---- forward, keeping every activation
+    const F32Pair dense_in{dense, nullptr, bot->dims[0]};
     for (int l = 0; l < nb; ++l) {
-        const float* in = l == 0 ? dense : F(W.bact[l - 1]);
-        const int ldin = l == 0 ? bot->dims[0] : W.ldb[l - 1];
-        if ((r = train_linear_fwd(B, bot->dims[l + 1], bot->dims[l], in, ldin, static_cast<const float*>(bot->W[l]),
-                                  ldf(bot->dims[l]), bot->b[l], F(W.bact[l]), W.ldb[l], true, st)))
+        const F32Pair in = l == 0 ? dense_in : P(W.bact[l - 1], W.ldb[l - 1]);
+        if ((r = train_linear_fwd(B, bot->dims[l + 1], bot->dims[l], in, P(W.bW[l], ldf(bot->dims[l])), bot->b[l],
+                                  F(W.bact[l][0]), F(W.bact[l][1]), W.ldb[l], true, err, st)))
             return r;
     }
-    const float* x_dense = F(W.bact[nb - 1]);   // ld = ldf(d) = d (d % 4 == 0 on this path)
+    const F32Pair xd_pair = P(W.bact[nb - 1], W.ldb[nb - 1]);   // ld = d (d % 4 == 0 on this path)
+    const float* x_dense = F(W.xd);
+    if ((r = launch_merge_pair(B, d, xd_pair.hi, xd_pair.lo, xd_pair.ld, F(W.xd), d, st))) return r;
     if ((r = launch_embbag(tm, T->data, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err, st))) return r;
     if ((r = launch_interact(B, K, d, x_dense, F(W.E), F(W.concat), W.ldc, DLRM_F32, st))) return r;
+    const int cw = top->dims[0];
+    if ((r = launch_split_pair(B, cw, F(W.concat), W.ldc, F(W.concat_p[0]), F(W.concat_p[1]), W.ldc, st))) return r;
+    const F32Pair concat_p = P(W.concat_p, W.ldc);
     for (int l = 0; l < nt; ++l) {
-        const float* in = l == 0 ? F(W.concat) : F(W.tact[l - 1]);
-        const int ldin = l == 0 ? W.ldc : W.ldt[l - 1];
-        if ((r = train_linear_fwd(B, top->dims[l + 1], top->dims[l], in, ldin, static_cast<const float*>(top->W[l]),
-                                  ldf(top->dims[l]), top->b[l], F(W.tact[l]), W.ldt[l], l < nt - 1, st)))
+        const F32Pair in = l == 0 ? concat_p : P(W.tact[l - 1], W.ldt[l - 1]);
+        const bool last = l == nt - 1;
+        if ((r = train_linear_fwd(B, top->dims[l + 1], top->dims[l], in, P(W.tW[l], ldf(top->dims[l])), top->b[l],
+                                  last ? F(W.z) : F(W.tact[l][0]), last ? nullptr : F(W.tact[l][1]), W.ldt[l], !last,
+                                  err, st)))
             return r;
     }
 
     // ---- loss and dL/dz
-    float* dz = F(W.g0);
-    const float* z = F(W.tact[nt - 1]);
-    if ((r = launch_bce(B, z, labels, dz, y_hat, F(W.lpart), GF(G.loss), st))) return r;
+    float* dz = F(W.dz);
+    if ((r = launch_bce(B, F(W.z), labels, dz, y_hat, F(W.lpart), GF(G.loss), st))) return r;
     if (loss && cudaMemcpyAsync(loss, GF(G.loss), sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return DLRM_ERR_CUDA;
 
-    // ---- top MLP backward: cur = dL/d(pre-activation of layer l), ld curld
-    float* cur = dz;
-    int curld = 1;
-    float* other = F(W.g1);
+    // ---- top MLP backward: cur = dL/d(pre-activation of layer l)
+    F32Pair cur{dz, nullptr, 1};
+    int pp = 0;   // next gradient pair buffer
     for (int l = nt - 1; l >= 0; --l) {
-        const float* in = l == 0 ? F(W.concat) : F(W.tact[l - 1]);
-        const int ldin = l == 0 ? W.ldc : W.ldt[l - 1];
+        const F32Pair in = l == 0 ? concat_p : P(W.tact[l - 1], W.ldt[l - 1]);
         const int N = top->dims[l + 1], Kin = top->dims[l];
-        if ((r = train_linear_wgrad(B, N, Kin, cur, curld, in, ldin, GF(G.tdW[l]), ldf(Kin), GF(G.tdb[l]),
-                                    F(W.wscratch), st)))
-            return r;
-        const int ldo = l == 0 ? W.ldc : W.ldt[l - 1];
-        if ((r = train_linear_dgrad(B, N, Kin, cur, curld, static_cast<const float*>(top->W[l]), ldf(Kin),
-                                    l == 0 ? nullptr : F(W.tact[l - 1]), ldo, other, ldo, st)))
-            return r;
-        float* t = cur;
-        cur = other;
-        other = t;
-        curld = ldo;
-    }
-    // cur = d(concat) [B][ldc]
-    float* dxd = other;   // gradient of the last bottom layer's pre-activation [B][d]
-    if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), cur, W.ldc, dxd, GF(G.dE), st))) return r;
-    cur = dxd;
-    curld = d;
-    other = (cur == F(W.g0)) ? F(W.g1) : F(W.g0);
-    for (int l = nb - 1; l >= 0; --l) {
-        const float* in = l == 0 ? dense : F(W.bact[l - 1]);
-        const int ldin = l == 0 ? bot->dims[0] : W.ldb[l - 1];
-        const int N = bot->dims[l + 1], Kin = bot->dims[l];
-        if ((r = train_linear_wgrad(B, N, Kin, cur, curld, in, ldin, GF(G.bdW[l]), ldf(Kin), GF(G.bdb[l]),
-                                    F(W.wscratch), st)))
+        const F32Pair Wp = P(W.tW[l], ldf(Kin));
+        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.tdW[l]), ldf(Kin), GF(G.tdb[l]), F(W.wscratch), err,
+                                    st)))
             return r;
         if (l > 0) {
-            if ((r = train_linear_dgrad(B, N, Kin, cur, curld, static_cast<const float*>(bot->W[l]), ldf(Kin),
-                                        F(W.bact[l - 1]), W.ldb[l - 1], other, W.ldb[l - 1], st)))
+            const int ldo = W.gmax;
+            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, in, F(W.g[pp][0]), F(W.g[pp][1]), ldo, err, st)))
                 return r;
-            float* t = cur;
-            cur = other;
-            other = t;
-            curld = W.ldb[l - 1];
+            cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), ldo};
+            pp ^= 1;
+        } else {
+            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, F32Pair{nullptr, nullptr, 0}, F(W.dcat), nullptr, W.ldc,
+                                        err, st)))
+                return r;
+        }
+    }
+    // d(concat) -> gradient of the last bottom layer's pre-activation (ReLU mask applied) and dE
+    if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;
+    if ((r = launch_split_pair(B, d, F(W.dxd), d, F(W.g[pp][0]), F(W.g[pp][1]), d, st))) return r;
+    cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), d};
+    pp ^= 1;
+    for (int l = nb - 1; l >= 0; --l) {
+        const F32Pair in = l == 0 ? dense_in : P(W.bact[l - 1], W.ldb[l - 1]);
+        const int N = bot->dims[l + 1], Kin = bot->dims[l];
+        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.bdW[l]), ldf(Kin), GF(G.bdb[l]), F(W.wscratch), err,
+                                    st)))
+            return r;
+        if (l > 0) {
+            const int ldo = W.gmax;
+            if ((r = train_linear_dgrad(B, N, Kin, cur, P(W.bW[l], ldf(Kin)), in, F(W.g[pp][0]), F(W.g[pp][1]), ldo,
+                                        err, st)))
+                return r;
+            cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), ldo};
+            pp ^= 1;
         }
     }
 

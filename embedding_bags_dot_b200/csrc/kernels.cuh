@@ -48,14 +48,48 @@ dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt
                              cudaStream_t st);
 
 // ---- training (fp32)
-dlrm_status train_linear_fwd(int M, int N, int K, const float* x, int ldx, const float* W, int ldw, const float* b,
-                             float* y, int ldy, bool relu, cudaStream_t st);
-dlrm_status train_linear_dgrad(int M, int N, int K, const float* dy, int lddy, const float* W, int ldw,
-                               const float* relu_of, int ldr, float* dx, int lddx, cudaStream_t st);
-int train_wgrad_splits(int N, int K, int M);
+// An fp32 matrix row-major with leading dimension ld, held either plain
+// (lo == nullptr, value = hi) or as a 3xTF32 pair: hi = value with its 13 low
+// mantissa bits cleared, lo = value - hi (value = hi + lo exactly).
+struct F32Pair {
+    const float* hi;
+    const float* lo;
+    int ld;
+};
+
+// Tensor-core 3xTF32 GEMMs (gemm_tf32.cu); operands must be pairs.
+bool tf32x3_supported(int M, int N, int K, F32Pair a, F32Pair b);
+dlrm_status tf32x3_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* bias, float* y_hi, float* y_lo,
+                       int ldy, ErrRecord* err, cudaStream_t st);
+dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mask, float* dx_hi, float* dx_lo,
+                         int lddx, ErrRecord* err, cudaStream_t st);
+int tf32x3_wgrad_splits(int N, int K, int M);
+size_t tf32x3_wgrad_scratch_floats(int N, int K, int M);
+dlrm_status tf32x3_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* scratch,
+                         ErrRecord* err, cudaStream_t st);
+// C[i][j] = sum_r A(i, r) B(j, r); A(i, r) = A[i][r] (K-major) or A[r][i] (a_mn), likewise B
+dlrm_status tf32x3_gemm(int I, int J, int R, F32Pair A, bool a_mn, F32Pair B, bool b_mn, float* C, int ldc,
+                        float* scratch, ErrRecord* err, cudaStream_t st);
+
+// CUDA-core fp32 GEMMs and helpers (train_gemm.cu). Inputs may be plain or
+// pairs; y_lo / dx_lo non-null selects a pair output.
+dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b, float* y, float* y_lo,
+                             int ldy, bool relu, ErrRecord* err, cudaStream_t st);
+// dx[m][k] = sum_n dy[m][n] W[n][k], zeroed where relu_of (post-ReLU value) <= 0 when relu_of.hi is given
+dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of, float* dx, float* dx_lo,
+                               int lddx, ErrRecord* err, cudaStream_t st);
 size_t train_wgrad_scratch_floats(int N, int K, int M);
-dlrm_status train_linear_wgrad(int M, int N, int K, const float* dy, int lddy, const float* x, int ldx, float* dW,
-                               int ldw, float* db, float* scratch, cudaStream_t st);
+// dW[n][k] = sum_m dy[m][n] x[m][k]; db[n] = sum_m dy[m][n]
+dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* db,
+                               float* scratch, ErrRecord* err, cudaStream_t st);
+// hi/lo pair of a plain [rows][cols] matrix
+dlrm_status launch_split_pair(int rows, int cols, const float* src, int lds, float* hi, float* lo, int ldd,
+                              cudaStream_t st);
+// plain[r][c] = hi[r][c] + lo[r][c]
+dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* lo, int lds, float* out, int ldo,
+                              cudaStream_t st);
+// out[n][k] = sum_{z < S} part[z][n][k] in increasing z (part split stride N * ldp)
+dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st);
 
 dlrm_status launch_bce(int B, const float* z, const float* y, float* dz, float* y_hat, float* partial, float* loss,
                        cudaStream_t st);

@@ -1,8 +1,13 @@
 // fp32 GEMMs of the training step (forward with saved activations, data
-// gradient, weight gradient). The training workload keeps every tensor in
-// fp32, so these run on the CUDA cores with fp32 accumulation.
+// gradient, weight gradient): dispatch between the tensor-core 3xTF32 kernel
+// (gemm_tf32.cu) and a CUDA-core fp32 kernel for the shapes it does not take
+// (the 13-wide first bottom layer, the one-column logit layer), plus the
+// pair-split, split-sum and bias-gradient helpers.
 //
-// One kernel covers the three operand layouts:
+// Operands are F32Pair: plain fp32, or a 3xTF32 (hi, lo) pair whose value is
+// hi + lo exactly; the CUDA-core kernel reads either and writes either.
+//
+// The CUDA-core kernel covers the three operand layouts:
 //   C(i, j) = sum_r A(i, r) B(j, r)
 //   A(i, r) = A[i*lda + r]  (AT = false)   or  A[r*lda + i]  (AT = true)
 //   B(j, r) = B[j*ldb + r]  (BT = false)   or  B[r*ldb + j]  (BT = true)
@@ -24,9 +29,10 @@ constexpr int TM = 64, TN = 64, TK = 16;
 enum Epi { EPI_BIAS = 0, EPI_BIAS_RELU = 1, EPI_MASK = 2, EPI_PLAIN = 3, EPI_PARTIAL = 4 };
 
 template <bool T>
-__device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* __restrict__ X, long long ld, long long i0,
-                                          long long r0, long long ni, long long nr, bool ones_col) {
-    // S[r][i] = X(i0 + i, r0 + r), zero outside, 1 for the synthesized column i == ni when ones_col
+__device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* __restrict__ X,
+                                          const float* __restrict__ Xlo, long long ld, long long i0, long long r0,
+                                          long long ni, long long nr, bool ones_col) {
+    // S[r][i] = X(i0 + i, r0 + r) (+ its lo part), zero outside, 1 for the synthesized column i == ni when ones_col
     if constexpr (!T) {
         const int i = threadIdx.x >> 2, r = (threadIdx.x & 3) * 4;
 #pragma unroll
@@ -34,7 +40,7 @@ __device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* _
             const long long gi = i0 + i, gr = r0 + r + e;
             float v = 0.f;
             if (gr < nr) {
-                if (gi < ni) v = X[gi * ld + gr];
+                if (gi < ni) v = Xlo ? X[gi * ld + gr] + Xlo[gi * ld + gr] : X[gi * ld + gr];
                 else if (ones_col && gi == ni) v = 1.f;
             }
             S[r + e][i] = v;
@@ -46,7 +52,7 @@ __device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* _
             const long long gi = i0 + i + e, gr = r0 + r;
             float v = 0.f;
             if (gr < nr) {
-                if (gi < ni) v = X[gr * ld + gi];
+                if (gi < ni) v = Xlo ? X[gr * ld + gi] + Xlo[gr * ld + gi] : X[gr * ld + gi];
                 else if (ones_col && gi == ni) v = 1.f;
             }
             S[r][i + e] = v;
@@ -54,14 +60,19 @@ __device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* _
     }
 }
 
+__device__ __forceinline__ float tf32_hi_part(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+
 // Output tile (i0.., j0..) of C(i, j), reduction over r in [r_begin, r_end).
 // B_ONES: B has a synthesized extra column j == NB of ones (weight-gradient bias term).
+// C_lo non-null: the output is written as a (hi, lo) pair.
 template <bool AT, bool BT, int EPI, bool B_ONES>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(long long NI, long long NJ, long long NR, const float* __restrict__ A,
-                                                       long long lda, const float* __restrict__ Bm, long long ldb,
-                                                       const float* __restrict__ bias, const float* __restrict__ mask,
-                                                       long long ldm, float* __restrict__ C, long long ldc,
-                                                       long long r_chunk, long long part_stride) {
+                                                       const float* __restrict__ A_lo, long long lda,
+                                                       const float* __restrict__ Bm, const float* __restrict__ B_lo,
+                                                       long long ldb, const float* __restrict__ bias,
+                                                       const float* __restrict__ mask, const float* __restrict__ mask_lo,
+                                                       long long ldm, float* __restrict__ C, float* __restrict__ C_lo,
+                                                       long long ldc, long long r_chunk, long long part_stride) {
     __shared__ float As[TK][TN + 4];
     __shared__ float Bs[TK][TN + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -75,8 +86,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(long long NI, long long N
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
     for (long long r0 = rb; r0 < re; r0 += TK) {
-        load_tile<AT>(As, A, lda, i0, r0, NI, re, false);
-        load_tile<BT>(Bs, Bm, ldb, j0, r0, NJ, re, B_ONES);
+        load_tile<AT>(As, A, A_lo, lda, i0, r0, NI, re, false);
+        load_tile<BT>(Bs, Bm, B_lo, ldb, j0, r0, NJ, re, B_ONES);
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < TK; ++kk) {
@@ -101,11 +112,19 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(long long NI, long long N
             float v = acc[x][y];
             if constexpr (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) v += bias[j];
             if constexpr (EPI == EPI_BIAS_RELU) v = v > 0.f ? v : 0.f;
-            if constexpr (EPI == EPI_MASK) v = (mask[i * ldm + j] > 0.f) ? v : 0.f;
-            if constexpr (EPI == EPI_PARTIAL)
+            if constexpr (EPI == EPI_MASK) {
+                const float m = mask_lo ? mask[i * ldm + j] + mask_lo[i * ldm + j] : mask[i * ldm + j];
+                v = (m > 0.f) ? v : 0.f;
+            }
+            if constexpr (EPI == EPI_PARTIAL) {
                 C[(long long)blockIdx.z * part_stride + i * (NJ + 1) + j] = v;
-            else
+            } else if (C_lo) {
+                const float h = tf32_hi_part(v);
+                C[i * ldc + j] = h;
+                C_lo[i * ldc + j] = v - h;
+            } else {
                 C[i * ldc + j] = v;
+            }
         }
     }
 }
@@ -123,45 +142,94 @@ __global__ void wgrad_reduce_kernel(int splits, long long NI, long long NJ, cons
     }
 }
 
+__global__ void split_pair_kernel(long long rows, int cols, const float* __restrict__ src, long long lds,
+                                  float* __restrict__ hi, float* __restrict__ lo, long long ldd) {
+    const long long n = rows * cols;
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+        const long long r = q / cols, c = q - r * cols;
+        const float v = src[r * lds + c];
+        const float h = tf32_hi_part(v);
+        hi[r * ldd + c] = h;
+        lo[r * ldd + c] = v - h;
+    }
+}
+
+__global__ void split_pair_vec_kernel(long long rows, int cols4, const float4* __restrict__ src, long long lds4,
+                                      float4* __restrict__ hi, float4* __restrict__ lo, long long ldd4) {
+    const long long n = rows * cols4;
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+        const long long r = q / cols4, c = q - r * cols4;
+        const float4 v = src[r * lds4 + c];
+        const float4 h = make_float4(tf32_hi_part(v.x), tf32_hi_part(v.y), tf32_hi_part(v.z), tf32_hi_part(v.w));
+        hi[r * ldd4 + c] = h;
+        lo[r * ldd4 + c] = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+    }
+}
+
+__global__ void merge_pair_kernel(long long rows, int cols, const float* __restrict__ hi,
+                                  const float* __restrict__ lo, long long lds, float* __restrict__ out, long long ldo) {
+    const long long n = rows * cols;
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+        const long long r = q / cols, c = q - r * cols;
+        out[r * ldo + c] = hi[r * lds + c] + lo[r * lds + c];
+    }
+}
+
+__global__ void split_sum_kernel(int S, long long N, int K, const float* __restrict__ part, long long ldp,
+                                 float* __restrict__ out, long long ldo) {
+    const long long n = N * K;
+    const long long zs = N * ldp;
+    for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
+        const long long i = q / K, j = q - i * K;
+        float s = 0.f;
+        for (int z = 0; z < S; ++z) s += part[z * zs + i * ldp + j];
+        out[i * ldo + j] = s;
+    }
+}
+
+// Column sums of a [M][N] pair over fixed row chunks: part[p][c] = sum of rows
+// [p*rows_per, (p+1)*rows_per), eight row-interleaved partial sums combined in order.
+__global__ void __launch_bounds__(256) colsum_partial_kernel(long long M, int N, const float* __restrict__ hi,
+                                                             const float* __restrict__ lo, long long ld,
+                                                             long long rows_per, float* __restrict__ part) {
+    __shared__ float red[8][33];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + tx;
+    const long long rb = (long long)blockIdx.y * rows_per;
+    const long long re = rb + rows_per < M ? rb + rows_per : M;
+    float s = 0.f;
+    if (c < N)
+        for (long long r = rb + ty; r < re; r += 8) s += lo ? hi[r * ld + c] + lo[r * ld + c] : hi[r * ld + c];
+    red[ty][tx] = s;
+    __syncthreads();
+    if (ty == 0 && c < N) {
+        float t = 0.f;
+#pragma unroll
+        for (int y = 0; y < 8; ++y) t += red[y][tx];
+        part[(long long)blockIdx.y * N + c] = t;
+    }
+}
+
+__global__ void colsum_final_kernel(int P, int N, const float* __restrict__ part, float* __restrict__ out) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= N) return;
+    float s = 0.f;
+    for (int p = 0; p < P; ++p) s += part[(long long)p * N + c];
+    out[c] = s;
+}
+
+int colsum_chunks(int M) {
+    const int p = (M + 511) / 512;
+    return p < 1 ? 1 : (p > 128 ? 128 : p);
+}
+
 dim3 grid_for(long long NI, long long NJ, int z) {
     return dim3((unsigned)((NJ + TN - 1) / TN), (unsigned)((NI + TM - 1) / TM), (unsigned)z);
 }
 
-}  // namespace
+int grid_stride_blocks(long long n) { return (int)((n + 255) / 256 < 8192 ? (n + 255) / 256 : 8192); }
 
-dlrm_status train_linear_fwd(int M, int N, int K, const float* x, int ldx, const float* W, int ldw, const float* b,
-                             float* y, int ldy, bool relu, cudaStream_t st) {
-    if (M == 0) return DLRM_OK;
-    if (relu)
-        gemm_f32_kernel<false, false, EPI_BIAS_RELU, false><<<grid_for(M, N, 1), 256, 0, st>>>(
-            M, N, K, x, ldx, W, ldw, b, nullptr, 0, y, ldy, K, 0);
-    else
-        gemm_f32_kernel<false, false, EPI_BIAS, false><<<grid_for(M, N, 1), 256, 0, st>>>(
-            M, N, K, x, ldx, W, ldw, b, nullptr, 0, y, ldy, K, 0);
-    DLRM_LAUNCH_CHECK();
-    return DLRM_OK;
-}
-
-dlrm_status train_linear_dgrad(int M, int N, int K, const float* dy, int lddy, const float* W, int ldw,
-                               const float* relu_of, int ldr, float* dx, int lddx, cudaStream_t st) {
-    // dx[m][k] = sum_n dy[m][n] W[n][k], zeroed where relu_of[m][k] <= 0 (if given)
-    if (M == 0) return DLRM_OK;
-    if (relu_of)
-        gemm_f32_kernel<false, true, EPI_MASK, false><<<grid_for(M, K, 1), 256, 0, st>>>(
-            M, K, N, dy, lddy, W, ldw, nullptr, relu_of, ldr, dx, lddx, N, 0);
-    else
-        gemm_f32_kernel<false, true, EPI_PLAIN, false><<<grid_for(M, K, 1), 256, 0, st>>>(
-            M, K, N, dy, lddy, W, ldw, nullptr, nullptr, 0, dx, lddx, N, 0);
-    DLRM_LAUNCH_CHECK();
-    return DLRM_OK;
-}
-
-size_t train_wgrad_scratch_floats(int N, int K, int M) {
-    const int splits = train_wgrad_splits(N, K, M);
-    return (size_t)splits * (size_t)N * (size_t)(K + 1);
-}
-
-int train_wgrad_splits(int N, int K, int M) {
+int simt_wgrad_splits(int N, int K, int M) {
     // enough blocks to fill the GPU; fixed per shape so results do not depend on the device
     const long long tiles = ((N + TM - 1) / TM) * (long long)((K + 1 + TN - 1) / TN);
     long long s = (1184 + tiles - 1) / tiles;
@@ -172,19 +240,110 @@ int train_wgrad_splits(int N, int K, int M) {
     return (int)s;
 }
 
-dlrm_status train_linear_wgrad(int M, int N, int K, const float* dy, int lddy, const float* x, int ldx, float* dW,
-                               int ldw, float* db, float* scratch, cudaStream_t st) {
+bool is_pair(F32Pair p) { return p.lo != nullptr; }
+
+}  // namespace
+
+dlrm_status launch_split_pair(int rows, int cols, const float* src, int lds, float* hi, float* lo, int ldd,
+                              cudaStream_t st) {
+    if (rows <= 0 || cols <= 0) return DLRM_OK;
+    const bool vec = cols % 4 == 0 && lds % 4 == 0 && ldd % 4 == 0 && ((uintptr_t)src & 15) == 0 &&
+                     ((uintptr_t)hi & 15) == 0 && ((uintptr_t)lo & 15) == 0;
+    if (vec) {
+        const long long n = (long long)rows * (cols / 4);
+        split_pair_vec_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(
+            rows, cols / 4, reinterpret_cast<const float4*>(src), lds / 4, reinterpret_cast<float4*>(hi),
+            reinterpret_cast<float4*>(lo), ldd / 4);
+    } else {
+        split_pair_kernel<<<grid_stride_blocks((long long)rows * cols), 256, 0, st>>>(rows, cols, src, lds, hi, lo,
+                                                                                       ldd);
+    }
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* lo, int lds, float* out, int ldo,
+                              cudaStream_t st) {
+    const long long n = (long long)rows * cols;
+    if (n <= 0) return DLRM_OK;
+    merge_pair_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(rows, cols, hi, lo, lds, out, ldo);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st) {
+    const long long n = (long long)N * K;
+    if (n == 0) return DLRM_OK;
+    split_sum_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(S, N, K, part, ldp, out, ldo);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b, float* y, float* y_lo,
+                             int ldy, bool relu, ErrRecord* err, cudaStream_t st) {
+    if (M == 0) return DLRM_OK;
+    if (relu && y_lo && tf32x3_supported(M, N, K, x, W))
+        return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, err, st);
+    if (relu)
+        gemm_f32_kernel<false, false, EPI_BIAS_RELU, false><<<grid_for(M, N, 1), 256, 0, st>>>(
+            M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
+    else
+        gemm_f32_kernel<false, false, EPI_BIAS, false><<<grid_for(M, N, 1), 256, 0, st>>>(
+            M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of, float* dx, float* dx_lo,
+                               int lddx, ErrRecord* err, cudaStream_t st) {
+    if (M == 0) return DLRM_OK;
+    const bool shape_ok = relu_of.hi ? (dx_lo && is_pair(relu_of)) : !dx_lo;
+    if (shape_ok && tf32x3_supported(M, K, N, dy, W))
+        return tf32x3_dgrad(M, N, K, dy, W, relu_of, dx, dx_lo, lddx, err, st);
+    if (relu_of.hi)
+        gemm_f32_kernel<false, true, EPI_MASK, false><<<grid_for(M, K, 1), 256, 0, st>>>(
+            M, K, N, dy.hi, dy.lo, dy.ld, W.hi, W.lo, W.ld, nullptr, relu_of.hi, relu_of.lo, relu_of.ld, dx, dx_lo,
+            lddx, N, 0);
+    else
+        gemm_f32_kernel<false, true, EPI_PLAIN, false><<<grid_for(M, K, 1), 256, 0, st>>>(
+            M, K, N, dy.hi, dy.lo, dy.ld, W.hi, W.lo, W.ld, nullptr, nullptr, nullptr, 0, dx, dx_lo, lddx, N, 0);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+size_t train_wgrad_scratch_floats(int N, int K, int M) {
+    const size_t simt = (size_t)simt_wgrad_splits(N, K, M) * (size_t)N * (size_t)(K + 1);
+    const size_t tc = tf32x3_wgrad_scratch_floats(N, K, M);
+    const size_t cs = (size_t)colsum_chunks(M) * (size_t)N;
+    return simt > tc ? (simt > cs ? simt : cs) : (tc > cs ? tc : cs);
+}
+
+dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* db,
+                               float* scratch, ErrRecord* err, cudaStream_t st) {
     // dW[n][k] = sum_m dy[m][n] x[m][k]; db[n] = sum_m dy[m][n]
-    const int splits = train_wgrad_splits(N, K, M);
+    if (N >= 16 && tf32x3_supported(N, K, M, dy, x)) {
+        dlrm_status r = tf32x3_wgrad(M, N, K, dy, x, dW, ldw, scratch, err, st);
+        if (r) return r;
+        // bias gradient: fixed-order column sums of dy (the split partials above are consumed by now)
+        const int P = colsum_chunks(M);
+        const long long rows_per = ((long long)M + P - 1) / P;
+        colsum_partial_kernel<<<dim3((unsigned)((N + 31) / 32), (unsigned)P), 256, 0, st>>>(M, N, dy.hi, dy.lo, dy.ld,
+                                                                                           rows_per, scratch);
+        DLRM_LAUNCH_CHECK();
+        colsum_final_kernel<<<(N + 255) / 256, 256, 0, st>>>(P, N, scratch, db);
+        DLRM_LAUNCH_CHECK();
+        return DLRM_OK;
+    }
+    const int splits = simt_wgrad_splits(N, K, M);
     long long chunk = ((long long)M + splits - 1) / splits;
     chunk = (chunk + TK - 1) / TK * TK;
     const long long pstride = (long long)N * (K + 1);
     gemm_f32_kernel<true, true, EPI_PARTIAL, true><<<grid_for(N, K + 1, splits), 256, 0, st>>>(
-        N, K, M, dy, lddy, x, ldx, nullptr, nullptr, 0, scratch, 0, chunk, pstride);
+        N, K, M, dy.hi, dy.lo, dy.ld, x.hi, x.lo, x.ld, nullptr, nullptr, nullptr, 0, scratch, nullptr, 0, chunk,
+        pstride);
     DLRM_LAUNCH_CHECK();
     const long long n = pstride;
-    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    wgrad_reduce_kernel<<<blocks, 256, 0, st>>>(splits, N, K, scratch, pstride, dW, ldw, db);
+    wgrad_reduce_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(splits, N, K, scratch, pstride, dW, ldw, db);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }

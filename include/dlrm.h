@@ -191,6 +191,27 @@ dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, 
                                      int64_t nnz, void* grads, uint32_t* rows, float* row_grads,
                                      int32_t* n_rows, dlrm_stream stream);
 
+/* fp32 GEMM of the training step, on the tensor cores at fp32 accuracy
+ * (the matrix products of the fully connected layers, "Deep Learning
+ * Recommendation Model (DLRM)", Key Method Details: bottom and top MLPs, and
+ * their gradients by the chain rule):
+ *   C[i][j] = sum_{r < R} A(i, r) B(j, r)        i < I, j < J
+ * A(i, r) = A[i*lda + r] (a_mn = 0) or A[r*lda + i] (a_mn = 1); B likewise
+ * with b_mn. All pointers are device fp32, 16-byte aligned; lda, ldb, ldc
+ * are multiples of 4 (ldc >= J). Each operand is split in `ws` into a TF32
+ * pair (hi = value with its 13 low mantissa bits cleared, lo = value - hi)
+ * and the product is summed as A_lo B_hi + A_hi B_lo + A_hi B_hi in fp32
+ * (error about 2^-20 of sum_r |A(i,r) B(j,r)|). Long reductions are cut into
+ * shape-determined r-ranges added in a fixed order: bit-reproducible.
+ * ws: 16-byte aligned, dlrm_gemm_f32_workspace_size(...) bytes, caller-owned.
+ * Returns DLRM_ERR_INVALID_ARG (sizes < 1, null, misaligned, ld),
+ * DLRM_ERR_WORKSPACE (ws null or misaligned), DLRM_ERR_UNSUPPORTED (no
+ * tensor-map support in the driver); device timeouts land in the error
+ * record read by dlrm_check_error. */
+size_t dlrm_gemm_f32_workspace_size(int I, int J, int R, int a_mn, int b_mn);
+dlrm_status dlrm_gemm_f32(int I, int J, int R, const float* A, int lda, int a_mn, const float* B, int ldb, int b_mn,
+                          float* C, int ldc, void* ws, dlrm_stream stream);
+
 /* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
 #define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
 
