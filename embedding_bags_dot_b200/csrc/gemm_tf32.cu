@@ -1,12 +1,18 @@
 // fp32 GEMMs of the training step on the tensor cores, 3xTF32:
 //   C(i, j) = sum_r A(i, r) B(j, r)
-// every fp32 operand x is held as a pair (hi, lo): hi = x with its 13 low
-// mantissa bits cleared (exactly a TF32 number), lo = x - hi (exact in fp32,
-// rounded to TF32 by the tensor core). The product is accumulated in fp32 as
+// every fp32 operand x is held as a pair (hi, lo): hi = x rounded to the
+// nearest TF32 number, lo = x - hi (exact in fp32, at most 12 significant
+// bits, taken to TF32 by the tensor core). Each product is formed as
 //   A_lo B_hi + A_hi B_lo + A_hi B_hi
-// (the dropped A_lo B_lo term and the TF32 rounding of lo are ~2^-21 of
-// |A||B| per product), so the result carries fp32-level error on a tensor
-// pipe that runs TF32 at half the bf16 rate.
+// (the dropped A_lo B_lo term and the TF32 rounding of lo are ~2^-23 of
+// |A||B|), on a tensor pipe that runs TF32 at half the bf16 rate.
+//
+// The tensor core's fp32 accumulation truncates at every MMA, which biases
+// long sums (measured: ~1e-5 of sum |terms| after 1024 same-sign terms). So no
+// accumulator lives longer than one 32-deep k-block: each block's partial
+// product is taken out of TMEM by the epilogue warps and added into fp32
+// registers with round-to-nearest, while the next block accumulates in the
+// other TMEM buffer.
 //
 // The three GEMMs of a fully connected layer ("Deep Learning Recommendation
 // Model (DLRM)", Key Method Details: FC layers; their gradients by the chain
@@ -24,10 +30,11 @@
 // tcgen05.mma.cta_group::2.kind::tf32 (M = 256, N = 256, K = 8); each CTA
 // stages its 128 rows of A and its 128 rows of B, hi and lo (64 KB per
 // 32-deep k-block, three stages), by TMA with 128-byte swizzle (32-byte
-// atoms for MN-major operands); the leader
-// issues 12 MMAs per k-block; 8 epilogue warps per CTA drain the
-// double-buffered TMEM accumulator, apply bias/ReLU or the ReLU mask, split
-// the result into its (hi, lo) pair and write it by TMA bulk tensor stores.
+// atoms for MN-major operands); the leader issues 12 MMAs per k-block into
+// one of two TMEM buffers; 8 epilogue warps per CTA add each finished block
+// into registers (128 fp32 per thread: 32 rows x 128 columns per warp), then
+// apply bias/ReLU or the ReLU mask, split the result into its (hi, lo) pair
+// and write it by TMA bulk tensor stores.
 // Every wait is bounded (timeout -> DLRM_ERR_TIMEOUT in the error record,
 // copies and MMAs drained, TMEM freed). No cluster-multicast load is used.
 #include <cuda.h>
@@ -46,6 +53,14 @@ constexpr int STAGE3_BYTES = 4 * PART3;       // A_hi, A_lo, B_hi, B_lo
 constexpr int SMEM3_BYTES = STAGES3 * STAGE3_BYTES + OUT_BYTES + 1024 + 256;
 static_assert(SMEM3_BYTES <= 227 * 1024, "shared memory");
 constexpr int PAIRS_REF = 74;                 // SM pairs assumed when choosing the split count (shape-only)
+// 12 warps: warpgroup 0 = TMA producer (warp 0), MMA issuer and TMEM owner
+// (warp 1), two idle warps; warpgroups 1 and 2 = 8 epilogue warps. The block
+// launches with 168 registers per thread (64,512 in all); warpgroup 0 gives
+// back to 40 and the epilogue warpgroups take 232 each:
+// 128 * 40 + 256 * 232 = 64,512.
+constexpr int THREADS3 = 384;
+constexpr int REGS_LOW = 40, REGS_HIGH = 232;
+static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= 168 * THREADS3, "register split exceeds the launch allocation");
 
 enum Epi3 { E3_RELU_PAIR = 0, E3_MASK_PAIR = 1, E3_PLAIN = 2 };
 
@@ -117,7 +132,15 @@ __device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* hi
     }
 }
 
-__device__ __forceinline__ float tf32_hi(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+// hi part of a 3xTF32 pair: v rounded to the nearest TF32 value (ties away
+// from zero), so that lo = v - hi is exact and has at most 12 significant bits;
+// magnitudes that would round up to infinity are truncated instead.
+__device__ __forceinline__ float tf32_hi(float v) {
+    const uint32_t u = __float_as_uint(v);
+    uint32_t r = u + 0x1000u;
+    if ((r & 0x7F800000u) == 0x7F800000u) r = u;
+    return __uint_as_float(r & 0xFFFFE000u);
+}
 
 // Stage one 32-row x 32-column fp32 chunk (128-byte swizzle) and store it.
 __device__ __forceinline__ void stage_store(const float (&v)[32], unsigned char* stage, uint32_t stage_s,
@@ -136,24 +159,20 @@ __device__ __forceinline__ void stage_store(const float (&v)[32], unsigned char*
     if (lane == 0) tma_store_3d(map, stage_s, x, y, z);
 }
 
-// Epilogue of one warp: rows i0 .. i0 + 31 (one per lane), columns jb .. jb + 127.
+// Final epilogue of one warp from its fp32 register accumulator: rows i0 ..
+// i0 + 31 (one per lane), columns jb .. jb + 127 (acc[c][e] = column jb + 32c + e).
 template <int EPI>
-__device__ __forceinline__ void epilogue3(uint32_t taddr, int i0, int jb, int I, int J, int z,
+__device__ __forceinline__ void epilogue3(float (&acc)[4][32], int i0, int jb, int I, int J, int z,
                                           const float* __restrict__ bias, const float* __restrict__ mhi,
                                           const float* __restrict__ mlo, long long ldm, const CUtensorMap* c0,
                                           const CUtensorMap* c1, unsigned char* stage, uint32_t stage_s) {
     const int lane = threadIdx.x & 31;
     const int i = i0 + lane;
-#pragma unroll 1
+#pragma unroll
     for (int c = 0; c < 4; ++c) {
         const int j0 = jb + 32 * c;
         if (j0 >= J) break;   // uniform across the warp
-        uint32_t r[32];
-        tmem_ld32_issue(taddr + 32 * c, r);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+        float (&v)[32] = acc[c];
         if constexpr (EPI == E3_RELU_PAIR) {
             if (j0 + 32 <= J) {
                 const float4* b4 = reinterpret_cast<const float4*>(bias + j0);
@@ -181,12 +200,12 @@ __device__ __forceinline__ void epilogue3(uint32_t taddr, int i0, int jb, int I,
                 if (j0 + 32 <= J) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 a = __ldg(reinterpret_cast<const float4*>(h) + q);
-                        const float4 b = __ldg(reinterpret_cast<const float4*>(l) + q);
-                        if (!(a.x + b.x > 0.f)) v[4 * q + 0] = 0.f;
-                        if (!(a.y + b.y > 0.f)) v[4 * q + 1] = 0.f;
-                        if (!(a.z + b.z > 0.f)) v[4 * q + 2] = 0.f;
-                        if (!(a.w + b.w > 0.f)) v[4 * q + 3] = 0.f;
+                        const float4 x = __ldg(reinterpret_cast<const float4*>(h) + q);
+                        const float4 y = __ldg(reinterpret_cast<const float4*>(l) + q);
+                        if (!(x.x + y.x > 0.f)) v[4 * q + 0] = 0.f;
+                        if (!(x.y + y.y > 0.f)) v[4 * q + 1] = 0.f;
+                        if (!(x.z + y.z > 0.f)) v[4 * q + 2] = 0.f;
+                        if (!(x.w + y.w > 0.f)) v[4 * q + 3] = 0.f;
                     }
                 } else {
 #pragma unroll
@@ -209,8 +228,20 @@ __device__ __forceinline__ void epilogue3(uint32_t taddr, int i0, int jb, int I,
     }
 }
 
+// acc[c] += the 32 TMEM columns at taddr + 32c, c = 0..3
+__device__ __forceinline__ void promote(float (&acc)[4][32], uint32_t taddr) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32_issue(taddr + 32 * c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[c][e] += __uint_as_float(r[e]);
+    }
+}
+
 template <bool AMN, bool BMN, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS3, 1)
     gemm3x_kernel(const __grid_constant__ Maps3 maps, int I, int J, int R, int r_chunk, int S,
                   const float* __restrict__ bias, const float* __restrict__ mhi, const float* __restrict__ mlo,
                   long long ldm, ErrRecord* err) {
@@ -260,6 +291,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int re = rb + r_chunk < R ? rb + r_chunk : R;
         nk = (re - rb + BR3 - 1) / BR3;
     };
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_LOW));
     if (warp == 0) {
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.a_hi)) : "memory");
@@ -300,24 +333,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0 && leader) {
             int s = 0;
             uint32_t ph = 0;
-            int it = 0;
-            for (int t = pair; t < ntiles && !timed_out; t += npair, ++it) {
+            uint32_t blk = 0;   // k-blocks issued so far: block n accumulates in TMEM buffer n & 1
+            for (int t = pair; t < ntiles && !timed_out; t += npair) {
                 int z, mb, nb, rb, nk;
                 tile_of(t, z, mb, nb, rb, nk);
-                const int acc = it & 1;
-                const uint32_t use = (uint32_t)(it >> 1);
-                if (!mbar_wait(&bars->tempty[acc], (use & 1u) ^ 1u, abort)) {
-                    timed_out = true;
-                    break;
-                }
-                fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * 256);
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&bars->full[s], ph, abort)) {
+                for (int kb = 0; kb < nk; ++kb, ++blk) {
+                    const int acc = (int)(blk & 1u);
+                    if (!mbar_wait(&bars->tempty[acc], ((blk >> 1) & 1u) ^ 1u, abort) ||
+                        !mbar_wait(&bars->full[s], ph, abort)) {
                         timed_out = true;
                         break;
                     }
                     fence_after();
+                    const uint32_t d = tmem + (uint32_t)(acc * 256);
                     const uint32_t sa = base + s * STAGE3_BYTES;
                     const uint32_t sb = sa + 2 * PART3;
 #pragma unroll
@@ -328,18 +356,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         const uint64_t a_lo = AMN ? sdesc_mn(sa + PART3 + ao) : sdesc(sa + PART3 + ao);
                         const uint64_t b_hi = BMN ? sdesc_mn(sb + bo) : sdesc(sb + bo);
                         const uint64_t b_lo = BMN ? sdesc_mn(sb + PART3 + bo) : sdesc(sb + PART3 + bo);
-                        umma2_tf32(d, a_lo, b_hi, ID, (kb | k) != 0);
+                        umma2_tf32(d, a_lo, b_hi, ID, k != 0);
                         umma2_tf32(d, a_hi, b_lo, ID, 1u);
                         umma2_tf32(d, a_hi, b_hi, ID, 1u);
                     }
                     umma2_commit_both(&bars->empty[s]);
+                    umma2_commit_both(&bars->tfull[acc]);
                     if (++s == STAGES3) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
-                if (timed_out) break;
-                umma2_commit_both(&bars->tfull[acc]);
             }
             if (timed_out) *abort = 1;
             umma2_commit_both(&bars->drain);
@@ -347,31 +374,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         } else if (lane == 0) {
             mbar_wait(&bars->drain, 0, abort, true);
         }
+    }
     } else {
-        const int ew = warp - 2;
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_HIGH));
+        // epilogue warps: every k-block's partial product is added into fp32
+        // registers (round to nearest) as soon as its accumulator is complete,
+        // so that the tensor core accumulates at most one 32-deep block at a time
+        const int ew = warp - 4;
         const int q = warp & 3;
         const int h = ew >> 2;
         unsigned char* stage = gbase + STAGES3 * STAGE3_BYTES + ew * STAGE_OUT_BYTES;
         const uint32_t stage_s = base + STAGES3 * STAGE3_BYTES + ew * STAGE_OUT_BYTES;
         const uint32_t lead_tempty0 = map_rank(su32(&bars->tempty[0]), 0);
         const uint32_t lead_tempty1 = map_rank(su32(&bars->tempty[1]), 0);
-        int it = 0;
-        for (int t = pair; t < ntiles && !timed_out; t += npair, ++it) {
+        uint32_t blk = 0;
+        for (int t = pair; t < ntiles && !timed_out; t += npair) {
             int z, mb, nb, rb, nk;
             tile_of(t, z, mb, nb, rb, nk);
-            const int acc = it & 1;
-            const uint32_t use = (uint32_t)(it >> 1);
-            if (!mbar_wait(&bars->tfull[acc], use & 1u, abort)) {
-                timed_out = true;
-                break;
+            float acc[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) acc[c][e] = 0.f;
+            for (int kb = 0; kb < nk; ++kb, ++blk) {
+                const int a = (int)(blk & 1u);
+                if (!mbar_wait(&bars->tfull[a], (blk >> 1) & 1u, abort)) {
+                    timed_out = true;
+                    break;
+                }
+                fence_after();
+                promote(acc, tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 256 + h * 128));
+                fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(a ? lead_tempty1 : lead_tempty0);
             }
-            fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + h * 128);
-            epilogue3<EPI>(taddr, mb * 256 + (int)rank * 128 + q * 32, nb * 256 + h * 128, I, J, z, bias, mhi, mlo,
+            if (timed_out) break;
+            epilogue3<EPI>(acc, mb * 256 + (int)rank * 128 + q * 32, nb * 256 + h * 128, I, J, z, bias, mhi, mlo,
                            ldm, &maps.c0, &maps.c1, stage, stage_s);
-            fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc ? lead_tempty1 : lead_tempty0);
         }
         if (timed_out) *abort = 1;
         if (lane == 0) bulk_wait_all0();
@@ -436,7 +475,7 @@ dlrm_status launch3(const Maps3& maps, int I, int J, int R, int r_chunk, int S, 
     const long long ntiles = (long long)((I + 255) / 256) * ((J + 255) / 256) * S;
     const int pairs = sm_count3() / 2;
     const int grid = 2 * (int)(ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS, SMEM3_BYTES, st>>>(maps, I, J, R, r_chunk, S, bias, mhi, mlo, (long long)ldm, err);
+    kern<<<grid, THREADS3, SMEM3_BYTES, st>>>(maps, I, J, R, r_chunk, S, bias, mhi, mlo, (long long)ldm, err);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }

@@ -60,7 +60,14 @@ __device__ __forceinline__ void load_tile(float (&S)[TK][TN + 4], const float* _
     }
 }
 
-__device__ __forceinline__ float tf32_hi_part(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+// hi part of a 3xTF32 pair: v rounded to the nearest TF32 value (ties away from
+// zero; magnitudes that would round up to infinity are truncated), lo = v - hi exactly.
+__device__ __forceinline__ float tf32_hi_part(float v) {
+    const uint32_t u = __float_as_uint(v);
+    uint32_t r = u + 0x1000u;
+    if ((r & 0x7F800000u) == 0x7F800000u) r = u;
+    return __uint_as_float(r & 0xFFFFE000u);
+}
 
 // Output tile (i0.., j0..) of C(i, j), reduction over r in [r_begin, r_end).
 // B_ONES: B has a synthesized extra column j == NB of ones (weight-gradient bias term).

@@ -65,6 +65,21 @@ def test_gemm_f32_exact_on_small_integers(a_mn, b_mn):
     assert np.array_equal(got, A64 @ B64.T)
 
 
+@pytest.mark.parametrize("R", [64, 1024, 65536])
+def test_gemm_f32_long_same_sign_sums_do_not_drift(R):
+    # all terms positive: an accumulator that rounds toward zero loses ~R/8 units in the last place
+    # (1e-5 of the sum at R = 1024); fp32 with round-to-nearest stays near 1e-7
+    I = J = 256
+    g = torch.Generator().manual_seed(R + 1)
+    A = torch.rand((I, R), generator=g)
+    B = torch.rand((J, R), generator=g)
+    got = _run(A, False, B, False, I, J, R)
+    A64, B64 = A.double().numpy(), B.double().numpy()
+    want = A64 @ B64.T
+    rel = np.abs(got - want) / want
+    assert rel.max() <= 1e-6, rel.max()
+
+
 def test_gemm_f32_bit_reproducible():
     I, J, R = 512, 384, 30000   # long reduction: split into fixed r-ranges
     g = torch.Generator().manual_seed(9)

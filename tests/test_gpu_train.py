@@ -2,14 +2,24 @@
 loss, every MLP gradient, the row-sorted embedding gradients (bit-exact row
 set and counts), the SGD update of touched rows only, and bit-reproducibility.
 
-Gradients are batch sums; each is judged against its own sum of |terms|
-(from the oracle): |gpu - oracle| <= 1e-5 * (|oracle| + sum|terms|).
+Two checks per tensor:
+  1. a first-order error bound: gradients are batch sums, each judged against
+     its own sum of |terms| propagated through the network (from the
+     oracle): |gpu - oracle| <= 1e-5 * (|oracle| + sum|terms|). It holds for
+     any correct fp32 evaluation order, but on the deep configurations the
+     propagated sizes are loose;
+  2. an fp32 error budget: the 50/90/99% quantiles of |gpu - oracle| may be at
+     most 16x those of the same training step run in plain fp32 by PyTorch on
+     the CPU (fp32_budget.py), plus 1e-7 of the tensor's largest entry. A
+     kernel that loses precision (say, products taken at TF32 width, or a
+     biased accumulator) fails this one.
 """
 import numpy as np
 import pytest
 import torch
 
 import embedding_bags_dot_b200 as E
+from fp32_budget import check_within_budget, train_grads_f32
 from gpucase import GpuModel, to_np
 from oracle import oracle as O
 from synth import CONFIGS, gen, shrink
@@ -81,6 +91,7 @@ def case(request):
     t = Trainer(cfg)
     model = O.model_from_config(cfg)
     ref = O.train_grads(model, t.batch.dense, t.batch.offsets, t.batch.indices, t.batch.labels, scales=True)
+    ref["f32"] = train_grads_f32(model, t.batch.dense, t.batch.offsets, t.batch.indices, t.batch.labels)
     return cfg, t, model, ref
 
 
@@ -89,10 +100,12 @@ def test_loss_and_dense_gradients(case):
     loss, y = t.backward()
     assert abs(loss - ref["loss"]) <= RTOL * abs(ref["loss"]), (loss, ref["loss"])
     assert np.abs(y - ref["y_hat"]).max() <= RTOL * 1.0
+    check_within_budget(y, ref["y_hat"], ref["f32"]["y_hat"], f"{cfg.name} y_hat")
     grads = t.dense_grads()
     for key in ("bot_dW", "bot_db", "top_dW", "top_db"):
-        for l, (gg, oo, ss) in enumerate(zip(grads[key], ref[key], ref[key + "_s"])):
+        for l, (gg, oo, ss, o32) in enumerate(zip(grads[key], ref[key], ref[key + "_s"], ref["f32"][key])):
             _close(gg, oo, ss, f"{cfg.name} {key}[{l}]")
+            check_within_budget(gg, oo, o32, f"{cfg.name} {key}[{l}]")
 
 
 def test_embedding_row_gradients_and_bookkeeping(case):
@@ -110,6 +123,8 @@ def test_embedding_row_gradients_and_bookkeeping(case):
     got_rows = rows.cpu().numpy()[:nr].astype(np.int64)
     assert np.array_equal(got_rows, touched), "touched rows must match bit-exactly, in increasing order"
     _close(to_np(rg)[:nr], ref["table_grad"][touched], ref["table_grad_s"][touched], f"{cfg.name} row grads")
+    check_within_budget(to_np(rg)[:nr], ref["table_grad"][touched], ref["f32"]["table_grad"][touched],
+                        f"{cfg.name} row grads")
 
 
 def test_sparse_sgd_updates_touched_rows_only(case):
