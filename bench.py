@@ -446,7 +446,13 @@ def run_train(args, cfg, rank, world, local_rank):
     total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][2]), world, dev)
     bwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     sgd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    samples = cfg.B * args.steps * world
+    # roofline of the dominant kernel, the 3xTF32 GEMM, on the largest layer of the step (top layer 2: the
+    # batch x 1024 x 1024 forward product), timed alone right after the step loop
+    I, J, R = cfg.B, cfg.top[2], cfg.top[1]
+    gemm_ms = max_over_ranks(time_tf32x3(I, J, R, dev, stream), world, dev)
+    _, peak_bf16, peak_kind = read_peaks()
+    peak_tf32 = peak_bf16 * TF32_PER_BF16
+    tensor_tflops = 3 * 2.0 * I * J * R / (gemm_ms * 1e-3) / 1e12
     if rank == 0:
         out = {"metric": "DLRM training samples/s on 1 B200 (forward + backward + sparse SGD)",
                "value": aggregate_rate(cfg.B * args.steps, world, total_ms), "unit": "samples/s", "n_gpus": world,
@@ -456,9 +462,48 @@ def run_train(args, cfg, rank, world, local_rank):
                "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "lr": cfg.lr,
                           "nnz_max": nnz_max},
                "kernels_ms_per_step": {"dlrm_backward": bwd, "dlrm_sparse_sgd": sgd},
+               "roofline": {"bound": "tensor", "achieved": tensor_tflops, "peak": peak_tf32, "unit": "TFLOP/s",
+                            "frac": tensor_tflops / peak_tf32, "traffic": None,
+                            "peak_kind": f"{peak_kind} bf16 burst x {TF32_PER_BF16:.3f} (nominal TF32:BF16)",
+                            "kernel": "gemm3x_kernel (dlrm_gemm_tf32x3)",
+                            "shape": f"{I}x{J}x{R} K-major x K-major",
+                            "flops_per_launch": "3 TF32 products x 2*I*J*R", "avg_launch_ms": gemm_ms,
+                            "fp32_equiv_tflops": 2.0 * I * J * R / (gemm_ms * 1e-3) / 1e12},
                "loss_last": float(loss.item()), "gpu_launches": int(n1 - n0), "clocks": clk}
         print(json.dumps(out), flush=True)
     return 0
+
+
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense TF32 : BF16 tensor rate of B200
+
+
+def time_tf32x3(I, J, R, dev, stream, reps=10, warmup=3):
+    """Average launch time (ms) of the 3xTF32 GEMM kernel alone (dlrm_gemm_tf32x3, operands already in pair form,
+    A [I][R] and B [J][R] K-major) on the given stream, CUDA events around each launch."""
+    import torch
+    import embedding_bags_dot_b200 as E
+    g = torch.Generator(device=dev).manual_seed(7)
+    A = torch.randn((I, R), device=dev, generator=g)
+    B = torch.randn((J, R), device=dev, generator=g) / R ** 0.5
+    Ah, Al, Bh, Bl = torch.empty_like(A), torch.empty_like(A), torch.empty_like(B), torch.empty_like(B)
+    E.dlrm_tf32_split(I, R, A, R, Ah, Al, R, stream=stream)
+    E.dlrm_tf32_split(J, R, B, R, Bh, Bl, R, stream=stream)
+    del A, B
+    C = torch.empty((I, J), device=dev)
+    ws = E.alloc_workspace(E.dlrm_gemm_tf32x3_workspace_size(I, J, R), dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for _ in range(warmup):
+        E.dlrm_gemm_tf32x3(I, J, R, Ah, Al, R, False, Bh, Bl, R, False, C, J, ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        E.dlrm_gemm_tf32x3(I, J, R, Ah, Al, R, False, Bh, Bl, R, False, C, J, ws, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    st = E.dlrm_check_error(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device error record after the GEMM timing: {st}")
+    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
 
 
 def run_latency(args, cfg, rank, world, local_rank):

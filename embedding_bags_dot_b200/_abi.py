@@ -78,6 +78,11 @@ _SIGS = {
     "dlrm_gemm_f32_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
     "dlrm_gemm_f32": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
                                 C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    "dlrm_tf32_split": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int,
+                                  C.c_void_p]),
+    "dlrm_gemm_tf32x3_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int]),
+    "dlrm_gemm_tf32x3": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                                   C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
 }
 
 
@@ -244,6 +249,24 @@ def dlrm_gemm_f32(I: int, J: int, R: int, A, lda: int, a_mn: bool, B, ldb: int, 
     (B likewise)."""
     return _check(lib().dlrm_gemm_f32(int(I), int(J), int(R), _ptr(A), int(lda), int(bool(a_mn)), _ptr(B), int(ldb),
                                       int(bool(b_mn)), _ptr(C), int(ldc), _ptr(ws), _stream(stream)), "dlrm_gemm_f32")
+
+
+def dlrm_tf32_split(rows: int, cols: int, src, lds: int, hi, lo, ldd: int, stream=None):
+    """hi = src rounded to the nearest TF32 value, lo = src - hi (exact)."""
+    return _check(lib().dlrm_tf32_split(int(rows), int(cols), _ptr(src), int(lds), _ptr(hi), _ptr(lo), int(ldd),
+                                        _stream(stream)), "dlrm_tf32_split")
+
+
+def dlrm_gemm_tf32x3_workspace_size(I: int, J: int, R: int) -> int:
+    return int(lib().dlrm_gemm_tf32x3_workspace_size(int(I), int(J), int(R)))
+
+
+def dlrm_gemm_tf32x3(I: int, J: int, R: int, A_hi, A_lo, lda: int, a_mn: bool, B_hi, B_lo, ldb: int, b_mn: bool, C,
+                     ldc: int, ws, stream=None):
+    """dlrm_gemm_f32 on operands already split by dlrm_tf32_split."""
+    return _check(lib().dlrm_gemm_tf32x3(int(I), int(J), int(R), _ptr(A_hi), _ptr(A_lo), int(lda), int(bool(a_mn)),
+                                         _ptr(B_hi), _ptr(B_lo), int(ldb), int(bool(b_mn)), _ptr(C), int(ldc),
+                                         _ptr(ws), _stream(stream)), "dlrm_gemm_tf32x3")
 
 
 # ----------------------------------------------------------------- training step (fp32)

@@ -63,4 +63,31 @@ dlrm_status dlrm_gemm_f32(int I, int J, int R, const float* A, int lda, int a_mn
     return r;
 }
 
+dlrm_status dlrm_tf32_split(int rows, int cols, const float* src, int lds, float* hi, float* lo, int ldd,
+                            dlrm_stream stream) {
+    if (rows < 0 || cols < 0 || lds < cols || ldd < cols) return DLRM_ERR_INVALID_ARG;
+    if ((long long)rows * cols > 0 && (!src || !hi || !lo)) return DLRM_ERR_INVALID_ARG;
+    return launch_split_pair(rows, cols, src, lds, hi, lo, ldd, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dlrm_gemm_tf32x3_workspace_size(int I, int J, int R) {
+    if (!args_ok(I, J, R)) return 0;
+    return align_up(DLRM_ERR_RECORD_BYTES, 256) + sizeof(float) * tf32x3_wgrad_scratch_floats(I, J, R);
+}
+
+dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float* A_lo, int lda, int a_mn,
+                             const float* B_hi, const float* B_lo, int ldb, int b_mn, float* C, int ldc, void* ws,
+                             dlrm_stream stream) {
+    if (!args_ok(I, J, R) || !A_hi || !A_lo || !B_hi || !B_lo || !C) return DLRM_ERR_INVALID_ARG;
+    const int a_cols = a_mn ? I : R, b_cols = b_mn ? J : R;
+    if (lda < a_cols || ldb < b_cols || ldc < J || lda % 4 || ldb % 4 || ldc % 4) return DLRM_ERR_INVALID_ARG;
+    const uintptr_t al = (uintptr_t)A_hi | (uintptr_t)A_lo | (uintptr_t)B_hi | (uintptr_t)B_lo | (uintptr_t)C;
+    if (al & 15) return DLRM_ERR_INVALID_ARG;
+    if (!ws || ((uintptr_t)ws & 15)) return DLRM_ERR_WORKSPACE;
+    char* w = static_cast<char*>(ws);
+    return tf32x3_gemm(I, J, R, F32Pair{A_hi, A_lo, lda}, a_mn != 0, F32Pair{B_hi, B_lo, ldb}, b_mn != 0, C, ldc,
+                       reinterpret_cast<float*>(w + align_up(DLRM_ERR_RECORD_BYTES, 256)),
+                       reinterpret_cast<ErrRecord*>(w), reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

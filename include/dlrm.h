@@ -212,6 +212,23 @@ size_t dlrm_gemm_f32_workspace_size(int I, int J, int R, int a_mn, int b_mn);
 dlrm_status dlrm_gemm_f32(int I, int J, int R, const float* A, int lda, int a_mn, const float* B, int ldb, int b_mn,
                           float* C, int ldc, void* ws, dlrm_stream stream);
 
+/* The two halves of dlrm_gemm_f32, for callers that keep operands in pair
+ * form (as the training step does for every activation and gradient).
+ * dlrm_tf32_split: hi[r][c] = src[r][c] rounded to the nearest TF32 value,
+ * lo[r][c] = src[r][c] - hi[r][c] (exact), for r < rows, c < cols; device
+ * fp32 pointers, leading dimensions in elements (lds >= cols, ldd >= cols).
+ * dlrm_gemm_tf32x3: the product of dlrm_gemm_f32 from pairs (A_hi, A_lo)
+ * and (B_hi, B_lo) that share the layout and leading dimension given; all
+ * pointers 16-byte aligned, lda/ldb/ldc multiples of 4. ws: 16-byte aligned,
+ * dlrm_gemm_tf32x3_workspace_size(I, J, R) bytes (error record and the
+ * partial sums of long reductions). Errors as dlrm_gemm_f32. */
+dlrm_status dlrm_tf32_split(int rows, int cols, const float* src, int lds, float* hi, float* lo, int ldd,
+                            dlrm_stream stream);
+size_t dlrm_gemm_tf32x3_workspace_size(int I, int J, int R);
+dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float* A_lo, int lda, int a_mn,
+                             const float* B_hi, const float* B_lo, int ldb, int b_mn, float* C, int ldc, void* ws,
+                             dlrm_stream stream);
+
 /* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
 #define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
 

@@ -7,7 +7,8 @@ measured, not guessed: the same model is run forward and backward in fp32 by
 PyTorch on the CPU (torch.nn.functional.embedding_bag, dense matmuls,
 autograd), and its distance to the fp64 oracle, per tensor and per quantile,
 is the budget. This module is a yardstick of fp32 precision only; the values
-the GPU is compared with are the oracle's.
+the GPU is compared with are the oracle's. (The 3xTF32 pair product that the
+GPU's GEMMs use is available here too, for study: tf32x3=True.)
 
 Reading of the training step used here (as in the oracle): ReLU after every
 bottom layer and every hidden top layer, the last top layer linear, Z = the
@@ -46,11 +47,31 @@ def _mm3(x, y):
     return (xl @ yh + xh @ yl) + xh @ yh
 
 
-def train_grads_f32(model, dense, offsets, indices, labels, tf32x3=False):
+class _MM1(torch.autograd.Function):
+    """a @ b.T with both operands rounded to TF32 (the precision a single TF32 product keeps)."""
+
+    @staticmethod
+    def forward(ctx, a, b):
+        ctx.save_for_backward(a, b)
+        return _tf32_round(a) @ _tf32_round(b).t()
+
+    @staticmethod
+    def backward(ctx, g):
+        a, b = ctx.saved_tensors
+        return _tf32_round(g) @ _tf32_round(b), _tf32_round(g.t()) @ _tf32_round(a)
+
+
+def train_grads_f32(model, dense, offsets, indices, labels, tf32x3=False, tf32x1=False):
     """Loss, y_hat and every gradient of the fp32 training step (CPU, float32). With tf32x3 the
-    matrix products of the MLPs (forward and both gradients) are taken as 3xTF32 pair products."""
+    matrix products of the MLPs (forward and both gradients) are taken as 3xTF32 pair products,
+    with tf32x1 as single TF32 products."""
     f = torch.float32
-    mm = (lambda a, W: _MM3.apply(a, W)) if tf32x3 else (lambda a, W: a @ W.t())  # noqa: E731
+    if tf32x3:
+        mm = lambda a, W: _MM3.apply(a, W)  # noqa: E731
+    elif tf32x1:
+        mm = lambda a, W: _MM1.apply(a, W)  # noqa: E731
+    else:
+        mm = lambda a, W: a @ W.t()  # noqa: E731
     K, d = model.K, model.d
     B = dense.shape[0]
     tables = torch.tensor(model.tables, dtype=f, requires_grad=True)
@@ -84,20 +105,21 @@ def train_grads_f32(model, dense, offsets, indices, labels, tf32x3=False):
     loss = (torch.nn.functional.softplus(z) - y * z).mean()
     loss.backward()
     g = lambda ts: [t.grad.double().numpy() for t in ts]  # noqa: E731
-    return {"loss": float(loss), "y_hat": torch.sigmoid(z).detach().double().numpy(), "bot_dW": g(bW),
+    return {"loss": float(loss.detach()), "y_hat": torch.sigmoid(z).detach().double().numpy(), "bot_dW": g(bW),
             "bot_db": g(bb), "top_dW": g(tW), "top_db": g(tb), "table_grad": tables.grad.double().numpy()}
 
 
-QUANTILES = (0.5, 0.9, 0.99)
-
-
 def check_within_budget(got, want, ref32, what, factor=16.0):
-    """Each listed quantile of |got - want| is at most `factor` times the same quantile
-    of |ref32 - want|, plus 1e-7 of max|want| (one fp32 rounding of the largest entry)."""
+    """The 50% and 90% quantiles of |got - want| (and the 99% one from 1000 entries up) are at most
+    `factor` times the same quantiles of |ref32 - want|, plus 1e-7 of max|want| (one fp32 rounding of
+    the largest entry). Tensors of fewer than 64 entries have no error distribution to compare; they
+    are left to the first-order bound."""
     got, want, ref32 = (np.asarray(a, np.float64).ravel() for a in (got, want, ref32))
+    if want.size < 64:
+        return
     floor = 1e-7 * float(np.abs(want).max(initial=0.0))
     e, e32 = np.abs(got - want), np.abs(ref32 - want)
-    for q in QUANTILES:
+    for q in (0.5, 0.9) + ((0.99,) if want.size >= 1000 else ()):
         a, b = float(np.quantile(e, q)), float(np.quantile(e32, q))
         assert a <= factor * b + floor, (f"{what}: error quantile {q} = {a:.3g} exceeds {factor} x fp32 budget "
                                          f"{b:.3g} (+{floor:.2g})")

@@ -88,3 +88,26 @@ def test_gemm_f32_bit_reproducible():
     a = _run(A, True, B, True, I, J, R)
     b = _run(A, True, B, True, I, J, R)
     assert np.array_equal(a, b)
+
+
+def test_split_and_pair_gemm_match_the_one_call_gemm():
+    I, J, R = 700, 300, 2000
+    g = torch.Generator().manual_seed(11)
+    _, A = _operand(I, R, False, g, "randn")
+    _, B = _operand(J, R, True, g, "randn")
+    want = _run(A, False, B, True, I, J, R)
+    Ad, Bd = A.cuda(), B.cuda()
+    Ah, Al = torch.empty_like(Ad), torch.empty_like(Ad)
+    Bh, Bl = torch.empty_like(Bd), torch.empty_like(Bd)
+    E.dlrm_tf32_split(Ad.shape[0], Ad.shape[1], Ad, Ad.shape[1], Ah, Al, Ad.shape[1])
+    E.dlrm_tf32_split(Bd.shape[0], Bd.shape[1], Bd, Bd.shape[1], Bh, Bl, Bd.shape[1])
+    # the split is exact and hi is a TF32 number (13 low mantissa bits clear)
+    assert torch.equal(Ah + Al, Ad)
+    assert int((Ah.view(torch.int32) & 0x1FFF).abs().max()) == 0
+    assert float((Al.abs() - Ah.abs() * 2.0 ** -11).max()) <= 0   # |lo| <= half a TF32 unit of |hi|
+    ldc = (J + 3) // 4 * 4
+    C = torch.full((I, ldc), float("nan"), device="cuda")
+    ws = E.alloc_workspace(E.dlrm_gemm_tf32x3_workspace_size(I, J, R))
+    E.dlrm_gemm_tf32x3(I, J, R, Ah, Al, Ad.shape[1], False, Bh, Bl, Bd.shape[1], True, C, ldc, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    assert np.array_equal(to_np(C)[:, :J], want)
