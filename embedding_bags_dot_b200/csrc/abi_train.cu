@@ -234,11 +234,19 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     }
     const F32Pair xd_pair = P(W.bact[nb - 1], W.ldb[nb - 1]);   // ld = d (d % 4 == 0 on this path)
     const float* x_dense = F(W.xd);
-    if ((r = launch_merge_pair(B, d, xd_pair.hi, xd_pair.lo, xd_pair.ld, F(W.xd), d, st))) return r;
+    // the warp-per-sample interaction reads and writes pairs; other shapes go through plain fp32 copies
+    const bool pair_inter = interact_pair_supported(K, d);
     if ((r = launch_embbag(tm, T->data, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err, st))) return r;
-    if ((r = launch_interact(B, K, d, x_dense, F(W.E), F(W.concat), W.ldc, DLRM_F32, st))) return r;
-    const int cw = top->dims[0];
-    if ((r = launch_split_pair(B, cw, F(W.concat), W.ldc, F(W.concat_p[0]), F(W.concat_p[1]), W.ldc, st))) return r;
+    if (pair_inter) {
+        if ((r = launch_interact_fwd_pair(B, K, d, xd_pair, F(W.E), F(W.concat_p[0]), F(W.concat_p[1]), W.ldc, st)))
+            return r;
+    } else {
+        if ((r = launch_merge_pair(B, d, xd_pair.hi, xd_pair.lo, xd_pair.ld, F(W.xd), d, st))) return r;
+        if ((r = launch_interact(B, K, d, x_dense, F(W.E), F(W.concat), W.ldc, DLRM_F32, st))) return r;
+        if ((r = launch_split_pair(B, top->dims[0], F(W.concat), W.ldc, F(W.concat_p[0]), F(W.concat_p[1]), W.ldc,
+                                   st)))
+            return r;
+    }
     const F32Pair concat_p = P(W.concat_p, W.ldc);
     for (int l = 0; l < nt; ++l) {
         const F32Pair in = l == 0 ? concat_p : P(W.tact[l - 1], W.ldt[l - 1]);
@@ -278,8 +286,14 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
         }
     }
     // d(concat) -> gradient of the last bottom layer's pre-activation (ReLU mask applied) and dE
-    if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;
-    if ((r = launch_split_pair(B, d, F(W.dxd), d, F(W.g[pp][0]), F(W.g[pp][1]), d, st))) return r;
+    if (pair_inter) {
+        if ((r = launch_interact_bwd_pair(B, K, d, xd_pair, F(W.E), F(W.dcat), W.ldc, F(W.g[pp][0]), F(W.g[pp][1]), d,
+                                          GF(G.dE), st)))
+            return r;
+    } else {
+        if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;
+        if ((r = launch_split_pair(B, d, F(W.dxd), d, F(W.g[pp][0]), F(W.g[pp][1]), d, st))) return r;
+    }
     cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), d};
     pp ^= 1;
     for (int l = nb - 1; l >= 0; --l) {

@@ -91,6 +91,13 @@ dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* 
 // out[n][k] = sum_{z < S} part[z][n][k] in increasing z (part split stride N * ldp)
 dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st);
 
+// Warp-per-sample fp32 interaction on pairs (interact_f32.cu), for K = 26 and d = 64 or 128.
+bool interact_pair_supported(int K, int d);
+dlrm_status launch_interact_fwd_pair(int B, int K, int d, F32Pair x_dense, const float* E, float* concat_hi,
+                                     float* concat_lo, int ldc, cudaStream_t st);
+dlrm_status launch_interact_bwd_pair(int B, int K, int d, F32Pair x_dense, const float* E, const float* dconcat,
+                                     int ldc, float* dx_hi, float* dx_lo, int lddx, float* dE, cudaStream_t st);
+
 dlrm_status launch_bce(int B, const float* z, const float* y, float* dz, float* y_hat, float* partial, float* loss,
                        cudaStream_t st);
 size_t interact_bwd_smem(int K, int d);

@@ -37,6 +37,7 @@ def _cases():
         "train-mix": shrink(tr, B=97, rows_cap=400).with_(bag="mix", seed=2),
         "tiny-train": CONFIGS["tiny"].with_(training=True, B=203),
         "train-hot-rows": shrink(tr, B=2000, rows_cap=50),   # long segments: many occurrences per row
+        "train-d64": shrink(tr, B=333, rows_cap=2000).with_(d=64, bottom=(13, 256, 64), top=(415, 256, 1), seed=5),
     }
 
 
