@@ -7,7 +7,13 @@
 // Operands are F32Pair: plain fp32, or a 3xTF32 (hi, lo) pair whose value is
 // hi + lo exactly; the CUDA-core kernel reads either and writes either.
 //
-// The CUDA-core kernel covers the three operand layouts:
+// Shapes the tensor cores do not take get kernels of their own: the 13-wide
+// first bottom layer (narrow_fwd_kernel; its weight gradient is a weighted
+// column sum of dy, one pass), the one-column logit layer (gemv_rows_kernel,
+// outer_mask_kernel, weighted column sums), and every bias gradient is a
+// fixed-order column sum (colsum_w_kernel).
+//
+// The general CUDA-core kernel covers the three operand layouts:
 //   C(i, j) = sum_r A(i, r) B(j, r)
 //   A(i, r) = A[i*lda + r]  (AT = false)   or  A[r*lda + i]  (AT = true)
 //   B(j, r) = B[j*ldb + r]  (BT = false)   or  B[r*ldb + j]  (BT = true)
@@ -194,35 +200,148 @@ __global__ void split_sum_kernel(int S, long long N, int K, const float* __restr
     }
 }
 
-// Column sums of a [M][N] pair over fixed row chunks: part[p][c] = sum of rows
-// [p*rows_per, (p+1)*rows_per), eight row-interleaved partial sums combined in order.
-__global__ void __launch_bounds__(256) colsum_partial_kernel(long long M, int N, const float* __restrict__ hi,
-                                                             const float* __restrict__ lo, long long ld,
-                                                             long long rows_per, float* __restrict__ part) {
-    __shared__ float red[8][33];
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    const int c = blockIdx.x * 32 + tx;
+// Weighted column sums over fixed row chunks:
+//   part[p][c][w] = sum_{b in chunk p} A(b, c) * Wt(b, w),  w < NW
+// A is [M][N] plain or a pair (value hi + lo); Wt(b, w) = X[b][w] for w < kx
+// and 1 for w == kx when `ones`, 0 beyond. Each thread owns four columns, the
+// warps of a block (CS_WARPS(NW)) take rows in turn, and their partials are
+// combined in warp order: a fixed summation order for every result.
+__host__ __device__ constexpr int CS_WARPS(int nw) { return nw > 4 ? 4 : 8; }
+
+template <int NW>
+__global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const float* __restrict__ ah,
+                                                       const float* __restrict__ al, long long lda,
+                                                       const float* __restrict__ X, long long ldx, int kx, bool ones,
+                                                       long long rows_per, float* __restrict__ part) {
+    constexpr int WARPS = CS_WARPS(NW);
+    __shared__ float red[WARPS][128 * NW + 1];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int c0 = blockIdx.x * 128 + 4 * lane;
     const long long rb = (long long)blockIdx.y * rows_per;
     const long long re = rb + rows_per < M ? rb + rows_per : M;
-    float s = 0.f;
-    if (c < N)
-        for (long long r = rb + ty; r < re; r += 8) s += lo ? hi[r * ld + c] + lo[r * ld + c] : hi[r * ld + c];
-    red[ty][tx] = s;
+    const bool vec = (lda & 3) == 0 && c0 + 4 <= N;
+    float acc[4][NW];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int q = 0; q < NW; ++q) acc[e][q] = 0.f;
+    for (long long r = rb + w; r < re; r += WARPS) {
+        float v[4];
+        if (vec) {
+            const float4 h = __ldg(reinterpret_cast<const float4*>(ah + r * lda + c0));
+            v[0] = h.x, v[1] = h.y, v[2] = h.z, v[3] = h.w;
+            if (al) {
+                const float4 l = __ldg(reinterpret_cast<const float4*>(al + r * lda + c0));
+                v[0] += l.x, v[1] += l.y, v[2] += l.z, v[3] += l.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                v[e] = (c0 + e < N) ? (al ? ah[r * lda + c0 + e] + al[r * lda + c0 + e] : ah[r * lda + c0 + e]) : 0.f;
+        }
+        float wt[NW];
+#pragma unroll
+        for (int q = 0; q < NW; ++q) wt[q] = q < kx ? __ldg(X + r * ldx + q) : ((ones && q == kx) ? 1.f : 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int q = 0; q < NW; ++q) acc[e][q] = fmaf(v[e], wt[q], acc[e][q]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int q = 0; q < NW; ++q) red[w][(4 * lane + e) * NW + q] = acc[e][q];
     __syncthreads();
-    if (ty == 0 && c < N) {
+    for (int i = threadIdx.x; i < 128 * NW; i += blockDim.x) {
+        const int c = blockIdx.x * 128 + i / NW;
+        if (c >= N) continue;
         float t = 0.f;
 #pragma unroll
-        for (int y = 0; y < 8; ++y) t += red[y][tx];
-        part[(long long)blockIdx.y * N + c] = t;
+        for (int y = 0; y < WARPS; ++y) t += red[y][i];
+        part[((long long)blockIdx.y * N + c) * NW + (i % NW)] = t;
     }
 }
 
-__global__ void colsum_final_kernel(int P, int N, const float* __restrict__ part, float* __restrict__ out) {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= N) return;
-    float s = 0.f;
-    for (int p = 0; p < P; ++p) s += part[(long long)p * N + c];
-    out[c] = s;
+// out(c, w) = sum_p part[p][c][w] in increasing p; w < kx -> dW[c * ldw + w], w == kx -> db[c]
+__global__ void colsum_w_final_kernel(int P, int N, int NW, int kx, bool ones, const float* __restrict__ part,
+                                      float* __restrict__ dW, long long ldw, float* __restrict__ db) {
+    const long long n = (long long)N * NW;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(i / NW), q = (int)(i % NW);
+        if (q > kx || (q == kx && !ones)) continue;
+        float s = 0.f;
+        for (int p = 0; p < P; ++p) s += part[(long long)p * n + i];
+        if (q < kx) dW[c * ldw + q] = s;
+        else db[c] = s;
+    }
+}
+
+// y[b][n] = act(sum_{k < K} x(b, k) W[n][k] + bias[n]) for K <= 16 (the 13 dense features), one thread
+// per output column with its weight row in registers; y written as a pair or plain.
+__global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int K, const float* __restrict__ xh,
+                                                         const float* __restrict__ xl, long long ldx,
+                                                         const float* __restrict__ W, const float* __restrict__ Wl,
+                                                         long long ldw, const float* __restrict__ bias, bool relu,
+                                                         float* __restrict__ yh, float* __restrict__ yl, long long ldy,
+                                                         long long rows_per) {
+    const int n = blockIdx.x * 128 + threadIdx.x;
+    if (n >= N) return;
+    float wr[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) wr[k] = k < K ? (Wl ? W[n * ldw + k] + Wl[n * ldw + k] : W[n * ldw + k]) : 0.f;
+    const float bn = bias[n];
+    const long long rb = (long long)blockIdx.y * rows_per;
+    const long long re = rb + rows_per < M ? rb + rows_per : M;
+    for (long long b = rb; b < re; ++b) {
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (k < K) s = fmaf(xl ? __ldg(xh + b * ldx + k) + __ldg(xl + b * ldx + k) : __ldg(xh + b * ldx + k), wr[k], s);
+        s += bn;
+        if (relu) s = s > 0.f ? s : 0.f;
+        if (yl) {
+            const float h = tf32_hi_part(s);
+            yh[b * ldy + n] = h;
+            yl[b * ldy + n] = s - h;
+        } else {
+            yh[b * ldy + n] = s;
+        }
+    }
+}
+
+// z[b] = sum_k x(b, k) w[k] + bias[0] (a one-column layer): one warp per row
+__global__ void __launch_bounds__(256) gemv_rows_kernel(long long M, int K, const float* __restrict__ xh,
+                                                        const float* __restrict__ xl, long long ldx,
+                                                        const float* __restrict__ w, const float* __restrict__ wl,
+                                                        const float* __restrict__ bias, float* __restrict__ z) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long b = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); b < M; b += warps) {
+        float s = 0.f;
+        for (int k = lane; k < K; k += 32) {
+            const float v = xl ? xh[b * ldx + k] + xl[b * ldx + k] : xh[b * ldx + k];
+            s = fmaf(v, wl ? __ldg(w + k) + __ldg(wl + k) : __ldg(w + k), s);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) z[b] = s + bias[0];
+    }
+}
+
+// dx[b][k] = dz[b] * w[k] where relu_of(b, k) > 0, else 0 (data gradient of a one-column layer), as a pair
+__global__ void outer_mask_kernel(long long M, int K, const float* __restrict__ dz, const float* __restrict__ w,
+                                  const float* __restrict__ wl, const float* __restrict__ mh, const float* __restrict__ ml, long long ldm,
+                                  float* __restrict__ dh, float* __restrict__ dl, long long ldd) {
+    const long long n = M * K;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const long long b = i / K;
+        const int k = (int)(i - b * K);
+        const float m = ml ? mh[b * ldm + k] + ml[b * ldm + k] : mh[b * ldm + k];
+        const float v = m > 0.f ? dz[b] * (wl ? __ldg(w + k) + __ldg(wl + k) : __ldg(w + k)) : 0.f;
+        const float h = tf32_hi_part(v);
+        dh[b * ldd + k] = h;
+        dl[b * ldd + k] = v - h;
+    }
 }
 
 int colsum_chunks(int M) {
@@ -286,11 +405,52 @@ dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, fl
     return DLRM_OK;
 }
 
+// Columns of a weighted column sum (launch_colsum_w) per chunk; chunks of 512 rows, at most 128.
+constexpr int CS_NW = 16;
+
+dlrm_status launch_colsum_w(int M, int N, F32Pair A, const float* X, int ldx, int kx, bool ones, float* dW, int ldw,
+                            float* db, float* scratch, cudaStream_t st) {
+    const int P = colsum_chunks(M);
+    const long long rows_per = ((long long)M + P - 1) / P;
+    const dim3 grid((unsigned)((N + 127) / 128), (unsigned)P);
+    const int nw = kx + (ones ? 1 : 0);
+    int NW;
+    if (nw <= 1) {
+        colsum_w_kernel<1><<<grid, 32 * CS_WARPS(1), 0, st>>>(M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones, rows_per,
+                                                              scratch);
+        NW = 1;
+    } else {
+        colsum_w_kernel<CS_NW><<<grid, 32 * CS_WARPS(CS_NW), 0, st>>>(M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones,
+                                                                      rows_per, scratch);
+        NW = CS_NW;
+    }
+    DLRM_LAUNCH_CHECK();
+    colsum_w_final_kernel<<<grid_stride_blocks((long long)N * NW), 256, 0, st>>>(P, N, NW, kx, ones, scratch, dW, ldw,
+                                                                               db);
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
 dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b, float* y, float* y_lo,
                              int ldy, bool relu, ErrRecord* err, cudaStream_t st) {
     if (M == 0) return DLRM_OK;
     if (relu && y_lo && tf32x3_supported(M, N, K, x, W))
         return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, err, st);
+    if (K <= 16) {
+        const long long rows_per = 256;
+        const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + rows_per - 1) / rows_per));
+        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy,
+                                                rows_per);
+        DLRM_LAUNCH_CHECK();
+        return DLRM_OK;
+    }
+    if (N == 1 && !relu && !y_lo) {
+        const long long blocks = (M + 7) / 8;
+        gemv_rows_kernel<<<(int)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, st>>>(M, K, x.hi, x.lo, x.ld, W.hi,
+                                                                                     W.lo, b, y);
+        DLRM_LAUNCH_CHECK();
+        return DLRM_OK;
+    }
     if (relu)
         gemm_f32_kernel<false, false, EPI_BIAS_RELU, false><<<grid_for(M, N, 1), 256, 0, st>>>(
             M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
@@ -307,6 +467,12 @@ dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pa
     const bool shape_ok = relu_of.hi ? (dx_lo && is_pair(relu_of)) : !dx_lo;
     if (shape_ok && tf32x3_supported(M, K, N, dy, W))
         return tf32x3_dgrad(M, N, K, dy, W, relu_of, dx, dx_lo, lddx, err, st);
+    if (N == 1 && relu_of.hi && dx_lo && !dy.lo) {
+        outer_mask_kernel<<<grid_stride_blocks((long long)M * K), 256, 0, st>>>(M, K, dy.hi, W.hi, W.lo, relu_of.hi,
+                                                                               relu_of.lo, relu_of.ld, dx, dx_lo, lddx);
+        DLRM_LAUNCH_CHECK();
+        return DLRM_OK;
+    }
     if (relu_of.hi)
         gemm_f32_kernel<false, true, EPI_MASK, false><<<grid_for(M, K, 1), 256, 0, st>>>(
             M, K, N, dy.hi, dy.lo, dy.ld, W.hi, W.lo, W.ld, nullptr, relu_of.hi, relu_of.lo, relu_of.ld, dx, dx_lo,
@@ -321,7 +487,7 @@ dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pa
 size_t train_wgrad_scratch_floats(int N, int K, int M) {
     const size_t simt = (size_t)simt_wgrad_splits(N, K, M) * (size_t)N * (size_t)(K + 1);
     const size_t tc = tf32x3_wgrad_scratch_floats(N, K, M);
-    const size_t cs = (size_t)colsum_chunks(M) * (size_t)N;
+    const size_t cs = (size_t)colsum_chunks(M) * (size_t)(N > K ? N : K) * CS_NW;
     return simt > tc ? (simt > cs ? simt : cs) : (tc > cs ? tc : cs);
 }
 
@@ -332,14 +498,17 @@ dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float
         dlrm_status r = tf32x3_wgrad(M, N, K, dy, x, dW, ldw, scratch, err, st);
         if (r) return r;
         // bias gradient: fixed-order column sums of dy (the split partials above are consumed by now)
-        const int P = colsum_chunks(M);
-        const long long rows_per = ((long long)M + P - 1) / P;
-        colsum_partial_kernel<<<dim3((unsigned)((N + 31) / 32), (unsigned)P), 256, 0, st>>>(M, N, dy.hi, dy.lo, dy.ld,
-                                                                                           rows_per, scratch);
-        DLRM_LAUNCH_CHECK();
-        colsum_final_kernel<<<(N + 255) / 256, 256, 0, st>>>(P, N, scratch, db);
-        DLRM_LAUNCH_CHECK();
-        return DLRM_OK;
+        return launch_colsum_w(M, N, dy, nullptr, 0, 0, true, nullptr, 0, db, scratch, st);
+    }
+    if (K < CS_NW && !x.lo) {
+        // narrow input (the 13 dense features): dW[n][k] and db[n] from one pass over dy
+        return launch_colsum_w(M, N, dy, x.hi, x.ld, K, true, dW, ldw, db, scratch, st);
+    }
+    if (N == 1 && !dy.lo) {
+        // one-column layer: dW[0][k] = sum_m x[m][k] dz[m], db[0] = sum_m dz[m]
+        dlrm_status r = launch_colsum_w(M, K, x, dy.hi, dy.ld, 1, false, dW, 1, nullptr, scratch, st);
+        if (r) return r;
+        return launch_colsum_w(M, 1, dy, nullptr, 0, 0, true, nullptr, 0, db, scratch, st);
     }
     const int splits = simt_wgrad_splits(N, K, M);
     long long chunk = ((long long)M + splits - 1) / splits;
