@@ -364,6 +364,117 @@ __global__ void piece_sum_kernel(int d, const long long* __restrict__ n_piece_de
     }
 }
 
+// Rows of 32 V floats, V per lane (d = 32, 64, 128): one 4/8/16-byte access per lane and row.
+template <int V>
+struct LaneVec {
+    float v[V];
+    __device__ __forceinline__ void load(const float* p) {
+        if constexpr (V == 4) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(p));
+            v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+        } else if constexpr (V == 2) {
+            const float2 t = __ldg(reinterpret_cast<const float2*>(p));
+            v[0] = t.x, v[1] = t.y;
+        } else {
+            v[0] = __ldg(p);
+        }
+    }
+    __device__ __forceinline__ void load_rw(const float* p) {
+        if constexpr (V == 4) {
+            const float4 t = *reinterpret_cast<const float4*>(p);
+            v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+        } else if constexpr (V == 2) {
+            const float2 t = *reinterpret_cast<const float2*>(p);
+            v[0] = t.x, v[1] = t.y;
+        } else {
+            v[0] = *p;
+        }
+    }
+    __device__ __forceinline__ void store(float* p) const {
+        if constexpr (V == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+        else if constexpr (V == 2) *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+        else *p = v[0];
+    }
+};
+
+// piece_sum_kernel for d = 32 V: the same sums in the same order, each occurrence's row read once by the
+// warp (16 bytes per lane at d = 128) with four rows in flight.
+template <int V>
+__global__ void piece_sum_vec_kernel(const long long* __restrict__ n_piece_dev, const int* __restrict__ piece_seg,
+                                     const long long* __restrict__ piece_base, const long long* __restrict__ seg_start,
+                                     const uint32_t* __restrict__ vals, const float* __restrict__ dE, int piece,
+                                     float* __restrict__ partial) {
+    constexpr int d = 32 * V;
+    const long long np = *n_piece_dev;
+    const int lane = threadIdx.x & 31;
+    const long long wstride = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long p = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < np; p += wstride) {
+        const int s = piece_seg[p];
+        const long long j = p - piece_base[s];
+        const long long beg = seg_start[s] + j * piece;
+        const long long end = beg + piece < seg_start[s + 1] ? beg + piece : seg_start[s + 1];
+        float acc[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = 0.f;
+        long long o = beg;
+        for (; o + 4 <= end; o += 4) {
+            LaneVec<V> r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) r[u].load(dE + (long long)vals[o + u] * d + V * lane);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] += r[u].v[e];
+        }
+        for (; o < end; ++o) {
+            LaneVec<V> r;
+            r.load(dE + (long long)vals[o] * d + V * lane);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] += r.v[e];
+        }
+        LaneVec<V> out;
+#pragma unroll
+        for (int e = 0; e < V; ++e) out.v[e] = acc[e];
+        out.store(partial + p * d + V * lane);
+    }
+}
+
+// seg_apply_kernel for d = 32 V (same sums, same order)
+template <int V>
+__global__ void seg_apply_vec_kernel(const long long* __restrict__ n_seg_dev, const long long* __restrict__ piece_base,
+                                     const uint32_t* __restrict__ seg_row, const float* __restrict__ partial, float lr,
+                                     float* __restrict__ table, float* __restrict__ grad_out) {
+    constexpr int d = 32 * V;
+    const long long ns = *n_seg_dev;
+    const int lane = threadIdx.x & 31;
+    const long long wstride = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long s = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < ns; s += wstride) {
+        float g[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) g[e] = 0.f;
+        for (long long p = piece_base[s]; p < piece_base[s + 1]; ++p) {
+            LaneVec<V> r;
+            r.load(partial + p * d + V * lane);
+#pragma unroll
+            for (int e = 0; e < V; ++e) g[e] += r.v[e];
+        }
+        if (table) {
+            float* w = table + (long long)seg_row[s] * d + V * lane;
+            LaneVec<V> t;
+            t.load_rw(w);
+#pragma unroll
+            for (int e = 0; e < V; ++e) t.v[e] -= lr * g[e];
+            t.store(w);
+        }
+        if (grad_out) {
+            LaneVec<V> o;
+#pragma unroll
+            for (int e = 0; e < V; ++e) o.v[e] = g[e];
+            o.store(grad_out + s * d + V * lane);
+        }
+    }
+}
+
 // One warp per segment: g = sum of its piece partials in order; T[row] -= lr * g if table is given,
 // and g is written to grad_out[s] if given.
 __global__ void seg_apply_kernel(int d, const long long* __restrict__ n_seg_dev, const long long* __restrict__ piece_base,
@@ -562,11 +673,29 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
     const int* piece_seg = reinterpret_cast<const int*>(base + L.piece_seg);
     float* partial = const_cast<float*>(reinterpret_cast<const float*>(base + L.partial));
     const int blocks = 148 * 8;
-    piece_sum_kernel<<<blocks, 256, 0, st>>>(d, &counts[3], piece_seg, piece_base, seg_start, vals, dE, SPARSE_PIECE,
-                                             partial);
+    // the vector kernels need d = 32, 64 or 128 and 16-byte aligned rows everywhere (dE, partials and the
+    // table are aligned by construction; a caller's grad_out may not be)
+    const bool vec = (d == 32 || d == 64 || d == 128) && (((uintptr_t)grad_out & 15) == 0);
+#define DLRM_SPARSE_VEC(V)                                                                                        \
+    piece_sum_vec_kernel<V><<<blocks, 256, 0, st>>>(&counts[3], piece_seg, piece_base, seg_start, vals, dE,        \
+                                                    SPARSE_PIECE, partial);                                         \
+    DLRM_LAUNCH_CHECK();                                                                                          \
+    seg_apply_vec_kernel<V><<<blocks, 256, 0, st>>>(&counts[2], piece_base, seg_row, partial, lr, table, grad_out); \
     DLRM_LAUNCH_CHECK();
-    seg_apply_kernel<<<blocks, 256, 0, st>>>(d, &counts[2], piece_base, seg_row, partial, lr, table, grad_out);
-    DLRM_LAUNCH_CHECK();
+    if (vec && d == 128) {
+        DLRM_SPARSE_VEC(4)
+    } else if (vec && d == 64) {
+        DLRM_SPARSE_VEC(2)
+    } else if (vec && d == 32) {
+        DLRM_SPARSE_VEC(1)
+    } else {
+        piece_sum_kernel<<<blocks, 256, 0, st>>>(d, &counts[3], piece_seg, piece_base, seg_start, vals, dE,
+                                                 SPARSE_PIECE, partial);
+        DLRM_LAUNCH_CHECK();
+        seg_apply_kernel<<<blocks, 256, 0, st>>>(d, &counts[2], piece_base, seg_row, partial, lr, table, grad_out);
+        DLRM_LAUNCH_CHECK();
+    }
+#undef DLRM_SPARSE_VEC
     if (rows_out) {
         cudaMemcpyAsync(rows_out, seg_row, sizeof(uint32_t) * L.cap, cudaMemcpyDeviceToDevice, st);
     }

@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const
     for (int e = 0; e < 4; ++e)
 #pragma unroll
         for (int q = 0; q < NW; ++q) acc[e][q] = 0.f;
+#pragma unroll 4
     for (long long r = rb + w; r < re; r += WARPS) {
         float v[4];
         if (vec) {
@@ -262,49 +263,71 @@ __global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const
     }
 }
 
-// out(c, w) = sum_p part[p][c][w] in increasing p; w < kx -> dW[c * ldw + w], w == kx -> db[c]
+// out(c, w) = sum over p of part[p][c][w], one warp per output: lane l adds p = l, l + 32, ... in order,
+// then a fixed butterfly across lanes; w < kx -> dW[c * ldw + w], w == kx -> db[c]
 __global__ void colsum_w_final_kernel(int P, int N, int NW, int kx, bool ones, const float* __restrict__ part,
                                       float* __restrict__ dW, long long ldw, float* __restrict__ db) {
     const long long n = (long long)N * NW;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long i = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n; i += warps) {
         const int c = (int)(i / NW), q = (int)(i % NW);
-        if (q > kx || (q == kx && !ones)) continue;
+        if (q > kx || (q == kx && !ones)) continue;   // uniform across the warp
         float s = 0.f;
-        for (int p = 0; p < P; ++p) s += part[(long long)p * n + i];
-        if (q < kx) dW[c * ldw + q] = s;
-        else db[c] = s;
+        for (int p = lane; p < P; p += 32) s += part[(long long)p * n + i];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) {
+            if (q < kx) dW[c * ldw + q] = s;
+            else db[c] = s;
+        }
     }
 }
 
-// y[b][n] = act(sum_{k < K} x(b, k) W[n][k] + bias[n]) for K <= 16 (the 13 dense features), one thread
-// per output column with its weight row in registers; y written as a pair or plain.
+// y[b][n] = act(sum_{k < K} x(b, k) W[n][k] + bias[n]) for K <= 16 (the 13 dense features): one thread
+// per output column with its weight row in registers; the block's rows of x are staged in shared memory
+// (read there as broadcasts), four rows per step; y written as a pair or plain.
+constexpr int NARROW_ROWS = 256;
 __global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int K, const float* __restrict__ xh,
                                                          const float* __restrict__ xl, long long ldx,
                                                          const float* __restrict__ W, const float* __restrict__ Wl,
                                                          long long ldw, const float* __restrict__ bias, bool relu,
-                                                         float* __restrict__ yh, float* __restrict__ yl, long long ldy,
-                                                         long long rows_per) {
+                                                         float* __restrict__ yh, float* __restrict__ yl, long long ldy) {
+    __shared__ float xs[NARROW_ROWS][17];
+    const long long rb = (long long)blockIdx.y * NARROW_ROWS;
+    const int nr = (int)(M - rb < NARROW_ROWS ? M - rb : NARROW_ROWS);
+    for (int q = threadIdx.x; q < nr * K; q += blockDim.x) {
+        const int r = q / K, k = q - r * K;
+        const long long g = (rb + r) * ldx + k;
+        xs[r][k] = xl ? xh[g] + xl[g] : xh[g];
+    }
+    __syncthreads();
     const int n = blockIdx.x * 128 + threadIdx.x;
     if (n >= N) return;
     float wr[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) wr[k] = k < K ? (Wl ? W[n * ldw + k] + Wl[n * ldw + k] : W[n * ldw + k]) : 0.f;
     const float bn = bias[n];
-    const long long rb = (long long)blockIdx.y * rows_per;
-    const long long re = rb + rows_per < M ? rb + rows_per : M;
-    for (long long b = rb; b < re; ++b) {
-        float s = 0.f;
+    for (int r0 = 0; r0 < nr; r0 += 4) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-            if (k < K) s = fmaf(xl ? __ldg(xh + b * ldx + k) + __ldg(xl + b * ldx + k) : __ldg(xh + b * ldx + k), wr[k], s);
-        s += bn;
-        if (relu) s = s > 0.f ? s : 0.f;
-        if (yl) {
-            const float h = tf32_hi_part(s);
-            yh[b * ldy + n] = h;
-            yl[b * ldy + n] = s - h;
-        } else {
-            yh[b * ldy + n] = s;
+            if (k < K)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) s[u] = fmaf(xs[r0 + u < nr ? r0 + u : r0][k], wr[k], s[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (r0 + u >= nr) break;
+            float v = s[u] + bn;
+            if (relu) v = v > 0.f ? v : 0.f;
+            const long long o = (rb + r0 + u) * ldy + n;
+            if (yl) {
+                const float h = tf32_hi_part(v);
+                yh[o] = h;
+                yl[o] = v - h;
+            } else {
+                yh[o] = v;
+            }
         }
     }
 }
@@ -425,8 +448,9 @@ dlrm_status launch_colsum_w(int M, int N, F32Pair A, const float* X, int ldx, in
         NW = CS_NW;
     }
     DLRM_LAUNCH_CHECK();
-    colsum_w_final_kernel<<<grid_stride_blocks((long long)N * NW), 256, 0, st>>>(P, N, NW, kx, ones, scratch, dW, ldw,
-                                                                               db);
+    const long long outs = (long long)N * NW;
+    colsum_w_final_kernel<<<(int)((outs + 7) / 8 < 148 * 16 ? (outs + 7) / 8 : 148 * 16), 256, 0, st>>>(
+        P, N, NW, kx, ones, scratch, dW, ldw, db);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -437,10 +461,8 @@ dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const fl
     if (relu && y_lo && tf32x3_supported(M, N, K, x, W))
         return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, err, st);
     if (K <= 16) {
-        const long long rows_per = 256;
-        const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + rows_per - 1) / rows_per));
-        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy,
-                                                rows_per);
+        const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + NARROW_ROWS - 1) / NARROW_ROWS));
+        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy);
         DLRM_LAUNCH_CHECK();
         return DLRM_OK;
     }
