@@ -225,7 +225,6 @@ __global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const
     for (int e = 0; e < 4; ++e)
 #pragma unroll
         for (int q = 0; q < NW; ++q) acc[e][q] = 0.f;
-#pragma unroll 4
     for (long long r = rb + w; r < re; r += WARPS) {
         float v[4];
         if (vec) {
