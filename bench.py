@@ -48,17 +48,29 @@ POOL = 8
 
 def workload_desc(cfg) -> str:
     rows = f"{min(cfg.rows)}..{max(cfg.rows)} rows" if len(set(cfg.rows)) > 1 else f"{cfg.rows[0]} rows each"
-    tb = sum(cfg.rows) * cfg.d * (4 if cfg.table_dtype == "f32" else 2) / 1e9
+    tb = sum(cfg.rows) * table_row_bytes(cfg) / 1e9
     return (f"{cfg.name}: B={cfg.B}, K={cfg.K} tables ({rows}, {tb:.1f} GB {cfg.table_dtype}), d={cfg.d}, "
             f"bags={cfg.bag}, indices={cfg.index}, bottom={'-'.join(map(str, cfg.bottom))}, "
             f"top={'-'.join(map(str, cfg.top))}")
 
 
+def table_row_bytes(cfg) -> int:
+    """Bytes of one stored table row (row-wise 8-bit: d codes + fp32 scale and offset, padded to 16)."""
+    if cfg.table_dtype == "u8row":
+        return (cfg.d + 8 + 15) // 16 * 16
+    return cfg.d * (4 if cfg.table_dtype == "f32" else 2)
+
+
+def quantizer():
+    """The library's row-wise 8-bit quantiser, for building uint8 tables on the device."""
+    import embedding_bags_dot_b200 as E
+    return lambda src, dst: E.dlrm_quantize_rows_u8(src, dst)
+
+
 def algorithmic_bytes(cfg, batch) -> int:
     """Bytes the fused gather + interaction must move for one batch."""
-    es_t = 4 if cfg.table_dtype == "f32" else 2
     es_o = 4 if cfg.mlp_dtype == "f32" else 2
-    rows = int(batch.indices.size) * cfg.d * es_t
+    rows = int(batch.indices.size) * table_row_bytes(cfg)
     return rows + 4 * batch.indices.size + 4 * (cfg.K * cfg.B + 1) + 4 * cfg.B * cfg.d + es_o * cfg.B * cfg.concat_width
 
 
@@ -230,7 +242,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     sd.build_fill()
 
     # model
-    tables = sd.tables_on_device(cfg, device=dev)
+    tables = sd.tables_on_device(cfg, device=dev, quantize=quantizer())
     T = E.Tables(tables, cfg.rows, cfg.d)
     bW, bb, bd = sd.mlp_on_device(cfg, "bottom", dev)
     tW, tb, td = sd.mlp_on_device(cfg, "top", dev)
@@ -363,11 +375,12 @@ def run_ours(args, cfg, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.table_dtype, "data": "synthetic",
             "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world, "per_gpu_batch": cfg.B,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": f"no flush: tables {sum(cfg.rows) * cfg.d * (4 if cfg.table_dtype == 'f32' else 2) / 1e9:.1f} GB "
+                       "l2": f"no flush: tables {sum(cfg.rows) * table_row_bytes(cfg) / 1e9:.1f} GB "
                              f"and a {POOL}-batch pool of {pool_bytes / 1e6:.0f} MB exceed the {L2_BYTES >> 20} MB L2"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
                          "frac": achieved / peak_hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)" if cfg.table_dtype == "bf16"
+                         "kernel": "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
+                                   if cfg.table_dtype in ("bf16", "u8row")
                                    else "embbag_interact_kernel (dlrm_embbag_interact_fwd)",
                          "algorithmic_bytes_per_launch": avg_algo, "avg_launch_ms": k2_avg},
             "kernels_ms_per_step": {"bottom_mlp": float(np.mean(bot_ms)), "embbag_interact": float(np.mean(k2_ms)),
@@ -396,7 +409,7 @@ def run_train(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     E.lib()
     sd.build_fill()
-    tables = sd.tables_on_device(cfg, device=dev)
+    tables = sd.tables_on_device(cfg, device=dev, quantize=quantizer())
     T = E.Tables(tables, cfg.rows, cfg.d)
     bot = E.MLP(*sd.mlp_on_device(cfg, "bottom", dev))
     top = E.MLP(*sd.mlp_on_device(cfg, "top", dev))
@@ -520,7 +533,7 @@ def run_latency(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     E.lib()
     sd.build_fill()
-    T = E.Tables(sd.tables_on_device(cfg, device=dev), cfg.rows, cfg.d)
+    T = E.Tables(sd.tables_on_device(cfg, device=dev, quantize=quantizer()), cfg.rows, cfg.d)
     bot = E.MLP(*sd.mlp_on_device(cfg, "bottom", dev))
     top = E.MLP(*sd.mlp_on_device(cfg, "top", dev))
     perms = {k: gen.table_permutation(cfg, k) for k in range(cfg.K)} if cfg.index.startswith("zipf") else None
@@ -544,7 +557,36 @@ def run_latency(args, cfg, rank, world, local_rank):
             ms.append(e0.elapsed_time(e1))
         ms.sort()
         med, p99 = ms[len(ms) // 2], ms[min(len(ms) - 1, int(0.99 * len(ms)))]
-        rows.append({"batch": B, "latency_ms_p50": med, "latency_ms_p99": p99, "samples_per_s": B / (med * 1e-3)})
+        row = {"batch": B, "latency_ms_p50": med, "latency_ms_p99": p99, "samples_per_s": B / (med * 1e-3)}
+        # the same forward captured once in a CUDA graph and replayed: no per-call host work (argument checks,
+        # tensor-map encoding, launches) between the events
+        try:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(st)
+            with torch.cuda.stream(side):
+                E.dlrm_forward(T, bot, top, B, bt["dense"], bt["offsets"], bt["indices"], y, ws, side)
+            torch.cuda.synchronize(dev)
+            with torch.cuda.graph(g):
+                cs = torch.cuda.current_stream(dev)
+                E.dlrm_forward(T, bot, top, B, bt["dense"], bt["offsets"], bt["indices"], y, ws, cs)
+            for _ in range(args.warmup):
+                g.replay()
+            gms = []
+            for _ in range(max(args.steps, 20)):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+                e1.synchronize()
+                gms.append(e0.elapsed_time(e1))
+            gms.sort()
+            row["graph_latency_ms_p50"] = gms[len(gms) // 2]
+            row["graph_latency_ms_p99"] = gms[min(len(gms) - 1, int(0.99 * len(gms)))]
+            del g
+        except Exception as exc:  # report, keep the eager numbers
+            row["graph_error"] = str(exc)[:200]
+        rows.append(row)
     # co-location: S streams, each serving its own small batches
     coloc = []
     Bc = min(256, cfg.B)

@@ -26,7 +26,9 @@ MAX_LAYERS = 16
 ERR_RECORD_BYTES = 256
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
-DT_CODE = {"f32": F32, "f16": F16, "bf16": BF16, torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+U8ROW = 3   # row-wise 8-bit table records (tables only)
+DT_CODE = {"f32": F32, "f16": F16, "bf16": BF16, "u8row": U8ROW, torch.float32: F32, torch.float16: F16,
+           torch.bfloat16: BF16, torch.uint8: U8ROW}
 DT_TORCH = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
 
 
@@ -76,6 +78,8 @@ _SIGS = {
     "dlrm_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
+    "dlrm_row_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "dlrm_quantize_rows_u8": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
                                 C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     "dlrm_tf32_split": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int,
@@ -142,7 +146,8 @@ def dlrm_ld(n: int, dt) -> int:
 # ----------------------------------------------------------------- model containers
 
 class Tables:
-    """K tables in one contiguous device buffer ([sum rows][d]) plus host row counts."""
+    """K tables in one contiguous device buffer ([sum rows][d], or [sum rows][record bytes] uint8 for
+    row-wise 8-bit tables) plus host row counts."""
 
     def __init__(self, data: torch.Tensor, rows, d: int):
         assert data.is_cuda and data.is_contiguous()
@@ -235,6 +240,18 @@ def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, 
     return _check(lib().dlrm_forward_noalloc(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                              _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(err_flags),
                                              _stream(stream)), "dlrm_forward_noalloc")
+
+
+def dlrm_row_bytes(d: int, dt) -> int:
+    return int(lib().dlrm_row_bytes(int(d), DT_CODE.get(dt, dt)))
+
+
+def dlrm_quantize_rows_u8(src, dst, stream=None):
+    """Row-wise 8-bit records dst (uint8 [rows][dlrm_row_bytes(d, U8ROW)]) from src (fp32 or bf16 [rows][d])."""
+    rows, d = src.shape
+    assert dst.dtype == torch.uint8 and dst.shape[0] == rows and dst.shape[1] == dlrm_row_bytes(d, U8ROW)
+    return _check(lib().dlrm_quantize_rows_u8(_ptr(src), DT_CODE[src.dtype], int(rows), int(d), _ptr(dst),
+                                              _stream(stream)), "dlrm_quantize_rows_u8")
 
 
 # ----------------------------------------------------------------- fp32 GEMM (tensor cores, 3xTF32)

@@ -20,11 +20,12 @@ namespace {
 
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline bool valid_dt(int dt) { return dt == DLRM_F32 || dt == DLRM_F16 || dt == DLRM_BF16; }
+inline bool valid_table_dt(int dt) { return valid_dt(dt) || dt == DLRM_U8ROW; }
 inline cudaStream_t cs(dlrm_stream s) { return reinterpret_cast<cudaStream_t>(s); }
 
 dlrm_status check_tables(const dlrm_tables* T, TableMeta& tm) {
     if (!T || !T->rows || !T->data) return DLRM_ERR_INVALID_ARG;
-    if (T->K < 1 || T->d < 1 || !valid_dt(T->dt)) return DLRM_ERR_INVALID_ARG;
+    if (T->K < 1 || T->d < 1 || !valid_table_dt(T->dt)) return DLRM_ERR_INVALID_ARG;
     if (T->K > DLRM_MAX_TABLES) return DLRM_ERR_UNSUPPORTED;
     if (!aligned16(T->data)) return DLRM_ERR_INVALID_ARG;
     long long acc = 0;
@@ -34,7 +35,8 @@ dlrm_status check_tables(const dlrm_tables* T, TableMeta& tm) {
         tm.rows[k] = T->rows[k];
         acc += T->rows[k];
     }
-    if (!gather_supported(T->d, T->dt)) return DLRM_ERR_UNSUPPORTED;
+    // uint8 records are read by the fused tensor-core kernel only (d = 64, 128)
+    if (T->dt == DLRM_U8ROW ? !(T->d == 64 || T->d == 128) : !gather_supported(T->d, T->dt)) return DLRM_ERR_UNSUPPORTED;
     return DLRM_OK;
 }
 

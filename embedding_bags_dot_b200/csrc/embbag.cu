@@ -353,6 +353,7 @@ static bool gather_geometry(int d, dlrm_dtype dt, Geometry& g) {
 }
 
 bool gather_supported(int d, dlrm_dtype dt) {
+    if (dt == DLRM_U8ROW) return false;   // only the fused tensor-core kernel reads uint8 records
     Geometry g;
     return gather_geometry(d, dt, g);
 }
@@ -396,7 +397,7 @@ dlrm_status launch_embbag(const TableMeta& tm, const void* tables, dlrm_dtype dt
                           const int32_t* offsets, const int32_t* indices, long long nnz, float* pooled,
                           int32_t* bag_len, ErrRecord* err, cudaStream_t st) {
     Geometry g;
-    if (!gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
+    if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     if ((size_t)sizeof(int) * K * 33 + (size_t)K * 32 > kSmemMax) return DLRM_ERR_UNSUPPORTED;
     switch (dt) {
         case DLRM_F32: return launch_embbag_t<float>(tm, tables, K, d, B, offsets, indices, nnz, pooled, bag_len, err, st, g);
@@ -455,10 +456,11 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                    const int32_t* offsets, const int32_t* indices, long long nnz,
                                    const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                    cudaStream_t st) {
-    Geometry g;
-    if (!gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt, tm.base[K - 1] + tm.rows[K - 1]))
-        return launch_embbag_interact_mma(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st);
+        return launch_embbag_interact_mma(tm, tables, dt, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt,
+                                          err, st);
+    Geometry g;
+    if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     switch (dt) {
         case DLRM_F32: return launch_fused_t<float>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
         case DLRM_BF16: return launch_fused_t<__nv_bfloat16>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);

@@ -1,4 +1,4 @@
-// Fused gather + interaction for bf16 tables on the tensor cores.
+// Fused gather + interaction for bf16 or row-wise uint8 tables on the tensor cores.
 //
 // Same operation as embbag.cu's fused kernel: per sample b, pool the K bags
 // into e_1..e_K ("DLRM", briansu.co, section 3), form X = [x_dense; e_1..e_K]
@@ -13,6 +13,11 @@
 //     row per lane. A one-row bag is copied global -> shared with cp.async,
 //     so every row of the sample is in flight at once without registers;
 //     a bag of several rows is summed in fp32 and rounded to bf16.
+//     Row-wise uint8 tables (Q): a one-row bag's record (d codes, fp32 scale,
+//     fp32 offset) is copied the same way, unswizzled, into the first bytes of
+//     its X row slot; once it has landed each lane reads its 8 codes and the
+//     scale/offset, the warp synchronises, and the lane writes the dequantised
+//     values (s q + m, rounded to bf16) as its swizzled 16-byte chunk.
 //  2. x_dense (fp32) is split into hi = bf16(x) and lo = bf16(x - hi); hi is
 //     row 0 of X and lo row K+1, so that Z_i0 = G[i][0] + G[K+1][i] keeps the
 //     dense vector's fp32 precision.
@@ -76,10 +81,19 @@ __device__ __forceinline__ uint32_t column_source(int c, int d, int P, int GS, u
 
 }  // namespace
 
-// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2). GL: lanes per row (d = 8 GL).
-template <int MT, int GL>
+// Dequantise 8 codes of a DLRM_U8ROW record: v = s q + m.
+__device__ __forceinline__ void dequant8(uint2 codes, float sc, float of, float (&v)[8]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        v[e] = fmaf(sc, (float)((codes.x >> (8 * e)) & 0xFFu), of);
+        v[4 + e] = fmaf(sc, (float)((codes.y >> (8 * e)) & 0xFFu), of);
+    }
+}
+
+// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2). GL: lanes per row (d = 8 GL). Q: row-wise uint8 tables.
+template <int MT, int GL, bool Q>
 __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_mma_kernel(
-    const __nv_bfloat16* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B,
+    const void* __restrict__ tables_v, const __grid_constant__ TableMeta tm, int K, int B,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, int warp_bytes, ErrRecord* err) {
     constexpr int d = 8 * GL;
@@ -91,6 +105,9 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     constexpr int GS = KP + 8;       // G row stride in floats (float2 staging without bank conflicts)
     constexpr int NG = 32 / GL;      // row groups per warp
     constexpr int NTILE = MT * (MT + 1);
+    constexpr int QRB = (d + 8 + 15) / 16 * 16;   // uint8 record bytes
+    const __nv_bfloat16* __restrict__ tables = static_cast<const __nv_bfloat16*>(tables_v);
+    const unsigned char* __restrict__ qtab = static_cast<const unsigned char*>(tables_v);
     // byte offset of 16-byte chunk c of X row r
     auto xoff = [](int r, int c) { return r * RS + 16 * (SWZ ? (c ^ (r & 7)) : c); };
     extern __shared__ __align__(16) unsigned char smem[];
@@ -169,7 +186,12 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
             const uint32_t code = code_s[k * S + s];
             const uint32_t dst = xw_s + (uint32_t)xoff(k + 1, g);
             if (code < CODE_MULTI) {
-                cp_async16(dst, tables + (long long)code * d + 8 * g);
+                if constexpr (Q) {
+                    if (16 * g < QRB)
+                        cp_async16(xw_s + (uint32_t)((k + 1) * RS + 16 * g), qtab + (long long)code * QRB + 16 * g);
+                } else {
+                    cp_async16(dst, tables + (long long)code * d + 8 * g);
+                }
             } else if (code == CODE_EMPTY) {
                 *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) = make_uint4(0, 0, 0, 0);
             } else {
@@ -177,10 +199,22 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                 float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int p = st; p < en; ++p) {
                     const int idx = __ldg(indices + p);
-                    if (idx >= 0 && (long long)idx < tm.rows[k])
-                        Chunk16<__nv_bfloat16>::add(ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g), a);
-                    else if (g == 0)
+                    if (idx >= 0 && (long long)idx < tm.rows[k]) {
+                        if constexpr (Q) {
+                            const unsigned char* rec = qtab + (tm.base[k] + idx) * (long long)QRB;
+                            const uint2 cq = __ldg(reinterpret_cast<const uint2*>(rec + 8 * g));
+                            const float2 so = __ldg(reinterpret_cast<const float2*>(rec + d));
+                            float v[8];
+                            dequant8(cq, so.x, so.y, v);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) a[e] += v[e];
+                        } else {
+                            Chunk16<__nv_bfloat16>::add(ldg16_stream(tables + (tm.base[k] + idx) * (long long)d + 8 * g),
+                                                        a);
+                        }
+                    } else if (g == 0) {
                         ++oob;
+                    }
                 }
                 *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) =
                     make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
@@ -206,6 +240,26 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         }
         cp_async_wait_all();
         __syncwarp();
+        if constexpr (Q) {
+            // one-row bags: staged records -> dequantised bf16 rows, in place (every lane reads before any writes)
+            for (int kk = 0; kk < (K + NG - 1) / NG; ++kk) {
+                const int k = kk * NG + gi;
+                const bool one = k < K && code_s[k * S + s] < CODE_MULTI;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if (one) {
+                    const unsigned char* rec = xw + (size_t)(k + 1) * RS;
+                    const uint2 cq = *reinterpret_cast<const uint2*>(rec + 8 * g);
+                    const float2 so = *reinterpret_cast<const float2*>(rec + d);
+                    float v[8];
+                    dequant8(cq, so.x, so.y, v);
+                    w = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                   pack_bf16(v[6], v[7]));
+                }
+                __syncwarp();
+                if (one) *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) = w;
+            }
+            __syncwarp();
+        }
 
         // ---- 3. lower-triangle Gram tiles on the tensor cores
         float acc[NTILE][4];
@@ -302,8 +356,9 @@ static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
 
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
                                    long long total_rows) {
-    if (dt != DLRM_BF16) return false;
+    if (dt != DLRM_BF16 && dt != DLRM_U8ROW) return false;
     if (!(d == 32 || d == 64 || d == 128 || d == 256)) return false;
+    if (dt == DLRM_U8ROW && !(d == 64 || d == 128)) return false;
     if (K + 2 > 64) return false;
     if (total_rows >= (long long)CODE_MULTI) return false;
     if (out_dt == DLRM_BF16 && (ld % 8 || ((uintptr_t)out & 15))) return false;
@@ -314,28 +369,35 @@ bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const vo
     return mma_smem(K, d, ld, MT, wb) <= 227 * 1024;
 }
 
-template <int MT, int GL>
+template <int MT, int GL, bool Q>
 static void launch_mma_t(const TableMeta& tm, const void* tables, int K, int B, const int32_t* offsets,
                          const int32_t* indices, long long nnz, const float* x_dense, void* out, int ld, int out_dt,
                          int warp_bytes, size_t smem, ErrRecord* err, cudaStream_t st) {
-    auto kern = embbag_interact_mma_kernel<MT, GL>;
+    auto kern = embbag_interact_mma_kernel<MT, GL, Q>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<(B + S - 1) / S, WARPS * 32, smem, st>>>(static_cast<const __nv_bfloat16*>(tables), tm, K, B, offsets,
-                                                    indices, nnz, x_dense, out, ld, out_dt, warp_bytes, err);
+    kern<<<(B + S - 1) / S, WARPS * 32, smem, st>>>(tables, tm, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt,
+                                                    warp_bytes, err);
 }
 
-dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, int K, int d, int B,
+dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st) {
     int MT, wb;
     const size_t smem = mma_smem(K, d, ld, MT, wb);
+    const bool q = dt == DLRM_U8ROW;
 #define DLRM_MMA_GL(MTV)                                                                                       \
     switch (d) {                                                                                               \
-        case 32: launch_mma_t<MTV, 4>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \
-        case 64: launch_mma_t<MTV, 8>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \
-        case 128: launch_mma_t<MTV, 16>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break; \
-        default: launch_mma_t<MTV, 32>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;  \
+        case 32: launch_mma_t<MTV, 4, false>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \
+        case 64:                                                                                               \
+            if (q) launch_mma_t<MTV, 8, true>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st);  \
+            else launch_mma_t<MTV, 8, false>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); \
+            break;                                                                                             \
+        case 128:                                                                                              \
+            if (q) launch_mma_t<MTV, 16, true>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); \
+            else launch_mma_t<MTV, 16, false>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); \
+            break;                                                                                             \
+        default: launch_mma_t<MTV, 32, false>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;  \
     }
     switch (MT) {
         case 1: DLRM_MMA_GL(1) break;

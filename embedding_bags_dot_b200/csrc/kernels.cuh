@@ -24,7 +24,7 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
 // d in {32, 64, 128, 256} and K + 2 <= 64; launch_embbag_interact picks it when supported.
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
                                    long long total_rows);
-dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, int K, int d, int B,
+dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st);
@@ -46,6 +46,9 @@ bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, in
 dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st);
+
+// DLRM_U8ROW record bytes of a row of width d (quant.cu)
+size_t u8row_bytes(int d);
 
 // ---- training (fp32)
 // An fp32 matrix row-major with leading dimension ld, held either plain

@@ -25,7 +25,13 @@
  *   - backward and SGD: the pages state none; the gradients below are the
  *     calculus of the forward definition, and SGD is w <- w - lr * grad.
  *
- * Arithmetic is fp64 throughout. Inputs arrive already widened to fp64
+ *   - row-wise 8-bit tables (the storage the fused gather path also reads):
+ *     the pages fix no format; the reading used is the min/max affine form
+ *     per row, computed in fp32 exactly as the library's quantiser specifies
+ *     (so both sides take the same integer decisions), and dequantised here
+ *     in fp64 as s q + m.
+ *
+ * Arithmetic is fp64 throughout (except the quantiser's fp32 codes). Inputs arrive already widened to fp64
  * (exactly) by the caller. Weights are [out][in] row-major with no padding.
  * Invalid indices (outside [0, m_k)) are skipped and counted; a bag whose
  * offsets are decreasing or outside [0, nnz] pools to zero and is counted.
@@ -582,4 +588,36 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
 /* Plain SGD: w <- w - lr * g, elementwise. */
 void oracle_sgd(int64_t n, double lr, double* w, const double* g) {
     for (int64_t q = 0; q < n; ++q) w[q] -= lr * g[q];
+}
+
+/* Row-wise 8-bit quantisation of fp32 rows (the DLRM_U8ROW storage). Per row,
+ * in fp32 with round-to-nearest: lo = min, hi = max, s = (hi - lo) / 255,
+ * q = rint((v - lo) / s) clamped to [0, 255] (q = 0 when s = 0), m = lo. */
+void oracle_quantize_rows_u8(int64_t rows, int d, const float* src, unsigned char* codes, float* scale,
+                             float* offset) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* v = src + r * d;
+        float lo = INFINITY, hi = -INFINITY;
+        for (int c = 0; c < d; ++c) {
+            lo = fminf(lo, v[c]);
+            hi = fmaxf(hi, v[c]);
+        }
+        const float s = (hi - lo) / 255.0f;
+        for (int c = 0; c < d; ++c) {
+            float q = 0.0f;
+            if (s > 0.0f) q = rintf((v[c] - lo) / s);
+            if (q < 0.0f) q = 0.0f;
+            if (q > 255.0f) q = 255.0f;
+            codes[r * d + c] = (unsigned char)q;
+        }
+        scale[r] = s;
+        offset[r] = lo;
+    }
+}
+
+/* Value of every entry of row-wise 8-bit rows: s * q + m, in fp64 (exact for fp32 s, m and 8-bit q). */
+void oracle_dequantize_rows_u8(int64_t rows, int d, const unsigned char* codes, const float* scale,
+                               const float* offset, double* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int c = 0; c < d; ++c) out[r * d + c] = (double)scale[r] * (double)codes[r * d + c] + (double)offset[r];
 }

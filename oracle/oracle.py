@@ -68,6 +68,8 @@ def _declare(lib):
     lib.oracle_train_grads.argtypes = [vp, i, l, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, vp, vp, vp, vp]
     lib.oracle_sgd.argtypes = [C.c_int64, d, vp, vp]
+    lib.oracle_quantize_rows_u8.argtypes = [C.c_int64, i, vp, vp, vp, vp]
+    lib.oracle_dequantize_rows_u8.argtypes = [C.c_int64, i, vp, vp, vp, vp]
     return lib
 
 
@@ -186,7 +188,7 @@ def model_from_config(cfg: Config, tables_stored: np.ndarray | None = None, rows
     bW, bb = layers_f64(bot, cfg.mlp_dtype)
     tW, tb = layers_f64(top, cfg.mlp_dtype)
     rows = np.asarray(cfg.rows if rows is None else rows, np.int64)
-    return Model(rows, cfg.d, gen.to_f64(tables_stored, cfg.table_dtype).reshape(-1, cfg.d), bW, bb, tW, tb)
+    return Model(rows, cfg.d, table_values(tables_stored, cfg.table_dtype).reshape(-1, cfg.d), bW, bb, tW, tb)
 
 
 def sub_batch(cfg: Config, batch: gen.Batch, samples: np.ndarray):
@@ -277,6 +279,50 @@ def train_grads(model: Model, dense, offsets, indices, labels, lib=None, scales:
     out.update({"loss": float(loss[0]), "y_hat": y, "bot_dW": bdW, "bot_db": bdb, "top_dW": tdW, "top_db": tdb,
                 "table_grad": tg, "row_count": cnt, "counts": (int(counts[0]), int(counts[1]))})
     return out
+
+
+def quantize_rows_u8(rows_f32: np.ndarray, lib=None):
+    """Row-wise 8-bit quantisation of fp32 rows [n][d]: (codes uint8 [n][d], scale fp32 [n], offset fp32 [n])."""
+    lib = lib or load()
+    v = np.ascontiguousarray(rows_f32, dtype=np.float32)
+    n, d = v.shape
+    codes = np.zeros((n, d), np.uint8)
+    scale = np.zeros(n, np.float32)
+    offset = np.zeros(n, np.float32)
+    if n:
+        lib.oracle_quantize_rows_u8(n, d, _p(v), _p(codes), _p(scale), _p(offset))
+    return codes, scale, offset
+
+
+def dequantize_rows_u8(codes: np.ndarray, scale: np.ndarray, offset: np.ndarray, lib=None) -> np.ndarray:
+    """fp64 values s * q + m of row-wise 8-bit rows."""
+    lib = lib or load()
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    n, d = codes.shape
+    out = np.zeros((n, d), np.float64)
+    if n:
+        lib.oracle_dequantize_rows_u8(n, d, _p(codes), _p(np.ascontiguousarray(scale, np.float32)),
+                                      _p(np.ascontiguousarray(offset, np.float32)), _p(out))
+    return out
+
+
+def u8_records(codes: np.ndarray, scale: np.ndarray, offset: np.ndarray) -> np.ndarray:
+    """The DLRM_U8ROW byte records [n][round_up(d + 8, 16)]: codes, fp32 scale, fp32 offset, zero padding."""
+    n, d = codes.shape
+    rb = (d + 8 + 15) // 16 * 16
+    rec = np.zeros((n, rb), np.uint8)
+    rec[:, :d] = codes
+    rec[:, d:d + 4] = np.ascontiguousarray(scale, np.float32).view(np.uint8).reshape(n, 4)
+    rec[:, d + 4:d + 8] = np.ascontiguousarray(offset, np.float32).view(np.uint8).reshape(n, 4)
+    return rec
+
+
+def table_values(stored: np.ndarray, dtype: str) -> np.ndarray:
+    """fp64 values of stored table rows; row-wise 8-bit tables are stored as their fp32 source rows
+    and quantised here."""
+    if dtype == "u8row":
+        return dequantize_rows_u8(*quantize_rows_u8(np.asarray(stored, np.float32)))
+    return gen.to_f64(stored, dtype)
 
 
 def sgd(w: np.ndarray, g: np.ndarray, lr: float, lib=None) -> np.ndarray:

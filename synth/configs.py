@@ -32,7 +32,7 @@ class Config:
     B: int                      # batch size (samples)
     rows: tuple                 # m_k, one per table
     d: int                      # shared embedding width
-    table_dtype: str            # "f32" | "f16" | "bf16"
+    table_dtype: str            # "f32" | "f16" | "bf16" | "u8row" (row-wise 8-bit: fp32 source rows, quantised by the user)
     mlp_dtype: str              # dtype of MLP weights and hidden activations
     bag: str                    # "one" | "poisson20" | "uniform100" | "fixed:<n>" | "mix"
     index: str                  # "uniform" | "zipf:<alpha>"
@@ -100,6 +100,10 @@ CONFIGS = {
     "train": Config("train", B=65536, rows=tuple(r // 4 for r in LARGE_ROWS), d=128, table_dtype="f32",
                     mlp_dtype="f32", bag="one", index="zipf:1.05", dense="log1p_poisson3",
                     bottom=(13, 512, 256, 128), top=(479, 1024, 1024, 512, 256, 1), training=True),
+    # The large forward with row-wise 8-bit tables (d uint8 codes + fp32 scale and offset per row).
+    "large-u8": Config("large-u8", B=65536, rows=LARGE_ROWS, d=128, table_dtype="u8row", mlp_dtype="bf16",
+                       bag="one", index="zipf:1.05", dense="log1p_poisson3",
+                       bottom=(13, 512, 256, 128), top=(479, 1024, 1024, 512, 256, 1)),
 }
 
 for _c in CONFIGS.values():

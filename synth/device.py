@@ -55,9 +55,24 @@ def host_to_torch(a: np.ndarray, dtype: str) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a))
 
 
-def tables_on_device(cfg: Config, device="cuda", on_device_fill: bool | None = None) -> torch.Tensor:
-    """All tables as one [sum rows][d] device tensor of the table dtype."""
+def tables_on_device(cfg: Config, device="cuda", on_device_fill: bool | None = None, quantize=None) -> torch.Tensor:
+    """All tables as one [sum rows][d] device tensor of the table dtype. Row-wise 8-bit tables
+    ("u8row") come back as uint8 records [sum rows][record bytes]: each table's fp32 source rows are
+    made on the device and handed to quantize(src_f32 [m][d], dst_records [m][rb]) (the caller's
+    quantiser, e.g. the library's dlrm_quantize_rows_u8)."""
     total = int(sum(cfg.rows))
+    if cfg.table_dtype == "u8row":
+        if quantize is None:
+            raise ValueError("row-wise 8-bit tables need a quantize callback")
+        rb = (cfg.d + 8 + 15) // 16 * 16
+        out = torch.empty((total, rb), dtype=torch.uint8, device=device)
+        base = 0
+        for k, m in enumerate(cfg.rows):
+            src = _fill_table_f32(cfg, k, m, device)
+            quantize(src, out[base:base + m])
+            del src
+            base += m
+        return out
     if on_device_fill is None:
         on_device_fill = total * cfg.d > (1 << 26)
     if not on_device_fill:
@@ -75,6 +90,20 @@ def tables_on_device(cfg: Config, device="cuda", on_device_fill: bool | None = N
             raise RuntimeError(f"synth_fill_table failed: cudaError {r}")
         base += m
     return out
+
+
+def _fill_table_f32(cfg: Config, k: int, m: int, device) -> torch.Tensor:
+    """fp32 source rows of table k on the device (the same values as gen.table_rows_f32)."""
+    src = torch.empty((m, cfg.d), dtype=torch.float32, device=device)
+    if m * cfg.d <= (1 << 24):
+        src.copy_(torch.from_numpy(gen.table_rows_f32(gen.table_seed(cfg), k, m, np.arange(m), cfg.d)))
+        return src
+    L = _fill_lib()
+    r = L.synth_fill_table(src.data_ptr(), DT_CODE["f32"], m, cfg.d, k, gen.table_seed(cfg),
+                           float(gen.table_scale(m)), torch.cuda.current_stream(device).cuda_stream)
+    if r != 0:
+        raise RuntimeError(f"synth_fill_table failed: cudaError {r}")
+    return src
 
 
 def mlp_on_device(cfg: Config, which: str, device="cuda"):

@@ -78,6 +78,8 @@ def table_rows(seed: int, table_id: int, m: int, row_ids: np.ndarray, d: int, dt
         return v.astype(np.float16)
     if dtype == "bf16":
         return f32_to_bf16_bits(v)
+    if dtype == "u8row":
+        return v   # row-wise 8-bit tables: the fp32 source rows; quantisation belongs to the consumers
     raise ValueError(dtype)
 
 

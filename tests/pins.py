@@ -341,7 +341,47 @@ def pin_sgd(lib):
     assert np.array_equal(out, np.array([1.0 - 0.005, -2.0 - 0.0025, 3.5 + 0.01]))
 
 
-ALL_PINS = [pin_embbag_golden, pin_embbag_closed_forms, pin_embbag_vs_library, pin_embbag_invalid,
+def pin_quant_golden(lib):
+    # hand-worked row (tests/golden/quant_u8_row.json)
+    g = _golden("quant_u8_row.json")
+    codes, s, m = O.quantize_rows_u8(np.array([g["row"]], np.float32), lib)
+    assert codes[0].tolist() == g["codes"], codes
+    assert s[0] == np.float32(g["scale"]) and m[0] == np.float32(g["offset"]), (s, m)
+    back = O.dequantize_rows_u8(codes, s, m, lib)
+    _close(back[0], np.array(g["row"]), rtol=0, atol=1e-6, what="dequantised worked row")
+
+
+def pin_quant_constant_row(lib):
+    codes, s, m = O.quantize_rows_u8(np.full((1, 16), -0.375, np.float32), lib)
+    assert s[0] == 0 and np.all(codes == 0) and m[0] == np.float32(-0.375)
+    assert np.all(O.dequantize_rows_u8(codes, s, m, lib) == -0.375)
+
+
+def pin_quant_rounding_bound(lib):
+    # nearest code: |s q + m - v| <= s / 2; the row's min and max map to codes 0 and 255
+    rng = np.random.default_rng(3)
+    v = (rng.standard_normal((200, 64)) * rng.uniform(1e-3, 10, (200, 1))).astype(np.float32)
+    codes, s, m = O.quantize_rows_u8(v, lib)
+    back = O.dequantize_rows_u8(codes, s, m, lib)
+    err = np.abs(back - v.astype(np.float64))
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 1e-5) + 1e-6 * np.abs(v).max(axis=1, keepdims=True))
+    assert np.all(codes.min(axis=1) == 0) and np.all(codes.max(axis=1) == 255)
+    assert np.all(m == v.min(axis=1))
+
+
+def pin_quant_brute_force(lib):
+    # the chosen code is the nearest of all 256 (up to the fp32 division that decides ties)
+    rng = np.random.default_rng(4)
+    v = rng.uniform(-2, 3, (64, 8)).astype(np.float32)
+    codes, s, m = O.quantize_rows_u8(v, lib)
+    grid = s[:, None, None].astype(np.float64) * np.arange(256)[None, None, :] + m[:, None, None]
+    dist = np.abs(grid - v[:, :, None].astype(np.float64))
+    chosen = np.take_along_axis(dist, codes[:, :, None].astype(np.int64), axis=2)[:, :, 0]
+    assert np.all(chosen <= dist.min(axis=2) + 1e-6 * s[:, None])
+
+
+ALL_PINS = [pin_quant_golden, pin_quant_constant_row, pin_quant_rounding_bound, pin_quant_brute_force,
+            pin_embbag_golden, pin_embbag_closed_forms, pin_embbag_vs_library, pin_embbag_invalid,
             pin_interact_golden, pin_interact_closed_forms, pin_interact_vs_library_and_symmetry,
             pin_mlp, pin_forward_zero_last_layer, pin_forward_golden, pin_forward_vs_library, pin_bce,
             pin_gradients_vs_autograd, pin_gradients_finite_difference, pin_sgd]
