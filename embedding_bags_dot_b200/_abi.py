@@ -79,6 +79,10 @@ _SIGS = {
                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
     "dlrm_row_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "dlrm_embbag_cat_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
+                                      C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "dlrm_forward_cat": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                                   C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_quantize_rows_u8": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
                                 C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
@@ -231,6 +235,22 @@ def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices,
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                      _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
                   "dlrm_forward")
+
+
+def dlrm_embbag_cat_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,
+                        stream=None):
+    """Concat-only interaction: concat rows [x_dense, e_1 .. e_K, zeros]."""
+    out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
+    return _check(lib().dlrm_embbag_cat_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
+                                            _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
+                                            _stream(stream)), "dlrm_embbag_cat_fwd")
+
+
+def dlrm_forward_cat(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
+    """dlrm_forward with the concat-only interaction (top MLP input width d (K + 1))."""
+    return _check(lib().dlrm_forward_cat(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
+                                         _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
+                  "dlrm_forward_cat")
 
 
 def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, err_flags=None,

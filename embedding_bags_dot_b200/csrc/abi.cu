@@ -76,7 +76,7 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
     FwdLayout L;
     size_t off = DLRM_ERR_RECORD_BYTES;
     const int K = T->K, d = T->d;
-    const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
+    const int ldc = dlrm_ld(top->dims[0], top->dt);   // the concat: d + K(K+1)/2 (dot) or d(K+1) (concat-only)
     L.x_dense = off;
     off = align_up(off + sizeof(float) * (size_t)B * d, 256);
     L.concat = off;
@@ -237,16 +237,20 @@ dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype 
                    static_cast<ErrRecord*>(ws), cs(stream));
 }
 
-dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+namespace {
+
+// The forward pass with the dot interaction (cat = false) or the concat-only one (cat = true).
+dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
-                         dlrm_stream stream) {
+                         dlrm_stream stream, bool cat) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
     if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
     if ((r = check_mlp(bot)) != DLRM_OK || (r = check_mlp(top)) != DLRM_OK) return r;
     const int K = T->K, d = T->d;
-    if (bot->dims[bot->n_layers] != d || top->dims[0] != d + K * (K + 1) / 2 || top->dims[top->n_layers] != 1)
+    const int width = cat ? d * (K + 1) : d + K * (K + 1) / 2;
+    if (bot->dims[bot->n_layers] != d || top->dims[0] != width || top->dims[top->n_layers] != 1)
         return DLRM_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
@@ -256,16 +260,47 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
     cudaStream_t st = cs(stream);
     float* x_dense = reinterpret_cast<float*>(w + L.x_dense);
     void* concat = w + L.concat;
-    const int ldc = dlrm_ld(d + K * (K + 1) / 2, top->dt);
+    const int ldc = dlrm_ld(width, top->dt);
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
     if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1,
                      w + L.cvt, err, st)))
         return r;
-    if ((r = launch_embbag_interact(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt,
-                                    reinterpret_cast<ErrRecord*>(w), st)))
-        return r;
+    r = cat ? launch_embbag_cat(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt, err,
+                                st)
+            : launch_embbag_interact(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt,
+                                     err, st);
+    if (r) return r;
     return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, w + L.cvt, err,
                    st);
+}
+
+}  // namespace
+
+dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                         const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
+                         dlrm_stream stream) {
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, false);
+}
+
+dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                             const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
+                             dlrm_stream stream) {
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, true);
+}
+
+dlrm_status dlrm_embbag_cat_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                                int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt, void* ws,
+                                dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_tables(T, tm);
+    if (r != DLRM_OK) return r;
+    if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
+    if (!valid_dt(out_dt) || ld < T->d * (T->K + 1)) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    if (!x_dense || !concat) return DLRM_ERR_INVALID_ARG;
+    return launch_embbag_cat(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, x_dense, concat, ld, out_dt,
+                             static_cast<ErrRecord*>(ws), cs(stream));
 }
 
 }  // extern "C"

@@ -227,6 +227,79 @@ __global__ void __launch_bounds__(256) embbag_kernel(const T* __restrict__ table
     report_warp(err, oob, bad);
 }
 
+// ------------------------------------------------------------------ concat-only interaction
+
+// Writes a pooled bag into its d-wide slot of a concat row, converted to OT
+// (16-byte stores where the slot is aligned, element stores otherwise).
+template <typename T, bool VEC, int NCH, typename OT>
+struct CatSink {
+    OT* base;          // slot of bag s is base + s * stride
+    long long stride;
+    int g, GL, n_ch;
+    bool vec_ok;
+    template <typename Acc>
+    __device__ __forceinline__ void operator()(int s, Acc& acc) {
+        constexpr int E = RowIO<T, VEC>::E;
+        OT* dst = base + s * stride;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int cg = g + GL * c;
+            if (cg < n_ch) {
+                OT* p = dst + cg * E;
+                if constexpr (E * sizeof(OT) % 16 == 0) {
+                    if (vec_ok) {
+#pragma unroll
+                        for (int h = 0; h < (int)(E * sizeof(OT) / 16); ++h) {
+                            OT t[16 / sizeof(OT)];
+#pragma unroll
+                            for (int e = 0; e < (int)(16 / sizeof(OT)); ++e)
+                                t[e] = Cvt<OT>::from_f(acc[c][h * (16 / sizeof(OT)) + e]);
+                            reinterpret_cast<uint4*>(p)[h] = *reinterpret_cast<const uint4*>(t);
+                        }
+                        continue;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) p[e] = Cvt<OT>::from_f(acc[c][e]);
+            }
+        }
+    }
+};
+
+// Concat-only interaction (the Wide & Deep alternative the pages contrast
+// DLRM with: embeddings concatenated with the dense vector, no dot products):
+// row b of out is [x_dense_b, e_1, ..., e_K, 0 padding up to ld], each e_k the
+// sum-pooled bag (k, b). The gather is K1's; only the destination differs.
+template <typename T, bool VEC, int NCH, typename OT>
+__global__ void __launch_bounds__(256) embbag_cat_kernel(const T* __restrict__ tables, const __grid_constant__ TableMeta tm,
+                                                         int K, int d, int n_ch, int GL, int B, int S,
+                                                         const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ indices, long long nnz,
+                                                         const float* __restrict__ x_dense, OT* __restrict__ out, int ld,
+                                                         bool vec_ok, ErrRecord* err) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    int* off_s = reinterpret_cast<int*>(smem);
+    unsigned char* bad_s = smem + sizeof(int) * K * (S + 1);
+    const int b0 = blockIdx.x * S;
+    const int nb = min(S, B - b0);
+    unsigned oob = 0, bad = 0;
+    load_tile_offsets(offsets, B, K, b0, nb, S, nnz, off_s, bad_s, nullptr, bad);
+    auto make_sink = [&](int k, int s0, int g) {
+        return CatSink<T, VEC, NCH, OT>{out + (long long)(b0 + s0) * ld + (long long)(k + 1) * d, (long long)ld, g, GL,
+                                        n_ch, vec_ok};
+    };
+    pool_tile<T, VEC, NCH, 4>(tables, tm, K, d, n_ch, GL, indices, off_s, bad_s, S, nb, oob, make_sink);
+    // x_dense in front, zero padding behind
+    const int tail = ld - d * (K + 1);
+    for (int q = threadIdx.x; q < nb * (d + tail); q += blockDim.x) {
+        const int s = q / (d + tail), c = q - s * (d + tail);
+        const long long b = b0 + s;
+        if (c < d) out[b * ld + c] = Cvt<OT>::from_f(x_dense[b * d + c]);
+        else out[b * ld + d * (K + 1) + (c - d)] = Cvt<OT>::from_f(0.f);
+    }
+    report_warp(err, oob, bad);
+}
+
 // ------------------------------------------------------------------ interaction on a smem tile
 
 __device__ __forceinline__ int pair_row(int p) {
@@ -467,6 +540,60 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
         case DLRM_F16: return launch_fused_t<__half>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
     }
     return DLRM_ERR_UNSUPPORTED;
+}
+
+template <typename T, typename OT>
+static dlrm_status launch_cat_t(const TableMeta& tm, const void* tables, int K, int d, int B, const int32_t* offsets,
+                                const int32_t* indices, long long nnz, const float* x_dense, void* out, int ld,
+                                ErrRecord* err, cudaStream_t st, const Geometry& g) {
+    const int S = 32;
+    const size_t smem = sizeof(int) * (size_t)K * (S + 1) + (size_t)K * S;
+    const dim3 grid((B + S - 1) / S);
+    const T* tb = static_cast<const T*>(tables);
+    OT* o = static_cast<OT*>(out);
+    const bool vec_ok = ((uintptr_t)out & 15) == 0 && ((size_t)d * sizeof(OT)) % 16 == 0 && ((size_t)ld * sizeof(OT)) % 16 == 0;
+#define DLRM_CAT(VEC, NCH)                                                                                       \
+    {                                                                                                            \
+        auto kern = embbag_cat_kernel<T, VEC, NCH, OT>;                                                          \
+        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+        kern<<<grid, 256, smem, st>>>(tb, tm, K, d, g.n_ch, g.GL, B, S, offsets, indices, nnz, x_dense, o, ld,   \
+                                      vec_ok, err);                                                              \
+    }
+    if (g.vec) {
+        if (g.NCH == 1) DLRM_CAT(true, 1) else if (g.NCH == 2) DLRM_CAT(true, 2) else DLRM_CAT(true, 4)
+    } else {
+        if (g.NCH == 1) DLRM_CAT(false, 1) else if (g.NCH == 2) DLRM_CAT(false, 2)
+        else if (g.NCH == 4) DLRM_CAT(false, 4) else DLRM_CAT(false, 8)
+    }
+#undef DLRM_CAT
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
+template <typename T>
+static dlrm_status launch_cat_out(const TableMeta& tm, const void* tables, int K, int d, int B, const int32_t* offsets,
+                                  const int32_t* indices, long long nnz, const float* x_dense, void* out, int ld,
+                                  dlrm_dtype out_dt, ErrRecord* err, cudaStream_t st, const Geometry& g) {
+    switch (out_dt) {
+        case DLRM_F32: return launch_cat_t<T, float>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st, g);
+        case DLRM_BF16: return launch_cat_t<T, __nv_bfloat16>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st, g);
+        case DLRM_F16: return launch_cat_t<T, __half>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st, g);
+        default: return DLRM_ERR_UNSUPPORTED;
+    }
+}
+
+dlrm_status launch_embbag_cat(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
+                              const int32_t* offsets, const int32_t* indices, long long nnz, const float* x_dense,
+                              void* out, int ld, dlrm_dtype out_dt, ErrRecord* err, cudaStream_t st) {
+    Geometry g;
+    if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
+    if ((size_t)sizeof(int) * K * 33 + (size_t)K * 32 > kSmemMax) return DLRM_ERR_UNSUPPORTED;
+    switch (dt) {
+        case DLRM_F32: return launch_cat_out<float>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
+        case DLRM_BF16: return launch_cat_out<__nv_bfloat16>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
+        case DLRM_F16: return launch_cat_out<__half>(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st, g);
+        default: return DLRM_ERR_UNSUPPORTED;
+    }
 }
 
 }  // namespace dlrm

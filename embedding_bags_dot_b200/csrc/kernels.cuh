@@ -47,6 +47,11 @@ dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st);
 
+// Concat-only interaction: out row b = [x_dense_b, e_1 .. e_K, zeros up to ld] (embbag.cu)
+dlrm_status launch_embbag_cat(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
+                              const int32_t* offsets, const int32_t* indices, long long nnz, const float* x_dense,
+                              void* out, int ld, dlrm_dtype out_dt, ErrRecord* err, cudaStream_t st);
+
 // DLRM_U8ROW record bytes of a row of width d (quant.cu)
 size_t u8row_bytes(int d);
 

@@ -213,6 +213,24 @@ dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, 
                                      int64_t nnz, void* grads, uint32_t* rows, float* row_grads,
                                      int32_t* n_rows, dlrm_stream stream);
 
+/* Concat-only interaction, the alternative the pages set DLRM against
+ * ("Deep Learning Recommendation Model (DLRM)", Key Method Details: Wide &
+ * Deep concatenates embeddings without explicit interactions; "DLRM",
+ * briansu.co, section 3: variants swap the interaction layer and keep the
+ * sparse/dense skeleton). Row b of concat ([B][ld], out_dt, ld >= d (K + 1))
+ * becomes [x_dense_b, e_1, ..., e_K, zeros up to ld] with e_k the sum-pooled
+ * bag (k, b); x_dense fp32 [B][d]. Bags, errors and dtypes as
+ * dlrm_embbag_interact_fwd (DLRM_U8ROW tables: DLRM_ERR_UNSUPPORTED). */
+dlrm_status dlrm_embbag_cat_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
+                                int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt, void* ws,
+                                dlrm_stream stream);
+
+/* dlrm_forward with the concat-only interaction: top->dims[0] must be
+ * d (K + 1). Workspace: dlrm_workspace_size(T, bot, top, B, 0). */
+dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                             const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
+                             dlrm_stream stream);
+
 /* fp32 GEMM of the training step, on the tensor cores at fp32 accuracy
  * (the matrix products of the fully connected layers, "Deep Learning
  * Recommendation Model (DLRM)", Key Method Details: bottom and top MLPs, and

@@ -621,3 +621,16 @@ void oracle_dequantize_rows_u8(int64_t rows, int d, const unsigned char* codes, 
     for (int64_t r = 0; r < rows; ++r)
         for (int c = 0; c < d; ++c) out[r * d + c] = (double)scale[r] * (double)codes[r * d + c] + (double)offset[r];
 }
+
+/* Concat-only interaction (the Wide & Deep alternative the pages contrast
+ * DLRM with, "Deep Learning Recommendation Model (DLRM)", Key Method Details):
+ * out[b] = [x_dense[b], e_1, ..., e_K], width d (K + 1). */
+void oracle_concat(int B, int K, int d, const double* x_dense, const double* pooled, double* out) {
+    const int64_t w = (int64_t)d * (K + 1);
+    for (int b = 0; b < B; ++b) {
+        double* o = out + (int64_t)b * w;
+        for (int t = 0; t < d; ++t) o[t] = x_dense[(int64_t)b * d + t];
+        for (int k = 0; k < K; ++k)
+            for (int t = 0; t < d; ++t) o[(int64_t)(k + 1) * d + t] = pooled[((int64_t)b * K + k) * d + t];
+    }
+}

@@ -69,6 +69,7 @@ def _declare(lib):
                                        vp, vp, vp, vp, vp]
     lib.oracle_sgd.argtypes = [C.c_int64, d, vp, vp]
     lib.oracle_quantize_rows_u8.argtypes = [C.c_int64, i, vp, vp, vp, vp]
+    lib.oracle_concat.argtypes = [i, i, i, vp, vp, vp]
     lib.oracle_dequantize_rows_u8.argtypes = [C.c_int64, i, vp, vp, vp, vp]
     return lib
 
@@ -238,6 +239,28 @@ def forward(model: Model, dense, offsets, indices, lib=None):
     s = model.struct()
     lib.oracle_forward(C.byref(s), B, indices.size, _p(dense), _p(offsets), _p(indices), _p(y), _p(z), _p(counts))
     return y, z, (int(counts[0]), int(counts[1]))
+
+
+def concat(x_dense: np.ndarray, pooled: np.ndarray, lib=None) -> np.ndarray:
+    """Concat-only interaction: [B][d] and [B][K][d] -> [B][d (K + 1)] = [x_dense, e_1 .. e_K]."""
+    lib = lib or load()
+    x_dense, pooled = _c64(x_dense), _c64(pooled)
+    B, K, d = pooled.shape
+    out = np.zeros((B, d * (K + 1)), np.float64)
+    lib.oracle_concat(B, K, d, _p(x_dense), _p(pooled), _p(out))
+    return out
+
+
+def forward_cat(model: Model, dense, offsets, indices, lib=None):
+    """The forward pass with the concat-only interaction: bottom MLP (ReLU after every layer), pooled
+    bags, [x_dense, e_1 .. e_K], top MLP (last layer linear), sigmoid. Returns (y_hat, logits, counts)."""
+    lib = lib or load()
+    dense = _c64(dense)
+    B = dense.shape[0]
+    x = mlp(model.bot_W, model.bot_b, dense, relu_last=True, lib=lib)
+    pooled, _, counts = embbag(model.tables, model.rows, model.d, B, offsets, indices, lib=lib)
+    z = mlp(model.top_W, model.top_b, concat(x, pooled, lib=lib), relu_last=False, lib=lib)[:, 0]
+    return 1.0 / (1.0 + np.exp(-z)), z, counts
 
 
 def bce(z, y, lib=None) -> float:

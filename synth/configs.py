@@ -38,10 +38,11 @@ class Config:
     index: str                  # "uniform" | "zipf:<alpha>"
     dense: str                  # "normal" | "log1p_poisson3"
     bottom: tuple               # layer widths, first is 13, last is d
-    top: tuple                  # layer widths, first is d + P, last is 1
+    top: tuple                  # layer widths, first is the concat width, last is 1
     training: bool = False
     lr: float = 0.01
     seed: int = 0
+    interaction: str = "dot"    # "dot": [x_dense, Z] (the pages' DLRM); "cat": [x_dense, e_1..e_K] (concat-only)
 
     @property
     def K(self) -> int:
@@ -54,7 +55,7 @@ class Config:
 
     @property
     def concat_width(self) -> int:
-        return self.d + self.P
+        return self.d + self.P if self.interaction == "dot" else self.d * (self.K + 1)
 
     @property
     def concat_ld(self) -> int:
@@ -69,7 +70,8 @@ class Config:
 
     def check(self) -> None:
         assert self.bottom[-1] == self.d, "bottom MLP must end at d"
-        assert self.top[0] == self.concat_width, "top MLP must start at d + K(K+1)/2"
+        assert self.interaction in ("dot", "cat")
+        assert self.top[0] == self.concat_width, "top MLP must start at the concat width"
         assert self.top[-1] == 1, "top MLP must end in one logit"
 
 
@@ -100,6 +102,10 @@ CONFIGS = {
     "train": Config("train", B=65536, rows=tuple(r // 4 for r in LARGE_ROWS), d=128, table_dtype="f32",
                     mlp_dtype="f32", bag="one", index="zipf:1.05", dense="log1p_poisson3",
                     bottom=(13, 512, 256, 128), top=(479, 1024, 1024, 512, 256, 1), training=True),
+    # The large forward with the concat-only interaction (top MLP input [x_dense, e_1..e_26] = 3456 wide).
+    "large-cat": Config("large-cat", B=65536, rows=LARGE_ROWS, d=128, table_dtype="bf16", mlp_dtype="bf16",
+                        bag="one", index="zipf:1.05", dense="log1p_poisson3",
+                        bottom=(13, 512, 256, 128), top=(3456, 1024, 1024, 512, 256, 1), interaction="cat"),
     # The large forward with row-wise 8-bit tables (d uint8 codes + fp32 scale and offset per row).
     "large-u8": Config("large-u8", B=65536, rows=LARGE_ROWS, d=128, table_dtype="u8row", mlp_dtype="bf16",
                        bag="one", index="zipf:1.05", dense="log1p_poisson3",

@@ -380,7 +380,39 @@ def pin_quant_brute_force(lib):
     assert np.all(chosen <= dist.min(axis=2) + 1e-6 * s[:, None])
 
 
-ALL_PINS = [pin_quant_golden, pin_quant_constant_row, pin_quant_rounding_bound, pin_quant_brute_force,
+def pin_concat(lib):
+    # layout: columns [0, d) are x_dense, [d (k + 1), d (k + 2)) are e_k; against torch.cat
+    rng = np.random.default_rng(11)
+    B, K, d = 5, 4, 3
+    x = rng.standard_normal((B, d))
+    p = rng.standard_normal((B, K, d))
+    got = O.concat(x, p, lib)
+    want = torch.cat([torch.from_numpy(x)] + [torch.from_numpy(p[:, k]) for k in range(K)], dim=1).numpy()
+    assert np.array_equal(got, want)
+    assert np.array_equal(got[:, :d], x) and np.array_equal(got[:, d * 3:d * 4], p[:, 2])
+
+
+def pin_forward_cat_vs_library(lib):
+    # bottom MLP, pooling, concat, top MLP, sigmoid in torch fp64 (embedding_bag, cat, linear)
+    cfg = shrink(CONFIGS["tiny"], B=20).with_(bag="mix", seed=5, interaction="cat", top=(16 * 9, 32, 1))
+    batch = gen.make_batches(cfg, (0,))[0]
+    model = O.model_from_config(cfg)
+    y, z, counts = O.forward_cat(model, batch.dense, batch.offsets, batch.indices, lib)
+    x = torch.from_numpy(np.asarray(batch.dense, np.float64))
+    for W, b in zip(model.bot_W, model.bot_b):
+        x = torch.relu(F.linear(x, torch.from_numpy(W), torch.from_numpy(b)))
+    pooled = torch_pool(model.tables, model.rows, model.d, cfg.B, batch.offsets, batch.indices)
+    h = torch.cat([x] + [pooled[:, k] for k in range(cfg.K)], dim=1)
+    for l, (W, b) in enumerate(zip(model.top_W, model.top_b)):
+        h = F.linear(h, torch.from_numpy(W), torch.from_numpy(b))
+        if l < len(model.top_W) - 1:
+            h = torch.relu(h)
+    _close(z, h[:, 0].numpy(), what="concat-only logits")
+    _close(y, torch.sigmoid(h[:, 0]).numpy(), what="concat-only y_hat")
+    assert counts == (0, 0)
+
+
+ALL_PINS = [pin_concat, pin_forward_cat_vs_library, pin_quant_golden, pin_quant_constant_row, pin_quant_rounding_bound, pin_quant_brute_force,
             pin_embbag_golden, pin_embbag_closed_forms, pin_embbag_vs_library, pin_embbag_invalid,
             pin_interact_golden, pin_interact_closed_forms, pin_interact_vs_library_and_symmetry,
             pin_mlp, pin_forward_zero_last_layer, pin_forward_golden, pin_forward_vs_library, pin_bce,

@@ -35,6 +35,8 @@ MUTANTS = {
     "sgd_sign": ("w[q] -= lr * g[q];", "w[q] += lr * g[q];"),
     "dense_grad_direct_part_dropped": ("for (int t = 0; t < d; ++t) g[t] += dc[t];", "(void)0;"),
     "oob_not_counted": ("if (r < 0 || r >= rows[k]) { ++oob; continue; }", "if (r < 0 || r >= rows[k]) { continue; }"),
+    "concat_dense_last": ("for (int t = 0; t < d; ++t) o[t] = x_dense[(int64_t)b * d + t];",
+                          "for (int t = 0; t < d; ++t) o[(int64_t)K * d + t] = x_dense[(int64_t)b * d + t];"),
     "quant_floor": ("if (s > 0.0f) q = rintf((v[c] - lo) / s);", "if (s > 0.0f) q = floorf((v[c] - lo) / s);"),
     "quant_scale_256": ("const float s = (hi - lo) / 255.0f;", "const float s = (hi - lo) / 256.0f;"),
     "quant_offset_hi": ("        offset[r] = lo;", "        offset[r] = hi;"),
