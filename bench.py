@@ -160,7 +160,7 @@ def oracle_rate(cfg, batch, n_samples: int, seed: int = 0):
     Bs, dense, offs, idx, _, rows, used = O.sub_batch(cfg, batch, samples)
     model = O.model_for_rows(cfg, used)
     t0 = time.perf_counter()
-    O.forward(model, dense, offs, idx)
+    (O.forward_cat if cfg.interaction == "cat" else O.forward)(model, dense, offs, idx)
     dt = time.perf_counter() - t0
     return Bs / dt, dt, O.threads(), Bs
 
@@ -272,7 +272,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         E.dlrm_mlp_fwd(bot, cfg.B, b["dense"], cfg.n_dense, x_dense, cfg.d, E.ACT_RELU, ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        E.dlrm_embbag_interact_fwd(T, cfg.B, b["offsets"], b["indices"], x_dense, concat, ldc, cfg.mlp_dtype, ws, stream)
+        if cfg.interaction == "cat":
+            E.dlrm_embbag_cat_fwd(T, cfg.B, b["offsets"], b["indices"], x_dense, concat, ldc, cfg.mlp_dtype, ws, stream)
+        else:
+            E.dlrm_embbag_interact_fwd(T, cfg.B, b["offsets"], b["indices"], x_dense, concat, ldc, cfg.mlp_dtype, ws,
+                                       stream)
         if ev is not None:
             ev[2].record(stream)
         E.dlrm_mlp_fwd(top, cfg.B, concat, ldc, y, 1, E.ACT_SIGMOID, ws, stream)
@@ -321,6 +325,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     for ev in consumed:
         ev.record(stream)
 
+    fwd = E.dlrm_forward_cat if cfg.interaction == "cat" else E.dlrm_forward
+
     def e2e_step(i):
         sl, hb = i & 1, host_b[i % POOL]
         cstream.wait_event(consumed[sl])
@@ -330,7 +336,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         copied[sl].record(cstream)
         stream.wait_event(copied[sl])
         n = hb["indices"].numel()
-        E.dlrm_forward(T, bot, top, cfg.B, slots[sl]["dense"], slots[sl]["offsets"], slots[sl]["indices"][:n],
+        fwd(T, bot, top, cfg.B, slots[sl]["dense"], slots[sl]["offsets"], slots[sl]["indices"][:n],
                        y_dev[sl], ws, stream)
         consumed[sl].record(stream)
         y_host[sl].copy_(y_dev[sl], non_blocking=True)
@@ -379,9 +385,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                              f"and a {POOL}-batch pool of {pool_bytes / 1e6:.0f} MB exceed the {L2_BYTES >> 20} MB L2"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
                          "frac": achieved / peak_hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
-                                   if cfg.table_dtype in ("bf16", "u8row")
-                                   else "embbag_interact_kernel (dlrm_embbag_interact_fwd)",
+                         "kernel": ("embbag_cat_kernel (dlrm_embbag_cat_fwd)" if cfg.interaction == "cat" else
+                                    "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
+                                    if cfg.table_dtype in ("bf16", "u8row")
+                                    else "embbag_interact_kernel (dlrm_embbag_interact_fwd)"),
                          "algorithmic_bytes_per_launch": avg_algo, "avg_launch_ms": k2_avg},
             "kernels_ms_per_step": {"bottom_mlp": float(np.mean(bot_ms)), "embbag_interact": float(np.mean(k2_ms)),
                                     "top_mlp": float(np.mean(top_ms))},

@@ -97,3 +97,21 @@ def test_skipped_indices_and_argument_errors():
         E.dlrm_forward(g.T, g.bot, g.top, cfg.B, torch.from_numpy(batch.dense).cuda(), offs,
                        torch.from_numpy(batch.indices).cuda(), y, g.ws)
     assert e.value.status == E.ERR_INVALID_ARG
+
+
+@pytest.mark.slow
+def test_large_cat_forward_full_size():
+    # the full 65,536-sample batch in the benchmark's launch configuration, checked on sampled outputs
+    cfg = CONFIGS["large-cat"]
+    batch = gen.make_batches(cfg, (0,))[0]
+    g = GpuModel(cfg)
+    bt = {k: torch.from_numpy(v).cuda() for k, v in (("dense", batch.dense), ("offsets", batch.offsets),
+                                                      ("indices", batch.indices))}
+    y = torch.empty(cfg.B, device="cuda")
+    E.dlrm_forward_cat(g.T, g.bot, g.top, cfg.B, bt["dense"], bt["offsets"], bt["indices"], y, g.ws)
+    assert E.dlrm_check_error(g.ws)[0] == 0
+    samples = np.sort(np.random.default_rng(8).choice(cfg.B, 256, replace=False))
+    Bs, dense, offs, idx, _, rows, used = O.sub_batch(cfg, batch, samples)
+    want, _, counts = O.forward_cat(O.model_for_rows(cfg, used), dense, offs, idx)
+    assert counts == (0, 0)
+    assert_close(to_np(y)[samples], want, "bf16", "large-cat y_hat (sampled)")
