@@ -29,6 +29,8 @@ struct TrainWs {
     size_t z, dz;                                            // logit and dL/dz [B]
     size_t g[2][2];                                          // gradient ping-pong pairs [B][gmax]
     size_t dcat, dxd;                                        // plain d(concat) [B][ldc], d(x_dense pre-act) [B][d]
+    size_t bbits[DLRM_MAX_LAYERS], tbits[DLRM_MAX_LAYERS];   // ReLU bitmasks of the saved activations
+    size_t csum;                                             // column sums per 32-row group of a gradient
     size_t wscratch, lpart, total;
     int ldb[DLRM_MAX_LAYERS], ldt[DLRM_MAX_LAYERS], ldc, gmax;
 };
@@ -79,6 +81,9 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
         for (int h = 0; h < 2; ++h) W.g[p][h] = take(sizeof(float) * (size_t)B * gmax);
     W.dcat = take(sizeof(float) * (size_t)B * W.ldc);
     W.dxd = take(sizeof(float) * (size_t)B * d);
+    for (int l = 0; l < nb; ++l) W.bbits[l] = take(sizeof(uint32_t) * (size_t)B * relu_bits_ld(bot->dims[l + 1]));
+    for (int l = 0; l < nt - 1; ++l) W.tbits[l] = take(sizeof(uint32_t) * (size_t)B * relu_bits_ld(top->dims[l + 1]));
+    W.csum = take(sizeof(float) * (size_t)((B + 31) / 32) * gmax);
     size_t ws = 0;
     for (int l = 0; l < nb; ++l)
         ws = std::max(ws, train_wgrad_scratch_floats(bot->dims[l + 1], bot->dims[l], B));
@@ -207,6 +212,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
     cudaStream_t st = cs(stream);
     auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
+    auto U = [&](size_t o) { return reinterpret_cast<uint32_t*>(w + o); };
     auto GF = [&](size_t o) { return reinterpret_cast<float*>(g + o); };
     const int nb = bot->n_layers, nt = top->n_layers;
 
@@ -229,7 +235,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     for (int l = 0; l < nb; ++l) {
         const F32Pair in = l == 0 ? dense_in : P(W.bact[l - 1], W.ldb[l - 1]);
         if ((r = train_linear_fwd(B, bot->dims[l + 1], bot->dims[l], in, P(W.bW[l], ldf(bot->dims[l])), bot->b[l],
-                                  F(W.bact[l][0]), F(W.bact[l][1]), W.ldb[l], true, err, st)))
+                                  F(W.bact[l][0]), F(W.bact[l][1]), W.ldb[l], true, U(W.bbits[l]), err, st)))
             return r;
     }
     const F32Pair xd_pair = P(W.bact[nb - 1], W.ldb[nb - 1]);   // ld = d (d % 4 == 0 on this path)
@@ -253,7 +259,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
         const bool last = l == nt - 1;
         if ((r = train_linear_fwd(B, top->dims[l + 1], top->dims[l], in, P(W.tW[l], ldf(top->dims[l])), top->b[l],
                                   last ? F(W.z) : F(W.tact[l][0]), last ? nullptr : F(W.tact[l][1]), W.ldt[l], !last,
-                                  err, st)))
+                                  last ? nullptr : U(W.tbits[l]), err, st)))
             return r;
     }
 
@@ -265,23 +271,26 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
 
     // ---- top MLP backward: cur = dL/d(pre-activation of layer l)
     F32Pair cur{dz, nullptr, 1};
-    int pp = 0;   // next gradient pair buffer
+    int pp = 0;           // next gradient pair buffer
+    bool csum_ok = false;  // W.csum holds the column sums of cur per 32-row group
     for (int l = nt - 1; l >= 0; --l) {
         const F32Pair in = l == 0 ? concat_p : P(W.tact[l - 1], W.ldt[l - 1]);
         const int N = top->dims[l + 1], Kin = top->dims[l];
         const F32Pair Wp = P(W.tW[l], ldf(Kin));
-        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.tdW[l]), ldf(Kin), GF(G.tdb[l]), F(W.wscratch), err,
-                                    st)))
+        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.tdW[l]), ldf(Kin), GF(G.tdb[l]),
+                                    csum_ok ? F(W.csum) : nullptr, F(W.wscratch), err, st)))
             return r;
+        csum_ok = false;
         if (l > 0) {
             const int ldo = W.gmax;
-            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, in, F(W.g[pp][0]), F(W.g[pp][1]), ldo, err, st)))
+            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, in, U(W.tbits[l - 1]), F(W.g[pp][0]), F(W.g[pp][1]), ldo,
+                                        F(W.csum), &csum_ok, err, st)))
                 return r;
             cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), ldo};
             pp ^= 1;
         } else {
-            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, F32Pair{nullptr, nullptr, 0}, F(W.dcat), nullptr, W.ldc,
-                                        err, st)))
+            if ((r = train_linear_dgrad(B, N, Kin, cur, Wp, F32Pair{nullptr, nullptr, 0}, nullptr, F(W.dcat), nullptr,
+                                        W.ldc, nullptr, nullptr, err, st)))
                 return r;
         }
     }
@@ -296,16 +305,19 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     }
     cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), d};
     pp ^= 1;
+    csum_ok = false;
     for (int l = nb - 1; l >= 0; --l) {
         const F32Pair in = l == 0 ? dense_in : P(W.bact[l - 1], W.ldb[l - 1]);
         const int N = bot->dims[l + 1], Kin = bot->dims[l];
-        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.bdW[l]), ldf(Kin), GF(G.bdb[l]), F(W.wscratch), err,
-                                    st)))
+        if ((r = train_linear_wgrad(B, N, Kin, cur, in, GF(G.bdW[l]), ldf(Kin), GF(G.bdb[l]),
+                                    csum_ok ? F(W.csum) : nullptr, F(W.wscratch), err, st)))
             return r;
+        csum_ok = false;
         if (l > 0) {
             const int ldo = W.gmax;
-            if ((r = train_linear_dgrad(B, N, Kin, cur, P(W.bW[l], ldf(Kin)), in, F(W.g[pp][0]), F(W.g[pp][1]), ldo,
-                                        err, st)))
+            // the first layer's bias gradient comes with its weight gradient (one pass over dy): no column sums
+            if ((r = train_linear_dgrad(B, N, Kin, cur, P(W.bW[l], ldf(Kin)), in, U(W.bbits[l - 1]), F(W.g[pp][0]),
+                                        F(W.g[pp][1]), ldo, l - 1 > 0 ? F(W.csum) : nullptr, &csum_ok, err, st)))
                 return r;
             cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), ldo};
             pp ^= 1;

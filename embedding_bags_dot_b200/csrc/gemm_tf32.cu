@@ -64,6 +64,18 @@ static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= 168 * THREADS3, "register spli
 
 enum Epi3 { E3_RELU_PAIR = 0, E3_MASK_PAIR = 1, E3_PLAIN = 2 };
 
+// Epilogue operands (unused ones null).
+struct Epi3Args {
+    const float* bias;          // E3_RELU_PAIR: bias[J]
+    const float* mhi;           // E3_MASK_PAIR without bits: the saved post-ReLU activation pair [I][ldm]
+    const float* mlo;
+    long long ldm;
+    uint32_t* bits_out;         // E3_RELU_PAIR: ReLU bitmask of the output, bit j % 32 of word [i][j / 32]
+    const uint32_t* bits_in;    // E3_MASK_PAIR: the saved activation's ReLU bitmask (instead of mhi/mlo)
+    long long ldbits;           // words per row of either bitmask
+    float* csum;                // E3_MASK_PAIR: column sums of each 32-row group of the output, [I / 32][J]
+};
+
 struct Bars3 {
     unsigned long long full[STAGES3];
     unsigned long long empty[STAGES3];
@@ -159,15 +171,43 @@ __device__ __forceinline__ void stage_store(const float (&v)[32], unsigned char*
     if (lane == 0) tma_store_3d(map, stage_s, x, y, z);
 }
 
+// Lane l ends with the sum over lanes of part[l] (part is consumed): the
+// column sums of a warp's 32 rows, a fixed summation tree.
+__device__ __forceinline__ float reduce_scatter32(float (&part)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int k = 0; k < w; ++k) {
+            const float send = upper ? part[k] : part[k + w];
+            const float keep = upper ? part[k + w] : part[k];
+            part[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return part[0];
+}
+
 // Final epilogue of one warp from its fp32 register accumulator: rows i0 ..
 // i0 + 31 (one per lane), columns jb .. jb + 127 (acc[c][e] = column jb + 32c + e).
 template <int EPI>
 __device__ __forceinline__ void epilogue3(float (&acc)[4][32], int i0, int jb, int I, int J, int z,
-                                          const float* __restrict__ bias, const float* __restrict__ mhi,
-                                          const float* __restrict__ mlo, long long ldm, const CUtensorMap* c0,
-                                          const CUtensorMap* c1, unsigned char* stage, uint32_t stage_s) {
+                                          const Epi3Args& ea, const CUtensorMap* c0, const CUtensorMap* c1,
+                                          unsigned char* stage, uint32_t stage_s) {
     const int lane = threadIdx.x & 31;
     const int i = i0 + lane;
+    const float* __restrict__ bias = ea.bias;
+    const float* __restrict__ mhi = ea.mhi;
+    const float* __restrict__ mlo = ea.mlo;
+    const long long ldm = ea.ldm;
+    // the saved activation's ReLU bits for this lane's row, one word per 32-column chunk, loaded up front
+    uint32_t mbits[4] = {0u, 0u, 0u, 0u};
+    if constexpr (EPI == E3_MASK_PAIR) {
+        if (ea.bits_in && i < I) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (jb + 32 * c < J) mbits[c] = __ldg(ea.bits_in + (long long)i * ea.ldbits + (jb + 32 * c) / 32);
+        }
+    }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const int j0 = jb + 32 * c;
@@ -192,9 +232,21 @@ __device__ __forceinline__ void epilogue3(float (&acc)[4][32], int i0, int jb, i
                 }
             }
         }
+        if constexpr (EPI == E3_RELU_PAIR) {
+            if (ea.bits_out && i < I) {
+                uint32_t b = 0u;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) b |= (v[e] > 0.f ? 1u : 0u) << e;
+                ea.bits_out[(long long)i * ea.ldbits + j0 / 32] = b;
+            }
+        }
         if constexpr (EPI == E3_MASK_PAIR) {
-            // ReLU'(pre-activation) from the saved post-ReLU value m = hi + lo: 1 where m > 0
-            if (i < I) {
+            // ReLU'(pre-activation): 1 where the saved post-ReLU value m = hi + lo is > 0
+            if (ea.bits_in) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (!((mbits[c] >> e) & 1u)) v[e] = 0.f;
+            } else if (i < I) {
                 const float* h = mhi + (long long)i * ldm + j0;
                 const float* l = mlo + (long long)i * ldm + j0;
                 if (j0 + 32 <= J) {
@@ -224,6 +276,13 @@ __device__ __forceinline__ void epilogue3(float (&acc)[4][32], int i0, int jb, i
 #pragma unroll
             for (int e = 0; e < 32; ++e) w[e] = v[e] - w[e];
             stage_store(w, stage, stage_s, c1, j0, i0, 0);
+            if constexpr (EPI == E3_MASK_PAIR) {
+                if (ea.csum && i0 < I) {   // uniform across the warp; groups wholly beyond I have no slot
+                    // rows beyond I hold zeros (their A rows are zero-filled), so they add nothing
+                    const float cs = reduce_scatter32(v, lane);
+                    if (j0 + lane < J) ea.csum[(long long)(i0 / 32) * J + j0 + lane] = cs;
+                }
+            }
         }
     }
 }
@@ -242,9 +301,8 @@ __device__ __forceinline__ void promote(float (&acc)[4][32], uint32_t taddr) {
 
 template <bool AMN, bool BMN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS3, 1)
-    gemm3x_kernel(const __grid_constant__ Maps3 maps, int I, int J, int R, int r_chunk, int S,
-                  const float* __restrict__ bias, const float* __restrict__ mhi, const float* __restrict__ mlo,
-                  long long ldm, ErrRecord* err) {
+    gemm3x_kernel(const __grid_constant__ Maps3 maps, int I, int J, int R, int r_chunk, int S, const Epi3Args ea,
+                  ErrRecord* err) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -409,8 +467,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS3, 1)
                 if (lane == 0) mbar_arrive_cluster(a ? lead_tempty1 : lead_tempty0);
             }
             if (timed_out) break;
-            epilogue3<EPI>(acc, mb * 256 + (int)rank * 128 + q * 32, nb * 256 + h * 128, I, J, z, bias, mhi, mlo,
-                           ldm, &maps.c0, &maps.c1, stage, stage_s);
+            epilogue3<EPI>(acc, mb * 256 + (int)rank * 128 + q * 32, nb * 256 + h * 128, I, J, z, ea, &maps.c0,
+                           &maps.c1, stage, stage_s);
         }
         if (timed_out) *abort = 1;
         if (lane == 0) bulk_wait_all0();
@@ -468,14 +526,14 @@ bool output_map(CUtensorMap* m, float* p, int I, int J, int ld, int S) {
 }
 
 template <bool AMN, bool BMN, int EPI>
-dlrm_status launch3(const Maps3& maps, int I, int J, int R, int r_chunk, int S, const float* bias, const float* mhi,
-                    const float* mlo, int ldm, ErrRecord* err, cudaStream_t st) {
+dlrm_status launch3(const Maps3& maps, int I, int J, int R, int r_chunk, int S, const Epi3Args& ea, ErrRecord* err,
+                    cudaStream_t st) {
     auto kern = gemm3x_kernel<AMN, BMN, EPI>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM3_BYTES);
     const long long ntiles = (long long)((I + 255) / 256) * ((J + 255) / 256) * S;
     const int pairs = sm_count3() / 2;
     const int grid = 2 * (int)(ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS3, SMEM3_BYTES, st>>>(maps, I, J, R, r_chunk, S, bias, mhi, mlo, (long long)ldm, err);
+    kern<<<grid, THREADS3, SMEM3_BYTES, st>>>(maps, I, J, R, r_chunk, S, ea, err);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -493,7 +551,7 @@ bool tf32x3_supported(int M, int N, int K, F32Pair a, F32Pair b) {
 }
 
 dlrm_status tf32x3_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* bias, float* y_hi, float* y_lo,
-                       int ldy, ErrRecord* err, cudaStream_t st) {
+                       int ldy, uint32_t* relu_bits, int ldbits, ErrRecord* err, cudaStream_t st) {
     using namespace tc;
     if (!tc::al16(bias) || !tc::al16(y_hi) || !tc::al16(y_lo) || ldy % 4) return DLRM_ERR_UNSUPPORTED;
     Maps3 m;
@@ -501,11 +559,16 @@ dlrm_status tf32x3_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b
         !operand_map(&m.b_hi, W.hi, false, N, K, W.ld) || !operand_map(&m.b_lo, W.lo, false, N, K, W.ld) ||
         !output_map(&m.c0, y_hi, M, N, ldy, 1) || !output_map(&m.c1, y_lo, M, N, ldy, 1))
         return DLRM_ERR_CUDA;
-    return launch3<false, false, E3_RELU_PAIR>(m, M, N, K, K, 1, bias, nullptr, nullptr, 0, err, st);
+    Epi3Args ea{};
+    ea.bias = bias;
+    ea.bits_out = relu_bits;
+    ea.ldbits = ldbits;
+    return launch3<false, false, E3_RELU_PAIR>(m, M, N, K, K, 1, ea, err, st);
 }
 
-dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mask, float* dx_hi, float* dx_lo,
-                         int lddx, ErrRecord* err, cudaStream_t st) {
+dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mask, const uint32_t* mask_bits,
+                         int ldbits, float* dx_hi, float* dx_lo, int lddx, float* csum, ErrRecord* err,
+                         cudaStream_t st) {
     // dx[m][k] = sum_n dy[m][n] W[n][k]; masked by (mask.hi + mask.lo > 0) when mask.hi is given
     // (a masked gradient is written as a (hi, lo) pair, an unmasked one plain)
     using namespace tc;
@@ -517,9 +580,17 @@ dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mas
         !output_map(&m.c0, dx_hi, M, K, lddx, 1) || (dx_lo && !output_map(&m.c1, dx_lo, M, K, lddx, 1)))
         return DLRM_ERR_CUDA;
     if (!dx_lo) m.c1 = m.c0;
-    if (mask.hi)
-        return launch3<false, true, E3_MASK_PAIR>(m, M, K, N, N, 1, nullptr, mask.hi, mask.lo, mask.ld, err, st);
-    return launch3<false, true, E3_PLAIN>(m, M, K, N, N, 1, nullptr, nullptr, nullptr, 0, err, st);
+    if (mask.hi) {
+        Epi3Args ea{};
+        ea.mhi = mask.hi;
+        ea.mlo = mask.lo;
+        ea.ldm = mask.ld;
+        ea.bits_in = mask_bits;
+        ea.ldbits = ldbits;
+        ea.csum = csum;
+        return launch3<false, true, E3_MASK_PAIR>(m, M, K, N, N, 1, ea, err, st);
+    }
+    return launch3<false, true, E3_PLAIN>(m, M, K, N, N, 1, Epi3Args{}, err, st);
 }
 
 int tf32x3_wgrad_splits(int N, int K, int M) {
@@ -566,13 +637,13 @@ dlrm_status tf32x3_gemm(int I, int J, int R, F32Pair A, bool a_mn, F32Pair Bm, b
     m.c1 = m.c0;
     dlrm_status r;
     if (a_mn && b_mn)
-        r = launch3<true, true, E3_PLAIN>(m, I, J, R, (int)chunk, S, nullptr, nullptr, nullptr, 0, err, st);
+        r = launch3<true, true, E3_PLAIN>(m, I, J, R, (int)chunk, S, Epi3Args{}, err, st);
     else if (a_mn)
-        r = launch3<true, false, E3_PLAIN>(m, I, J, R, (int)chunk, S, nullptr, nullptr, nullptr, 0, err, st);
+        r = launch3<true, false, E3_PLAIN>(m, I, J, R, (int)chunk, S, Epi3Args{}, err, st);
     else if (b_mn)
-        r = launch3<false, true, E3_PLAIN>(m, I, J, R, (int)chunk, S, nullptr, nullptr, nullptr, 0, err, st);
+        r = launch3<false, true, E3_PLAIN>(m, I, J, R, (int)chunk, S, Epi3Args{}, err, st);
     else
-        r = launch3<false, false, E3_PLAIN>(m, I, J, R, (int)chunk, S, nullptr, nullptr, nullptr, 0, err, st);
+        r = launch3<false, false, E3_PLAIN>(m, I, J, R, (int)chunk, S, Epi3Args{}, err, st);
     if (r || S == 1) return r;
     return launch_split_sum(S, I, J, scratch, ldp, C, ldc, st);
 }

@@ -67,10 +67,14 @@ struct F32Pair {
 
 // Tensor-core 3xTF32 GEMMs (gemm_tf32.cu); operands must be pairs.
 bool tf32x3_supported(int M, int N, int K, F32Pair a, F32Pair b);
+// relu_bits (optional): the output's ReLU bitmask, bit j % 32 of word [m][j / 32], ldbits words per row.
 dlrm_status tf32x3_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* bias, float* y_hi, float* y_lo,
-                       int ldy, ErrRecord* err, cudaStream_t st);
-dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mask, float* dx_hi, float* dx_lo,
-                         int lddx, ErrRecord* err, cudaStream_t st);
+                       int ldy, uint32_t* relu_bits, int ldbits, ErrRecord* err, cudaStream_t st);
+// mask_bits (optional): the saved activation's ReLU bitmask, read instead of the pair; csum (optional):
+// column sums of each 32-row group of the masked output, [ceil(M / 32)][K].
+dlrm_status tf32x3_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair mask, const uint32_t* mask_bits,
+                         int ldbits, float* dx_hi, float* dx_lo, int lddx, float* csum, ErrRecord* err,
+                         cudaStream_t st);
 int tf32x3_wgrad_splits(int N, int K, int M);
 size_t tf32x3_wgrad_scratch_floats(int N, int K, int M);
 dlrm_status tf32x3_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* scratch,
@@ -81,15 +85,23 @@ dlrm_status tf32x3_gemm(int I, int J, int R, F32Pair A, bool a_mn, F32Pair B, bo
 
 // CUDA-core fp32 GEMMs and helpers (train_gemm.cu). Inputs may be plain or
 // pairs; y_lo / dx_lo non-null selects a pair output.
+// ReLU bitmasks of saved activations: ceil(n / 32) words per row (bit j % 32 of word j / 32).
+inline int relu_bits_ld(int n) { return (n + 31) / 32; }
+
+// relu_bits (optional, with relu): the output's ReLU bitmask is written too.
 dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b, float* y, float* y_lo,
-                             int ldy, bool relu, ErrRecord* err, cudaStream_t st);
-// dx[m][k] = sum_n dy[m][n] W[n][k], zeroed where relu_of (post-ReLU value) <= 0 when relu_of.hi is given
-dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of, float* dx, float* dx_lo,
-                               int lddx, ErrRecord* err, cudaStream_t st);
+                             int ldy, bool relu, uint32_t* relu_bits, ErrRecord* err, cudaStream_t st);
+// dx[m][k] = sum_n dy[m][n] W[n][k], zeroed where relu_of (post-ReLU value) <= 0 when relu_of.hi is given;
+// relu_bits (optional) is relu_of's bitmask. If csum is given and *csum_done comes back true, csum holds
+// the column sums of dx per 32-row group ([ceil(M / 32)][K]) for the next layer's bias gradient.
+dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of,
+                               const uint32_t* relu_bits, float* dx, float* dx_lo, int lddx, float* csum,
+                               bool* csum_done, ErrRecord* err, cudaStream_t st);
 size_t train_wgrad_scratch_floats(int N, int K, int M);
-// dW[n][k] = sum_m dy[m][n] x[m][k]; db[n] = sum_m dy[m][n]
+// dW[n][k] = sum_m dy[m][n] x[m][k]; db[n] = sum_m dy[m][n] (from csum, the column sums of dy per
+// 32-row group, when given)
 dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* db,
-                               float* scratch, ErrRecord* err, cudaStream_t st);
+                               const float* csum, float* scratch, ErrRecord* err, cudaStream_t st);
 // hi/lo pair of a plain [rows][cols] matrix
 dlrm_status launch_split_pair(int rows, int cols, const float* src, int lds, float* hi, float* lo, int ldd,
                               cudaStream_t st);

@@ -283,6 +283,36 @@ __global__ void colsum_w_final_kernel(int P, int N, int NW, int kx, bool ones, c
     }
 }
 
+// bits[m][j / 32] bit j % 32 = (y(m, j) > 0), y plain or a pair: one warp per (row, 32 columns)
+__global__ void relu_bits_kernel(long long M, int N, const float* __restrict__ yh, const float* __restrict__ yl,
+                                 long long ldy, uint32_t* __restrict__ bits, long long ldbits) {
+    const int lane = threadIdx.x & 31;
+    const long long words = M * ldbits;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long q = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); q < words; q += warps) {
+        const long long m = q / ldbits;
+        const int j = (int)(q - m * ldbits) * 32 + lane;
+        bool pos = false;
+        if (j < N) pos = (yl ? yh[m * ldy + j] + yl[m * ldy + j] : yh[m * ldy + j]) > 0.f;
+        const uint32_t w = __ballot_sync(0xffffffffu, pos);
+        if (lane == 0) bits[q] = w;
+    }
+}
+
+// db[j] = sum over 32-row groups g of csum[g][j] in increasing g (one warp per column: lane l adds
+// g = l, l + 32, ... in order, then a fixed butterfly)
+__global__ void csum_final_kernel(int G, int J, const float* __restrict__ csum, float* __restrict__ db) {
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); j < J; j += warps) {
+        float s = 0.f;
+        for (int g = lane; g < G; g += 32) s += csum[(long long)g * J + j];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) db[j] = s;
+    }
+}
+
 // y[b][n] = act(sum_{k < K} x(b, k) W[n][k] + bias[n]) for K <= 16 (the 13 dense features): one thread
 // per output column with its weight row in registers; the block's rows of x are staged in shared memory
 // (read there as broadcasts), four rows per step; y written as a pair or plain.
@@ -291,7 +321,8 @@ __global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int
                                                          const float* __restrict__ xl, long long ldx,
                                                          const float* __restrict__ W, const float* __restrict__ Wl,
                                                          long long ldw, const float* __restrict__ bias, bool relu,
-                                                         float* __restrict__ yh, float* __restrict__ yl, long long ldy) {
+                                                         float* __restrict__ yh, float* __restrict__ yl, long long ldy,
+                                                         uint32_t* __restrict__ bits, long long ldbits) {
     __shared__ float xs[NARROW_ROWS][17];
     const long long rb = (long long)blockIdx.y * NARROW_ROWS;
     const int nr = (int)(M - rb < NARROW_ROWS ? M - rb : NARROW_ROWS);
@@ -302,11 +333,12 @@ __global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int
     }
     __syncthreads();
     const int n = blockIdx.x * 128 + threadIdx.x;
-    if (n >= N) return;
+    const bool active = n < N;   // inactive lanes stay for the bitmask ballots
     float wr[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) wr[k] = k < K ? (Wl ? W[n * ldw + k] + Wl[n * ldw + k] : W[n * ldw + k]) : 0.f;
-    const float bn = bias[n];
+    for (int k = 0; k < 16; ++k)
+        wr[k] = (active && k < K) ? (Wl ? W[n * ldw + k] + Wl[n * ldw + k] : W[n * ldw + k]) : 0.f;
+    const float bn = active ? bias[n] : 0.f;
     for (int r0 = 0; r0 < nr; r0 += 4) {
         float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -316,16 +348,22 @@ __global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int
                 for (int u = 0; u < 4; ++u) s[u] = fmaf(xs[r0 + u < nr ? r0 + u : r0][k], wr[k], s[u]);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            if (r0 + u >= nr) break;
+            if (r0 + u >= nr) break;   // uniform across the block
             float v = s[u] + bn;
             if (relu) v = v > 0.f ? v : 0.f;
             const long long o = (rb + r0 + u) * ldy + n;
-            if (yl) {
-                const float h = tf32_hi_part(v);
-                yh[o] = h;
-                yl[o] = v - h;
-            } else {
-                yh[o] = v;
+            if (active) {
+                if (yl) {
+                    const float h = tf32_hi_part(v);
+                    yh[o] = h;
+                    yl[o] = v - h;
+                } else {
+                    yh[o] = v;
+                }
+            }
+            if (bits) {
+                const uint32_t w = __ballot_sync(0xffffffffu, active && v > 0.f);
+                if ((threadIdx.x & 31) == 0 && n < N) bits[(rb + r0 + u) * ldbits + n / 32] = w;
             }
         }
     }
@@ -455,13 +493,15 @@ dlrm_status launch_colsum_w(int M, int N, F32Pair A, const float* X, int ldx, in
 }
 
 dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const float* b, float* y, float* y_lo,
-                             int ldy, bool relu, ErrRecord* err, cudaStream_t st) {
+                             int ldy, bool relu, uint32_t* relu_bits, ErrRecord* err, cudaStream_t st) {
     if (M == 0) return DLRM_OK;
+    if (!relu) relu_bits = nullptr;
     if (relu && y_lo && tf32x3_supported(M, N, K, x, W))
-        return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, err, st);
+        return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, relu_bits, relu_bits_ld(N), err, st);
     if (K <= 16) {
         const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + NARROW_ROWS - 1) / NARROW_ROWS));
-        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy);
+        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy,
+                                                relu_bits, relu_bits_ld(N));
         DLRM_LAUNCH_CHECK();
         return DLRM_OK;
     }
@@ -479,15 +519,28 @@ dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const fl
         gemm_f32_kernel<false, false, EPI_BIAS, false><<<grid_for(M, N, 1), 256, 0, st>>>(
             M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
     DLRM_LAUNCH_CHECK();
+    if (relu_bits) {
+        const long long words = (long long)M * relu_bits_ld(N);
+        relu_bits_kernel<<<grid_stride_blocks(words * 32), 256, 0, st>>>(M, N, y, y_lo, ldy, relu_bits,
+                                                                         relu_bits_ld(N));
+        DLRM_LAUNCH_CHECK();
+    }
     return DLRM_OK;
 }
 
-dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of, float* dx, float* dx_lo,
-                               int lddx, ErrRecord* err, cudaStream_t st) {
+dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pair relu_of,
+                               const uint32_t* relu_bits, float* dx, float* dx_lo, int lddx, float* csum,
+                               bool* csum_done, ErrRecord* err, cudaStream_t st) {
+    if (csum_done) *csum_done = false;
     if (M == 0) return DLRM_OK;
     const bool shape_ok = relu_of.hi ? (dx_lo && is_pair(relu_of)) : !dx_lo;
-    if (shape_ok && tf32x3_supported(M, K, N, dy, W))
-        return tf32x3_dgrad(M, N, K, dy, W, relu_of, dx, dx_lo, lddx, err, st);
+    if (shape_ok && tf32x3_supported(M, K, N, dy, W)) {
+        float* cs = relu_of.hi ? csum : nullptr;
+        dlrm_status r = tf32x3_dgrad(M, N, K, dy, W, relu_of, relu_of.hi ? relu_bits : nullptr, relu_bits_ld(K), dx,
+                                     dx_lo, lddx, cs, err, st);
+        if (!r && cs && csum_done) *csum_done = true;
+        return r;
+    }
     if (N == 1 && relu_of.hi && dx_lo && !dy.lo) {
         outer_mask_kernel<<<grid_stride_blocks((long long)M * K), 256, 0, st>>>(M, K, dy.hi, W.hi, W.lo, relu_of.hi,
                                                                                relu_of.lo, relu_of.ld, dx, dx_lo, lddx);
@@ -513,11 +566,18 @@ size_t train_wgrad_scratch_floats(int N, int K, int M) {
 }
 
 dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float* dW, int ldw, float* db,
-                               float* scratch, ErrRecord* err, cudaStream_t st) {
+                               const float* csum, float* scratch, ErrRecord* err, cudaStream_t st) {
     // dW[n][k] = sum_m dy[m][n] x[m][k]; db[n] = sum_m dy[m][n]
     if (N >= 16 && tf32x3_supported(N, K, M, dy, x)) {
         dlrm_status r = tf32x3_wgrad(M, N, K, dy, x, dW, ldw, scratch, err, st);
         if (r) return r;
+        if (csum) {
+            // bias gradient from the column sums per 32-row group that the data-gradient epilogue left
+            const int G = (M + 31) / 32;
+            csum_final_kernel<<<(N + 7) / 8 < 148 * 8 ? (N + 7) / 8 : 148 * 8, 256, 0, st>>>(G, N, csum, db);
+            DLRM_LAUNCH_CHECK();
+            return DLRM_OK;
+        }
         // bias gradient: fixed-order column sums of dy (the split partials above are consumed by now)
         return launch_colsum_w(M, N, dy, nullptr, 0, 0, true, nullptr, 0, db, scratch, st);
     }
