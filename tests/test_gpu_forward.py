@@ -20,6 +20,7 @@ def _cases():
         "tiny-ragged-mix": shrink(t, B=203).with_(bag="mix", seed=1),
         "medium-small": shrink(m, B=197, rows_cap=5000),
         "large-small": shrink(l, B=261, rows_cap=20000),
+        "large-batch3": shrink(l, B=3, rows_cap=2000),          # serving-size batch: small-batch layer kernel
         "stress-small": shrink(s, B=37, rows_cap=3000).with_(bag="uniform100"),
         "f16-d64-mix": shrink(m, B=77, rows_cap=700).with_(table_dtype="f16", mlp_dtype="f16", bag="mix"),
         "f32-d3-mix": shrink(t, B=45, rows_cap=50).with_(d=3, bag="mix", bottom=(13, 8, 3), top=(3 + 36, 16, 1)),

@@ -73,3 +73,27 @@ def test_linear_tc_two_layers_bf16_hidden(act):
     if act == E.ACT_SIGMOID:
         want = 1 / (1 + np.exp(-want))
     assert_close(to_np(out), want, "bf16", "two-layer bf16 MLP", scale_mlp(Ws, bs, xs, sigmoid=(act == E.ACT_SIGMOID)))
+
+
+# batches of at most 16 rows take the warp-per-column CUDA-core kernel (8 rows per block tile)
+@pytest.mark.parametrize("M,N,K", [(1, 256, 479), (5, 1024, 1024), (8, 40, 13), (16, 300, 200), (9, 64, 5)])
+@pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
+def test_linear_small_batch(M, N, K, dt):
+    if dt == "f32":
+        g = torch.Generator().manual_seed(M * 3 + N)
+        ld = E.dlrm_ld(K, "f32")
+        x = torch.zeros((M, ld))
+        x[:, :K] = torch.randn((M, K), generator=g)
+        W = torch.zeros((N, ld))
+        W[:, :K] = torch.randn((N, K), generator=g) / np.sqrt(K)
+        b = torch.randn(N, generator=g) * 0.1
+    else:
+        x, W, b, ld = _layer(M, N, K, dt, seed=M * 11 + N)
+    mlp = E.MLP([W.cuda()], [b.cuda()], [K, N])
+    out = torch.full((M, N), float("nan"), device="cuda")
+    ws = E.alloc_workspace(1 << 20)
+    E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, N, E.ACT_RELU, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    xs, Ws, bs = x[:, :K].double().numpy(), W[:, :K].double().numpy(), b.double().numpy()
+    want = O.mlp([Ws], [bs], xs, relu_last=True)
+    assert_close(to_np(out), want, "f32", f"small-batch linear {M}x{N}x{K} {dt}", scale_mlp([Ws], [bs], xs))
