@@ -4,9 +4,8 @@
 // "Output": a sigmoid on the top MLP's output).
 //
 // This file holds the CUDA-core paths: a tiled FFMA GEMM used for fp32
-// layers and for layers the tensor-core path does not take, a warp-per-column
-// kernel for batches of at most 16 rows, and a warp-per-row GEMV for the
-// single-logit last layer with its activation.
+// layers and for layers the tensor-core path does not take, and a
+// warp-per-row GEMV for the single-logit last layer with its activation.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -89,81 +88,6 @@ __global__ void __launch_bounds__(256) gemv_kernel(int M, int K, const TA* __res
     if (lane == 0) y[row * ldy] = activate<ACT>(s + bias[0]);
 }
 
-// Small batches (M <= 16, the latency-bound serving case): one warp per
-// output column reads its weight row once with 16-byte loads, for up to 8
-// rows of x staged in shared memory as fp32; blockIdx.y takes the next 8
-// rows. A weight matrix is read by all SMs at once instead of streaming
-// through the tile pipeline of the tensor-core kernel.
-constexpr int SKINNY_ROWS = 8;
-template <typename TA, typename TW, typename TC, int ACT>
-__global__ void __launch_bounds__(256) linear_skinny_kernel(int M, int N, int K, const TA* __restrict__ A, int lda,
-                                                            const TW* __restrict__ W, int ldw,
-                                                            const float* __restrict__ bias, TC* __restrict__ C,
-                                                            int ldc) {
-    extern __shared__ float xs[];   // [SKINNY_ROWS][K]
-    const int m0 = blockIdx.y * SKINNY_ROWS;
-    const int nm = min(SKINNY_ROWS, M - m0);
-    for (int q = threadIdx.x; q < SKINNY_ROWS * K; q += blockDim.x) {
-        const int m = q / K, k = q - m * K;
-        xs[q] = m < nm ? Cvt<TA>::to_f(A[(long long)(m0 + m) * lda + k]) : 0.f;
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (n >= N) return;
-    const TW* w = W + (long long)n * ldw;
-    float acc[SKINNY_ROWS];
-#pragma unroll
-    for (int m = 0; m < SKINNY_ROWS; ++m) acc[m] = 0.f;
-    for (int k0 = 8 * lane; k0 < K; k0 += 256) {
-        float wv[8];
-        if (k0 + 8 <= K) {
-            if constexpr (sizeof(TW) == 2) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(w + k0));
-                const TW* t = reinterpret_cast<const TW*>(&raw);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) wv[e] = Cvt<TW>::to_f(t[e]);
-            } else {
-                const float4 a = __ldg(reinterpret_cast<const float4*>(w + k0));
-                const float4 b = __ldg(reinterpret_cast<const float4*>(w + k0 + 4));
-                wv[0] = a.x, wv[1] = a.y, wv[2] = a.z, wv[3] = a.w, wv[4] = b.x, wv[5] = b.y, wv[6] = b.z, wv[7] = b.w;
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) wv[e] = k0 + e < K ? Cvt<TW>::to_f(w[k0 + e]) : 0.f;
-        }
-#pragma unroll
-        for (int m = 0; m < SKINNY_ROWS; ++m) {
-            const float* x = xs + m * K + k0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (k0 + e < K) acc[m] = fmaf(x[e], wv[e], acc[m]);
-        }
-    }
-#pragma unroll
-    for (int m = 0; m < SKINNY_ROWS; ++m)
-#pragma unroll
-        for (int o = 16; o; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
-    if (lane < nm) {
-        float v = 0.f;
-#pragma unroll
-        for (int m = 0; m < SKINNY_ROWS; ++m)
-            if (m == lane) v = acc[m];
-        C[(long long)(m0 + lane) * ldc + n] = Cvt<TC>::from_f(activate<ACT>(v + bias[n]));
-    }
-}
-
-template <typename TA, typename TW, typename TC, int ACT>
-static void run_skinny(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias, void* C,
-                       int ldc, cudaStream_t st) {
-    auto kern = linear_skinny_kernel<TA, TW, TC, ACT>;
-    const size_t smem = sizeof(float) * SKINNY_ROWS * (size_t)K;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const dim3 grid((N + 7) / 8, (M + SKINNY_ROWS - 1) / SKINNY_ROWS);
-    kern<<<grid, 256, smem, st>>>(M, N, K, static_cast<const TA*>(A), lda, static_cast<const TW*>(W), ldw, bias,
-                                  static_cast<TC*>(C), ldc);
-}
-
 template <typename TA, typename TW, typename TC, int ACT>
 static void run_ffma(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias, void* C,
                      int ldc, cudaStream_t st) {
@@ -180,20 +104,9 @@ static void run_gemv(int M, int K, const void* A, int lda, const void* W, const 
                                                           static_cast<const TW*>(W), bias, static_cast<float*>(C), ldc);
 }
 
-// layers the skinny kernel takes: a few rows, whose fp32 copy fits the shared memory, 16-byte weight rows
-static bool skinny_ok(int M, int K, int ldw, size_t w_es) {
-    return M <= 2 * SKINNY_ROWS && sizeof(float) * SKINNY_ROWS * (size_t)K <= 200 * 1024 && (ldw * w_es) % 16 == 0;
-}
-
 template <typename TA, typename TW, typename TC>
 static void dispatch_act(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias,
                          void* C, int ldc, int act, cudaStream_t st) {
-    if (skinny_ok(M, K, ldw, sizeof(TW)) && ((uintptr_t)W & 15) == 0) {
-        if (act == DLRM_ACT_RELU) run_skinny<TA, TW, TC, DLRM_ACT_RELU>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
-        else if (act == DLRM_ACT_SIGMOID) run_skinny<TA, TW, TC, DLRM_ACT_SIGMOID>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
-        else run_skinny<TA, TW, TC, DLRM_ACT_NONE>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
-        return;
-    }
     if (act == DLRM_ACT_RELU) run_ffma<TA, TW, TC, DLRM_ACT_RELU>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
     else if (act == DLRM_ACT_SIGMOID) run_ffma<TA, TW, TC, DLRM_ACT_SIGMOID>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
     else run_ffma<TA, TW, TC, DLRM_ACT_NONE>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
@@ -280,9 +193,7 @@ dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, i
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
                           ErrRecord* err, cudaStream_t st) {
     if (M == 0) return DLRM_OK;
-    // a handful of rows: the warp-per-column CUDA-core kernel beats the tensor-core pipeline's fill
-    const bool small = M <= 16 && N > 1;
-    if (!small && N > 1 && linear_tc_supported(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc))
+    if (N > 1 && linear_tc_supported(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc))
         return launch_linear_tc(M, N, K, A, a_dt, lda, W, ldw, bias, C, c_dt, ldc, act, err, st);
     return launch_linear_ffma(M, N, K, A, a_dt, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st);
 }

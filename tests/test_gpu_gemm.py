@@ -75,7 +75,7 @@ def test_linear_tc_two_layers_bf16_hidden(act):
     assert_close(to_np(out), want, "bf16", "two-layer bf16 MLP", scale_mlp(Ws, bs, xs, sigmoid=(act == E.ACT_SIGMOID)))
 
 
-# batches of at most 16 rows take the warp-per-column CUDA-core kernel (8 rows per block tile)
+# serving-size batches (a handful of rows) through the same layer path
 @pytest.mark.parametrize("M,N,K", [(1, 256, 479), (5, 1024, 1024), (8, 40, 13), (16, 300, 200), (9, 64, 5)])
 @pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
 def test_linear_small_batch(M, N, K, dt):
