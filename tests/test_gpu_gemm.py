@@ -97,3 +97,29 @@ def test_linear_small_batch(M, N, K, dt):
     xs, Ws, bs = x[:, :K].double().numpy(), W[:, :K].double().numpy(), b.double().numpy()
     want = O.mlp([Ws], [bs], xs, relu_last=True)
     assert_close(to_np(out), want, "f32", f"small-batch linear {M}x{N}x{K} {dt}", scale_mlp([Ws], [bs], xs))
+
+
+# the bottom-MLP shape (K0 <= 64 -> 512 -> 256 -> N3) runs as one fused tensor-core kernel
+@pytest.mark.parametrize("B", [1, 127, 300, 1000, 20000])
+@pytest.mark.parametrize("dt,n3", [("bf16", 128), ("f16", 64), ("bf16", 256)])
+def test_fused_bottom_mlp(B, dt, n3):
+    g = torch.Generator().manual_seed(B + n3)
+    dims = [13, 512, 256, n3]
+    Ws, bs, Wd, bd = [], [], [], []
+    for l in range(3):
+        K, N = dims[l], dims[l + 1]
+        W = torch.zeros((N, E.dlrm_ld(K, dt)), dtype=TD[dt])
+        W[:, :K] = (torch.randn((N, K), generator=g) * np.sqrt(2.0 / K)).to(TD[dt])
+        b = torch.randn(N, generator=g) * 0.1
+        Ws.append(W[:, :K].double().numpy())
+        bs.append(b.double().numpy())
+        Wd.append(W.cuda())
+        bd.append(b.cuda())
+    x = torch.randn((B, 13), generator=g).abs()   # dense features: log1p-like, non-negative
+    mlp = E.MLP(Wd, bd, dims)
+    out = torch.full((B, n3), float("nan"), device="cuda")
+    ws = E.alloc_workspace(1 << 24)
+    E.dlrm_mlp_fwd(mlp, B, x.cuda(), 13, out, n3, E.ACT_RELU, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    want = O.mlp(Ws, bs, x.double().numpy(), relu_last=True)
+    assert_close(to_np(out), want, "bf16", f"fused bottom MLP B={B} {dt} N3={n3}", scale_mlp(Ws, bs, x.double().numpy()))
