@@ -99,8 +99,6 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
 // tensor-core path.
 dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out, int ld_out,
                     int final_act, void* act0, void* act1, void* cvt, ErrRecord* err, cudaStream_t st) {
-    if (bottom_mlp_fused_supported(m, in_dt, out, ld_out, final_act))
-        return launch_bottom_mlp_fused(m, B, static_cast<const float*>(in), ld_in, out, ld_out, final_act, err, st);
     const void* cur = in;
     dlrm_dtype cur_dt = in_dt;
     int cur_ld = ld_in;

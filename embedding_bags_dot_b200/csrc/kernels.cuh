@@ -55,12 +55,6 @@ dlrm_status launch_embbag_cat(const TableMeta& tm, const void* tables, dlrm_dtyp
 // DLRM_U8ROW record bytes of a row of width d (quant.cu)
 size_t u8row_bytes(int d);
 
-// The whole bottom MLP (K0 <= 64 -> 512 -> 256 -> N3, 16-bit weights, fp32 in/out) in one
-// tensor-core kernel (mlp_fused.cu).
-bool bottom_mlp_fused_supported(const dlrm_mlp* m, dlrm_dtype in_dt, const void* out, int ld_out, int final_act);
-dlrm_status launch_bottom_mlp_fused(const dlrm_mlp* m, int B, const float* dense, int ldd, float* out, int ld_out,
-                                    int final_act, ErrRecord* err, cudaStream_t st);
-
 // ---- training (fp32)
 // An fp32 matrix row-major with leading dimension ld, held either plain
 // (lo == nullptr, value = hi) or as a 3xTF32 pair: hi = value with its 13 low

@@ -99,7 +99,7 @@ def test_linear_small_batch(M, N, K, dt):
     assert_close(to_np(out), want, "f32", f"small-batch linear {M}x{N}x{K} {dt}", scale_mlp([Ws], [bs], xs))
 
 
-# the bottom-MLP shape (K0 <= 64 -> 512 -> 256 -> N3) runs as one fused tensor-core kernel
+# the bottom-MLP shape (13 dense features -> 512 -> 256 -> N3) through dlrm_mlp_fwd, many batch sizes
 @pytest.mark.parametrize("B", [1, 127, 300, 1000, 20000])
 @pytest.mark.parametrize("dt,n3", [("bf16", 128), ("f16", 64), ("bf16", 256)])
 def test_fused_bottom_mlp(B, dt, n3):
