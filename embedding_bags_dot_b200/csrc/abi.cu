@@ -114,6 +114,11 @@ dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, 
         const int K = m->dims[l], N = m->dims[l + 1];
         const int ldw = dlrm_ld(K, m->dt);
         dlrm_status r;
+        // last hidden layer followed by the one-column sigmoid output: one kernel, the hidden output unstored
+        if (l == m->n_layers - 2 && m->dims[l + 2] == 1 && final_act == DLRM_ACT_SIGMOID && ld_out == 1 &&
+            linear_tc_logit_supported(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l]))
+            return launch_linear_tc_logit(B, N, K, cur, cur_dt, cur_ld, m->W[l], ldw, m->b[l], m->W[l + 1],
+                                          m->b[l + 1], out, err, st);
         if (l == m->n_layers - 1) {
             r = launch_linear(B, N, K, cur, cur_dt, cur_ld, m->W[l], m->dt, ldw, m->b[l], out, DLRM_F32, ld_out,
                               final_act, err, st);

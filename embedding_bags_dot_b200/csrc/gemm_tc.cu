@@ -187,11 +187,23 @@ __global__ void __launch_bounds__(THREADS, 1)
 // leader's full barrier; the MMA commits are multicast to both CTAs' empty and
 // accumulator-full barriers; both CTAs' epilogues release the accumulator on
 // the leader's barrier. Each CTA's TMEM holds the 128 rows of its M half.
+// ACT_RELU_LOGIT: the layer's ReLU output h (N <= 256, one tile wide) is not
+// stored; the epilogue forms the next, one-column layer instead:
+// y[m] = sigmoid(sum_j h[m][j] w[j] + b), one thread per row summing its
+// columns in order.
+constexpr int ACT_RELU_LOGIT = 16;
+template <typename TW>
+struct LogitArgs {
+    const TW* w;       // [N] weights of the one-column layer
+    const float* b;    // its bias (one float)
+    float* y;          // [M] output
+};
+
 template <typename TC, int ACT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     linear_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
                       const __grid_constant__ CUtensorMap mapC, int M, int N, int K, const float* __restrict__ bias,
-                      uint32_t id, ErrRecord* err) {
+                      uint32_t id, ErrRecord* err, LogitArgs<TC> la) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -324,8 +336,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             fence_after();
             const int mb = t / nbn, nb = t - mb * nbn;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2 + h * (BN2 / 2));
-            epilogue_tma<TC, ACT, BN2 / 2>(taddr, mb * 256 + (int)rank * 128 + q * 32, nb * BN2 + h * (BN2 / 2), N,
-                                           bias, &mapC, stage, stage_s);
+            if constexpr (ACT == ACT_RELU_LOGIT) {
+                // the first warp of each lane quadrant reads all N <= 256 columns of its 32 rows (the same TMEM
+                // lanes as its partner); the partner only releases the accumulator
+                if (h == 0) {
+                    const uint32_t row_addr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2);
+                    float part = 0.f;
+#pragma unroll 1
+                    for (int c = 0; c < BN2 / 32; ++c) {
+                        const int j0 = 32 * c;
+                        if (j0 >= N) break;   // uniform across the warp
+                        uint32_t r[32];
+                        tmem_ld32_issue(row_addr + 32 * c, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (j0 + e < N) {
+                                const float v = fmaxf(__uint_as_float(r[e]) + __ldg(bias + j0 + e), 0.f);
+                                part = fmaf(v, Cvt<TC>::to_f(la.w[j0 + e]), part);
+                            }
+                        }
+                    }
+                    const long long row = (long long)mb * 256 + (int)rank * 128 + q * 32 + lane;
+                    if (row < M) la.y[row] = 1.f / (1.f + expf(-(part + __ldg(la.b))));
+                }
+            } else {
+                epilogue_tma<TC, ACT, BN2 / 2>(taddr, mb * 256 + (int)rank * 128 + q * 32, nb * BN2 + h * (BN2 / 2),
+                                               N, bias, &mapC, stage, stage_s);
+            }
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? lead_tempty1 : lead_tempty0);
@@ -401,18 +439,43 @@ static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const 
 
 template <typename TC, int ACT>
 static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc, int M, int N, int K,
-                             const float* bias, uint32_t id, ErrRecord* err, cudaStream_t st) {
+                             const float* bias, uint32_t id, ErrRecord* err, cudaStream_t st,
+                             LogitArgs<TC> la = LogitArgs<TC>{nullptr, nullptr, nullptr}) {
     auto kern = linear_tc2_kernel<TC, ACT>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
     const int ntiles = ((M + 255) / 256) * ((N + BN2 - 1) / BN2);
     const int pairs = sm_count() / 2;
     const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err);
+    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err, la);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
 
 }  // namespace tc
+
+bool linear_tc_logit_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                               dlrm_dtype w_dt, int ldw, const float* bias) {
+    // the SM-pair kernel (M >= 4096) with the whole layer output in one 256-wide tile
+    if (M < 256 * 16 || N > tc::BN2) return false;
+    if (a_dt != w_dt || a_dt == DLRM_F32 || N < 2 || K < 1 || (lda % 8) || (ldw % 8)) return false;
+    if (((uintptr_t)A & 15) || ((uintptr_t)W & 15) || ((uintptr_t)bias & 15)) return false;
+    return tc::encode_fn() != nullptr;
+}
+
+dlrm_status launch_linear_tc_logit(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                                   int ldw, const float* bias, const void* w_next, const float* b_next, float* y,
+                                   ErrRecord* err, cudaStream_t st) {
+    CUtensorMap ma, mw;
+    if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) || !tc::make_map(&mw, W, a_dt, K, N, ldw, tc::BN2 / 2))
+        return DLRM_ERR_CUDA;
+    const int fmt = a_dt == DLRM_BF16 ? 1 : 0;
+    if (a_dt == DLRM_BF16)
+        return tc::launch_t2<__nv_bfloat16, tc::ACT_RELU_LOGIT>(
+            ma, mw, mw, M, N, K, bias, tc::idesc2(fmt), err, st,
+            tc::LogitArgs<__nv_bfloat16>{static_cast<const __nv_bfloat16*>(w_next), b_next, y});
+    return tc::launch_t2<__half, tc::ACT_RELU_LOGIT>(ma, mw, mw, M, N, K, bias, tc::idesc2(fmt), err, st,
+                                                     tc::LogitArgs<__half>{static_cast<const __half*>(w_next), b_next, y});
+}
 
 bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, dlrm_dtype w_dt,
                          int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc) {

@@ -55,6 +55,14 @@ dlrm_status launch_embbag_cat(const TableMeta& tm, const void* tables, dlrm_dtyp
 // DLRM_U8ROW record bytes of a row of width d (quant.cu)
 size_t u8row_bytes(int d);
 
+// A hidden ReLU layer (N <= 256, M >= 4096, 16-bit) whose output feeds a one-column layer with a
+// sigmoid: y[m] = sigmoid(relu(A W^T + bias)[m] . w_next + b_next), the hidden output never stored.
+bool linear_tc_logit_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                               dlrm_dtype w_dt, int ldw, const float* bias);
+dlrm_status launch_linear_tc_logit(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
+                                   int ldw, const float* bias, const void* w_next, const float* b_next, float* y,
+                                   ErrRecord* err, cudaStream_t st);
+
 // ---- training (fp32)
 // An fp32 matrix row-major with leading dimension ld, held either plain
 // (lo == nullptr, value = hi) or as a 3xTF32 pair: hi = value with its 13 low

@@ -123,3 +123,33 @@ def test_fused_bottom_mlp(B, dt, n3):
     assert E.dlrm_check_error(ws)[0] == 0
     want = O.mlp(Ws, bs, x.double().numpy(), relu_last=True)
     assert_close(to_np(out), want, "bf16", f"fused bottom MLP B={B} {dt} N3={n3}", scale_mlp(Ws, bs, x.double().numpy()))
+
+
+# at 4096+ rows the last hidden layer (width <= 256) and the one-column sigmoid output run as one kernel
+@pytest.mark.parametrize("B,h,dt", [(4096, 256, "bf16"), (5000, 200, "bf16"), (4100, 256, "f16"), (3000, 256, "bf16")])
+def test_last_hidden_layer_with_logit(B, h, dt):
+    g = torch.Generator().manual_seed(B + h)
+    dims = [479, 512, h, 1]
+    Ws, bs, Wd, bd = [], [], [], []
+    for l in range(3):
+        K, N = dims[l], dims[l + 1]
+        W = torch.zeros((N, E.dlrm_ld(K, dt)), dtype=TD[dt])
+        W[:, :K] = (torch.randn((N, K), generator=g) * np.sqrt(2.0 / K)).to(TD[dt])
+        b = torch.randn(N, generator=g) * 0.1
+        Ws.append(W[:, :K].double().numpy())
+        bs.append(b.double().numpy())
+        Wd.append(W.cuda())
+        bd.append(b.cuda())
+    ld = E.dlrm_ld(479, dt)
+    x = torch.zeros((B, ld), dtype=TD[dt])
+    x[:, :479] = torch.randn((B, 479), generator=g).to(TD[dt])
+    mlp = E.MLP(Wd, bd, dims)
+    y = torch.full((B, 1), float("nan"), device="cuda")
+    ws = E.alloc_workspace(1 << 26)
+    E.dlrm_mlp_fwd(mlp, B, x.cuda(), ld, y, 1, E.ACT_SIGMOID, ws)
+    assert E.dlrm_check_error(ws)[0] == 0
+    xs = x[:, :479].double().numpy()
+    z = O.mlp(Ws, bs, xs, relu_last=False)
+    want = 1 / (1 + np.exp(-z))
+    assert_close(to_np(y), want, "bf16", f"last hidden layer + logit B={B} h={h} {dt}",
+                 scale_mlp(Ws, bs, xs, sigmoid=True))
