@@ -13,11 +13,13 @@
 //     row per lane. A one-row bag is copied global -> shared with cp.async,
 //     so every row of the sample is in flight at once without registers;
 //     a bag of several rows is summed in fp32 and rounded to bf16.
-//     Row-wise uint8 tables (Q): a one-row bag's record (d codes, fp32 scale,
-//     fp32 offset) is copied the same way, unswizzled, into the first bytes of
+//     Row-wise uint8 tables (Q), a sample with a bag of several rows (or a
+//     non-finite x_dense): a one-row bag's record (d codes, fp32 scale s, fp32
+//     offset m) is copied the same way, unswizzled, into the first bytes of
 //     its X row slot; once it has landed each lane reads its 8 codes and the
 //     scale/offset, the warp synchronises, and the lane writes the dequantised
 //     values (s q + m, rounded to bf16) as its swizzled 16-byte chunk.
+//     Every other uint8 sample takes the integer route (5. below).
 //  2. x_dense (fp32) is split into hi = bf16(x) and lo = bf16(x - hi); hi is
 //     row 0 of X and lo row K+1, so that Z_i0 = G[i][0] + G[K+1][i] keeps the
 //     dense vector's fp32 precision.
@@ -28,6 +30,19 @@
 //  4. G is staged in shared memory, the x_dense low-half terms are folded into
 //     column 0, and each lane writes fixed 8-column chunks of the concat row
 //     whose sources in G are computed once per block.
+//  5. Row-wise uint8 tables, samples whose bags hold at most one row: the
+//     codes are never converted. Each bag's d codes go by cp.async straight
+//     into row 1+k of an 8-bit tile, its (s, m) into a per-row slot; row 0 is
+//     all ones; x_dense is quantised per sample to 24 bits,
+//     x ~ sx qx + mn with qx = 65536 h + 256 u + l, and its three byte planes
+//     are rows K+1..K+3. One u8 x u8 -> s32 Gram on the tensor cores
+//     (mma.sync m16n8k32) then holds, exactly, every <q_i, q_j>, the code sums
+//     S_i = <q_i, 1> and the plane products. With e_i = s_i q_i + m_i,
+//       Z_ij = s_i s_j <q_i, q_j> + s_i S_i m_j + s_j S_j m_i + d m_i m_j,
+//     and the same with (sx, mn, <q_i, qx>, sum qx) for the x_dense column;
+//     the affine terms are applied in fp32 while the concat row is written.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -61,6 +76,14 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -90,7 +113,177 @@ __device__ __forceinline__ void dequant8(uint2 codes, float sc, float of, float 
     }
 }
 
-// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2). GL: lanes per row (d = 8 GL). Q: row-wise uint8 tables.
+// Layout of a warp's region on the integer route: KP+1 16-byte row slots
+// (s, m, s S, 0) -- slot 0 for x_dense, slots 1..K for the bags, slot KP all
+// zero for padding columns -- then the 8-bit tile X8 (KP rows of d bytes),
+// which the staged Gram (fp32, row stride KP + 8) overwrites after the MMAs.
+
+// One sample on the integer route: bags of at most one row, finite x_dense
+// (minimum mn, range = max - mn). Writes the whole concat row.
+template <int MT, int GL>
+__device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, const uint32_t* code_k, int K,
+                                          const unsigned char* __restrict__ qtab, const float4* xv, float mn,
+                                          float range, const uint32_t (&srcr)[SRC_CACHE][4], const uint16_t* src_s,
+                                          int nzc, const float* __restrict__ xrow, void* out, size_t row0, int ld,
+                                          int out_dt, int lane) {
+    constexpr int d = 8 * GL;
+    constexpr int KP = 16 * MT;
+    constexpr int GS = KP + 8;
+    constexpr int CH = d / 16;               // 16-byte chunks of an 8-bit row
+    constexpr int NG8 = 32 / CH;             // rows per round of the gather
+    constexpr int QRB = (d + 8 + 15) / 16 * 16;
+    constexpr int NTILE = MT * (MT + 1);
+    constexpr uint32_t ZERO_SLOT = KP * GS;
+    constexpr int X8 = (KP + 1) * 16;     // start of the 8-bit tile
+    // 128-byte rows: chunk c of row r at c ^ (r & 7); 64-byte rows: c ^ ((r >> 1) & 3). Either way the
+    // 8 rows an ldmatrix reads fall in 8 distinct 16-byte bank groups.
+    auto xoff8 = [](int r, int c) { return X8 + r * d + 16 * (d == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3))); };
+    float4* meta = reinterpret_cast<float4*>(xw);
+    float* G = reinterpret_cast<float*>(xw + X8);
+    const int P0 = K + 1;                    // x_dense byte planes: P0 (weight 1), P0+1 (256), P0+2 (65536)
+
+    // codes of the one-row bags, row 1+k; their (s, m) into slot 1+k; empty bags are all zero
+    {
+        const int gi = lane / CH, g = lane % CH;
+        for (int k = gi; k < K; k += NG8) {
+            const uint32_t code = code_k[k * S];
+            if (code < CODE_MULTI)
+                cp_async16(xw_s + (uint32_t)xoff8(k + 1, g), qtab + (long long)code * QRB + 16 * g);
+            else
+                *reinterpret_cast<uint4*>(xw + xoff8(k + 1, g)) = make_uint4(0, 0, 0, 0);
+        }
+        for (int k = lane; k < K; k += 32) {
+            const uint32_t code = code_k[k * S];
+            if (code < CODE_MULTI)
+                cp_async16(xw_s + 16u * (uint32_t)(k + 1), qtab + (long long)code * QRB + d);
+            else
+                meta[k + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    // row 0: ones; rows K+4 .. KP-1: zero; slot KP: zero
+    if (lane < CH) *reinterpret_cast<uint4*>(xw + xoff8(0, lane)) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+    for (int q = lane; q < (KP - K - 4) * CH; q += 32)
+        reinterpret_cast<uint4*>(xw + X8 + (K + 4) * d)[q] = make_uint4(0, 0, 0, 0);
+    if (lane == 0) meta[KP] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // x_dense -> 24-bit codes qx = rint((x - mn) / sx), sx = range / (2^24 - 1), as three byte planes
+    constexpr float QMAX = 16777215.f;
+    const float inv = range > 0.f ? QMAX / range : 0.f;
+    const float sx = range / QMAX;
+#pragma unroll
+    for (int q = 0; q < (d + 127) / 128; ++q) {
+        const int c = 4 * lane + 128 * q;
+        if (c < d) {
+            const float4 x = xv[q];
+            uint32_t qv[4];
+            qv[0] = (uint32_t)fminf(rintf((x.x - mn) * inv), QMAX);
+            qv[1] = (uint32_t)fminf(rintf((x.y - mn) * inv), QMAX);
+            qv[2] = (uint32_t)fminf(rintf((x.z - mn) * inv), QMAX);
+            qv[3] = (uint32_t)fminf(rintf((x.w - mn) * inv), QMAX);
+            const uint32_t lo01 = __byte_perm(qv[0], qv[1], 0x0040), lo23 = __byte_perm(qv[2], qv[3], 0x0040);
+            const uint32_t mi01 = __byte_perm(qv[0], qv[1], 0x0051), mi23 = __byte_perm(qv[2], qv[3], 0x0051);
+            const uint32_t hi01 = __byte_perm(qv[0], qv[1], 0x0062), hi23 = __byte_perm(qv[2], qv[3], 0x0062);
+            const int ch = c / 16, byte = c % 16;
+            *reinterpret_cast<uint32_t*>(xw + xoff8(P0, ch) + byte) = __byte_perm(lo01, lo23, 0x5410);
+            *reinterpret_cast<uint32_t*>(xw + xoff8(P0 + 1, ch) + byte) = __byte_perm(mi01, mi23, 0x5410);
+            *reinterpret_cast<uint32_t*>(xw + xoff8(P0 + 2, ch) + byte) = __byte_perm(hi01, hi23, 0x5410);
+        }
+    }
+    cp_async_wait_all();
+    __syncwarp();
+
+    // exact integer Gram of the lower-triangle tiles
+    int acc[NTILE][4];
+#pragma unroll
+    for (int t = 0; t < NTILE; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0;
+#pragma unroll
+    for (int ks = 0; ks < d / 32; ++ks) {
+        uint32_t a[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+            ldmatrix_x4(xw_s + (uint32_t)xoff8(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a[mt]);
+        int t = 0;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+            for (int nt = 0; nt <= 2 * mt + 1; ++nt, ++t)
+                mma_u8(acc[t], a[mt], a[nt >> 1][(nt & 1) ? 1 : 0], a[nt >> 1][(nt & 1) ? 3 : 2]);
+        }
+    }
+    __syncwarp();  // every lane's ldmatrix of X8 is done before G overwrites it
+
+    // stage G in fp32 (every entry is below 2^24, so exact)
+    {
+        const int gr = lane >> 2, tc = (lane & 3) * 2;
+        int t = 0;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+            for (int nt = 0; nt <= 2 * mt + 1; ++nt, ++t) {
+                float* p0 = G + (16 * mt + gr) * GS + 8 * nt + tc;
+                *reinterpret_cast<float2*>(p0) = make_float2((float)acc[t][0], (float)acc[t][1]);
+                *reinterpret_cast<float2*>(p0 + 8 * GS) = make_float2((float)acc[t][2], (float)acc[t][3]);
+            }
+        }
+        if (lane == 0) G[ZERO_SLOT] = 0.f;
+    }
+    __syncwarp();
+    // per bag: slot (s, m, s S); column 0 of its Gram row becomes <q_i, qx>
+    const float* Gx0 = G + P0 * GS;
+    for (int i = 1 + lane; i <= K; i += 32) {
+        const float S_i = G[i * GS];
+        G[i * GS] = fmaf(65536.f, Gx0[2 * GS + i], fmaf(256.f, Gx0[GS + i], Gx0[i]));
+        const float4 sm = meta[i];
+        meta[i] = make_float4(sm.x, sm.y, sm.x * S_i, 0.f);
+    }
+    if (lane == 0) {
+        const float Sx = fmaf(65536.f, Gx0[2 * GS], fmaf(256.f, Gx0[GS], Gx0[0]));
+        meta[0] = make_float4(sx, mn, sx * Sx, 0.f);
+    }
+    __syncwarp();
+
+    // Z for the Gram entry at `src`: s_i s_j g + t_i m_j + t_j m_i + d m_i m_j
+    auto zval = [&](uint32_t src) {
+        const int i = (int)(src / GS), j = (int)(src - (uint32_t)i * GS);
+        const float4 a = meta[i], c = meta[j];
+        return fmaf(a.x * c.x, G[src], fmaf(a.z, c.y, fmaf(c.z, a.y, (float)d * a.y * c.y)));
+    };
+    if (out_dt == DLRM_BF16) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out) + row0;
+        uint4* zrow = reinterpret_cast<uint4*>(orow) + d / 8;
+#pragma unroll
+        for (int q = 0; q < (d + 127) / 128; ++q) {
+            const int c = 4 * lane + 128 * q;
+            if (c < d) {
+                const float4 x = xv[q];
+                reinterpret_cast<uint2*>(orow)[c / 4] = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < SRC_CACHE; ++j) {
+            const int c8 = lane + 32 * j;
+            if (c8 < nzc) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = zval((srcr[j][e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
+                zrow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                      pack_bf16(f[6], f[7]));
+            }
+        }
+        for (int c8 = lane + 32 * SRC_CACHE; c8 < nzc; c8 += 32) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = zval(src_s[8 * c8 + e]);
+            zrow[c8] = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                                  pack_bf16(f[6], f[7]));
+        }
+    } else {
+        for (int c = lane; c < ld; c += 32) store_as(out, row0 + c, c < d ? xrow[c] : zval(src_s[c - d]), out_dt);
+    }
+    __syncwarp();  // the region is reused by the next sample
+}
+
+// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2; K + 4 with Q). GL: lanes per row (d = 8 GL).
+// Q: row-wise uint8 tables.
 template <int MT, int GL, bool Q>
 __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_mma_kernel(
     const void* __restrict__ tables_v, const __grid_constant__ TableMeta tm, int K, int B,
@@ -179,6 +372,33 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         for (int q = 0; q < (d + 127) / 128; ++q) {
             const int c = 4 * lane + 128 * q;
             xv[q] = c < d ? *reinterpret_cast<const float4*>(x_dense + b * d + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+
+        if constexpr (Q) {
+            // ---- 5. integer route, unless a bag holds several rows or x_dense is not finite
+            float mn = INFINITY, mx = -INFINITY;
+            bool slow = false;
+#pragma unroll
+            for (int q = 0; q < (d + 127) / 128; ++q) {
+                if (4 * lane + 128 * q < d) {
+                    const float4 x = xv[q];
+                    mn = fminf(fminf(mn, x.x), fminf(x.y, fminf(x.z, x.w)));
+                    mx = fmaxf(fmaxf(mx, x.x), fmaxf(x.y, fmaxf(x.z, x.w)));
+                    slow |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+                }
+            }
+            for (int k = lane; k < K; k += 32) slow |= code_s[k * S + s] == CODE_MULTI;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            const float range = mx - mn;
+            if (!__any_sync(0xffffffffu, slow) && isfinite(range)) {
+                u8_sample<MT, GL>(xw, xw_s, code_s + s, K, qtab, xv, mn, range, srcr, src_s, nzc, x_dense + b * d,
+                                  out, (size_t)b * ld, ld, out_dt, lane);
+                continue;
+            }
         }
 
         // ---- 1. gather: X rows 1..K
@@ -340,17 +560,20 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
 
 // ------------------------------------------------------------------ host side
 
-static int mma_warp_bytes(int K, int d, int& MT) {
-    MT = (K + 2 + 15) / 16;
+// Bytes of a warp's region: the bf16 tile or its staged Gram, and for uint8 tables (q) also the integer
+// route's row slots plus its 8-bit tile or staged Gram.
+static int mma_warp_bytes(int K, int d, bool q, int& MT) {
+    MT = (K + (q ? 4 : 2) + 15) / 16;
     const int KP = 16 * MT;
     const int RS = d >= 64 ? 2 * d : 2 * d + 16;
-    const int x = KP * RS;
-    const int gbytes = RS + (KP * (KP + 8) + 1) * 4;
-    return ((x > gbytes ? x : gbytes) + 15) & ~15;
+    const int gf = (KP * (KP + 8) + 1) * 4;
+    int bytes = std::max(KP * RS, RS + gf);
+    if (q) bytes = std::max(bytes, (KP + 1) * 16 + std::max(KP * d, gf));
+    return (bytes + 15) & ~15;
 }
 
-static size_t mma_smem(int K, int d, int ld, int& MT, int& warp_bytes) {
-    warp_bytes = mma_warp_bytes(K, d, MT);
+static size_t mma_smem(int K, int d, bool q, int ld, int& MT, int& warp_bytes) {
+    warp_bytes = mma_warp_bytes(K, d, q, MT);
     return (size_t)WARPS * warp_bytes + sizeof(uint32_t) * (size_t)K * S + sizeof(uint16_t) * (size_t)(ld - d + 8);
 }
 
@@ -359,14 +582,14 @@ bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const vo
     if (dt != DLRM_BF16 && dt != DLRM_U8ROW) return false;
     if (!(d == 32 || d == 64 || d == 128 || d == 256)) return false;
     if (dt == DLRM_U8ROW && !(d == 64 || d == 128)) return false;
-    if (K + 2 > 64) return false;
+    if (K + (dt == DLRM_U8ROW ? 4 : 2) > 64) return false;
     if (total_rows >= (long long)CODE_MULTI) return false;
     if (out_dt == DLRM_BF16 && (ld % 8 || ((uintptr_t)out & 15))) return false;
     if (ld - d > 8 * 0x1FFF) return false;
     const int P = K * (K + 1) / 2;
     if (P + d > ld || ld > 0x7FFF) return false;
     int MT, wb;
-    return mma_smem(K, d, ld, MT, wb) <= 227 * 1024;
+    return mma_smem(K, d, dt == DLRM_U8ROW, ld, MT, wb) <= 227 * 1024;
 }
 
 template <int MT, int GL, bool Q>
@@ -384,8 +607,8 @@ dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, 
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st) {
     int MT, wb;
-    const size_t smem = mma_smem(K, d, ld, MT, wb);
     const bool q = dt == DLRM_U8ROW;
+    const size_t smem = mma_smem(K, d, q, ld, MT, wb);
 #define DLRM_MMA_GL(MTV)                                                                                       \
     switch (d) {                                                                                               \
         case 32: launch_mma_t<MTV, 4, false>(tm, tables, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt, wb, smem, err, st); break;   \

@@ -70,7 +70,7 @@ def test_forward_and_fused_concat(name):
     assert counts == (0, 0)
     assert_close(y, want, "u8row", f"{name} y_hat")
     # the fused kernel alone, bf16 concat
-    x = np.random.default_rng(1).standard_normal((cfg.B, cfg.d)).astype(np.float32)
+    x = _dense_with_edge_rows(cfg.B, cfg.d, 1)
     ld = E.dlrm_ld(cfg.concat_width, "bf16")
     out = torch.full((cfg.B, ld), float("nan"), dtype=torch.bfloat16, device="cuda")
     E.dlrm_embbag_interact_fwd(g.T, cfg.B, bt["offsets"], bt["indices"], torch.from_numpy(x).cuda(), out, ld, "bf16",
@@ -86,6 +86,64 @@ def test_forward_and_fused_concat(name):
     assert_close(got[:, :cfg.concat_width], want_c, "u8row", f"{name} concat", scale_concat(x, pooled_s))
     assert np.all(got[:, cfg.concat_width:] == 0)
     del base, rows
+
+
+def _dense_with_edge_rows(B, d, seed):
+    """Normal x_dense plus rows the per-sample 24-bit quantisation of x_dense must handle:
+    constant rows (range 0), all-zero rows and rows with one large outlier."""
+    x = np.random.default_rng(seed).standard_normal((B, d)).astype(np.float32)
+    x[::5] = 0.5
+    x[1::7] = 0.0
+    x[2::11, 3] = 1.0e4
+    x[3::13] = np.abs(x[3::13]) + 100.0
+    return x
+
+
+def _empty_bags(offsets, indices, K, B, pred):
+    """The CSR batch with every bag (k, b) for which pred(k, b) holds emptied."""
+    lens = np.diff(offsets.astype(np.int64))
+    keep = np.ones(len(indices), bool)
+    for k in range(K):
+        for b in range(B):
+            if pred(k, b):
+                q = k * B + b
+                keep[offsets[q]:offsets[q + 1]] = False
+                lens[q] = 0
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32), indices[keep].copy()
+
+
+@pytest.mark.parametrize("name", ["u8-d128-onehot", "u8-d64-onehot"])
+def test_integer_route_fp32_concat_is_tight(name):
+    """One-row bags take the integer route: exact u8 x u8 Gram, fp32 affine terms, 24-bit x_dense. With an
+    fp32 concat (no bf16 rounding of the output) the error has two sources: x_dense quantised to 24 bits of
+    its per-sample range (at most ~1.5 range 2^-24 per element) and the fp32 rounding of the affine terms,
+    which are as large as sum |e - m| |x - min x|. On ordinary rows both stay below 1e-5 of the magnitude
+    scale sum |e_i| |x_j|; a row with one x_dense element 1e4 times the rest, met by an embedding element
+    near zero, reaches a few 1e-5, so those rows get 1e-4. The dequantising route (bf16 rows) is at ~2e-3."""
+    cfg = CASES["u8-d128-onehot"] if name == "u8-d128-onehot" else shrink(
+        CONFIGS["medium"], B=211, rows_cap=3000).with_(table_dtype="u8row", mlp_dtype="bf16", bag="one", seed=8)
+    batch = gen.make_batches(cfg, (0,))[0]
+    # some bags emptied: tables 0, 5, 10, ... for every third sample
+    offs, idx = _empty_bags(batch.offsets, batch.indices, cfg.K, cfg.B, lambda k, b: k % 5 == 0 and b % 3 == 0)
+    g = GpuModel(cfg)
+    x = _dense_with_edge_rows(cfg.B, cfg.d, 2)
+    ld = E.dlrm_ld(cfg.concat_width, "f32")
+    out = torch.full((cfg.B, ld), float("nan"), dtype=torch.float32, device="cuda")
+    E.dlrm_embbag_interact_fwd(g.T, cfg.B, torch.from_numpy(offs).cuda(), torch.from_numpy(idx).cuda(),
+                               torch.from_numpy(x).cuda(), out, ld, "f32", g.ws)
+    assert E.dlrm_check_error(g.ws)[0] == 0
+    model = O.model_from_config(cfg)
+    pooled, _, _ = O.embbag(model.tables, np.asarray(cfg.rows, np.int64), cfg.d, cfg.B, offs, idx)
+    pooled_s = O.embbag(np.abs(model.tables), np.asarray(cfg.rows, np.int64), cfg.d, cfg.B, offs, idx)[0]
+    want = O.interact(x, pooled)
+    scale = scale_concat(x, pooled_s)
+    got = to_np(out)[:, :cfg.concat_width]
+    rel = np.abs(got - want) / (scale + 1e-300)
+    outlier = np.zeros(cfg.B, bool)
+    outlier[2::11] = True
+    worst = (float(rel[~outlier].max()), float(rel[outlier].max()))
+    assert worst[0] <= 1e-5 and worst[1] <= 1e-4, f"{name}: worst of scale, ordinary/outlier rows {worst}"
+    assert np.all(to_np(out)[:, cfg.concat_width:] == 0)
 
 
 def test_invalid_bags_and_unsupported_entry_points():
