@@ -55,6 +55,7 @@ _SIGS = {
     "dlrm_ld": (C.c_int, [C.c_int, C.c_int]),
     "dlrm_status_str": (C.c_char_p, [C.c_int]),
     "dlrm_workspace_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
+    "dlrm_mlp_workspace_size": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
     "dlrm_check_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_embbag_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
                                   C.c_void_p, C.c_void_p]),
@@ -195,6 +196,20 @@ def dlrm_workspace_size(T: Tables, bot: MLP, top: MLP, B: int, training: int = 0
     return int(lib().dlrm_workspace_size(_ref(T), _ref(bot), _ref(top), int(B), int(training)))
 
 
+def dlrm_mlp_workspace_size(mlp: MLP, B: int, in_dt) -> int:
+    return int(lib().dlrm_mlp_workspace_size(mlp.ref(), int(B), int(DT_CODE.get(in_dt, in_dt))))
+
+
+def _need_ws(ws, nbytes: int, where: str) -> None:
+    """The C entry points cannot see the workspace's size: refuse a tensor smaller than the call needs
+    before anything is launched. A size of 0 (the query found the arguments invalid) leaves the
+    diagnosis to the entry point itself."""
+    if not isinstance(ws, torch.Tensor) or nbytes <= 0:
+        return
+    if ws.numel() * ws.element_size() < nbytes:
+        raise DlrmError(ERR_WORKSPACE, where)
+
+
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """Zero-filled workspace (the error record must start at zero)."""
     return torch.zeros(max(int(nbytes), ERR_RECORD_BYTES), dtype=torch.uint8, device=device)
@@ -208,6 +223,7 @@ def dlrm_check_error(ws: torch.Tensor, stream=None):
 
 
 def dlrm_embbag_fwd(T: Tables, B: int, offsets, indices, pooled, bag_len=None, ws=None, stream=None):
+    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_fwd")
     return _check(lib().dlrm_embbag_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
                                         _ptr(pooled), _ptr(bag_len), _ptr(ws), _stream(stream)), "dlrm_embbag_fwd")
 
@@ -221,17 +237,20 @@ def dlrm_interact_fwd(B: int, K: int, d: int, x_dense, pooled, concat, ld: int, 
 def dlrm_embbag_interact_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,
                              stream=None):
     out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
+    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_interact_fwd")
     return _check(lib().dlrm_embbag_interact_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
                                                  _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
                                                  _stream(stream)), "dlrm_embbag_interact_fwd")
 
 
 def dlrm_mlp_fwd(mlp: MLP, B: int, inp, ld_in: int, out, ld_out: int, final_act: int, ws, stream=None):
+    _need_ws(ws, dlrm_mlp_workspace_size(mlp, B, inp.dtype) if B > 0 else ERR_RECORD_BYTES, "dlrm_mlp_fwd")
     return _check(lib().dlrm_mlp_fwd(mlp.ref(), int(B), _ptr(inp), DT_CODE[inp.dtype], int(ld_in), _ptr(out),
                                      int(ld_out), int(final_act), _ptr(ws), _stream(stream)), "dlrm_mlp_fwd")
 
 
 def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
+    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward")
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                      _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
                   "dlrm_forward")
@@ -241,6 +260,7 @@ def dlrm_embbag_cat_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld
                         stream=None):
     """Concat-only interaction: concat rows [x_dense, e_1 .. e_K, zeros]."""
     out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
+    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_cat_fwd")
     return _check(lib().dlrm_embbag_cat_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
                                             _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
                                             _stream(stream)), "dlrm_embbag_cat_fwd")
@@ -248,6 +268,7 @@ def dlrm_embbag_cat_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld
 
 def dlrm_forward_cat(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
     """dlrm_forward with the concat-only interaction (top MLP input width d (K + 1))."""
+    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward_cat")
     return _check(lib().dlrm_forward_cat(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                          _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
                   "dlrm_forward_cat")
@@ -284,6 +305,7 @@ def dlrm_gemm_f32(I: int, J: int, R: int, A, lda: int, a_mn: bool, B, ldb: int, 
                   stream=None):
     """C[i][j] = sum_r A(i, r) B(j, r) in fp32 on the tensor cores; A(i, r) = A[i][r], or A[r][i] when a_mn
     (B likewise)."""
+    _need_ws(ws, dlrm_gemm_f32_workspace_size(I, J, R, a_mn, b_mn), "dlrm_gemm_f32")
     return _check(lib().dlrm_gemm_f32(int(I), int(J), int(R), _ptr(A), int(lda), int(bool(a_mn)), _ptr(B), int(ldb),
                                       int(bool(b_mn)), _ptr(C), int(ldc), _ptr(ws), _stream(stream)), "dlrm_gemm_f32")
 
@@ -301,6 +323,7 @@ def dlrm_gemm_tf32x3_workspace_size(I: int, J: int, R: int) -> int:
 def dlrm_gemm_tf32x3(I: int, J: int, R: int, A_hi, A_lo, lda: int, a_mn: bool, B_hi, B_lo, ldb: int, b_mn: bool, C,
                      ldc: int, ws, stream=None):
     """dlrm_gemm_f32 on operands already split by dlrm_tf32_split."""
+    _need_ws(ws, dlrm_gemm_tf32x3_workspace_size(I, J, R), "dlrm_gemm_tf32x3")
     return _check(lib().dlrm_gemm_tf32x3(int(I), int(J), int(R), _ptr(A_hi), _ptr(A_lo), int(lda), int(bool(a_mn)),
                                          _ptr(B_hi), _ptr(B_lo), int(ldb), int(bool(b_mn)), _ptr(C), int(ldc),
                                          _ptr(ws), _stream(stream)), "dlrm_gemm_tf32x3")
@@ -325,6 +348,7 @@ def dlrm_grads_offsets(T: Tables, bot: MLP, top: MLP, B: int, nnz: int) -> dict:
 
 def dlrm_backward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, labels, grads, ws, loss=None,
                   y_hat=None, stream=None):
+    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 1), "dlrm_backward")
     return _check(lib().dlrm_backward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                       _ptr(indices), int(indices.numel()), _ptr(labels), _ptr(loss), _ptr(y_hat),
                                       _ptr(grads), _ptr(ws), _stream(stream)), "dlrm_backward")

@@ -6,6 +6,8 @@
 
 #include <atomic>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -66,6 +68,26 @@ size_t hidden_bytes(const dlrm_mlp* m, int B) {
         if (b > w) w = b;
     }
     return w * (size_t)B;
+}
+
+// dlrm_mlp_fwd's workspace after the error record: `nact` activation buffers of `act` bytes (the
+// widest hidden layer output; none for one layer, one for two), then the input converted to the MLP's
+// dtype when it comes in another one.
+struct MlpWs {
+    size_t act, cvt, total;
+    int nact;
+};
+
+MlpWs mlp_ws(const dlrm_mlp* m, int B, dlrm_dtype in_dt) {
+    MlpWs w{};
+    size_t row = 0;
+    for (int l = 1; l < m->n_layers; ++l) row = std::max(row, (size_t)dlrm_ld(m->dims[l], m->dt) * esize(m->dt));
+    w.act = align_up(row * (size_t)B, 256);
+    w.nact = m->n_layers >= 3 ? 2 : m->n_layers - 1;
+    const bool conv = in_dt != m->dt && m->dt != DLRM_F32;
+    w.cvt = conv ? align_up((size_t)dlrm_ld(m->dims[0], m->dt) * esize(m->dt) * (size_t)B, 256) : 0;
+    w.total = DLRM_ERR_RECORD_BYTES + (size_t)w.nact * w.act + w.cvt;
+    return w;
 }
 
 struct FwdLayout {
@@ -236,10 +258,15 @@ dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype 
     if (B == 0) return DLRM_OK;
     if (!in || !out) return DLRM_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
-    const size_t h = align_up(hidden_bytes(mlp, B), 256);
+    const MlpWs L = mlp_ws(mlp, B, in_dt);
     char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
-    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + h, w + 2 * h,
+    return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + L.act, w + (size_t)L.nact * L.act,
                    static_cast<ErrRecord*>(ws), cs(stream));
+}
+
+size_t dlrm_mlp_workspace_size(const dlrm_mlp* mlp, int B, dlrm_dtype in_dt) {
+    if (check_mlp(mlp) != DLRM_OK || B < 0 || !valid_dt(in_dt)) return 0;
+    return mlp_ws(mlp, B, in_dt).total;
 }
 
 namespace {

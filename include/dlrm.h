@@ -156,9 +156,19 @@ dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t*
  * hidden layer; after the last layer `final_act` (none, ReLU or sigmoid).
  *   in    [B][ld_in] of in_dt, dims[0] logical columns
  *   out   out, fp32 [B][ld_out], dims[n_layers] logical columns
- *   ws    workspace from dlrm_workspace_size for this MLP as `top` (or bottom) */
+ *   ws    16-byte aligned, at least dlrm_mlp_workspace_size(mlp, B, in_dt)
+ *         bytes (dlrm_workspace_size of a model with this MLP as top or
+ *         bottom is enough); the hidden activations live there. The size is
+ *         not passed, so it cannot be checked here: a smaller buffer is
+ *         written past its end. */
 dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in,
                          float* out, int ld_out, int final_act, void* ws, dlrm_stream stream);
+
+/* Bytes of workspace dlrm_mlp_fwd needs for this MLP, batch and input dtype:
+ * the error record, one or two buffers of the widest hidden-layer output and,
+ * when in_dt differs from a 16-bit MLP dtype, the converted input.
+ * 0 for an invalid MLP, B < 0 or an invalid in_dt. */
+size_t dlrm_mlp_workspace_size(const dlrm_mlp* mlp, int B, dlrm_dtype in_dt);
 
 /* Whole forward pass ([S] sections 3-4):
  *   y_hat = sigmoid(top([x_dense, vec(Z)])),  x_dense = bottom(dense) with ReLU after every bottom layer,

@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -86,3 +87,41 @@ def test_product_path_has_no_cpu_fallback():
     for f in glob.glob(os.path.join(ROOT, "embedding_bags_dot_b200", "**", "*.*"), recursive=True):
         if f.endswith((".py", ".cu", ".cuh")):
             assert "import oracle" not in open(f).read() and "from oracle" not in open(f).read(), f
+
+
+def _cpu_mlp(dims, dt):
+    E = pytest.importorskip("embedding_bags_dot_b200")
+    td = {"f32": torch.float32, "bf16": torch.bfloat16}[dt]
+    Ws = [torch.zeros((dims[l + 1], E.dlrm_ld(dims[l], dt)), dtype=td) for l in range(len(dims) - 1)]
+    bs = [torch.zeros(dims[l + 1]) for l in range(len(dims) - 1)]
+    return E.MLP(Ws, bs, dims)
+
+
+def test_mlp_workspace_size_follows_the_documented_layout(lib):
+    """Error record (256 B), then one activation buffer per alternating hidden output (none for one layer,
+    one for two, two otherwise) of the widest hidden output, then the input converted to a 16-bit MLP
+    dtype when it comes in another dtype; every piece rounded up to 256 bytes."""
+    import embedding_bags_dot_b200 as E
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    B = 1000
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), B, "f32") == 256
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "bf16"), B, "f32") == 256 + a256(16 * 2 * B)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 512, 128], "bf16"), B, "f32") == 256 + a256(512 * 2 * B) + a256(16 * 2 * B)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 512, 256, 128], "bf16"), B, "bf16") == 256 + 2 * a256(512 * 2 * B)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([479, 1024, 1024, 512, 256, 1], "bf16"), 77, "bf16") == \
+        256 + 2 * a256(1024 * 2 * 77)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 100, 3], "f32"), 5, "f32") == 256 + a256(100 * 4 * 5)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), -1, "f32") == 0
+
+
+def test_bindings_refuse_a_short_workspace_before_launching(lib):
+    import embedding_bags_dot_b200 as E
+    mlp = _cpu_mlp([13, 512, 256, 128], "bf16")
+    B = 1000
+    need = E.dlrm_mlp_workspace_size(mlp, B, torch.float32)
+    x, out = torch.zeros((B, 13)), torch.zeros((B, 128))
+    before = E.dlrm_launch_count()
+    with pytest.raises(E.DlrmError) as e:
+        E.dlrm_mlp_fwd(mlp, B, x, 13, out, 128, E.ACT_RELU, torch.zeros(need - 16, dtype=torch.uint8))
+    assert e.value.status == E.ERR_WORKSPACE
+    assert E.dlrm_launch_count() == before

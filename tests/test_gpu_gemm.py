@@ -40,7 +40,7 @@ def test_linear_tc_fp32_out(M, N, K, dt):
     mlp = E.MLP([W.cuda()], [b.cuda()], [K, N])
     out = torch.full((M, N + 4 - N % 4 if N % 4 else N), float("nan"), device="cuda")
     ldo = out.shape[1]
-    ws = E.alloc_workspace(1 << 20)
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, M, x.dtype))
     E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, ldo, E.ACT_NONE, ws)
     assert E.dlrm_check_error(ws)[0] == 0
     xs = x[:, :K].double().numpy()
@@ -63,7 +63,7 @@ def test_linear_tc_two_layers_bf16_hidden(act):
     b2 = torch.randn(N, generator=g) * 0.1
     mlp = E.MLP([W1.cuda(), W2.cuda()], [b1.cuda(), b2.cuda()], [K, H, N])
     out = torch.empty((M, N), device="cuda")
-    ws = E.alloc_workspace(1 << 22)
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, M, x.dtype))
     E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, N, act, ws)
     assert E.dlrm_check_error(ws)[0] == 0
     Ws = [W1[:, :K].double().numpy(), W2.double().numpy()]
@@ -91,7 +91,7 @@ def test_linear_small_batch(M, N, K, dt):
         x, W, b, ld = _layer(M, N, K, dt, seed=M * 11 + N)
     mlp = E.MLP([W.cuda()], [b.cuda()], [K, N])
     out = torch.full((M, N), float("nan"), device="cuda")
-    ws = E.alloc_workspace(1 << 20)
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, M, x.dtype))
     E.dlrm_mlp_fwd(mlp, M, x.cuda(), ld, out, N, E.ACT_RELU, ws)
     assert E.dlrm_check_error(ws)[0] == 0
     xs, Ws, bs = x[:, :K].double().numpy(), W[:, :K].double().numpy(), b.double().numpy()
@@ -118,7 +118,7 @@ def test_fused_bottom_mlp(B, dt, n3):
     x = torch.randn((B, 13), generator=g).abs()   # dense features: log1p-like, non-negative
     mlp = E.MLP(Wd, bd, dims)
     out = torch.full((B, n3), float("nan"), device="cuda")
-    ws = E.alloc_workspace(1 << 24)
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, x.dtype))
     E.dlrm_mlp_fwd(mlp, B, x.cuda(), 13, out, n3, E.ACT_RELU, ws)
     assert E.dlrm_check_error(ws)[0] == 0
     want = O.mlp(Ws, bs, x.double().numpy(), relu_last=True)
@@ -145,7 +145,7 @@ def test_last_hidden_layer_with_logit(B, h, dt):
     x[:, :479] = torch.randn((B, 479), generator=g).to(TD[dt])
     mlp = E.MLP(Wd, bd, dims)
     y = torch.full((B, 1), float("nan"), device="cuda")
-    ws = E.alloc_workspace(1 << 26)
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, x.dtype))
     E.dlrm_mlp_fwd(mlp, B, x.cuda(), ld, y, 1, E.ACT_SIGMOID, ws)
     assert E.dlrm_check_error(ws)[0] == 0
     xs = x[:, :479].double().numpy()
