@@ -5,42 +5,42 @@
 // and write [x_dense, Z_10, Z_20, Z_21, ...] with Z_ij = <X_i, X_j>, j < i
 // ("DLRM", briansu.co, section 4, equations "Interaction" and "Output").
 //
-// Block prologue (all threads): the tile's CSR offsets are read once,
-// coalesced, and every bag is resolved to a code: the global row of a
-// one-row bag, "empty" (no rows, bad offsets or an out-of-range index), or
-// "several rows". Then one warp owns one sample at a time:
-//  1. gather: lanes form groups of GL = d/8 lanes, one 16-byte chunk of a bf16
-//     row per lane. A one-row bag is copied global -> shared with cp.async,
-//     so every row of the sample is in flight at once without registers;
-//     a bag of several rows is summed in fp32 and rounded to bf16.
-//     Row-wise uint8 tables (Q), a sample with a bag of several rows (or a
-//     non-finite x_dense): a one-row bag's record (d codes, fp32 scale s, fp32
-//     offset m) is copied the same way, unswizzled, into the first bytes of
-//     its X row slot; once it has landed each lane reads its 8 codes and the
-//     scale/offset, the warp synchronises, and the lane writes the dequantised
-//     values (s q + m, rounded to bf16) as its swizzled 16-byte chunk.
-//     Every other uint8 sample takes the integer route (5. below).
-//  2. x_dense (fp32) is split into hi = bf16(x) and lo = bf16(x - hi); hi is
-//     row 0 of X and lo row K+1, so that Z_i0 = G[i][0] + G[K+1][i] keeps the
-//     dense vector's fp32 precision.
-//  3. Gram G = X X^T over the Kp = 16*MT padded rows with
-//     mma.sync.m16n8k16 (bf16 in, fp32 accumulate), lower-triangle tiles only.
-//     The same ldmatrix fragments serve as A and as B (B = X^T), so X is read
-//     from shared memory once per sample.
+// Block prologue: one warp per table, one lane per sample of the 32-sample
+// tile; each lane reads its bag's two CSR offsets and resolves the bag to a
+// code: the global row of a one-row bag, "empty" (no rows, bad offsets or an
+// out-of-range index) or "several rows". Then one warp owns one sample at a
+// time:
+//  1. gather: lane k issues ONE bulk copy (cp.async.bulk, completing on the
+//     warp's mbarrier) for the whole row of a one-row bag k, straight into row
+//     1+k of the sample's tile. Tile rows are unswizzled and padded by one
+//     16-byte chunk, so the 8 rows an ldmatrix reads land in 8 distinct bank
+//     groups. Empty bags are zeroed and bags of several rows are summed in
+//     fp32 by lane groups while the copies are in flight.
+//  2. bf16 tables: x_dense (fp32) is split into hi = bf16(x) and
+//     lo = bf16(x - hi); hi is row 0 and lo row K+1, so that
+//     Z_i0 = G[i][0] + G[K+1][i] keeps the dense vector's fp32 precision.
+//  3. Gram G = X X^T over the 16*MT padded rows with mma.sync.m16n8k16 (bf16
+//     in, fp32 accumulate), lower-triangle tiles only. The same ldmatrix
+//     fragments serve as A and as B (B = X^T), so X is read from shared memory
+//     once per sample. Rows past the sample's last one are never written: they
+//     only reach Gram entries that nothing reads.
 //  4. G is staged in shared memory, the x_dense low-half terms are folded into
 //     column 0, and each lane writes fixed 8-column chunks of the concat row
 //     whose sources in G are computed once per block.
-//  5. Row-wise uint8 tables, samples whose bags hold at most one row: the
-//     codes are never converted. Each bag's d codes go by cp.async straight
-//     into row 1+k of an 8-bit tile, its (s, m) into a per-row slot; row 0 is
-//     all ones; x_dense is quantised per sample to 24 bits,
-//     x ~ sx qx + mn with qx = 65536 h + 256 u + l, and its three byte planes
-//     are rows K+1..K+3. One u8 x u8 -> s32 Gram on the tensor cores
-//     (mma.sync m16n8k32) then holds, exactly, every <q_i, q_j>, the code sums
-//     S_i = <q_i, 1> and the plane products. With e_i = s_i q_i + m_i,
+//  5. Row-wise uint8 tables, samples whose bags hold at most one row (and
+//     whose x_dense is finite): the codes are never converted. Each record
+//     (d codes, fp32 scale s, fp32 offset m) is copied whole into row 1+k of
+//     an 8-bit tile whose row stride is the record size; row 0 is all ones;
+//     x_dense is quantised per sample to 24 bits, x ~ sx qx + mn with
+//     qx = 65536 h + 256 u + l, and its three byte planes are rows K+1..K+3.
+//     One u8 x u8 -> s32 Gram (mma.sync m16n8k32) then holds, exactly, every
+//     <q_i, q_j>, the code sums S_i = <q_i, 1> and the plane products. With
+//     e_i = s_i q_i + m_i,
 //       Z_ij = s_i s_j <q_i, q_j> + s_i S_i m_j + s_j S_j m_i + d m_i m_j,
 //     and the same with (sx, mn, <q_i, qx>, sum qx) for the x_dense column;
 //     the affine terms are applied in fp32 while the concat row is written.
+//     Other uint8 samples take steps 1-4 with each one-row record copied into
+//     its bf16 row slot and dequantised there (s q + m, rounded to bf16).
 #include <algorithm>
 
 #include "common.cuh"
@@ -52,10 +52,13 @@ namespace {
 
 constexpr int WARPS = 8;
 constexpr int SPW = 4;               // samples per warp per block
-constexpr int S = WARPS * SPW;       // samples per block
+constexpr int S = WARPS * SPW;       // samples per block: one lane each in the prologue
+static_assert(S == 32, "the prologue maps the block's samples to the lanes of a warp");
 constexpr uint32_t CODE_EMPTY = 0xFFFFFFFFu;
 constexpr uint32_t CODE_MULTI = 0xFFFFFFFEu;
 constexpr int SRC_CACHE = 1;         // concat chunks per lane whose sources stay in registers
+constexpr int WAIT_TRIES = 1 << 20;  // bound on the mbarrier polls for one sample's rows (~1 s at 1 us each)
+constexpr unsigned FULL = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -84,11 +87,44 @@ __device__ __forceinline__ void mma_u8(int (&c)[4], const uint32_t (&a)[4], uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// ---- one-row bags: bulk copies completing on the warp's mbarrier
+__device__ __forceinline__ void bar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+// The phase's single arrival, announcing the bytes its copies will deliver.
+__device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Orders this thread's earlier generic shared-memory accesses before later bulk-copy writes.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Bounded wait for the phase of the given parity; false if it never completed. Each poll suspends for
+// at most about 1 us (the hint, in ns), so the bound is time-like, not a count of instructions.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    for (int i = 0; i < WAIT_TRIES; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(1000u)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+// Position of the n-th (0-based) set bit of m, or -1.
+__device__ __forceinline__ int nth_bit(unsigned long long m, int n) {
+    for (int t = 0; t < n; ++t) m &= m - 1;
+    return m ? __ffsll((long long)m) - 1 : -1;
+}
+__device__ __forceinline__ unsigned long long drop_bits(unsigned long long m, int n) {
+    for (int t = 0; t < n; ++t) m &= m - 1;
+    return m;
 }
 
 // Source of concat column c (c >= d) in the staged Gram G (row stride GS):
@@ -102,8 +138,6 @@ __device__ __forceinline__ uint32_t column_source(int c, int d, int P, int GS, u
     return (uint32_t)(i * GS + (p - i * (i - 1) / 2));
 }
 
-}  // namespace
-
 // Dequantise 8 codes of a DLRM_U8ROW record: v = s q + m.
 __device__ __forceinline__ void dequant8(uint2 codes, float sc, float of, float (&v)[8]) {
 #pragma unroll
@@ -113,58 +147,48 @@ __device__ __forceinline__ void dequant8(uint2 codes, float sc, float of, float 
     }
 }
 
-// Layout of a warp's region on the integer route: KP+1 16-byte row slots
-// (s, m, s S, 0) -- slot 0 for x_dense, slots 1..K for the bags, slot KP all
-// zero for padding columns -- then the 8-bit tile X8 (KP rows of d bytes),
-// which the staged Gram (fp32, row stride KP + 8) overwrites after the MMAs.
+// Byte offset of the integer route's (s, m, s S, 0) slots: after the 8-bit tile and the staged Gram.
+__host__ __device__ constexpr int u8_meta_offset(int K, int KP, int qrb) {
+    return (std::max((K + 4) * qrb, (KP * (KP + 8) + 1) * 4) + 15) / 16 * 16;
+}
 
-// One sample on the integer route: bags of at most one row, finite x_dense
-// (minimum mn, range = max - mn). Writes the whole concat row.
+// The bag masks of one sample: bit k set for bag k.
+struct BagMasks {
+    unsigned long long one, multi, empty;
+};
+
+// One sample on the integer route (every bag holds at most one row, x_dense finite with minimum mn and
+// range max - mn). The records' bulk copies into rows 1..K (stride QRB) are already issued on `bar`.
+// Writes the whole concat row.
 template <int MT, int GL>
-__device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, const uint32_t* code_k, int K,
-                                          const unsigned char* __restrict__ qtab, const float4* xv, float mn,
-                                          float range, const uint32_t (&srcr)[SRC_CACHE][4], const uint16_t* src_s,
-                                          int nzc, const float* __restrict__ xrow, void* out, size_t row0, int ld,
-                                          int out_dt, int lane) {
+__device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, int K, const BagMasks& bm,
+                                          uint32_t bar, uint32_t parity, bool& timed_out, const float4* xv,
+                                          float mn, float range, const uint32_t (&srcr)[SRC_CACHE][4],
+                                          const uint16_t* src_s, int nzc, const float* __restrict__ xrow,
+                                          void* out, size_t row0, int ld, int out_dt, int lane) {
     constexpr int d = 8 * GL;
     constexpr int KP = 16 * MT;
     constexpr int GS = KP + 8;
-    constexpr int CH = d / 16;               // 16-byte chunks of an 8-bit row
-    constexpr int NG8 = 32 / CH;             // rows per round of the gather
-    constexpr int QRB = (d + 8 + 15) / 16 * 16;
+    constexpr int QRB = (d + 8 + 15) / 16 * 16;   // record bytes = 8-bit tile row stride
+    constexpr int CHQ = QRB / 16;                 // 16-byte chunks of a record
+    constexpr int NGQ = 32 / CHQ;                 // records zeroed per round
     constexpr int NTILE = MT * (MT + 1);
     constexpr uint32_t ZERO_SLOT = KP * GS;
-    constexpr int X8 = (KP + 1) * 16;     // start of the 8-bit tile
-    // 128-byte rows: chunk c of row r at c ^ (r & 7); 64-byte rows: c ^ ((r >> 1) & 3). Either way the
-    // 8 rows an ldmatrix reads fall in 8 distinct 16-byte bank groups.
-    auto xoff8 = [](int r, int c) { return X8 + r * d + 16 * (d == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3))); };
-    float4* meta = reinterpret_cast<float4*>(xw);
-    float* G = reinterpret_cast<float*>(xw + X8);
-    const int P0 = K + 1;                    // x_dense byte planes: P0 (weight 1), P0+1 (256), P0+2 (65536)
+    float* G = reinterpret_cast<float*>(xw);
+    float4* meta = reinterpret_cast<float4*>(xw + u8_meta_offset(K, KP, QRB));
+    const int P0 = K + 1;                         // x_dense byte planes: P0 (weight 1), P0+1 (256), P0+2 (65536)
 
-    // codes of the one-row bags, row 1+k; their (s, m) into slot 1+k; empty bags are all zero
+    // empty bags: codes and (s, m) all zero
     {
-        const int gi = lane / CH, g = lane % CH;
-        for (int k = gi; k < K; k += NG8) {
-            const uint32_t code = code_k[k * S];
-            if (code < CODE_MULTI)
-                cp_async16(xw_s + (uint32_t)xoff8(k + 1, g), qtab + (long long)code * QRB + 16 * g);
-            else
-                *reinterpret_cast<uint4*>(xw + xoff8(k + 1, g)) = make_uint4(0, 0, 0, 0);
-        }
-        for (int k = lane; k < K; k += 32) {
-            const uint32_t code = code_k[k * S];
-            if (code < CODE_MULTI)
-                cp_async16(xw_s + 16u * (uint32_t)(k + 1), qtab + (long long)code * QRB + d);
-            else
-                meta[k + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int gq = lane / CHQ, cq = lane % CHQ;
+        for (unsigned long long rest = bm.empty; rest; rest = drop_bits(rest, NGQ)) {
+            const int k = gq < NGQ ? nth_bit(rest, gq) : -1;
+            if (k >= 0) *reinterpret_cast<uint4*>(xw + (k + 1) * QRB + 16 * cq) = make_uint4(0, 0, 0, 0);
         }
     }
-    // row 0: ones; rows K+4 .. KP-1: zero; slot KP: zero
-    if (lane < CH) *reinterpret_cast<uint4*>(xw + xoff8(0, lane)) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
-    for (int q = lane; q < (KP - K - 4) * CH; q += 32)
-        reinterpret_cast<uint4*>(xw + X8 + (K + 4) * d)[q] = make_uint4(0, 0, 0, 0);
-    if (lane == 0) meta[KP] = make_float4(0.f, 0.f, 0.f, 0.f);
+    // row 0: ones
+    if (lane < d / 16)
+        *reinterpret_cast<uint4*>(xw + 16 * lane) = make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
     // x_dense -> 24-bit codes qx = rint((x - mn) / sx), sx = range / (2^24 - 1), as three byte planes
     constexpr float QMAX = 16777215.f;
     const float inv = range > 0.f ? QMAX / range : 0.f;
@@ -182,13 +206,12 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, cons
             const uint32_t lo01 = __byte_perm(qv[0], qv[1], 0x0040), lo23 = __byte_perm(qv[2], qv[3], 0x0040);
             const uint32_t mi01 = __byte_perm(qv[0], qv[1], 0x0051), mi23 = __byte_perm(qv[2], qv[3], 0x0051);
             const uint32_t hi01 = __byte_perm(qv[0], qv[1], 0x0062), hi23 = __byte_perm(qv[2], qv[3], 0x0062);
-            const int ch = c / 16, byte = c % 16;
-            *reinterpret_cast<uint32_t*>(xw + xoff8(P0, ch) + byte) = __byte_perm(lo01, lo23, 0x5410);
-            *reinterpret_cast<uint32_t*>(xw + xoff8(P0 + 1, ch) + byte) = __byte_perm(mi01, mi23, 0x5410);
-            *reinterpret_cast<uint32_t*>(xw + xoff8(P0 + 2, ch) + byte) = __byte_perm(hi01, hi23, 0x5410);
+            *reinterpret_cast<uint32_t*>(xw + P0 * QRB + c) = __byte_perm(lo01, lo23, 0x5410);
+            *reinterpret_cast<uint32_t*>(xw + (P0 + 1) * QRB + c) = __byte_perm(mi01, mi23, 0x5410);
+            *reinterpret_cast<uint32_t*>(xw + (P0 + 2) * QRB + c) = __byte_perm(hi01, hi23, 0x5410);
         }
     }
-    cp_async_wait_all();
+    if (!bar_wait(bar, parity)) timed_out = true;
     __syncwarp();
 
     // exact integer Gram of the lower-triangle tiles
@@ -200,7 +223,7 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, cons
         uint32_t a[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
-            ldmatrix_x4(xw_s + (uint32_t)xoff8(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a[mt]);
+            ldmatrix_x4(xw_s + (uint32_t)((16 * mt + (lane & 15)) * QRB + 16 * (2 * ks + (lane >> 4))), a[mt]);
         int t = 0;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -209,7 +232,14 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, cons
                 mma_u8(acc[t], a[mt], a[nt >> 1][(nt & 1) ? 1 : 0], a[nt >> 1][(nt & 1) ? 3 : 2]);
         }
     }
-    __syncwarp();  // every lane's ldmatrix of X8 is done before G overwrites it
+    // each bag's (s, m) from its record, before G overwrites the tile
+    float2 sm[(KP + 31) / 32];
+#pragma unroll
+    for (int w = 0; w < (KP + 31) / 32; ++w) {
+        const int k = lane + 32 * w;
+        sm[w] = k < K ? *reinterpret_cast<const float2*>(xw + (k + 1) * QRB + d) : make_float2(0.f, 0.f);
+    }
+    __syncwarp();  // every lane's reads of the tile are done before G overwrites it
 
     // stage G in fp32 (every entry is below 2^24, so exact)
     {
@@ -229,16 +259,20 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, cons
     __syncwarp();
     // per bag: slot (s, m, s S); column 0 of its Gram row becomes <q_i, qx>
     const float* Gx0 = G + P0 * GS;
-    for (int i = 1 + lane; i <= K; i += 32) {
-        const float S_i = G[i * GS];
-        G[i * GS] = fmaf(65536.f, Gx0[2 * GS + i], fmaf(256.f, Gx0[GS + i], Gx0[i]));
-        const float4 sm = meta[i];
-        meta[i] = make_float4(sm.x, sm.y, sm.x * S_i, 0.f);
+#pragma unroll
+    for (int w = 0; w < (KP + 31) / 32; ++w) {
+        const int i = lane + 32 * w + 1;
+        if (i <= K) {
+            const float S_i = G[i * GS];
+            G[i * GS] = fmaf(65536.f, Gx0[2 * GS + i], fmaf(256.f, Gx0[GS + i], Gx0[i]));
+            meta[i] = make_float4(sm[w].x, sm[w].y, sm[w].x * S_i, 0.f);
+        }
     }
     if (lane == 0) {
         const float Sx = fmaf(65536.f, Gx0[2 * GS], fmaf(256.f, Gx0[GS], Gx0[0]));
         meta[0] = make_float4(sx, mn, sx * Sx, 0.f);
     }
+    if (lane == 1) meta[KP] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncwarp();
 
     // Z for the Gram entry at `src`: s_i s_j g + t_i m_j + t_j m_i + d m_i m_j
@@ -279,10 +313,11 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, cons
     } else {
         for (int c = lane; c < ld; c += 32) store_as(out, row0 + c, c < d ? xrow[c] : zval(src_s[c - d]), out_dt);
     }
-    __syncwarp();  // the region is reused by the next sample
 }
 
-// MT: m-tiles of 16 rows (Kp = 16 MT >= K + 2; K + 4 with Q). GL: lanes per row (d = 8 GL).
+}  // namespace
+
+// MT: m-tiles of 16 rows (16 MT >= K + 2; K + 4 with Q). GL: lanes per row (d = 8 GL).
 // Q: row-wise uint8 tables.
 template <int MT, int GL, bool Q>
 __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_mma_kernel(
@@ -291,28 +326,27 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, int warp_bytes, ErrRecord* err) {
     constexpr int d = 8 * GL;
     constexpr int KP = 16 * MT;
-    // X rows: d >= 64 uses 2d-byte rows whose 16-byte chunks are XOR-swizzled by (row & 7); d = 32
-    // pads rows to an odd number of chunks. Either way ldmatrix reads 8 rows without bank conflicts.
-    constexpr bool SWZ = d >= 64;
-    constexpr int RS = SWZ ? 2 * d : 2 * d + 16;
+    constexpr int RS = 2 * d + 16;   // bf16 tile row: 2d bytes plus one pad chunk (conflict-free ldmatrix)
     constexpr int GS = KP + 8;       // G row stride in floats (float2 staging without bank conflicts)
     constexpr int NG = 32 / GL;      // row groups per warp
     constexpr int NTILE = MT * (MT + 1);
     constexpr int QRB = (d + 8 + 15) / 16 * 16;   // uint8 record bytes
+    constexpr int ROWB = Q ? QRB : 2 * d;         // bytes of one table row in global memory
+    constexpr bool TWO = KP > 32;                 // K may exceed 32: two bags per lane
     const __nv_bfloat16* __restrict__ tables = static_cast<const __nv_bfloat16*>(tables_v);
     const unsigned char* __restrict__ qtab = static_cast<const unsigned char*>(tables_v);
-    // byte offset of 16-byte chunk c of X row r
-    auto xoff = [](int r, int c) { return r * RS + 16 * (SWZ ? (c ^ (r & 7)) : c); };
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = K * (K + 1) / 2;
     const int L = K + 1;             // row holding the low half of x_dense
+    const int KS = K | 1;            // code_s row stride (odd: the prologue's writes are conflict-free)
     unsigned char* xw = smem + (size_t)warp * warp_bytes;
     unsigned char* tail = smem + (size_t)WARPS * warp_bytes;
-    int* off_s = reinterpret_cast<int*>(smem);   // prologue only: lives in the X regions until samples start
-    uint32_t* code_s = reinterpret_cast<uint32_t*>(tail);
-    uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + K * S);   // sources of columns d .. ld-1
-    const int nzc = (ld - d) / 8;                                    // 8-column chunks after x_dense
+    uint32_t* code_s = reinterpret_cast<uint32_t*>(tail);                       // [S][KS]
+    uint16_t* src_s = reinterpret_cast<uint16_t*>(code_s + S * KS);             // sources of columns d .. ld-1
+    const int bar_off = (S * KS * 4 + (ld - d + 8) * 2 + 7) & ~7;
+    const uint32_t bar = (uint32_t)__cvta_generic_to_shared(tail + bar_off) + 8u * (uint32_t)warp;
+    const int nzc = (ld - d) / 8;                                               // 8-column chunks after x_dense
     constexpr uint32_t ZERO_SLOT = KP * GS;
     const bool bf16_out = out_dt == DLRM_BF16;
 
@@ -320,29 +354,30 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const int nb = min(S, B - b0);
     unsigned oob = 0, bad = 0;
 
-    // ---- block prologue: tile offsets, bag codes, concat column sources
-    for (int q = threadIdx.x; q < K * (nb + 1); q += blockDim.x) {
-        const int k = q / (nb + 1), s = q - k * (nb + 1);
-        off_s[k * (S + 1) + s] = offsets[(long long)k * B + b0 + s];
+    // ---- block prologue: bag codes (warp per table, lane per sample), concat column sources, barriers
+    for (int k = warp; k < K; k += WARPS) {
+        if (lane < nb) {
+            const long long o = (long long)k * B + b0 + lane;
+            const long long st = offsets[o], en = offsets[o + 1];
+            uint32_t code = CODE_EMPTY;
+            if (st < 0 || en < st || en > nnz) {
+                ++bad;
+            } else if (en - st == 1) {
+                const int idx = __ldg(indices + st);
+                if (idx >= 0 && (long long)idx < tm.rows[k])
+                    code = (uint32_t)(tm.base[k] + idx);
+                else
+                    ++oob;
+            } else if (en - st > 1) {
+                code = CODE_MULTI;
+            }
+            code_s[lane * KS + k] = code;
+        }
     }
     for (int c = d + threadIdx.x; c < ld; c += blockDim.x) src_s[c - d] = (uint16_t)column_source(c, d, P, GS, ZERO_SLOT);
-    __syncthreads();
-    for (int q = threadIdx.x; q < K * nb; q += blockDim.x) {
-        const int k = q / nb, s = q - k * nb;
-        const long long st = off_s[k * (S + 1) + s], en = off_s[k * (S + 1) + s + 1];
-        uint32_t code = CODE_EMPTY;
-        if (st < 0 || en < st || en > nnz) {
-            ++bad;
-        } else if (en - st == 1) {
-            const int idx = __ldg(indices + st);
-            if (idx >= 0 && (long long)idx < tm.rows[k])
-                code = (uint32_t)(tm.base[k] + idx);
-            else
-                ++oob;
-        } else if (en - st > 1) {
-            code = CODE_MULTI;
-        }
-        code_s[k * S + s] = code;
+    if (lane == 0) {
+        bar_init(bar);
+        fence_proxy_async();
     }
     __syncthreads();
 
@@ -360,6 +395,8 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const uint32_t xw_s = (uint32_t)__cvta_generic_to_shared(xw);
     float* G = reinterpret_cast<float*>(xw + RS);
     const int gi = lane / GL, g = lane % GL;
+    uint32_t parity = 0;
+    bool timed_out = false;
 
     for (int r = 0; r < SPW; ++r) {
         const int s = warp * SPW + r;
@@ -374,47 +411,77 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
             xv[q] = c < d ? *reinterpret_cast<const float4*>(x_dense + b * d + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 
+        // this sample's bags: lane k holds bag k (and k + 32)
+        const uint32_t* cs = code_s + s * KS;
+        const uint32_t c0 = lane < K ? cs[lane] : CODE_EMPTY;
+        const uint32_t c1 = TWO && lane + 32 < K ? cs[lane + 32] : CODE_EMPTY;
+        BagMasks bm;
+        bm.one = __ballot_sync(FULL, c0 < CODE_MULTI);
+        bm.multi = __ballot_sync(FULL, c0 == CODE_MULTI);
+        bm.empty = __ballot_sync(FULL, lane < K && c0 == CODE_EMPTY);
+        if (TWO) {
+            bm.one |= (unsigned long long)__ballot_sync(FULL, c1 < CODE_MULTI) << 32;
+            bm.multi |= (unsigned long long)__ballot_sync(FULL, c1 == CODE_MULTI) << 32;
+            bm.empty |= (unsigned long long)__ballot_sync(FULL, lane + 32 < K && c1 == CODE_EMPTY) << 32;
+        }
+
+        // uint8 tables: the integer route unless a bag holds several rows or x_dense is not finite
+        bool int_route = false;
+        float mn = 0.f, range = 0.f;
         if constexpr (Q) {
-            // ---- 5. integer route, unless a bag holds several rows or x_dense is not finite
-            float mn = INFINITY, mx = -INFINITY;
-            bool slow = false;
+            float mx = -INFINITY;
+            mn = INFINITY;
+            bool nonfinite = false;
 #pragma unroll
             for (int q = 0; q < (d + 127) / 128; ++q) {
                 if (4 * lane + 128 * q < d) {
                     const float4 x = xv[q];
                     mn = fminf(fminf(mn, x.x), fminf(x.y, fminf(x.z, x.w)));
                     mx = fmaxf(fmaxf(mx, x.x), fmaxf(x.y, fmaxf(x.z, x.w)));
-                    slow |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+                    nonfinite |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
                 }
             }
-            for (int k = lane; k < K; k += 32) slow |= code_s[k * S + s] == CODE_MULTI;
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
             }
-            const float range = mx - mn;
-            if (!__any_sync(0xffffffffu, slow) && isfinite(range)) {
-                u8_sample<MT, GL>(xw, xw_s, code_s + s, K, qtab, xv, mn, range, srcr, src_s, nzc, x_dense + b * d,
-                                  out, (size_t)b * ld, ld, out_dt, lane);
+            range = mx - mn;
+            int_route = bm.multi == 0 && !__any_sync(FULL, nonfinite) && isfinite(range);
+        }
+
+        // ---- 1. one bulk copy per one-row bag (after the previous sample's accesses to the region)
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) bar_expect(bar, (uint32_t)__popcll(bm.one) * ROWB);
+        __syncwarp();
+        {
+            const int stride = Q && int_route ? QRB : RS;
+            if (c0 < CODE_MULTI)
+                bulk_row(xw_s + (uint32_t)((lane + 1) * stride),
+                         Q ? (const void*)(qtab + (long long)c0 * QRB) : (const void*)(tables + (long long)c0 * d),
+                         ROWB, bar);
+            if (TWO && c1 < CODE_MULTI)
+                bulk_row(xw_s + (uint32_t)((lane + 33) * stride),
+                         Q ? (const void*)(qtab + (long long)c1 * QRB) : (const void*)(tables + (long long)c1 * d),
+                         ROWB, bar);
+        }
+        if constexpr (Q) {
+            if (int_route) {
+                u8_sample<MT, GL>(xw, xw_s, K, bm, bar, parity, timed_out, xv, mn, range, srcr, src_s, nzc,
+                                  x_dense + b * d, out, (size_t)b * ld, ld, out_dt, lane);
+                parity ^= 1u;
+                __syncwarp();  // the region is reused by the next sample
                 continue;
             }
         }
 
-        // ---- 1. gather: X rows 1..K
-        for (int k = gi; k < K; k += NG) {
-            const uint32_t code = code_s[k * S + s];
-            const uint32_t dst = xw_s + (uint32_t)xoff(k + 1, g);
-            if (code < CODE_MULTI) {
-                if constexpr (Q) {
-                    if (16 * g < QRB)
-                        cp_async16(xw_s + (uint32_t)((k + 1) * RS + 16 * g), qtab + (long long)code * QRB + 16 * g);
-                } else {
-                    cp_async16(dst, tables + (long long)code * d + 8 * g);
-                }
-            } else if (code == CODE_EMPTY) {
-                *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) = make_uint4(0, 0, 0, 0);
-            } else {
+        // empty bags -> zero rows; bags of several rows -> fp32 sums rounded to bf16 (NG bags at a time)
+        for (unsigned long long rest = bm.empty | bm.multi; rest; rest = drop_bits(rest, NG)) {
+            const int k = nth_bit(rest, gi);
+            if (k < 0) continue;
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if ((bm.multi >> k) & 1ull) {
                 const int st = offsets[(long long)k * B + b], en = offsets[(long long)k * B + b + 1];
                 float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int p = st; p < en; ++p) {
@@ -436,13 +503,10 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                         ++oob;
                     }
                 }
-                *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) =
-                    make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+                w = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
             }
+            *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) = w;
         }
-        // zero the padding rows K+2 .. KP-1 (G of the previous sample may have overwritten them)
-        for (int q = lane; q < (KP - K - 2) * (RS / 16); q += 32)
-            reinterpret_cast<uint4*>(xw + (size_t)(K + 2) * RS)[q] = make_uint4(0, 0, 0, 0);
 
         // ---- 2. x_dense -> rows 0 (hi) and K+1 (lo)
 #pragma unroll
@@ -452,22 +516,22 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                 const float4 x = xv[q];
                 const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
                 const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-                *reinterpret_cast<uint2*>(xw + xoff(0, c / 8) + 2 * (c % 8)) =
+                *reinterpret_cast<uint2*>(xw + 2 * c) =
                     make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
-                *reinterpret_cast<uint2*>(xw + xoff(L, c / 8) + 2 * (c % 8)) =
+                *reinterpret_cast<uint2*>(xw + L * RS + 2 * c) =
                     make_uint2(pack_bf16(x.x - f01.x, x.y - f01.y), pack_bf16(x.z - f23.x, x.w - f23.y));
             }
         }
-        cp_async_wait_all();
+        if (!bar_wait(bar, parity)) timed_out = true;
+        parity ^= 1u;
         __syncwarp();
         if constexpr (Q) {
-            // one-row bags: staged records -> dequantised bf16 rows, in place (every lane reads before any writes)
-            for (int kk = 0; kk < (K + NG - 1) / NG; ++kk) {
-                const int k = kk * NG + gi;
-                const bool one = k < K && code_s[k * S + s] < CODE_MULTI;
+            // one-row bags: records -> dequantised bf16 rows, in place (every lane reads before any writes)
+            for (unsigned long long rest = bm.one; rest; rest = drop_bits(rest, NG)) {
+                const int k = nth_bit(rest, gi);
                 uint4 w = make_uint4(0, 0, 0, 0);
-                if (one) {
-                    const unsigned char* rec = xw + (size_t)(k + 1) * RS;
+                if (k >= 0) {
+                    const unsigned char* rec = xw + (k + 1) * RS;
                     const uint2 cq = *reinterpret_cast<const uint2*>(rec + 8 * g);
                     const float2 so = *reinterpret_cast<const float2*>(rec + d);
                     float v[8];
@@ -476,7 +540,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                                    pack_bf16(v[6], v[7]));
                 }
                 __syncwarp();
-                if (one) *reinterpret_cast<uint4*>(xw + xoff(k + 1, g)) = w;
+                if (k >= 0) *reinterpret_cast<uint4*>(xw + (k + 1) * RS + 16 * g) = w;
             }
             __syncwarp();
         }
@@ -490,7 +554,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
             uint32_t a[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
-                ldmatrix_x4(xw_s + (uint32_t)xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a[mt]);
+                ldmatrix_x4(xw_s + (uint32_t)((16 * mt + (lane & 15)) * RS + 16 * (2 * ks + (lane >> 4))), a[mt]);
             int t = 0;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
@@ -555,26 +619,36 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         }
         __syncwarp();  // X / G reused by the next sample
     }
+    if (timed_out && lane == 0) atomicOr(&err->flags, ERR_TIMEOUT);
     report_warp(err, oob, bad);
 }
 
 // ------------------------------------------------------------------ host side
 
-// Bytes of a warp's region: the bf16 tile or its staged Gram, and for uint8 tables (q) also the integer
-// route's row slots plus its 8-bit tile or staged Gram.
+// Bytes of a warp's region. bf16 tile: rows 0..K+1 of 2d+16 bytes, or row 0 plus the staged Gram; uint8
+// tables add the integer route's tile (rows 0..K+3 of one record each) or Gram, then its (s, m, s S) slots.
 static int mma_warp_bytes(int K, int d, bool q, int& MT) {
     MT = (K + (q ? 4 : 2) + 15) / 16;
     const int KP = 16 * MT;
-    const int RS = d >= 64 ? 2 * d : 2 * d + 16;
+    const int RS = 2 * d + 16;
     const int gf = (KP * (KP + 8) + 1) * 4;
-    int bytes = std::max(KP * RS, RS + gf);
-    if (q) bytes = std::max(bytes, (KP + 1) * 16 + std::max(KP * d, gf));
+    int bytes = std::max((K + 2) * RS, RS + gf);
+    if (q) {
+        const int qrb = (d + 8 + 15) / 16 * 16;
+        bytes = std::max(bytes, u8_meta_offset(K, KP, qrb) + (KP + 1) * 16);
+    }
     return (bytes + 15) & ~15;
 }
 
+// Rows past a sample's last one are read by ldmatrix but never written; the last warp's may reach past
+// its region and the tail, so the allocation ends with enough slack to keep those reads inside it.
 static size_t mma_smem(int K, int d, bool q, int ld, int& MT, int& warp_bytes) {
     warp_bytes = mma_warp_bytes(K, d, q, MT);
-    return (size_t)WARPS * warp_bytes + sizeof(uint32_t) * (size_t)K * S + sizeof(uint16_t) * (size_t)(ld - d + 8);
+    const int KP = 16 * MT;
+    const size_t tail = (((size_t)S * (K | 1) * 4 + (size_t)(ld - d + 8) * 2 + 7) & ~(size_t)7) + 8 * WARPS;
+    const size_t reach = (size_t)KP * std::max(2 * d + 16, q ? (d + 8 + 15) / 16 * 16 : 0);
+    const size_t slack = reach > (size_t)warp_bytes + tail ? reach - warp_bytes - tail : 0;
+    return (size_t)WARPS * warp_bytes + tail + ((slack + 15) & ~(size_t)15);
 }
 
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
