@@ -97,7 +97,7 @@ struct FwdLayout {
 FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
     FwdLayout L;
     size_t off = DLRM_ERR_RECORD_BYTES;
-    const int K = T->K, d = T->d;
+    const int d = T->d;
     const int ldc = dlrm_ld(top->dims[0], top->dt);   // the concat: d + K(K+1)/2 (dot) or d(K+1) (concat-only)
     L.x_dense = off;
     off = align_up(off + sizeof(float) * (size_t)B * d, 256);

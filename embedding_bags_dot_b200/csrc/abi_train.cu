@@ -22,9 +22,9 @@ inline cudaStream_t cs(dlrm_stream s) { return reinterpret_cast<cudaStream_t>(s)
 struct TrainWs {
     size_t bW[DLRM_MAX_LAYERS][2], tW[DLRM_MAX_LAYERS][2];   // weight pairs, ld ldf(in)
     size_t bact[DLRM_MAX_LAYERS][2];                         // bottom outputs (pairs), ld ldb
-    size_t xd;                                               // x_dense plain [B][d]
-    size_t E;                                                // pooled [B][K][d]
-    size_t concat, concat_p[2];                              // [B][ldc] plain and pair
+    size_t xd;                                               // x_dense plain [B][d] (fallback path only)
+    size_t E;                                                // pooled [B][K][d] (fallback path only)
+    size_t concat, concat_p[2];                              // [B][ldc] plain (fallback only) and pair
     size_t tact[DLRM_MAX_LAYERS][2];                         // top hidden outputs (pairs), ld ldt
     size_t z, dz;                                            // logit and dL/dz [B]
     size_t g[2][2];                                          // gradient ping-pong pairs [B][gmax]
@@ -33,6 +33,7 @@ struct TrainWs {
     size_t csum;                                             // column sums per 32-row group of a gradient
     size_t wscratch, lpart, total;
     int ldb[DLRM_MAX_LAYERS], ldt[DLRM_MAX_LAYERS], ldc, gmax;
+    bool tc;                                                 // fused tensor-core interaction (no E, xd, concat, dxd)
 };
 
 struct Grads {
@@ -63,10 +64,14 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
         for (int h = 0; h < 2; ++h) W.bact[l][h] = take(sizeof(float) * (size_t)B * W.ldb[l]);
         gmax = std::max(gmax, W.ldb[l]);
     }
-    W.xd = take(sizeof(float) * (size_t)B * d);
-    W.E = take(sizeof(float) * (size_t)B * K * d);
     W.ldc = ldf(d + K * (K + 1) / 2);
-    W.concat = take(sizeof(float) * (size_t)B * W.ldc);
+    long long total_rows = 0;
+    for (int k = 0; k < K; ++k) total_rows += T->rows[k];
+    // the fused tensor-core interaction gathers the bags itself: no pooled vectors, no plain-fp32 copies
+    W.tc = interact_tc_supported(K, d, total_rows, W.ldc);
+    W.xd = W.tc ? 0 : take(sizeof(float) * (size_t)B * d);
+    W.E = W.tc ? 0 : take(sizeof(float) * (size_t)B * K * d);
+    W.concat = W.tc ? 0 : take(sizeof(float) * (size_t)B * W.ldc);
     for (int h = 0; h < 2; ++h) W.concat_p[h] = take(sizeof(float) * (size_t)B * W.ldc);
     for (int l = 0; l < nt - 1; ++l) {
         W.ldt[l] = ldf(top->dims[l + 1]);
@@ -80,7 +85,7 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
     for (int p = 0; p < 2; ++p)
         for (int h = 0; h < 2; ++h) W.g[p][h] = take(sizeof(float) * (size_t)B * gmax);
     W.dcat = take(sizeof(float) * (size_t)B * W.ldc);
-    W.dxd = take(sizeof(float) * (size_t)B * d);
+    W.dxd = W.tc ? 0 : take(sizeof(float) * (size_t)B * d);
     for (int l = 0; l < nb; ++l) W.bbits[l] = take(sizeof(uint32_t) * (size_t)B * relu_bits_ld(bot->dims[l + 1]));
     for (int l = 0; l < nt - 1; ++l) W.tbits[l] = take(sizeof(uint32_t) * (size_t)B * relu_bits_ld(top->dims[l + 1]));
     W.csum = take(sizeof(float) * (size_t)((B + 31) / 32) * gmax);
@@ -239,14 +244,17 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
             return r;
     }
     const F32Pair xd_pair = P(W.bact[nb - 1], W.ldb[nb - 1]);   // ld = d (d % 4 == 0 on this path)
-    const float* x_dense = F(W.xd);
-    // the warp-per-sample interaction reads and writes pairs; other shapes go through plain fp32 copies
-    const bool pair_inter = interact_pair_supported(K, d);
-    if ((r = launch_embbag(tm, T->data, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err, st))) return r;
-    if (pair_inter) {
-        if ((r = launch_interact_fwd_pair(B, K, d, xd_pair, F(W.E), F(W.concat_p[0]), F(W.concat_p[1]), W.ldc, st)))
+    const float* x_dense = W.tc ? nullptr : F(W.xd);
+    const float* tables = static_cast<const float*>(T->data);
+    // the fused tensor-core interaction gathers the bags and reads/writes pairs; other shapes pool the bags
+    // first and go through plain fp32 copies
+    if (W.tc) {
+        if ((r = launch_interact_fwd_tc(tm, tables, K, d, B, offsets, indices, nnz, xd_pair, F(W.concat_p[0]),
+                                        F(W.concat_p[1]), W.ldc, err, st)))
             return r;
     } else {
+        if ((r = launch_embbag(tm, T->data, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err, st)))
+            return r;
         if ((r = launch_merge_pair(B, d, xd_pair.hi, xd_pair.lo, xd_pair.ld, F(W.xd), d, st))) return r;
         if ((r = launch_interact(B, K, d, x_dense, F(W.E), F(W.concat), W.ldc, DLRM_F32, st))) return r;
         if ((r = launch_split_pair(B, top->dims[0], F(W.concat), W.ldc, F(W.concat_p[0]), F(W.concat_p[1]), W.ldc,
@@ -295,9 +303,9 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
         }
     }
     // d(concat) -> gradient of the last bottom layer's pre-activation (ReLU mask applied) and dE
-    if (pair_inter) {
-        if ((r = launch_interact_bwd_pair(B, K, d, xd_pair, F(W.E), F(W.dcat), W.ldc, F(W.g[pp][0]), F(W.g[pp][1]), d,
-                                          GF(G.dE), st)))
+    if (W.tc) {
+        if ((r = launch_interact_bwd_tc(tm, tables, K, d, B, offsets, indices, nnz, xd_pair, F(W.dcat), W.ldc,
+                                        F(W.g[pp][0]), F(W.g[pp][1]), d, GF(G.dE), err, st)))
             return r;
     } else {
         if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;

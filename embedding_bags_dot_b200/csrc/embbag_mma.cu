@@ -43,12 +43,15 @@
 //     its bf16 row slot and dequantised there (s q + m, rounded to bf16).
 #include <algorithm>
 
+#include "async_copy.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace dlrm {
 
 namespace {
+
+using namespace ac;
 
 constexpr int WARPS = 8;
 constexpr int SPW = 4;               // samples per warp per block
@@ -57,18 +60,11 @@ static_assert(S == 32, "the prologue maps the block's samples to the lanes of a 
 constexpr uint32_t CODE_EMPTY = 0xFFFFFFFFu;
 constexpr uint32_t CODE_MULTI = 0xFFFFFFFEu;
 constexpr int SRC_CACHE = 1;         // concat chunks per lane whose sources stay in registers
-constexpr int WAIT_TRIES = 1 << 20;  // bound on the mbarrier polls for one sample's rows (~1 s at 1 us each)
 constexpr unsigned FULL = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
 }
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -85,46 +81,6 @@ __device__ __forceinline__ void mma_u8(int (&c)[4], const uint32_t (&a)[4], uint
         "{%0,%1,%2,%3};"
         : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// ---- one-row bags: bulk copies completing on the warp's mbarrier
-__device__ __forceinline__ void bar_init(uint32_t bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-}
-// The phase's single arrival, announcing the bytes its copies will deliver.
-__device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-// Orders this thread's earlier generic shared-memory accesses before later bulk-copy writes.
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-// Bounded wait for the phase of the given parity; false if it never completed. Each poll suspends for
-// at most about 1 us (the hint, in ns), so the bound is time-like, not a count of instructions.
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-    for (int i = 0; i < WAIT_TRIES; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(1000u)
-            : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
-
-// Position of the n-th (0-based) set bit of m, or -1.
-__device__ __forceinline__ int nth_bit(unsigned long long m, int n) {
-    for (int t = 0; t < n; ++t) m &= m - 1;
-    return m ? __ffsll((long long)m) - 1 : -1;
-}
-__device__ __forceinline__ unsigned long long drop_bits(unsigned long long m, int n) {
-    for (int t = 0; t < n; ++t) m &= m - 1;
-    return m;
 }
 
 // Source of concat column c (c >= d) in the staged Gram G (row stride GS):

@@ -119,12 +119,18 @@ dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* 
 // out[n][k] = sum_{z < S} part[z][n][k] in increasing z (part split stride N * ldp)
 dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st);
 
-// Warp-per-sample fp32 interaction on pairs (interact_f32.cu), for K = 26 and d = 64 or 128.
-bool interact_pair_supported(int K, int d);
-dlrm_status launch_interact_fwd_pair(int B, int K, int d, F32Pair x_dense, const float* E, float* concat_hi,
-                                     float* concat_lo, int ldc, cudaStream_t st);
-dlrm_status launch_interact_bwd_pair(int B, int K, int d, F32Pair x_dense, const float* E, const float* dconcat,
-                                     int ldc, float* dx_hi, float* dx_lo, int lddx, float* dE, cudaStream_t st);
+// Warp-per-sample fp32 interaction of the training step with the gather fused in (interact_tc.cu):
+// fp32 tables, K + 1 <= 32, d in {32, 64, 128}; 3xTF32 on the tensor cores. The forward reads the bags
+// itself (counting skipped indices and bad bags in err) and writes the concat as a TF32 pair; the
+// backward gathers the same rows again and writes dx_dense (pair, ReLU-masked) and dE [B][K][d].
+bool interact_tc_supported(int K, int d, long long total_rows, int ldc);
+dlrm_status launch_interact_fwd_tc(const TableMeta& tm, const float* tables, int K, int d, int B,
+                                   const int32_t* offsets, const int32_t* indices, long long nnz, F32Pair x_dense,
+                                   float* concat_hi, float* concat_lo, int ldc, ErrRecord* err, cudaStream_t st);
+dlrm_status launch_interact_bwd_tc(const TableMeta& tm, const float* tables, int K, int d, int B,
+                                   const int32_t* offsets, const int32_t* indices, long long nnz, F32Pair x_dense,
+                                   const float* dconcat, int ldc, float* dx_hi, float* dx_lo, int lddx, float* dE,
+                                   ErrRecord* err, cudaStream_t st);
 
 dlrm_status launch_bce(int B, const float* z, const float* y, float* dz, float* y_hat, float* partial, float* loss,
                        cudaStream_t st);
