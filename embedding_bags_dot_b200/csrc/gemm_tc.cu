@@ -189,9 +189,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 // the leader's barrier. Each CTA's TMEM holds the 128 rows of its M half.
 // ACT_RELU_LOGIT: the layer's ReLU output h (N <= 256, one tile wide) is not
 // stored; the epilogue forms the next, one-column layer instead:
-// y[m] = sigmoid(sum_j h[m][j] w[j] + b), one thread per row summing its
-// columns in order.
+// y[m] = sigmoid(sum_j h[m][j] w[j] + b). Both epilogue warps of a TMEM lane
+// quadrant take 128 columns of the quadrant's 32 rows (one thread per row,
+// columns in order, bias and w read from shared memory); the two partial sums
+// of a row meet in a shared slot by atomic exchange, and the thread that finds
+// its partner's sum there finishes the row. No warp waits on the other.
 constexpr int ACT_RELU_LOGIT = 16;
+constexpr uint32_t LOGIT_EMPTY = 0x7FC0DEADu;   // slot holding no partial sum (a NaN no arithmetic produces)
 template <typename TW>
 struct LogitArgs {
     const TW* w;       // [N] weights of the one-column layer
@@ -234,6 +238,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars->tmem_base)),
                      "r"(TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    if constexpr (ACT == ACT_RELU_LOGIT) {
+        // each epilogue warp's (unused) output stage: [0, 128) bias and [128, 256) w of its 128 columns;
+        // the quadrant's first warp also holds the exchange slots [256, 320): two tile parities x 32 rows
+        if (warp >= 2) {
+            const int ew = warp - 2, h = ew >> 2;
+            float* bw = reinterpret_cast<float*>(gbase + STAGES2 * STAGE2_BYTES + ew * STAGE_OUT_BYTES);
+            for (int j = lane; j < BN2 / 2; j += 32) {
+                const int col = h * (BN2 / 2) + j;
+                bw[j] = col < N ? __ldg(bias + col) : 0.f;
+                bw[BN2 / 2 + j] = col < N ? Cvt<TC>::to_f(la.w[col]) : 0.f;
+            }
+            if (h == 0)
+                for (int j = lane; j < 64; j += 32) bw[BN2 + j] = __uint_as_float(LOGIT_EMPTY);
+        }
     }
     fence_before();
     cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA signal
@@ -337,28 +356,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int mb = t / nbn, nb = t - mb * nbn;
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2 + h * (BN2 / 2));
             if constexpr (ACT == ACT_RELU_LOGIT) {
-                // the first warp of each lane quadrant reads all N <= 256 columns of its 32 rows (the same TMEM
-                // lanes as its partner); the partner only releases the accumulator
-                if (h == 0) {
-                    const uint32_t row_addr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN2);
-                    float part = 0.f;
+                const float* bw = reinterpret_cast<const float*>(stage);
+                float part = 0.f;
 #pragma unroll 1
-                    for (int c = 0; c < BN2 / 32; ++c) {
-                        const int j0 = 32 * c;
-                        if (j0 >= N) break;   // uniform across the warp
-                        uint32_t r[32];
-                        tmem_ld32_issue(row_addr + 32 * c, r);
-                        tmem_ld_wait();
+                for (int c = 0; c < BN2 / 64; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_issue(taddr + 32 * c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            if (j0 + e < N) {
-                                const float v = fmaxf(__uint_as_float(r[e]) + __ldg(bias + j0 + e), 0.f);
-                                part = fmaf(v, Cvt<TC>::to_f(la.w[j0 + e]), part);
-                            }
-                        }
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 bb = *reinterpret_cast<const float4*>(bw + 32 * c + e);
+                        const float4 ww = *reinterpret_cast<const float4*>(bw + BN2 / 2 + 32 * c + e);
+                        part = fmaf(fmaxf(__uint_as_float(r[e]) + bb.x, 0.f), ww.x, part);
+                        part = fmaf(fmaxf(__uint_as_float(r[e + 1]) + bb.y, 0.f), ww.y, part);
+                        part = fmaf(fmaxf(__uint_as_float(r[e + 2]) + bb.z, 0.f), ww.z, part);
+                        part = fmaf(fmaxf(__uint_as_float(r[e + 3]) + bb.w, 0.f), ww.w, part);
                     }
+                }
+                // the row's two halves meet in the quadrant's slot for this accumulator; the slot is next used two
+                // tiles later, after both warps have released this accumulator
+                float* slot = reinterpret_cast<float*>(gbase + STAGES2 * STAGE2_BYTES + ((q + 2) & 3) * STAGE_OUT_BYTES) +
+                              BN2 + 32 * acc + lane;
+                const float other = atomicExch(slot, part);
+                if (__float_as_uint(other) != LOGIT_EMPTY) {
+                    *slot = __uint_as_float(LOGIT_EMPTY);
                     const long long row = (long long)mb * 256 + (int)rank * 128 + q * 32 + lane;
-                    if (row < M) la.y[row] = 1.f / (1.f + expf(-(part + __ldg(la.b))));
+                    if (row < M) la.y[row] = 1.f / (1.f + expf(-((part + other) + __ldg(la.b))));
                 }
             } else {
                 epilogue_tma<TC, ACT, BN2 / 2>(taddr, mb * 256 + (int)rank * 128 + q * 32, nb * BN2 + h * (BN2 / 2),
