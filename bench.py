@@ -13,9 +13,12 @@ log; the benchmark cycles a pool of 8 batches.
 
 value:  samples/s with inputs resident in HBM, device time (CUDA events),
         max over ranks; each rank runs an independent replica (weak scaling).
-e2e:    the same through dlrm_forward with every step's batch copied from pinned
-        host memory and y_hat copied back inside the timed region (the copy of
-        step i+1 runs on a copy stream while step i computes).
+e2e:    the same through dlrm_forward (dlrm_forward_cat for the concat-only
+        interaction) with every step's batch copied from pinned host memory and
+        y_hat copied back inside the timed region (the copy of step i+1 runs on
+        a copy stream while step i computes; y_hat of step i goes back on a
+        third stream while step i+1 computes, and the timing ends after the
+        last one has arrived).
 roofline: the fused gather + interaction kernel against measured HBM
         bandwidth, with algorithmic bytes = gathered rows + indices + offsets +
         x_dense read + concat write.
@@ -327,13 +330,16 @@ def run_ours(args, cfg, rank, world, local_rank):
     # memory (copy stream, two staging slots so the next batch's copy overlaps this step's forward)
     # and copies y_hat back.
     cstream = torch.cuda.Stream(dev)
-    maxn = {k: max(hb[k].numel() for hb in host_b) for k in ("dense", "offsets", "indices")}
+    ostream = torch.cuda.Stream(dev)     # y_hat device -> host, overlapping the next step's forward
+    in_keys = ("dense", "offsets", "indices")
+    maxn = {k: max(hb[k].numel() for hb in host_b) for k in in_keys}
     slots = [{k: torch.empty(maxn[k], dtype=host_b[0][k].dtype, device=dev) for k in maxn} for _ in range(2)]
     y_dev = [torch.empty(cfg.B, dtype=torch.float32, device=dev) for _ in range(2)]
     y_host = [torch.empty(cfg.B, dtype=torch.float32).pin_memory() for _ in range(2)]
     copied = [torch.cuda.Event() for _ in range(2)]
     consumed = [torch.cuda.Event() for _ in range(2)]
-    for ev in consumed:
+    read_back = [torch.cuda.Event() for _ in range(2)]
+    for ev in consumed + read_back:
         ev.record(stream)
 
     fwd = E.dlrm_forward_cat if cfg.interaction == "cat" else E.dlrm_forward
@@ -342,15 +348,19 @@ def run_ours(args, cfg, rank, world, local_rank):
         sl, hb = i & 1, host_b[i % POOL]
         cstream.wait_event(consumed[sl])
         with torch.cuda.stream(cstream):
-            for k in ("dense", "offsets", "indices"):
+            for k in in_keys:
                 slots[sl][k][:hb[k].numel()].copy_(hb[k].view(-1), non_blocking=True)
         copied[sl].record(cstream)
         stream.wait_event(copied[sl])
+        stream.wait_event(read_back[sl])          # y_dev[sl] of step i-2 has been copied out
         n = hb["indices"].numel()
         fwd(T, bot, top, cfg.B, slots[sl]["dense"], slots[sl]["offsets"], slots[sl]["indices"][:n],
-                       y_dev[sl], ws, stream)
+            y_dev[sl], ws, stream)
         consumed[sl].record(stream)
-        y_host[sl].copy_(y_dev[sl], non_blocking=True)
+        ostream.wait_event(consumed[sl])
+        with torch.cuda.stream(ostream):
+            y_host[sl].copy_(y_dev[sl], non_blocking=True)
+        read_back[sl].record(ostream)
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -360,11 +370,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     cstream.wait_event(e0)
     for i in range(args.steps):
         e2e_step(i)
+    stream.wait_stream(ostream)                   # the last step's y_hat is on the host
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    h2d = int(np.mean([sum(hb[k].numel() * hb[k].element_size() for k in ("dense", "offsets", "indices"))
-                       for hb in host_b]))
+    h2d = int(np.mean([sum(hb[k].numel() * hb[k].element_size() for k in in_keys) for hb in host_b]))
     d2h = cfg.B * 4
 
     # max over ranks

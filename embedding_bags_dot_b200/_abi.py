@@ -56,6 +56,10 @@ _SIGS = {
     "dlrm_status_str": (C.c_char_p, [C.c_int]),
     "dlrm_workspace_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
     "dlrm_mlp_workspace_size": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
+    "dlrm_forward_lengths": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                       C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_offsets_from_lengths_workspace_size": (C.c_size_t, [C.c_int64]),
+    "dlrm_offsets_from_lengths": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_check_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_embbag_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
                                   C.c_void_p, C.c_void_p]),
@@ -254,6 +258,30 @@ def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices,
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                      _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
                   "dlrm_forward")
+
+
+def dlrm_forward_lengths(T: Tables, bot: MLP, top: MLP, B: int, dense, lengths, indices, y_hat, ws, stream=None):
+    """dlrm_forward with uint8 bag lengths [K * B] in place of CSR offsets."""
+    if lengths.dtype != torch.uint8:
+        raise DlrmError(ERR_INVALID_ARG, "dlrm_forward_lengths")
+    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward_lengths")
+    return _check(lib().dlrm_forward_lengths(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(lengths),
+                                             _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws),
+                                             _stream(stream)), "dlrm_forward_lengths")
+
+
+def dlrm_offsets_from_lengths_workspace_size(n: int) -> int:
+    return int(lib().dlrm_offsets_from_lengths_workspace_size(int(n)))
+
+
+def dlrm_offsets_from_lengths(lengths, offsets, ws, stream=None):
+    """offsets[i] = sum of lengths[0..i) for i <= n; uint8 lengths [n], int32 offsets [n + 1]."""
+    n = lengths.numel()
+    if lengths.dtype != torch.uint8 or offsets.dtype != torch.int32 or offsets.numel() < n + 1:
+        raise DlrmError(ERR_INVALID_ARG, "dlrm_offsets_from_lengths")
+    _need_ws(ws, dlrm_offsets_from_lengths_workspace_size(n), "dlrm_offsets_from_lengths")
+    return _check(lib().dlrm_offsets_from_lengths(_ptr(lengths), int(n), _ptr(offsets), _ptr(ws), _stream(stream)),
+                  "dlrm_offsets_from_lengths")
 
 
 def dlrm_embbag_cat_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,

@@ -91,7 +91,7 @@ MlpWs mlp_ws(const dlrm_mlp* m, int B, dlrm_dtype in_dt) {
 }
 
 struct FwdLayout {
-    size_t x_dense, concat, act0, act1, cvt, total;
+    size_t x_dense, concat, act0, act1, cvt, offs, lscratch, total;
 };
 
 FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
@@ -112,6 +112,12 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
     off = align_up(off + h, 256);
     L.cvt = off;
     off = align_up(off + h, 256);
+    // offsets derived from bag lengths (dlrm_forward_lengths) and the scan's chunk sums
+    const long long nbags = (long long)T->K * B;
+    L.offs = off;
+    off = align_up(off + sizeof(int32_t) * (size_t)(nbags + 1), 256);
+    L.lscratch = off;
+    off = align_up(off + sizeof(int) * lengths_scratch_ints(nbags), 256);
     L.total = off;
     return L;
 }
@@ -312,6 +318,39 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
                          dlrm_stream stream) {
     return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, false);
+}
+
+dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
+                                 const float* dense, const uint8_t* lengths, const int32_t* indices, int64_t nnz,
+                                 float* y_hat, void* ws, dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_tables(T, tm);
+    if (r != DLRM_OK) return r;
+    if (B < 0 || nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
+    if (B > 0 && !lengths) return DLRM_ERR_INVALID_ARG;
+    if ((r = check_mlp(bot)) != DLRM_OK || (r = check_mlp(top)) != DLRM_OK) return r;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    const FwdLayout L = fwd_layout(T, bot, top, B);
+    char* w = static_cast<char*>(ws);
+    int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offs);
+    if ((r = launch_offsets_from_lengths(lengths, (long long)T->K * B, offsets, reinterpret_cast<int*>(w + L.lscratch),
+                                         cs(stream))) != DLRM_OK)
+        return r;
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, false);
+}
+
+size_t dlrm_offsets_from_lengths_workspace_size(int64_t n) {
+    if (n < 0) return 0;
+    return DLRM_ERR_RECORD_BYTES + sizeof(int) * lengths_scratch_ints(n);
+}
+
+dlrm_status dlrm_offsets_from_lengths(const uint8_t* lengths, int64_t n, int32_t* offsets, void* ws,
+                                      dlrm_stream stream) {
+    if (n < 0 || (n > 0 && !lengths) || !offsets) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    return launch_offsets_from_lengths(lengths, n, offsets,
+                                       reinterpret_cast<int*>(static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES), cs(stream));
 }
 
 dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,

@@ -38,6 +38,10 @@ dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, i
                           ErrRecord* err, cudaStream_t st);
 
 // out[b][c] = in[b][c] (converted) for c < K, zero up to ldo.
+// offsets[i] = sum of lengths[0..i) for i <= n, uint8 lengths (lengths.cu); scratch: lengths_scratch_ints(n) ints.
+size_t lengths_scratch_ints(long long n);
+dlrm_status launch_offsets_from_lengths(const uint8_t* lengths, long long n, int32_t* offsets, int* scratch,
+                                        cudaStream_t st);
 dlrm_status launch_convert(int B, int K, const void* in, dlrm_dtype in_dt, int ldi, void* out, dlrm_dtype out_dt,
                            int ldo, cudaStream_t st);
 

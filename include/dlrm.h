@@ -178,6 +178,28 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat,
                          void* ws, dlrm_stream stream);
 
+/* dlrm_forward with the bags given by their lengths instead of CSR offsets
+ * (the pages fix no input format; this is a compact form of the same bags):
+ *   lengths  uint8 [K * B], bag (k, b) at k * B + b (the order of the
+ *            offsets), each bag's index count (at most 255); the bags'
+ *            indices follow one another in `indices` in that order.
+ * The offsets are derived on the device into the workspace (prefix sums), so
+ * a caller copying inputs from host memory moves 1 byte per bag instead of 4.
+ * The result is identical to dlrm_forward on offsets[i] = sum of
+ * lengths[0..i). Lengths that do not add up to nnz are caught like bad offsets.
+ * Workspace: dlrm_workspace_size(T, bot, top, B, 0). */
+dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
+                                 const float* dense, const uint8_t* lengths, const int32_t* indices, int64_t nnz,
+                                 float* y_hat, void* ws, dlrm_stream stream);
+
+/* offsets[i] = sum_{j < i} lengths[j] for 0 <= i <= n (int32 out, device
+ * pointers, the scan dlrm_forward_lengths runs). ws: 16-byte aligned,
+ * dlrm_offsets_from_lengths_workspace_size(n) bytes (error record, then the
+ * scan's chunk sums). The total must stay below 2^31. */
+size_t dlrm_offsets_from_lengths_workspace_size(int64_t n);
+dlrm_status dlrm_offsets_from_lengths(const uint8_t* lengths, int64_t n, int32_t* offsets, void* ws,
+                                      dlrm_stream stream);
+
 /* ------------------------------------------------------------ training step
  * fp32 tables and MLPs only (DLRM_ERR_UNSUPPORTED otherwise); d % 4 == 0.
  * The pages state the loss ([N] Key Method Details: binary cross-entropy);
