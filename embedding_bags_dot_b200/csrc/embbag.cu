@@ -585,6 +585,8 @@ static dlrm_status launch_cat_out(const TableMeta& tm, const void* tables, int K
 dlrm_status launch_embbag_cat(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
                               const int32_t* offsets, const int32_t* indices, long long nnz, const float* x_dense,
                               void* out, int ld, dlrm_dtype out_dt, ErrRecord* err, cudaStream_t st) {
+    if (embbag_cat_bulk_supported(dt, out_dt, K, d, ld, out, tm.base[K - 1] + tm.rows[K - 1]))
+        return launch_embbag_cat_bulk(tm, tables, dt, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st);
     Geometry g;
     if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     if ((size_t)sizeof(int) * K * 33 + (size_t)K * 32 > kSmemMax) return DLRM_ERR_UNSUPPORTED;

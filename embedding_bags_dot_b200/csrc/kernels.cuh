@@ -22,6 +22,13 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
 
 // Tensor-core (mma.sync) variant of launch_embbag_interact for bf16 tables with
 // d in {32, 64, 128, 256} and K + 2 <= 64; launch_embbag_interact picks it when supported.
+// Concat-only interaction for tables stored in the concat's dtype (embbag_cat_bulk.cu): each sample's row is
+// assembled in shared memory from bulk-copied table rows and written with one bulk store.
+bool embbag_cat_bulk_supported(dlrm_dtype dt, dlrm_dtype out_dt, int K, int d, int ld, const void* out,
+                               long long total_rows);
+dlrm_status launch_embbag_cat_bulk(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
+                                   const int32_t* offsets, const int32_t* indices, long long nnz,
+                                   const float* x_dense, void* out, int ld, ErrRecord* err, cudaStream_t st);
 bool embbag_interact_mma_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
                                    long long total_rows);
 dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
