@@ -88,6 +88,10 @@ def read_peaks():
 
 # the files the fused gather + interaction kernel is compiled from (its traffic record is keyed on them)
 K2_SOURCES = ("embedding_bags_dot_b200/csrc/embbag_mma.cu", "embedding_bags_dot_b200/csrc/async_copy.cuh")
+CAT_SOURCES = ("embedding_bags_dot_b200/csrc/embbag_cat_bulk.cu", "embedding_bags_dot_b200/csrc/async_copy.cuh")
+# full-size DRAM traffic records of the dominant kernel, per workload: (summary, the kernel's sources)
+TRAFFIC = {"large": ("profiles/embbag_interact_large_traffic.json", K2_SOURCES),
+           "large-cat": ("profiles/embbag_cat_large_traffic.json", CAT_SOURCES)}
 
 
 def source_hash(src_rels) -> str:
@@ -394,7 +398,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                "sample": f"{used} random samples of batch 0, fp64 forward in {dt:.1f} s"}
 
     if rank == 0:
-        traffic = kernel_traffic("profiles/embbag_interact_large_traffic.json", K2_SOURCES) if cfg.name == "large" else None
+        traffic = kernel_traffic(*TRAFFIC[cfg.name]) if cfg.name in TRAFFIC else None
         out = {
             "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -405,7 +409,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                              f"and a {POOL}-batch pool of {pool_bytes / 1e6:.0f} MB exceed the {L2_BYTES >> 20} MB L2"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
                          "frac": achieved / peak_hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": ("embbag_cat_kernel (dlrm_embbag_cat_fwd)" if cfg.interaction == "cat" else
+                         "kernel": ("embbag_cat_bulk_kernel (dlrm_embbag_cat_fwd)" if cfg.interaction == "cat" else
                                     "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
                                     if cfg.table_dtype in ("bf16", "u8row")
                                     else "embbag_interact_kernel (dlrm_embbag_interact_fwd)"),
