@@ -125,3 +125,31 @@ def test_bindings_refuse_a_short_workspace_before_launching(lib):
         E.dlrm_mlp_fwd(mlp, B, x, 13, out, 128, E.ACT_RELU, torch.zeros(need - 16, dtype=torch.uint8))
     assert e.value.status == E.ERR_WORKSPACE
     assert E.dlrm_launch_count() == before
+
+
+def test_lengths_workspace_and_argument_checks(lib):
+    """dlrm_offsets_from_lengths needs the error record plus one int per 8,192-length chunk (and one more);
+    the bindings refuse lengths that are not uint8 and offsets that are not int32 or too short, before
+    anything is launched."""
+    import embedding_bags_dot_b200 as E
+    for n, chunks in ((0, 0), (1, 1), (8192, 1), (8193, 2), (1_703_936, 208)):
+        assert E.dlrm_offsets_from_lengths_workspace_size(n) == 256 + 4 * (chunks + 1)
+    assert E.dlrm_offsets_from_lengths_workspace_size(-1) == 0
+    before = E.dlrm_launch_count()
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    for lens, offs in ((torch.zeros(10, dtype=torch.int32), torch.zeros(11, dtype=torch.int32)),
+                       (torch.zeros(10, dtype=torch.uint8), torch.zeros(11, dtype=torch.int64)),
+                       (torch.zeros(10, dtype=torch.uint8), torch.zeros(10, dtype=torch.int32))):
+        with pytest.raises(E.DlrmError) as e:
+            E.dlrm_offsets_from_lengths(lens, offs, ws)
+        assert e.value.status == E.ERR_INVALID_ARG
+    with pytest.raises(E.DlrmError) as e:
+        E.dlrm_offsets_from_lengths(torch.zeros(100_000, dtype=torch.uint8), torch.zeros(100_001, dtype=torch.int32),
+                                    torch.zeros(64, dtype=torch.uint8))
+    assert e.value.status == E.ERR_WORKSPACE
+    mlp = _cpu_mlp([13, 64], "f32")
+    with pytest.raises(E.DlrmError) as e:
+        E.dlrm_forward_lengths(None, mlp, mlp, 4, torch.zeros((4, 13)), torch.zeros(8, dtype=torch.int32),
+                               torch.zeros(8, dtype=torch.int32), torch.zeros(4), ws)
+    assert e.value.status == E.ERR_INVALID_ARG
+    assert E.dlrm_launch_count() == before
