@@ -131,9 +131,10 @@ dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* 
 dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st);
 
 // Warp-per-sample fp32 interaction of the training step with the gather fused in (interact_tc.cu):
-// fp32 tables, K + 1 <= 32, d in {32, 64, 128}; 3xTF32 on the tensor cores. The forward reads the bags
-// itself (counting skipped indices and bad bags in err) and writes the concat as a TF32 pair; the
-// backward gathers the same rows again and writes dx_dense (pair, ReLU-masked) and dE [B][K][d].
+// fp32 tables, K = 26, d in {64, 128}. The forward reads the bags itself (counting skipped indices and
+// bad bags in err), forms the Gram as 3xTF32 on the tensor cores and writes the concat as a TF32 pair;
+// the backward gathers the same rows again and writes dx_dense (pair, ReLU-masked) and dE [B][K][d]
+// from the CUDA cores.
 bool interact_tc_supported(int K, int d, long long total_rows, int ldc);
 dlrm_status launch_interact_fwd_tc(const TableMeta& tm, const float* tables, int K, int d, int B,
                                    const int32_t* offsets, const int32_t* indices, long long nnz, F32Pair x_dense,
