@@ -30,6 +30,9 @@ def _cases():
                                                                         top=(64 * 27, 256, 1), seed=3),
         "cat-f16-d5": shrink(t, B=45, rows_cap=50).with_(d=5, table_dtype="f16", mlp_dtype="f16", bag="mix",
                                                          interaction="cat", bottom=(13, 8, 5), top=(45, 16, 1)),
+        # f16 tables into an f16 concat (the forward's): rows assembled in shared memory, one bulk store each
+        "cat-d64-f16-mix": shrink(m, B=77, rows_cap=2000).with_(table_dtype="f16", mlp_dtype="f16", bag="mix",
+                                                                interaction="cat", top=(64 * 27, 256, 1), seed=8),
     }
 
 

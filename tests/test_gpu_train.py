@@ -177,3 +177,26 @@ def test_training_step_is_bit_reproducible():
         results.append([t.g.tables.cpu()] + [w.cpu() for w in t.g.bot.Ws + t.g.top.Ws + t.g.bot.bs + t.g.top.bs])
     for a, b in zip(*results):
         assert torch.equal(a, b)
+
+
+def test_training_step_with_skipped_indices():
+    """Out-of-range indices in a training batch (the fused interaction's forward validates the bags): they
+    are skipped exactly where the oracle skips them, counted once per occurrence by the forward, and the
+    loss and y_hat still follow the oracle."""
+    cfg = shrink(CONFIGS["train"], B=150, rows_cap=1500).with_(name="train-oob", bag="mix", seed=11)
+    t = Trainer(cfg)
+    idx = t.batch.indices.copy()
+    idx[::9] = 10 ** 7                                  # past the end of every table
+    t.bt["indices"] = torch.from_numpy(idx).cuda()
+    g = t.g
+    loss = torch.zeros(1, device="cuda")
+    y = torch.zeros(cfg.B, device="cuda")
+    E.dlrm_backward(g.T, g.bot, g.top, cfg.B, t.bt["dense"], t.bt["offsets"], t.bt["indices"], t.bt["labels"],
+                    t.grads, g.ws, loss=loss, y_hat=y)
+    st = E.dlrm_check_error(g.ws)
+    ref = O.train_grads(O.model_from_config(cfg), t.batch.dense, t.batch.offsets, idx, t.batch.labels, scales=True)
+    n_oob = int(ref["counts"][0])
+    assert n_oob == idx[::9].size
+    assert st[0] == E.ERR_INDEX_OOB and st[2] == n_oob, (st, n_oob)
+    assert abs(float(loss.item()) - ref["loss"]) <= RTOL * abs(ref["loss"])
+    assert np.abs(to_np(y) - ref["y_hat"]).max() <= RTOL
