@@ -165,8 +165,33 @@ __global__ void convert_kernel(int B, int K, const TI* __restrict__ in, int ldi,
     }
 }
 
+// One thread per row, 16-bit output rows written as 16-byte chunks (ldo % 8 == 0, 16-byte aligned rows):
+// no per-element index division.
+template <typename TI, typename TO>
+__global__ void convert_rows_kernel(int B, int K, const TI* __restrict__ in, int ldi, TO* __restrict__ out, int ldo) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
+        const TI* src = in + (long long)b * ldi;
+        TO* dst = out + (long long)b * ldo;
+        for (int c0 = 0; c0 < ldo; c0 += 8) {
+            TO t[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = Cvt<TO>::from_f(c0 + e < K ? Cvt<TI>::to_f(src[c0 + e]) : 0.f);
+            *reinterpret_cast<uint4*>(dst + c0) = *reinterpret_cast<const uint4*>(t);
+        }
+    }
+}
+
 template <typename TI>
 static void convert_to(int B, int K, const void* in, int ldi, void* out, dlrm_dtype out_dt, int ldo, cudaStream_t st) {
+    if (out_dt != DLRM_F32 && ldo % 8 == 0 && ((uintptr_t)out & 15) == 0) {
+        const int blocks = (B + 255) / 256 < 148 * 8 ? (B + 255) / 256 : 148 * 8;
+        const TI* i = static_cast<const TI*>(in);
+        if (out_dt == DLRM_BF16)
+            convert_rows_kernel<TI, __nv_bfloat16><<<blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__nv_bfloat16*>(out), ldo);
+        else
+            convert_rows_kernel<TI, __half><<<blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__half*>(out), ldo);
+        return;
+    }
     long long blocks = ((long long)B * ldo + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
