@@ -196,8 +196,8 @@ def run_reference(args, cfg, rank):
     if rank != 0:
         return 0
     batch = gen.make_batches(cfg, (0,))[0]
-    # size one step at about 1/(steps + warmup) of ~2 minutes of CPU time
-    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    # size one step at 1/(steps + warmup) of ~2 minutes of CPU time, whatever the step count
+    budget = 120.0 / max(1, args.steps + args.warmup)
     rate0, _, cores, _ = oracle_rate(cfg, batch, 32)
     n = int(min(cfg.B, max(16, rate0 * budget)))
     for w in range(args.warmup):
@@ -661,7 +661,9 @@ def run_latency(args, cfg, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 1000 for a forward workload, 100 for training, 20 for the "
+                         "reference arm and --latency; long enough for several clock samples)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="large", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -674,6 +676,10 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = CONFIGS[args.workload]
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" or args.latency else (100 if cfg.training else 1000)
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
     if args.batch or args.rows_cap:
         from synth import shrink
         cfg = shrink(cfg, B=args.batch, rows_cap=args.rows_cap, name=f"{cfg.name}-profile")
