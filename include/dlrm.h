@@ -223,7 +223,11 @@ dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const 
  * gradients of the mean loss for every MLP weight and bias, the gradient of
  * every pooled bag, and the occurrences of the batch sorted by table row
  * (stable, so equal rows keep occurrence order). loss (device, 1 float) and
- * y_hat (device, fp32 [B]) are optional outputs. Bit-reproducible. */
+ * y_hat (device, fp32 [B]) are optional outputs. Bit-reproducible.
+ * Skipped (out-of-range) indices and bags with bad offsets are handled as in
+ * dlrm_forward and counted once per call in the error record at the start of
+ * `ws` (read with dlrm_check_error); occurrences beyond the gradient buffer's
+ * capacity (nnz larger than the one it was sized for) are counted as bad. */
 dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                           const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
                           float* loss, float* y_hat, void* grads, void* ws, dlrm_stream stream);
