@@ -288,67 +288,6 @@ static void linear_backward(int B, int n_in, int n_out, const double* W, const d
     }
 }
 
-/* ---- magnitude companions (error yardstick for fp32 results; not part of the method)
- *
- * First-order running error bounds: every computed quantity gets a "size",
- * the same computation run on absolute values, so that its rounding error in
- * fp32 is a small multiple of u * size. Forward: size(W a + b) = |W| size(a)
- * + |b|; a ReLU unit is dropped (size 0, exact zero output) only when its
- * pre-activation is below zero by more than kink_eps of its size, since one
- * that close to zero may take either branch in fp32. Backward: the size of a
- * gradient sums |upstream gradient size| x |W| or x size(activation). */
-
-/* Forward size of one layer: fs_out[b][o] for every sample. */
-static void linear_forward_magnitude(int B, int n_in, int n_out, const double* W, const double* bias,
-                                     const double* A, const double* fs_in, double* fs_out, int relu,
-                                     double kink_eps) {
-#pragma omp parallel for schedule(static)
-    for (int b = 0; b < B; ++b) {
-        for (int o = 0; o < n_out; ++o) {
-            const double* w = W + (int64_t)o * n_in;
-            double pre = bias[o], size = fabs(bias[o]);
-            for (int i = 0; i < n_in; ++i) {
-                pre += w[i] * A[(int64_t)b * n_in + i];
-                size += fabs(w[i]) * fs_in[(int64_t)b * n_in + i];
-            }
-            fs_out[(int64_t)b * n_out + o] = (!relu || pre > 0.0 || fabs(pre) <= kink_eps * size) ? size : 0.0;
-        }
-    }
-}
-
-/* Backward size of one layer: sY (size of dL/d output) is dropped where the
- * unit's forward size is 0, then sW = sum_b sY fs_A, sb = sum_b sY, sA = sY |W|. */
-static void linear_backward_magnitude(int B, int n_in, int n_out, const double* W, const double* fs_A,
-                                      const double* fs_Y, double* sY, double* sW, double* sb, double* sA, int relu) {
-    if (relu) {
-        for (int64_t q = 0; q < (int64_t)B * n_out; ++q)
-            if (!(fs_Y[q] > 0.0)) sY[q] = 0.0;
-    }
-#pragma omp parallel for schedule(static)
-    for (int o = 0; o < n_out; ++o) {
-        double a = 0.0;
-        for (int b = 0; b < B; ++b) a += sY[(int64_t)b * n_out + o];
-        if (sb) sb[o] = a;
-        if (sW) {
-            for (int i = 0; i < n_in; ++i) {
-                double s = 0.0;
-                for (int b = 0; b < B; ++b) s += sY[(int64_t)b * n_out + o] * fs_A[(int64_t)b * n_in + i];
-                sW[(int64_t)o * n_in + i] = s;
-            }
-        }
-    }
-    if (sA) {
-#pragma omp parallel for schedule(static)
-        for (int b = 0; b < B; ++b) {
-            for (int i = 0; i < n_in; ++i) {
-                double s = 0.0;
-                for (int o = 0; o < n_out; ++o) s += sY[(int64_t)b * n_out + o] * fabs(W[(int64_t)o * n_in + i]);
-                sA[(int64_t)b * n_in + i] = s;
-            }
-        }
-    }
-}
-
 /* Forward + backward of the whole model on one batch.
  * Outputs:
  *   loss                      mean BCE
@@ -356,18 +295,12 @@ static void linear_backward_magnitude(int B, int n_in, int n_out, const double* 
  *   bot_dW[l] [out][in], bot_db[l] [out], top_dW[l], top_db[l]: batch-summed gradients of the mean loss
  *   table_grad [sum rows][d]  gradient of every table row (zero for rows no valid index touches)
  *   row_count  [sum rows]     number of valid occurrences of each row in the batch
- *   counts[0..1]              as oracle_embbag
- * Optional (NULL to skip): *_s arrays of the same shapes receive, for every
- * gradient, the size of what it sums: the same backward chain run on
- * magnitudes (|dL/dz|, |W|, |activations|), an error yardstick for the fp32
- * GPU result; not part of the method. */
+ *   counts[0..1]              as oracle_embbag */
 void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* dense,
                         const int32_t* offsets, const int32_t* indices, const double* labels,
                         double* loss, double* y_hat,
                         double* const* bot_dW, double* const* bot_db, double* const* top_dW, double* const* top_db,
-                        double* table_grad, int64_t* row_count, long* counts,
-                        double* const* bot_dW_s, double* const* bot_db_s, double* const* top_dW_s,
-                        double* const* top_db_s, double* table_grad_s) {
+                        double* table_grad, int64_t* row_count, long* counts) {
     int K = M->K, d = M->d;
     int width = d + K * (K + 1) / 2;
     int64_t* base = (int64_t*)malloc(sizeof(int64_t) * (K > 0 ? K : 1));
@@ -476,110 +409,6 @@ void oracle_train_grads(const oracle_model* M, int B, long nnz, const double* de
     }
     free(dX); free(dY);
 
-    /* Magnitude companion pass (only when scales are requested). */
-    if (bot_dW_s || bot_db_s || top_dW_s || top_db_s || table_grad_s) {
-        const double KINK_EPS = 1e-4;   /* well above the fp32 forward's relative rounding */
-        double** bfs = (double**)malloc(sizeof(double*) * (M->n_bot + 1));
-        double** tfs = (double**)malloc(sizeof(double*) * (M->n_top + 1));
-        for (int l = 0; l <= M->n_bot; ++l) bfs[l] = (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]);
-        for (int l = 0; l <= M->n_top; ++l) tfs[l] = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
-        for (int64_t q = 0; q < (int64_t)B * M->bot_dims[0]; ++q) bfs[0][q] = fabs(dense[q]);
-        for (int l = 0; l < M->n_bot; ++l)
-            linear_forward_magnitude(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], M->bot_b[l], bot_act[l],
-                                     bfs[l], bfs[l + 1], 1, KINK_EPS);
-        const double* xfs = bfs[M->n_bot];
-        /* pooled sizes: sum of |rows| of each bag */
-        double* Efs = (double*)calloc((size_t)B * (K > 0 ? K : 1) * d, sizeof(double));
-        for (int k = 0; k < K; ++k)
-            for (int b = 0; b < B; ++b) {
-                int64_t start = offsets[(int64_t)k * B + b], end = offsets[(int64_t)k * B + b + 1];
-                if (start < 0 || end < start || end > nnz) continue;
-                double* e = Efs + ((int64_t)b * K + k) * d;
-                for (int64_t p = start; p < end; ++p) {
-                    int64_t r = indices[p];
-                    if (r < 0 || r >= M->rows[k]) continue;
-                    for (int t = 0; t < d; ++t) e[t] += fabs(M->tables[(base[k] + r) * d + t]);
-                }
-            }
-        /* concat sizes */
-#pragma omp parallel for schedule(static)
-        for (int b = 0; b < B; ++b) {
-            double* c = tfs[0] + (int64_t)b * width;
-            for (int t = 0; t < d; ++t) c[t] = xfs[(int64_t)b * d + t];
-            int p = d;
-            for (int i = 1; i <= K; ++i)
-                for (int j = 0; j < i; ++j) {
-                    const double* fi = Efs + ((int64_t)b * K + (i - 1)) * d;
-                    const double* fj = (j == 0) ? xfs + (int64_t)b * d : Efs + ((int64_t)b * K + (j - 1)) * d;
-                    double s2 = 0.0;
-                    for (int t = 0; t < d; ++t) s2 += fi[t] * fj[t];
-                    c[p++] = s2;
-                }
-        }
-        for (int l = 0; l < M->n_top; ++l)
-            linear_forward_magnitude(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], M->top_b[l], top_act[l],
-                                     tfs[l], tfs[l + 1], l < M->n_top - 1, KINK_EPS);
-        /* backward sizes: |dL/dz| plus the sigmoid's slope (<= 1/4) times the logit's size */
-        double* sY = (double*)malloc(sizeof(double) * (size_t)B);
-        for (int b = 0; b < B; ++b) sY[b] = (fabs(sigmoid(z[b]) - labels[b]) + 0.25 * tfs[M->n_top][b]) / B;
-        for (int l = M->n_top - 1; l >= 0; --l) {
-            double* sA = (double*)malloc(sizeof(double) * (size_t)B * M->top_dims[l]);
-            linear_backward_magnitude(B, M->top_dims[l], M->top_dims[l + 1], M->top_W[l], tfs[l], tfs[l + 1], sY,
-                                      top_dW_s ? top_dW_s[l] : NULL, top_db_s ? top_db_s[l] : NULL, sA,
-                                      l < M->n_top - 1);
-            free(sY);
-            sY = sA;
-        }
-        double* sX = (double*)calloc((size_t)B * (K + 1) * d, sizeof(double));
-#pragma omp parallel for schedule(static)
-        for (int b = 0; b < B; ++b) {
-            const double* sc = sY + (int64_t)b * width;
-            double* g = sX + (int64_t)b * (K + 1) * d;
-            for (int t = 0; t < d; ++t) g[t] += sc[t];
-            int p = d;
-            for (int i = 1; i <= K; ++i) {
-                const double* fi = Efs + ((int64_t)b * K + (i - 1)) * d;
-                for (int j = 0; j < i; ++j) {
-                    const double* fj = (j == 0) ? xfs + (int64_t)b * d : Efs + ((int64_t)b * K + (j - 1)) * d;
-                    double sz = sc[p++];
-                    for (int t = 0; t < d; ++t) {
-                        g[(int64_t)i * d + t] += sz * fj[t];
-                        g[(int64_t)j * d + t] += sz * fi[t];
-                    }
-                }
-            }
-        }
-        double* sB = (double*)malloc(sizeof(double) * (size_t)B * d);
-        for (int b = 0; b < B; ++b) memcpy(sB + (int64_t)b * d, sX + (int64_t)b * (K + 1) * d, sizeof(double) * d);
-        for (int l = M->n_bot - 1; l >= 0; --l) {
-            double* sA = (l > 0) ? (double*)malloc(sizeof(double) * (size_t)B * M->bot_dims[l]) : NULL;
-            linear_backward_magnitude(B, M->bot_dims[l], M->bot_dims[l + 1], M->bot_W[l], bfs[l], bfs[l + 1], sB,
-                                      bot_dW_s ? bot_dW_s[l] : NULL, bot_db_s ? bot_db_s[l] : NULL, sA, 1);
-            free(sB);
-            sB = sA;
-        }
-        if (table_grad_s) {
-            memset(table_grad_s, 0, sizeof(double) * (size_t)total_rows * d);
-            for (int k = 0; k < K; ++k)
-                for (int b = 0; b < B; ++b) {
-                    int64_t start = offsets[(int64_t)k * B + b], end = offsets[(int64_t)k * B + b + 1];
-                    if (start < 0 || end < start || end > nnz) continue;
-                    const double* g = sX + ((int64_t)b * (K + 1) + (k + 1)) * d;
-                    for (int64_t p = start; p < end; ++p) {
-                        int64_t r = indices[p];
-                        if (r < 0 || r >= M->rows[k]) continue;
-                        for (int t = 0; t < d; ++t) table_grad_s[(base[k] + r) * d + t] += g[t];
-                    }
-                }
-        }
-        free(sX);
-        free(sY);
-        free(Efs);
-        for (int l = 0; l <= M->n_bot; ++l) free(bfs[l]);
-        for (int l = 0; l <= M->n_top; ++l) free(tfs[l]);
-        free(bfs);
-        free(tfs);
-    }
     for (int l = 0; l <= M->n_bot; ++l) free(bot_act[l]);
     for (int l = 0; l <= M->n_top; ++l) free(top_act[l]);
     free(bot_act); free(top_act); free(E); free(lens); free(base);

@@ -65,8 +65,7 @@ def _declare(lib):
     lib.oracle_forward.argtypes = [vp, i, l, vp, vp, vp, vp, vp, vp]
     lib.oracle_bce.argtypes = [i, vp, vp]
     lib.oracle_bce.restype = d
-    lib.oracle_train_grads.argtypes = [vp, i, l, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                       vp, vp, vp, vp, vp]
+    lib.oracle_train_grads.argtypes = [vp, i, l, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.oracle_sgd.argtypes = [C.c_int64, d, vp, vp]
     lib.oracle_quantize_rows_u8.argtypes = [C.c_int64, i, vp, vp, vp, vp]
     lib.oracle_concat.argtypes = [i, i, i, vp, vp, vp]
@@ -269,9 +268,8 @@ def bce(z, y, lib=None) -> float:
     return float(lib.oracle_bce(z.size, _p(z), _p(y)))
 
 
-def train_grads(model: Model, dense, offsets, indices, labels, lib=None, scales: bool = False) -> dict:
-    """Loss, y_hat, all MLP gradients, per-row table gradients and occurrence counts.
-    With scales=True also the sum of |terms| of every batch-summed gradient (keys *_s)."""
+def train_grads(model: Model, dense, offsets, indices, labels, lib=None) -> dict:
+    """Loss, y_hat, all MLP gradients, per-row table gradients and occurrence counts."""
     lib = lib or load()
     dense, offsets, indices, labels = _c64(dense), _i32(offsets), _i32(indices), _c64(labels)
     B = dense.shape[0]
@@ -286,19 +284,9 @@ def train_grads(model: Model, dense, offsets, indices, labels, lib=None, scales:
     y = np.zeros(B, np.float64)
     counts = np.zeros(2, np.int64)
     out = {}
-    if scales:
-        sc = {k: [np.zeros_like(a) for a in v] for k, v in (("bot_dW_s", bdW), ("bot_db_s", bdb), ("top_dW_s", tdW),
-                                                              ("top_db_s", tdb))}
-        sc["table_grad_s"] = np.zeros_like(tg)
-        extra = [ptr(sc["bot_dW_s"]), ptr(sc["bot_db_s"]), ptr(sc["top_dW_s"]), ptr(sc["top_db_s"]),
-                 _p(sc["table_grad_s"])]
-        out.update(sc)
-    else:
-        extra = [None] * 5
     s = model.struct()
     lib.oracle_train_grads(C.byref(s), B, indices.size, _p(dense), _p(offsets), _p(indices), _p(labels),
-                           _p(loss), _p(y), ptr(bdW), ptr(bdb), ptr(tdW), ptr(tdb), _p(tg), _p(cnt), _p(counts),
-                           *extra)
+                           _p(loss), _p(y), ptr(bdW), ptr(bdb), ptr(tdW), ptr(tdb), _p(tg), _p(cnt), _p(counts))
     out.update({"loss": float(loss[0]), "y_hat": y, "bot_dW": bdW, "bot_db": bdb, "top_dW": tdW, "top_db": tdb,
                 "table_grad": tg, "row_count": cnt, "counts": (int(counts[0]), int(counts[1]))})
     return out

@@ -8,6 +8,8 @@ import pytest
 import torch
 
 import embedding_bags_dot_b200 as E
+import error_bound as EB
+import train_checks as TC
 from gpucase import GpuModel, assert_close, scale_concat, to_np
 from oracle import oracle as O
 from synth import CONFIGS, gen
@@ -106,13 +108,12 @@ def test_train_step_full_size():
     S = np.array(sorted(sample_set))
     Bs, dense, offs3, idx3, labels3, rws3, used3 = O.sub_batch(cfg, batch, S)
     m3 = O.model_for_rows(cfg, used3)
-    ref = O.train_grads(m3, dense, offs3, idx3, labels3, scales=True)
+    ref = O.train_grads(m3, dense, offs3, idx3, labels3)
+    bd = EB.bounds(m3, dense, offs3, idx3, labels3, oracle_grads=ref)
     factor = Bs / cfg.B   # the oracle's mean over |S| samples vs the GPU's mean over B
     got_g = to_np(rg[torch.from_numpy(pick).long().cuda()])
     for q, (r, k) in enumerate(zip(uk[pick], table_of)):
         local_row = np.searchsorted(used3[k], r - base[k])
         ci = int(np.sum([len(u) for u in used3[:k]])) + local_row
-        want = ref["table_grad"][ci] * factor
-        sc = ref["table_grad_s"][ci] * factor
-        err = np.abs(got_g[q] - want)
-        assert np.all(err <= 1e-5 * (np.abs(want) + sc)), (q, float(err.max()), float(sc.max()))
+        TC.check_grad(got_g[q], ref["table_grad"][ci] * factor, bd["table_grad_S2"][ci] * factor,
+                      bd["table_grad_F"][ci] * factor, f"full-size row {r}")
