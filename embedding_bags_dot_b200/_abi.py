@@ -52,50 +52,53 @@ _lock = threading.Lock()
 
 _SIGS = {
     "dlrm_launch_count": (C.c_uint64, []),
+    "dlrm_set_wait_polls": (C.c_int, [C.c_int64]),
     "dlrm_ld": (C.c_int, [C.c_int, C.c_int]),
     "dlrm_status_str": (C.c_char_p, [C.c_int]),
     "dlrm_workspace_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
     "dlrm_mlp_workspace_size": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
     "dlrm_forward_lengths": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
-                                       C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+                                       C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_offsets_from_lengths_workspace_size": (C.c_size_t, [C.c_int64]),
-    "dlrm_offsets_from_lengths": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
-    "dlrm_check_error": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_offsets_from_lengths": (C.c_int, [C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "dlrm_check_error": (C.c_int, [C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p]),
     "dlrm_embbag_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
-                                  C.c_void_p, C.c_void_p]),
+                                  C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_interact_fwd": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int,
                                     C.c_void_p]),
     "dlrm_embbag_interact_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p,
-                                           C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+                                           C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_mlp_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int,
-                               C.c_void_p, C.c_void_p]),
+                               C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_forward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
-                               C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+                               C.c_int64, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_grads_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64]),
     "dlrm_grads_offsets": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_backward": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
-                                C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+                                C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
+                                C.c_size_t, C.c_void_p]),
     "dlrm_sparse_sgd": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_void_p,
-                                  C.c_void_p, C.c_void_p]),
+                                  C.c_size_t, C.c_void_p, C.c_void_p]),
     "dlrm_embedding_row_grads": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int64, C.c_void_p,
-                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+                                           C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_forward_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                        C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
     "dlrm_row_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "dlrm_embbag_cat_fwd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p,
-                                      C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+                                      C.c_int, C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_forward_cat": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
-                                   C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]),
+                                   C.c_int64, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_quantize_rows_u8": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int, C.c_void_p, C.c_void_p]),
     "dlrm_gemm_f32": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
-                                C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+                                C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]),
     "dlrm_tf32_split": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int,
                                   C.c_void_p]),
     "dlrm_gemm_tf32x3_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_int]),
     "dlrm_gemm_tf32x3": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
-                                   C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+                                   C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_size_t,
+                                   C.c_void_p]),
 }
 
 
@@ -146,6 +149,11 @@ def _stream(stream):
 
 def dlrm_launch_count() -> int:
     return int(lib().dlrm_launch_count())
+
+
+def dlrm_set_wait_polls(polls: int) -> None:
+    """Test hook: polls of the first bounded waits on the current device (< 0: the defaults)."""
+    _check(lib().dlrm_set_wait_polls(int(polls)), "dlrm_set_wait_polls")
 
 
 def dlrm_ld(n: int, dt) -> int:
@@ -204,14 +212,11 @@ def dlrm_mlp_workspace_size(mlp: MLP, B: int, in_dt) -> int:
     return int(lib().dlrm_mlp_workspace_size(mlp.ref(), int(B), int(DT_CODE.get(in_dt, in_dt))))
 
 
-def _need_ws(ws, nbytes: int, where: str) -> None:
-    """The C entry points cannot see the workspace's size: refuse a tensor smaller than the call needs
-    before anything is launched. A size of 0 (the query found the arguments invalid) leaves the
-    diagnosis to the entry point itself."""
-    if not isinstance(ws, torch.Tensor) or nbytes <= 0:
-        return
-    if ws.numel() * ws.element_size() < nbytes:
-        raise DlrmError(ERR_WORKSPACE, where)
+def _nbytes(buf) -> int:
+    """Size in bytes of a caller buffer (a tensor), passed to the C entry points, which refuse short ones."""
+    if buf is None:
+        return 0
+    return int(buf.numel() * buf.element_size())
 
 
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
@@ -222,14 +227,14 @@ def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
 def dlrm_check_error(ws: torch.Tensor, stream=None):
     """Returns (status, flags, n_skipped_indices, n_bad_bags) and clears the record."""
     info = (C.c_int64 * 3)()
-    s = lib().dlrm_check_error(_ptr(ws), _stream(stream), info)
+    s = lib().dlrm_check_error(_ptr(ws), _nbytes(ws), _stream(stream), info)
     return int(s), int(info[0]), int(info[1]), int(info[2])
 
 
 def dlrm_embbag_fwd(T: Tables, B: int, offsets, indices, pooled, bag_len=None, ws=None, stream=None):
-    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_fwd")
     return _check(lib().dlrm_embbag_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
-                                        _ptr(pooled), _ptr(bag_len), _ptr(ws), _stream(stream)), "dlrm_embbag_fwd")
+                                        _ptr(pooled), _ptr(bag_len), _ptr(ws), _nbytes(ws), _stream(stream)),
+                  "dlrm_embbag_fwd")
 
 
 def dlrm_interact_fwd(B: int, K: int, d: int, x_dense, pooled, concat, ld: int, out_dt=None, stream=None):
@@ -241,33 +246,30 @@ def dlrm_interact_fwd(B: int, K: int, d: int, x_dense, pooled, concat, ld: int, 
 def dlrm_embbag_interact_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,
                              stream=None):
     out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
-    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_interact_fwd")
     return _check(lib().dlrm_embbag_interact_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
                                                  _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
-                                                 _stream(stream)), "dlrm_embbag_interact_fwd")
+                                                 _nbytes(ws), _stream(stream)), "dlrm_embbag_interact_fwd")
 
 
 def dlrm_mlp_fwd(mlp: MLP, B: int, inp, ld_in: int, out, ld_out: int, final_act: int, ws, stream=None):
-    _need_ws(ws, dlrm_mlp_workspace_size(mlp, B, inp.dtype) if B > 0 else ERR_RECORD_BYTES, "dlrm_mlp_fwd")
     return _check(lib().dlrm_mlp_fwd(mlp.ref(), int(B), _ptr(inp), DT_CODE[inp.dtype], int(ld_in), _ptr(out),
-                                     int(ld_out), int(final_act), _ptr(ws), _stream(stream)), "dlrm_mlp_fwd")
+                                     int(ld_out), int(final_act), _ptr(ws), _nbytes(ws), _stream(stream)),
+                  "dlrm_mlp_fwd")
 
 
 def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
-    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward")
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
-                                     _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
-                  "dlrm_forward")
+                                     _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _nbytes(ws),
+                                     _stream(stream)), "dlrm_forward")
 
 
 def dlrm_forward_lengths(T: Tables, bot: MLP, top: MLP, B: int, dense, lengths, indices, y_hat, ws, stream=None):
     """dlrm_forward with uint8 bag lengths [K * B] in place of CSR offsets."""
     if lengths.dtype != torch.uint8:
         raise DlrmError(ERR_INVALID_ARG, "dlrm_forward_lengths")
-    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward_lengths")
     return _check(lib().dlrm_forward_lengths(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(lengths),
                                              _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws),
-                                             _stream(stream)), "dlrm_forward_lengths")
+                                             _nbytes(ws), _stream(stream)), "dlrm_forward_lengths")
 
 
 def dlrm_offsets_from_lengths_workspace_size(n: int) -> int:
@@ -279,27 +281,24 @@ def dlrm_offsets_from_lengths(lengths, offsets, ws, stream=None):
     n = lengths.numel()
     if lengths.dtype != torch.uint8 or offsets.dtype != torch.int32 or offsets.numel() < n + 1:
         raise DlrmError(ERR_INVALID_ARG, "dlrm_offsets_from_lengths")
-    _need_ws(ws, dlrm_offsets_from_lengths_workspace_size(n), "dlrm_offsets_from_lengths")
-    return _check(lib().dlrm_offsets_from_lengths(_ptr(lengths), int(n), _ptr(offsets), _ptr(ws), _stream(stream)),
-                  "dlrm_offsets_from_lengths")
+    return _check(lib().dlrm_offsets_from_lengths(_ptr(lengths), int(n), _ptr(offsets), _ptr(ws), _nbytes(ws),
+                                                  _stream(stream)), "dlrm_offsets_from_lengths")
 
 
 def dlrm_embbag_cat_fwd(T: Tables, B: int, offsets, indices, x_dense, concat, ld: int, out_dt=None, ws=None,
                         stream=None):
     """Concat-only interaction: concat rows [x_dense, e_1 .. e_K, zeros]."""
     out_dt = DT_CODE[concat.dtype] if out_dt is None else DT_CODE.get(out_dt, out_dt)
-    _need_ws(ws, ERR_RECORD_BYTES, "dlrm_embbag_cat_fwd")
     return _check(lib().dlrm_embbag_cat_fwd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()),
                                             _ptr(x_dense), _ptr(concat), int(ld), int(out_dt), _ptr(ws),
-                                            _stream(stream)), "dlrm_embbag_cat_fwd")
+                                            _nbytes(ws), _stream(stream)), "dlrm_embbag_cat_fwd")
 
 
 def dlrm_forward_cat(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
     """dlrm_forward with the concat-only interaction (top MLP input width d (K + 1))."""
-    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 0), "dlrm_forward_cat")
     return _check(lib().dlrm_forward_cat(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
-                                         _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _stream(stream)),
-                  "dlrm_forward_cat")
+                                         _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _nbytes(ws),
+                                         _stream(stream)), "dlrm_forward_cat")
 
 
 def dlrm_forward_noalloc(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, err_flags=None,
@@ -333,9 +332,9 @@ def dlrm_gemm_f32(I: int, J: int, R: int, A, lda: int, a_mn: bool, B, ldb: int, 
                   stream=None):
     """C[i][j] = sum_r A(i, r) B(j, r) in fp32 on the tensor cores; A(i, r) = A[i][r], or A[r][i] when a_mn
     (B likewise)."""
-    _need_ws(ws, dlrm_gemm_f32_workspace_size(I, J, R, a_mn, b_mn), "dlrm_gemm_f32")
     return _check(lib().dlrm_gemm_f32(int(I), int(J), int(R), _ptr(A), int(lda), int(bool(a_mn)), _ptr(B), int(ldb),
-                                      int(bool(b_mn)), _ptr(C), int(ldc), _ptr(ws), _stream(stream)), "dlrm_gemm_f32")
+                                      int(bool(b_mn)), _ptr(C), int(ldc), _ptr(ws), _nbytes(ws), _stream(stream)),
+                  "dlrm_gemm_f32")
 
 
 def dlrm_tf32_split(rows: int, cols: int, src, lds: int, hi, lo, ldd: int, stream=None):
@@ -351,10 +350,9 @@ def dlrm_gemm_tf32x3_workspace_size(I: int, J: int, R: int) -> int:
 def dlrm_gemm_tf32x3(I: int, J: int, R: int, A_hi, A_lo, lda: int, a_mn: bool, B_hi, B_lo, ldb: int, b_mn: bool, C,
                      ldc: int, ws, stream=None):
     """dlrm_gemm_f32 on operands already split by dlrm_tf32_split."""
-    _need_ws(ws, dlrm_gemm_tf32x3_workspace_size(I, J, R), "dlrm_gemm_tf32x3")
     return _check(lib().dlrm_gemm_tf32x3(int(I), int(J), int(R), _ptr(A_hi), _ptr(A_lo), int(lda), int(bool(a_mn)),
                                          _ptr(B_hi), _ptr(B_lo), int(ldb), int(bool(b_mn)), _ptr(C), int(ldc),
-                                         _ptr(ws), _stream(stream)), "dlrm_gemm_tf32x3")
+                                         _ptr(ws), _nbytes(ws), _stream(stream)), "dlrm_gemm_tf32x3")
 
 
 # ----------------------------------------------------------------- training step (fp32)
@@ -376,21 +374,22 @@ def dlrm_grads_offsets(T: Tables, bot: MLP, top: MLP, B: int, nnz: int) -> dict:
 
 def dlrm_backward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, labels, grads, ws, loss=None,
                   y_hat=None, stream=None):
-    _need_ws(ws, dlrm_workspace_size(T, bot, top, B, 1), "dlrm_backward")
     return _check(lib().dlrm_backward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                       _ptr(indices), int(indices.numel()), _ptr(labels), _ptr(loss), _ptr(y_hat),
-                                      _ptr(grads), _ptr(ws), _stream(stream)), "dlrm_backward")
+                                      _ptr(grads), _nbytes(grads), _ptr(ws), _nbytes(ws), _stream(stream)),
+                  "dlrm_backward")
 
 
 def dlrm_sparse_sgd(T: Tables, bot: MLP, top: MLP, B: int, nnz: int, lr: float, grads, n_touched=None, stream=None):
     return _check(lib().dlrm_sparse_sgd(T.ref(), bot.ref(), top.ref(), int(B), int(nnz), float(lr), _ptr(grads),
-                                        _ptr(n_touched), _stream(stream)), "dlrm_sparse_sgd")
+                                        _nbytes(grads), _ptr(n_touched), _stream(stream)), "dlrm_sparse_sgd")
 
 
 def dlrm_embedding_row_grads(T: Tables, bot: MLP, top: MLP, B: int, nnz: int, grads, rows, row_grads, n_rows,
                              stream=None):
     return _check(lib().dlrm_embedding_row_grads(T.ref(), bot.ref(), top.ref(), int(B), int(nnz), _ptr(grads),
-                                                 _ptr(rows), _ptr(row_grads), _ptr(n_rows), _stream(stream)),
+                                                 _nbytes(grads), _ptr(rows), _ptr(row_grads), _ptr(n_rows),
+                                                 _stream(stream)),
                   "dlrm_embedding_row_grads")
 
 

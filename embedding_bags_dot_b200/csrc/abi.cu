@@ -170,6 +170,13 @@ extern "C" {
 
 uint64_t dlrm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+dlrm_status dlrm_set_wait_polls(int64_t polls) {
+    if (set_wait_polls_gemm_tc(polls) != cudaSuccess || set_wait_polls_embbag_mma(polls) != cudaSuccess ||
+        set_wait_polls_embbag_cat(polls) != cudaSuccess || set_wait_polls_interact_tc(polls) != cudaSuccess)
+        return DLRM_ERR_CUDA;
+    return DLRM_OK;
+}
+
 int dlrm_ld(int n, dlrm_dtype dt) {
     const int per = 16 / (int)esize(dt);
     return (n + per - 1) / per * per;
@@ -199,8 +206,9 @@ size_t dlrm_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm
     return t > f ? t : f;
 }
 
-dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info) {
+dlrm_status dlrm_check_error(void* ws, size_t ws_bytes, dlrm_stream stream, int64_t* info) {
     if (!ws) return DLRM_ERR_INVALID_ARG;
+    if (ws_bytes < DLRM_ERR_RECORD_BYTES) return DLRM_ERR_WORKSPACE;
     ErrRecord h;
     if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, cs(stream)) != cudaSuccess) return DLRM_ERR_CUDA;
     if (cudaStreamSynchronize(cs(stream)) != cudaSuccess) return DLRM_ERR_CUDA;
@@ -217,12 +225,13 @@ dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info) {
 }
 
 dlrm_status dlrm_embbag_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
-                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, dlrm_stream stream) {
+                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, size_t ws_bytes,
+                            dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
     if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < DLRM_ERR_RECORD_BYTES) return DLRM_ERR_WORKSPACE;
     if (B > 0 && (!pooled || !aligned16(pooled))) return DLRM_ERR_INVALID_ARG;
     if (B == 0) return DLRM_OK;
     return launch_embbag(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, pooled, bag_len,
@@ -242,13 +251,13 @@ dlrm_status dlrm_interact_fwd(int B, int K, int d, const float* x_dense, const f
 
 dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
                                      int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt,
-                                     void* ws, dlrm_stream stream) {
+                                     void* ws, size_t ws_bytes, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
     if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
     if (!valid_dt(out_dt) || ld < T->d + T->K * (T->K + 1) / 2) return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < DLRM_ERR_RECORD_BYTES) return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
     if (!x_dense || !concat || !aligned16(x_dense) || !aligned16(concat)) return DLRM_ERR_INVALID_ARG;
     return launch_embbag_interact(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, x_dense, concat, ld,
@@ -256,15 +265,15 @@ dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t*
 }
 
 dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out,
-                         int ld_out, int final_act, void* ws, dlrm_stream stream) {
+                         int ld_out, int final_act, void* ws, size_t ws_bytes, dlrm_stream stream) {
     dlrm_status r = check_mlp(mlp);
     if (r != DLRM_OK) return r;
     if (B < 0 || !valid_dt(in_dt) || ld_in < mlp->dims[0] || ld_out < mlp->dims[mlp->n_layers]) return DLRM_ERR_INVALID_ARG;
     if (final_act < DLRM_ACT_NONE || final_act > DLRM_ACT_SIGMOID) return DLRM_ERR_INVALID_ARG;
     if (B == 0) return DLRM_OK;
     if (!in || !out) return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
     const MlpWs L = mlp_ws(mlp, B, in_dt);
+    if (!ws || !aligned16(ws) || ws_bytes < L.total) return DLRM_ERR_WORKSPACE;
     char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
     return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + L.act, w + (size_t)L.nact * L.act,
                    static_cast<ErrRecord*>(ws), cs(stream));
@@ -275,12 +284,15 @@ size_t dlrm_mlp_workspace_size(const dlrm_mlp* mlp, int B, dlrm_dtype in_dt) {
     return mlp_ws(mlp, B, in_dt).total;
 }
 
-namespace {
+}  // extern "C"
 
-// The forward pass with the dot interaction (cat = false) or the concat-only one (cat = true).
-dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
-                         const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
-                         dlrm_stream stream, bool cat) {
+namespace dlrm {
+
+// Every host-side check of the forward pass (dot interaction, or concat-only when cat), in the order the
+// entry points apply them, before anything is launched. ws_bytes is the workspace's size.
+dlrm_status forward_check(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                          const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* y_hat,
+                          const void* ws, size_t ws_bytes, bool cat) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
@@ -290,9 +302,27 @@ dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
     const int width = cat ? d * (K + 1) : d + K * (K + 1) / 2;
     if (bot->dims[bot->n_layers] != d || top->dims[0] != width || top->dims[top->n_layers] != 1)
         return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
-    if (B == 0) return DLRM_OK;
-    if (!dense || !y_hat) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < fwd_layout(T, bot, top, B).total) return DLRM_ERR_WORKSPACE;
+    if (B > 0 && (!dense || !y_hat)) return DLRM_ERR_INVALID_ARG;
+    return DLRM_OK;
+}
+
+}  // namespace dlrm
+
+extern "C" {
+
+namespace {
+
+// The forward pass with the dot interaction (cat = false) or the concat-only one (cat = true).
+dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                         const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
+                         size_t ws_bytes, dlrm_stream stream, bool cat) {
+    dlrm_status r = forward_check(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, ws_bytes, cat);
+    if (r != DLRM_OK || B == 0) return r;
+    TableMeta tm;
+    check_tables(T, tm);
+    const int K = T->K, d = T->d;
+    const int width = cat ? d * (K + 1) : d + K * (K + 1) / 2;
     const FwdLayout L = fwd_layout(T, bot, top, B);
     char* w = static_cast<char*>(ws);
     cudaStream_t st = cs(stream);
@@ -316,13 +346,13 @@ dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
 
 dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
-                         dlrm_stream stream) {
-    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, false);
+                         size_t ws_bytes, dlrm_stream stream) {
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, ws_bytes, stream, false);
 }
 
 dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
                                  const float* dense, const uint8_t* lengths, const int32_t* indices, int64_t nnz,
-                                 float* y_hat, void* ws, dlrm_stream stream) {
+                                 float* y_hat, void* ws, size_t ws_bytes, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
@@ -334,10 +364,13 @@ dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, cons
     const FwdLayout L = fwd_layout(T, bot, top, B);
     char* w = static_cast<char*>(ws);
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offs);
+    // every check of the forward pass before the scan is launched (the scan's output stands in for the offsets)
+    if ((r = forward_check(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, ws_bytes, false)) != DLRM_OK)
+        return r;
     if ((r = launch_offsets_from_lengths(lengths, (long long)T->K * B, offsets, reinterpret_cast<int*>(w + L.lscratch),
                                          cs(stream))) != DLRM_OK)
         return r;
-    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, false);
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, ws_bytes, stream, false);
 }
 
 size_t dlrm_offsets_from_lengths_workspace_size(int64_t n) {
@@ -346,28 +379,28 @@ size_t dlrm_offsets_from_lengths_workspace_size(int64_t n) {
 }
 
 dlrm_status dlrm_offsets_from_lengths(const uint8_t* lengths, int64_t n, int32_t* offsets, void* ws,
-                                      dlrm_stream stream) {
+                                      size_t ws_bytes, dlrm_stream stream) {
     if (n < 0 || (n > 0 && !lengths) || !offsets) return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < dlrm_offsets_from_lengths_workspace_size(n)) return DLRM_ERR_WORKSPACE;
     return launch_offsets_from_lengths(lengths, n, offsets,
                                        reinterpret_cast<int*>(static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES), cs(stream));
 }
 
 dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                              const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
-                             dlrm_stream stream) {
-    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, stream, true);
+                             size_t ws_bytes, dlrm_stream stream) {
+    return forward_impl(T, bot, top, B, dense, offsets, indices, nnz, y_hat, ws, ws_bytes, stream, true);
 }
 
 dlrm_status dlrm_embbag_cat_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
                                 int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt, void* ws,
-                                dlrm_stream stream) {
+                                size_t ws_bytes, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_tables(T, tm);
     if (r != DLRM_OK) return r;
     if ((r = check_bags(B, offsets, indices, nnz)) != DLRM_OK) return r;
     if (!valid_dt(out_dt) || ld < T->d * (T->K + 1)) return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws)) return DLRM_ERR_WORKSPACE;
+    if (!ws || !aligned16(ws) || ws_bytes < DLRM_ERR_RECORD_BYTES) return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
     if (!x_dense || !concat) return DLRM_ERR_INVALID_ARG;
     return launch_embbag_cat(tm, T->data, T->dt, T->K, T->d, B, offsets, indices, nnz, x_dense, concat, ld, out_dt,

@@ -44,13 +44,13 @@ size_t dlrm_gemm_f32_workspace_size(int I, int J, int R, int a_mn, int b_mn) {
 }
 
 dlrm_status dlrm_gemm_f32(int I, int J, int R, const float* A, int lda, int a_mn, const float* B, int ldb, int b_mn,
-                          float* C, int ldc, void* ws, dlrm_stream stream) {
+                          float* C, int ldc, void* ws, size_t ws_bytes, dlrm_stream stream) {
     if (!args_ok(I, J, R) || !A || !B || !C) return DLRM_ERR_INVALID_ARG;
     const int a_cols = a_mn ? I : R, b_cols = b_mn ? J : R;
     if (lda < a_cols || ldb < b_cols || ldc < J || ldc % 4 || ((uintptr_t)C & 15)) return DLRM_ERR_INVALID_ARG;
-    if (!ws || ((uintptr_t)ws & 15)) return DLRM_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const GemmWs W = gemm_ws(I, J, R, a_mn, b_mn);
+    if (!ws || ((uintptr_t)ws & 15) || ws_bytes < W.total) return DLRM_ERR_WORKSPACE;
     char* w = static_cast<char*>(ws);
     auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
@@ -77,13 +77,13 @@ size_t dlrm_gemm_tf32x3_workspace_size(int I, int J, int R) {
 
 dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float* A_lo, int lda, int a_mn,
                              const float* B_hi, const float* B_lo, int ldb, int b_mn, float* C, int ldc, void* ws,
-                             dlrm_stream stream) {
+                             size_t ws_bytes, dlrm_stream stream) {
     if (!args_ok(I, J, R) || !A_hi || !A_lo || !B_hi || !B_lo || !C) return DLRM_ERR_INVALID_ARG;
     const int a_cols = a_mn ? I : R, b_cols = b_mn ? J : R;
     if (lda < a_cols || ldb < b_cols || ldc < J || lda % 4 || ldb % 4 || ldc % 4) return DLRM_ERR_INVALID_ARG;
     const uintptr_t al = (uintptr_t)A_hi | (uintptr_t)A_lo | (uintptr_t)B_hi | (uintptr_t)B_lo | (uintptr_t)C;
     if (al & 15) return DLRM_ERR_INVALID_ARG;
-    if (!ws || ((uintptr_t)ws & 15)) return DLRM_ERR_WORKSPACE;
+    if (!ws || ((uintptr_t)ws & 15) || ws_bytes < dlrm_gemm_tf32x3_workspace_size(I, J, R)) return DLRM_ERR_WORKSPACE;
     char* w = static_cast<char*>(ws);
     return tf32x3_gemm(I, J, R, F32Pair{A_hi, A_lo, lda}, a_mn != 0, F32Pair{B_hi, B_lo, ldb}, b_mn != 0, C, ldc,
                        reinterpret_cast<float*>(w + align_up(DLRM_ERR_RECORD_BYTES, 256)),

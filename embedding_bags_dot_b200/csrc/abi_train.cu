@@ -201,12 +201,15 @@ dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const 
 
 dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                           const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
-                          float* loss, float* y_hat, void* grads, void* ws, dlrm_stream stream) {
+                          float* loss, float* y_hat, void* grads, size_t grads_bytes, void* ws, size_t ws_bytes,
+                          dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
     if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws) || !grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
+    if (ws_bytes < dlrm_workspace_size(T, bot, top, B, 1) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
+        return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
     if (!dense || !offsets || (nnz > 0 && !indices) || !labels) return DLRM_ERR_INVALID_ARG;
     const int K = T->K, d = T->d;
@@ -341,12 +344,13 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
 }
 
 dlrm_status dlrm_sparse_sgd(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
-                            float lr, void* grads, int32_t* n_touched, dlrm_stream stream) {
+                            float lr, void* grads, size_t grads_bytes, int32_t* n_touched, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
     if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
-    if (!grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
+    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
+        return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
     const Grads G = grads_layout(T, bot, top, B, nnz);
     const char* g = static_cast<const char*>(grads);
@@ -371,13 +375,14 @@ dlrm_status dlrm_sparse_sgd(const dlrm_tables* T, const dlrm_mlp* bot, const dlr
 }
 
 dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
-                                     int64_t nnz, void* grads, uint32_t* rows, float* row_grads,
-                                     int32_t* n_rows, dlrm_stream stream) {
+                                     int64_t nnz, const void* grads, size_t grads_bytes, uint32_t* rows,
+                                     float* row_grads, int32_t* n_rows, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
     if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
-    if (!grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
+    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
+        return DLRM_ERR_WORKSPACE;
     if (!rows || !row_grads || !n_rows) return DLRM_ERR_INVALID_ARG;
     if (B == 0) return DLRM_OK;
     const Grads G = grads_layout(T, bot, top, B, nnz);

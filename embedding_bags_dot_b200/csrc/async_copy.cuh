@@ -31,10 +31,16 @@ __device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t
 }
 // Orders this thread's earlier generic shared-memory accesses before later bulk-copy writes.
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-// Bounded wait for the phase of the given parity; false if it never completed. Each poll suspends for
-// at most about 1 us (the hint, in ns), so the bound is time-like, not a count of instructions.
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-    for (int i = 0; i < WAIT_TRIES; ++i) {
+// Polls of the first wait for a sample's rows on this device (WAIT_TRIES unless a test lowered it with
+// dlrm_set_wait_polls to make that wait run out). Each translation unit that includes this header has its
+// own copy, set through its own set_rows_wait_tries_* function.
+static __device__ int g_rows_wait_tries = WAIT_TRIES;
+
+// Bounded wait for the phase of the given parity; false if it never completed within `tries` polls. Each
+// poll suspends for at most about 1 us (the hint, in ns), so the bound is time-like, not a count of
+// instructions.
+__device__ __forceinline__ bool bar_wait_n(uint32_t bar, uint32_t parity, int tries) {
+    for (int i = 0; i < tries; ++i) {
         uint32_t ok;
         asm volatile(
             "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
@@ -44,6 +50,24 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
         if (ok) return true;
     }
     return false;
+}
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) { return bar_wait_n(bar, parity, WAIT_TRIES); }
+
+// The warp's wait for the rows of one phase (call with the whole warp converged), first with `tries` polls
+// (a kernel reads g_rows_wait_tries once at its start). If any lane gives up, every lane waits again with
+// the full bound, so that no copy is still landing in the region when the caller stops using it, and
+// false is returned on every lane.
+__device__ __forceinline__ bool rows_ready(uint32_t bar, uint32_t parity, int tries) {
+    const bool ok = bar_wait_n(bar, parity, tries);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    bar_wait_n(bar, parity, WAIT_TRIES);
+    return false;
+}
+
+// Host side: sets this translation unit's first-wait bound on the current device (tries < 0: the default).
+static inline cudaError_t set_rows_wait_tries_here(int tries) {
+    const int v = tries < 0 ? WAIT_TRIES : tries;
+    return cudaMemcpyToSymbol(g_rows_wait_tries, &v, sizeof(v));
 }
 
 // Position of the n-th (0-based) set bit of m, or -1.

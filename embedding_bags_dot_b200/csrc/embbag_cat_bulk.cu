@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(CW * 32) embbag_cat_bulk_kernel(const T* __res
 
     uint32_t parity = 0;
     bool timed_out = false;
+    const int first_tries = g_rows_wait_tries;
     constexpr int E16 = 16 / (int)sizeof(T);       // elements per 16-byte chunk
     const int nch = d / E16;                       // chunks per bag slot
     for (int r = 0; r < CSPW; ++r) {
@@ -139,7 +140,10 @@ __global__ void __launch_bounds__(CW * 32) embbag_cat_bulk_kernel(const T* __res
                 reinterpret_cast<uint4*>(slot)[ch] = *reinterpret_cast<const uint4*>(t);
             }
         }
-        if (!bar_wait(bar, parity)) timed_out = true;
+        if (!rows_ready(bar, parity, first_tries)) {   // rows landed (drained): stop this warp's samples
+            timed_out = true;
+            break;
+        }
         parity ^= 1u;
         // ordinary stores into the buffer become visible to the bulk store
         fence_proxy_async();
@@ -186,6 +190,10 @@ dlrm_status launch_embbag_cat_bulk(const TableMeta& tm, const void* tables, dlrm
 #undef DLRM_CAT_BULK
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
+}
+
+cudaError_t set_wait_polls_embbag_cat(long long polls) {
+    return ac::set_rows_wait_tries_here(polls < 0 ? -1 : (int)(polls < ac::WAIT_TRIES ? polls : ac::WAIT_TRIES));
 }
 
 }  // namespace dlrm

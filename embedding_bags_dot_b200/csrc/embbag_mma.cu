@@ -118,7 +118,7 @@ struct BagMasks {
 // Writes the whole concat row.
 template <int MT, int GL>
 __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, int K, const BagMasks& bm,
-                                          uint32_t bar, uint32_t parity, bool& timed_out, const float4* xv,
+                                          uint32_t bar, uint32_t parity, int tries, bool& timed_out, const float4* xv,
                                           float mn, float range, const uint32_t (&srcr)[SRC_CACHE][4],
                                           const uint16_t* src_s, int nzc, const float* __restrict__ xrow,
                                           void* out, size_t row0, int ld, int out_dt, int lane) {
@@ -167,7 +167,10 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, int 
             *reinterpret_cast<uint32_t*>(xw + (P0 + 2) * QRB + c) = __byte_perm(hi01, hi23, 0x5410);
         }
     }
-    if (!bar_wait(bar, parity)) timed_out = true;
+    if (!rows_ready(bar, parity, tries)) {   // rows landed (drained); the caller stops after this sample
+        timed_out = true;
+        return;
+    }
     __syncwarp();
 
     // exact integer Gram of the lower-triangle tiles
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const int gi = lane / GL, g = lane % GL;
     uint32_t parity = 0;
     bool timed_out = false;
+    const int first_tries = g_rows_wait_tries;
 
     for (int r = 0; r < SPW; ++r) {
         const int s = warp * SPW + r;
@@ -424,10 +428,11 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
         }
         if constexpr (Q) {
             if (int_route) {
-                u8_sample<MT, GL>(xw, xw_s, K, bm, bar, parity, timed_out, xv, mn, range, srcr, src_s, nzc,
-                                  x_dense + b * d, out, (size_t)b * ld, ld, out_dt, lane);
+                u8_sample<MT, GL>(xw, xw_s, K, bm, bar, parity, first_tries, timed_out, xv, mn, range, srcr, src_s,
+                                  nzc, x_dense + b * d, out, (size_t)b * ld, ld, out_dt, lane);
                 parity ^= 1u;
                 __syncwarp();  // the region is reused by the next sample
+                if (timed_out) break;
                 continue;
             }
         }
@@ -478,7 +483,10 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                     make_uint2(pack_bf16(x.x - f01.x, x.y - f01.y), pack_bf16(x.z - f23.x, x.w - f23.y));
             }
         }
-        if (!bar_wait(bar, parity)) timed_out = true;
+        if (!rows_ready(bar, parity, first_tries)) {   // rows landed (drained): stop this warp's samples
+            timed_out = true;
+            break;
+        }
         parity ^= 1u;
         __syncwarp();
         if constexpr (Q) {
@@ -661,6 +669,10 @@ dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, 
 #undef DLRM_MMA_GL
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
+}
+
+cudaError_t set_wait_polls_embbag_mma(long long polls) {
+    return ac::set_rows_wait_tries_here(polls < 0 ? -1 : (int)(polls < ac::WAIT_TRIES ? polls : ac::WAIT_TRIES));
 }
 
 }  // namespace dlrm

@@ -26,6 +26,10 @@
 namespace dlrm {
 namespace tc {
 
+// Polls of the ordinary waits of linear_tc_kernel on this device (WAIT_LIMIT unless a test lowered it
+// with dlrm_set_wait_polls to make them run out). The drains after a timeout always use WAIT_LIMIT.
+static __device__ long long g_tc1_wait_polls = WAIT_LIMIT;
+
 template <typename TC, int ACT>
 __global__ void __launch_bounds__(THREADS, 1)
     linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
@@ -65,6 +69,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tmem = bars->tmem_base;
     volatile int* abort = &bars->abort;
     bool timed_out = false;
+    const long long lim = g_tc1_wait_polls;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -75,7 +80,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x) {
                 const int mb = t / nbn, nb = t - mb * nbn;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&bars->empty[s], ph ^ 1u, abort)) {
+                    if (!mbar_wait_n(&bars->empty[s], ph ^ 1u, abort, lim)) {
                         timed_out = true;
                         break;
                     }
@@ -89,16 +94,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             }
-            if (timed_out) {
-                *abort = 1;
-                // drain: every stage whose load may still be in flight completes its full phase
-                for (int q = 0; q < STAGES; ++q) {
-                    if (--s < 0) {
-                        s = STAGES - 1;
-                        ph ^= 1u;
-                    }
-                    mbar_wait(&bars->full[s], ph, abort, true);
+            if (timed_out) *abort = 1;
+            // drain, also when another role gave up: every stage whose load may still be in flight
+            // completes its full phase before the CTA may exit (a stage never loaded, or already
+            // consumed, passes at once)
+            for (int q = 0; q < STAGES; ++q) {
+                if (--s < 0) {
+                    s = STAGES - 1;
+                    ph ^= 1u;
                 }
+                mbar_wait(&bars->full[s], ph, abort, true);
             }
         }
     } else if (warp == 1) {
@@ -110,14 +115,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
                 const int acc = i & 1;
                 const uint32_t use = (uint32_t)(i >> 1);
-                if (!mbar_wait(&bars->tempty[acc], (use & 1u) ^ 1u, abort)) {
+                if (!mbar_wait_n(&bars->tempty[acc], (use & 1u) ^ 1u, abort, lim)) {
                     timed_out = true;
                     break;
                 }
                 fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&bars->full[s], ph, abort)) {
+                    if (!mbar_wait_n(&bars->full[s], ph, abort, lim)) {
                         timed_out = true;
                         break;
                     }
@@ -150,7 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
             const int acc = i & 1;
             const uint32_t use = (uint32_t)(i >> 1);
-            if (!mbar_wait(&bars->tfull[acc], use & 1u, abort)) {
+            if (!mbar_wait_n(&bars->tfull[acc], use & 1u, abort, lim)) {
                 timed_out = true;
                 break;
             }
@@ -475,6 +480,11 @@ static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, const
 }
 
 }  // namespace tc
+
+cudaError_t set_wait_polls_gemm_tc(long long polls) {
+    const long long v = polls < 0 ? tc::WAIT_LIMIT : polls;
+    return cudaMemcpyToSymbol(tc::g_tc1_wait_polls, &v, sizeof(v));
+}
 
 bool linear_tc_logit_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
                                dlrm_dtype w_dt, int ldw, const float* bias) {

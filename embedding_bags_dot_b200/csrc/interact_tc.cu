@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(FW * 32, 2) interact_fwd_tc_kernel(
     unsigned oob = 0, bad = 0;
     bool timed_out = false;
     uint32_t parity = 0;
+    const int first_tries = g_rows_wait_tries;
     const long long nw = (long long)gridDim.x * FW;
     for (long long b = (long long)blockIdx.x * FW + warp; b < B; b += nw) {
         float4 h[NX], l[NX];
@@ -200,7 +201,10 @@ __global__ void __launch_bounds__(FW * 32, 2) interact_fwd_tc_kernel(
                 *reinterpret_cast<float4*>(X + c) =
                     make_float4(h[q].x + l[q].x, h[q].y + l[q].y, h[q].z + l[q].z, h[q].w + l[q].w);
         }
-        if (!bar_wait(bar, parity)) timed_out = true;
+        if (!rows_ready(bar, parity, first_tries)) {   // rows landed (drained): stop this warp's samples
+            timed_out = true;
+            break;
+        }
         parity ^= 1u;
         __syncwarp();
 
@@ -307,6 +311,7 @@ __global__ void __launch_bounds__(BW * 32, 3) interact_bwd_fma_kernel(
     unsigned oob = 0, bad = 0;
     bool timed_out = false;
     uint32_t parity = 0;
+    const int first_tries = g_rows_wait_tries;
     const long long nw = (long long)gridDim.x * BW;
     long long b = (long long)blockIdx.x * BW + warp;
     if (b < B) gather_rows<D, D>(R, R_s, tables, tm, K, B, b, offsets, indices, nnz, bar, false, oob, bad, lane);
@@ -328,7 +333,10 @@ __global__ void __launch_bounds__(BW * 32, 3) interact_bwd_fma_kernel(
 #pragma unroll
             for (int e = 0; e < V; ++e) x[0][e] = h[e] + l[e];
         }
-        if (!bar_wait(bar, parity)) timed_out = true;
+        if (!rows_ready(bar, parity, first_tries)) {   // rows landed (drained): stop this warp's samples
+            timed_out = true;
+            break;
+        }
         parity ^= 1u;
         __syncwarp();
 #pragma unroll
@@ -486,6 +494,10 @@ dlrm_status launch_interact_bwd_tc(const TableMeta& tm, const float* tables, int
 #undef DLRM_BWD
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
+}
+
+cudaError_t set_wait_polls_interact_tc(long long polls) {
+    return ac::set_rows_wait_tries_here(polls < 0 ? -1 : (int)(polls < ac::WAIT_TRIES ? polls : ac::WAIT_TRIES));
 }
 
 }  // namespace dlrm

@@ -169,5 +169,14 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
                                 cudaStream_t st);
 dlrm_status launch_sgd(long long n, float lr, float* w, const float* g, cudaStream_t st);
 size_t train_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B);
+// Test hook behind dlrm_set_wait_polls: the first-wait bound of each file's kernels on the current device.
+cudaError_t set_wait_polls_gemm_tc(long long polls);
+cudaError_t set_wait_polls_embbag_mma(long long polls);
+cudaError_t set_wait_polls_embbag_cat(long long polls);
+cudaError_t set_wait_polls_interact_tc(long long polls);
+// Every host-side check of dlrm_forward (cat = false) or dlrm_forward_cat (cat = true), ws_bytes included.
+dlrm_status forward_check(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                          const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* y_hat,
+                          const void* ws, size_t ws_bytes, bool cat);
 
 }  // namespace dlrm

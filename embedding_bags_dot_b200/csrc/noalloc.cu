@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "kernels.cuh"
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DLRM_NOALLOC_SCRATCH_BYTES];
 
@@ -48,15 +49,17 @@ cudaError_t scratch_address(void** out) {
 extern "C" dlrm_status dlrm_forward_noalloc(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
                                             const float* dense, const int32_t* offsets, const int32_t* indices,
                                             int64_t nnz, float* y_hat, uint32_t* err_flags, dlrm_stream stream) {
-    const size_t need = dlrm_workspace_size(T, bot, top, B, 0);
-    if (need == 0) return DLRM_ERR_INVALID_ARG;
-    if (need > (size_t)DLRM_NOALLOC_SCRATCH_BYTES) return DLRM_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return DLRM_ERR_CUDA;
+    // Every check dlrm_forward makes, with the array as its workspace, before anything is queued: a
+    // refused call returns the same status as dlrm_forward and leaves err_flags and the array alone.
+    dlrm_status r = dlrm::forward_check(T, bot, top, B, dense, offsets, indices, nnz, y_hat, scratch,
+                                        DLRM_NOALLOC_SCRATCH_BYTES, false);
+    if (r != DLRM_OK) return r;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // The array keeps the previous call's contents: the error record must start at zero.
     if (cudaMemsetAsync(scratch, 0, DLRM_ERR_RECORD_BYTES, st) != cudaSuccess) return DLRM_ERR_CUDA;
-    const dlrm_status r = dlrm_forward(T, bot, top, B, dense, offsets, indices, nnz, y_hat, scratch, stream);
+    r = dlrm_forward(T, bot, top, B, dense, offsets, indices, nnz, y_hat, scratch, DLRM_NOALLOC_SCRATCH_BYTES, stream);
     if (r != DLRM_OK) return r;
     if (err_flags && cudaMemcpyAsync(err_flags, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return DLRM_ERR_CUDA;

@@ -51,15 +51,20 @@ __device__ __forceinline__ bool mbar_try(unsigned long long* b, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete. Gives up
-// early when another role has already aborted (unless ignore_abort).
-__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, volatile int* abort,
-                                          bool ignore_abort = false) {
-    for (long long i = 0; i < WAIT_LIMIT; ++i) {
+// Bounded wait (at most `limit` polls) for the phase with the given parity to
+// complete. Gives up early when another role has already aborted (unless
+// ignore_abort).
+__device__ __forceinline__ bool mbar_wait_n(unsigned long long* b, uint32_t parity, volatile int* abort,
+                                            long long limit, bool ignore_abort = false) {
+    for (long long i = 0; i < limit; ++i) {
         if (mbar_try(b, parity)) return true;
         if (!ignore_abort && (i & 255) == 255 && *abort) return false;
     }
     return false;
+}
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, volatile int* abort,
+                                          bool ignore_abort = false) {
+    return mbar_wait_n(b, parity, abort, WAIT_LIMIT, ignore_abort);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, unsigned long long* bar, int x,

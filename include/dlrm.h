@@ -20,6 +20,11 @@
  *    index contributes nothing, the offending bag pools to zero, and the
  *    event is recorded in the error record at the start of the workspace;
  *    dlrm_check_error() reads and clears it.
+ *  - Every caller-provided scratch buffer (workspace `ws`, gradient buffer
+ *    `grads`) comes with its size in bytes (`ws_bytes`, `grads_bytes`). A
+ *    buffer smaller than the call needs (the matching *_size query) or not
+ *    16-byte aligned is refused with DLRM_ERR_WORKSPACE before anything is
+ *    launched; the library never writes past the size it is given.
  *  - Bags are CSR, table-major: bag (k, b) of table k and sample b holds
  *    indices[offsets[k*B + b] .. offsets[k*B + b + 1]), each a row id local to
  *    table k. offsets has K*B + 1 int32 entries; nnz < 2^31.
@@ -110,6 +115,19 @@ dlrm_status dlrm_quantize_rows_u8(const void* src, dlrm_dtype src_dt, int64_t ro
  * (all devices, all streams). Used to count launches inside a timed region. */
 uint64_t dlrm_launch_count(void);
 
+/* Test hook, no counterpart in the pages: sets, on the current device, how
+ * many times the first bounded wait of the row-gathering kernels (the bulk
+ * copies of a sample's rows) and the ordinary waits of the single-CTA
+ * tensor-core layer (batches below 4,096 rows) poll before giving up;
+ * polls < 0 restores the defaults (about a second). A test sets 0 to make
+ * those waits run out at once and checks that the call returns, that
+ * dlrm_check_error reports DLRM_ERR_TIMEOUT, and that the next call (after
+ * restoring) is correct. After giving up, a kernel still waits with the full
+ * bound for the copies it has in flight, frees its tensor memory and returns;
+ * outputs of the samples or tiles it did not finish are undefined. Not for
+ * production use; synchronise the device before and after calling it. */
+dlrm_status dlrm_set_wait_polls(int64_t polls);
+
 /* Human-readable name of a status code (static string). */
 const char* dlrm_status_str(dlrm_status s);
 
@@ -124,7 +142,7 @@ size_t dlrm_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm
  * DLRM_ERR_INDEX_OOB if any index was out of range, else DLRM_ERR_TIMEOUT if
  * a bounded wait gave up, else DLRM_OK. If `info` (host, 3 entries) is not
  * NULL it receives {flags, skipped indices, bad bags}. */
-dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info);
+dlrm_status dlrm_check_error(void* ws, size_t ws_bytes, dlrm_stream stream, int64_t* info);
 
 /* Sum-pooled embedding bags ([S] section 3: each sparse feature looks up a
  * row of its own table; a bag of several ids sums their rows, an empty bag
@@ -132,9 +150,10 @@ dlrm_status dlrm_check_error(void* ws, dlrm_stream stream, int64_t* info);
  *   pooled   out, fp32 [B][K][d]
  *   bag_len  out, optional (may be NULL): int32 [K*B], end - start of each bag
  *            (0 for a bag with bad offsets)
- *   ws       workspace holding the error record (>= DLRM_ERR_RECORD_BYTES) */
+ *   ws       workspace holding the error record (ws_bytes >= DLRM_ERR_RECORD_BYTES) */
 dlrm_status dlrm_embbag_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
-                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, dlrm_stream stream);
+                            int64_t nnz, float* pooled, int32_t* bag_len, void* ws, size_t ws_bytes,
+                            dlrm_stream stream);
 
 /* Pairwise dot-product interaction and concat ([S] section 4, equations
  * "Interaction" and "Output"; [N] Core Idea: self-interactions excluded).
@@ -150,19 +169,18 @@ dlrm_status dlrm_interact_fwd(int B, int K, int d, const float* x_dense, const f
  * chip and only the concat rows are written. Same arguments and errors. */
 dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
                                      int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt,
-                                     void* ws, dlrm_stream stream);
+                                     void* ws, size_t ws_bytes, dlrm_stream stream);
 
 /* MLP forward ([N] Key Method Details: FC layers with ReLU). ReLU after every
  * hidden layer; after the last layer `final_act` (none, ReLU or sigmoid).
  *   in    [B][ld_in] of in_dt, dims[0] logical columns
  *   out   out, fp32 [B][ld_out], dims[n_layers] logical columns
- *   ws    16-byte aligned, at least dlrm_mlp_workspace_size(mlp, B, in_dt)
- *         bytes (dlrm_workspace_size of a model with this MLP as top or
- *         bottom is enough); the hidden activations live there. The size is
- *         not passed, so it cannot be checked here: a smaller buffer is
- *         written past its end. */
+ *   ws    16-byte aligned, ws_bytes >= dlrm_mlp_workspace_size(mlp, B, in_dt)
+ *         (dlrm_workspace_size of a model with this MLP as top or bottom is
+ *         enough); the hidden activations live there. A smaller ws_bytes is
+ *         refused with DLRM_ERR_WORKSPACE before any launch. */
 dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in,
-                         float* out, int ld_out, int final_act, void* ws, dlrm_stream stream);
+                         float* out, int ld_out, int final_act, void* ws, size_t ws_bytes, dlrm_stream stream);
 
 /* Bytes of workspace dlrm_mlp_fwd needs for this MLP, batch and input dtype:
  * the error record, one or two buffers of the widest hidden-layer output and,
@@ -173,10 +191,11 @@ size_t dlrm_mlp_workspace_size(const dlrm_mlp* mlp, int B, dlrm_dtype in_dt);
 /* Whole forward pass ([S] sections 3-4):
  *   y_hat = sigmoid(top([x_dense, vec(Z)])),  x_dense = bottom(dense) with ReLU after every bottom layer,
  * hidden top layers with ReLU, last top layer linear (dims must end in 1).
- *   dense  fp32 [B][bot->dims[0]];  y_hat out, fp32 [B] */
+ *   dense  fp32 [B][bot->dims[0]];  y_hat out, fp32 [B]
+ *   ws     ws_bytes >= dlrm_workspace_size(T, bot, top, B, 0) */
 dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                          const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat,
-                         void* ws, dlrm_stream stream);
+                         void* ws, size_t ws_bytes, dlrm_stream stream);
 
 /* dlrm_forward with the bags given by their lengths instead of CSR offsets
  * (the pages fix no input format; this is a compact form of the same bags):
@@ -190,7 +209,7 @@ dlrm_status dlrm_forward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
  * Workspace: dlrm_workspace_size(T, bot, top, B, 0). */
 dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
                                  const float* dense, const uint8_t* lengths, const int32_t* indices, int64_t nnz,
-                                 float* y_hat, void* ws, dlrm_stream stream);
+                                 float* y_hat, void* ws, size_t ws_bytes, dlrm_stream stream);
 
 /* offsets[i] = sum_{j < i} lengths[j] for 0 <= i <= n (int32 out, device
  * pointers, the scan dlrm_forward_lengths runs). ws: 16-byte aligned,
@@ -198,7 +217,7 @@ dlrm_status dlrm_forward_lengths(const dlrm_tables* T, const dlrm_mlp* bot, cons
  * scan's chunk sums). The total must stay below 2^31. */
 size_t dlrm_offsets_from_lengths_workspace_size(int64_t n);
 dlrm_status dlrm_offsets_from_lengths(const uint8_t* lengths, int64_t n, int32_t* offsets, void* ws,
-                                      dlrm_stream stream);
+                                      size_t ws_bytes, dlrm_stream stream);
 
 /* ------------------------------------------------------------ training step
  * fp32 tables and MLPs only (DLRM_ERR_UNSUPPORTED otherwise); d % 4 == 0.
@@ -226,28 +245,31 @@ dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const 
  * y_hat (device, fp32 [B]) are optional outputs. Bit-reproducible.
  * Skipped (out-of-range) indices and bags with bad offsets are handled as in
  * dlrm_forward and counted once per call in the error record at the start of
- * `ws` (read with dlrm_check_error); occurrences beyond the gradient buffer's
- * capacity (nnz larger than the one it was sized for) are counted as bad. */
+ * `ws` (read with dlrm_check_error). grads_bytes must be at least
+ * dlrm_grads_size(T, bot, top, B, nnz) and ws_bytes at least
+ * dlrm_workspace_size(T, bot, top, B, 1). */
 dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                           const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
-                          float* loss, float* y_hat, void* grads, void* ws, dlrm_stream stream);
+                          float* loss, float* y_hat, void* grads, size_t grads_bytes, void* ws, size_t ws_bytes,
+                          dlrm_stream stream);
 
 /* SGD step from a gradient buffer filled by dlrm_backward on the same batch
  * shape: every table row the batch touched gets T[r] -= lr * g_r, where g_r
  * sums the gradients of the bags that use row r (once per occurrence) in
  * occurrence order; untouched rows are not written. Then W -= lr * dW and
  * b -= lr * db for every MLP layer. n_touched (device int32, optional)
- * receives the number of distinct rows updated. */
+ * receives the number of distinct rows updated. grads_bytes: as dlrm_backward. */
 dlrm_status dlrm_sparse_sgd(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
-                            float lr, void* grads, int32_t* n_touched, dlrm_stream stream);
+                            float lr, void* grads, size_t grads_bytes, int32_t* n_touched, dlrm_stream stream);
 
 /* The per-row embedding gradients dlrm_sparse_sgd would apply, without
  * applying them: rows (device uint32 [nnz]) gets the touched rows as global
  * row ids (base_k + r) in increasing order, row_grads (device fp32 [nnz][d])
- * their summed gradients, n_rows (device int32) their count. */
+ * their summed gradients, n_rows (device int32) their count. grads_bytes:
+ * as dlrm_backward. */
 dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
-                                     int64_t nnz, void* grads, uint32_t* rows, float* row_grads,
-                                     int32_t* n_rows, dlrm_stream stream);
+                                     int64_t nnz, const void* grads, size_t grads_bytes, uint32_t* rows,
+                                     float* row_grads, int32_t* n_rows, dlrm_stream stream);
 
 /* Concat-only interaction, the alternative the pages set DLRM against
  * ("Deep Learning Recommendation Model (DLRM)", Key Method Details: Wide &
@@ -259,13 +281,13 @@ dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, 
  * dlrm_embbag_interact_fwd (DLRM_U8ROW tables: DLRM_ERR_UNSUPPORTED). */
 dlrm_status dlrm_embbag_cat_fwd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices,
                                 int64_t nnz, const float* x_dense, void* concat, int ld, dlrm_dtype out_dt, void* ws,
-                                dlrm_stream stream);
+                                size_t ws_bytes, dlrm_stream stream);
 
 /* dlrm_forward with the concat-only interaction: top->dims[0] must be
  * d (K + 1). Workspace: dlrm_workspace_size(T, bot, top, B, 0). */
 dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
                              const int32_t* offsets, const int32_t* indices, int64_t nnz, float* y_hat, void* ws,
-                             dlrm_stream stream);
+                             size_t ws_bytes, dlrm_stream stream);
 
 /* fp32 GEMM of the training step, on the tensor cores at fp32 accuracy
  * (the matrix products of the fully connected layers, "Deep Learning
@@ -279,14 +301,14 @@ dlrm_status dlrm_forward_cat(const dlrm_tables* T, const dlrm_mlp* bot, const dl
  * and the product is summed as A_lo B_hi + A_hi B_lo + A_hi B_hi in fp32
  * (error about 2^-20 of sum_r |A(i,r) B(j,r)|). Long reductions are cut into
  * shape-determined r-ranges added in a fixed order: bit-reproducible.
- * ws: 16-byte aligned, dlrm_gemm_f32_workspace_size(...) bytes, caller-owned.
+ * ws: 16-byte aligned, ws_bytes >= dlrm_gemm_f32_workspace_size(...), caller-owned.
  * Returns DLRM_ERR_INVALID_ARG (sizes < 1, null, misaligned, ld),
- * DLRM_ERR_WORKSPACE (ws null or misaligned), DLRM_ERR_UNSUPPORTED (no
+ * DLRM_ERR_WORKSPACE (ws null, misaligned or short), DLRM_ERR_UNSUPPORTED (no
  * tensor-map support in the driver); device timeouts land in the error
  * record read by dlrm_check_error. */
 size_t dlrm_gemm_f32_workspace_size(int I, int J, int R, int a_mn, int b_mn);
 dlrm_status dlrm_gemm_f32(int I, int J, int R, const float* A, int lda, int a_mn, const float* B, int ldb, int b_mn,
-                          float* C, int ldc, void* ws, dlrm_stream stream);
+                          float* C, int ldc, void* ws, size_t ws_bytes, dlrm_stream stream);
 
 /* The two halves of dlrm_gemm_f32, for callers that keep operands in pair
  * form (as the training step does for every activation and gradient).
@@ -303,7 +325,7 @@ dlrm_status dlrm_tf32_split(int rows, int cols, const float* src, int lds, float
 size_t dlrm_gemm_tf32x3_workspace_size(int I, int J, int R);
 dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float* A_lo, int lda, int a_mn,
                              const float* B_hi, const float* B_lo, int ldb, int b_mn, float* C, int ldc, void* ws,
-                             dlrm_stream stream);
+                             size_t ws_bytes, dlrm_stream stream);
 
 /* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
 #define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -333,11 +355,15 @@ dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float
  *    previous call's contents. Calls whose work overlaps on the GPU (other
  *    streams, other host threads) race on it; order them on one stream or
  *    serialise them.
- *  - Errors: device-detected input errors are handled as in dlrm_forward
- *    (skipped index, empty bag). The error record is cleared at the start
- *    of each call; if err_flags (device, optional) is not NULL it receives
- *    this call's flags once the call's work completes: bit 0 = an index was
- *    out of range, bit 1 = a bag had bad offsets. */
+ *  - Errors: every argument check of dlrm_forward runs first, and a refused
+ *    call returns the status dlrm_forward would return, having queued
+ *    nothing and written neither the array nor err_flags. Device-detected
+ *    input errors are handled as in dlrm_forward (skipped index, empty bag).
+ *    The error record is cleared at the start of each accepted call; if
+ *    err_flags (device, optional) is not NULL it receives this call's flags
+ *    once the call's work completes: bit 0 = an index was out of range,
+ *    bit 1 = a bag had bad offsets. On any status other than DLRM_OK,
+ *    err_flags is left as it was. */
 dlrm_status dlrm_forward_noalloc(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B,
                                  const float* dense, const int32_t* offsets, const int32_t* indices, int64_t nnz,
                                  float* y_hat, uint32_t* err_flags, dlrm_stream stream);

@@ -60,11 +60,12 @@ def test_host_side_helpers(lib):
 def test_argument_checks_without_gpu(lib):
     import embedding_bags_dot_b200 as E
     # null tables / null everything: rejected before any CUDA call
-    assert lib.dlrm_embbag_fwd(None, 4, None, None, 0, None, None, None, None) == E.ERR_INVALID_ARG
-    assert lib.dlrm_forward(None, None, None, 4, None, None, None, 0, None, None, None) == E.ERR_INVALID_ARG
+    assert lib.dlrm_embbag_fwd(None, 4, None, None, 0, None, None, None, 0, None) == E.ERR_INVALID_ARG
+    assert lib.dlrm_forward(None, None, None, 4, None, None, None, 0, None, None, 0, None) == E.ERR_INVALID_ARG
     assert lib.dlrm_interact_fwd(4, 0, 8, None, None, None, 64, 0, None) == E.ERR_INVALID_ARG
     assert lib.dlrm_interact_fwd(4, 300, 8, None, None, None, 10 ** 6, 0, None) == E.ERR_UNSUPPORTED
-    assert lib.dlrm_check_error(None, None, None) == E.ERR_INVALID_ARG
+    assert lib.dlrm_check_error(None, 0, None, None) == E.ERR_INVALID_ARG
+    assert lib.dlrm_check_error(256, 255, None, None) == E.ERR_WORKSPACE
     # workspace size from host structs only (fake, never dereferenced, device pointers)
     rows = (C.c_int64 * 3)(10, 20, 30)
     T = E._abi.dlrm_tables(256, rows, 3, 16, E.F32)
@@ -114,7 +115,61 @@ def test_mlp_workspace_size_follows_the_documented_layout(lib):
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), -1, "f32") == 0
 
 
-def test_bindings_refuse_a_short_workspace_before_launching(lib):
+def _fake_model(E, K=3, d=16, B=100, dt=None):
+    """Host structs of a small fp32 model whose device pointers are fake (16-byte aligned, never
+    dereferenced: every call below returns from its host-side checks)."""
+    dt = E.F32 if dt is None else dt
+    keep = {}
+    keep["rows"] = (C.c_int64 * K)(*[10 * (k + 1) for k in range(K)])
+    keep["T"] = E._abi.dlrm_tables(1 << 20, keep["rows"], K, d, dt)
+    keep["db"] = (C.c_int * 3)(13, 32, d)
+    keep["dt"] = (C.c_int * 3)(d + K * (K + 1) // 2, 8, 1)
+    keep["W"] = (C.c_void_p * 2)(2 << 20, 3 << 20)
+    keep["b"] = (C.c_void_p * 2)(4 << 20, 5 << 20)
+    keep["bot"] = E._abi.dlrm_mlp(2, keep["db"], keep["W"], keep["b"], dt)
+    keep["top"] = E._abi.dlrm_mlp(2, keep["dt"], keep["W"], keep["b"], dt)
+    return keep
+
+
+def test_c_abi_refuses_a_short_buffer_before_launching(lib):
+    """Through the C ABI itself (no binding in between): every entry point that takes caller scratch
+    memory refuses a buffer one byte shorter than its size query, with DLRM_ERR_WORKSPACE and no launch,
+    and accepts the exact size as far as the host-side checks go."""
+    import embedding_bags_dot_b200 as E
+    m = _fake_model(E)
+    T, bot, top = C.byref(m["T"]), C.byref(m["bot"]), C.byref(m["top"])
+    B, nnz, fake = 100, 300, 6 << 20
+    before = E.dlrm_launch_count()
+    need = lib.dlrm_workspace_size(T, bot, top, B, 0)
+    assert lib.dlrm_forward(T, bot, top, B, fake, fake, fake, nnz, fake, fake, need - 1, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_forward_cat(T, bot, top, B, fake, fake, fake, nnz, fake, fake, need - 1, None) == E.ERR_INVALID_ARG
+    assert lib.dlrm_forward_lengths(T, bot, top, B, fake, fake, fake, nnz, fake, fake, need - 1, None) == E.ERR_WORKSPACE
+    need_m = lib.dlrm_mlp_workspace_size(bot, B, E.F32)
+    assert lib.dlrm_mlp_fwd(bot, B, fake, E.F32, 13, fake, 16, E.ACT_RELU, fake, need_m - 1, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_embbag_fwd(T, B, fake, fake, nnz, fake, None, fake, E.ERR_RECORD_BYTES - 1, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_embbag_interact_fwd(T, B, fake, fake, nnz, fake, fake, 24, E.F32, fake, E.ERR_RECORD_BYTES - 1,
+                                        None) == E.ERR_WORKSPACE
+    need_t = lib.dlrm_workspace_size(T, bot, top, B, 1)
+    need_g = lib.dlrm_grads_size(T, bot, top, B, nnz)
+    assert need_t > 0 and need_g > 0
+    args = (T, bot, top, B, fake, fake, fake, nnz, fake, None, None)
+    assert lib.dlrm_backward(*args, fake, need_g, fake, need_t - 1, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_backward(*args, fake, need_g - 1, fake, need_t, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_sparse_sgd(T, bot, top, B, nnz, 0.01, fake, need_g - 1, None, None) == E.ERR_WORKSPACE
+    assert lib.dlrm_embedding_row_grads(T, bot, top, B, nnz, fake, need_g - 1, fake, fake, fake, None) == E.ERR_WORKSPACE
+    for a_mn, b_mn in ((0, 0), (1, 1)):
+        need_f = lib.dlrm_gemm_f32_workspace_size(64, 48, 40, a_mn, b_mn)
+        assert lib.dlrm_gemm_f32(64, 48, 40, fake, 64, a_mn, fake, 48, b_mn, fake, 48, fake, need_f - 1, None) == \
+            E.ERR_WORKSPACE
+    need_x = lib.dlrm_gemm_tf32x3_workspace_size(64, 48, 40)
+    assert lib.dlrm_gemm_tf32x3(64, 48, 40, fake, fake, 40, 0, fake, fake, 40, 0, fake, 48, fake, need_x - 1, None) == \
+        E.ERR_WORKSPACE
+    assert lib.dlrm_offsets_from_lengths(fake, 1000, fake, fake,
+                                         lib.dlrm_offsets_from_lengths_workspace_size(1000) - 1, None) == E.ERR_WORKSPACE
+    assert E.dlrm_launch_count() == before
+
+
+def test_bindings_pass_the_buffer_size_through(lib):
     import embedding_bags_dot_b200 as E
     mlp = _cpu_mlp([13, 512, 256, 128], "bf16")
     B = 1000
@@ -122,7 +177,7 @@ def test_bindings_refuse_a_short_workspace_before_launching(lib):
     x, out = torch.zeros((B, 13)), torch.zeros((B, 128))
     before = E.dlrm_launch_count()
     with pytest.raises(E.DlrmError) as e:
-        E.dlrm_mlp_fwd(mlp, B, x, 13, out, 128, E.ACT_RELU, torch.zeros(need - 16, dtype=torch.uint8))
+        E.dlrm_mlp_fwd(mlp, B, x, 13, out, 128, E.ACT_RELU, torch.zeros(need - 16, dtype=torch.uint8), stream=0)
     assert e.value.status == E.ERR_WORKSPACE
     assert E.dlrm_launch_count() == before
 
@@ -141,15 +196,15 @@ def test_lengths_workspace_and_argument_checks(lib):
                        (torch.zeros(10, dtype=torch.uint8), torch.zeros(11, dtype=torch.int64)),
                        (torch.zeros(10, dtype=torch.uint8), torch.zeros(10, dtype=torch.int32))):
         with pytest.raises(E.DlrmError) as e:
-            E.dlrm_offsets_from_lengths(lens, offs, ws)
+            E.dlrm_offsets_from_lengths(lens, offs, ws, stream=0)
         assert e.value.status == E.ERR_INVALID_ARG
     with pytest.raises(E.DlrmError) as e:
         E.dlrm_offsets_from_lengths(torch.zeros(100_000, dtype=torch.uint8), torch.zeros(100_001, dtype=torch.int32),
-                                    torch.zeros(64, dtype=torch.uint8))
+                                    torch.zeros(64, dtype=torch.uint8), stream=0)
     assert e.value.status == E.ERR_WORKSPACE
     mlp = _cpu_mlp([13, 64], "f32")
     with pytest.raises(E.DlrmError) as e:
         E.dlrm_forward_lengths(None, mlp, mlp, 4, torch.zeros((4, 13)), torch.zeros(8, dtype=torch.int32),
-                               torch.zeros(8, dtype=torch.int32), torch.zeros(4), ws)
+                               torch.zeros(8, dtype=torch.int32), torch.zeros(4), ws, stream=0)
     assert e.value.status == E.ERR_INVALID_ARG
     assert E.dlrm_launch_count() == before

@@ -96,12 +96,14 @@ def test_host_argument_errors(tiny):
     nnz = batch.indices.size
     P = lambda t: t.data_ptr()  # noqa: E731
     # null tables
-    assert L.dlrm_embbag_fwd(None, cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, P(g.ws), s) == E.ERR_INVALID_ARG
+    nws = g.ws.numel()
+    assert L.dlrm_embbag_fwd(None, cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, P(g.ws), nws, s) == E.ERR_INVALID_ARG
     # nnz out of range
-    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), 2 ** 31, P(pooled), None, P(g.ws), s) == E.ERR_INVALID_ARG
-    # missing workspace, misaligned output
-    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, None, s) == E.ERR_WORKSPACE
-    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled) + 4, None, P(g.ws), s) == E.ERR_INVALID_ARG
+    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), 2 ** 31, P(pooled), None, P(g.ws), nws, s) == E.ERR_INVALID_ARG
+    # missing or short workspace, misaligned output
+    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, None, 0, s) == E.ERR_WORKSPACE
+    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, P(g.ws), 255, s) == E.ERR_WORKSPACE
+    assert L.dlrm_embbag_fwd(g.T.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled) + 4, None, P(g.ws), nws, s) == E.ERR_INVALID_ARG
     # concat leading dimension too small
     x = torch.zeros((cfg.B, cfg.d), device="cuda")
     out = torch.zeros((cfg.B, 64), device="cuda")
