@@ -77,6 +77,17 @@ def algorithmic_bytes(cfg, batch) -> int:
     return rows + 4 * batch.indices.size + 4 * (cfg.K * cfg.B + 1) + 4 * cfg.B * cfg.d + es_o * cfg.B * cfg.concat_width
 
 
+def fused_kernel_name(cfg) -> str:
+    """The gather + interaction kernel the library dispatches to for this workload."""
+    if cfg.interaction == "cat":
+        return "embbag_cat_bulk_kernel (dlrm_embbag_cat_fwd)"
+    if cfg.table_dtype in ("bf16", "u8row") and cfg.K + (4 if cfg.table_dtype == "u8row" else 2) <= 64:
+        return "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
+    if cfg.table_dtype == "bf16" and cfg.mlp_dtype == "bf16" and cfg.d in (64, 128) and cfg.K <= 128:
+        return "embbag_interact_wide_kernel (dlrm_embbag_interact_fwd)"
+    return "embbag_interact_kernel (dlrm_embbag_interact_fwd)"
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -183,6 +194,32 @@ def oracle_rate(cfg, batch, n_samples: int, seed: int = 0):
     return Bs / dt, dt, O.threads(), Bs
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_on_one_core(cfg, batch, target_s: float):
+    """The same oracle measurement with its OpenMP pool cut to one thread."""
+    from oracle import oracle as O
+    lib = O.load()
+    n_all = O.threads()
+    lib.oracle_set_threads(1)
+    try:
+        rate, dt, cores, used = calibrated_oracle(cfg, batch, target_s)
+    finally:
+        lib.oracle_set_threads(n_all)
+    return rate, dt, cores, used
+
+
 def calibrated_oracle(cfg, batch, target_s: float):
     n = 64
     rate, dt, cores, used = oracle_rate(cfg, batch, n)
@@ -213,7 +250,8 @@ def run_reference(args, cfg, rank):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
-                            "sample": f"{n} random samples of batch 0 per step (fp64 forward, host cores)"},
+                            "sample": f"{n} random samples of batch 0 per step (fp64 forward, host cores)",
+                            "cpu_model": cpu_model()},
            "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
@@ -409,10 +447,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                              f"and a {POOL}-batch pool of {pool_bytes / 1e6:.0f} MB exceed the {L2_BYTES >> 20} MB L2"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak_hbm, "unit": "GB/s",
                          "frac": achieved / peak_hbm, "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": ("embbag_cat_bulk_kernel (dlrm_embbag_cat_fwd)" if cfg.interaction == "cat" else
-                                    "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
-                                    if cfg.table_dtype in ("bf16", "u8row")
-                                    else "embbag_interact_kernel (dlrm_embbag_interact_fwd)"),
+                         "kernel": fused_kernel_name(cfg),
                          "algorithmic_bytes_per_launch": avg_algo, "avg_launch_ms": k2_avg},
             "kernels_ms_per_step": {"bottom_mlp": float(np.mean(bot_ms)), "embbag_interact": float(np.mean(k2_ms)),
                                     "top_mlp": float(np.mean(top_ms))},

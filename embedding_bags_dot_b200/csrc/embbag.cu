@@ -532,6 +532,8 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
     if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt, tm.base[K - 1] + tm.rows[K - 1]))
         return launch_embbag_interact_mma(tm, tables, dt, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt,
                                           err, st);
+    if (embbag_interact_wide_supported(dt, K, d, ld, out, out_dt))
+        return launch_embbag_interact_wide(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st);
     Geometry g;
     if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     switch (dt) {

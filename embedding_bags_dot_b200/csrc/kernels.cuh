@@ -35,6 +35,11 @@ dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, 
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st);
+// Many tables (K up to 128, bf16 tables and concat, d = 64 or 128): U-deep row gather and mma.sync Gram.
+bool embbag_interact_wide_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt);
+dlrm_status launch_embbag_interact_wide(const TableMeta& tm, const void* tables, int K, int d, int B,
+                                        const int32_t* offsets, const int32_t* indices, long long nnz,
+                                        const float* x_dense, void* out, int ld, ErrRecord* err, cudaStream_t st);
 
 // One fully connected layer: C[M][N] = act(A[M][K] W[N][K]^T + bias), fp32 accumulation.
 // A has dtype a_dt (ld lda), W has dtype w_dt (ld ldw), C has dtype c_dt (ld ldc).

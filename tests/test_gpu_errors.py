@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import embedding_bags_dot_b200 as E
-from gpucase import GpuModel, assert_close, scale_pooled, to_np
+from gpucase import GpuModel, assert_close, scale_concat, scale_pooled, to_np
 from oracle import oracle as O
 from synth import CONFIGS, gen, shrink
 from synth import device as sd
@@ -16,11 +16,15 @@ from synth import device as sd
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["f32", "bf16"])
+@pytest.fixture(scope="module", params=["f32", "bf16", "bf16-many"])
 def tiny(request):
-    # bf16 with d = 16 x 8 = 128 takes the tensor-core fused path; f32 the CUDA-core one
+    # bf16 with d = 16 x 8 = 128 takes the tensor-core fused path; f32 the CUDA-core one; 70 bf16 tables of
+    # d = 64 the many-table fused path
     if request.param == "f32":
         cfg = shrink(CONFIGS["tiny"], B=70).with_(bag="mix", seed=4)
+    elif request.param == "bf16-many":
+        cfg = shrink(CONFIGS["stress"], B=70, rows_cap=1000).with_(rows=(1000,) * 70, bag="mix", seed=4,
+                                                                   top=(64 + 2485, 64, 1))
     else:
         cfg = shrink(CONFIGS["large"], B=70, rows_cap=1000).with_(rows=(1000,) * 8, bag="mix", seed=4,
                                                                   top=(128 + 36, 64, 1))
@@ -87,6 +91,31 @@ def test_forward_records_errors_and_completes(tiny):
     assert_close(to_np(y), want, cfg.table_dtype, "forward with skipped indices")
 
 
+def test_fused_interaction_with_bad_bags(tiny):
+    """The fused gather + interaction skips out-of-range indices and pools bags with bad offsets to zero,
+    as the oracle does, and counts both."""
+    cfg, batch, g = tiny
+    offs = batch.offsets.copy()
+    idx = batch.indices.copy()
+    idx[::11] = cfg.rows[0] + 3
+    offs[7] = offs[6] - 1
+    offs[2 * cfg.B + 33] = -1
+    bt = sd.batch_on_device(batch)
+    x = np.random.default_rng(9).standard_normal((cfg.B, cfg.d)).astype(np.float32)
+    out = torch.full((cfg.B, cfg.concat_ld), float("nan"), dtype=sd.TORCH_DT[cfg.mlp_dtype], device="cuda")
+    E.dlrm_embbag_interact_fwd(g.T, cfg.B, torch.from_numpy(offs).cuda(), torch.from_numpy(idx).cuda(),
+                               torch.from_numpy(x).cuda(), out, cfg.concat_ld, cfg.mlp_dtype, g.ws)
+    st = E.dlrm_check_error(g.ws)
+    model = O.model_from_config(cfg)
+    pooled, _, counts = O.embbag(model.tables, cfg.rows, cfg.d, cfg.B, offs, idx)
+    assert counts[0] > 0 and counts[1] >= 2
+    assert st == (E.ERR_BAD_OFFSETS, 3, counts[0], counts[1])
+    want = O.interact(x, pooled)
+    sc = scale_concat(x, scale_pooled(model, cfg.B, offs, idx))
+    tol = "f32" if cfg.table_dtype == "f32" else "bf16"
+    assert_close(to_np(out)[:, :want.shape[1]], want, tol, "fused concat with bad bags", sc)
+
+
 def test_host_argument_errors(tiny):
     cfg, batch, g = tiny
     L = E.lib()
@@ -112,16 +141,16 @@ def test_host_argument_errors(tiny):
     assert L.dlrm_interact_fwd(cfg.B, 257, cfg.d, P(x), P(pooled), P(out), 10 ** 6, 0, s) == E.ERR_UNSUPPORTED
     # a table with zero rows
     bad = E.Tables(g.tables, [0] + list(cfg.rows[1:]), cfg.d)
-    assert L.dlrm_embbag_fwd(bad.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, P(g.ws), s) == E.ERR_INVALID_ARG
+    assert L.dlrm_embbag_fwd(bad.ref(), cfg.B, P(bt["offsets"]), P(bt["indices"]), nnz, P(pooled), None, P(g.ws), nws, s) == E.ERR_INVALID_ARG
     # unsupported row width: d = 301 fp32 is neither a 16-byte multiple <= 2 KB nor <= 256
     t300 = torch.zeros((10, 301), device="cuda")
     T300 = E.Tables(t300, [10], 301)
-    assert L.dlrm_embbag_fwd(T300.ref(), 1, P(bt["offsets"]), P(bt["indices"]), 0, P(pooled), None, P(g.ws), s) == E.ERR_UNSUPPORTED
+    assert L.dlrm_embbag_fwd(T300.ref(), 1, P(bt["offsets"]), P(bt["indices"]), 0, P(pooled), None, P(g.ws), nws, s) == E.ERR_UNSUPPORTED
     # forward with a top MLP whose input width does not match d + K(K+1)/2
     y = torch.empty(cfg.B, device="cuda")
-    assert L.dlrm_forward(g.T.ref(), g.bot.ref(), g.bot.ref(), cfg.B, P(bt["dense"]), P(bt["offsets"]), P(bt["indices"]), nnz, P(y), P(g.ws), s) == E.ERR_INVALID_ARG
+    assert L.dlrm_forward(g.T.ref(), g.bot.ref(), g.bot.ref(), cfg.B, P(bt["dense"]), P(bt["offsets"]), P(bt["indices"]), nnz, P(y), P(g.ws), nws, s) == E.ERR_INVALID_ARG
     # B = 0 is a valid no-op
-    assert L.dlrm_forward(g.T.ref(), g.bot.ref(), g.top.ref(), 0, None, None, None, 0, None, P(g.ws), s) == E.OK
+    assert L.dlrm_forward(g.T.ref(), g.bot.ref(), g.top.ref(), 0, None, None, None, 0, None, P(g.ws), nws, s) == E.OK
     torch.cuda.synchronize()
     assert E.dlrm_check_error(g.ws) == (0, 0, 0, 0)
 

@@ -37,6 +37,14 @@ def _cases():
                                                                 bag="mix", bottom=(13, 32, 256), top=(256 + 36, 32, 1)),
         "bf16-d32-K62": shrink(t, B=35).with_(rows=(300,) * 62, d=32, table_dtype="bf16", mlp_dtype="bf16",
                                                bottom=(13, 16, 32), top=(32 + 1953, 16, 1)),
+        # many tables (K + 2 > 64): row gather U deep and the Gram on mma.sync, m-tile counts 4..8
+        "bf16-d64-K63-mix": shrink(s, B=29, rows_cap=500).with_(rows=(500,) * 63, bag="mix", seed=6,
+                                                                 top=(64 + 2016, 64, 1)),
+        "bf16-d128-K70-u100": shrink(s, B=13, rows_cap=900).with_(rows=(900,) * 70, d=128, seed=7,
+                                                                   bottom=(13, 64, 128), top=(128 + 2485, 64, 1)),
+        "bf16-d64-K128-mix": shrink(s, B=9, rows_cap=300).with_(rows=(300,) * 128, bag="mix", seed=8,
+                                                                 top=(64 + 8256, 32, 1)),
+        "bf16-d64-K100-batch1": shrink(s, B=1, rows_cap=1000),
     }
 
 
