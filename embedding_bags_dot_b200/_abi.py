@@ -53,6 +53,22 @@ _lock = threading.Lock()
 _SIGS = {
     "dlrm_launch_count": (C.c_uint64, []),
     "dlrm_set_wait_polls": (C.c_int, [C.c_int64]),
+    "dlrm_pooled_assemble": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_void_p, C.c_void_p]),
+    "dlrm_pooled_split": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    C.c_void_p, C.c_void_p]),
+    "dlrm_embbag_sgd_scratch_size": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int64]),
+    "dlrm_backward_pooled_workspace_size": (C.c_size_t, [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int]),
+    "dlrm_grads_pooled_size": (C.c_size_t, [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int]),
+    "dlrm_grads_pooled_offsets": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                            C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dlrm_backward_pooled": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                       C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
+                                       C.c_size_t, C.c_void_p]),
+    "dlrm_mlp_sgd": (C.c_int, [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_int, C.c_float, C.c_void_p, C.c_size_t,
+                               C.c_void_p]),
+    "dlrm_embbag_sgd": (C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_float,
+                                  C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p]),
     "dlrm_ld": (C.c_int, [C.c_int, C.c_int]),
     "dlrm_status_str": (C.c_char_p, [C.c_int]),
     "dlrm_workspace_size": (C.c_size_t, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
@@ -391,6 +407,69 @@ def dlrm_embedding_row_grads(T: Tables, bot: MLP, top: MLP, B: int, nnz: int, gr
                                                  _nbytes(grads), _ptr(rows), _ptr(row_grads), _ptr(n_rows),
                                                  _stream(stream)),
                   "dlrm_embedding_row_grads")
+
+
+# ----------------------------------------------------------------- table-wise model parallelism
+
+def _parts_args(first_table, n_tables, ptrs):
+    n = len(first_table)
+    return (n, (C.c_int * n)(*[int(x) for x in first_table]), (C.c_int * n)(*[int(x) for x in n_tables]),
+            (C.c_void_p * n)(*ptrs))
+
+
+def dlrm_pooled_assemble(B: int, K: int, d: int, first_table, n_tables, parts, out, stream=None):
+    """out[b][first_p + j] = parts[p][b][j] for every part p (fp32 device tensors)."""
+    n, ft, nt, pp = _parts_args(first_table, n_tables, [_ptr(p) for p in parts])
+    return _check(lib().dlrm_pooled_assemble(int(B), int(K), int(d), n, ft, nt, pp, _ptr(out), _stream(stream)),
+                  "dlrm_pooled_assemble")
+
+
+def dlrm_pooled_split(B: int, K: int, d: int, first_table, n_tables, inp, parts, stream=None):
+    """parts[p][b][j] = inp[b][first_p + j] (the inverse of dlrm_pooled_assemble)."""
+    n, ft, nt, pp = _parts_args(first_table, n_tables, [_ptr(p) for p in parts])
+    return _check(lib().dlrm_pooled_split(int(B), int(K), int(d), n, ft, nt, _ptr(inp), pp, _stream(stream)),
+                  "dlrm_pooled_split")
+
+
+def dlrm_embbag_sgd_scratch_size(T: Tables, B: int, nnz: int) -> int:
+    return int(lib().dlrm_embbag_sgd_scratch_size(T.ref(), int(B), int(nnz)))
+
+
+def dlrm_embbag_sgd(T: Tables, B: int, offsets, indices, dE, lr: float, scratch, n_touched=None, stream=None):
+    """T[r] -= lr * (sum of dE over the occurrences of row r), for the rows the bags touch."""
+    return _check(lib().dlrm_embbag_sgd(T.ref(), int(B), _ptr(offsets), _ptr(indices), int(indices.numel()), _ptr(dE),
+                                        float(lr), _ptr(scratch), _nbytes(scratch), _ptr(n_touched), _stream(stream)),
+                  "dlrm_embbag_sgd")
+
+
+def dlrm_backward_pooled_workspace_size(K: int, d: int, bot: MLP, top: MLP, B: int) -> int:
+    return int(lib().dlrm_backward_pooled_workspace_size(int(K), int(d), bot.ref(), top.ref(), int(B)))
+
+
+def dlrm_grads_pooled_size(K: int, d: int, bot: MLP, top: MLP, B: int) -> int:
+    return int(lib().dlrm_grads_pooled_size(int(K), int(d), bot.ref(), top.ref(), int(B)))
+
+
+def dlrm_grads_pooled_offsets(K: int, d: int, bot: MLP, top: MLP, B: int) -> dict:
+    nb, nt = len(bot.Ws), len(top.Ws)
+    arrs = [(C.c_size_t * n)() for n in (nb, nb, nt, nt)]
+    dE, loss, end = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    _check(lib().dlrm_grads_pooled_offsets(int(K), int(d), bot.ref(), top.ref(), int(B), *arrs, C.byref(dE),
+                                           C.byref(loss), C.byref(end)), "dlrm_grads_pooled_offsets")
+    return {"bot_dW": list(arrs[0]), "bot_db": list(arrs[1]), "top_dW": list(arrs[2]), "top_db": list(arrs[3]),
+            "dE": dE.value, "loss": loss.value, "dense_end": end.value}
+
+
+def dlrm_backward_pooled(K: int, d: int, bot: MLP, top: MLP, B: int, dense, pooled, labels, grads, ws, loss=None,
+                         y_hat=None, stream=None):
+    return _check(lib().dlrm_backward_pooled(int(K), int(d), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(pooled),
+                                             _ptr(labels), _ptr(loss), _ptr(y_hat), _ptr(grads), _nbytes(grads),
+                                             _ptr(ws), _nbytes(ws), _stream(stream)), "dlrm_backward_pooled")
+
+
+def dlrm_mlp_sgd(K: int, d: int, bot: MLP, top: MLP, B: int, lr: float, grads, stream=None):
+    return _check(lib().dlrm_mlp_sgd(int(K), int(d), bot.ref(), top.ref(), int(B), float(lr), _ptr(grads),
+                                     _nbytes(grads), _stream(stream)), "dlrm_mlp_sgd")
 
 
 def grads_view(grads: torch.Tensor, off: int, shape) -> torch.Tensor:

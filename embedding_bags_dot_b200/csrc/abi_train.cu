@@ -44,7 +44,9 @@ struct Grads {
 
 int ldf(int n) { return dlrm_ld(n, DLRM_F32); }
 
-TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
+// Layout for K tables of width d holding total_rows rows; allow_tc = false forces the path that reads pooled
+// vectors (the caller's, or the ones the step pools itself).
+TrainWs train_ws(int K, int d, long long total_rows, bool allow_tc, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
     TrainWs W;
     size_t off = DLRM_ERR_RECORD_BYTES;
     auto take = [&](size_t bytes) {
@@ -52,7 +54,6 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
         off = align_up(off + bytes, 256);
         return o;
     };
-    const int K = T->K, d = T->d;
     const int nb = bot->n_layers, nt = top->n_layers;
     for (int l = 0; l < nb; ++l)
         for (int h = 0; h < 2; ++h) W.bW[l][h] = take(sizeof(float) * (size_t)bot->dims[l + 1] * ldf(bot->dims[l]));
@@ -65,10 +66,8 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
         gmax = std::max(gmax, W.ldb[l]);
     }
     W.ldc = ldf(d + K * (K + 1) / 2);
-    long long total_rows = 0;
-    for (int k = 0; k < K; ++k) total_rows += T->rows[k];
     // the fused tensor-core interaction gathers the bags itself: no pooled vectors, no plain-fp32 copies
-    W.tc = interact_tc_supported(K, d, total_rows, W.ldc);
+    W.tc = allow_tc && interact_tc_supported(K, d, total_rows, W.ldc);
     W.xd = W.tc ? 0 : take(sizeof(float) * (size_t)B * d);
     W.E = W.tc ? 0 : take(sizeof(float) * (size_t)B * K * d);
     W.concat = W.tc ? 0 : take(sizeof(float) * (size_t)B * W.ldc);
@@ -100,7 +99,7 @@ TrainWs train_ws(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top,
     return W;
 }
 
-Grads grads_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, long long nnz) {
+Grads grads_layout(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, long long nnz) {
     Grads G;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -116,9 +115,9 @@ Grads grads_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* to
         G.tdW[l] = take(sizeof(float) * (size_t)top->dims[l + 1] * ldf(top->dims[l]));
         G.tdb[l] = take(sizeof(float) * (size_t)top->dims[l + 1]);
     }
-    G.dE = take(sizeof(float) * (size_t)B * T->K * T->d);
+    G.dE = take(sizeof(float) * (size_t)B * K * d);
     G.loss = take(sizeof(float));
-    G.sp = sparse_layout((long long)T->K * B, nnz, T->d);
+    G.sp = sparse_layout((long long)K * B, nnz, d);
     G.sparse = take(G.sp.total);
     G.total = off;
     return G;
@@ -167,7 +166,7 @@ namespace dlrm {
 size_t train_workspace_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
     TableMeta tm;
     if (check_train(T, bot, top, B, tm) != DLRM_OK) return 0;
-    return train_ws(T, bot, top, B).total;
+    return train_ws(T->K, T->d, total_rows_of(tm, T->K), true, bot, top, B).total;
 }
 }  // namespace dlrm
 
@@ -176,7 +175,7 @@ extern "C" {
 size_t dlrm_grads_size(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz) {
     TableMeta tm;
     if (check_train(T, bot, top, B, tm) != DLRM_OK || nnz < 0) return 0;
-    return grads_layout(T, bot, top, B, nnz).total;
+    return grads_layout(T->K, T->d, bot, top, B, nnz).total;
 }
 
 dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
@@ -185,7 +184,7 @@ dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const 
     TableMeta tm;
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
-    const Grads G = grads_layout(T, bot, top, B, nnz);
+    const Grads G = grads_layout(T->K, T->d, bot, top, B, nnz);
     for (int l = 0; l < bot->n_layers; ++l) {
         if (bot_dW) bot_dW[l] = G.bdW[l];
         if (bot_db) bot_db[l] = G.bdb[l];
@@ -199,26 +198,21 @@ dlrm_status dlrm_grads_offsets(const dlrm_tables* T, const dlrm_mlp* bot, const 
     return DLRM_OK;
 }
 
-dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
-                          const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
-                          float* loss, float* y_hat, void* grads, size_t grads_bytes, void* ws, size_t ws_bytes,
-                          dlrm_stream stream) {
-    TableMeta tm;
-    dlrm_status r = check_train(T, bot, top, B, tm);
-    if (r) return r;
-    if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws) || !grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
-    if (ws_bytes < dlrm_workspace_size(T, bot, top, B, 1) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
-        return DLRM_ERR_WORKSPACE;
-    if (B == 0) return DLRM_OK;
-    if (!dense || !offsets || (nnz > 0 && !indices) || !labels) return DLRM_ERR_INVALID_ARG;
-    const int K = T->K, d = T->d;
-    const TrainWs W = train_ws(T, bot, top, B);
-    const Grads G = grads_layout(T, bot, top, B, nnz);
+}  // extern "C"
+
+namespace {
+
+// The training step's forward and backward on one batch. With pooled == nullptr it gathers the bags of the
+// tables itself (tm, tables, offsets, indices) and finishes with the row-sorted preparation of the sparse
+// update; with pooled ([B][K][d] fp32) the given vectors stand in for the pooled bags and no row is touched.
+dlrm_status backward_impl(int K, int d, const TableMeta& tm, const float* tables, const dlrm_mlp* bot,
+                          const dlrm_mlp* top, int B, const float* dense, const int32_t* offsets,
+                          const int32_t* indices, int64_t nnz, const float* pooled, const float* labels, float* loss,
+                          float* y_hat, void* grads, void* ws, const TrainWs& W, const Grads& G, cudaStream_t st) {
+    dlrm_status r;
     char* w = static_cast<char*>(ws);
     char* g = static_cast<char*>(grads);
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
-    cudaStream_t st = cs(stream);
     auto F = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
     auto U = [&](size_t o) { return reinterpret_cast<uint32_t*>(w + o); };
     auto GF = [&](size_t o) { return reinterpret_cast<float*>(g + o); };
@@ -248,7 +242,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     }
     const F32Pair xd_pair = P(W.bact[nb - 1], W.ldb[nb - 1]);   // ld = d (d % 4 == 0 on this path)
     const float* x_dense = W.tc ? nullptr : F(W.xd);
-    const float* tables = static_cast<const float*>(T->data);
+    const float* E = pooled ? pooled : (W.tc ? nullptr : F(W.E));
     // the fused tensor-core interaction gathers the bags and reads/writes pairs; other shapes pool the bags
     // first and go through plain fp32 copies
     if (W.tc) {
@@ -256,10 +250,11 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
                                         F(W.concat_p[1]), W.ldc, err, st)))
             return r;
     } else {
-        if ((r = launch_embbag(tm, T->data, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err, st)))
+        if (!pooled && (r = launch_embbag(tm, tables, DLRM_F32, K, d, B, offsets, indices, nnz, F(W.E), nullptr, err,
+                                          st)))
             return r;
         if ((r = launch_merge_pair(B, d, xd_pair.hi, xd_pair.lo, xd_pair.ld, F(W.xd), d, st))) return r;
-        if ((r = launch_interact(B, K, d, x_dense, F(W.E), F(W.concat), W.ldc, DLRM_F32, st))) return r;
+        if ((r = launch_interact(B, K, d, x_dense, E, F(W.concat), W.ldc, DLRM_F32, st))) return r;
         if ((r = launch_split_pair(B, top->dims[0], F(W.concat), W.ldc, F(W.concat_p[0]), F(W.concat_p[1]), W.ldc,
                                    st)))
             return r;
@@ -311,7 +306,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
                                         F(W.g[pp][0]), F(W.g[pp][1]), d, GF(G.dE), err, st)))
             return r;
     } else {
-        if ((r = launch_interact_bwd(B, K, d, x_dense, F(W.E), F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;
+        if ((r = launch_interact_bwd(B, K, d, x_dense, E, F(W.dcat), W.ldc, F(W.dxd), GF(G.dE), st))) return r;
         if ((r = launch_split_pair(B, d, F(W.dxd), d, F(W.g[pp][0]), F(W.g[pp][1]), d, st))) return r;
     }
     cur = F32Pair{F(W.g[pp][0]), F(W.g[pp][1]), d};
@@ -336,6 +331,7 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     }
 
     // ---- embedding rows: sort occurrences by row, cut segments and pieces
+    if (pooled) return DLRM_OK;
     int sorted_buf = 0;
     if ((r = launch_sparse_prepare(K, B, tm, total_rows_of(tm, K), offsets, indices, nnz, g + G.sparse, G.sp, err,
                                    &sorted_buf, st)))
@@ -343,16 +339,134 @@ dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_
     return DLRM_OK;
 }
 
+// Shapes of the pooled-input step: the same MLP and width rules as check_train, for K vectors of width d.
+dlrm_status check_pooled(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
+    if (K < 1 || d < 1 || B < 0 || !bot || !top || !bot->dims || !top->dims || !bot->W || !bot->b || !top->W ||
+        !top->b)
+        return DLRM_ERR_INVALID_ARG;
+    if (K > DLRM_MAX_TABLES || bot->n_layers < 1 || top->n_layers < 1 || bot->n_layers > DLRM_MAX_LAYERS ||
+        top->n_layers > DLRM_MAX_LAYERS)
+        return DLRM_ERR_UNSUPPORTED;
+    if (bot->dt != DLRM_F32 || top->dt != DLRM_F32) return DLRM_ERR_UNSUPPORTED;
+    for (int l = 0; l <= bot->n_layers; ++l)
+        if (bot->dims[l] < 1) return DLRM_ERR_INVALID_ARG;
+    for (int l = 0; l <= top->n_layers; ++l)
+        if (top->dims[l] < 1) return DLRM_ERR_INVALID_ARG;
+    for (int l = 0; l < bot->n_layers; ++l)
+        if (!bot->W[l] || !bot->b[l]) return DLRM_ERR_INVALID_ARG;
+    for (int l = 0; l < top->n_layers; ++l)
+        if (!top->W[l] || !top->b[l]) return DLRM_ERR_INVALID_ARG;
+    if (bot->dims[bot->n_layers] != d || top->dims[0] != d + K * (K + 1) / 2 || top->dims[top->n_layers] != 1)
+        return DLRM_ERR_INVALID_ARG;
+    if (d % 4 || interact_bwd_smem(K, d) > 227 * 1024 || interact_smem_per_sample(K, d) > 227 * 1024)
+        return DLRM_ERR_UNSUPPORTED;
+    return DLRM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dlrm_status dlrm_backward(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                          const int32_t* offsets, const int32_t* indices, int64_t nnz, const float* labels,
+                          float* loss, float* y_hat, void* grads, size_t grads_bytes, void* ws, size_t ws_bytes,
+                          dlrm_stream stream) {
+    TableMeta tm;
+    dlrm_status r = check_train(T, bot, top, B, tm);
+    if (r) return r;
+    if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || !grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
+    if (ws_bytes < dlrm_workspace_size(T, bot, top, B, 1) || grads_bytes < grads_layout(T->K, T->d, bot, top, B, nnz).total)
+        return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    if (!dense || !offsets || (nnz > 0 && !indices) || !labels) return DLRM_ERR_INVALID_ARG;
+    const int K = T->K, d = T->d;
+    const TrainWs W = train_ws(K, d, total_rows_of(tm, K), true, bot, top, B);
+    const Grads G = grads_layout(K, d, bot, top, B, nnz);
+    return backward_impl(K, d, tm, static_cast<const float*>(T->data), bot, top, B, dense, offsets, indices, nnz,
+                         nullptr, labels, loss, y_hat, grads, ws, W, G, cs(stream));
+}
+
+size_t dlrm_backward_pooled_workspace_size(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
+    if (check_pooled(K, d, bot, top, B) != DLRM_OK) return 0;
+    return train_ws(K, d, 0, false, bot, top, B).total;
+}
+
+size_t dlrm_grads_pooled_size(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
+    if (check_pooled(K, d, bot, top, B) != DLRM_OK) return 0;
+    return grads_layout(K, d, bot, top, B, 0).total;
+}
+
+dlrm_status dlrm_grads_pooled_offsets(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, size_t* bot_dW,
+                                      size_t* bot_db, size_t* top_dW, size_t* top_db, size_t* dE, size_t* loss,
+                                      size_t* dense_end) {
+    dlrm_status r = check_pooled(K, d, bot, top, B);
+    if (r) return r;
+    const Grads G = grads_layout(K, d, bot, top, B, 0);
+    for (int l = 0; l < bot->n_layers; ++l) {
+        if (bot_dW) bot_dW[l] = G.bdW[l];
+        if (bot_db) bot_db[l] = G.bdb[l];
+    }
+    for (int l = 0; l < top->n_layers; ++l) {
+        if (top_dW) top_dW[l] = G.tdW[l];
+        if (top_db) top_db[l] = G.tdb[l];
+    }
+    if (dE) *dE = G.dE;
+    if (loss) *loss = G.loss;
+    if (dense_end) *dense_end = G.dE;
+    return DLRM_OK;
+}
+
+dlrm_status dlrm_backward_pooled(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                                 const float* pooled, const float* labels, float* loss, float* y_hat, void* grads,
+                                 size_t grads_bytes, void* ws, size_t ws_bytes, dlrm_stream stream) {
+    dlrm_status r = check_pooled(K, d, bot, top, B);
+    if (r) return r;
+    if (!ws || !aligned16(ws) || !grads || !aligned16(grads)) return DLRM_ERR_WORKSPACE;
+    const TrainWs W = train_ws(K, d, 0, false, bot, top, B);
+    const Grads G = grads_layout(K, d, bot, top, B, 0);
+    if (ws_bytes < W.total || grads_bytes < G.total) return DLRM_ERR_WORKSPACE;
+    if (B == 0) return DLRM_OK;
+    if (!dense || !pooled || !labels || !aligned16(pooled)) return DLRM_ERR_INVALID_ARG;
+    TableMeta tm;
+    return backward_impl(K, d, tm, nullptr, bot, top, B, dense, nullptr, nullptr, 0, pooled, labels, loss, y_hat,
+                         grads, ws, W, G, cs(stream));
+}
+
+dlrm_status dlrm_mlp_sgd(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, float lr, const void* grads,
+                         size_t grads_bytes, dlrm_stream stream) {
+    dlrm_status r = check_pooled(K, d, bot, top, B);
+    if (r) return r;
+    const Grads G = grads_layout(K, d, bot, top, B, 0);
+    if (!grads || !aligned16(grads) || grads_bytes < G.dE) return DLRM_ERR_WORKSPACE;
+    const char* g = static_cast<const char*>(grads);
+    cudaStream_t st = cs(stream);
+    for (int l = 0; l < bot->n_layers; ++l) {
+        const long long n = (long long)bot->dims[l + 1] * ldf(bot->dims[l]);
+        if ((r = launch_sgd(n, lr, static_cast<float*>(bot->W[l]), reinterpret_cast<const float*>(g + G.bdW[l]), st)) ||
+            (r = launch_sgd(bot->dims[l + 1], lr, bot->b[l], reinterpret_cast<const float*>(g + G.bdb[l]), st)))
+            return r;
+    }
+    for (int l = 0; l < top->n_layers; ++l) {
+        const long long n = (long long)top->dims[l + 1] * ldf(top->dims[l]);
+        if ((r = launch_sgd(n, lr, static_cast<float*>(top->W[l]), reinterpret_cast<const float*>(g + G.tdW[l]), st)) ||
+            (r = launch_sgd(top->dims[l + 1], lr, top->b[l], reinterpret_cast<const float*>(g + G.tdb[l]), st)))
+            return r;
+    }
+    return DLRM_OK;
+}
+
+
 dlrm_status dlrm_sparse_sgd(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B, int64_t nnz,
                             float lr, void* grads, size_t grads_bytes, int32_t* n_touched, dlrm_stream stream) {
     TableMeta tm;
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
     if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
-    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
+    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T->K, T->d, bot, top, B, nnz).total)
         return DLRM_ERR_WORKSPACE;
     if (B == 0) return DLRM_OK;
-    const Grads G = grads_layout(T, bot, top, B, nnz);
+    const Grads G = grads_layout(T->K, T->d, bot, top, B, nnz);
     const char* g = static_cast<const char*>(grads);
     cudaStream_t st = cs(stream);
     const int sorted = radix_passes(total_rows_of(tm, T->K)) & 1;
@@ -381,11 +495,11 @@ dlrm_status dlrm_embedding_row_grads(const dlrm_tables* T, const dlrm_mlp* bot, 
     dlrm_status r = check_train(T, bot, top, B, tm);
     if (r) return r;
     if (nnz < 0 || nnz >= (int64_t(1) << 31)) return DLRM_ERR_INVALID_ARG;
-    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T, bot, top, B, nnz).total)
+    if (!grads || !aligned16(grads) || grads_bytes < grads_layout(T->K, T->d, bot, top, B, nnz).total)
         return DLRM_ERR_WORKSPACE;
     if (!rows || !row_grads || !n_rows) return DLRM_ERR_INVALID_ARG;
     if (B == 0) return DLRM_OK;
-    const Grads G = grads_layout(T, bot, top, B, nnz);
+    const Grads G = grads_layout(T->K, T->d, bot, top, B, nnz);
     const char* g = static_cast<const char*>(grads);
     const int sorted = radix_passes(total_rows_of(tm, T->K)) & 1;
     return launch_sparse_apply(T->d, g + G.sparse, G.sp, sorted, reinterpret_cast<const float*>(g + G.dE), 0.f,

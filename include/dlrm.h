@@ -327,6 +327,73 @@ dlrm_status dlrm_gemm_tf32x3(int I, int J, int R, const float* A_hi, const float
                              const float* B_hi, const float* B_lo, int ldb, int b_mn, float* C, int ldc, void* ws,
                              size_t ws_bytes, dlrm_stream stream);
 
+/* ------------------------------------------------- table-wise model parallelism
+ * The pages' system keeps the embedding tables model-parallel and the fully
+ * connected layers data-parallel, with an all-to-all of the lookup results
+ * between the two (arXiv 1906.00091 index page, Abstract; the
+ * science.uptrusthq.com citation snippet on all-to-all communication of the
+ * embedding lookups; "DLRM", briansu.co, section 5). Each rank owns a
+ * contiguous range of tables, pools its own tables' bags for the whole
+ * batch (dlrm_embbag_fwd), and the caller's collective (NCCL all-to-all)
+ * sends each rank the rows of its batch shard. These calls place the
+ * received blocks and apply the owner's sparse update.
+ *
+ * dlrm_pooled_assemble: parts[p] (device, fp32 [B][n_tables[p]][d]) holds
+ * tables first_table[p] .. first_table[p] + n_tables[p] - 1; the parts must
+ * tile 0 .. K-1 in order (first_table[0] = 0, each next part starting where
+ * the previous ends). out (device, fp32 [B][K][d]) receives every part in
+ * its columns. first_table, n_tables and parts are host arrays of n_parts
+ * entries. Strided device-to-device copies on `stream`, no kernel.
+ * dlrm_pooled_split: the inverse (in [B][K][d] -> parts), for the gradients
+ * of the pooled vectors on their way back to the owners.
+ * DLRM_ERR_INVALID_ARG for parts that do not tile 0 .. K-1 or null pointers. */
+dlrm_status dlrm_pooled_assemble(int B, int K, int d, int n_parts, const int* first_table, const int* n_tables,
+                                 const float* const* parts, float* out, dlrm_stream stream);
+dlrm_status dlrm_pooled_split(int B, int K, int d, int n_parts, const int* first_table, const int* n_tables,
+                              const float* in, float* const* parts, dlrm_stream stream);
+
+/* The data-parallel half of a sharded training step, for one rank's batch
+ * shard: dlrm_backward with the pooled vectors given instead of tables and
+ * bags. pooled: device fp32 [B][K][d], 16-byte aligned (the vectors the
+ * all-to-all brought, placed by dlrm_pooled_assemble). The forward (bottom
+ * MLP, interaction, top MLP, sigmoid), the mean BCE loss over these B samples
+ * and the backward run as in dlrm_backward; grads receives every MLP
+ * gradient and, at the dE offset, the gradient of every pooled vector
+ * [B][K][d] (to be split per owner with dlrm_pooled_split and sent back). No
+ * row of any table is read or written. Offsets inside grads:
+ * dlrm_grads_pooled_offsets (dense_end: the MLP gradients occupy bytes
+ * [0, dense_end), one contiguous range for the data-parallel all-reduce).
+ * Sizes: grads_bytes >= dlrm_grads_pooled_size(...), ws_bytes >=
+ * dlrm_backward_pooled_workspace_size(...). fp32 MLPs, d % 4 == 0. */
+size_t dlrm_backward_pooled_workspace_size(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B);
+size_t dlrm_grads_pooled_size(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B);
+dlrm_status dlrm_grads_pooled_offsets(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, size_t* bot_dW,
+                                      size_t* bot_db, size_t* top_dW, size_t* top_db, size_t* dE, size_t* loss,
+                                      size_t* dense_end);
+dlrm_status dlrm_backward_pooled(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, const float* dense,
+                                 const float* pooled, const float* labels, float* loss, float* y_hat, void* grads,
+                                 size_t grads_bytes, void* ws, size_t ws_bytes, dlrm_stream stream);
+/* W -= lr * dW and b -= lr * db for every layer of both MLPs, from a
+ * gradient buffer laid out by dlrm_grads_pooled_offsets (grads_bytes >=
+ * dense_end). */
+dlrm_status dlrm_mlp_sgd(int K, int d, const dlrm_mlp* bot, const dlrm_mlp* top, int B, float lr, const void* grads,
+                         size_t grads_bytes, dlrm_stream stream);
+
+/* The owner's half of the sparse SGD step (the update dlrm_sparse_sgd applies
+ * to the embedding rows), from the gradient of every pooled bag of its own
+ * tables: T[r] -= lr * g_r for every row r a valid index of the batch
+ * touches, with g_r = sum of dE[b][k] over the occurrences of r in bag (k, b),
+ * added in occurrence order (bit-reproducible); untouched rows are not
+ * written. fp32 tables only (d % 4 == 0); bags as dlrm_embbag_fwd (skipped
+ * indices and bad bags contribute nothing). dE: device fp32 [B][K][d], 16-byte
+ * aligned. scratch: 16-byte aligned, scratch_bytes >=
+ * dlrm_embbag_sgd_scratch_size(T, B, nnz) (error record, then the sort and
+ * segment arrays). n_touched (device int32, optional): rows updated. */
+size_t dlrm_embbag_sgd_scratch_size(const dlrm_tables* T, int B, int64_t nnz);
+dlrm_status dlrm_embbag_sgd(const dlrm_tables* T, int B, const int32_t* offsets, const int32_t* indices, int64_t nnz,
+                            const float* dE, float lr, void* scratch, size_t scratch_bytes, int32_t* n_touched,
+                            dlrm_stream stream);
+
 /* Size of the device scratch array that dlrm_forward_noalloc uses (32 MiB). */
 #define DLRM_NOALLOC_SCRATCH_BYTES (32u << 20)
 
