@@ -74,9 +74,40 @@ size_t hidden_bytes(const dlrm_mlp* m, int B) {
 // widest hidden layer output; none for one layer, one for two), then the input converted to the MLP's
 // dtype when it comes in another one.
 struct MlpWs {
-    size_t act, cvt, total;
+    size_t act, cvt, f32tc, total;
     int nact;
 };
+
+// fp32 MLPs run their layers on the tensor cores as 3xTF32 GEMMs, whose operands are (hi, lo) pairs: the
+// split weights of every layer, the split input, two pair buffers for the hidden outputs and the last
+// layer's pair output. Byte offsets relative to the start of this region.
+struct F32TcWs {
+    size_t w[DLRM_MAX_LAYERS][2], in[2], act[2][2], total;
+    int ld_in, ld_act;
+};
+
+F32TcWs f32tc_ws(const dlrm_mlp* m, int B) {
+    F32TcWs W{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    int widest = 1, widest_in = 1;
+    for (int l = 0; l < m->n_layers; ++l) {
+        for (int h = 0; h < 2; ++h) W.w[l][h] = take(sizeof(float) * (size_t)m->dims[l + 1] * dlrm_ld(m->dims[l], DLRM_F32));
+        widest = std::max(widest, m->dims[l + 1]);
+        widest_in = std::max(widest_in, m->dims[l]);
+    }
+    W.ld_in = dlrm_ld(widest_in, DLRM_F32);   // the split input, or any layer's input merged back to plain
+    W.ld_act = dlrm_ld(widest, DLRM_F32);
+    for (int h = 0; h < 2; ++h) W.in[h] = take(sizeof(float) * (size_t)B * W.ld_in);
+    for (int p = 0; p < 2; ++p)
+        for (int h = 0; h < 2; ++h) W.act[p][h] = take(sizeof(float) * (size_t)B * W.ld_act);
+    W.total = off;
+    return W;
+}
 
 MlpWs mlp_ws(const dlrm_mlp* m, int B, dlrm_dtype in_dt) {
     MlpWs w{};
@@ -86,12 +117,13 @@ MlpWs mlp_ws(const dlrm_mlp* m, int B, dlrm_dtype in_dt) {
     w.nact = m->n_layers >= 3 ? 2 : m->n_layers - 1;
     const bool conv = in_dt != m->dt && m->dt != DLRM_F32;
     w.cvt = conv ? align_up((size_t)dlrm_ld(m->dims[0], m->dt) * esize(m->dt) * (size_t)B, 256) : 0;
-    w.total = DLRM_ERR_RECORD_BYTES + (size_t)w.nact * w.act + w.cvt;
+    w.f32tc = m->dt == DLRM_F32 ? f32tc_ws(m, B).total : 0;
+    w.total = DLRM_ERR_RECORD_BYTES + (size_t)w.nact * w.act + w.cvt + w.f32tc;
     return w;
 }
 
 struct FwdLayout {
-    size_t x_dense, concat, act0, act1, cvt, offs, lscratch, total;
+    size_t x_dense, concat, act0, act1, cvt, offs, lscratch, f32tc, total;
 };
 
 FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* top, int B) {
@@ -118,6 +150,11 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
     off = align_up(off + sizeof(int32_t) * (size_t)(nbags + 1), 256);
     L.lscratch = off;
     off = align_up(off + sizeof(int) * lengths_scratch_ints(nbags), 256);
+    // fp32 MLPs: the 3xTF32 pair buffers of the larger of the two (one MLP runs at a time)
+    const size_t f32 = std::max(bot->dt == DLRM_F32 ? f32tc_ws(bot, B).total : 0,
+                                top->dt == DLRM_F32 ? f32tc_ws(top, B).total : 0);
+    L.f32tc = off;
+    off = align_up(off + f32, 256);
     L.total = off;
     return L;
 }
@@ -125,8 +162,58 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
 // The MLP chain: ReLU after hidden layers, final_act after the last layer. An fp32 input
 // to a 16-bit MLP is first converted (into cvt) so that every layer can take the
 // tensor-core path.
+// A layer of an fp32 MLP goes to the 3xTF32 tensor-core GEMM when the output is wide enough to fill its
+// tiles and the batch fills the GPU; the first bottom layer (13 inputs) and one-column layers stay on the
+// CUDA cores.
+bool f32_layer_on_tc(int M, int N, int K) { return M >= 1024 && N >= 16 && K > 16; }
+
+// fp32 MLP: hidden layers as (hi, lo) pairs in the tensor-core buffers at `tc` (F32TcWs layout); a layer
+// that stays on the CUDA cores reads and writes the same pairs; the last layer writes `out` plain.
+dlrm_status run_mlp_f32(const dlrm_mlp* m, int B, const float* in, int ld_in, float* out, int ld_out, int final_act,
+                        char* tc, ErrRecord* err, cudaStream_t st) {
+    const F32TcWs W = f32tc_ws(m, B);
+    auto F = [&](size_t o) { return reinterpret_cast<float*>(tc + o); };
+    dlrm_status r;
+    F32Pair cur{in, nullptr, ld_in};
+    for (int l = 0; l < m->n_layers; ++l) {
+        const int K = m->dims[l], N = m->dims[l + 1], ldw = dlrm_ld(K, DLRM_F32);
+        const bool last = l == m->n_layers - 1;
+        const bool use_tc = f32_layer_on_tc(B, N, K) && (!last || final_act == DLRM_ACT_RELU);
+        if (!use_tc && last) {
+            // plain input for the CUDA-core layer (and its activation): merge a pair first
+            if (cur.lo) {
+                if ((r = launch_merge_pair(B, K, cur.hi, cur.lo, cur.ld, F(W.in[0]), W.ld_in, st))) return r;
+                cur = F32Pair{F(W.in[0]), nullptr, W.ld_in};
+            }
+            return launch_linear(B, N, K, cur.hi, DLRM_F32, cur.ld, m->W[l], DLRM_F32, ldw, m->b[l], out, DLRM_F32,
+                                 ld_out, final_act, err, st);
+        }
+        const F32Pair Wp{F(W.w[l][0]), F(W.w[l][1]), ldw};
+        if ((r = launch_split_pair(N, K, static_cast<const float*>(m->W[l]), ldw, F(W.w[l][0]), F(W.w[l][1]), ldw, st)))
+            return r;
+        if (use_tc && !cur.lo) {
+            if ((r = launch_split_pair(B, K, cur.hi, cur.ld, F(W.in[0]), F(W.in[1]), W.ld_in, st))) return r;
+            cur = F32Pair{F(W.in[0]), F(W.in[1]), W.ld_in};
+        }
+        const int p = l & 1;
+        float* yh = F(W.act[p][0]);
+        float* yl = F(W.act[p][1]);
+        if ((r = train_linear_fwd(B, N, K, cur, Wp, m->b[l], yh, yl, W.ld_act, true, nullptr, err, st))) return r;
+        cur = F32Pair{yh, yl, W.ld_act};
+        if (last) return launch_merge_pair(B, N, yh, yl, W.ld_act, out, ld_out, st);
+    }
+    return DLRM_OK;
+}
+
 dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, int ld_in, float* out, int ld_out,
-                    int final_act, void* act0, void* act1, void* cvt, ErrRecord* err, cudaStream_t st) {
+                    int final_act, void* act0, void* act1, void* cvt, ErrRecord* err, cudaStream_t st,
+                    char* f32tc = nullptr) {
+    if (m->dt == DLRM_F32 && in_dt == DLRM_F32 && f32tc) {
+        bool any = false;
+        for (int l = 0; l < m->n_layers; ++l) any |= f32_layer_on_tc(B, m->dims[l + 1], m->dims[l]);
+        if (any)
+            return run_mlp_f32(m, B, static_cast<const float*>(in), ld_in, out, ld_out, final_act, f32tc, err, st);
+    }
     const void* cur = in;
     dlrm_dtype cur_dt = in_dt;
     int cur_ld = ld_in;
@@ -276,7 +363,7 @@ dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype 
     if (!ws || !aligned16(ws) || ws_bytes < L.total) return DLRM_ERR_WORKSPACE;
     char* w = static_cast<char*>(ws) + DLRM_ERR_RECORD_BYTES;
     return run_mlp(mlp, B, in, in_dt, ld_in, out, ld_out, final_act, w, w + L.act, w + (size_t)L.nact * L.act,
-                   static_cast<ErrRecord*>(ws), cs(stream));
+                   static_cast<ErrRecord*>(ws), cs(stream), L.f32tc ? w + (size_t)L.nact * L.act + L.cvt : nullptr);
 }
 
 size_t dlrm_mlp_workspace_size(const dlrm_mlp* mlp, int B, dlrm_dtype in_dt) {
@@ -331,7 +418,7 @@ dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
     const int ldc = dlrm_ld(width, top->dt);
     ErrRecord* err = reinterpret_cast<ErrRecord*>(w);
     if ((r = run_mlp(bot, B, dense, DLRM_F32, bot->dims[0], x_dense, d, DLRM_ACT_RELU, w + L.act0, w + L.act1,
-                     w + L.cvt, err, st)))
+                     w + L.cvt, err, st, w + L.f32tc)))
         return r;
     r = cat ? launch_embbag_cat(tm, T->data, T->dt, K, d, B, offsets, indices, nnz, x_dense, concat, ldc, top->dt, err,
                                 st)
@@ -339,7 +426,7 @@ dlrm_status forward_impl(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_m
                                      err, st);
     if (r) return r;
     return run_mlp(top, B, concat, top->dt, ldc, y_hat, 1, DLRM_ACT_SIGMOID, w + L.act0, w + L.act1, w + L.cvt, err,
-                   st);
+                   st, w + L.f32tc);
 }
 
 }  // namespace

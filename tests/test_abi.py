@@ -101,17 +101,25 @@ def _cpu_mlp(dims, dt):
 def test_mlp_workspace_size_follows_the_documented_layout(lib):
     """Error record (256 B), then one activation buffer per alternating hidden output (none for one layer,
     one for two, two otherwise) of the widest hidden output, then the input converted to a 16-bit MLP
-    dtype when it comes in another dtype; every piece rounded up to 256 bytes."""
+    dtype when it comes in another dtype, then (fp32 MLPs) the 3xTF32 pair buffers; every piece rounded up
+    to 256 bytes."""
     import embedding_bags_dot_b200 as E
     a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
     B = 1000
-    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), B, "f32") == 256
+
+    def f32tc(dims, B):
+        """fp32 MLPs add their 3xTF32 pair buffers: split weights, split input, two hidden pair buffers."""
+        ldf = lambda n: (n + 3) // 4 * 4  # noqa: E731
+        w = sum(2 * a256(4 * dims[l + 1] * ldf(dims[l])) for l in range(len(dims) - 1))
+        return w + 2 * a256(4 * B * ldf(max(dims[:-1]))) + 4 * a256(4 * B * ldf(max(dims[1:])))
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), B, "f32") == 256 + f32tc([13, 64], B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "bf16"), B, "f32") == 256 + a256(16 * 2 * B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 512, 128], "bf16"), B, "f32") == 256 + a256(512 * 2 * B) + a256(16 * 2 * B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 512, 256, 128], "bf16"), B, "bf16") == 256 + 2 * a256(512 * 2 * B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([479, 1024, 1024, 512, 256, 1], "bf16"), 77, "bf16") == \
         256 + 2 * a256(1024 * 2 * 77)
-    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 100, 3], "f32"), 5, "f32") == 256 + a256(100 * 4 * 5)
+    assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 100, 3], "f32"), 5, "f32") == \
+        256 + a256(100 * 4 * 5) + f32tc([13, 100, 3], 5)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), -1, "f32") == 0
 
 
