@@ -432,8 +432,12 @@ def run_ours(args, cfg, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, dt, cores, used = calibrated_oracle(cfg, batches[0], args.cpu_seconds)
+        r1, dt1, c1, used1 = oracle_on_one_core(cfg, batches[0], args.cpu_seconds / 3)
         cpu = {"value": rate, "unit": "samples/s", "cores": cores, "kind": "oracle",
-               "sample": f"{used} random samples of batch 0, fp64 forward in {dt:.1f} s"}
+               "sample": f"{used} random samples of batch 0, fp64 forward in {dt:.1f} s",
+               "cpu_model": cpu_model(),
+               "one_core": {"value": r1, "cores": c1,
+                            "sample": f"{used1} random samples of batch 0, fp64 forward in {dt1:.1f} s"}}
 
     if rank == 0:
         traffic = kernel_traffic(*TRAFFIC[cfg.name]) if cfg.name in TRAFFIC else None
