@@ -204,6 +204,35 @@ __device__ __forceinline__ void pool_tile(const T* __restrict__ tables, const Ta
     }
 }
 
+// Pool every bag of the tile, one bag per work item: items (table k, sample s) are taken from a shared
+// counter by lane groups, so that long and short bags even out across the groups, with U rows in flight
+// per lane. The counter (shared, zeroed before the block's first __syncthreads) is consumed.
+template <typename T, bool VEC, int NCH, int U, typename MakeSink>
+__device__ __forceinline__ void pool_items(const T* __restrict__ tables, const TableMeta& tm, int K, int d, int n_ch,
+                                           int GL, const int32_t* __restrict__ indices, const int* off_s,
+                                           const unsigned char* bad_s, int S, int nb, unsigned& oob,
+                                           MakeSink make_sink, int* counter) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane & (GL - 1);
+    const int leader = lane & ~(GL - 1);
+    const unsigned gmask = GL == 32 ? 0xffffffffu : ((1u << GL) - 1u) << leader;
+    const int n_items = K * nb;
+    for (;;) {
+        int it = 0;
+        if (g == 0) it = atomicAdd(counter, 1);
+        it = __shfl_sync(gmask, it, leader);
+        if (it >= n_items) break;
+        const int k = it / nb, s = it - k * nb;
+        const T* table = tables + tm.base[k] * (long long)d;
+        auto sink = make_sink(k, s, g);
+        const bool isbad = bad_s[k * S + s];
+        int one[2];
+        one[0] = isbad ? 0 : off_s[k * (S + 1) + s];
+        one[1] = isbad ? 0 : off_s[k * (S + 1) + s + 1];
+        walk_bags<T, VEC, NCH, U>(table, tm.rows[k], d, n_ch, indices, one, 1, g, GL, oob, sink);
+    }
+}
+
 // ------------------------------------------------------------------ K1: pooling only
 
 template <typename T, bool VEC, int NCH>
@@ -381,15 +410,18 @@ __global__ void __launch_bounds__(256) embbag_interact_kernel(
     float* X = reinterpret_cast<float*>(smem);
     int* off_s = reinterpret_cast<int*>(smem + sizeof(float) * (size_t)S * n1 * xs);
     unsigned char* bad_s = reinterpret_cast<unsigned char*>(off_s + K * (S + 1));
+    int* counter = reinterpret_cast<int*>(bad_s + (((size_t)K * S + 3) & ~(size_t)3));
     const int b0 = blockIdx.x * S;
     const int nb = min(S, B - b0);
     unsigned oob = 0, bad = 0;
+    if (threadIdx.x == 0) *counter = 0;
     load_dense_rows(x_dense, d, b0, nb, X, xs, n1);
     load_tile_offsets(offsets, B, K, b0, nb, S, nnz, off_s, bad_s, nullptr, bad);
     auto make_sink = [&](int k, int s0, int g) {
         return RowSink<T, VEC, NCH>{X + ((long long)s0 * n1 + 1 + k) * xs, (long long)n1 * xs, g, GL, n_ch};
     };
-    pool_tile<T, VEC, NCH, 4>(tables, tm, K, d, n_ch, GL, indices, off_s, bad_s, S, nb, oob, make_sink);
+    constexpr int U = NCH >= 4 ? 2 : (NCH == 2 ? 4 : 8);
+    pool_items<T, VEC, NCH, U>(tables, tm, K, d, n_ch, GL, indices, off_s, bad_s, S, nb, oob, make_sink, counter);
     __syncthreads();
     interact_tile(X, xs, K, d, nb, b0, out, ld, out_dt);
     report_warp(err, oob, bad);
@@ -499,9 +531,12 @@ static dlrm_status launch_fused_t(const TableMeta& tm, const void* tables, int K
                                   const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                   cudaStream_t st, const Geometry& g) {
     const size_t per = interact_smem_per_sample(K, d);
-    const auto extra = [&](int S) { return sizeof(int) * (size_t)K * (S + 1) + (size_t)K * S; };
+    const auto extra = [&](int S) { return sizeof(int) * (size_t)K * (S + 1) + (((size_t)K * S + 3) & ~(size_t)3) + 16; };
     int S = (int)(kSmemBudget / per);
     S = S < 1 ? 1 : (S > 8 ? 8 : S);
+    // enough blocks for about four per SM, so that small batches still spread over the GPU
+    const int s_fill = B / (148 * 4);
+    if (s_fill < S) S = s_fill < 1 ? 1 : s_fill;
     while (S > 1 && per * S + extra(S) > kSmemMax) --S;
     const size_t smem = per * S + extra(S);
     if (smem > kSmemMax) return DLRM_ERR_UNSUPPORTED;
