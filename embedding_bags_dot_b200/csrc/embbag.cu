@@ -74,11 +74,15 @@ __device__ __forceinline__ void walk_bags(const T* __restrict__ table, long long
     int p = off[0];
     const int pend = off[nb];
     int bag_end = off[1];
+    int idx[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) idx[u] = (p + u < pend) ? __ldg(indices + p + u) : -1;
     while (p < pend) {
         const int n = min(U, pend - p);
-        int idx[U];
+        // the next step's indices are loaded while this step's rows are in flight
+        int nxt[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) idx[u] = (u < n) ? __ldg(indices + p + u) : -1;
+        for (int u = 0; u < U; ++u) nxt[u] = (p + n + u < pend) ? __ldg(indices + p + n + u) : -1;
         LdT<T, VEC> v[U][NCH];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -108,6 +112,8 @@ __device__ __forceinline__ void walk_bags(const T* __restrict__ table, long long
             }
         }
         p += n;
+#pragma unroll
+        for (int u = 0; u < U; ++u) idx[u] = nxt[u];
     }
     while (s < nb) {
         sink(s, acc);

@@ -36,6 +36,7 @@ namespace {
 using namespace ac;
 
 constexpr int WW = 8;                 // warps per block
+constexpr int NC = 2;                 // 16-column blocks of the Gram accumulated at a time per m-tile
 constexpr unsigned FULLW = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t pack_bf16w(float lo, float hi) {
@@ -84,7 +85,7 @@ __host__ __device__ inline WideLayout wide_layout(int d, int MT, int ld) {
 
 // GL: lanes per row (d = 8 GL); MT: 16-row m-tiles of the e tile (16 MT >= K); U: rows in flight per lane.
 template <int GL, int MT, int U>
-__global__ void __launch_bounds__(WW * 32, 2) embbag_interact_wide_kernel(
+__global__ void __launch_bounds__(WW * 32, 3) embbag_interact_wide_kernel(
     const __nv_bfloat16* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B, int S,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, __nv_bfloat16* __restrict__ out, int ld, ErrRecord* err) {
@@ -141,10 +142,14 @@ __global__ void __launch_bounds__(WW * 32, 2) embbag_interact_wide_kernel(
         } else {
             const __nv_bfloat16* tab = tables + tm.base[k] * (long long)d + 8 * g;
             const long long m = tm.rows[k];
-            for (long long p = st; p < en; p += U) {
-                int idx[U];
+            // the next U indices are loaded while this step's rows are in flight
+            int idx[U];
 #pragma unroll
-                for (int u = 0; u < U; ++u) idx[u] = p + u < en ? __ldg(indices + p + u) : -1;
+            for (int u = 0; u < U; ++u) idx[u] = st + u < en ? __ldg(indices + st + u) : -1;
+            for (long long p = st; p < en; p += U) {
+                int nxt[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) nxt[u] = p + U + u < en ? __ldg(indices + p + U + u) : -1;
                 uint4 v[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -154,6 +159,8 @@ __global__ void __launch_bounds__(WW * 32, 2) embbag_interact_wide_kernel(
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) Chunk16<__nv_bfloat16>::add(v[u], acc);
+#pragma unroll
+                for (int u = 0; u < U; ++u) idx[u] = nxt[u];
             }
         }
         *reinterpret_cast<uint4*>(tile_of(s) + k * L.RS + 16 * g) =
@@ -173,41 +180,50 @@ __global__ void __launch_bounds__(WW * 32, 2) embbag_interact_wide_kernel(
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
             if (mt % WPS != wsub || 16 * mt >= K) continue;
-            float acc[2 * MT][4];
-            float ax[4] = {0.f, 0.f, 0.f, 0.f};
+            // the lower-triangle n8 tiles of this m-tile in chunks of NC 16-column blocks (few accumulators
+            // live at a time), the x tile with the first chunk
 #pragma unroll
-            for (int t = 0; t < 2 * mt + 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+            for (int c0 = 0; c0 <= mt; c0 += NC) {
+                float acc[2 * NC][4];
+                float ax[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < d / 16; ++ks) {
-                uint32_t a[4];
-                ldmatrix_x4(tile_s + (uint32_t)((16 * mt + (lane & 15)) * L.RS + 16 * (2 * ks + (lane >> 4))), a);
+                for (int t = 0; t < 2 * NC; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 #pragma unroll
-                for (int n2 = 0; n2 <= mt; ++n2) {
-                    uint32_t b[4];
-                    if (n2 == mt) {
-                        b[0] = a[0]; b[1] = a[1]; b[2] = a[2]; b[3] = a[3];
-                    } else {
-                        ldmatrix_x4(tile_s + (uint32_t)((16 * n2 + (lane & 15)) * L.RS + 16 * (2 * ks + (lane >> 4))), b);
+                for (int ks = 0; ks < d / 16; ++ks) {
+                    uint32_t a[4];
+                    ldmatrix_x4(tile_s + (uint32_t)((16 * mt + (lane & 15)) * L.RS + 16 * (2 * ks + (lane >> 4))), a);
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) {
+                        const int n2 = c0 + j;
+                        if (n2 > mt) break;
+                        uint32_t b[4];
+                        if (n2 == mt) {
+                            b[0] = a[0]; b[1] = a[1]; b[2] = a[2]; b[3] = a[3];
+                        } else {
+                            ldmatrix_x4(tile_s + (uint32_t)((16 * n2 + (lane & 15)) * L.RS + 16 * (2 * ks + (lane >> 4))), b);
+                        }
+                        mma_bf16w(acc[2 * j], a, b[0], b[2]);
+                        mma_bf16w(acc[2 * j + 1], a, b[1], b[3]);
                     }
-                    mma_bf16w(acc[2 * n2], a, b[0], b[2]);
-                    mma_bf16w(acc[2 * n2 + 1], a, b[1], b[3]);
+                    if (c0 == 0) {
+                        uint32_t x0, x1;
+                        ldmatrix_x2(xt_s + (uint32_t)((lane & 7) * L.RS + 16 * (2 * ks + ((lane >> 3) & 1))), x0, x1);
+                        mma_bf16w(ax, a, x0, x1);
+                    }
                 }
-                uint32_t x0, x1;
-                ldmatrix_x2(xt_s + (uint32_t)((lane & 7) * L.RS + 16 * (2 * ks + ((lane >> 3) & 1))), x0, x1);
-                mma_bf16w(ax, a, x0, x1);
-            }
-            // rows r = 16 mt + gr (+ 8) hold e_{r+1}: Z_{r+1, c+1} for c < r, and Z_{r+1, 0}
+                // rows r = 16 mt + gr (+ 8) hold e_{r+1}: Z_{r+1, c+1} for c < r, and (first chunk) Z_{r+1, 0}
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = 16 * mt + gr + 8 * h;
-                if (r >= K) continue;
-                const int base = d + (r + 1) * r / 2;          // concat column of Z_{r+1, 0}
-                if (tc == 0) orow[base] = __float2bfloat16_rn(ax[2 * h] + ax[2 * h + 1]);
+                for (int h = 0; h < 2; ++h) {
+                    const int r = 16 * mt + gr + 8 * h;
+                    if (r >= K) continue;
+                    const int base = d + (r + 1) * r / 2;          // concat column of Z_{r+1, 0}
+                    if (c0 == 0 && tc == 0) orow[base] = __float2bfloat16_rn(ax[2 * h] + ax[2 * h + 1]);
 #pragma unroll
-                for (int t = 0; t < 2 * mt + 2; ++t) {
-                    const int c = 8 * t + tc;
-                    if (c < r) orow[base + 1 + c] = __float2bfloat16_rn(acc[t][2 * h]);
-                    if (c + 1 < r) orow[base + 2 + c] = __float2bfloat16_rn(acc[t][2 * h + 1]);
+                    for (int t = 0; t < 2 * NC; ++t) {
+                        const int c = 16 * c0 + 8 * t + tc;
+                        if (c < r) orow[base + 1 + c] = __float2bfloat16_rn(acc[t][2 * h]);
+                        if (c + 1 < r) orow[base + 2 + c] = __float2bfloat16_rn(acc[t][2 * h + 1]);
+                    }
                 }
             }
         }
@@ -230,10 +246,13 @@ static size_t wide_smem(int d, int MT, int ld, int S) {
     return (size_t)S * wide_layout(d, MT, ld).per_sample + 16;
 }
 
-// Samples per block: 4 when two blocks fit an SM, else 2, else 1 (0: does not fit).
+// Samples per block: the most that still lets three blocks share an SM (the register budget allows three),
+// else the most that let two, else 1
+// (0: does not fit).
 static int wide_samples(int d, int MT, int ld) {
-    for (int S : {4, 2})
-        if (2 * wide_smem(d, MT, ld, S) <= 228 * 1024 - 2048) return S;
+    for (int blocks : {3, 2})
+        for (int S : {4, 2, 1})
+            if ((size_t)blocks * (wide_smem(d, MT, ld, S) + 1024) <= 228 * 1024) return S;
     return wide_smem(d, MT, ld, 1) <= 227 * 1024 ? 1 : 0;
 }
 
