@@ -259,6 +259,7 @@ uint64_t dlrm_launch_count(void) { return g_launches.load(std::memory_order_rela
 
 dlrm_status dlrm_set_wait_polls(int64_t polls) {
     if (set_wait_polls_gemm_tc(polls) != cudaSuccess || set_wait_polls_embbag_mma(polls) != cudaSuccess ||
+        set_wait_polls_embbag_pipe(polls) != cudaSuccess ||
         set_wait_polls_embbag_cat(polls) != cudaSuccess || set_wait_polls_interact_tc(polls) != cudaSuccess)
         return DLRM_ERR_CUDA;
     return DLRM_OK;

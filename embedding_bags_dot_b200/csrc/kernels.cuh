@@ -35,6 +35,14 @@ dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, 
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st);
+// bf16 tables into a bf16 concat, K + 2 <= 64: persistent warps, next sample's rows in flight during this one's
+// Gram and store, Z written from the accumulators, one bulk store per row.
+bool embbag_interact_pipe_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
+                                    long long total_rows);
+dlrm_status launch_embbag_interact_pipe(const TableMeta& tm, const void* tables, int K, int d, int B,
+                                        const int32_t* offsets, const int32_t* indices, long long nnz,
+                                        const float* x_dense, void* out, int ld, ErrRecord* err, cudaStream_t st);
+cudaError_t set_wait_polls_embbag_pipe(long long polls);
 // Many tables (K up to 128, bf16 tables and concat, d = 64 or 128): U-deep row gather and mma.sync Gram.
 bool embbag_interact_wide_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt);
 dlrm_status launch_embbag_interact_wide(const TableMeta& tm, const void* tables, int K, int d, int B,
