@@ -79,15 +79,19 @@ template <typename T> struct Chunk16;
 template <> struct Chunk16<float> {
     static constexpr int E = 4;
     static __device__ __forceinline__ void add(const uint4& v, float* a) {
-        a[0] += __uint_as_float(v.x); a[1] += __uint_as_float(v.y);
-        a[2] += __uint_as_float(v.z); a[3] += __uint_as_float(v.w);
+        const float2 lo = __fadd2_rn(make_float2(a[0], a[1]), make_float2(__uint_as_float(v.x), __uint_as_float(v.y)));
+        const float2 hi = __fadd2_rn(make_float2(a[2], a[3]), make_float2(__uint_as_float(v.z), __uint_as_float(v.w)));
+        a[0] = lo.x; a[1] = lo.y; a[2] = hi.x; a[3] = hi.y;
     }
 };
 template <> struct Chunk16<__nv_bfloat16> {
     static constexpr int E = 8;
     static __device__ __forceinline__ void add2(unsigned w, float* a) {
-        a[0] += __uint_as_float(w << 16);
-        a[1] += __uint_as_float(w & 0xffff0000u);
+        // both halves widened exactly, then one packed two-lane fp32 add (round to nearest)
+        const float2 s = __fadd2_rn(make_float2(a[0], a[1]),
+                                    make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
+        a[0] = s.x;
+        a[1] = s.y;
     }
     static __device__ __forceinline__ void add(const uint4& v, float* a) {
         add2(v.x, a); add2(v.y, a + 2); add2(v.z, a + 4); add2(v.w, a + 6);

@@ -148,14 +148,24 @@ __global__ void __launch_bounds__(WW * 32, 3) embbag_interact_wide_kernel(
             for (int u = 0; u < U; ++u) idx[u] = st + u < en ? __ldg(indices + st + u) : -1;
             for (long long p = st; p < en; p += U) {
                 int nxt[U];
+                if (p + 2 * U <= en) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) nxt[u] = p + U + u < en ? __ldg(indices + p + U + u) : -1;
+                    for (int u = 0; u < U; ++u) nxt[u] = __ldg(indices + p + U + u);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) nxt[u] = p + U + u < en ? __ldg(indices + p + U + u) : -1;
+                }
                 uint4 v[U];
+                unsigned okm = 0;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const bool ok = idx[u] >= 0 && (long long)idx[u] < m;
-                    if (g == 0 && p + u < en && !ok) ++oob;
+                    const bool ok = (unsigned long long)(unsigned)idx[u] < (unsigned long long)m;   // -1: past the bag
+                    okm |= (unsigned)ok << u;
                     v[u] = ok ? ldg16_stream(tab + (long long)idx[u] * d) : make_uint4(0, 0, 0, 0);
+                }
+                if (g == 0) {   // indices of the bag that are out of range (not the slots past its end)
+                    const int n = en - p < U ? (int)(en - p) : U;
+                    oob += __popc(~okm & ((1u << n) - 1u));
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) Chunk16<__nv_bfloat16>::add(v[u], acc);
