@@ -100,8 +100,8 @@ F32TcWs f32tc_ws(const dlrm_mlp* m, int B) {
         widest = std::max(widest, m->dims[l + 1]);
         widest_in = std::max(widest_in, m->dims[l]);
     }
-    W.ld_in = dlrm_ld(widest_in, DLRM_F32);   // the split input, or any layer's input merged back to plain
-    W.ld_act = dlrm_ld(widest, DLRM_F32);
+    W.ld_in = dlrm_ld(std::max(widest_in, widest), DLRM_F32);   // plain buffers: any layer's input or output
+    W.ld_act = W.ld_in;                                            // pair buffers: likewise
     for (int h = 0; h < 2; ++h) W.in[h] = take(sizeof(float) * (size_t)B * W.ld_in);
     for (int p = 0; p < 2; ++p)
         for (int h = 0; h < 2; ++h) W.act[p][h] = take(sizeof(float) * (size_t)B * W.ld_act);
@@ -162,45 +162,59 @@ FwdLayout fwd_layout(const dlrm_tables* T, const dlrm_mlp* bot, const dlrm_mlp* 
 // The MLP chain: ReLU after hidden layers, final_act after the last layer. An fp32 input
 // to a 16-bit MLP is first converted (into cvt) so that every layer can take the
 // tensor-core path.
-// A layer of an fp32 MLP goes to the 3xTF32 tensor-core GEMM when the output is wide enough to fill its
-// tiles and the batch fills the GPU; the first bottom layer (13 inputs) and one-column layers stay on the
-// CUDA cores.
-bool f32_layer_on_tc(int M, int N, int K) { return M >= 1024 && N >= 16 && K > 16; }
+// A layer of an fp32 MLP goes to the 3xTF32 tensor-core GEMM (256x256 tiles on SM pairs) when the batch
+// gives it enough tiles to be worth the pair conversions: at 2,048 rows (the medium configuration) the
+// CUDA-core layers measured faster in total. The 13-wide first bottom layer stays on the CUDA cores.
+bool f32_layer_on_tc(int M, int N, int K) { return M >= 4096 && N >= 64 && K > 16; }
 
-// fp32 MLP: hidden layers as (hi, lo) pairs in the tensor-core buffers at `tc` (F32TcWs layout); a layer
-// that stays on the CUDA cores reads and writes the same pairs; the last layer writes `out` plain.
+// fp32 MLP with tensor-core layers: buffers in `tc` (F32TcWs layout): two (hi, lo) pair buffers for the
+// tensor-core layers' inputs and outputs, two plain buffers for the CUDA-core layers'. A tensor-core layer
+// takes a pair (a plain input is split first), a CUDA-core layer a plain input (a pair is merged first);
+// the last layer writes `out` plain.
 dlrm_status run_mlp_f32(const dlrm_mlp* m, int B, const float* in, int ld_in, float* out, int ld_out, int final_act,
                         char* tc, ErrRecord* err, cudaStream_t st) {
     const F32TcWs W = f32tc_ws(m, B);
     auto F = [&](size_t o) { return reinterpret_cast<float*>(tc + o); };
+    float* pairs[2][2] = {{F(W.act[0][0]), F(W.act[0][1])}, {F(W.act[1][0]), F(W.act[1][1])}};
+    float* plain[2] = {F(W.in[0]), F(W.in[1])};
     dlrm_status r;
+    // cur: the layer input; where = 0/1 for pair buffer 0/1, 2/3 for plain buffer 0/1, -1 for the caller's input
     F32Pair cur{in, nullptr, ld_in};
+    int where = -1;
     for (int l = 0; l < m->n_layers; ++l) {
         const int K = m->dims[l], N = m->dims[l + 1], ldw = dlrm_ld(K, DLRM_F32);
         const bool last = l == m->n_layers - 1;
-        const bool use_tc = f32_layer_on_tc(B, N, K) && (!last || final_act == DLRM_ACT_RELU);
-        if (!use_tc && last) {
-            // plain input for the CUDA-core layer (and its activation): merge a pair first
-            if (cur.lo) {
-                if ((r = launch_merge_pair(B, K, cur.hi, cur.lo, cur.ld, F(W.in[0]), W.ld_in, st))) return r;
-                cur = F32Pair{F(W.in[0]), nullptr, W.ld_in};
+        if (!(f32_layer_on_tc(B, N, K) && (!last || final_act == DLRM_ACT_RELU))) {
+            if (cur.lo) {                       // merge the pair into a plain buffer
+                if ((r = launch_merge_pair(B, K, cur.hi, cur.lo, cur.ld, plain[0], W.ld_in, st))) return r;
+                cur = F32Pair{plain[0], nullptr, W.ld_in};
+                where = 2;
             }
-            return launch_linear(B, N, K, cur.hi, DLRM_F32, cur.ld, m->W[l], DLRM_F32, ldw, m->b[l], out, DLRM_F32,
-                                 ld_out, final_act, err, st);
+            if (last)
+                return launch_linear(B, N, K, cur.hi, DLRM_F32, cur.ld, m->W[l], DLRM_F32, ldw, m->b[l], out, DLRM_F32,
+                                     ld_out, final_act, err, st);
+            const int dst = where == 2 ? 1 : 0;
+            if ((r = launch_linear(B, N, K, cur.hi, DLRM_F32, cur.ld, m->W[l], DLRM_F32, ldw, m->b[l], plain[dst],
+                                   DLRM_F32, W.ld_in, DLRM_ACT_RELU, err, st)))
+                return r;
+            cur = F32Pair{plain[dst], nullptr, W.ld_in};
+            where = 2 + dst;
+            continue;
         }
-        const F32Pair Wp{F(W.w[l][0]), F(W.w[l][1]), ldw};
+        if (!cur.lo) {                          // split the plain input into a pair buffer
+            if ((r = launch_split_pair(B, K, cur.hi, cur.ld, pairs[0][0], pairs[0][1], W.ld_act, st))) return r;
+            cur = F32Pair{pairs[0][0], pairs[0][1], W.ld_act};
+            where = 0;
+        }
         if ((r = launch_split_pair(N, K, static_cast<const float*>(m->W[l]), ldw, F(W.w[l][0]), F(W.w[l][1]), ldw, st)))
             return r;
-        if (use_tc && !cur.lo) {
-            if ((r = launch_split_pair(B, K, cur.hi, cur.ld, F(W.in[0]), F(W.in[1]), W.ld_in, st))) return r;
-            cur = F32Pair{F(W.in[0]), F(W.in[1]), W.ld_in};
-        }
-        const int p = l & 1;
-        float* yh = F(W.act[p][0]);
-        float* yl = F(W.act[p][1]);
-        if ((r = train_linear_fwd(B, N, K, cur, Wp, m->b[l], yh, yl, W.ld_act, true, nullptr, err, st))) return r;
-        cur = F32Pair{yh, yl, W.ld_act};
-        if (last) return launch_merge_pair(B, N, yh, yl, W.ld_act, out, ld_out, st);
+        const int dst = where == 0 ? 1 : 0;
+        if ((r = train_linear_fwd(B, N, K, cur, F32Pair{F(W.w[l][0]), F(W.w[l][1]), ldw}, m->b[l], pairs[dst][0],
+                                  pairs[dst][1], W.ld_act, true, nullptr, err, st)))
+            return r;
+        cur = F32Pair{pairs[dst][0], pairs[dst][1], W.ld_act};
+        where = dst;
+        if (last) return launch_merge_pair(B, N, cur.hi, cur.lo, cur.ld, out, ld_out, st);
     }
     return DLRM_OK;
 }

@@ -111,7 +111,7 @@ def test_mlp_workspace_size_follows_the_documented_layout(lib):
         """fp32 MLPs add their 3xTF32 pair buffers: split weights, split input, two hidden pair buffers."""
         ldf = lambda n: (n + 3) // 4 * 4  # noqa: E731
         w = sum(2 * a256(4 * dims[l + 1] * ldf(dims[l])) for l in range(len(dims) - 1))
-        return w + 2 * a256(4 * B * ldf(max(dims[:-1]))) + 4 * a256(4 * B * ldf(max(dims[1:])))
+        return w + 6 * a256(4 * B * ldf(max(dims)))
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "f32"), B, "f32") == 256 + f32tc([13, 64], B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 64], "bf16"), B, "f32") == 256 + a256(16 * 2 * B)
     assert E.dlrm_mlp_workspace_size(_cpu_mlp([13, 512, 128], "bf16"), B, "f32") == 256 + a256(512 * 2 * B) + a256(16 * 2 * B)

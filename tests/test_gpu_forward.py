@@ -20,7 +20,7 @@ def _cases():
         "tiny-ragged-mix": shrink(t, B=203).with_(bag="mix", seed=1),
         "medium-small": shrink(m, B=197, rows_cap=5000),
         # a batch large enough for the fp32 MLP layers to run on the tensor cores (3xTF32 pairs)
-        "medium-b1536": shrink(m, B=1536, rows_cap=800).with_(seed=4),
+        "medium-b4200": shrink(m, B=4200, rows_cap=300).with_(seed=4, bag="fixed:3"),
         "large-small": shrink(l, B=261, rows_cap=20000),
         "large-batch3": shrink(l, B=3, rows_cap=2000),          # serving-size batch: small-batch layer kernel
         "stress-small": shrink(s, B=37, rows_cap=3000).with_(bag="uniform100"),
@@ -131,7 +131,7 @@ def test_embbag_interact_fwd(name):
     assert np.all(got[:, want.shape[1]:] == 0.0)
 
 
-@pytest.mark.parametrize("name", ["tiny", "medium-small", "medium-b1536", "large-small", "stress-small", "f16-d64-mix"])
+@pytest.mark.parametrize("name", ["tiny", "medium-small", "medium-b4200", "large-small", "stress-small", "f16-d64-mix"])
 def test_mlp_fwd(name):
     cfg = CASES[name]
     g = GpuModel(cfg)
