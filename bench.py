@@ -81,8 +81,6 @@ def fused_kernel_name(cfg) -> str:
     """The gather + interaction kernel the library dispatches to for this workload."""
     if cfg.interaction == "cat":
         return "embbag_cat_bulk_kernel (dlrm_embbag_cat_fwd)"
-    if cfg.table_dtype == "bf16" and cfg.mlp_dtype == "bf16" and cfg.K + 2 <= 64 and cfg.d in (32, 64, 128, 256):
-        return "embbag_interact_pipe_kernel (dlrm_embbag_interact_fwd)"
     if cfg.table_dtype in ("bf16", "u8row") and cfg.K + (4 if cfg.table_dtype == "u8row" else 2) <= 64:
         return "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
     if cfg.table_dtype == "bf16" and cfg.mlp_dtype == "bf16" and cfg.d in (64, 128) and cfg.K <= 128:
@@ -100,7 +98,7 @@ def read_peaks():
 
 
 # the files the fused gather + interaction kernel is compiled from (its traffic record is keyed on them)
-K2_SOURCES = ("embedding_bags_dot_b200/csrc/embbag_pipe.cu", "embedding_bags_dot_b200/csrc/async_copy.cuh",
+K2_SOURCES = ("embedding_bags_dot_b200/csrc/embbag_mma.cu", "embedding_bags_dot_b200/csrc/async_copy.cuh",
               "embedding_bags_dot_b200/csrc/common.cuh")
 CAT_SOURCES = ("embedding_bags_dot_b200/csrc/embbag_cat_bulk.cu", "embedding_bags_dot_b200/csrc/async_copy.cuh",
                "embedding_bags_dot_b200/csrc/common.cuh")

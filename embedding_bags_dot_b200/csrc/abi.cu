@@ -228,6 +228,9 @@ dlrm_status run_mlp(const dlrm_mlp* m, int B, const void* in, dlrm_dtype in_dt, 
         if (any)
             return run_mlp_f32(m, B, static_cast<const float*>(in), ld_in, out, ld_out, final_act, f32tc, err, st);
     }
+    // three bf16 layers from fp32 input (the bottom MLP): one kernel, the hidden activations never in HBM
+    if (mlp3_tc_supported(m, B, in_dt, ld_in, out, ld_out, final_act))
+        return launch_mlp3_tc(m, B, static_cast<const float*>(in), ld_in, out, ld_out, err, st);
     const void* cur = in;
     dlrm_dtype cur_dt = in_dt;
     int cur_ld = ld_in;
@@ -273,7 +276,7 @@ uint64_t dlrm_launch_count(void) { return g_launches.load(std::memory_order_rela
 
 dlrm_status dlrm_set_wait_polls(int64_t polls) {
     if (set_wait_polls_gemm_tc(polls) != cudaSuccess || set_wait_polls_embbag_mma(polls) != cudaSuccess ||
-        set_wait_polls_embbag_pipe(polls) != cudaSuccess ||
+        set_wait_polls_mlp3(polls) != cudaSuccess ||
         set_wait_polls_embbag_cat(polls) != cudaSuccess || set_wait_polls_interact_tc(polls) != cudaSuccess)
         return DLRM_ERR_CUDA;
     return DLRM_OK;

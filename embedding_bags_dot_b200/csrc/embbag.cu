@@ -570,8 +570,6 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                    const int32_t* offsets, const int32_t* indices, long long nnz,
                                    const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                    cudaStream_t st) {
-    if (embbag_interact_pipe_supported(dt, K, d, ld, out, out_dt, tm.base[K - 1] + tm.rows[K - 1]))
-        return launch_embbag_interact_pipe(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st);
     if (embbag_interact_mma_supported(dt, K, d, ld, out, out_dt, tm.base[K - 1] + tm.rows[K - 1]))
         return launch_embbag_interact_mma(tm, tables, dt, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt,
                                           err, st);

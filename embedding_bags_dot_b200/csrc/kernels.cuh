@@ -35,14 +35,6 @@ dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, 
                                        const int32_t* offsets, const int32_t* indices, long long nnz,
                                        const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
                                        cudaStream_t st);
-// bf16 tables into a bf16 concat, K + 2 <= 64: persistent warps, next sample's rows in flight during this one's
-// Gram and store, Z written from the accumulators, one bulk store per row.
-bool embbag_interact_pipe_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt,
-                                    long long total_rows);
-dlrm_status launch_embbag_interact_pipe(const TableMeta& tm, const void* tables, int K, int d, int B,
-                                        const int32_t* offsets, const int32_t* indices, long long nnz,
-                                        const float* x_dense, void* out, int ld, ErrRecord* err, cudaStream_t st);
-cudaError_t set_wait_polls_embbag_pipe(long long polls);
 // Many tables (K up to 128, bf16 tables and concat, d = 64 or 128): U-deep row gather and mma.sync Gram.
 bool embbag_interact_wide_supported(dlrm_dtype dt, int K, int d, int ld, const void* out, dlrm_dtype out_dt);
 dlrm_status launch_embbag_interact_wide(const TableMeta& tm, const void* tables, int K, int d, int B,
@@ -56,6 +48,15 @@ dlrm_status launch_embbag_interact_wide(const TableMeta& tm, const void* tables,
 dlrm_status launch_linear(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
                           dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act,
                           ErrRecord* err, cudaStream_t st);
+
+// Three bf16 layers in one tensor-core kernel (mlp3_tc.cu): fp32 input [B][ld_in] with dims[0] <= 16,
+// h1 and h2 kept on chip, fp32 ReLU output [B][ld_out]; dims[1] <= 512, dims[2] <= 256, dims[3] <= 128, each a
+// multiple of 64.
+bool mlp3_tc_supported(const dlrm_mlp* m, int B, dlrm_dtype in_dt, int ld_in, const void* out, int ld_out,
+                       int final_act);
+dlrm_status launch_mlp3_tc(const dlrm_mlp* m, int B, const float* in, int ld_in, float* out, int ld_out, ErrRecord* err,
+                           cudaStream_t st);
+cudaError_t set_wait_polls_mlp3(long long polls);
 
 // out[b][c] = in[b][c] (converted) for c < K, zero up to ldo.
 // offsets[i] = sum of lengths[0..i) for i <= n, uint8 lengths (lengths.cu); scratch: lengths_scratch_ints(n) ints.

@@ -117,8 +117,9 @@ uint64_t dlrm_launch_count(void);
 
 /* Test hook, no counterpart in the pages: sets, on the current device, how
  * many times the first bounded wait of the row-gathering kernels (the bulk
- * copies of a sample's rows) and the ordinary waits of the single-CTA
- * tensor-core layer (batches below 4,096 rows) poll before giving up;
+ * copies of a sample's rows), the ordinary waits of the single-CTA
+ * tensor-core layer (batches below 4,096 rows) and those of the one-kernel
+ * three-layer MLP (the bf16 bottom MLP) poll before giving up;
  * polls < 0 restores the defaults (about a second). A test sets 0 to make
  * those waits run out at once and checks that the call returns, that
  * dlrm_check_error reports DLRM_ERR_TIMEOUT, and that the next call (after
@@ -178,7 +179,12 @@ dlrm_status dlrm_embbag_interact_fwd(const dlrm_tables* T, int B, const int32_t*
  *   ws    16-byte aligned, ws_bytes >= dlrm_mlp_workspace_size(mlp, B, in_dt)
  *         (dlrm_workspace_size of a model with this MLP as top or bottom is
  *         enough); the hidden activations live there. A smaller ws_bytes is
- *         refused with DLRM_ERR_WORKSPACE before any launch. */
+ *         refused with DLRM_ERR_WORKSPACE before any launch.
+ * Three bf16 layers on fp32 input with final_act ReLU (the bottom MLP), with
+ * dims[0] <= 16 and dims[1..3] multiples of 64 up to 512 / 256 / 128, run as
+ * one kernel whose hidden activations stay on chip (same roundings: input and
+ * hidden outputs to bf16, fp32 accumulation). Padding columns of a weight row
+ * (between dims[l] and its leading dimension) are never read there. */
 dlrm_status dlrm_mlp_fwd(const dlrm_mlp* mlp, int B, const void* in, dlrm_dtype in_dt, int ld_in,
                          float* out, int ld_out, int final_act, void* ws, size_t ws_bytes, dlrm_stream stream);
 

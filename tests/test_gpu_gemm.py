@@ -101,7 +101,7 @@ def test_linear_small_batch(M, N, K, dt):
 
 # the bottom-MLP shape (13 dense features -> 512 -> 256 -> N3) through dlrm_mlp_fwd, many batch sizes
 @pytest.mark.parametrize("B", [1, 127, 300, 1000, 20000])
-@pytest.mark.parametrize("dt,n3", [("bf16", 128), ("f16", 64), ("bf16", 256)])
+@pytest.mark.parametrize("dt,n3", [("bf16", 128), ("f16", 64), ("bf16", 256), ("bf16", 64)])
 def test_fused_bottom_mlp(B, dt, n3):
     g = torch.Generator().manual_seed(B + n3)
     dims = [13, 512, 256, n3]
@@ -123,6 +123,37 @@ def test_fused_bottom_mlp(B, dt, n3):
     assert E.dlrm_check_error(ws)[0] == 0
     want = O.mlp(Ws, bs, x.double().numpy(), relu_last=True)
     assert_close(to_np(out), want, "bf16", f"fused bottom MLP B={B} {dt} N3={n3}", scale_mlp(Ws, bs, x.double().numpy()))
+
+
+# three bf16 layers from fp32 input run as one kernel (h1, h2 kept on chip) for widths that are multiples of 64
+# up to 512 / 256 / 128 and up to 16 inputs: other widths, ragged batches, a K below 16
+@pytest.mark.parametrize("dims", [(13, 192, 128, 64), (7, 64, 64, 128), (16, 512, 64, 64), (1, 448, 192, 128)])
+@pytest.mark.parametrize("B", [1, 129, 4999])
+def test_three_layer_mlp_one_kernel(dims, B):
+    g = torch.Generator().manual_seed(B * 5 + dims[1])
+    Ws, bs, Wd, bd = [], [], [], []
+    for l in range(3):
+        K, N = dims[l], dims[l + 1]
+        W = torch.zeros((N, E.dlrm_ld(K, "bf16")), dtype=torch.bfloat16)
+        W[:, :K] = (torch.randn((N, K), generator=g) * np.sqrt(2.0 / K)).bfloat16()
+        if K % 8:
+            W[:, K:] = float("nan")    # row padding is never read as a weight
+        b = torch.randn(N, generator=g) * 0.1
+        Ws.append(W[:, :K].double().numpy())
+        bs.append(b.double().numpy())
+        Wd.append(W.cuda())
+        bd.append(b.cuda())
+    x = torch.randn((B, dims[0]), generator=g)
+    mlp = E.MLP(Wd, bd, list(dims))
+    out = torch.full((B, dims[3]), float("nan"), device="cuda")
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, x.dtype))
+    n0 = E.dlrm_launch_count()
+    E.dlrm_mlp_fwd(mlp, B, x.cuda(), dims[0], out, dims[3], E.ACT_RELU, ws)
+    assert E.dlrm_launch_count() - n0 == 1, "three layers, one launch"
+    assert E.dlrm_check_error(ws)[0] == 0
+    xs = x.bfloat16().double().numpy()     # the input rounded to bf16, as every bf16 layer path does
+    want = O.mlp(Ws, bs, xs, relu_last=True)
+    assert_close(to_np(out), want, "bf16", f"one-kernel MLP {dims} B={B}", scale_mlp(Ws, bs, xs))
 
 
 # at 4096+ rows the last hidden layer (width <= 256) and the one-column sigmoid output run as one kernel

@@ -1,8 +1,8 @@
 """Bounded device waits that run out (failure detection without a GPU fault).
 
 dlrm_set_wait_polls(0) makes the first bounded wait of the row-gathering
-kernels and the ordinary waits of the single-CTA tensor-core layer give up at
-once. Each call below must still return, report DLRM_ERR_TIMEOUT through
+kernels and the ordinary waits of the single-CTA tensor-core layer and of the
+one-kernel three-layer MLP give up at once. Each call below must still return, report DLRM_ERR_TIMEOUT through
 dlrm_check_error (the kernel drained its own copies and MMAs, freed its tensor
 memory and returned), and, after the default is restored, the same call on
 the same stream must give exactly the result of a call that never timed out.
@@ -61,6 +61,22 @@ def test_tensor_core_layer_wait_runs_out():
     x = torch.randn(B, dims[0], device="cuda").to(torch.bfloat16)
     out = torch.empty(B, dims[-1], device="cuda")
     ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, torch.bfloat16))
+    _timed_out_then_recovers(lambda: E.dlrm_mlp_fwd(mlp, B, x, dims[0], out, dims[-1], E.ACT_RELU, ws), ws, out)
+
+
+def test_one_kernel_mlp_wait_runs_out():
+    """Three bf16 layers in one kernel (weight ring, layer-1 chunks and h2 staged on chip, three accumulators)."""
+    torch.manual_seed(1)
+    dims = [13, 512, 256, 128]
+    Ws = [torch.zeros(dims[l + 1], E.dlrm_ld(dims[l], "bf16"), device="cuda", dtype=torch.bfloat16) for l in range(3)]
+    for l in range(3):
+        Ws[l][:, :dims[l]] = (torch.randn(dims[l + 1], dims[l], device="cuda") * 0.1).bfloat16()
+    bs = [torch.randn(dims[l + 1], device="cuda") * 0.1 for l in range(3)]
+    mlp = E.MLP(Ws, bs, dims)
+    B = 1000
+    x = torch.randn(B, dims[0], device="cuda")
+    out = torch.empty(B, dims[-1], device="cuda")
+    ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, torch.float32))
     _timed_out_then_recovers(lambda: E.dlrm_mlp_fwd(mlp, B, x, dims[0], out, dims[-1], E.ACT_RELU, ws), ws, out)
 
 
