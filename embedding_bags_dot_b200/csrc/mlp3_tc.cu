@@ -1,6 +1,6 @@
-// Three fully connected layers in one tensor-core kernel, for the bottom MLP of
-// DLRM ("Deep Learning Recommendation Model (DLRM)", nadeemcite summary, Key
-// Method Details: the dense features go through FC layers with ReLU):
+// Three fully connected layers in one kernel, for the bottom MLP of DLRM
+// ("Deep Learning Recommendation Model (DLRM)", nadeemcite summary, Key Method
+// Details: the dense features go through FC layers with ReLU):
 //   h1 = relu(x W1^T + b1), h2 = relu(h1 W2^T + b2), y = relu(h2 W3^T + b3)
 // with x fp32 [M][n0 <= 16] (rounded to bf16, as the layer-by-layer path does),
 // bf16 weights, h1 and h2 rounded to bf16, fp32 accumulation and fp32 output.
@@ -11,20 +11,22 @@
 //   warp 0      TMA producer: W1 once (n1 x 16, 32-byte swizzle, resident),
 //               then per tile the 64-deep k-blocks of W2 and of W3 through a
 //               4-stage ring (128-byte swizzle);
-//   warp 1      allocates the 512 TMEM columns and one thread issues the MMAs;
-//   warps 2..9  epilogue (two warps per TMEM lane quadrant, half the columns
-//               each): x -> bf16 tile, and every accumulator -> bias, ReLU ->
-//               the next layer's operand in shared memory or the fp32 output.
-// Layer 1 runs in 64-column chunks: chunk j of h1 is exactly k-block j of
-// layer 2's A operand. The MMA thread keeps layer 1 LAG chunks ahead of layer
-// 2 (M=128, N=64, K=16 into one of four TMEM slots), so the epilogue's work on
-// a chunk overlaps the layer-2 MMAs of the chunks before it. The four 16 KB
-// slots of the operand ring hold the h1 chunks, then, once layer 2 is done,
-// the k-blocks of h2 for layer 3.
-// TMEM: layer-2 accumulator [0, 256), whose first n3 columns then hold the
-// layer-3 accumulator; layer-1 slots [256, 512). Biases sit in shared memory.
-// All waits are bounded: on timeout the kernel records DLRM_ERR_TIMEOUT,
-// drains its own copies and MMAs, frees TMEM and returns.
+//   warp 1      allocates 512 TMEM columns; one thread issues the tcgen05 MMAs
+//               of layers 2 and 3;
+//   warps 2..9  two per TMEM lane quadrant (32 rows), half the columns each.
+// Layer 1 (K = 16) is too thin for the tcgen05 pipe: the epilogue warps
+// compute it themselves, 64 columns at a time, with mma.sync (x fragments
+// straight from global memory, W1 fragments by ldmatrix, accumulators started
+// at the bias), and write the ReLU'd bf16 chunk with stmatrix into one of four
+// 16 KB operand tiles. Chunk j of h1 is exactly k-block j of layer 2's A
+// operand, so the epilogue runs up to four chunks ahead of the layer-2 MMAs.
+// Once layer 2 is done the four tiles take h2 (bias, ReLU, bf16 from TMEM)
+// for layer 3, whose accumulator alternates between two TMEM buffers so that
+// its epilogue overlaps the next tile.
+// TMEM: layer-2 accumulator [0, 256), layer-3 accumulators [256, 384) and
+// [384, 512). Biases sit in shared memory. All waits are bounded: on timeout
+// the kernel records DLRM_ERR_TIMEOUT, drains its own copies and MMAs, frees
+// TMEM and returns.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -36,27 +38,26 @@ namespace tc {
 namespace {
 
 constexpr int M3_THREADS = 64 + 32 * EPI_WARPS;
-constexpr int SLOTS = 4;                               // layer-1 TMEM slots and operand-ring tiles
-constexpr int LAG = 3;                                 // layer-1 chunks issued ahead of layer 2
+constexpr int SLOTS = 4;                               // operand-ring tiles (h1 chunks, then h2)
 constexpr int W_STAGES = 4;
 constexpr int W_STAGE_BYTES = 256 * BK * 2;            // one k-block of up to 256 weight rows
 constexpr int TILE_BYTES = BM * BK * 2;                // one 128 x 64 bf16 operand tile
 constexpr int OFF_W1 = 0;                              // n1 / 64 chunks of 64 rows x 32 bytes
-constexpr int OFF_X0 = 16 * 1024;                      // 128 x 32-byte tile
-constexpr int OFF_BIAS = 20 * 1024;                    // b1 | b2 | b3, up to 896 floats
-constexpr int OFF_ACT = 24 * 1024;                     // SLOTS operand tiles (h1 chunks, then h2)
+constexpr int OFF_BIAS = 16 * 1024;                    // b1 | b2 | b3, up to 896 floats
+constexpr int OFF_ACT = 20 * 1024;                     // SLOTS operand tiles
 constexpr int OFF_WR = OFF_ACT + SLOTS * TILE_BYTES;   // weight ring
 constexpr int OFF_BARS = OFF_WR + W_STAGES * W_STAGE_BYTES;
 constexpr int M3_SMEM = OFF_BARS + 512 + 1024;
-constexpr uint32_t COL_ACC = 0, COL_A1 = 256;
+constexpr uint32_t COL_ACC2 = 0, COL_ACC3 = 256;
 static_assert(M3_SMEM <= 227 * 1024, "shared memory of the fused MLP");
+static_assert(OFF_ACT % 1024 == 0 && OFF_WR % 1024 == 0, "swizzled tiles are 1024-byte aligned");
 
 struct Bars3 {
     unsigned long long wfull[W_STAGES], wempty[W_STAGES];
-    unsigned long long w1full, x0full, x0empty;
-    unsigned long long a1full[SLOTS], a1empty[SLOTS];   // layer-1 TMEM slots
+    unsigned long long w1full;
     unsigned long long s1full[SLOTS], s1empty[SLOTS];   // h1 chunk tiles in the operand ring
-    unsigned long long acc2full, s2full, s2empty, acc3full, acc3empty;
+    unsigned long long acc2full, acc2empty, s2full, s2empty;
+    unsigned long long acc3full[2], acc3empty[2];
     unsigned long long drain;
     unsigned int tmem_base;
     int abort;
@@ -65,16 +66,6 @@ static_assert(sizeof(Bars3) <= 512, "barrier block");
 
 static __device__ long long g_mlp3_wait_polls = WAIT_LIMIT;
 
-// K-major operand with 32-byte swizzle (rows of 16 bf16): 8-row groups of 256 bytes.
-__device__ __forceinline__ uint64_t sdesc32(uint32_t addr) {
-    uint64_t d = (uint64_t)((addr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)1 << 16;
-    d |= (uint64_t)(256 >> 4) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)6 << 61;
-    return d;
-}
-
 __host__ __device__ constexpr uint32_t idesc_mn(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
@@ -82,6 +73,24 @@ __host__ __device__ constexpr uint32_t idesc_mn(int m, int n) {
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // 32 accumulator columns of one row + bias (shared memory), ReLU, rounded to bf16 and stored as four 16-byte
@@ -102,7 +111,7 @@ __device__ __forceinline__ void store_bf16_chunks(const uint32_t (&r)[32], const
     }
 }
 
-// Uses of slot s per tile (chunks j < nc1 with j % SLOTS == s) and the global use count of chunk j of tile i.
+// Global use count of operand slot j % SLOTS by chunk j of tile i (uses per tile: chunks with that slot).
 __device__ __forceinline__ uint32_t slot_use(int i, int j, int nc1) {
     const int s = j % SLOTS;
     const int per = (nc1 - s + SLOTS - 1) / SLOTS;
@@ -130,19 +139,18 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
             mbar_init(&bars->wempty[s], 1);
         }
         mbar_init(&bars->w1full, 1);
-        mbar_init(&bars->x0full, 4);
-        mbar_init(&bars->x0empty, 1);
         for (int a = 0; a < SLOTS; ++a) {
-            mbar_init(&bars->a1full[a], 1);
-            mbar_init(&bars->a1empty[a], EPI_WARPS);
             mbar_init(&bars->s1full[a], EPI_WARPS);
             mbar_init(&bars->s1empty[a], 1);
         }
         mbar_init(&bars->acc2full, 1);
+        mbar_init(&bars->acc2empty, EPI_WARPS);
         mbar_init(&bars->s2full, EPI_WARPS);
         mbar_init(&bars->s2empty, 1);
-        mbar_init(&bars->acc3full, 1);
-        mbar_init(&bars->acc3empty, EPI_WARPS);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bars->acc3full[a], 1);
+            mbar_init(&bars->acc3empty[a], EPI_WARPS);
+        }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -161,12 +169,12 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
     volatile int* abort = &bars->abort;
     bool timed_out = false;
     const long long lim = g_mlp3_wait_polls;
+    const bool any = (int)blockIdx.x < ntiles;
 
     if (warp == 0) {
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW2)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW3)) : "memory");
-            const bool any = (int)blockIdx.x < ntiles;
             if (any) {
                 mbar_expect_tx(&bars->w1full, (uint32_t)(nc1 * 64 * 32));
                 for (int j = 0; j < nc1; ++j) tma_load_2d(base + OFF_W1 + j * 2048, &mapW1, &bars->w1full, 0, 64 * j);
@@ -203,59 +211,40 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id1 = idesc_mn(BM, 64), id2 = idesc_mn(BM, n2), id3 = idesc_mn(BM, n3);
+            const uint32_t id2 = idesc_mn(BM, n2), id3 = idesc_mn(BM, n3);
             int ws = 0;
             uint32_t wph = 0;
-            if ((int)blockIdx.x < ntiles && !mbar_wait_n(&bars->w1full, 0, abort, lim)) timed_out = true;
             int i = 0;
             for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
                 const uint32_t ip = (uint32_t)i & 1u;
-                if (!mbar_wait_n(&bars->x0full, ip, abort, lim)) {
-                    timed_out = true;
-                    break;
-                }
-                for (int jj = 0; jj < nc1 + LAG && !timed_out; ++jj) {
-                    if (jj < nc1) {   // layer 1, chunk jj -> TMEM slot jj % SLOTS
-                        const int sl = jj % SLOTS;
-                        const uint32_t u = slot_use(i, jj, nc1);
-                        if (!mbar_wait_n(&bars->a1empty[sl], (u & 1u) ^ 1u, abort, lim)) {
-                            timed_out = true;
-                            break;
-                        }
-                        fence_after();
-                        umma(tmem + COL_A1 + 64 * sl, sdesc32(base + OFF_X0), sdesc32(base + OFF_W1 + jj * 2048), id1, 0);
-                        umma_commit(&bars->a1full[sl]);
-                        if (jj == nc1 - 1) umma_commit(&bars->x0empty);
+                // layer 2: k-block j is h1 chunk j (operand slot j % SLOTS)
+                for (int j = 0; j < nc1; ++j) {
+                    const int sl = j % SLOTS;
+                    const uint32_t u = slot_use(i, j, nc1);
+                    if ((j == 0 && !mbar_wait_n(&bars->acc2empty, ip ^ 1u, abort, lim)) ||
+                        !mbar_wait_n(&bars->s1full[sl], u & 1u, abort, lim) ||
+                        !mbar_wait_n(&bars->wfull[ws], wph, abort, lim)) {
+                        timed_out = true;
+                        break;
                     }
-                    if (jj >= LAG) {   // layer 2, k-block j = h1 chunk j (operand slot j % SLOTS)
-                        const int j = jj - LAG, sl = j % SLOTS;
-                        const uint32_t u = slot_use(i, j, nc1);
-                        if (j == 0 && !mbar_wait_n(&bars->acc3empty, ip ^ 1u, abort, lim)) {
-                            timed_out = true;
-                            break;
-                        }
-                        if (!mbar_wait_n(&bars->s1full[sl], u & 1u, abort, lim) ||
-                            !mbar_wait_n(&bars->wfull[ws], wph, abort, lim)) {
-                            timed_out = true;
-                            break;
-                        }
-                        fence_after();
-                        const uint32_t a = base + OFF_ACT + sl * TILE_BYTES, w = base + OFF_WR + ws * W_STAGE_BYTES;
+                    fence_after();
+                    const uint32_t a = base + OFF_ACT + sl * TILE_BYTES, w = base + OFF_WR + ws * W_STAGE_BYTES;
 #pragma unroll
-                        for (int k = 0; k < BK / 16; ++k)
-                            umma(tmem + COL_ACC, sdesc(a + k * 32), sdesc(w + k * 32), id2, (j | k) != 0);
-                        umma_commit(&bars->wempty[ws]);
-                        umma_commit(&bars->s1empty[sl]);
-                        if (++ws == W_STAGES) {
-                            ws = 0;
-                            wph ^= 1u;
-                        }
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma(tmem + COL_ACC2, sdesc(a + k * 32), sdesc(w + k * 32), id2, (j | k) != 0);
+                    umma_commit(&bars->wempty[ws]);
+                    umma_commit(&bars->s1empty[sl]);
+                    if (++ws == W_STAGES) {
+                        ws = 0;
+                        wph ^= 1u;
                     }
                 }
                 if (timed_out) break;
                 umma_commit(&bars->acc2full);
-                // layer 3 on h2 (operand slots 0 .. n2/64 - 1), accumulator in the first n3 columns
-                if (!mbar_wait_n(&bars->s2full, ip, abort, lim)) {
+                // layer 3 on h2 (operand slots 0 .. n2/64 - 1) into accumulator i & 1
+                const uint32_t d3 = tmem + COL_ACC3 + 128 * ip;
+                if (!mbar_wait_n(&bars->s2full, ip, abort, lim) ||
+                    !mbar_wait_n(&bars->acc3empty[ip], (((uint32_t)i >> 1) & 1u) ^ 1u, abort, lim)) {
                     timed_out = true;
                     break;
                 }
@@ -268,8 +257,7 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
                     fence_after();
                     const uint32_t a = base + OFF_ACT + kb * TILE_BYTES, w = base + OFF_WR + ws * W_STAGE_BYTES;
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        umma(tmem + COL_ACC, sdesc(a + k * 32), sdesc(w + k * 32), id3, (kb | k) != 0);
+                    for (int k = 0; k < BK / 16; ++k) umma(d3, sdesc(a + k * 32), sdesc(w + k * 32), id3, (kb | k) != 0);
                     umma_commit(&bars->wempty[ws]);
                     if (++ws == W_STAGES) {
                         ws = 0;
@@ -277,7 +265,7 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
                     }
                 }
                 if (timed_out) break;
-                umma_commit(&bars->acc3full);
+                umma_commit(&bars->acc3full[ip]);
                 umma_commit(&bars->s2empty);
             }
             if (timed_out) *abort = 1;
@@ -286,107 +274,37 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
         }
     } else {
         const int ew = warp - 2;
-        const int q = warp & 3;                  // TMEM lane quadrant
+        const int q = warp & 3;                  // TMEM lane quadrant: rows 32 q .. 32 q + 31
         const int h = ew >> 2;                   // half of the columns
-        const int r = q * 32 + lane;             // row of the tile
-        const int rsw = r & 7;                   // 128-byte swizzle phase of the row
+        const int r = q * 32 + lane;             // this thread's row for the TMEM epilogues
+        const int rsw = r & 7;                   // 128-byte swizzle phase of that row
         const uint32_t lanes = (uint32_t)(q * 32) << 16;
+        const int gr = lane >> 2, tc = 2 * (lane & 3);
         const float* bs1 = bias_s;
         const float* bs2 = bias_s + n1;
         const float* bs3 = bias_s + n1 + n2;
-        // x rows of a tile, loaded one tile ahead by the first warp of each quadrant
-        float xr[16];
+        // x fragments (mma.sync A layout) of rows 32 q + 16 mt + {gr, gr + 8}, columns {tc, tc+1, tc+8, tc+9}
+        float xf[2][8];
         auto load_x = [&](int t) {
-            const long long row = (long long)t * BM + r;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) xr[k] = (row < M && k < n0) ? __ldg(x + row * ldx + k) : 0.f;
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const long long row = (long long)t * BM + q * 32 + 16 * mt + gr + 8 * ((e >> 1) & 1);
+                    const int k = tc + (e & 1) + 8 * (e >> 2);
+                    xf[mt][e] = (row < M && k < n0) ? __ldg(x + row * ldx + k) : 0.f;
+                }
         };
-        // x (registers) -> bf16, row r of the 32-byte swizzled tile
-        auto store_x = [&]() {
-            unsigned char* dst = g + OFF_X0 + r * 32;
-            const int sw = (r >> 2) & 1;
-            *reinterpret_cast<uint4*>(dst + 16 * (0 ^ sw)) =
-                make_uint4(pack2(xr[0], xr[1]), pack2(xr[2], xr[3]), pack2(xr[4], xr[5]), pack2(xr[6], xr[7]));
-            *reinterpret_cast<uint4*>(dst + 16 * (1 ^ sw)) =
-                make_uint4(pack2(xr[8], xr[9]), pack2(xr[10], xr[11]), pack2(xr[12], xr[13]), pack2(xr[14], xr[15]));
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->x0full);
-        };
-        if (h == 0 && (int)blockIdx.x < ntiles) {
-            load_x(blockIdx.x);
-            store_x();
-            if ((int)(blockIdx.x + gridDim.x) < ntiles) load_x(blockIdx.x + gridDim.x);
-        }
-        int i = 0;
-        for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
-            const uint32_t ip = (uint32_t)i & 1u;
-            // layer-1 chunks -> h1 tiles in the operand ring
-            for (int j = 0; j < nc1; ++j) {
-                const int sl = j % SLOTS;
-                const uint32_t u = slot_use(i, j, nc1);
-                if (!mbar_wait_n(&bars->a1full[sl], u & 1u, abort, lim)) {
-                    timed_out = true;
-                    break;
-                }
-                fence_after();
-                uint32_t acc[32];
-                tmem_ld32_issue(tmem + lanes + COL_A1 + 64 * sl + 32 * h, acc);
-                tmem_ld_wait();
-                fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->a1empty[sl]);
-                // the slot's previous reader: layer 2 on chunk j - SLOTS of this tile, else the last tile's layer 3
-                const bool ok = j >= SLOTS ? mbar_wait_n(&bars->s1empty[sl], (u & 1u) ^ 1u, abort, lim)
-                                           : mbar_wait_n(&bars->s2empty, ip ^ 1u, abort, lim);
-                if (!ok) {
-                    timed_out = true;
-                    break;
-                }
-                store_bf16_chunks(acc, bs1 + 64 * j + 32 * h, g + OFF_ACT + sl * TILE_BYTES + r * 128, 4 * h, rsw);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->s1full[sl]);
-            }
-            if (timed_out) break;
-            // the next tile's x, once this tile's layer 1 has read the x tile
-            if (h == 0 && t + (int)gridDim.x < ntiles) {
-                if (!mbar_wait_n(&bars->x0empty, ip, abort, lim)) {
-                    timed_out = true;
-                    break;
-                }
-                store_x();
-                if (t + 2 * (int)gridDim.x < ntiles) load_x(t + 2 * gridDim.x);
-            }
-            // layer-2 accumulator -> h2 tiles (layer 2 has finished reading the ring)
-            if (!mbar_wait_n(&bars->acc2full, ip, abort, lim)) {
-                timed_out = true;
-                break;
-            }
+        // layer-3 accumulator of tile tt (local index ii) -> fp32 output rows
+        auto out_tile = [&](int tt, int ii) -> bool {
+            const uint32_t b = (uint32_t)ii & 1u;
+            if (!mbar_wait_n(&bars->acc3full[b], ((uint32_t)ii >> 1) & 1u, abort, lim)) return false;
             fence_after();
-            for (int cb = 0; cb < n2 / 64; ++cb) {
-                const int col = h * (n2 / 2) + 32 * cb;
-                uint32_t acc[32];
-                tmem_ld32_issue(tmem + lanes + COL_ACC + col, acc);
-                tmem_ld_wait();
-                store_bf16_chunks(acc, bs2 + col, g + OFF_ACT + (col / 64) * TILE_BYTES + r * 128, (col % 64) / 8,
-                                  rsw);
-            }
-            fence_before();
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->s2full);
-            // layer-3 accumulator -> fp32 output rows
-            if (!mbar_wait_n(&bars->acc3full, ip, abort, lim)) {
-                timed_out = true;
-                break;
-            }
-            fence_after();
-            const long long row = (long long)t * BM + r;
+            const long long row = (long long)tt * BM + r;
             for (int cb = 0; cb < n3 / 64; ++cb) {
                 const int col = h * (n3 / 2) + 32 * cb;
                 uint32_t acc[32];
-                tmem_ld32_issue(tmem + lanes + COL_ACC + col, acc);
+                tmem_ld32_issue(tmem + lanes + COL_ACC3 + 128 * b + col, acc);
                 tmem_ld_wait();
                 if (row < M) {
                     float4* o = reinterpret_cast<float4*>(out + row * ldo + col);
@@ -403,8 +321,102 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
             }
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->acc3empty);
+            if (lane == 0) mbar_arrive(&bars->acc3empty[b]);
+            return true;
+        };
+        if (any) {
+            load_x(blockIdx.x);
+            if (!mbar_wait_n(&bars->w1full, 0, abort, lim)) timed_out = true;
         }
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
+            const uint32_t ip = (uint32_t)i & 1u;
+            uint32_t af[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int p = 0; p < 4; ++p) af[mt][p] = pack2(xf[mt][2 * p], xf[mt][2 * p + 1]);
+            if (t + (int)gridDim.x < ntiles) load_x(t + gridDim.x);   // the next tile's x, a tile ahead
+            // layer 1, chunk j: 32 rows x 32 columns per warp on mma.sync -> h1 tile j % SLOTS
+            for (int j = 0; j < nc1; ++j) {
+                const int sl = j % SLOTS;
+                const uint32_t u = slot_use(i, j, nc1);
+                uint32_t bf[2][4];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int n = 32 * h + 16 * hh + (lane & 15);         // W1 row within chunk j
+                    ldsm_x4(base + OFF_W1 + j * 2048 + n * 32 + 16 * ((lane >> 4) ^ ((n >> 2) & 1)), bf[hh]);
+                }
+                float acc[2][4][4];
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const float2 bb = *reinterpret_cast<const float2*>(bs1 + 64 * j + 32 * h + 8 * nt + tc);
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        acc[mt][nt][0] = bb.x;
+                        acc[mt][nt][1] = bb.y;
+                        acc[mt][nt][2] = bb.x;
+                        acc[mt][nt][3] = bb.y;
+                        mma16816(acc[mt][nt], af[mt], bf[nt >> 1][(nt & 1) ? 1 : 0], bf[nt >> 1][(nt & 1) ? 3 : 2]);
+                    }
+                }
+                // the slot's previous reader: layer 2 on chunk j - SLOTS of this tile, else the last tile's layer 3
+                const bool ok = j >= SLOTS ? mbar_wait_n(&bars->s1empty[sl], (u & 1u) ^ 1u, abort, lim)
+                                           : mbar_wait_n(&bars->s2empty, ip ^ 1u, abort, lim);
+                if (!ok) {
+                    timed_out = true;
+                    break;
+                }
+                const uint32_t slot = base + OFF_ACT + sl * TILE_BYTES;
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t v[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {   // matrix m: n-tile 2 np + (m >> 1), rows gr (+8 if m odd)
+                            const float* c = acc[mt][2 * np + (m >> 1)];
+                            v[m] = (m & 1) ? pack2(fmaxf(c[2], 0.f), fmaxf(c[3], 0.f))
+                                           : pack2(fmaxf(c[0], 0.f), fmaxf(c[1], 0.f));
+                        }
+                        const int m = lane >> 3;
+                        const int row = q * 32 + 16 * mt + 8 * (m & 1) + (lane & 7);
+                        const int kc = 4 * h + 2 * np + (m >> 1);
+                        stsm_x4(slot + row * 128 + 16 * (kc ^ (row & 7)), v[0], v[1], v[2], v[3]);
+                    }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s1full[sl]);
+            }
+            if (timed_out) break;
+            // layer-2 accumulator -> h2 tiles (layer 2 has finished reading the ring)
+            if (!mbar_wait_n(&bars->acc2full, ip, abort, lim)) {
+                timed_out = true;
+                break;
+            }
+            fence_after();
+            for (int cb = 0; cb < n2 / 64; ++cb) {
+                const int col = h * (n2 / 2) + 32 * cb;
+                uint32_t acc[32];
+                tmem_ld32_issue(tmem + lanes + COL_ACC2 + col, acc);
+                tmem_ld_wait();
+                store_bf16_chunks(acc, bs2 + col, g + OFF_ACT + (col / 64) * TILE_BYTES + r * 128, (col % 64) / 8,
+                                  rsw);
+            }
+            fence_before();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->acc2empty);
+                mbar_arrive(&bars->s2full);
+            }
+            // the previous tile's output while this tile's layer 3 runs
+            if (i > 0 && !out_tile(t - (int)gridDim.x, i - 1)) {
+                timed_out = true;
+                break;
+            }
+        }
+        if (!timed_out && i > 0 && !out_tile(blockIdx.x + (i - 1) * (int)gridDim.x, i - 1)) timed_out = true;
         if (timed_out) *abort = 1;
     }
 
