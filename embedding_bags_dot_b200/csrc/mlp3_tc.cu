@@ -20,8 +20,6 @@
 // at the bias), and write the ReLU'd bf16 chunk with stmatrix into one of four
 // 16 KB operand tiles. Chunk j of h1 is exactly k-block j of layer 2's A
 // operand, so the epilogue runs up to four chunks ahead of the layer-2 MMAs.
-// Each CTA starts layers 2 and 3 at its own k-block (blockIdx modulo the
-// count), so that concurrent CTAs read different weight lines.
 // Once layer 2 is done the four tiles take h2 (bias, ReLU, bf16 from TMEM)
 // for layer 3, whose accumulator alternates between two TMEM buffers so that
 // its epilogue overlaps the next tile.
@@ -134,9 +132,6 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = (M + BM - 1) / BM;
     const int nc1 = n1 / 64, nk3 = n2 / 64;
-    // every CTA walks the k-blocks of layers 2 and 3 from its own starting block, so that the CTAs do not all
-    // fetch the same weight lines at the same moment
-    const int rot2 = (int)(blockIdx.x % (unsigned)nc1), rot3 = (int)(blockIdx.x % (unsigned)nk3);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < W_STAGES; ++s) {
@@ -193,9 +188,9 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
                         break;
                     }
                     const bool l2 = kb < nc1;
-                    const int blk = l2 ? (rot2 + kb) % nc1 : (rot3 + kb - nc1) % nk3;
                     mbar_expect_tx(&bars->wfull[s], (uint32_t)((l2 ? n2 : n3) * BK * 2));
-                    tma_load_2d(base + OFF_WR + s * W_STAGE_BYTES, l2 ? &mapW2 : &mapW3, &bars->wfull[s], blk * BK, 0);
+                    tma_load_2d(base + OFF_WR + s * W_STAGE_BYTES, l2 ? &mapW2 : &mapW3, &bars->wfull[s],
+                                (l2 ? kb : kb - nc1) * BK, 0);
                     if (++s == W_STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -222,7 +217,7 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
             int i = 0;
             for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
                 const uint32_t ip = (uint32_t)i & 1u;
-                // layer 2, step j: k-block (rot2 + j) % nc1 = the h1 chunk in operand slot j % SLOTS
+                // layer 2: k-block j is h1 chunk j (operand slot j % SLOTS)
                 for (int j = 0; j < nc1; ++j) {
                     const int sl = j % SLOTS;
                     const uint32_t u = slot_use(i, j, nc1);
@@ -260,7 +255,7 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
                         break;
                     }
                     fence_after();
-                    const uint32_t a = base + OFF_ACT + ((rot3 + kb) % nk3) * TILE_BYTES, w = base + OFF_WR + ws * W_STAGE_BYTES;
+                    const uint32_t a = base + OFF_ACT + kb * TILE_BYTES, w = base + OFF_WR + ws * W_STAGE_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) umma(d3, sdesc(a + k * 32), sdesc(w + k * 32), id3, (kb | k) != 0);
                     umma_commit(&bars->wempty[ws]);
@@ -342,20 +337,20 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
 #pragma unroll
                 for (int p = 0; p < 4; ++p) af[mt][p] = pack2(xf[mt][2 * p], xf[mt][2 * p + 1]);
             if (t + (int)gridDim.x < ntiles) load_x(t + gridDim.x);   // the next tile's x, a tile ahead
-            // layer 1, step j = chunk c: 32 rows x 32 columns per warp on mma.sync -> h1 tile j % SLOTS
+            // layer 1, chunk j: 32 rows x 32 columns per warp on mma.sync -> h1 tile j % SLOTS
             for (int j = 0; j < nc1; ++j) {
-                const int sl = j % SLOTS, c = (rot2 + j) % nc1;
+                const int sl = j % SLOTS;
                 const uint32_t u = slot_use(i, j, nc1);
                 uint32_t bf[2][4];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int n = 32 * h + 16 * hh + (lane & 15);         // W1 row within chunk c
-                    ldsm_x4(base + OFF_W1 + c * 2048 + n * 32 + 16 * ((lane >> 4) ^ ((n >> 2) & 1)), bf[hh]);
+                    const int n = 32 * h + 16 * hh + (lane & 15);         // W1 row within chunk j
+                    ldsm_x4(base + OFF_W1 + j * 2048 + n * 32 + 16 * ((lane >> 4) ^ ((n >> 2) & 1)), bf[hh]);
                 }
                 float acc[2][4][4];
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    const float2 bb = *reinterpret_cast<const float2*>(bs1 + 64 * c + 32 * h + 8 * nt + tc);
+                    const float2 bb = *reinterpret_cast<const float2*>(bs1 + 64 * j + 32 * h + 8 * nt + tc);
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
                         acc[mt][nt][0] = bb.x;
