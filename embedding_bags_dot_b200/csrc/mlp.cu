@@ -18,52 +18,71 @@ __device__ __forceinline__ float activate(float v) {
     return v;
 }
 
-// 64 x 64 output tile per 256-thread block, 16-deep k slices through smem,
-// 4 x 4 outputs per thread.
+// 64 x 64 output tile per 256-thread block, 16-deep k slices through shared
+// memory, 4 x 4 outputs per thread. Software-pipelined: the next slice's
+// global loads are issued into registers before the current slice's
+// multiply-adds, and the slices alternate between two shared buffers, so each
+// slice costs one barrier and its load latency hides behind the arithmetic.
 template <typename TA, typename TW, typename TC, int ACT>
 __global__ void __launch_bounds__(256) linear_ffma_kernel(int M, int N, int K, const TA* __restrict__ A, int lda,
                                                           const TW* __restrict__ W, int ldw,
                                                           const float* __restrict__ bias, TC* __restrict__ C,
                                                           int ldc) {
-    __shared__ float As[16][64 + 4];
-    __shared__ float Ws[16][64 + 4];
+    constexpr int RM = 64, TM = 4;   // tile rows, output rows per thread
+    __shared__ __align__(16) float As[2][16][RM + 4];
+    __shared__ __align__(16) float Ws[2][16][64 + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const long long m0 = (long long)blockIdx.y * 64;
+    const long long m0 = (long long)blockIdx.y * RM;
     const int n0 = blockIdx.x * 64;
-    float acc[4][4];
+    float acc[TM][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    // this thread's loads: row lr of the A and W tiles, k = k0 + lk .. k0 + lk + 3
     const int lr = threadIdx.x >> 2, lk = (threadIdx.x & 3) * 4;
-    for (int k0 = 0; k0 < K; k0 += 16) {
+    const long long gm = m0 + lr;
+    const int gn = n0 + lr;
+    float ra[4], rw[4];
+    auto load = [&](int k0) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int gk = k0 + lk + e;
-            const long long gm = m0 + lr;
-            const int gn = n0 + lr;
-            As[lk + e][lr] = (gm < M && gk < K) ? Cvt<TA>::to_f(A[gm * lda + gk]) : 0.f;
-            Ws[lk + e][lr] = (gn < N && gk < K) ? Cvt<TW>::to_f(W[(long long)gn * ldw + gk]) : 0.f;
+            ra[e] = (gm < M && gk < K) ? Cvt<TA>::to_f(A[gm * lda + gk]) : 0.f;
+            rw[e] = (gn < N && gk < K) ? Cvt<TW>::to_f(W[(long long)gn * ldw + gk]) : 0.f;
         }
-        __syncthreads();
+    };
+    auto stage = [&](int b) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            As[b][lk + e][lr] = ra[e];
+            Ws[b][lk + e][lr] = rw[e];
+        }
+    };
+    load(0);
+    stage(0);
+    __syncthreads();
+    int b = 0;
+    for (int k0 = 0; k0 < K; k0 += 16, b ^= 1) {
+        const bool more = k0 + 16 < K;
+        if (more) load(k0 + 16);   // in flight during this slice's multiply-adds
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
-            float a[4], w[4];
+            const float4 a = *reinterpret_cast<const float4*>(&As[b][kk][ty * 4]);
+            const float av[TM] = {a.x, a.y, a.z, a.w};
+            const float4 w = *reinterpret_cast<const float4*>(&Ws[b][kk][tx * 4]);
+            const float wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = As[kk][ty * 4 + i];
-                w[i] = Ws[kk][tx * 4 + i];
-            }
+            for (int i = 0; i < TM; ++i)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], wv[j], acc[i][j]);
         }
+        if (more) stage(b ^ 1);    // the other buffer: its last readers finished before the previous barrier
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const long long m = m0 + ty * 4 + i;
+    for (int i = 0; i < TM; ++i) {
+        const long long m = m0 + ty * TM + i;
         if (m >= M) continue;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

@@ -128,7 +128,7 @@ def test_fused_bottom_mlp(B, dt, n3):
 # three bf16 layers from fp32 input run as one kernel (h1, h2 kept on chip) for widths that are multiples of 64
 # up to 512 / 256 / 128 and up to 16 inputs: other widths, ragged batches, a K below 16
 @pytest.mark.parametrize("dims", [(13, 192, 128, 64), (7, 64, 64, 128), (16, 512, 64, 64), (1, 448, 192, 128)])
-@pytest.mark.parametrize("B", [1, 129, 4999])
+@pytest.mark.parametrize("B", [1, 129, 256, 300, 4999])   # from 256 rows on, SM pairs share each weight k-block
 def test_three_layer_mlp_one_kernel(dims, B):
     g = torch.Generator().manual_seed(B * 5 + dims[1])
     Ws, bs, Wd, bd = [], [], [], []

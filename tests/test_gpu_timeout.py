@@ -64,7 +64,8 @@ def test_tensor_core_layer_wait_runs_out():
     _timed_out_then_recovers(lambda: E.dlrm_mlp_fwd(mlp, B, x, dims[0], out, dims[-1], E.ACT_RELU, ws), ws, out)
 
 
-def test_one_kernel_mlp_wait_runs_out():
+@pytest.mark.parametrize("B", [100, 1000])    # one CTA per 128-row tile; SM pairs from 256 rows on
+def test_one_kernel_mlp_wait_runs_out(B):
     """Three bf16 layers in one kernel (weight ring, layer-1 chunks and h2 staged on chip, three accumulators)."""
     torch.manual_seed(1)
     dims = [13, 512, 256, 128]
@@ -73,7 +74,6 @@ def test_one_kernel_mlp_wait_runs_out():
         Ws[l][:, :dims[l]] = (torch.randn(dims[l + 1], dims[l], device="cuda") * 0.1).bfloat16()
     bs = [torch.randn(dims[l + 1], device="cuda") * 0.1 for l in range(3)]
     mlp = E.MLP(Ws, bs, dims)
-    B = 1000
     x = torch.randn(B, dims[0], device="cuda")
     out = torch.empty(B, dims[-1], device="cuda")
     ws = E.alloc_workspace(E.dlrm_mlp_workspace_size(mlp, B, torch.float32))
