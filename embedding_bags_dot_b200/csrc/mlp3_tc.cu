@@ -18,7 +18,7 @@
 // compute it themselves, 64 columns at a time, with mma.sync (x fragments
 // straight from global memory, W1 fragments by ldmatrix, accumulators started
 // at the bias), and write the ReLU'd bf16 chunk with stmatrix into one of four
-// 16 KB operand tiles. Chunk j of h1 is exactly k-block j of layer 2's A
+// 16 KB operand tiles; the two warp groups take alternate chunks. Chunk j of h1 is exactly k-block j of layer 2's A
 // operand, so the epilogue runs up to four chunks ahead of the layer-2 MMAs.
 // Once layer 2 is done the four tiles take h2 (bias, ReLU, bf16 from TMEM)
 // for layer 3, whose accumulator alternates between two TMEM buffers so that
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
         }
         mbar_init(&bars->w1full, 1);
         for (int a = 0; a < SLOTS; ++a) {
-            mbar_init(&bars->s1full[a], EPI_WARPS);
+            mbar_init(&bars->s1full[a], EPI_WARPS / 2);   // one warp group writes a chunk
             mbar_init(&bars->s1empty[a], 1);
         }
         mbar_init(&bars->acc2full, 1);
@@ -337,53 +337,60 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
 #pragma unroll
                 for (int p = 0; p < 4; ++p) af[mt][p] = pack2(xf[mt][2 * p], xf[mt][2 * p + 1]);
             if (t + (int)gridDim.x < ntiles) load_x(t + gridDim.x);   // the next tile's x, a tile ahead
-            // layer 1, chunk j: 32 rows x 32 columns per warp on mma.sync -> h1 tile j % SLOTS
-            for (int j = 0; j < nc1; ++j) {
+            // layer 1, chunk j on mma.sync -> h1 tile j % SLOTS: the two warp groups (h = 0, 1) take alternate
+            // chunks, each warp 32 rows x 64 columns, so two chunks are in progress at a time
+            for (int j = h; j < nc1; j += 2) {
                 const int sl = j % SLOTS;
                 const uint32_t u = slot_use(i, j, nc1);
-                uint32_t bf[2][4];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int n = 32 * h + 16 * hh + (lane & 15);         // W1 row within chunk j
-                    ldsm_x4(base + OFF_W1 + j * 2048 + n * 32 + 16 * ((lane >> 4) ^ ((n >> 2) & 1)), bf[hh]);
-                }
-                float acc[2][4][4];
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const float2 bb = *reinterpret_cast<const float2*>(bs1 + 64 * j + 32 * h + 8 * nt + tc);
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        acc[mt][nt][0] = bb.x;
-                        acc[mt][nt][1] = bb.y;
-                        acc[mt][nt][2] = bb.x;
-                        acc[mt][nt][3] = bb.y;
-                        mma16816(acc[mt][nt], af[mt], bf[nt >> 1][(nt & 1) ? 1 : 0], bf[nt >> 1][(nt & 1) ? 3 : 2]);
-                    }
-                }
-                // the slot's previous reader: layer 2 on chunk j - SLOTS of this tile, else the last tile's layer 3
-                const bool ok = j >= SLOTS ? mbar_wait_n(&bars->s1empty[sl], (u & 1u) ^ 1u, abort, lim)
-                                           : mbar_wait_n(&bars->s2empty, ip ^ 1u, abort, lim);
-                if (!ok) {
-                    timed_out = true;
-                    break;
-                }
                 const uint32_t slot = base + OFF_ACT + sl * TILE_BYTES;
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int cc = 0; cc < 2; ++cc) {   // columns 32 cc .. 32 cc + 31 of the chunk
+                    uint32_t bf[2][4];
 #pragma unroll
-                    for (int np = 0; np < 2; ++np) {
-                        uint32_t v[4];
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {   // matrix m: n-tile 2 np + (m >> 1), rows gr (+8 if m odd)
-                            const float* c = acc[mt][2 * np + (m >> 1)];
-                            v[m] = (m & 1) ? pack2(fmaxf(c[2], 0.f), fmaxf(c[3], 0.f))
-                                           : pack2(fmaxf(c[0], 0.f), fmaxf(c[1], 0.f));
-                        }
-                        const int m = lane >> 3;
-                        const int row = q * 32 + 16 * mt + 8 * (m & 1) + (lane & 7);
-                        const int kc = 4 * h + 2 * np + (m >> 1);
-                        stsm_x4(slot + row * 128 + 16 * (kc ^ (row & 7)), v[0], v[1], v[2], v[3]);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int n = 32 * cc + 16 * hh + (lane & 15);         // W1 row within chunk j
+                        ldsm_x4(base + OFF_W1 + j * 2048 + n * 32 + 16 * ((lane >> 4) ^ ((n >> 2) & 1)), bf[hh]);
                     }
+                    float acc[2][4][4];
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const float2 bb = *reinterpret_cast<const float2*>(bs1 + 64 * j + 32 * cc + 8 * nt + tc);
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt) {
+                            acc[mt][nt][0] = bb.x;
+                            acc[mt][nt][1] = bb.y;
+                            acc[mt][nt][2] = bb.x;
+                            acc[mt][nt][3] = bb.y;
+                            mma16816(acc[mt][nt], af[mt], bf[nt >> 1][(nt & 1) ? 1 : 0], bf[nt >> 1][(nt & 1) ? 3 : 2]);
+                        }
+                    }
+                    // the slot's previous reader: layer 2 on chunk j - SLOTS of this tile, else the last tile's layer 3
+                    if (cc == 0) {
+                        const bool ok = j >= SLOTS ? mbar_wait_n(&bars->s1empty[sl], (u & 1u) ^ 1u, abort, lim)
+                                                   : mbar_wait_n(&bars->s2empty, ip ^ 1u, abort, lim);
+                        if (!ok) {
+                            timed_out = true;
+                            break;
+                        }
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int np = 0; np < 2; ++np) {
+                            uint32_t v[4];
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {   // matrix m: n-tile 2 np + (m >> 1), rows gr (+8 if m odd)
+                                const float* c = acc[mt][2 * np + (m >> 1)];
+                                v[m] = (m & 1) ? pack2(fmaxf(c[2], 0.f), fmaxf(c[3], 0.f))
+                                               : pack2(fmaxf(c[0], 0.f), fmaxf(c[1], 0.f));
+                            }
+                            const int m = lane >> 3;
+                            const int row = q * 32 + 16 * mt + 8 * (m & 1) + (lane & 7);
+                            const int kc = 4 * cc + 2 * np + (m >> 1);
+                            stsm_x4(slot + row * 128 + 16 * (kc ^ (row & 7)), v[0], v[1], v[2], v[3]);
+                        }
+                }
+                if (timed_out) break;
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s1full[sl]);
