@@ -184,16 +184,35 @@ class ClockSampler:
 # --------------------------------------------------------------------------- oracle (CPU baseline)
 
 def oracle_rate(cfg, batch, n_samples: int, seed: int = 0):
-    """samples/s of the fp64 oracle forward on n_samples drawn from the batch (excluding input prep)."""
+    """samples/s of the fp64 oracle on n_samples drawn from the batch (excluding input prep): the forward, or for
+    a training workload the forward and backward (loss, MLP and row gradients; the update itself is negligible)."""
     from oracle import oracle as O
     rng = np.random.default_rng(seed)
     samples = np.sort(rng.choice(cfg.B, size=min(n_samples, cfg.B), replace=False))
-    Bs, dense, offs, idx, _, rows, used = O.sub_batch(cfg, batch, samples)
+    Bs, dense, offs, idx, labels, rows, used = O.sub_batch(cfg, batch, samples)
     model = O.model_for_rows(cfg, used)
     t0 = time.perf_counter()
-    (O.forward_cat if cfg.interaction == "cat" else O.forward)(model, dense, offs, idx)
+    if cfg.training:
+        O.train_grads(model, dense, offs, idx, labels)
+    else:
+        (O.forward_cat if cfg.interaction == "cat" else O.forward)(model, dense, offs, idx)
     dt = time.perf_counter() - t0
     return Bs / dt, dt, O.threads(), Bs
+
+
+def oracle_what(cfg) -> str:
+    return "fp64 forward + backward" if cfg.training else "fp64 forward"
+
+
+def cpu_baseline(cfg, batch, seconds: float) -> dict:
+    """The oracle on all host cores and on one core, on bounded random samples of the batch."""
+    rate, dt, cores, used = calibrated_oracle(cfg, batch, seconds)
+    r1, dt1, c1, used1 = oracle_on_one_core(cfg, batch, seconds / 3)
+    return {"value": rate, "unit": "samples/s", "cores": cores, "kind": "oracle",
+            "sample": f"{used} random samples of batch 0, {oracle_what(cfg)} in {dt:.1f} s",
+            "cpu_model": cpu_model(),
+            "one_core": {"value": r1, "cores": c1,
+                         "sample": f"{used1} random samples of batch 0, {oracle_what(cfg)} in {dt1:.1f} s"}}
 
 
 def cpu_model() -> str:
@@ -252,7 +271,7 @@ def run_reference(args, cfg, rank):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": "samples/s", "cores": cores, "kind": "oracle",
-                            "sample": f"{n} random samples of batch 0 per step (fp64 forward, host cores)",
+                            "sample": f"{n} random samples of batch 0 per step ({oracle_what(cfg)}, host cores)",
                             "cpu_model": cpu_model()},
            "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -433,13 +452,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, cores, used = calibrated_oracle(cfg, batches[0], args.cpu_seconds)
-        r1, dt1, c1, used1 = oracle_on_one_core(cfg, batches[0], args.cpu_seconds / 3)
-        cpu = {"value": rate, "unit": "samples/s", "cores": cores, "kind": "oracle",
-               "sample": f"{used} random samples of batch 0, fp64 forward in {dt:.1f} s",
-               "cpu_model": cpu_model(),
-               "one_core": {"value": r1, "cores": c1,
-                            "sample": f"{used1} random samples of batch 0, fp64 forward in {dt1:.1f} s"}}
+        cpu = cpu_baseline(cfg, batches[0], args.cpu_seconds)
 
     if rank == 0:
         traffic = kernel_traffic(*TRAFFIC[cfg.name]) if cfg.name in TRAFFIC else None
@@ -538,6 +551,9 @@ def run_train(args, cfg, rank, world, local_rank):
     _, peak_bf16, peak_kind = read_peaks()
     peak_tf32 = peak_bf16 * TF32_PER_BF16
     tensor_tflops = 3 * 2.0 * I * J * R / (gemm_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, batches[0], args.cpu_seconds)
     if rank == 0:
         out = {"metric": "DLRM training samples/s on 1 B200 (forward + backward + sparse SGD)",
                "value": aggregate_rate(cfg.B * args.steps, world, total_ms), "unit": "samples/s", "n_gpus": world,
@@ -554,7 +570,7 @@ def run_train(args, cfg, rank, world, local_rank):
                             "shape": f"{I}x{J}x{R} K-major x K-major",
                             "flops_per_launch": "3 TF32 products x 2*I*J*R", "avg_launch_ms": gemm_ms,
                             "fp32_equiv_tflops": 2.0 * I * J * R / (gemm_ms * 1e-3) / 1e12},
-               "loss_last": float(loss.item()), "gpu_launches": int(n1 - n0), "clocks": clk}
+               "cpu_baseline": cpu, "loss_last": float(loss.item()), "gpu_launches": int(n1 - n0), "clocks": clk}
         print(json.dumps(out), flush=True)
     return 0
 
