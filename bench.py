@@ -242,11 +242,15 @@ def oracle_on_one_core(cfg, batch, target_s: float):
 
 
 def calibrated_oracle(cfg, batch, target_s: float):
+    """The oracle on a sample sized to take about target_s: grown at most 8x per measurement, so that a rate
+    that falls with the sample size (the training oracle's) cannot overshoot the time budget."""
     n = 64
     rate, dt, cores, used = oracle_rate(cfg, batch, n)
-    n2 = int(min(cfg.B, max(n, rate * target_s)))
-    if n2 > n:
-        rate, dt, cores, used = oracle_rate(cfg, batch, n2, seed=1)
+    seed = 1
+    while dt < target_s / 2 and n < cfg.B:
+        n = int(min(cfg.B, 8 * n, max(n + 1, rate * target_s)))
+        rate, dt, cores, used = oracle_rate(cfg, batch, n, seed=seed)
+        seed += 1
     return rate, dt, cores, used
 
 

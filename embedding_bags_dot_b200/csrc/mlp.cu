@@ -92,6 +92,134 @@ __global__ void __launch_bounds__(256) linear_ffma_kernel(int M, int N, int K, c
     }
 }
 
+// fp32 A and W (rows 16-byte aligned): RM x 64 output tile per 256-thread block (RM = 64, or 32 when the
+// 64-row grid would leave more than half of the SMs idle), 32-deep k slices in a
+// 3-stage shared-memory ring filled by cp.async (16-byte copies straight from global memory, zero-filled past
+// M, N and K), so that two slices are always in flight while the block multiplies the third. Thread (ty, tx)
+// owns rows ty + 16 i (i < RM / 16) and columns tx + 16 j (j < 4): its A and W reads are 16-byte vectors along k, the
+// 16 W rows a warp reads fall in distinct bank groups (row stride 36 floats), and every output row is written
+// by 16 consecutive threads.
+namespace f32p {
+constexpr int BK = 32, LDS = BK + 4, STAGES = 3;
+constexpr int TILE_FLOATS = 64 * LDS;   // one 64-row tile; an RM-row A tile uses the first RM rows of it
+constexpr int SMEM = STAGES * 2 * TILE_FLOATS * 4;
+}  // namespace f32p
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename TC, int ACT, int RM>
+__global__ void __launch_bounds__(256) linear_f32_pipe_kernel(int M, int N, int K, const float* __restrict__ A,
+                                                              int lda, const float* __restrict__ W, int ldw,
+                                                              const float* __restrict__ bias, TC* __restrict__ C,
+                                                              int ldc) {
+    using namespace f32p;
+    constexpr int TM = RM / 16;   // output rows per thread
+    extern __shared__ __align__(16) float fsm[];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const long long m0 = (long long)blockIdx.y * RM;
+    const int n0 = blockIdx.x * 64;
+    const int nk = (K + BK - 1) / BK;
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(fsm);
+    // this thread's copies: rows lr and lr + 32 of both tiles, 16-byte column chunk lc of the slice
+    const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 4;
+    auto issue = [&](int kt) {
+        const int st = kt % STAGES;
+        const int k = kt * BK + lc;
+        const uint32_t bytes = k < K ? (uint32_t)(min(4, K - k) * 4) : 0u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = lr + 32 * h;
+            const long long gm = m0 + r;
+            const int gn = n0 + r;
+            if (r < RM) {
+                const uint32_t da = sbase + (uint32_t)(((st * 2) * TILE_FLOATS + r * LDS + lc) * 4);
+                cp_async16(da, gm < M && bytes ? A + gm * lda + k : A, gm < M ? bytes : 0u);
+            }
+            const uint32_t dw = sbase + (uint32_t)(((st * 2 + 1) * TILE_FLOATS + r * LDS + lc) * 4);
+            cp_async16(dw, gn < N && bytes ? W + (long long)gn * ldw + k : W, gn < N ? bytes : 0u);
+        }
+    };
+    float acc[TM][4];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < STAGES - 1; ++kt) {
+        if (kt < nk) issue(kt);
+        cp_async_commit();
+    }
+    for (int kt = 0; kt < nk; ++kt) {
+        cp_async_wait<STAGES - 2>();   // slice kt has landed (this thread's copies)
+        __syncthreads();               // ... and every thread's; the slot refilled below was last read before this
+        if (kt + STAGES - 1 < nk) issue(kt + STAGES - 1);
+        cp_async_commit();
+        const float* As = fsm + (kt % STAGES) * 2 * TILE_FLOATS;
+        const float* Ws = As + TILE_FLOATS;
+#pragma unroll
+        for (int kk = 0; kk < BK; kk += 4) {
+            float4 a[TM], w[4];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) a[i] = *reinterpret_cast<const float4*>(As + (ty + 16 * i) * LDS + kk);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(Ws + (tx + 16 * j) * LDS + kk);
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float t = acc[i][j];
+                    t = fmaf(a[i].x, w[j].x, t);
+                    t = fmaf(a[i].y, w[j].y, t);
+                    t = fmaf(a[i].z, w[j].z, t);
+                    t = fmaf(a[i].w, w[j].w, t);
+                    acc[i][j] = t;
+                }
+        }
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+        const long long m = m0 + ty + 16 * i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + tx + 16 * j;
+            if (n < N) C[m * ldc + n] = Cvt<TC>::from_f(activate<ACT>(acc[i][j] + bias[n]));
+        }
+    }
+}
+
+template <typename TC, int ACT>
+static void run_f32_pipe(int M, int N, int K, const float* A, int lda, const float* W, int ldw, const float* bias,
+                         void* C, int ldc, cudaStream_t st) {
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (2LL * ((N + 63) / 64) * ((M + 63) / 64) < sms) {
+        auto kern = linear_f32_pipe_kernel<TC, ACT, 32>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, f32p::SMEM);
+        const dim3 grid((N + 63) / 64, (M + 31) / 32);
+        kern<<<grid, 256, f32p::SMEM, st>>>(M, N, K, A, lda, W, ldw, bias, static_cast<TC*>(C), ldc);
+    } else {
+        auto kern = linear_f32_pipe_kernel<TC, ACT, 64>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, f32p::SMEM);
+        const dim3 grid((N + 63) / 64, (M + 63) / 64);
+        kern<<<grid, 256, f32p::SMEM, st>>>(M, N, K, A, lda, W, ldw, bias, static_cast<TC*>(C), ldc);
+    }
+}
+
+template <typename TC>
+static void dispatch_f32_pipe(int M, int N, int K, const float* A, int lda, const float* W, int ldw,
+                              const float* bias, void* C, int ldc, int act, cudaStream_t st) {
+    if (act == DLRM_ACT_RELU) run_f32_pipe<TC, DLRM_ACT_RELU>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+    else if (act == DLRM_ACT_SIGMOID) run_f32_pipe<TC, DLRM_ACT_SIGMOID>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+    else run_f32_pipe<TC, DLRM_ACT_NONE>(M, N, K, A, lda, W, ldw, bias, C, ldc, st);
+}
+
 // N == 1: one warp per row.
 template <typename TA, typename TW, int ACT>
 __global__ void __launch_bounds__(256) gemv_kernel(int M, int K, const TA* __restrict__ A, int lda,
@@ -162,6 +290,19 @@ static dlrm_status dispatch_w(int M, int N, int K, const void* A, int lda, const
 dlrm_status launch_linear_ffma(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W,
                                dlrm_dtype w_dt, int ldw, const float* bias, void* C, dlrm_dtype c_dt, int ldc,
                                int act, cudaStream_t st) {
+    // fp32 operands whose rows are 16-byte aligned: the cp.async pipeline
+    if (a_dt == DLRM_F32 && w_dt == DLRM_F32 && N > 1 && lda % 4 == 0 && ldw % 4 == 0 &&
+        !((uintptr_t)A & 15) && !((uintptr_t)W & 15)) {
+        const float* a = static_cast<const float*>(A);
+        const float* w = static_cast<const float*>(W);
+        switch (c_dt) {
+            case DLRM_F32: dispatch_f32_pipe<float>(M, N, K, a, lda, w, ldw, bias, C, ldc, act, st); break;
+            case DLRM_BF16: dispatch_f32_pipe<__nv_bfloat16>(M, N, K, a, lda, w, ldw, bias, C, ldc, act, st); break;
+            case DLRM_F16: dispatch_f32_pipe<__half>(M, N, K, a, lda, w, ldw, bias, C, ldc, act, st); break;
+        }
+        DLRM_LAUNCH_CHECK();
+        return DLRM_OK;
+    }
     dlrm_status r = DLRM_ERR_UNSUPPORTED;
     switch (a_dt) {
         case DLRM_F32: r = dispatch_w<float>(M, N, K, A, lda, W, w_dt, ldw, bias, C, c_dt, ldc, act, st); break;
