@@ -85,6 +85,8 @@ def fused_kernel_name(cfg) -> str:
         return "embbag_interact_mma_kernel (dlrm_embbag_interact_fwd)"
     if cfg.table_dtype == "bf16" and cfg.mlp_dtype == "bf16" and cfg.d in (64, 128) and cfg.K <= 128:
         return "embbag_interact_wide_kernel (dlrm_embbag_interact_fwd)"
+    if cfg.table_dtype == "f32" and cfg.d in (16, 32, 64, 128):
+        return "embbag_interact_f32_kernel (dlrm_embbag_interact_fwd)"
     return "embbag_interact_kernel (dlrm_embbag_interact_fwd)"
 
 

@@ -433,6 +433,89 @@ __global__ void __launch_bounds__(256) embbag_interact_kernel(
     report_warp(err, oob, bad);
 }
 
+// ------------------------------------------------------------------ K2 for fp32 tables of d = 4 GL
+
+// fp32 tables with 16-byte rows of d = 16, 32, 64 or 128 floats (the medium and tiny configurations): the
+// generic kernel's interaction on the block's fp32 tile, with a leaner gather. Work items (table k, sample s)
+// are taken NG at a time per warp from a shared counter, one bag per lane group of GL = d/4 lanes (16 bytes
+// of a row per lane); the group walks the bag U rows at a time with the next U indices loaded while the
+// rows are in flight, one range test per row against the table's row count (an index past the bag reads
+// as -1, i.e. out of range), out-of-range indices counted from one bit mask per step, fp32 sums with packed
+// adds, and the pooled row stored as one 16-byte vector per lane into row 1 + k of the sample's tile.
+template <int GL, int U>
+__global__ void __launch_bounds__(256) embbag_interact_f32_kernel(
+    const float* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B, int S, int xs,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
+    const float* __restrict__ x_dense, void* out, int ld, int out_dt, ErrRecord* err) {
+    constexpr int d = 4 * GL;
+    constexpr int NG = 32 / GL;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int n1 = K + 1;
+    float* X = reinterpret_cast<float*>(smem);
+    int* counter = reinterpret_cast<int*>(smem + sizeof(float) * (size_t)S * n1 * xs);
+    const int lane = threadIdx.x & 31;
+    const int g = lane % GL, grp = lane / GL;
+    const int b0 = blockIdx.x * S;
+    const int nb = min(S, B - b0);
+    unsigned oob = 0, bad = 0;
+    if (threadIdx.x == 0) *counter = 0;
+    load_dense_rows(x_dense, d, b0, nb, X, xs, n1);
+    __syncthreads();
+    const int n_items = K * nb;
+    for (;;) {
+        int it0 = 0;
+        if (lane == 0) it0 = atomicAdd(counter, NG);
+        it0 = __shfl_sync(0xffffffffu, it0, 0);
+        if (it0 >= n_items) break;
+        const int it = it0 + grp;
+        if (it >= n_items) continue;
+        const int k = it / nb, s = it - k * nb;
+        const long long o = (long long)k * B + b0 + s;
+        const long long st = offsets[o], en = offsets[o + 1];
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (st < 0 || en < st || en > nnz) {
+            if (g == 0) ++bad;
+        } else {
+            const float* tab = tables + tm.base[k] * (long long)d + 4 * g;
+            const unsigned long long m = (unsigned long long)tm.rows[k];
+            int idx[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) idx[u] = st + u < en ? __ldg(indices + st + u) : -1;
+            for (long long p = st; p < en; p += U) {
+                int nxt[U];
+                if (p + 2 * U <= en) {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) nxt[u] = __ldg(indices + p + U + u);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) nxt[u] = p + U + u < en ? __ldg(indices + p + U + u) : -1;
+                }
+                uint4 v[U];
+                unsigned okm = 0;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const bool ok = (unsigned long long)(unsigned)idx[u] < m;   // -1: past the bag
+                    okm |= (unsigned)ok << u;
+                    v[u] = ok ? ldg16_stream(tab + (long long)idx[u] * d) : make_uint4(0, 0, 0, 0);
+                }
+                if (g == 0) {   // out-of-range indices of the bag (not the slots past its end)
+                    const int n = en - p < U ? (int)(en - p) : U;
+                    oob += __popc(~okm & ((1u << n) - 1u));
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) Chunk16<float>::add(v[u], acc);
+#pragma unroll
+                for (int u = 0; u < U; ++u) idx[u] = nxt[u];
+            }
+        }
+        *reinterpret_cast<float4*>(X + ((long long)s * n1 + 1 + k) * xs + 4 * g) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    __syncthreads();
+    interact_tile(X, xs, K, d, nb, b0, out, ld, out_dt);
+    report_warp(err, oob, bad);
+}
+
 // ------------------------------------------------------------------ host launchers
 
 struct Geometry {
@@ -566,6 +649,46 @@ static dlrm_status launch_fused_t(const TableMeta& tm, const void* tables, int K
     return DLRM_OK;
 }
 
+static dlrm_status launch_fused_f32(const TableMeta& tm, const void* tables, int K, int d, int B,
+                                    const int32_t* offsets, const int32_t* indices, long long nnz,
+                                    const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
+                                    cudaStream_t st) {
+    const size_t per = interact_smem_per_sample(K, d);
+    const float* tb = static_cast<const float*>(tables);
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // S samples per block: as few as keep the whole grid resident at once (one wave: a partial second wave
+    // would leave most SMs idle while it runs), at most 8 and within the shared-memory budget
+#define DLRM_KF(GLV)                                                                                           \
+    {                                                                                                          \
+        auto kern = embbag_interact_f32_kernel<GLV, 8>;                                                        \
+        int S = 1;                                                                                             \
+        for (;; ++S) {                                                                                         \
+            const size_t sm = per * S + 16;                                                                    \
+            if (S > 1 && (S > 8 || sm > kSmemMax)) { --S; break; }                                            \
+            int occ = 0;                                                                                       \
+            if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, sm) != cudaSuccess || occ < 1) occ = 1; \
+            if ((long long)(B + S - 1) / S <= (long long)occ * sms) break;                                    \
+        }                                                                                                      \
+        const size_t smem = per * S + 16;                                                                      \
+        if (smem > kSmemMax) return DLRM_ERR_UNSUPPORTED;                                                      \
+        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+        const dim3 grid((B + S - 1) / S);                                                                      \
+        kern<<<grid, 256, smem, st>>>(tb, tm, K, B, S, xstride(d), offsets, indices, nnz, x_dense, out, ld,    \
+                                      (int)out_dt, err);                                                       \
+    }
+    switch (d) {
+        case 16: DLRM_KF(4) break;
+        case 32: DLRM_KF(8) break;
+        case 64: DLRM_KF(16) break;
+        default: DLRM_KF(32) break;
+    }
+#undef DLRM_KF
+    DLRM_LAUNCH_CHECK();
+    return DLRM_OK;
+}
+
 dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,
                                    const int32_t* offsets, const int32_t* indices, long long nnz,
                                    const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
@@ -575,6 +698,8 @@ dlrm_status launch_embbag_interact(const TableMeta& tm, const void* tables, dlrm
                                           err, st);
     if (embbag_interact_wide_supported(dt, K, d, ld, out, out_dt))
         return launch_embbag_interact_wide(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, err, st);
+    if (dt == DLRM_F32 && (d == 16 || d == 32 || d == 64 || d == 128) && K >= 1)
+        return launch_fused_f32(tm, tables, K, d, B, offsets, indices, nnz, x_dense, out, ld, out_dt, err, st);
     Geometry g;
     if (dt == DLRM_U8ROW || !gather_geometry(d, dt, g)) return DLRM_ERR_UNSUPPORTED;
     switch (dt) {
