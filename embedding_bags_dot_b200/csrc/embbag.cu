@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 
+#include <mutex>
 #include <type_traits>
 
 namespace dlrm {
@@ -649,6 +650,27 @@ static dlrm_status launch_fused_t(const TableMeta& tm, const void* tables, int K
     return DLRM_OK;
 }
 
+// Resident blocks per SM of embbag_interact_f32_kernel<GL> with `smem` bytes of dynamic shared memory: asked
+// of the runtime once per (GL, smem) and kept (a property of the code and the GPU model; one model per process).
+template <typename Query>
+static int f32_occupancy(int gl, size_t smem, Query query) {
+    struct Entry {
+        int gl;
+        size_t smem;
+        int occ;
+    };
+    static Entry cache[32];
+    static int used = 0;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].gl == gl && cache[i].smem == smem) return cache[i].occ;
+    int occ = 1;
+    query(occ);
+    cache[used < 32 ? used++ : (int)(smem % 32)] = Entry{gl, smem, occ};
+    return occ;
+}
+
 static dlrm_status launch_fused_f32(const TableMeta& tm, const void* tables, int K, int d, int B,
                                     const int32_t* offsets, const int32_t* indices, long long nnz,
                                     const float* x_dense, void* out, int ld, dlrm_dtype out_dt, ErrRecord* err,
@@ -666,9 +688,10 @@ static dlrm_status launch_fused_f32(const TableMeta& tm, const void* tables, int
         for (;; ++S) {                                                                                         \
             const size_t sm = per * S + 16;                                                                    \
             if (S > 1 && (S > 8 || sm > kSmemMax)) { --S; break; }                                            \
-            int occ = 0;                                                                                       \
-            if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, sm) != cudaSuccess || occ < 1) occ = 1; \
+            int occ = f32_occupancy(GLV, sm, [&](int& o) {                                                   \
+                if (sm > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+                if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, 256, sm) != cudaSuccess || o < 1) o = 1; \
+            });                                                                                                \
             if ((long long)(B + S - 1) / S <= (long long)occ * sms) break;                                    \
         }                                                                                                      \
         const size_t smem = per * S + 16;                                                                      \
