@@ -448,6 +448,7 @@ __global__ void __launch_bounds__(256) embbag_interact_f32_kernel(
     const float* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B, int S, int xs,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, ErrRecord* err) {
+    pdl_wait();   // programmatic dependent: the previous kernel's outputs are visible from here on
     constexpr int d = 4 * GL;
     constexpr int NG = 32 / GL;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -698,8 +699,8 @@ static dlrm_status launch_fused_f32(const TableMeta& tm, const void* tables, int
         if (smem > kSmemMax) return DLRM_ERR_UNSUPPORTED;                                                      \
         if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         const dim3 grid((B + S - 1) / S);                                                                      \
-        kern<<<grid, 256, smem, st>>>(tb, tm, K, B, S, xstride(d), offsets, indices, nnz, x_dense, out, ld,    \
-                                      (int)out_dt, err);                                                       \
+        (void)launch_pdl(kern, grid, dim3(256), smem, st, tb, tm, K, B, S, xstride(d), offsets, indices, nnz,   \
+                         x_dense, out, ld, (int)out_dt, err);                                                  \
     }
     switch (d) {
         case 16: DLRM_KF(4) break;

@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(CW * 32) embbag_cat_bulk_kernel(const T* __res
                                                                   const int32_t* __restrict__ indices, long long nnz,
                                                                   const float* __restrict__ x_dense, T* __restrict__ out,
                                                                   int ld, int warp_bytes, ErrRecord* err) {
+    pdl_wait();   // programmatic dependent: the previous kernel's outputs are visible from here on
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     T* row = reinterpret_cast<T*>(smem + (size_t)warp * warp_bytes);
@@ -183,8 +184,8 @@ dlrm_status launch_embbag_cat_bulk(const TableMeta& tm, const void* tables, dlrm
     {                                                                                                           \
         auto kern = embbag_cat_bulk_kernel<TT>;                                                                 \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-        kern<<<grid, CW * 32, smem, st>>>(static_cast<const TT*>(tables), tm, K, d, B, offsets, indices, nnz,   \
-                                          x_dense, static_cast<TT*>(out), ld, wb, err);                         \
+        (void)launch_pdl(kern, dim3(grid), dim3(CW * 32), smem, st, static_cast<const TT*>(tables), tm, K, d, B, \
+                         offsets, indices, nnz, x_dense, static_cast<TT*>(out), ld, wb, err);                   \
     }
     if (dt == DLRM_BF16) DLRM_CAT_BULK(__nv_bfloat16) else if (dt == DLRM_F16) DLRM_CAT_BULK(__half) else DLRM_CAT_BULK(float)
 #undef DLRM_CAT_BULK

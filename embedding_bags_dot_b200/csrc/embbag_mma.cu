@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
     const void* __restrict__ tables_v, const __grid_constant__ TableMeta tm, int K, int B,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, int warp_bytes, ErrRecord* err) {
+    pdl_wait();   // programmatic dependent: the previous kernel's outputs are visible from here on
     constexpr int d = 8 * GL;
     constexpr int KP = 16 * MT;
     constexpr int RS = 2 * d + 16;   // bf16 tile row: 2d bytes plus one pad chunk (conflict-free ldmatrix)
@@ -636,8 +637,8 @@ static void launch_mma_t(const TableMeta& tm, const void* tables, int K, int B, 
                          int warp_bytes, size_t smem, ErrRecord* err, cudaStream_t st) {
     auto kern = embbag_interact_mma_kernel<MT, GL, Q>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<(B + S - 1) / S, WARPS * 32, smem, st>>>(tables, tm, K, B, offsets, indices, nnz, x_dense, out, ld, out_dt,
-                                                    warp_bytes, err);
+    (void)launch_pdl(kern, dim3((B + S - 1) / S), dim3(WARPS * 32), smem, st, tables, tm, K, B, offsets, indices, nnz,
+                     x_dense, out, ld, out_dt, warp_bytes, err);
 }
 
 dlrm_status launch_embbag_interact_mma(const TableMeta& tm, const void* tables, dlrm_dtype dt, int K, int d, int B,

@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(WW * 32, 3) embbag_interact_wide_kernel(
     const __nv_bfloat16* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int B, int S,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, __nv_bfloat16* __restrict__ out, int ld, ErrRecord* err) {
+    pdl_wait();   // programmatic dependent: the previous kernel's outputs are visible from here on
     constexpr int d = 8 * GL;
     constexpr int NG = 32 / GL;                   // lane groups per warp
     const WideLayout L = wide_layout(d, MT, ld);
@@ -284,8 +285,8 @@ static void launch_wide_t(const TableMeta& tm, const void* tables, int K, int B,
     const size_t smem = wide_smem(d, MT, ld, S);
     auto kern = embbag_interact_wide_kernel<GL, MT, 8>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<(B + S - 1) / S, WW * 32, smem, st>>>(static_cast<const __nv_bfloat16*>(tables), tm, K, B, S, offsets,
-                                                 indices, nnz, x_dense, static_cast<__nv_bfloat16*>(out), ld, err);
+    (void)launch_pdl(kern, dim3((B + S - 1) / S), dim3(WW * 32), smem, st, static_cast<const __nv_bfloat16*>(tables), tm,
+                     K, B, S, offsets, indices, nnz, x_dense, static_cast<__nv_bfloat16*>(out), ld, err);
 }
 
 dlrm_status launch_embbag_interact_wide(const TableMeta& tm, const void* tables, int K, int d, int B,

@@ -3,20 +3,28 @@
 // the bottom/top MLP layers of DLRM ("Deep Learning Recommendation Model
 // (DLRM)", nadeemcite summary, Key Method Details: FC layers with ReLU).
 //
-// sm_100a design: a persistent kernel, one 192-thread CTA per SM.
-//   warp 0      TMA producer: 128x64 tiles of A and 256x64 tiles of W (both
-//               K-major, 128-byte swizzle) into a 4-stage shared-memory ring;
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
-//               and one thread issues tcgen05.mma (M=128, N=256, K=16);
+// sm_100a design: a persistent kernel, one 320-thread CTA per SM.
+//   warp 0      TMA producer: 128x64 tiles of A and BNTx64 tiles of W (both
+//               K-major, 128-byte swizzle) into a shared-memory ring;
+//   warp 1      allocates 2 BNT TMEM columns (two 128 x BNT fp32
+//               accumulators) and one thread issues tcgen05.mma (M=128,
+//               N=BNT, K=16);
 //   warps 2..9  epilogue: tcgen05.ld of the finished accumulator (each warp
-//               owns the 32 TMEM lanes of its quadrant and half of the
+//               owns the 32 TMEM lanes of its quadrant and a share of the
 //               columns), bias, activation, conversion into a 128-byte
 //               swizzled shared-memory stage written out by TMA bulk tensor
 //               stores, while the MMA warp already fills the other accumulator.
+// Two tile widths: BNT = 256 (4-stage ring), and BNT = 64 (8-stage ring) for
+// small batches, where a layer has few 128-row tiles: four times the CTAs, each
+// streaming a quarter of the weights, with twice the loads in flight. Below 128
+// rows the A box holds only the batch's rows (rounded up to 8); the MMA still
+// reads 128 rows, and the rows past the box only reach accumulator rows that
+// are never stored.
 // Shared-memory stages are released by tcgen05.commit onto an mbarrier. All
 // waits are bounded: on timeout the kernel records DLRM_ERR_TIMEOUT in the
 // error record, drains its own copies and MMAs (again bounded), frees TMEM
-// and returns. No cluster multicast is used.
+// and returns. No cluster multicast is used. Launched as a programmatic
+// dependent: barriers and TMEM are set up before pdl_wait().
 #include <cuda.h>
 
 #include "common.cuh"
@@ -30,23 +38,49 @@ namespace tc {
 // with dlrm_set_wait_polls to make them run out). The drains after a timeout always use WAIT_LIMIT.
 static __device__ long long g_tc1_wait_polls = WAIT_LIMIT;
 
-template <typename TC, int ACT>
+// Shared-memory plan of the single-CTA kernel for tile width BNT.
+template <int BNT>
+struct Tile1 {
+    static constexpr int NS = BNT == BN ? STAGES : 8;     // ring stages
+    static constexpr int W_BYTES = BNT * BK * 2;
+    static constexpr int STAGE = A_BYTES + W_BYTES;
+    static constexpr int TMEM = 2 * BNT;
+    static constexpr int SMEM = NS * STAGE + OUT_BYTES + 1024 + 256;
+    // epilogue columns per warp: half the tile per warp of a quadrant, or the whole tile for the first
+    // warp when half of it is narrower than one 128-byte chunk of 16-bit output
+    static constexpr int WC = BNT >= 128 ? BNT / 2 : BNT;
+};
+
+template <int NS>
+struct BarsN {
+    unsigned long long full[NS];
+    unsigned long long empty[NS];
+    unsigned long long tfull[2];
+    unsigned long long tempty[2];
+    unsigned long long drain;
+    unsigned int tmem_base;
+    int abort;
+};
+
+template <typename TC, int ACT, int BNT>
 __global__ void __launch_bounds__(THREADS, 1)
     linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW,
                      const __grid_constant__ CUtensorMap mapC, int M, int N, int K, const float* __restrict__ bias,
-                     uint32_t id, ErrRecord* err) {
+                     uint32_t id, uint32_t a_tx, ErrRecord* err) {
+    using T = Tile1<BNT>;
+    constexpr int NS = T::NS;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    Bars* bars = reinterpret_cast<Bars*>(gbase + STAGES * STAGE_BYTES + OUT_BYTES);
+    BarsN<NS>* bars = reinterpret_cast<BarsN<NS>*>(gbase + NS * T::STAGE + OUT_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nbn = (N + BN - 1) / BN;
+    const int nbn = (N + BNT - 1) / BNT;
     const int ntiles = ((M + BM - 1) / BM) * nbn;
     const int nk = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
@@ -60,12 +94,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars->tmem_base)),
-                     "r"(TMEM_COLS));
+                     "r"(T::TMEM));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW)) : "memory");
     }
     fence_before();
     __syncthreads();
     fence_after();
+    pdl_wait();      // the previous kernel's outputs (A) are complete and visible from here on
     const uint32_t tmem = bars->tmem_base;
     volatile int* abort = &bars->abort;
     bool timed_out = false;
@@ -73,8 +112,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapA)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapW)) : "memory");
             int s = 0;
             uint32_t ph = 0;
             for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x) {
@@ -84,11 +121,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         timed_out = true;
                         break;
                     }
-                    const uint32_t sa = base + s * STAGE_BYTES;
-                    mbar_expect_tx(&bars->full[s], STAGE_BYTES);
+                    const uint32_t sa = base + s * T::STAGE;
+                    mbar_expect_tx(&bars->full[s], a_tx + T::W_BYTES);
                     tma_load_2d(sa, &mapA, &bars->full[s], kb * BK, mb * BM);
-                    tma_load_2d(sa + A_BYTES, &mapW, &bars->full[s], kb * BK, nb * BN);
-                    if (++s == STAGES) {
+                    tma_load_2d(sa + A_BYTES, &mapW, &bars->full[s], kb * BK, nb * BNT);
+                    if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -98,9 +135,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             // drain, also when another role gave up: every stage whose load may still be in flight
             // completes its full phase before the CTA may exit (a stage never loaded, or already
             // consumed, passes at once)
-            for (int q = 0; q < STAGES; ++q) {
+            for (int q = 0; q < NS; ++q) {
                 if (--s < 0) {
-                    s = STAGES - 1;
+                    s = NS - 1;
                     ph ^= 1u;
                 }
                 mbar_wait(&bars->full[s], ph, abort, true);
@@ -120,19 +157,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 fence_after();
-                const uint32_t d = tmem + (uint32_t)(acc * BN);
+                const uint32_t d = tmem + (uint32_t)(acc * BNT);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait_n(&bars->full[s], ph, abort, lim)) {
                         timed_out = true;
                         break;
                     }
                     fence_after();
-                    const uint32_t sa = base + s * STAGE_BYTES;
+                    const uint32_t sa = base + s * T::STAGE;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
                         umma(d, sdesc(sa + k * 32), sdesc(sa + A_BYTES + k * 32), id_, (kb | k) != 0);
                     umma_commit(&bars->empty[s]);
-                    if (++s == STAGES) {
+                    if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -148,9 +185,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         const int ew = warp - 2;   // epilogue warp 0..7
         const int q = warp & 3;    // TMEM lane quadrant this warp may access
-        const int h = ew >> 2;     // which half of the tile's columns
-        unsigned char* stage = gbase + STAGES * STAGE_BYTES + ew * STAGE_OUT_BYTES;
-        const uint32_t stage_s = base + STAGES * STAGE_BYTES + ew * STAGE_OUT_BYTES;
+        const int h = ew >> 2;     // which share of the tile's columns
+        const bool active = h * T::WC < BNT;
+        unsigned char* stage = gbase + NS * T::STAGE + ew * STAGE_OUT_BYTES;
+        const uint32_t stage_s = base + NS * T::STAGE + ew * STAGE_OUT_BYTES;
         int i = 0;
         for (int t = blockIdx.x; t < ntiles && !timed_out; t += gridDim.x, ++i) {
             const int acc = i & 1;
@@ -160,10 +198,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             }
             fence_after();
-            const int mb = t / nbn, nb = t - mb * nbn;
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + h * (BN / 2));
-            epilogue_tma<TC, ACT, BN / 2>(taddr, mb * BM + q * 32, nb * BN + h * (BN / 2), N, bias, &mapC, stage,
-                                          stage_s);
+            if (active) {
+                const int mb = t / nbn, nb = t - mb * nbn;
+                const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BNT + h * T::WC);
+                epilogue_tma<TC, ACT, T::WC>(taddr, mb * BM + q * 32, nb * BNT + h * T::WC, N, bias, &mapC, stage,
+                                             stage_s);
+            }
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->tempty[acc]);
@@ -177,7 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(T::TMEM));
     }
 }
 
@@ -244,6 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                      "r"(TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
+    pdl_wait();      // the previous kernel's outputs (A) are complete and visible from here on
     if constexpr (ACT == ACT_RELU_LOGIT) {
         // each epilogue warp's (unused) output stage: [0, 128) bias and [128, 256) w of its 128 columns;
         // the quadrant's first warp also holds the exchange slots [256, 320): two tile parities x 32 rows
@@ -453,15 +494,15 @@ static int sm_count() {
     return n[dev];
 }
 
-template <typename TC, int ACT>
+template <typename TC, int ACT, int BNT>
 static dlrm_status launch_t(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& mc, int M, int N, int K,
-                            const float* bias, uint32_t id, ErrRecord* err, cudaStream_t st) {
-    auto kern = linear_tc_kernel<TC, ACT>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    const int ntiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+                            const float* bias, uint32_t id, uint32_t a_tx, ErrRecord* err, cudaStream_t st) {
+    auto kern = linear_tc_kernel<TC, ACT, BNT>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile1<BNT>::SMEM);
+    const int ntiles = ((M + BM - 1) / BM) * ((N + BNT - 1) / BNT);
     const int grid = ntiles < sm_count() ? ntiles : sm_count();
-    kern<<<grid, THREADS, SMEM_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err);
-    DLRM_LAUNCH_CHECK();
+    DLRM_PDL_CHECK(launch_pdl(kern, dim3(grid), dim3(THREADS), (size_t)Tile1<BNT>::SMEM, st, ma, mw, mc, M, N, K, bias,
+                              id, a_tx, err));
     return DLRM_OK;
 }
 
@@ -474,8 +515,8 @@ static dlrm_status launch_t2(const CUtensorMap& ma, const CUtensorMap& mw, const
     const int ntiles = ((M + 255) / 256) * ((N + BN2 - 1) / BN2);
     const int pairs = sm_count() / 2;
     const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS, SMEM2_BYTES, st>>>(ma, mw, mc, M, N, K, bias, id, err, la);
-    DLRM_LAUNCH_CHECK();
+    DLRM_PDL_CHECK(launch_pdl(kern, dim3(grid), dim3(THREADS), (size_t)SMEM2_BYTES, st, ma, mw, mc, M, N, K, bias, id,
+                              err, la));
     return DLRM_OK;
 }
 
@@ -524,26 +565,28 @@ bool linear_tc_supported(int M, int N, int K, const void* A, dlrm_dtype a_dt, in
 dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt, int lda, const void* W, int ldw,
                              const float* bias, void* C, dlrm_dtype c_dt, int ldc, int act, ErrRecord* err,
                              cudaStream_t st) {
-    // 256-row tiles on SM pairs when there are enough of them to fill the GPU, 128-row tiles otherwise
+    // 256-row tiles on SM pairs when there are enough of them to fill the GPU; otherwise 128-row tiles,
+    // 64 columns wide when 256-wide tiles would leave most SMs idle
     const bool pair = M >= 256 * 16;
+    const bool narrow = !pair && (long long)((M + tc::BM - 1) / tc::BM) * ((N + tc::BN - 1) / tc::BN) * 2 <= tc::sm_count();
+    const int bnt = pair ? tc::BN2 / 2 : narrow ? 64 : tc::BN;
+    // A box: the batch's rows (rounded up to 8) when they fit one tile, else a whole tile
+    const int a_rows = M < tc::BM ? (M + 7) & ~7 : tc::BM;
     CUtensorMap ma, mw, mc;
-    if (!tc::make_map(&ma, A, a_dt, K, M, lda, tc::BM) ||
-        !tc::make_map(&mw, W, a_dt, K, N, ldw, pair ? tc::BN2 / 2 : tc::BN) ||
+    if (!tc::make_map(&ma, A, a_dt, K, M, lda, pair ? tc::BM : a_rows) || !tc::make_map(&mw, W, a_dt, K, N, ldw, bnt) ||
         !tc::make_map(&mc, C, c_dt, N, M, ldc, 32, c_dt == DLRM_F32 ? 32 : 64))
         return DLRM_ERR_CUDA;
     const int fmt = a_dt == DLRM_BF16 ? 1 : 0;
-    const uint32_t id = pair ? tc::idesc2(fmt) : tc::idesc(fmt);
-#define DLRM_TC(TC)                                                                                             \
-    switch (act) {                                                                                              \
-        case DLRM_ACT_RELU:                                                                                     \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_RELU>(ma, mw, mc, M, N, K, bias, id, err, st)              \
-                        : tc::launch_t<TC, DLRM_ACT_RELU>(ma, mw, mc, M, N, K, bias, id, err, st);              \
-        case DLRM_ACT_SIGMOID:                                                                                  \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_SIGMOID>(ma, mw, mc, M, N, K, bias, id, err, st)           \
-                        : tc::launch_t<TC, DLRM_ACT_SIGMOID>(ma, mw, mc, M, N, K, bias, id, err, st);           \
-        default:                                                                                                \
-            return pair ? tc::launch_t2<TC, DLRM_ACT_NONE>(ma, mw, mc, M, N, K, bias, id, err, st)              \
-                        : tc::launch_t<TC, DLRM_ACT_NONE>(ma, mw, mc, M, N, K, bias, id, err, st);              \
+    const uint32_t a_tx = (uint32_t)a_rows * tc::BK * 2;
+#define DLRM_TC_ACT(TC, ACT)                                                                                    \
+    return pair     ? tc::launch_t2<TC, ACT>(ma, mw, mc, M, N, K, bias, tc::idesc2(fmt), err, st)               \
+           : narrow ? tc::launch_t<TC, ACT, 64>(ma, mw, mc, M, N, K, bias, tc::idesc(fmt, 64), a_tx, err, st)   \
+                    : tc::launch_t<TC, ACT, tc::BN>(ma, mw, mc, M, N, K, bias, tc::idesc(fmt), a_tx, err, st);
+#define DLRM_TC(TC)                                       \
+    switch (act) {                                        \
+        case DLRM_ACT_RELU: DLRM_TC_ACT(TC, DLRM_ACT_RELU)       \
+        case DLRM_ACT_SIGMOID: DLRM_TC_ACT(TC, DLRM_ACT_SIGMOID) \
+        default: DLRM_TC_ACT(TC, DLRM_ACT_NONE)                  \
     }
     if (c_dt == DLRM_F32) {
         DLRM_TC(float)
@@ -553,6 +596,7 @@ dlrm_status launch_linear_tc(int M, int N, int K, const void* A, dlrm_dtype a_dt
         DLRM_TC(__half)
     }
 #undef DLRM_TC
+#undef DLRM_TC_ACT
 }
 
 }  // namespace dlrm

@@ -6,6 +6,8 @@
 // This file holds the CUDA-core paths: a tiled FFMA GEMM used for fp32
 // layers and for layers the tensor-core path does not take, and a
 // warp-per-row GEMV for the single-logit last layer with its activation.
+// Every kernel here is launched as a programmatic dependent and waits
+// (pdl_wait) before its first access to global memory.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -28,6 +30,7 @@ __global__ void __launch_bounds__(256) linear_ffma_kernel(int M, int N, int K, c
                                                           const TW* __restrict__ W, int ldw,
                                                           const float* __restrict__ bias, TC* __restrict__ C,
                                                           int ldc) {
+    pdl_wait();
     constexpr int RM = 64, TM = 4;   // tile rows, output rows per thread
     __shared__ __align__(16) float As[2][16][RM + 4];
     __shared__ __align__(16) float Ws[2][16][64 + 4];
@@ -117,6 +120,7 @@ __global__ void __launch_bounds__(256) linear_f32_pipe_kernel(int M, int N, int 
                                                               int lda, const float* __restrict__ W, int ldw,
                                                               const float* __restrict__ bias, TC* __restrict__ C,
                                                               int ldc) {
+    pdl_wait();
     using namespace f32p;
     constexpr int TM = RM / 16;   // output rows per thread
     extern __shared__ __align__(16) float fsm[];
@@ -203,12 +207,14 @@ static void run_f32_pipe(int M, int N, int K, const float* A, int lda, const flo
         auto kern = linear_f32_pipe_kernel<TC, ACT, 32>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, f32p::SMEM);
         const dim3 grid((N + 63) / 64, (M + 31) / 32);
-        kern<<<grid, 256, f32p::SMEM, st>>>(M, N, K, A, lda, W, ldw, bias, static_cast<TC*>(C), ldc);
+        (void)launch_pdl(kern, grid, dim3(256), (size_t)f32p::SMEM, st, M, N, K, A, lda, W, ldw, bias,
+                         static_cast<TC*>(C), ldc);
     } else {
         auto kern = linear_f32_pipe_kernel<TC, ACT, 64>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, f32p::SMEM);
         const dim3 grid((N + 63) / 64, (M + 63) / 64);
-        kern<<<grid, 256, f32p::SMEM, st>>>(M, N, K, A, lda, W, ldw, bias, static_cast<TC*>(C), ldc);
+        (void)launch_pdl(kern, grid, dim3(256), (size_t)f32p::SMEM, st, M, N, K, A, lda, W, ldw, bias,
+                         static_cast<TC*>(C), ldc);
     }
 }
 
@@ -225,6 +231,7 @@ template <typename TA, typename TW, int ACT>
 __global__ void __launch_bounds__(256) gemv_kernel(int M, int K, const TA* __restrict__ A, int lda,
                                                    const TW* __restrict__ w, const float* __restrict__ bias,
                                                    float* __restrict__ y, int ldy) {
+    pdl_wait();
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= M) return;
@@ -239,16 +246,15 @@ template <typename TA, typename TW, typename TC, int ACT>
 static void run_ffma(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const float* bias, void* C,
                      int ldc, cudaStream_t st) {
     const dim3 grid((N + 63) / 64, (M + 63) / 64);
-    linear_ffma_kernel<TA, TW, TC, ACT><<<grid, 256, 0, st>>>(M, N, K, static_cast<const TA*>(A), lda,
-                                                              static_cast<const TW*>(W), ldw, bias,
-                                                              static_cast<TC*>(C), ldc);
+    (void)launch_pdl(linear_ffma_kernel<TA, TW, TC, ACT>, grid, dim3(256), 0, st, M, N, K, static_cast<const TA*>(A),
+                     lda, static_cast<const TW*>(W), ldw, bias, static_cast<TC*>(C), ldc);
 }
 
 template <typename TA, typename TW, int ACT>
 static void run_gemv(int M, int K, const void* A, int lda, const void* W, const float* bias, void* C, int ldc,
                      cudaStream_t st) {
-    gemv_kernel<TA, TW, ACT><<<(M + 7) / 8, 256, 0, st>>>(M, K, static_cast<const TA*>(A), lda,
-                                                          static_cast<const TW*>(W), bias, static_cast<float*>(C), ldc);
+    (void)launch_pdl(gemv_kernel<TA, TW, ACT>, dim3((M + 7) / 8), dim3(256), 0, st, M, K, static_cast<const TA*>(A),
+                     lda, static_cast<const TW*>(W), bias, static_cast<float*>(C), ldc);
 }
 
 template <typename TA, typename TW, typename TC>
@@ -317,6 +323,7 @@ dlrm_status launch_linear_ffma(int M, int N, int K, const void* A, dlrm_dtype a_
 // out[b][c] = in[b][c] converted to out_dt for c < K, 0 for K <= c < ldo.
 template <typename TI, typename TO>
 __global__ void convert_kernel(int B, int K, const TI* __restrict__ in, int ldi, TO* __restrict__ out, int ldo) {
+    pdl_wait();
     const long long n = (long long)B * ldo;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
         const long long b = q / ldo;
@@ -329,6 +336,7 @@ __global__ void convert_kernel(int B, int K, const TI* __restrict__ in, int ldi,
 // no per-element index division.
 template <typename TI, typename TO>
 __global__ void convert_rows_kernel(int B, int K, const TI* __restrict__ in, int ldi, TO* __restrict__ out, int ldo) {
+    pdl_wait();
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
         const TI* src = in + (long long)b * ldi;
         TO* dst = out + (long long)b * ldo;
@@ -347,9 +355,11 @@ static void convert_to(int B, int K, const void* in, int ldi, void* out, dlrm_dt
         const int blocks = (B + 255) / 256 < 148 * 8 ? (B + 255) / 256 : 148 * 8;
         const TI* i = static_cast<const TI*>(in);
         if (out_dt == DLRM_BF16)
-            convert_rows_kernel<TI, __nv_bfloat16><<<blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__nv_bfloat16*>(out), ldo);
+            (void)launch_pdl(convert_rows_kernel<TI, __nv_bfloat16>, dim3(blocks), dim3(256), 0, st, B, K, i, ldi,
+                             static_cast<__nv_bfloat16*>(out), ldo);
         else
-            convert_rows_kernel<TI, __half><<<blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__half*>(out), ldo);
+            (void)launch_pdl(convert_rows_kernel<TI, __half>, dim3(blocks), dim3(256), 0, st, B, K, i, ldi,
+                             static_cast<__half*>(out), ldo);
         return;
     }
     long long blocks = ((long long)B * ldo + 255) / 256;
@@ -357,11 +367,14 @@ static void convert_to(int B, int K, const void* in, int ldi, void* out, dlrm_dt
     if (blocks < 1) blocks = 1;
     const TI* i = static_cast<const TI*>(in);
     if (out_dt == DLRM_BF16)
-        convert_kernel<TI, __nv_bfloat16><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__nv_bfloat16*>(out), ldo);
+        (void)launch_pdl(convert_kernel<TI, __nv_bfloat16>, dim3((int)blocks), dim3(256), 0, st, B, K, i, ldi,
+                         static_cast<__nv_bfloat16*>(out), ldo);
     else if (out_dt == DLRM_F16)
-        convert_kernel<TI, __half><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<__half*>(out), ldo);
+        (void)launch_pdl(convert_kernel<TI, __half>, dim3((int)blocks), dim3(256), 0, st, B, K, i, ldi,
+                         static_cast<__half*>(out), ldo);
     else
-        convert_kernel<TI, float><<<(int)blocks, 256, 0, st>>>(B, K, i, ldi, static_cast<float*>(out), ldo);
+        (void)launch_pdl(convert_kernel<TI, float>, dim3((int)blocks), dim3(256), 0, st, B, K, i, ldi,
+                         static_cast<float*>(out), ldo);
 }
 
 dlrm_status launch_convert(int B, int K, const void* in, dlrm_dtype in_dt, int ldi, void* out, dlrm_dtype out_dt,

@@ -26,7 +26,8 @@
 // TMEM: layer-2 accumulator [0, 256), layer-3 accumulators [256, 384) and
 // [384, 512). Biases sit in shared memory. All waits are bounded: on timeout
 // the kernel records DLRM_ERR_TIMEOUT, drains its own copies and MMAs, frees
-// TMEM and returns.
+// TMEM and returns. Launched as a programmatic dependent: barriers and TMEM are
+// set up before pdl_wait().
 #include <cuda.h>
 
 #include "common.cuh"
@@ -155,13 +156,14 @@ __global__ void __launch_bounds__(M3_THREADS, 1)
         bars->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int c = threadIdx.x; c < n1 + n2 + n3; c += blockDim.x)
-        bias_s[c] = c < n1 ? __ldg(b1 + c) : c < n1 + n2 ? __ldg(b2 + c - n1) : __ldg(b3 + c - n1 - n2);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&bars->tmem_base)),
                      "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    pdl_wait();      // the previous kernel on the stream has completed; global memory from here on
+    for (int c = threadIdx.x; c < n1 + n2 + n3; c += blockDim.x)
+        bias_s[c] = c < n1 ? __ldg(b1 + c) : c < n1 + n2 ? __ldg(b2 + c - n1) : __ldg(b3 + c - n1 - n2);
     fence_before();
     __syncthreads();
     fence_after();
@@ -491,9 +493,8 @@ dlrm_status launch_mlp3_tc(const dlrm_mlp* m, int B, const float* in, int ld_in,
     cudaFuncSetAttribute(tc::mlp3_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::M3_SMEM);
     const int ntiles = (B + tc::BM - 1) / tc::BM;
     const int grid = ntiles < tc::sm_count_here() ? ntiles : tc::sm_count_here();
-    tc::mlp3_tc_kernel<<<grid, tc::M3_THREADS, tc::M3_SMEM, st>>>(m1, m2, m3, in, ld_in, n0, B, n1, n2, n3, m->b[0],
-                                                                  m->b[1], m->b[2], out, ld_out, err);
-    DLRM_LAUNCH_CHECK();
+    DLRM_PDL_CHECK(launch_pdl(tc::mlp3_tc_kernel, dim3(grid), dim3(tc::M3_THREADS), (size_t)tc::M3_SMEM, st, m1, m2, m3,
+                              in, ld_in, n0, B, n1, n2, n3, m->b[0], m->b[1], m->b[2], out, ld_out, err));
     return DLRM_OK;
 }
 

@@ -88,9 +88,9 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {
     return d;
 }
 
-// kind::f16 instruction descriptor: fp32 accumulate, A/B bf16 (1) or fp16 (0), both K-major.
-__host__ __device__ constexpr uint32_t idesc(int ab_fmt) {
-    return (1u << 4) | ((uint32_t)ab_fmt << 7) | ((uint32_t)ab_fmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+// kind::f16 instruction descriptor: fp32 accumulate, A/B bf16 (1) or fp16 (0), both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc(int ab_fmt, int n = BN) {
+    return (1u << 4) | ((uint32_t)ab_fmt << 7) | ((uint32_t)ab_fmt << 10) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(BM >> 4) << 24);
 }
 

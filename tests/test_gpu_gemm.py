@@ -29,11 +29,14 @@ def _layer(M, N, K, dt, seed):
     return x, W, b, ld
 
 
-# M >= 4096 takes the SM-pair (cta_group::2, 256x256 tile) kernel, smaller M the single-SM one
+# M >= 4096 takes the SM-pair (cta_group::2, 256x256 tile) kernel, smaller M the single-SM one: 128 x 64
+# tiles while 128 x 256 tiles would fill at most half the SMs (below 128 rows the A box holds only the
+# batch's rows), 128 x 256 tiles otherwise ((3000, 1024, 479), (4000, 600, 100))
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (333, 200, 100), (1000, 1024, 479), (65, 40, 16),
                                    (4096, 512, 1024), (300, 768, 256), (129, 257, 65),
                                    (5000, 300, 200), (8192, 1024, 479), (4100, 40, 16), (70000, 256, 512),
-                                   (5000, 512, 13), (100, 64, 5)])
+                                   (5000, 512, 13), (100, 64, 5), (3000, 1024, 479), (4000, 600, 100),
+                                   (2, 1000, 1024)])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 def test_linear_tc_fp32_out(M, N, K, dt):
     x, W, b, ld = _layer(M, N, K, dt, seed=M * 7 + N + K)
