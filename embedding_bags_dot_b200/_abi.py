@@ -267,13 +267,26 @@ def dlrm_embbag_interact_fwd(T: Tables, B: int, offsets, indices, x_dense, conca
                                                  _nbytes(ws), _stream(stream)), "dlrm_embbag_interact_fwd")
 
 
+def _need(t, dtype, rows: int, ld: int, width: int, where: str) -> None:
+    """Refuses a buffer of the wrong dtype, or too short for `rows` rows of `width` values `ld` apart: the C
+    entry points receive bare pointers and would read or write past its end."""
+    if t is None or (dtype is not None and t.dtype != dtype) or \
+            (rows > 0 and t.numel() < (rows - 1) * ld + width):
+        raise DlrmError(ERR_INVALID_ARG, where)
+
+
 def dlrm_mlp_fwd(mlp: MLP, B: int, inp, ld_in: int, out, ld_out: int, final_act: int, ws, stream=None):
+    """out: fp32 [B][ld_out] (the last layer's output is always fp32); inp: [B][ld_in] fp32 or the MLP dtype."""
+    _need(inp, None, int(B), int(ld_in), mlp.dims[0], "dlrm_mlp_fwd")
+    _need(out, torch.float32, int(B), int(ld_out), mlp.dims[-1], "dlrm_mlp_fwd")
     return _check(lib().dlrm_mlp_fwd(mlp.ref(), int(B), _ptr(inp), DT_CODE[inp.dtype], int(ld_in), _ptr(out),
                                      int(ld_out), int(final_act), _ptr(ws), _nbytes(ws), _stream(stream)),
                   "dlrm_mlp_fwd")
 
 
 def dlrm_forward(T: Tables, bot: MLP, top: MLP, B: int, dense, offsets, indices, y_hat, ws, stream=None):
+    _need(dense, torch.float32, int(B), bot.dims[0], bot.dims[0], "dlrm_forward")
+    _need(y_hat, torch.float32, int(B), 1, 1, "dlrm_forward")
     return _check(lib().dlrm_forward(T.ref(), bot.ref(), top.ref(), int(B), _ptr(dense), _ptr(offsets),
                                      _ptr(indices), int(indices.numel()), _ptr(y_hat), _ptr(ws), _nbytes(ws),
                                      _stream(stream)), "dlrm_forward")

@@ -190,6 +190,25 @@ def test_bindings_pass_the_buffer_size_through(lib):
     assert E.dlrm_launch_count() == before
 
 
+def test_bindings_refuse_a_mistyped_or_short_tensor(lib):
+    """The C entry points take bare pointers; the binding refuses, before any launch, an MLP output that is
+    not fp32 (the last layer always writes fp32) or too short, and a too-short input. A bf16 output buffer,
+    half the bytes the layer writes, once made an experiment write past its end on the GPU."""
+    import embedding_bags_dot_b200 as E
+    mlp = _cpu_mlp([479, 1024], "bf16")
+    B = 64
+    ws = torch.zeros(E.dlrm_mlp_workspace_size(mlp, B, torch.bfloat16), dtype=torch.uint8)
+    x = torch.zeros((B, 480), dtype=torch.bfloat16)
+    before = E.dlrm_launch_count()
+    for inp, out in [(x, torch.zeros((B, 1024), dtype=torch.bfloat16)),        # output not fp32
+                     (x, torch.zeros((B - 1, 1024))),                          # output one row short
+                     (x[: B - 1], torch.zeros((B, 1024)))]:                    # input one row short
+        with pytest.raises(E.DlrmError) as e:
+            E.dlrm_mlp_fwd(mlp, B, inp, 480, out, 1024, E.ACT_RELU, ws, stream=0)
+        assert e.value.status == E.ERR_INVALID_ARG
+    assert E.dlrm_launch_count() == before
+
+
 def test_lengths_workspace_and_argument_checks(lib):
     """dlrm_offsets_from_lengths needs the error record plus one int per 8,192-length chunk (and one more);
     the bindings refuse lengths that are not uint8 and offsets that are not int32 or too short, before
