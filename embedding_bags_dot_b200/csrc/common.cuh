@@ -116,7 +116,7 @@ struct TableMeta {
 };
 
 // ----------------------------------------------------------------- programmatic dependent launch
-// The kernels of the forward pass are launched with programmatic stream
+// Every kernel of this library is launched with programmatic stream
 // serialisation (launch_pdl): a kernel is scheduled as soon as every block of
 // the kernel before it on the stream has exited (the implicit trigger at a
 // block's exit, not the kernel's completion), and sets up its shared

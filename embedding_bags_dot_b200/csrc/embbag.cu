@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(256) embbag_kernel(const T* __restrict__ table
                                                      const int32_t* __restrict__ indices, long long nnz,
                                                      float* __restrict__ pooled, int32_t* __restrict__ bag_len,
                                                      ErrRecord* err) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char smem[];
     int* off_s = reinterpret_cast<int*>(smem);
     unsigned char* bad_s = smem + sizeof(int) * K * (S + 1);
@@ -313,6 +314,7 @@ __global__ void __launch_bounds__(256) embbag_cat_kernel(const T* __restrict__ t
                                                          const int32_t* __restrict__ indices, long long nnz,
                                                          const float* __restrict__ x_dense, OT* __restrict__ out, int ld,
                                                          bool vec_ok, ErrRecord* err) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char smem[];
     int* off_s = reinterpret_cast<int*>(smem);
     unsigned char* bad_s = smem + sizeof(int) * K * (S + 1);
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(256) interact_kernel(int B, int K, int d, int 
                                                        const float* __restrict__ x_dense,
                                                        const float* __restrict__ pooled, void* out, int ld,
                                                        int out_dt) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char smem[];
     float* X = reinterpret_cast<float*>(smem);
     const int b0 = blockIdx.x * S;
@@ -412,6 +415,7 @@ __global__ void __launch_bounds__(256) embbag_interact_kernel(
     const T* __restrict__ tables, const __grid_constant__ TableMeta tm, int K, int d, int n_ch, int GL, int B, int S,
     int xs, const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ x_dense, void* out, int ld, int out_dt, ErrRecord* err) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char smem[];
     const int n1 = K + 1;
     float* X = reinterpret_cast<float*>(smem);
@@ -576,7 +580,7 @@ static dlrm_status launch_embbag_t(const TableMeta& tm, const void* tables, int 
     {                                                                                                      \
         auto kern = embbag_kernel<T, VEC, NCH>;                                                            \
         if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        kern<<<grid, 256, smem, st>>>(tb, tm, K, d, g.n_ch, g.GL, B, S, offsets, indices, nnz, pooled, bag_len, err); \
+        (void)launch_pdl(kern, dim3(grid), dim3(256), (size_t)(smem), st, tb, tm, K, d, g.n_ch, g.GL, B, S, offsets, indices, nnz, pooled, bag_len, err); \
     }
     if (g.vec) {
         if (g.NCH == 1) DLRM_K1(true, 1) else if (g.NCH == 2) DLRM_K1(true, 2) else DLRM_K1(true, 4)
@@ -611,7 +615,7 @@ dlrm_status launch_interact(int B, int K, int d, const float* x_dense, const flo
     S = S < 1 ? 1 : (S > 8 ? 8 : S);
     const size_t smem = per * S;
     if (smem > 48 * 1024) cudaFuncSetAttribute(interact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    interact_kernel<<<(B + S - 1) / S, 256, smem, st>>>(B, K, d, S, xstride(d), x_dense, pooled, out, ld, (int)out_dt);
+    (void)launch_pdl(interact_kernel, dim3((B + S - 1) / S), dim3(256), (size_t)(smem), st, B, K, d, S, xstride(d), x_dense, pooled, out, ld, (int)out_dt);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -637,7 +641,7 @@ static dlrm_status launch_fused_t(const TableMeta& tm, const void* tables, int K
     {                                                                                                      \
         auto kern = embbag_interact_kernel<T, VEC, NCH>;                                                   \
         if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        kern<<<grid, 256, smem, st>>>(tb, tm, K, d, g.n_ch, g.GL, B, S, xstride(d), offsets, indices, nnz, x_dense, \
+        (void)launch_pdl(kern, dim3(grid), dim3(256), (size_t)(smem), st, tb, tm, K, d, g.n_ch, g.GL, B, S, xstride(d), offsets, indices, nnz, x_dense, \
                                       out, ld, (int)out_dt, err);                                         \
     }
     if (g.vec) {
@@ -748,7 +752,7 @@ static dlrm_status launch_cat_t(const TableMeta& tm, const void* tables, int K, 
     {                                                                                                            \
         auto kern = embbag_cat_kernel<T, VEC, NCH, OT>;                                                          \
         if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        kern<<<grid, 256, smem, st>>>(tb, tm, K, d, g.n_ch, g.GL, B, S, offsets, indices, nnz, x_dense, o, ld,   \
+        (void)launch_pdl(kern, dim3(grid), dim3(256), (size_t)(smem), st, tb, tm, K, d, g.n_ch, g.GL, B, S, offsets, indices, nnz, x_dense, o, ld,   \
                                       vec_ok, err);                                                              \
     }
     if (g.vec) {

@@ -303,6 +303,7 @@ template <bool AMN, bool BMN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS3, 1)
     gemm3x_kernel(const __grid_constant__ Maps3 maps, int I, int J, int R, int r_chunk, int S, const Epi3Args ea,
                   ErrRecord* err) {
+    pdl_wait();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = su32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -533,7 +534,7 @@ dlrm_status launch3(const Maps3& maps, int I, int J, int R, int r_chunk, int S, 
     const long long ntiles = (long long)((I + 255) / 256) * ((J + 255) / 256) * S;
     const int pairs = sm_count3() / 2;
     const int grid = 2 * (int)(ntiles < pairs ? ntiles : pairs);
-    kern<<<grid, THREADS3, SMEM3_BYTES, st>>>(maps, I, J, R, r_chunk, S, ea, err);
+    (void)launch_pdl(kern, dim3(grid), dim3(THREADS3), (size_t)(SMEM3_BYTES), st, maps, I, J, R, r_chunk, S, ea, err);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }

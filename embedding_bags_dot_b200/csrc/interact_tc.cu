@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(FW * 32, 2) interact_fwd_tc_kernel(
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ indices, long long nnz,
     const float* __restrict__ xh, const float* __restrict__ xl, int ldx, float* __restrict__ ch,
     float* __restrict__ cl, int ldc, int warp_bytes, ErrRecord* err) {
+    pdl_wait();
     constexpr int RS = D + 4;        // X row stride in floats: rows 16 bytes apart modulo 128 (conflict-free ldmatrix)
     constexpr int GS = KP + 8;       // G row stride in floats
     constexpr uint32_t ZERO_SLOT = KP * GS;
@@ -282,6 +283,7 @@ __global__ void __launch_bounds__(BW * 32, 3) interact_bwd_fma_kernel(
     const float* __restrict__ xh, const float* __restrict__ xl, int ldx, const float* __restrict__ dcat, int ldc,
     float* __restrict__ dxh, float* __restrict__ dxl, int lddx, float* __restrict__ dE, int warp_bytes,
     ErrRecord* err) {
+    pdl_wait();
     constexpr int K = N1 - 1;
     constexpr int D = 32 * V;
     constexpr int SR = (N1 + 3) / 4 * 4;   // row stride of the symmetric dZ matrix
@@ -464,7 +466,7 @@ dlrm_status launch_interact_fwd_tc(const TableMeta& tm, const float* tables, int
     {                                                                                                      \
         auto kern = interact_fwd_tc_kernel<DV>;                                                            \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                \
-        kern<<<grid, FW * 32, smem, st>>>(tables, tm, K, B, offsets, indices, nnz, x_dense.hi, x_dense.lo, \
+        (void)launch_pdl(kern, dim3(grid), dim3(FW * 32), (size_t)(smem), st, tables, tm, K, B, offsets, indices, nnz, x_dense.hi, x_dense.lo, \
                                           x_dense.ld, concat_hi, concat_lo, ldc, wb, err);                 \
     }
     if (d == 128) DLRM_FWD_TC(128) else DLRM_FWD_TC(64)
@@ -487,7 +489,7 @@ dlrm_status launch_interact_bwd_tc(const TableMeta& tm, const float* tables, int
     {                                                                                                        \
         auto kern = interact_bwd_fma_kernel<27, VV>;                                                         \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                  \
-        kern<<<grid, BW * 32, smem, st>>>(tables, tm, B, offsets, indices, nnz, x_dense.hi, x_dense.lo,      \
+        (void)launch_pdl(kern, dim3(grid), dim3(BW * 32), (size_t)(smem), st, tables, tm, B, offsets, indices, nnz, x_dense.hi, x_dense.lo,      \
                                           x_dense.ld, dconcat, ldc, dx_hi, dx_lo, lddx, dE, wb, err);        \
     }
     if (d == 128) DLRM_BWD(4) else DLRM_BWD(2)

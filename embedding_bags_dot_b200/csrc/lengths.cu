@@ -46,6 +46,7 @@ __device__ __forceinline__ void load_slice(const uint8_t* __restrict__ lengths, 
 
 __global__ void __launch_bounds__(LTHREADS) chunk_sums_kernel(const uint8_t* __restrict__ lengths, long long n,
                                                               int* __restrict__ sums) {
+    pdl_wait();
     __shared__ int tmp[32];
     uint8_t v[LPER];
     load_slice(lengths, n, (long long)blockIdx.x * LCH + (long long)threadIdx.x * LPER, v);
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(LTHREADS) chunk_sums_kernel(const uint8_t* __r
 
 __global__ void __launch_bounds__(LTHREADS) chunk_scan_kernel(const uint8_t* __restrict__ lengths, long long n,
                                                               const int* __restrict__ sums, int32_t* __restrict__ offsets) {
+    pdl_wait();
     __shared__ int tmp[32];
     __shared__ int scan[LTHREADS];
     // this chunk's offset: the sums of the chunks before it
@@ -98,9 +100,9 @@ dlrm_status launch_offsets_from_lengths(const uint8_t* lengths, long long n, int
     if (n == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t), st) == cudaSuccess ? DLRM_OK : DLRM_ERR_CUDA;
     const long long nb = (n + LCH - 1) / LCH;
     if (nb > 0x7FFFFFFF) return DLRM_ERR_UNSUPPORTED;
-    chunk_sums_kernel<<<(int)nb, LTHREADS, 0, st>>>(lengths, n, scratch);
+    (void)launch_pdl(chunk_sums_kernel, dim3((int)nb), dim3(LTHREADS), (size_t)(0), st, lengths, n, scratch);
     DLRM_LAUNCH_CHECK();
-    chunk_scan_kernel<<<(int)nb, LTHREADS, 0, st>>>(lengths, n, scratch, offsets);
+    (void)launch_pdl(chunk_scan_kernel, dim3((int)nb), dim3(LTHREADS), (size_t)(0), st, lengths, n, scratch, offsets);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }

@@ -12,6 +12,7 @@ namespace {
 template <typename T>
 __global__ void quantize_rows_kernel(const T* __restrict__ src, long long rows, int d, unsigned char* __restrict__ dst,
                                      long long rb) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
@@ -68,10 +69,10 @@ dlrm_status dlrm_quantize_rows_u8(const void* src, dlrm_dtype src_dt, int64_t ro
     const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
     const long long rb = (long long)u8row_bytes(d);
     if (src_dt == DLRM_F32)
-        quantize_rows_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), rows, d,
+        (void)launch_pdl(quantize_rows_kernel<float>, dim3(grid), dim3(256), (size_t)(0), st, static_cast<const float*>(src), rows, d,
                                                           static_cast<unsigned char*>(dst), rb);
     else
-        quantize_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), rows, d,
+        (void)launch_pdl(quantize_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(256), (size_t)(0), st, static_cast<const __nv_bfloat16*>(src), rows, d,
                                                                   static_cast<unsigned char*>(dst), rb);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;

@@ -32,6 +32,7 @@ constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;  // 4096
 
 __global__ void bce_kernel(int B, const float* __restrict__ z, const float* __restrict__ y, float* __restrict__ dz,
                            float* __restrict__ y_hat, float* __restrict__ partial) {
+    pdl_wait();
     __shared__ float red[256];
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     float l = 0.f;
@@ -54,6 +55,7 @@ __global__ void bce_kernel(int B, const float* __restrict__ z, const float* __re
 
 // Fixed-order sum of n partials (one block), divided by B.
 __global__ void mean_reduce_kernel(int n, const float* __restrict__ partial, int B, float* __restrict__ out) {
+    pdl_wait();
     __shared__ float red[1024];
     float s = 0.f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) s += partial[i];
@@ -72,6 +74,7 @@ __global__ void mean_reduce_kernel(int n, const float* __restrict__ partial, int
 __global__ void interact_bwd_kernel(int B, int K, int d, const float* __restrict__ x_dense,
                                     const float* __restrict__ E, const float* __restrict__ dconcat, int ldc,
                                     float* __restrict__ dx_dense, float* __restrict__ dE) {
+    pdl_wait();
     extern __shared__ float sm[];
     const int n1 = K + 1;
     float* X = sm;
@@ -130,6 +133,7 @@ __device__ __forceinline__ long long block_scan_incl(long long v, long long* tmp
 // Per-block sums of in[0..n) (n read from n_dev if not null).
 __global__ void scan_reduce_kernel(const int* __restrict__ in, long long n_host, const long long* n_dev,
                                    long long per_block, long long* __restrict__ block_sums) {
+    pdl_wait();
     __shared__ long long tmp[32];
     const long long n = n_dev ? *n_dev : n_host;
     const long long b0 = (long long)blockIdx.x * per_block;
@@ -141,6 +145,7 @@ __global__ void scan_reduce_kernel(const int* __restrict__ in, long long n_host,
 
 // Exclusive scan of the block sums (one block, sequential chunks in order). total -> *total.
 __global__ void scan_blocks_kernel(long long* __restrict__ sums, int nblocks, long long* __restrict__ total) {
+    pdl_wait();
     __shared__ long long tmp[32];
     long long carry = 0;
     for (int base = 0; base < nblocks; base += blockDim.x) {
@@ -161,6 +166,7 @@ __global__ void scan_blocks_kernel(long long* __restrict__ sums, int nblocks, lo
 __global__ void scan_down_kernel(const int* __restrict__ in, long long n_host, const long long* n_dev,
                                  long long per_block, const long long* __restrict__ block_off,
                                  long long* __restrict__ out) {
+    pdl_wait();
     __shared__ long long tmp[32];
     const long long n = n_dev ? *n_dev : n_host;
     const long long b0 = (long long)blockIdx.x * per_block;
@@ -185,6 +191,7 @@ __global__ void scan_down_kernel(const int* __restrict__ in, long long n_host, c
 // Valid length of bag kb (0 for bad offsets).
 __global__ void bag_len_kernel(long long KB, const int32_t* __restrict__ offsets, long long nnz, int* __restrict__ len,
                                ErrRecord* err) {
+    pdl_wait();
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < KB; q += (long long)gridDim.x * blockDim.x) {
         const long long st = offsets[q], en = offsets[q + 1];
         const bool isbad = st < 0 || en < st || en > nnz;
@@ -198,6 +205,7 @@ __global__ void occ_keys_kernel(int K, int B, const __grid_constant__ TableMeta 
                                 const int32_t* __restrict__ indices, const int* __restrict__ len,
                                 const long long* __restrict__ occ_off, long long cap, uint32_t invalid,
                                 uint32_t* __restrict__ keys, uint32_t* __restrict__ vals, ErrRecord* err) {
+    pdl_wait();
     unsigned over = 0;
     const long long KB = (long long)K * B;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < KB; q += (long long)gridDim.x * blockDim.x) {
@@ -229,6 +237,7 @@ __global__ void occ_keys_kernel(int K, int B, const __grid_constant__ TableMeta 
 __global__ void __launch_bounds__(SORT_THREADS) radix_hist_kernel(const uint32_t* __restrict__ keys,
                                                                   const long long* __restrict__ n_dev, int shift,
                                                                   int* __restrict__ counts, int nblocks) {
+    pdl_wait();
     __shared__ int h[RADIX];
     for (int i = threadIdx.x; i < RADIX; i += blockDim.x) h[i] = 0;
     __syncthreads();
@@ -249,6 +258,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(const uint3
                                                                      const long long* __restrict__ goff, int nblocks,
                                                                      uint32_t* __restrict__ kout,
                                                                      uint32_t* __restrict__ vout) {
+    pdl_wait();
     constexpr int W = SORT_THREADS / 32;
     __shared__ int wcount[W][RADIX];
     __shared__ long long base[W][RADIX];
@@ -302,6 +312,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(const uint3
 // head[i] = 1 if sorted key i starts a new row (valid keys only: key < invalid).
 __global__ void seg_head_kernel(const uint32_t* __restrict__ keys, const long long* __restrict__ n_dev,
                                 uint32_t invalid, int* __restrict__ head) {
+    pdl_wait();
     const long long n = *n_dev;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
         head[i] = (keys[i] < invalid && (i == 0 || keys[i] != keys[i - 1])) ? 1 : 0;
@@ -312,6 +323,7 @@ __global__ void seg_fill_kernel(const uint32_t* __restrict__ keys, const long lo
                                 uint32_t invalid, const int* __restrict__ head, const long long* __restrict__ seg_id,
                                 long long* __restrict__ seg_start, uint32_t* __restrict__ seg_row,
                                 int* __restrict__ seg_pieces, int piece) {
+    pdl_wait();
     const long long n = *n_dev;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
         if (head[i]) {
@@ -329,6 +341,7 @@ __global__ void seg_fill_kernel(const uint32_t* __restrict__ keys, const long lo
 // pieces of segment s = ceil(len / piece)
 __global__ void seg_pieces_kernel(const long long* __restrict__ n_seg_dev, const long long* __restrict__ seg_start,
                                   int piece, int* __restrict__ seg_pieces) {
+    pdl_wait();
     const long long ns = *n_seg_dev;
     for (long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x; s < ns; s += (long long)gridDim.x * blockDim.x)
         seg_pieces[s] = (int)((seg_start[s + 1] - seg_start[s] + piece - 1) / piece);
@@ -337,6 +350,7 @@ __global__ void seg_pieces_kernel(const long long* __restrict__ n_seg_dev, const
 // piece_seg[p] = segment of piece p
 __global__ void piece_owner_kernel(const long long* __restrict__ n_seg_dev, const long long* __restrict__ piece_base,
                                    int* __restrict__ piece_seg) {
+    pdl_wait();
     const long long ns = *n_seg_dev;
     for (long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x; s < ns; s += (long long)gridDim.x * blockDim.x)
         for (long long p = piece_base[s]; p < piece_base[s + 1]; ++p) piece_seg[p] = (int)s;
@@ -347,6 +361,7 @@ __global__ void piece_sum_kernel(int d, const long long* __restrict__ n_piece_de
                                  const long long* __restrict__ piece_base, const long long* __restrict__ seg_start,
                                  const uint32_t* __restrict__ vals, const float* __restrict__ dE, int piece,
                                  float* __restrict__ partial) {
+    pdl_wait();
     const long long np = *n_piece_dev;
     const int lane = threadIdx.x & 31;
     const long long wstride = (long long)gridDim.x * (blockDim.x >> 5);
@@ -403,6 +418,7 @@ __global__ void piece_sum_vec_kernel(const long long* __restrict__ n_piece_dev, 
                                      const long long* __restrict__ piece_base, const long long* __restrict__ seg_start,
                                      const uint32_t* __restrict__ vals, const float* __restrict__ dE, int piece,
                                      float* __restrict__ partial) {
+    pdl_wait();
     constexpr int d = 32 * V;
     const long long np = *n_piece_dev;
     const int lane = threadIdx.x & 31;
@@ -443,6 +459,7 @@ template <int V>
 __global__ void seg_apply_vec_kernel(const long long* __restrict__ n_seg_dev, const long long* __restrict__ piece_base,
                                      const uint32_t* __restrict__ seg_row, const float* __restrict__ partial, float lr,
                                      float* __restrict__ table, float* __restrict__ grad_out) {
+    pdl_wait();
     constexpr int d = 32 * V;
     const long long ns = *n_seg_dev;
     const int lane = threadIdx.x & 31;
@@ -479,6 +496,7 @@ __global__ void seg_apply_vec_kernel(const long long* __restrict__ n_seg_dev, co
 __global__ void seg_apply_kernel(int d, const long long* __restrict__ n_seg_dev, const long long* __restrict__ piece_base,
                                  const uint32_t* __restrict__ seg_row, const float* __restrict__ partial, float lr,
                                  float* __restrict__ table, float* __restrict__ grad_out) {
+    pdl_wait();
     const long long ns = *n_seg_dev;
     const int lane = threadIdx.x & 31;
     const long long wstride = (long long)gridDim.x * (blockDim.x >> 5);
@@ -496,13 +514,16 @@ __global__ void seg_apply_kernel(int d, const long long* __restrict__ n_seg_dev,
 }
 
 __global__ void sgd_kernel(long long n, float lr, float* __restrict__ w, const float* __restrict__ g) {
+    pdl_wait();
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
         w[i] -= lr * g[i];
 }
 
-__global__ void copy_count_kernel(const long long* __restrict__ src, int32_t* __restrict__ dst) { *dst = (int32_t)*src; }
+__global__ void copy_count_kernel(const long long* __restrict__ src, int32_t* __restrict__ dst) {
+    pdl_wait(); *dst = (int32_t)*src; }
 
 __global__ void clamp_count_kernel(long long* v, long long cap) {
+    pdl_wait();
     if (*v > cap) *v = cap;
 }
 
@@ -519,9 +540,9 @@ int grid_cap(long long n, int threads, int cap = 148 * 16) {
 dlrm_status launch_bce(int B, const float* z, const float* y, float* dz, float* y_hat, float* partial, float* loss,
                        cudaStream_t st) {
     const int nb = (B + 255) / 256;
-    bce_kernel<<<nb, 256, 0, st>>>(B, z, y, dz, y_hat, partial);
+    (void)launch_pdl(bce_kernel, dim3(nb), dim3(256), (size_t)(0), st, B, z, y, dz, y_hat, partial);
     DLRM_LAUNCH_CHECK();
-    mean_reduce_kernel<<<1, 1024, 0, st>>>(nb, partial, B, loss);
+    (void)launch_pdl(mean_reduce_kernel, dim3(1), dim3(1024), (size_t)(0), st, nb, partial, B, loss);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -534,7 +555,7 @@ dlrm_status launch_interact_bwd(int B, int K, int d, const float* x_dense, const
     if (smem > 227 * 1024) return DLRM_ERR_UNSUPPORTED;
     if (smem > 48 * 1024) cudaFuncSetAttribute(interact_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int grid = B < 148 * 8 ? B : 148 * 8;
-    interact_bwd_kernel<<<grid, 256, smem, st>>>(B, K, d, x_dense, E, dconcat, ldc, dx_dense, dE);
+    (void)launch_pdl(interact_bwd_kernel, dim3(grid), dim3(256), (size_t)(smem), st, B, K, d, x_dense, E, dconcat, ldc, dx_dense, dE);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -544,11 +565,11 @@ static dlrm_status scan_ints(const int* in, long long n_upper, const long long* 
                              long long* block_sums, long long* total, cudaStream_t st) {
     const long long per_block = 8192;
     const int nblocks = (int)((n_upper + per_block - 1) / per_block) + 1;
-    scan_reduce_kernel<<<nblocks, 1024, 0, st>>>(in, n_upper, n_dev, per_block, block_sums);
+    (void)launch_pdl(scan_reduce_kernel, dim3(nblocks), dim3(1024), (size_t)(0), st, in, n_upper, n_dev, per_block, block_sums);
     DLRM_LAUNCH_CHECK();
-    scan_blocks_kernel<<<1, 1024, 0, st>>>(block_sums, nblocks, total);
+    (void)launch_pdl(scan_blocks_kernel, dim3(1), dim3(1024), (size_t)(0), st, block_sums, nblocks, total);
     DLRM_LAUNCH_CHECK();
-    scan_down_kernel<<<nblocks, 1024, 0, st>>>(in, n_upper, n_dev, per_block, block_sums, out);
+    (void)launch_pdl(scan_down_kernel, dim3(nblocks), dim3(1024), (size_t)(0), st, in, n_upper, n_dev, per_block, block_sums, out);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -613,17 +634,17 @@ dlrm_status launch_sparse_prepare(int K, int B, const TableMeta& tm, long long t
     const uint32_t invalid = (uint32_t)total_rows;
     const int bits = key_bits(total_rows);
 
-    bag_len_kernel<<<grid_cap(KB, 256), 256, 0, st>>>(KB, offsets, nnz, bag_len, err);
+    (void)launch_pdl(bag_len_kernel, dim3(grid_cap(KB, 256)), dim3(256), (size_t)(0), st, KB, offsets, nnz, bag_len, err);
     DLRM_LAUNCH_CHECK();
     dlrm_status r = scan_ints(bag_len, KB, nullptr, occ_off, sums, &counts[0], st);
     if (r) return r;
     // n_occ = min(total occurrences, capacity)
     uint32_t* keys[2] = {reinterpret_cast<uint32_t*>(base + L.keys[0]), reinterpret_cast<uint32_t*>(base + L.keys[1])};
     uint32_t* vals[2] = {reinterpret_cast<uint32_t*>(base + L.vals[0]), reinterpret_cast<uint32_t*>(base + L.vals[1])};
-    occ_keys_kernel<<<grid_cap(KB, 256), 256, 0, st>>>(K, B, tm, offsets, indices, bag_len, occ_off, L.cap, invalid,
+    (void)launch_pdl(occ_keys_kernel, dim3(grid_cap(KB, 256)), dim3(256), (size_t)(0), st, K, B, tm, offsets, indices, bag_len, occ_off, L.cap, invalid,
                                                         keys[0], vals[0], err);
     DLRM_LAUNCH_CHECK();
-    clamp_count_kernel<<<1, 1, 0, st>>>(&counts[0], L.cap);
+    (void)launch_pdl(clamp_count_kernel, dim3(1), dim3(1), (size_t)(0), st, &counts[0], L.cap);
     DLRM_LAUNCH_CHECK();
 
     const int nsb = (int)sort_blocks(L.cap);
@@ -631,10 +652,10 @@ dlrm_status launch_sparse_prepare(int K, int B, const TableMeta& tm, long long t
     long long* hist_off = reinterpret_cast<long long*>(base + L.hist_off);
     int cur = 0;
     for (int shift = 0; shift < bits; shift += RADIX_BITS) {
-        radix_hist_kernel<<<nsb, SORT_THREADS, 0, st>>>(keys[cur], &counts[0], shift, hist, nsb);
+        (void)launch_pdl(radix_hist_kernel, dim3(nsb), dim3(SORT_THREADS), (size_t)(0), st, keys[cur], &counts[0], shift, hist, nsb);
         DLRM_LAUNCH_CHECK();
         if ((r = scan_ints(hist, (long long)RADIX * nsb, nullptr, hist_off, sums, nullptr, st))) return r;
-        radix_scatter_kernel<<<nsb, SORT_THREADS, 0, st>>>(keys[cur], vals[cur], &counts[0], shift, hist_off, nsb,
+        (void)launch_pdl(radix_scatter_kernel, dim3(nsb), dim3(SORT_THREADS), (size_t)(0), st, keys[cur], vals[cur], &counts[0], shift, hist_off, nsb,
                                                             keys[cur ^ 1], vals[cur ^ 1]);
         DLRM_LAUNCH_CHECK();
         cur ^= 1;
@@ -647,16 +668,16 @@ dlrm_status launch_sparse_prepare(int K, int B, const TableMeta& tm, long long t
     int* seg_pieces = reinterpret_cast<int*>(base + L.seg_pieces);
     long long* piece_base = reinterpret_cast<long long*>(base + L.piece_base);
     int* piece_seg = reinterpret_cast<int*>(base + L.piece_seg);
-    seg_head_kernel<<<grid_cap(L.cap, 256), 256, 0, st>>>(keys[cur], &counts[0], invalid, head);
+    (void)launch_pdl(seg_head_kernel, dim3(grid_cap(L.cap, 256)), dim3(256), (size_t)(0), st, keys[cur], &counts[0], invalid, head);
     DLRM_LAUNCH_CHECK();
     if ((r = scan_ints(head, L.cap, &counts[0], seg_id, sums, &counts[2], st))) return r;
-    seg_fill_kernel<<<grid_cap(L.cap, 256), 256, 0, st>>>(keys[cur], &counts[0], invalid, head, seg_id, seg_start, seg_row,
+    (void)launch_pdl(seg_fill_kernel, dim3(grid_cap(L.cap, 256)), dim3(256), (size_t)(0), st, keys[cur], &counts[0], invalid, head, seg_id, seg_start, seg_row,
                                                           seg_pieces, SPARSE_PIECE);
     DLRM_LAUNCH_CHECK();
-    seg_pieces_kernel<<<grid_cap(L.cap, 256), 256, 0, st>>>(&counts[2], seg_start, SPARSE_PIECE, seg_pieces);
+    (void)launch_pdl(seg_pieces_kernel, dim3(grid_cap(L.cap, 256)), dim3(256), (size_t)(0), st, &counts[2], seg_start, SPARSE_PIECE, seg_pieces);
     DLRM_LAUNCH_CHECK();
     if ((r = scan_ints(seg_pieces, L.cap, &counts[2], piece_base, sums, &counts[3], st))) return r;
-    piece_owner_kernel<<<grid_cap(L.cap, 256), 256, 0, st>>>(&counts[2], piece_base, piece_seg);
+    (void)launch_pdl(piece_owner_kernel, dim3(grid_cap(L.cap, 256)), dim3(256), (size_t)(0), st, &counts[2], piece_base, piece_seg);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -676,10 +697,10 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
     // table are aligned by construction; a caller's grad_out may not be)
     const bool vec = (d == 32 || d == 64 || d == 128) && (((uintptr_t)grad_out & 15) == 0);
 #define DLRM_SPARSE_VEC(V)                                                                                        \
-    piece_sum_vec_kernel<V><<<blocks, 256, 0, st>>>(&counts[3], piece_seg, piece_base, seg_start, vals, dE,        \
+    (void)launch_pdl(piece_sum_vec_kernel<V>, dim3(blocks), dim3(256), (size_t)(0), st, &counts[3], piece_seg, piece_base, seg_start, vals, dE,        \
                                                     SPARSE_PIECE, partial);                                         \
     DLRM_LAUNCH_CHECK();                                                                                          \
-    seg_apply_vec_kernel<V><<<blocks, 256, 0, st>>>(&counts[2], piece_base, seg_row, partial, lr, table, grad_out); \
+    (void)launch_pdl(seg_apply_vec_kernel<V>, dim3(blocks), dim3(256), (size_t)(0), st, &counts[2], piece_base, seg_row, partial, lr, table, grad_out); \
     DLRM_LAUNCH_CHECK();
     if (vec && d == 128) {
         DLRM_SPARSE_VEC(4)
@@ -688,10 +709,10 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
     } else if (vec && d == 32) {
         DLRM_SPARSE_VEC(1)
     } else {
-        piece_sum_kernel<<<blocks, 256, 0, st>>>(d, &counts[3], piece_seg, piece_base, seg_start, vals, dE,
+        (void)launch_pdl(piece_sum_kernel, dim3(blocks), dim3(256), (size_t)(0), st, d, &counts[3], piece_seg, piece_base, seg_start, vals, dE,
                                                  SPARSE_PIECE, partial);
         DLRM_LAUNCH_CHECK();
-        seg_apply_kernel<<<blocks, 256, 0, st>>>(d, &counts[2], piece_base, seg_row, partial, lr, table, grad_out);
+        (void)launch_pdl(seg_apply_kernel, dim3(blocks), dim3(256), (size_t)(0), st, d, &counts[2], piece_base, seg_row, partial, lr, table, grad_out);
         DLRM_LAUNCH_CHECK();
     }
 #undef DLRM_SPARSE_VEC
@@ -699,7 +720,7 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
         cudaMemcpyAsync(rows_out, seg_row, sizeof(uint32_t) * L.cap, cudaMemcpyDeviceToDevice, st);
     }
     if (n_rows_out) {
-        copy_count_kernel<<<1, 1, 0, st>>>(&counts[2], n_rows_out);
+        (void)launch_pdl(copy_count_kernel, dim3(1), dim3(1), (size_t)(0), st, &counts[2], n_rows_out);
         DLRM_LAUNCH_CHECK();
     }
     return DLRM_OK;
@@ -707,7 +728,7 @@ dlrm_status launch_sparse_apply(int d, const char* base, const SparseLayout& L, 
 
 dlrm_status launch_sgd(long long n, float lr, float* w, const float* g, cudaStream_t st) {
     if (n <= 0) return DLRM_OK;
-    sgd_kernel<<<grid_cap(n, 256), 256, 0, st>>>(n, lr, w, g);
+    (void)launch_pdl(sgd_kernel, dim3(grid_cap(n, 256)), dim3(256), (size_t)(0), st, n, lr, w, g);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }

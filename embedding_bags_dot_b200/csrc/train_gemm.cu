@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(long long NI, long long N
                                                        const float* __restrict__ mask, const float* __restrict__ mask_lo,
                                                        long long ldm, float* __restrict__ C, float* __restrict__ C_lo,
                                                        long long ldc, long long r_chunk, long long part_stride) {
+    pdl_wait();
     __shared__ float As[TK][TN + 4];
     __shared__ float Bs[TK][TN + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(long long NI, long long N
 // dW[i][j] = sum over splits (in order) of part[s][i][j]; db[i] from column NJ.
 __global__ void wgrad_reduce_kernel(int splits, long long NI, long long NJ, const float* __restrict__ part,
                                     long long part_stride, float* __restrict__ dW, long long ldw, float* __restrict__ db) {
+    pdl_wait();
     const long long n = NI * (NJ + 1);
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
         float s = 0.f;
@@ -157,6 +159,7 @@ __global__ void wgrad_reduce_kernel(int splits, long long NI, long long NJ, cons
 
 __global__ void split_pair_kernel(long long rows, int cols, const float* __restrict__ src, long long lds,
                                   float* __restrict__ hi, float* __restrict__ lo, long long ldd) {
+    pdl_wait();
     const long long n = rows * cols;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
         const long long r = q / cols, c = q - r * cols;
@@ -169,6 +172,7 @@ __global__ void split_pair_kernel(long long rows, int cols, const float* __restr
 
 __global__ void split_pair_vec_kernel(long long rows, int cols4, const float4* __restrict__ src, long long lds4,
                                       float4* __restrict__ hi, float4* __restrict__ lo, long long ldd4) {
+    pdl_wait();
     const long long n = rows * cols4;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
         const long long r = q / cols4, c = q - r * cols4;
@@ -181,6 +185,7 @@ __global__ void split_pair_vec_kernel(long long rows, int cols4, const float4* _
 
 __global__ void merge_pair_kernel(long long rows, int cols, const float* __restrict__ hi,
                                   const float* __restrict__ lo, long long lds, float* __restrict__ out, long long ldo) {
+    pdl_wait();
     const long long n = rows * cols;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
         const long long r = q / cols, c = q - r * cols;
@@ -190,6 +195,7 @@ __global__ void merge_pair_kernel(long long rows, int cols, const float* __restr
 
 __global__ void split_sum_kernel(int S, long long N, int K, const float* __restrict__ part, long long ldp,
                                  float* __restrict__ out, long long ldo) {
+    pdl_wait();
     const long long n = N * K;
     const long long zs = N * ldp;
     for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < n; q += (long long)gridDim.x * blockDim.x) {
@@ -213,6 +219,7 @@ __global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const
                                                        const float* __restrict__ al, long long lda,
                                                        const float* __restrict__ X, long long ldx, int kx, bool ones,
                                                        long long rows_per, float* __restrict__ part) {
+    pdl_wait();
     constexpr int WARPS = CS_WARPS(NW);
     __shared__ float red[WARPS][128 * NW + 1];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -266,6 +273,7 @@ __global__ void __launch_bounds__(256) colsum_w_kernel(long long M, int N, const
 // then a fixed butterfly across lanes; w < kx -> dW[c * ldw + w], w == kx -> db[c]
 __global__ void colsum_w_final_kernel(int P, int N, int NW, int kx, bool ones, const float* __restrict__ part,
                                       float* __restrict__ dW, long long ldw, float* __restrict__ db) {
+    pdl_wait();
     const long long n = (long long)N * NW;
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -286,6 +294,7 @@ __global__ void colsum_w_final_kernel(int P, int N, int NW, int kx, bool ones, c
 // bits[m][j / 32] bit j % 32 = (y(m, j) > 0), y plain or a pair: one warp per (row, 32 columns)
 __global__ void relu_bits_kernel(long long M, int N, const float* __restrict__ yh, const float* __restrict__ yl,
                                  long long ldy, uint32_t* __restrict__ bits, long long ldbits) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long words = M * ldbits;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -302,6 +311,7 @@ __global__ void relu_bits_kernel(long long M, int N, const float* __restrict__ y
 // db[j] = sum over 32-row groups g of csum[g][j] in increasing g (one warp per column: lane l adds
 // g = l, l + 32, ... in order, then a fixed butterfly)
 __global__ void csum_final_kernel(int G, int J, const float* __restrict__ csum, float* __restrict__ db) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
     for (int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); j < J; j += warps) {
@@ -323,6 +333,7 @@ __global__ void __launch_bounds__(128) narrow_fwd_kernel(long long M, int N, int
                                                          long long ldw, const float* __restrict__ bias, bool relu,
                                                          float* __restrict__ yh, float* __restrict__ yl, long long ldy,
                                                          uint32_t* __restrict__ bits, long long ldbits) {
+    pdl_wait();
     __shared__ float xs[NARROW_ROWS][17];
     const long long rb = (long long)blockIdx.y * NARROW_ROWS;
     const int nr = (int)(M - rb < NARROW_ROWS ? M - rb : NARROW_ROWS);
@@ -374,6 +385,7 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(long long M, int K, cons
                                                         const float* __restrict__ xl, long long ldx,
                                                         const float* __restrict__ w, const float* __restrict__ wl,
                                                         const float* __restrict__ bias, float* __restrict__ z) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long b = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); b < M; b += warps) {
@@ -392,6 +404,7 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(long long M, int K, cons
 __global__ void outer_mask_kernel(long long M, int K, const float* __restrict__ dz, const float* __restrict__ w,
                                   const float* __restrict__ wl, const float* __restrict__ mh, const float* __restrict__ ml, long long ldm,
                                   float* __restrict__ dh, float* __restrict__ dl, long long ldd) {
+    pdl_wait();
     const long long n = M * K;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
         const long long b = i / K;
@@ -437,11 +450,11 @@ dlrm_status launch_split_pair(int rows, int cols, const float* src, int lds, flo
                      ((uintptr_t)hi & 15) == 0 && ((uintptr_t)lo & 15) == 0;
     if (vec) {
         const long long n = (long long)rows * (cols / 4);
-        split_pair_vec_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(
+        (void)launch_pdl(split_pair_vec_kernel, dim3(grid_stride_blocks(n)), dim3(256), (size_t)(0), st, 
             rows, cols / 4, reinterpret_cast<const float4*>(src), lds / 4, reinterpret_cast<float4*>(hi),
             reinterpret_cast<float4*>(lo), ldd / 4);
     } else {
-        split_pair_kernel<<<grid_stride_blocks((long long)rows * cols), 256, 0, st>>>(rows, cols, src, lds, hi, lo,
+        (void)launch_pdl(split_pair_kernel, dim3(grid_stride_blocks((long long)rows * cols)), dim3(256), (size_t)(0), st, rows, cols, src, lds, hi, lo,
                                                                                        ldd);
     }
     DLRM_LAUNCH_CHECK();
@@ -452,7 +465,7 @@ dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* 
                               cudaStream_t st) {
     const long long n = (long long)rows * cols;
     if (n <= 0) return DLRM_OK;
-    merge_pair_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(rows, cols, hi, lo, lds, out, ldo);
+    (void)launch_pdl(merge_pair_kernel, dim3(grid_stride_blocks(n)), dim3(256), (size_t)(0), st, rows, cols, hi, lo, lds, out, ldo);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -460,7 +473,7 @@ dlrm_status launch_merge_pair(int rows, int cols, const float* hi, const float* 
 dlrm_status launch_split_sum(int S, int N, int K, const float* part, int ldp, float* out, int ldo, cudaStream_t st) {
     const long long n = (long long)N * K;
     if (n == 0) return DLRM_OK;
-    split_sum_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(S, N, K, part, ldp, out, ldo);
+    (void)launch_pdl(split_sum_kernel, dim3(grid_stride_blocks(n)), dim3(256), (size_t)(0), st, S, N, K, part, ldp, out, ldo);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
@@ -476,17 +489,17 @@ dlrm_status launch_colsum_w(int M, int N, F32Pair A, const float* X, int ldx, in
     const int nw = kx + (ones ? 1 : 0);
     int NW;
     if (nw <= 1) {
-        colsum_w_kernel<1><<<grid, 32 * CS_WARPS(1), 0, st>>>(M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones, rows_per,
+        (void)launch_pdl(colsum_w_kernel<1>, dim3(grid), dim3(32 * CS_WARPS(1)), (size_t)(0), st, M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones, rows_per,
                                                               scratch);
         NW = 1;
     } else {
-        colsum_w_kernel<CS_NW><<<grid, 32 * CS_WARPS(CS_NW), 0, st>>>(M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones,
+        (void)launch_pdl(colsum_w_kernel<CS_NW>, dim3(grid), dim3(32 * CS_WARPS(CS_NW)), (size_t)(0), st, M, N, A.hi, A.lo, A.ld, X, ldx, kx, ones,
                                                                       rows_per, scratch);
         NW = CS_NW;
     }
     DLRM_LAUNCH_CHECK();
     const long long outs = (long long)N * NW;
-    colsum_w_final_kernel<<<(int)((outs + 7) / 8 < 148 * 16 ? (outs + 7) / 8 : 148 * 16), 256, 0, st>>>(
+    (void)launch_pdl(colsum_w_final_kernel, dim3((int)((outs + 7) / 8 < 148 * 16 ? (outs + 7) / 8 : 148 * 16)), dim3(256), (size_t)(0), st, 
         P, N, NW, kx, ones, scratch, dW, ldw, db);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
@@ -500,28 +513,28 @@ dlrm_status train_linear_fwd(int M, int N, int K, F32Pair x, F32Pair W, const fl
         return tf32x3_fwd(M, N, K, x, W, b, y, y_lo, ldy, relu_bits, relu_bits_ld(N), err, st);
     if (K <= 16) {
         const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + NARROW_ROWS - 1) / NARROW_ROWS));
-        narrow_fwd_kernel<<<grid, 128, 0, st>>>(M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy,
+        (void)launch_pdl(narrow_fwd_kernel, dim3(grid), dim3(128), (size_t)(0), st, M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, relu, y, y_lo, ldy,
                                                 relu_bits, relu_bits_ld(N));
         DLRM_LAUNCH_CHECK();
         return DLRM_OK;
     }
     if (N == 1 && !relu && !y_lo) {
         const long long blocks = (M + 7) / 8;
-        gemv_rows_kernel<<<(int)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, st>>>(M, K, x.hi, x.lo, x.ld, W.hi,
+        (void)launch_pdl(gemv_rows_kernel, dim3((int)(blocks < 148 * 16 ? blocks : 148 * 16)), dim3(256), (size_t)(0), st, M, K, x.hi, x.lo, x.ld, W.hi,
                                                                                      W.lo, b, y);
         DLRM_LAUNCH_CHECK();
         return DLRM_OK;
     }
     if (relu)
-        gemm_f32_kernel<false, false, EPI_BIAS_RELU, false><<<grid_for(M, N, 1), 256, 0, st>>>(
+        (void)launch_pdl(gemm_f32_kernel<false, false, EPI_BIAS_RELU, false>, dim3(grid_for(M, N, 1)), dim3(256), (size_t)(0), st, 
             M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
     else
-        gemm_f32_kernel<false, false, EPI_BIAS, false><<<grid_for(M, N, 1), 256, 0, st>>>(
+        (void)launch_pdl(gemm_f32_kernel<false, false, EPI_BIAS, false>, dim3(grid_for(M, N, 1)), dim3(256), (size_t)(0), st, 
             M, N, K, x.hi, x.lo, x.ld, W.hi, W.lo, W.ld, b, nullptr, nullptr, 0, y, y_lo, ldy, K, 0);
     DLRM_LAUNCH_CHECK();
     if (relu_bits) {
         const long long words = (long long)M * relu_bits_ld(N);
-        relu_bits_kernel<<<grid_stride_blocks(words * 32), 256, 0, st>>>(M, N, y, y_lo, ldy, relu_bits,
+        (void)launch_pdl(relu_bits_kernel, dim3(grid_stride_blocks(words * 32)), dim3(256), (size_t)(0), st, M, N, y, y_lo, ldy, relu_bits,
                                                                          relu_bits_ld(N));
         DLRM_LAUNCH_CHECK();
     }
@@ -542,17 +555,17 @@ dlrm_status train_linear_dgrad(int M, int N, int K, F32Pair dy, F32Pair W, F32Pa
         return r;
     }
     if (N == 1 && relu_of.hi && dx_lo && !dy.lo) {
-        outer_mask_kernel<<<grid_stride_blocks((long long)M * K), 256, 0, st>>>(M, K, dy.hi, W.hi, W.lo, relu_of.hi,
+        (void)launch_pdl(outer_mask_kernel, dim3(grid_stride_blocks((long long)M * K)), dim3(256), (size_t)(0), st, M, K, dy.hi, W.hi, W.lo, relu_of.hi,
                                                                                relu_of.lo, relu_of.ld, dx, dx_lo, lddx);
         DLRM_LAUNCH_CHECK();
         return DLRM_OK;
     }
     if (relu_of.hi)
-        gemm_f32_kernel<false, true, EPI_MASK, false><<<grid_for(M, K, 1), 256, 0, st>>>(
+        (void)launch_pdl(gemm_f32_kernel<false, true, EPI_MASK, false>, dim3(grid_for(M, K, 1)), dim3(256), (size_t)(0), st, 
             M, K, N, dy.hi, dy.lo, dy.ld, W.hi, W.lo, W.ld, nullptr, relu_of.hi, relu_of.lo, relu_of.ld, dx, dx_lo,
             lddx, N, 0);
     else
-        gemm_f32_kernel<false, true, EPI_PLAIN, false><<<grid_for(M, K, 1), 256, 0, st>>>(
+        (void)launch_pdl(gemm_f32_kernel<false, true, EPI_PLAIN, false>, dim3(grid_for(M, K, 1)), dim3(256), (size_t)(0), st, 
             M, K, N, dy.hi, dy.lo, dy.ld, W.hi, W.lo, W.ld, nullptr, nullptr, nullptr, 0, dx, dx_lo, lddx, N, 0);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
@@ -574,7 +587,7 @@ dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float
         if (csum) {
             // bias gradient from the column sums per 32-row group that the data-gradient epilogue left
             const int G = (M + 31) / 32;
-            csum_final_kernel<<<(N + 7) / 8 < 148 * 8 ? (N + 7) / 8 : 148 * 8, 256, 0, st>>>(G, N, csum, db);
+            (void)launch_pdl(csum_final_kernel, dim3((N + 7) / 8 < 148 * 8 ? (N + 7) / 8 : 148 * 8), dim3(256), (size_t)(0), st, G, N, csum, db);
             DLRM_LAUNCH_CHECK();
             return DLRM_OK;
         }
@@ -595,12 +608,12 @@ dlrm_status train_linear_wgrad(int M, int N, int K, F32Pair dy, F32Pair x, float
     long long chunk = ((long long)M + splits - 1) / splits;
     chunk = (chunk + TK - 1) / TK * TK;
     const long long pstride = (long long)N * (K + 1);
-    gemm_f32_kernel<true, true, EPI_PARTIAL, true><<<grid_for(N, K + 1, splits), 256, 0, st>>>(
+    (void)launch_pdl(gemm_f32_kernel<true, true, EPI_PARTIAL, true>, dim3(grid_for(N, K + 1, splits)), dim3(256), (size_t)(0), st, 
         N, K, M, dy.hi, dy.lo, dy.ld, x.hi, x.lo, x.ld, nullptr, nullptr, nullptr, 0, scratch, nullptr, 0, chunk,
         pstride);
     DLRM_LAUNCH_CHECK();
     const long long n = pstride;
-    wgrad_reduce_kernel<<<grid_stride_blocks(n), 256, 0, st>>>(splits, N, K, scratch, pstride, dW, ldw, db);
+    (void)launch_pdl(wgrad_reduce_kernel, dim3(grid_stride_blocks(n)), dim3(256), (size_t)(0), st, splits, N, K, scratch, pstride, dW, ldw, db);
     DLRM_LAUNCH_CHECK();
     return DLRM_OK;
 }
