@@ -78,8 +78,10 @@ def test_linear_tc_two_layers_bf16_hidden(act):
     assert_close(to_np(out), want, "bf16", "two-layer bf16 MLP", scale_mlp(Ws, bs, xs, sigmoid=(act == E.ACT_SIGMOID)))
 
 
-# serving-size batches (a handful of rows) through the same layer path
-@pytest.mark.parametrize("M,N,K", [(1, 256, 479), (5, 1024, 1024), (8, 40, 13), (16, 300, 200), (9, 64, 5)])
+# serving-size batches (a handful of rows) through the same layer path: the A box holds the batch's rows
+# rounded up to 8, and the 128-row MMA's rows past them never reach the output
+@pytest.mark.parametrize("M,N,K", [(1, 256, 479), (5, 1024, 1024), (8, 40, 13), (16, 300, 200), (9, 64, 5),
+                                   (32, 512, 1024), (33, 512, 1024), (31, 1000, 1100)])
 @pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
 def test_linear_small_batch(M, N, K, dt):
     if dt == "f32":
