@@ -14,6 +14,11 @@
  *    buffer (tables, weights, inputs, outputs, workspace); the library never
  *    allocates device memory and keeps no pointer after a call returns.
  *  - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *    Its kernels are launched as programmatic dependents (each may start its
+ *    setup while the previous kernel on the stream finishes, and waits for
+ *    that kernel's completion before touching global memory), so the calls
+ *    keep plain stream order with any other work on the stream and can be
+ *    captured in CUDA graphs.
  *    Host-detectable argument errors return a status before anything is
  *    launched. Errors found on the device (an index outside its table, bag
  *    offsets that decrease or leave [0, nnz]) never trap: the offending
