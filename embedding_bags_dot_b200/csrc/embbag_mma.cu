@@ -103,7 +103,7 @@ __device__ __forceinline__ void dequant8(uint2 codes, float sc, float of, float 
     }
 }
 
-// Byte offset of the integer route's (s, m, s S, 0) slots: after the 8-bit tile and the staged Gram.
+// Byte offset of the integer route's (s, m, u, 0) slots: after the 8-bit tile and the staged Gram.
 __host__ __device__ constexpr int u8_meta_offset(int K, int KP, int qrb) {
     return (std::max((K + 4) * qrb, (KP * (KP + 8) + 1) * 4) + 15) / 16 * 16;
 }
@@ -216,7 +216,7 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, int 
         if (lane == 0) G[ZERO_SLOT] = 0.f;
     }
     __syncwarp();
-    // per bag: slot (s, m, s S); column 0 of its Gram row becomes <q_i, qx>
+    // per bag: slot (s, m, u = s S + (d/2) m); column 0 of its Gram row becomes <q_i, qx>
     const float* Gx0 = G + P0 * GS;
 #pragma unroll
     for (int w = 0; w < (KP + 31) / 32; ++w) {
@@ -224,21 +224,22 @@ __device__ __forceinline__ void u8_sample(unsigned char* xw, uint32_t xw_s, int 
         if (i <= K) {
             const float S_i = G[i * GS];
             G[i * GS] = fmaf(65536.f, Gx0[2 * GS + i], fmaf(256.f, Gx0[GS + i], Gx0[i]));
-            meta[i] = make_float4(sm[w].x, sm[w].y, sm[w].x * S_i, 0.f);
+            meta[i] = make_float4(sm[w].x, sm[w].y, fmaf(0.5f * (float)d, sm[w].y, sm[w].x * S_i), 0.f);
         }
     }
     if (lane == 0) {
         const float Sx = fmaf(65536.f, Gx0[2 * GS], fmaf(256.f, Gx0[GS], Gx0[0]));
-        meta[0] = make_float4(sx, mn, sx * Sx, 0.f);
+        meta[0] = make_float4(sx, mn, fmaf(0.5f * (float)d, mn, sx * Sx), 0.f);
     }
     if (lane == 1) meta[KP] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncwarp();
 
-    // Z for the Gram entry at `src`: s_i s_j g + t_i m_j + t_j m_i + d m_i m_j
+    // Z for the Gram entry at `src`: s_i s_j g + t_i m_j + t_j m_i + d m_i m_j (t = s S), written as
+    // s_i s_j g + u_i m_j + u_j m_i with u = t + (d/2) m
     auto zval = [&](uint32_t src) {
         const int i = (int)(src / GS), j = (int)(src - (uint32_t)i * GS);
         const float4 a = meta[i], c = meta[j];
-        return fmaf(a.x * c.x, G[src], fmaf(a.z, c.y, fmaf(c.z, a.y, (float)d * a.y * c.y)));
+        return fmaf(a.x * c.x, G[src], fmaf(a.z, c.y, c.z * a.y));
     };
     if (out_dt == DLRM_BF16) {
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(out) + row0;
@@ -402,11 +403,10 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
                     nonfinite |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
                 }
             }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-            }
+            // warp-wide min and max (a non-finite x_dense sends the sample to the dequantising route
+            // whatever these return)
+            asm volatile("redux.sync.min.f32 %0, %0, 0xffffffff;" : "+f"(mn));
+            asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mx));
             range = mx - mn;
             int_route = bm.multi == 0 && !__any_sync(FULL, nonfinite) && isfinite(range);
         }
@@ -591,7 +591,7 @@ __global__ void __launch_bounds__(WARPS * 32, MT >= 3 ? 2 : 3) embbag_interact_m
 // ------------------------------------------------------------------ host side
 
 // Bytes of a warp's region. bf16 tile: rows 0..K+1 of 2d+16 bytes, or row 0 plus the staged Gram; uint8
-// tables add the integer route's tile (rows 0..K+3 of one record each) or Gram, then its (s, m, s S) slots.
+// tables add the integer route's tile (rows 0..K+3 of one record each) or Gram, then its (s, m, u) slots.
 static int mma_warp_bytes(int K, int d, bool q, int& MT) {
     MT = (K + (q ? 4 : 2) + 15) / 16;
     const int KP = 16 * MT;
