@@ -90,6 +90,37 @@ def test_product_path_has_no_cpu_fallback():
             assert "import oracle" not in open(f).read() and "from oracle" not in open(f).read(), f
 
 
+def _kernel_bodies(src):
+    """(name, body) of every __global__ function definition in a CUDA source."""
+    out = []
+    for m in re.finditer(r"__global__", src):
+        head_end = src.index("{\n", m.end())
+        name = re.findall(r"(\w+)\s*\(", src[m.end():head_end])
+        depth, i = 0, head_end
+        while True:
+            depth += {"{": 1, "}": -1}.get(src[i], 0)
+            i += 1
+            if depth == 0:
+                break
+        out.append((name[-1] if name else "?", src[head_end:i]))
+    return out
+
+
+def test_every_kernel_is_a_programmatic_dependent_that_waits():
+    """Every kernel is launched through launch_pdl (no <<<>>> launches), waits (pdl_wait) before it may
+    touch global memory, and never lets its dependent start early (no griddepcontrol.launch_dependents)."""
+    srcs = glob.glob(os.path.join(ROOT, "embedding_bags_dot_b200", "csrc", "*.cu"))
+    n = 0
+    for f in srcs:
+        src = open(f).read()
+        assert "<<<" not in src, f"{f}: a launch bypasses launch_pdl"
+        assert "launch_dependents" not in src, f"{f}: a kernel triggers its dependent early"
+        for name, body in _kernel_bodies(src):
+            assert "pdl_wait();" in body, f"{os.path.basename(f)}: {name} never waits for the previous kernel"
+            n += 1
+    assert n >= 50
+
+
 def _cpu_mlp(dims, dt):
     E = pytest.importorskip("embedding_bags_dot_b200")
     td = {"f32": torch.float32, "bf16": torch.bfloat16}[dt]
